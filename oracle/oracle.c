@@ -1,0 +1,429 @@
+/*
+ * oracle.c -- plain, slow CPU restatement of the lightning indexer and its
+ * per-query top-k: the dense full-prefix form, PIVOT's grouped form (Reuse
+ * and Refine) and the MTP decode form.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing on the product path may link or call
+ * this file: only the tests, the smoke check and the benchmark's CPU-baseline
+ * leg do.  It shares no code, header or constant with the CUDA library.
+ *
+ * Every score is accumulated in double from inputs decoded exactly (bf16 or
+ * fp32).  Every selection is a full sort.  No blocking, fusion or reordering
+ * beyond what each definition states.
+ *
+ * Sources (pages are cited by title and by the part of the page):
+ *  - "PIVOT: Efficient Query-Group Indexing for Token-Level Sparse Attention"
+ *    (arXiv 2607.24593):
+ *      Method, first paragraph: every query is scored against its whole
+ *        prefix by the indexer score, Eq. (1), then keeps a top-k set.
+ *        The text of Eq. (1) did not survive; the reading used here is the
+ *        DSA lightning-indexer score
+ *            I[t,s] = sum_j w[t,j] * max(0, q[t,j] . k[s]),   s <= t,
+ *        which matches observation O3 of the same page (a per-head ReLU of
+ *        q_{t,j} . k_s, summed over heads).
+ *      Method, grouping paragraph: contiguous groups of a fixed size g that
+ *        never cross a request boundary; the last group may be smaller.
+ *      Experimental setup: the proxy is the mean of the group's queries;
+ *        PIVOT-Reuse shares the proxy's top-k; k = 2048, c = 2k.
+ *      Abstract: one shared full-prefix traversal yields a candidate set,
+ *        then PIVOT-Refine re-scores it with each member's own indexer.
+ *      Method, decode paragraph: the decode group is the current query plus
+ *        the MTP draft queries of the same step.
+ *  - Readings where the pages are silent (each also listed in the design
+ *    notes): proxy of w = mean of w; proxy arithmetic = fp32 sum in member
+ *    order, IEEE division, then round-to-nearest-even to bf16 for bf16
+ *    queries; ties in the top-k go to the lower index; the output lists the
+ *    selected positions in ascending order, padded with -1; Reuse member i
+ *    takes the proxy ranking restricted to its own prefix s <= t_i; the
+ *    shared scan of a group covers the prefix of its last member.
+ *
+ * Build: gcc -O2 -std=c11 -fPIC -shared -ffp-contract=off -pthread
+ *        -o liboracle.so oracle.c      (see oracle/build.py)
+ * -ffp-contract=off keeps every float operation of the proxy step separately
+ * rounded, as its definition states.
+ */
+#include <math.h>
+#include <pthread.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+enum { ORA_BF16 = 0, ORA_F32 = 1 };
+enum { ORA_DENSE = 0, ORA_REUSE = 1, ORA_REFINE = 2 };
+
+/* ---------------------------------------------------------------- inputs */
+
+static double bf16_bits_to_double(uint16_t b) {
+    uint32_t u = (uint32_t)b << 16;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return (double)f;
+}
+
+/* element i of a bf16 (bit pattern) or fp32 array, exactly, as a double */
+static double load_elem(const void *base, int dtype, size_t i) {
+    if (dtype == ORA_BF16) return bf16_bits_to_double(((const uint16_t *)base)[i]);
+    return (double)((const float *)base)[i];
+}
+
+/* round-to-nearest-even of a finite float to a bf16 bit pattern */
+static uint16_t float_to_bf16_rne(float f) {
+    uint32_t u;
+    memcpy(&u, &f, sizeof u);
+    u += 0x7FFFu + ((u >> 16) & 1u);
+    return (uint16_t)(u >> 16);
+}
+
+/* --------------------------------------------------------------- Eq. (1) */
+
+/* I[t,s] = sum_j w[t,j] * max(0, sum_i q[t,j,i] * k[s,i]).
+ * q_row: element offset of q[t,0,0] in q; k_row: offset of k[s,0] in k. */
+static double index_score(const void *q, size_t q_row, const void *k, size_t k_row,
+                          const float *w_row, int H, int d, int dtype) {
+    double total = 0.0;
+    for (int j = 0; j < H; ++j) {
+        double dot = 0.0;
+        for (int i = 0; i < d; ++i)
+            dot += load_elem(q, dtype, q_row + (size_t)j * d + i) * load_elem(k, dtype, k_row + i);
+        if (dot > 0.0) total += (double)w_row[j] * dot;
+    }
+    return total;
+}
+
+/* ------------------------------------------------------------- selection */
+
+typedef struct {
+    double score;
+    int pos;
+} cand_t;
+
+/* higher score first; equal scores: lower position first */
+static int by_score_desc_pos_asc(const void *a, const void *b) {
+    const cand_t *x = (const cand_t *)a, *y = (const cand_t *)b;
+    if (x->score > y->score) return -1;
+    if (x->score < y->score) return 1;
+    return (x->pos > y->pos) - (x->pos < y->pos);
+}
+
+static int int_asc(const void *a, const void *b) {
+    int x = *(const int *)a, y = *(const int *)b;
+    return (x > y) - (x < y);
+}
+
+/* The first min(k, n) candidates in (score desc, pos asc) order, written as
+ * ascending positions, then -1 up to k.  Sorts c in place. */
+static void select_topk(cand_t *c, int n, int k, int *out) {
+    qsort(c, (size_t)n, sizeof(cand_t), by_score_desc_pos_asc);
+    int m = n < k ? n : k;
+    for (int i = 0; i < m; ++i) out[i] = c[i].pos;
+    qsort(out, (size_t)m, sizeof(int), int_asc);
+    for (int i = m; i < k; ++i) out[i] = -1;
+}
+
+/* ------------------------------------------------------------ exported */
+
+/* Scores of one query row against n consecutive keys starting at key row
+ * key0: out[s] = I[q_row, key0 + s].  q_row indexes q [*, H, d] and w [*, H]. */
+int ora_score_row(const void *q, const void *k, const float *w, int dtype, int H, int d,
+                  long long q_row, long long key0, int n, double *out) {
+    if (!q || !k || !w || !out || H <= 0 || d <= 0 || n < 0) return 1;
+    for (int s = 0; s < n; ++s)
+        out[s] = index_score(q, (size_t)q_row * H * d, k, (size_t)(key0 + s) * d,
+                             w + (size_t)q_row * H, H, d, dtype);
+    return 0;
+}
+
+/* The selection rule alone, applied to given scores (used to re-select on
+ * scores exported by another implementation).  pos may be NULL (= 0..n-1). */
+int ora_select(const double *scores, const int *pos, int n, int k, int *out) {
+    if (n < 0 || k <= 0 || !out) return 1;
+    cand_t *c = (cand_t *)malloc(sizeof(cand_t) * (size_t)(n > 0 ? n : 1));
+    if (!c) return 2;
+    for (int i = 0; i < n; ++i) {
+        c[i].score = scores[i];
+        c[i].pos = pos ? pos[i] : i;
+    }
+    select_topk(c, n, k, out);
+    free(c);
+    return 0;
+}
+
+/* Locate global row r among requests given by cu_seqlens. */
+static int find_request(const int *cu, int num_seqs, long long r) {
+    int lo = 0, hi = num_seqs - 1;
+    while (lo < hi) {
+        int mid = (lo + hi + 1) / 2;
+        if (cu[mid] <= r) lo = mid; else hi = mid - 1;
+    }
+    return lo;
+}
+
+/* Proxy of a group: per head and dimension the fp32 sum of the members'
+ * queries in member order, divided by the group size (IEEE fp32), rounded
+ * to bf16 for bf16 queries; w-proxy likewise in fp32.  Members are rows
+ * m0, m0+1, ..., m0+cnt-1 of q [*, H, d] and w [*, H].
+ * qbar receives H*d elements in dtype format, wbar H floats. */
+static void group_proxy(const void *q, const float *w, int dtype, int H, int d,
+                        long long m0, int cnt, void *qbar, float *wbar) {
+    for (int j = 0; j < H; ++j) {
+        for (int i = 0; i < d; ++i) {
+            float sum = 0.0f;
+            for (int m = 0; m < cnt; ++m)
+                sum = sum + (float)load_elem(q, dtype, (size_t)(m0 + m) * H * d + (size_t)j * d + i);
+            float mean = sum / (float)cnt;
+            if (dtype == ORA_BF16) ((uint16_t *)qbar)[(size_t)j * d + i] = float_to_bf16_rne(mean);
+            else ((float *)qbar)[(size_t)j * d + i] = mean;
+        }
+        float ws = 0.0f;
+        for (int m = 0; m < cnt; ++m) ws = ws + w[(size_t)(m0 + m) * H + j];
+        wbar[j] = ws / (float)cnt;
+    }
+}
+
+/* Exported for tests of the proxy step alone. */
+int ora_group_proxy(const void *q, const float *w, int dtype, int H, int d, long long m0, int cnt,
+                    void *qbar, float *wbar) {
+    if (!q || !w || !qbar || !wbar || cnt <= 0) return 1;
+    group_proxy(q, w, dtype, H, d, m0, cnt, qbar, wbar);
+    return 0;
+}
+
+/* One grouped selection.
+ *   q, w: query rows; members are rows m0 .. m0+cnt-1; member t positions
+ *         are pos0 .. pos0+cnt-1 (request-local); the group's last member
+ *         sits at t_last = pos0+cnt-1.
+ *   keys: key rows key0 + s for s = 0 .. t_last.
+ *   mode: ORA_REUSE or ORA_REFINE; c: candidate budget (Refine).
+ *   member: which member (0..cnt-1) to produce; out: k entries. */
+static int grouped_member_topk(const void *q, const void *k, const float *w, int dtype, int H, int d,
+                               long long m0, int cnt, int pos0, long long key0, int topk, int c,
+                               int mode, int member, int *out) {
+    int t_last = pos0 + cnt - 1;
+    int n = t_last + 1;
+    size_t esz = dtype == ORA_BF16 ? 2 : 4;
+    void *qbar = malloc(esz * (size_t)H * d);
+    float *wbar = (float *)malloc(sizeof(float) * (size_t)H);
+    cand_t *pc = (cand_t *)malloc(sizeof(cand_t) * (size_t)n);
+    if (!qbar || !wbar || !pc) { free(qbar); free(wbar); free(pc); return 2; }
+    group_proxy(q, w, dtype, H, d, m0, cnt, qbar, wbar);
+    /* one shared scan of the group's full prefix with the proxy */
+    for (int s = 0; s < n; ++s) {
+        pc[s].score = index_score(qbar, 0, k, (size_t)(key0 + s) * d, wbar, H, d, dtype);
+        pc[s].pos = s;
+    }
+    int t = pos0 + member;
+    int rc = 0;
+    if (mode == ORA_REUSE) {
+        /* the proxy ranking, restricted to the member's own prefix */
+        select_topk(pc, t + 1, topk, out);
+    } else {
+        /* candidate set C: the proxy's top-min(c, n) over the whole prefix */
+        qsort(pc, (size_t)n, sizeof(cand_t), by_score_desc_pos_asc);
+        int nc = n < c ? n : c;
+        cand_t *mc = (cand_t *)malloc(sizeof(cand_t) * (size_t)(nc > 0 ? nc : 1));
+        if (!mc) { rc = 2; goto done; }
+        int m = 0;
+        for (int i = 0; i < nc; ++i) {
+            int s = pc[i].pos;
+            if (s > t) continue; /* the member's causal mask */
+            mc[m].score = index_score(q, (size_t)(m0 + member) * H * d, k, (size_t)(key0 + s) * d,
+                                      w + (size_t)(m0 + member) * H, H, d, dtype);
+            mc[m].pos = s;
+            ++m;
+        }
+        select_topk(mc, m, topk, out);
+        free(mc);
+    }
+done:
+    free(qbar);
+    free(wbar);
+    free(pc);
+    return rc;
+}
+
+/* ------------------------------------------------------ threaded drivers */
+
+typedef struct {
+    int kind; /* 0 dense, 1 pivot, 2 decode */
+    const void *q, *k;
+    const float *w;
+    int dtype, H, d, topk, g, c, mode;
+    const int *cu;
+    int num_seqs;
+    const long long *rows;
+    int nrows;
+    /* decode */
+    const int *kv_len;
+    int G, n_max;
+    int *out;
+    int next;
+    int rc;
+    pthread_mutex_t lock;
+} job_t;
+
+static int take(job_t *J) {
+    pthread_mutex_lock(&J->lock);
+    int i = J->next++;
+    pthread_mutex_unlock(&J->lock);
+    return i;
+}
+
+static void set_rc(job_t *J, int rc) {
+    if (!rc) return;
+    pthread_mutex_lock(&J->lock);
+    if (!J->rc) J->rc = rc;
+    pthread_mutex_unlock(&J->lock);
+}
+
+static void run_dense_row(job_t *J, int i) {
+    long long r = J->rows[i];
+    int b = find_request(J->cu, J->num_seqs, r);
+    int t = (int)(r - J->cu[b]);
+    cand_t *c = (cand_t *)malloc(sizeof(cand_t) * (size_t)(t + 1));
+    if (!c) { set_rc(J, 2); return; }
+    for (int s = 0; s <= t; ++s) {
+        c[s].score = index_score(J->q, (size_t)r * J->H * J->d, J->k, (size_t)(J->cu[b] + s) * J->d,
+                                 J->w + (size_t)r * J->H, J->H, J->d, J->dtype);
+        c[s].pos = s;
+    }
+    select_topk(c, t + 1, J->topk, J->out + (size_t)i * J->topk);
+    free(c);
+}
+
+static void run_pivot_row(job_t *J, int i) {
+    long long r = J->rows[i];
+    int b = find_request(J->cu, J->num_seqs, r);
+    int n = J->cu[b + 1] - J->cu[b];
+    int t = (int)(r - J->cu[b]);
+    int lo = (t / J->g) * J->g;
+    int hi = lo + J->g < n ? lo + J->g : n;
+    set_rc(J, grouped_member_topk(J->q, J->k, J->w, J->dtype, J->H, J->d, J->cu[b] + lo, hi - lo, lo,
+                                  J->cu[b], J->topk, J->c, J->mode, t - lo,
+                                  J->out + (size_t)i * J->topk));
+}
+
+/* decode: rows[i] is a request b; writes G rows of topk. */
+static void run_decode_req(job_t *J, int i) {
+    int b = (int)J->rows[i];
+    int n = J->kv_len[b];
+    int G = J->G, H = J->H, d = J->d;
+    int *out = J->out + (size_t)i * G * J->topk;
+    long long key0 = (long long)b * J->n_max;
+    long long m0 = (long long)b * G; /* query rows of q [B*G, H, d] */
+    if (J->mode == ORA_DENSE) {
+        for (int m = 0; m < G; ++m) {
+            int t = n - G + m;
+            cand_t *c = (cand_t *)malloc(sizeof(cand_t) * (size_t)(t + 1));
+            if (!c) { set_rc(J, 2); return; }
+            for (int s = 0; s <= t; ++s) {
+                c[s].score = index_score(J->q, (size_t)(m0 + m) * H * d, J->k, (size_t)(key0 + s) * d,
+                                         J->w + (size_t)(m0 + m) * H, H, d, J->dtype);
+                c[s].pos = s;
+            }
+            select_topk(c, t + 1, J->topk, out + (size_t)m * J->topk);
+            free(c);
+        }
+    } else {
+        for (int m = 0; m < G; ++m)
+            set_rc(J, grouped_member_topk(J->q, J->k, J->w, J->dtype, H, d, m0, G, n - G, key0,
+                                          J->topk, J->c, J->mode, m, out + (size_t)m * J->topk));
+    }
+}
+
+static void *worker(void *arg) {
+    job_t *J = (job_t *)arg;
+    for (;;) {
+        int i = take(J);
+        if (i >= J->nrows) break;
+        if (J->kind == 0) run_dense_row(J, i);
+        else if (J->kind == 1) run_pivot_row(J, i);
+        else run_decode_req(J, i);
+    }
+    return NULL;
+}
+
+static int run_job(job_t *J, int nthreads) {
+    if (nthreads < 1) nthreads = 1;
+    if (nthreads > 256) nthreads = 256;
+    pthread_t th[256];
+    J->next = 0;
+    J->rc = 0;
+    pthread_mutex_init(&J->lock, NULL);
+    int started = 0;
+    for (int i = 0; i < nthreads; ++i)
+        if (pthread_create(&th[i], NULL, worker, J) == 0) ++started;
+    if (!started) worker(J);
+    for (int i = 0; i < started; ++i) pthread_join(th[i], NULL);
+    pthread_mutex_destroy(&J->lock);
+    return J->rc;
+}
+
+static int check_requests(const int *cu, int num_seqs) {
+    if (!cu || num_seqs <= 0 || cu[0] != 0) return 1;
+    for (int b = 0; b < num_seqs; ++b)
+        if (cu[b + 1] < cu[b]) return 1;
+    return 0;
+}
+
+/* Dense top-k for the given global query rows.
+ * q [T,H,d], k [T,d] (bf16 bits or fp32), w [T,H] fp32; cu_seqlens host
+ * [num_seqs+1]; out [nrows, topk] int32. */
+int ora_dense_topk(const void *q, const void *k, const float *w, int dtype, const int *cu_seqlens,
+                   int num_seqs, int H, int d, int topk, const long long *rows, int nrows, int *out,
+                   int nthreads) {
+    if (!q || !k || !w || !out || (nrows > 0 && !rows) || H <= 0 || d <= 0 || topk <= 0) return 1;
+    if (check_requests(cu_seqlens, num_seqs)) return 1;
+    for (int i = 0; i < nrows; ++i)
+        if (rows[i] < 0 || rows[i] >= cu_seqlens[num_seqs]) return 1;
+    job_t J;
+    memset(&J, 0, sizeof J);
+    J.kind = 0; J.q = q; J.k = k; J.w = w; J.dtype = dtype; J.H = H; J.d = d; J.topk = topk;
+    J.cu = cu_seqlens; J.num_seqs = num_seqs; J.rows = rows; J.nrows = nrows; J.out = out;
+    return run_job(&J, nthreads);
+}
+
+/* PIVOT top-k (mode ORA_REUSE or ORA_REFINE) for the given global member
+ * rows; same layouts as ora_dense_topk; g >= 1; Refine needs c >= topk. */
+int ora_pivot_topk(const void *q, const void *k, const float *w, int dtype, const int *cu_seqlens,
+                   int num_seqs, int H, int d, int topk, int g, int c, int mode,
+                   const long long *rows, int nrows, int *out, int nthreads) {
+    if (!q || !k || !w || !out || (nrows > 0 && !rows) || H <= 0 || d <= 0 || topk <= 0 || g <= 0)
+        return 1;
+    if (mode != ORA_REUSE && mode != ORA_REFINE) return 1;
+    if (mode == ORA_REFINE && c < topk) return 1;
+    if (check_requests(cu_seqlens, num_seqs)) return 1;
+    for (int i = 0; i < nrows; ++i)
+        if (rows[i] < 0 || rows[i] >= cu_seqlens[num_seqs]) return 1;
+    job_t J;
+    memset(&J, 0, sizeof J);
+    J.kind = 1; J.q = q; J.k = k; J.w = w; J.dtype = dtype; J.H = H; J.d = d; J.topk = topk;
+    J.g = g; J.c = c; J.mode = mode; J.cu = cu_seqlens; J.num_seqs = num_seqs; J.rows = rows;
+    J.nrows = nrows; J.out = out;
+    return run_job(&J, nthreads);
+}
+
+/* Decode top-k for the given requests.
+ * q [B,G,H,d], kcache [B,n_max,d], w [B,G,H]; kv_len host [B] with
+ * G <= kv_len[b] <= n_max; query m of request b sits at position
+ * kv_len[b]-G+m and the cache already holds the keys of the group.
+ * mode ORA_DENSE, ORA_REUSE or ORA_REFINE (c >= topk); out [nreqs,G,topk]. */
+int ora_decode_topk(const void *q, const void *kcache, const float *w, int dtype, const int *kv_len,
+                    int B, int G, int n_max, int H, int d, int topk, int c, int mode,
+                    const long long *reqs, int nreqs, int *out, int nthreads) {
+    if (!q || !kcache || !w || !kv_len || !out || (nreqs > 0 && !reqs) || H <= 0 || d <= 0 ||
+        topk <= 0 || G <= 0)
+        return 1;
+    if (mode != ORA_DENSE && mode != ORA_REUSE && mode != ORA_REFINE) return 1;
+    if (mode == ORA_REFINE && c < topk) return 1;
+    for (int i = 0; i < nreqs; ++i) {
+        if (reqs[i] < 0 || reqs[i] >= B) return 1;
+        int n = kv_len[reqs[i]];
+        if (n < G || n > n_max) return 1;
+    }
+    job_t J;
+    memset(&J, 0, sizeof J);
+    J.kind = 2; J.q = q; J.k = kcache; J.w = w; J.dtype = dtype; J.H = H; J.d = d; J.topk = topk;
+    J.c = c; J.mode = mode; J.kv_len = kv_len; J.G = G; J.n_max = n_max; J.rows = reqs;
+    J.nrows = nreqs; J.out = out;
+    return run_job(&J, nthreads);
+}
