@@ -1,0 +1,175 @@
+/*
+ * idx.h -- C ABI of the B200 lightning-indexer + top-k library (libidx.so).
+ *
+ * The operation (PIVOT: "Efficient Query-Group Indexing for Token-Level
+ * Sparse Attention", Method, first paragraph, Eq. (1); the equation text is
+ * missing from the page, the DSA lightning-indexer form is used):
+ *
+ *     I[t,s] = sum_j w[t,j] * max(0, q[t,j] . k[s]),     0 <= s <= t,
+ *
+ * with t, s positions inside one request, followed by a per-query top-k:
+ * the k keys of highest score, ties to the lower position, listed in
+ * ascending position and padded with -1 when the prefix holds fewer than k.
+ *
+ * Grouped form (same page, Method, grouping paragraph; Experimental setup;
+ * Abstract): each request is cut into contiguous groups of g queries (the
+ * last one may be shorter, none crosses a request).  A group's proxy query
+ * is the mean of its members' queries (fp32 sum in member order, IEEE
+ * division, rounded to bf16 for bf16 inputs) and its proxy weight the mean
+ * of their w (fp32).  One scan of the group's full prefix (up to its last
+ * member) with the proxy gives
+ *   - IDX_MODE_REUSE:  each member takes the proxy ranking restricted to its
+ *                      own prefix (s <= t_member), first k entries;
+ *   - IDX_MODE_REFINE: the proxy's top-c positions form the candidate set C;
+ *                      each member re-scores C with its own q and w, masks
+ *                      s > t_member and takes its own top-k.
+ *
+ * Decode form (same page, Method, decode paragraph): the G queries of one
+ * MTP step form one group; query m of request b sits at position
+ * kv_len[b] - G + m and the cache already holds the keys of the group.
+ *
+ * Conventions shared by every entry point:
+ *   - All tensor pointers are DEVICE pointers, row-major and contiguous.
+ *     bf16 tensors hold IEEE bfloat16; fp32 tensors IEEE binary32.
+ *   - The caller owns every buffer.  The library never allocates device
+ *     memory on these paths: scratch space is the caller's workspace `ws`
+ *     of at least `*_workspace_size(...)` bytes, 256-byte aligned.
+ *   - Every call is asynchronous on `stream` (NULL = legacy default stream).
+ *     Argument errors are returned synchronously and nothing is launched.
+ *     Device-side anomalies (a bounded wait that ran out, a scratch overflow)
+ *     set a status word inside `ws`; read it with idx_device_status().
+ *   - Indices are request-local positions (int32).  Selected scores, when
+ *     requested, are the fp32 scores the selection used; padding slots get
+ *     index -1 and score -INFINITY.
+ *   - A workspace may be used by one call at a time; calls that share a
+ *     workspace must be ordered on one stream.
+ */
+#ifndef IDX_H
+#define IDX_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st *idx_stream_t; /* same object as cudaStream_t */
+
+typedef enum {
+    IDX_OK = 0,
+    IDX_ERR_INVALID = 1,     /* bad argument (shape, pointer, k > c, ...) */
+    IDX_ERR_UNSUPPORTED = 2, /* valid but not supported (e.g. a request longer than 2^20) */
+    IDX_ERR_WORKSPACE = 3,   /* ws NULL, misaligned or smaller than *_workspace_size() */
+    IDX_ERR_CUDA = 4,        /* a CUDA runtime call failed (launch, memset, ...) */
+    IDX_ERR_TIMEOUT = 5,     /* device: a bounded wait ran out; the results are invalid */
+    IDX_ERR_OVERFLOW = 6     /* device: a scratch buffer overflowed; the results are invalid */
+} idx_status;
+
+typedef enum { IDX_BF16 = 0, IDX_F32 = 1 } idx_dtype;
+
+typedef enum { IDX_MODE_DENSE = 0, IDX_MODE_REUSE = 1, IDX_MODE_REFINE = 2 } idx_mode;
+
+/* ------------------------------------------------------------ prefill */
+
+/* Workspace bytes for idx_dense_topk.  T = total tokens of the packed batch,
+ * num_seqs = number of requests.  Returns 0 for invalid arguments. */
+size_t idx_dense_workspace_size(int T, int H, int d, int topk, int num_seqs, idx_dtype dtype);
+
+/* Dense indexer + top-k over a packed batch of requests (PIVOT page,
+ * Method, first paragraph: every query scores its whole causal prefix).
+ *   q          [T, H, d]  dtype       query of row t, head j
+ *   k          [T, d]     dtype       key of row s (shared by all heads)
+ *   w          [T, H]     fp32        head weights of row t
+ *   cu_seqlens [num_seqs+1] int32     device; request b is rows
+ *                                     cu_seqlens[b] .. cu_seqlens[b+1]-1,
+ *                                     cu_seqlens[0] = 0, cu_seqlens[num_seqs] = T
+ *   out_idx    [T, topk]  int32       selected request-local positions
+ *   out_score  [T, topk]  fp32 or NULL
+ * Requirements: T >= 1, H >= 1, d >= 1 and d % 8 == 0, topk >= 1,
+ * every request no longer than 2^20 tokens (else IDX_ERR_UNSUPPORTED). */
+idx_status idx_dense_topk(const void *q, const void *k, const float *w, const int *cu_seqlens,
+                          int num_seqs, int T, int H, int d, int topk, idx_dtype dtype,
+                          int *out_idx, float *out_score, void *ws, size_t ws_bytes,
+                          idx_stream_t stream);
+
+/* Workspace bytes for idx_pivot_topk (mode REUSE or REFINE). */
+size_t idx_pivot_workspace_size(int T, int H, int d, int topk, int num_seqs, idx_dtype dtype, int g,
+                                int c, idx_mode mode);
+
+/* PIVOT grouped indexer + top-k (Reuse or Refine) over a packed batch.
+ * Same tensors and layouts as idx_dense_topk, plus
+ *   g     group size (>= 1); groups are request-local [m*g, min((m+1)*g, n))
+ *   c     candidate budget for REFINE (c >= topk); ignored for REUSE
+ *   mode  IDX_MODE_REUSE or IDX_MODE_REFINE */
+idx_status idx_pivot_topk(const void *q, const void *k, const float *w, const int *cu_seqlens,
+                          int num_seqs, int T, int H, int d, int topk, idx_dtype dtype, int g, int c,
+                          idx_mode mode, int *out_idx, float *out_score, void *ws, size_t ws_bytes,
+                          idx_stream_t stream);
+
+/* ------------------------------------------------------------- decode */
+
+/* Workspace bytes for idx_decode_topk. */
+size_t idx_decode_workspace_size(int B, int G, int n_max, int H, int d, int topk, int c, idx_mode mode,
+                                 idx_dtype dtype);
+
+/* One decode step of the indexer for B requests of G MTP queries each
+ * (PIVOT page, Method, decode paragraph).
+ *   q       [B, G, H, d]  dtype   query m of request b (position kv_len[b]-G+m)
+ *   kcache  [B, n_max, d] dtype   keys of request b at rows 0 .. kv_len[b]-1
+ *   kv_len  [B] int32             device; G <= kv_len[b] <= n_max (else the
+ *                                 request's rows are written as all -1 and
+ *                                 the status word records IDX_ERR_INVALID)
+ *   w       [B, G, H] fp32
+ *   mode    DENSE (each query scans its own prefix), REUSE or REFINE (the G
+ *           queries are one group; c as in idx_pivot_topk)
+ *   out_idx [B, G, topk] int32, out_score [B, G, topk] fp32 or NULL */
+idx_status idx_decode_topk(const void *q, const void *kcache, const int *kv_len, const float *w,
+                           int B, int G, int n_max, int H, int d, int topk, int c, idx_mode mode,
+                           idx_dtype dtype, int *out_idx, float *out_score, void *ws,
+                           size_t ws_bytes, idx_stream_t stream);
+
+/* ------------------------------------------------------ status, debug */
+
+/* Synchronises `stream`, returns the device status recorded in `ws` by the
+ * last call that used it (IDX_OK, IDX_ERR_TIMEOUT, IDX_ERR_OVERFLOW or
+ * IDX_ERR_INVALID), or IDX_ERR_CUDA if the synchronisation itself failed. */
+idx_status idx_device_status(const void *ws, idx_stream_t stream);
+
+/* A static, human-readable name of a status code. */
+const char *idx_status_string(idx_status s);
+
+/* Test hook: the fp32 scores the selection of the preceding call used, for
+ * a list of scored rows, written as out[i * ld + s] for s = 0 .. bound(i)
+ * (other entries untouched).  `stage` selects what is exported:
+ *   0: dense query rows (rows[] = global query rows; same arguments as
+ *      idx_dense_topk),
+ *   1: PIVOT proxy rows (rows[] = proxy indices in request order; same
+ *      arguments as idx_pivot_topk),
+ *   2: PIVOT Refine member re-scores over the candidate set (rows[] = global
+ *      member rows; out[i * ld + j] is the score of candidate j of the
+ *      member's group, j < c; requires that idx_pivot_topk ran on `ws`).
+ * rows is a DEVICE int32 array.  The scores come from the same kernels and
+ * arithmetic as the selection, so re-selecting on them reproduces out_idx. */
+idx_status idx_debug_scores(int stage, const void *q, const void *k, const float *w,
+                            const int *cu_seqlens, int num_seqs, int T, int H, int d, idx_dtype dtype,
+                            int g, int c, int topk, const int *rows, int nrows, float *out, long long ld,
+                            void *ws, size_t ws_bytes, idx_stream_t stream);
+
+/* Test hook for decode: stage 0 = dense query scores (row i = b*G+m, over
+ * s < kv_len[b]-G+m+1), stage 1 = proxy scores of request b (row i = b),
+ * stage 2 = Refine member re-scores over C (row i = b*G+m, j < c). */
+idx_status idx_debug_decode_scores(int stage, const void *q, const void *kcache, const int *kv_len,
+                                   const float *w, int B, int G, int n_max, int H, int d, int topk,
+                                   int c, idx_mode mode, idx_dtype dtype, float *out, long long ld,
+                                   void *ws, size_t ws_bytes, idx_stream_t stream);
+
+/* Which score kernel serves a shape: 1 = tcgen05 tensor-core kernel,
+ * 0 = SIMT kernel.  (bf16 with H = 64 and d = 128 uses the tensor cores.) */
+int idx_uses_tensor_cores(int H, int d, idx_dtype dtype);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* IDX_H */

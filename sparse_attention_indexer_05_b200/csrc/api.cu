@@ -1,0 +1,513 @@
+// api.cu -- the C ABI of libidx (include/idx.h): argument checks, workspace
+// layout and the launch sequence of each entry point.  No entry point
+// allocates device memory; every call is asynchronous on its stream.
+#include <math.h>
+#include <string.h>
+
+#include "../../include/idx.h"
+#include "common.cuh"
+#include "internal.h"
+
+using namespace idx;
+
+namespace {
+
+constexpr size_t kAlign = 256;
+constexpr size_t kMaxSmem = 232448;  // opt-in shared memory per block on sm_100
+
+size_t up(size_t x, size_t a = kAlign) { return (x + a - 1) / a * a; }
+
+// Candidate buffer capacity per scored row for a streaming top-ksel over
+// rows of at most n keys.  A random key order appends about
+// ksel * (1 + ln(n / ksel)) keys; 1.5x that leaves room for the histogram's
+// coarse threshold.  At least 2*ksel + 256 so that a compaction (cut to
+// ksel) always frees more than one tile's worth of appends; never more
+// than n, which cannot overflow at all.
+unsigned cap_for(long long ksel, long long n) {
+    if (n < 1) n = 1;
+    const long long nn = (long long)up((size_t)n, 32);
+    if (n <= ksel) return (unsigned)nn;
+    const double est = 1.5 * (double)ksel * (1.0 + log((double)n / (double)ksel));
+    long long cap = (long long)up((size_t)ceil(est), 256);
+    if (cap < 2 * ksel + 256) cap = 2 * ksel + 256;
+    if (cap > nn) cap = nn;
+    return (unsigned)cap;
+}
+
+struct Carve {
+    size_t off = 0;
+    size_t take(size_t bytes) {
+        const size_t o = off;
+        off = up(off + bytes);
+        return o;
+    }
+};
+
+size_t esize(idx_dtype dt) { return dt == IDX_F32 ? 4 : 2; }
+
+long long nbound(int T) { return T < kMaxLen ? T : kMaxLen; }
+
+struct PrefillWs {
+    PlanLayout pl;
+    long long R;          // scored rows (queries or proxies, upper bound)
+    unsigned cap, ksel;
+    size_t status, plan, slot, qbar, wbar, cnt, buf, cand, msc, total;
+};
+
+PrefillWs prefill_ws(int T, int H, int d, int topk, int S, idx_dtype dt, int g, int c, idx_mode mode) {
+    PrefillWs L{};
+    const bool pivot = mode != IDX_MODE_DENSE;
+    L.R = pivot ? ((long long)T + (long long)S * (g - 1)) / g : T;
+    L.pl.S = S;
+    L.pl.maxblk = (int)((L.R + RB - 1) / RB + S);
+    L.pl.maxtiles = (int)(nbound(T) / KT + 1);
+    L.ksel = mode == IDX_MODE_REUSE ? (unsigned)(topk + g - 1) : mode == IDX_MODE_REFINE ? (unsigned)c
+                                                                                       : (unsigned)topk;
+    L.cap = cap_for(L.ksel, nbound(T));
+    Carve cv;
+    L.status = cv.take(16);
+    L.plan = cv.take(L.pl.words() * 4);
+    L.slot = cv.take((size_t)(L.R > T ? L.R : T) * 4);
+    L.qbar = pivot ? cv.take((size_t)L.R * H * d * esize(dt)) : 0;
+    L.wbar = pivot ? cv.take((size_t)L.R * H * 4) : 0;
+    L.cnt = cv.take((size_t)L.R * 4);
+    L.buf = cv.take((size_t)L.R * L.cap * 8);
+    L.cand = mode == IDX_MODE_REFINE ? cv.take((size_t)L.R * c * 4) : 0;
+    L.msc = mode == IDX_MODE_REFINE ? cv.take((size_t)T * c * 4) : 0;
+    L.total = cv.off;
+    return L;
+}
+
+struct DecodeWs {
+    size_t status, qbar, wbar, spill, cand, msc, total;
+};
+
+DecodeWs decode_ws(int B, int G, int n_max, int H, int d, int c, idx_mode mode, idx_dtype dt) {
+    DecodeWs L{};
+    Carve cv;
+    const int rows = mode == IDX_MODE_DENSE ? B * G : B;
+    L.status = cv.take(16);
+    L.qbar = mode != IDX_MODE_DENSE ? cv.take((size_t)B * H * d * esize(dt)) : 0;
+    L.wbar = mode != IDX_MODE_DENSE ? cv.take((size_t)B * H * 4) : 0;
+    L.spill = cv.take((size_t)rows * n_max * 4);
+    L.cand = mode == IDX_MODE_REFINE ? cv.take((size_t)B * c * 4) : 0;
+    L.msc = mode == IDX_MODE_REFINE ? cv.take((size_t)B * G * c * 4) : 0;
+    L.total = cv.off;
+    return L;
+}
+
+bool shape_ok(int H, int d, idx_dtype dt) {
+    if (H < 1 || d < 8 || d % 8 != 0 || (dt != IDX_BF16 && dt != IDX_F32)) return false;
+    return true;
+}
+
+bool path_ok(int H, int d, idx_dtype dt) {
+    return tc_supported(H, d, (int)dt) || simt_smem_bytes(H, d, (int)dt) <= kMaxSmem;
+}
+
+idx_status cuda_st(cudaError_t e) { return e == cudaSuccess ? IDX_OK : IDX_ERR_CUDA; }
+
+#define TRY_CUDA(x)                                  \
+    do {                                             \
+        cudaError_t e_ = (x);                        \
+        if (e_ != cudaSuccess) return IDX_ERR_CUDA;  \
+    } while (0)
+
+__global__ void scatter_slots(const int *rows, int nrows, int R, int *slot, unsigned *status) {
+    const int i = blockIdx.x * blockDim.x + threadIdx.x;
+    if (i >= nrows) return;
+    const int r = rows[i];
+    if (r < 0 || r >= R) {
+        atomicOr(status, ST_INVALID);
+        return;
+    }
+    slot[r] = i;
+}
+
+__global__ void copy_rows(const float *src, long long src_ld, const int *rows, int nrows, int R, int ncols,
+                          float *dst, long long ld, unsigned *status) {
+    const int i = blockIdx.y;
+    if (i >= nrows) return;
+    const int r = rows[i];
+    if (r < 0 || r >= R) {
+        if (threadIdx.x == 0 && blockIdx.x == 0) atomicOr(status, ST_INVALID);
+        return;
+    }
+    for (int j = blockIdx.x * blockDim.x + threadIdx.x; j < ncols; j += gridDim.x * blockDim.x)
+        dst[(long long)i * ld + j] = src[(long long)r * src_ld + j];
+}
+
+struct Prefill {
+    const void *q, *k;
+    const float *w;
+    const int *cu;
+    int S, T, H, d, topk;
+    idx_dtype dt;
+    int g, c;
+    idx_mode mode;
+    char *ws;
+    PrefillWs L;
+    cudaStream_t st;
+
+    unsigned *status() const { return reinterpret_cast<unsigned *>(ws + L.status); }
+    int *plan() const { return reinterpret_cast<int *>(ws + L.plan); }
+
+    ScoreArgs score_args(bool proxies) const {
+        ScoreArgs a{};
+        a.q = proxies ? (const void *)(ws + L.qbar) : q;
+        a.k = k;
+        a.w = proxies ? reinterpret_cast<const float *>(ws + L.wbar) : w;
+        a.cu = cu;
+        a.S = S; a.T = T; a.H = H; a.d = d;
+        a.g = proxies ? g : 1;
+        a.plan = plan();
+        a.pl = L.pl;
+        a.sink = SINK_FILTER;
+        a.buf = reinterpret_cast<unsigned long long *>(ws + L.buf);
+        a.cap = L.cap;
+        a.ksel = L.ksel;
+        a.cnt = reinterpret_cast<unsigned *>(ws + L.cnt);
+        a.status = status();
+        return a;
+    }
+
+    cudaError_t score(const ScoreArgs &a) const {
+        // the persistent score kernels pull row blocks from plan[3]
+        cudaError_t e = cudaMemsetAsync(plan() + 3, 0, 4, st);
+        if (e != cudaSuccess) return e;
+        return tc_supported(H, d, (int)dt) ? launch_score_tc(a, st) : launch_score_simt(a, (int)dt, st);
+    }
+
+    cudaError_t prepare() const {
+        cudaError_t e = cudaMemsetAsync(status(), 0, 4, st);
+        if (e != cudaSuccess) return e;
+        e = launch_plan(cu, S, T, mode == IDX_MODE_DENSE ? 1 : g, plan(), L.pl, status(), st);
+        if (e != cudaSuccess) return e;
+        if (mode != IDX_MODE_DENSE)
+            e = launch_proxy(q, w, cu, S, T, H, d, g, (int)dt, plan(), L.pl, ws + L.qbar,
+                             reinterpret_cast<float *>(ws + L.wbar), (int)L.R, st);
+        return e;
+    }
+
+    SelectArgs select_args(int kind, int nrows, int kk, int *oi, float *os) const {
+        SelectArgs s{};
+        s.kind = kind;
+        s.nrows = nrows;
+        s.k = kk;
+        s.out_idx = oi;
+        s.out_score = os;
+        s.cu = cu;
+        s.S = S;
+        s.g = mode == IDX_MODE_DENSE ? 1 : g;
+        s.plan = plan();
+        s.pl = L.pl;
+        s.buf = reinterpret_cast<const unsigned long long *>(ws + L.buf);
+        s.cap = L.cap;
+        s.cnt = reinterpret_cast<const unsigned *>(ws + L.cnt);
+        s.c = c;
+        s.cand = reinterpret_cast<const int *>(ws + L.cand);
+        s.scores = reinterpret_cast<const float *>(ws + L.msc);
+        s.ld = c;
+        s.bitmap_words = (int)(nbound(T) / 32 + 1);
+        s.status = status();
+        return s;
+    }
+
+    GatherArgs gather_args() const {
+        GatherArgs a{};
+        a.q = q; a.k = k; a.w = w;
+        a.cand = reinterpret_cast<const int *>(ws + L.cand);
+        a.c = c; a.H = H; a.d = d;
+        a.nitems = (int)L.R;
+        a.mode = 0;
+        a.cu = cu; a.S = S; a.g = g;
+        a.plan = plan(); a.pl = L.pl;
+        a.out = reinterpret_cast<float *>(ws + L.msc);
+        a.status = status();
+        return a;
+    }
+};
+
+idx_status check_prefill(const void *q, const void *k, const float *w, const int *cu, int S, int T, int H,
+                         int d, int topk, idx_dtype dt, const int *out_idx, void *ws, size_t ws_bytes,
+                         size_t need) {
+    if (!q || !k || !w || !cu || !out_idx) return IDX_ERR_INVALID;
+    if (S < 1 || T < 1 || topk < 1 || !shape_ok(H, d, dt)) return IDX_ERR_INVALID;
+    if (!path_ok(H, d, dt)) return IDX_ERR_UNSUPPORTED;
+    if (!ws || (reinterpret_cast<uintptr_t>(ws) % kAlign) != 0 || ws_bytes < need) return IDX_ERR_WORKSPACE;
+    return IDX_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *idx_status_string(idx_status s) {
+    switch (s) {
+    case IDX_OK: return "IDX_OK";
+    case IDX_ERR_INVALID: return "IDX_ERR_INVALID";
+    case IDX_ERR_UNSUPPORTED: return "IDX_ERR_UNSUPPORTED";
+    case IDX_ERR_WORKSPACE: return "IDX_ERR_WORKSPACE";
+    case IDX_ERR_CUDA: return "IDX_ERR_CUDA";
+    case IDX_ERR_TIMEOUT: return "IDX_ERR_TIMEOUT";
+    case IDX_ERR_OVERFLOW: return "IDX_ERR_OVERFLOW";
+    }
+    return "IDX_ERR_UNKNOWN";
+}
+
+int idx_uses_tensor_cores(int H, int d, idx_dtype dtype) { return tc_supported(H, d, (int)dtype) ? 1 : 0; }
+
+size_t idx_dense_workspace_size(int T, int H, int d, int topk, int num_seqs, idx_dtype dtype) {
+    if (T < 1 || num_seqs < 1 || topk < 1 || !shape_ok(H, d, dtype)) return 0;
+    return prefill_ws(T, H, d, topk, num_seqs, dtype, 1, topk, IDX_MODE_DENSE).total;
+}
+
+idx_status idx_dense_topk(const void *q, const void *k, const float *w, const int *cu_seqlens, int num_seqs,
+                          int T, int H, int d, int topk, idx_dtype dtype, int *out_idx, float *out_score,
+                          void *ws, size_t ws_bytes, idx_stream_t stream) {
+    const size_t need = idx_dense_workspace_size(T, H, d, topk, num_seqs, dtype);
+    idx_status s = check_prefill(q, k, w, cu_seqlens, num_seqs, T, H, d, topk, dtype, out_idx, ws, ws_bytes,
+                                 need);
+    if (s != IDX_OK) return s;
+    Prefill P{q, k, w, cu_seqlens, num_seqs, T, H, d, topk, dtype, 1, topk, IDX_MODE_DENSE,
+              static_cast<char *>(ws), prefill_ws(T, H, d, topk, num_seqs, dtype, 1, topk, IDX_MODE_DENSE),
+              reinterpret_cast<cudaStream_t>(stream)};
+    TRY_CUDA(P.prepare());
+    TRY_CUDA(P.score(P.score_args(false)));
+    return cuda_st(launch_select(P.select_args(SEL_DENSE_CAND, T, topk, out_idx, out_score), P.st));
+}
+
+size_t idx_pivot_workspace_size(int T, int H, int d, int topk, int num_seqs, idx_dtype dtype, int g, int c,
+                                idx_mode mode) {
+    if (T < 1 || num_seqs < 1 || topk < 1 || g < 1 || !shape_ok(H, d, dtype)) return 0;
+    if (mode != IDX_MODE_REUSE && mode != IDX_MODE_REFINE) return 0;
+    if (mode == IDX_MODE_REFINE && c < topk) return 0;
+    return prefill_ws(T, H, d, topk, num_seqs, dtype, g, c, mode).total;
+}
+
+idx_status idx_pivot_topk(const void *q, const void *k, const float *w, const int *cu_seqlens, int num_seqs,
+                          int T, int H, int d, int topk, idx_dtype dtype, int g, int c, idx_mode mode,
+                          int *out_idx, float *out_score, void *ws, size_t ws_bytes, idx_stream_t stream) {
+    if (g < 1 || (mode != IDX_MODE_REUSE && mode != IDX_MODE_REFINE)) return IDX_ERR_INVALID;
+    if (mode == IDX_MODE_REFINE && c < topk) return IDX_ERR_INVALID;
+    if (mode == IDX_MODE_REUSE) c = topk;
+    const size_t need = idx_pivot_workspace_size(T, H, d, topk, num_seqs, dtype, g, c, mode);
+    idx_status s = check_prefill(q, k, w, cu_seqlens, num_seqs, T, H, d, topk, dtype, out_idx, ws, ws_bytes,
+                                 need);
+    if (s != IDX_OK) return s;
+    Prefill P{q, k, w, cu_seqlens, num_seqs, T, H, d, topk, dtype, g, c, mode, static_cast<char *>(ws),
+              prefill_ws(T, H, d, topk, num_seqs, dtype, g, c, mode), reinterpret_cast<cudaStream_t>(stream)};
+    TRY_CUDA(P.prepare());
+    TRY_CUDA(P.score(P.score_args(true)));
+    if (mode == IDX_MODE_REUSE)
+        return cuda_st(launch_select(P.select_args(SEL_REUSE_CAND, T, topk, out_idx, out_score), P.st));
+    int *cand = reinterpret_cast<int *>(P.ws + P.L.cand);
+    TRY_CUDA(launch_select(P.select_args(SEL_PROXY_TO_C, (int)P.L.R, c, cand, nullptr), P.st));
+    const GatherArgs ga = P.gather_args();
+    TRY_CUDA(tc_supported(H, d, (int)dtype) ? launch_gather_tc(ga, P.st) : launch_gather_simt(ga, (int)dtype, P.st));
+    return cuda_st(launch_select(P.select_args(SEL_MEMBER_SCORES, T, topk, out_idx, out_score), P.st));
+}
+
+size_t idx_decode_workspace_size(int B, int G, int n_max, int H, int d, int topk, int c, idx_mode mode,
+                                 idx_dtype dtype) {
+    if (B < 1 || G < 1 || G > RB || n_max < G || n_max > kMaxLen || topk < 1 || !shape_ok(H, d, dtype))
+        return 0;
+    if (mode != IDX_MODE_DENSE && mode != IDX_MODE_REUSE && mode != IDX_MODE_REFINE) return 0;
+    if (mode == IDX_MODE_REFINE && c < topk) return 0;
+    return decode_ws(B, G, n_max, H, d, c, mode, dtype).total;
+}
+
+namespace {
+
+struct Decode {
+    const void *q, *kc;
+    const int *kv;
+    const float *w;
+    int B, G, n_max, H, d, topk, c;
+    idx_mode mode;
+    idx_dtype dt;
+    char *ws;
+    DecodeWs L;
+    cudaStream_t st;
+
+    unsigned *status() const { return reinterpret_cast<unsigned *>(ws + L.status); }
+
+    DecodeArgs dargs(bool proxy, float *spill) const {
+        DecodeArgs a{};
+        a.q = proxy ? (const void *)(ws + L.qbar) : q;
+        a.kc = kc;
+        a.w = proxy ? reinterpret_cast<const float *>(ws + L.wbar) : w;
+        a.kv_len = kv;
+        a.B = B; a.G = G; a.Gq = proxy ? 1 : G; a.n_max = n_max; a.H = H; a.d = d;
+        a.chunk_tiles = 64;
+        a.spill = spill;
+        a.status = status();
+        return a;
+    }
+    cudaError_t scan(const DecodeArgs &a) const {
+        return tc_supported(H, d, (int)dt) && (a.Gq * H) <= 256 ? launch_decode_tc(a, st)
+                                                                : launch_decode_simt(a, (int)dt, st);
+    }
+    SelectArgs sargs(int kind, int nrows, int kk, int *oi, float *os, const float *scores, long long ld) const {
+        SelectArgs s{};
+        s.kind = kind; s.nrows = nrows; s.k = kk; s.out_idx = oi; s.out_score = os;
+        s.scores = scores; s.ld = ld;
+        s.cand = reinterpret_cast<const int *>(ws + L.cand);
+        s.c = c;
+        s.kv_len = kv; s.G = G; s.n_max = n_max;
+        s.bitmap_words = n_max / 32 + 1;
+        s.status = status();
+        return s;
+    }
+    GatherArgs gargs() const {
+        GatherArgs a{};
+        a.q = q; a.k = kc; a.w = w;
+        a.cand = reinterpret_cast<const int *>(ws + L.cand);
+        a.c = c; a.H = H; a.d = d;
+        a.nitems = B;
+        a.mode = 1;
+        a.G = G; a.n_max = n_max; a.kv_len = kv;
+        a.out = reinterpret_cast<float *>(ws + L.msc);
+        a.status = status();
+        return a;
+    }
+};
+
+idx_status check_decode(const void *q, const void *kc, const int *kv, const float *w, int B, int G, int n_max,
+                        int H, int d, int topk, int c, idx_mode mode, idx_dtype dt, const int *out_idx,
+                        void *ws, size_t ws_bytes) {
+    if (!q || !kc || !kv || !w || !out_idx) return IDX_ERR_INVALID;
+    if (B < 1 || G < 1 || n_max < G || topk < 1 || !shape_ok(H, d, dt)) return IDX_ERR_INVALID;
+    if (mode != IDX_MODE_DENSE && mode != IDX_MODE_REUSE && mode != IDX_MODE_REFINE) return IDX_ERR_INVALID;
+    if (mode == IDX_MODE_REFINE && c < topk) return IDX_ERR_INVALID;
+    if (G > RB || n_max > kMaxLen || !path_ok(H, d, dt)) return IDX_ERR_UNSUPPORTED;
+    const size_t need = idx_decode_workspace_size(B, G, n_max, H, d, topk, c, mode, dt);
+    if (!ws || (reinterpret_cast<uintptr_t>(ws) % kAlign) != 0 || ws_bytes < need) return IDX_ERR_WORKSPACE;
+    return IDX_OK;
+}
+
+}  // namespace
+
+idx_status idx_decode_topk(const void *q, const void *kcache, const int *kv_len, const float *w, int B, int G,
+                           int n_max, int H, int d, int topk, int c, idx_mode mode, idx_dtype dtype,
+                           int *out_idx, float *out_score, void *ws, size_t ws_bytes, idx_stream_t stream) {
+    idx_status s = check_decode(q, kcache, kv_len, w, B, G, n_max, H, d, topk, c, mode, dtype, out_idx, ws,
+                                ws_bytes);
+    if (s != IDX_OK) return s;
+    Decode D{q, kcache, kv_len, w, B, G, n_max, H, d, topk, c, mode, dtype, static_cast<char *>(ws),
+             decode_ws(B, G, n_max, H, d, c, mode, dtype), reinterpret_cast<cudaStream_t>(stream)};
+    TRY_CUDA(cudaMemsetAsync(D.status(), 0, 4, D.st));
+    float *spill = reinterpret_cast<float *>(D.ws + D.L.spill);
+    if (mode == IDX_MODE_DENSE) {
+        TRY_CUDA(D.scan(D.dargs(false, spill)));
+        return cuda_st(launch_select(D.sargs(SEL_DEC_DENSE, B * G, topk, out_idx, out_score, spill, n_max), D.st));
+    }
+    TRY_CUDA(launch_decode_proxy(q, w, B, G, H, d, (int)dtype, D.ws + D.L.qbar,
+                                 reinterpret_cast<float *>(D.ws + D.L.wbar), D.st));
+    TRY_CUDA(D.scan(D.dargs(true, spill)));
+    if (mode == IDX_MODE_REUSE)
+        return cuda_st(launch_select(D.sargs(SEL_DEC_REUSE, B * G, topk, out_idx, out_score, spill, n_max), D.st));
+    int *cand = reinterpret_cast<int *>(D.ws + D.L.cand);
+    TRY_CUDA(launch_select(D.sargs(SEL_DEC_PROXY_TO_C, B, c, cand, nullptr, spill, n_max), D.st));
+    const GatherArgs ga = D.gargs();
+    TRY_CUDA(tc_supported(H, d, (int)dtype) && G * H <= 256 ? launch_gather_tc(ga, D.st)
+                                                            : launch_gather_simt(ga, (int)dtype, D.st));
+    const float *msc = reinterpret_cast<const float *>(D.ws + D.L.msc);
+    return cuda_st(launch_select(D.sargs(SEL_DEC_MEMBER, B * G, topk, out_idx, out_score, msc, c), D.st));
+}
+
+idx_status idx_device_status(const void *ws, idx_stream_t stream) {
+    if (!ws) return IDX_ERR_WORKSPACE;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    unsigned h = 0;
+    if (cudaMemcpyAsync(&h, ws, 4, cudaMemcpyDeviceToHost, st) != cudaSuccess) return IDX_ERR_CUDA;
+    if (cudaStreamSynchronize(st) != cudaSuccess) return IDX_ERR_CUDA;
+    if (h & ST_TIMEOUT) return IDX_ERR_TIMEOUT;
+    if (h & ST_OVERFLOW) return IDX_ERR_OVERFLOW;
+    if (h & ST_INVALID) return IDX_ERR_INVALID;
+    return IDX_OK;
+}
+
+idx_status idx_debug_scores(int stage, const void *q, const void *k, const float *w, const int *cu_seqlens,
+                            int num_seqs, int T, int H, int d, idx_dtype dtype, int g, int c, int topk,
+                            const int *rows, int nrows, float *out, long long ld, void *ws, size_t ws_bytes,
+                            idx_stream_t stream) {
+    if (!rows || !out || nrows < 0 || ld < 1 || stage < 0 || stage > 2) return IDX_ERR_INVALID;
+    const idx_mode mode = stage == 0 ? IDX_MODE_DENSE : (stage == 2 || c > 0 ? IDX_MODE_REFINE : IDX_MODE_REUSE);
+    const int gg = stage == 0 ? 1 : g;
+    const int cc = mode == IDX_MODE_REFINE ? c : topk;
+    if (gg < 1 || (mode == IDX_MODE_REFINE && cc < topk)) return IDX_ERR_INVALID;
+    const size_t need = mode == IDX_MODE_DENSE
+                            ? idx_dense_workspace_size(T, H, d, topk, num_seqs, dtype)
+                            : idx_pivot_workspace_size(T, H, d, topk, num_seqs, dtype, gg, cc, mode);
+    int dummy = 0;
+    idx_status s = check_prefill(q, k, w, cu_seqlens, num_seqs, T, H, d, topk, dtype, &dummy, ws, ws_bytes, need);
+    if (s != IDX_OK) return s;
+    Prefill P{q, k, w, cu_seqlens, num_seqs, T, H, d, topk, dtype, gg, cc, mode, static_cast<char *>(ws),
+              prefill_ws(T, H, d, topk, num_seqs, dtype, gg, cc, mode), reinterpret_cast<cudaStream_t>(stream)};
+    if (nrows == 0) return IDX_OK;
+    if (stage == 2) {
+        TRY_CUDA(cudaMemsetAsync(P.status(), 0, 4, P.st));
+        for (int r0 = 0; r0 < nrows; r0 += 65535) {
+            const int nr = nrows - r0 < 65535 ? nrows - r0 : 65535;
+            dim3 grid((c + 255) / 256 < 64 ? (c + 255) / 256 : 64, nr);
+            copy_rows<<<grid, 256, 0, P.st>>>(reinterpret_cast<const float *>(P.ws + P.L.msc), c, rows + r0, nr,
+                                              T, c, out + (long long)r0 * ld, ld, P.status());
+            TRY_CUDA(cudaGetLastError());
+        }
+        return IDX_OK;
+    }
+    TRY_CUDA(P.prepare());
+    int *slot = reinterpret_cast<int *>(P.ws + P.L.slot);
+    const long long R = stage == 0 ? T : P.L.R;
+    TRY_CUDA(cudaMemsetAsync(slot, 0xFF, (size_t)R * 4, P.st));
+    scatter_slots<<<(nrows + 255) / 256, 256, 0, P.st>>>(rows, nrows, (int)R, slot, P.status());
+    TRY_CUDA(cudaGetLastError());
+    ScoreArgs a = P.score_args(stage == 1);
+    a.sink = SINK_SPILL;
+    a.spill = out;
+    a.ld = ld;
+    a.slot_of_row = slot;
+    return cuda_st(P.score(a));
+}
+
+idx_status idx_debug_decode_scores(int stage, const void *q, const void *kcache, const int *kv_len, const float *w,
+                                   int B, int G, int n_max, int H, int d, int topk, int c, idx_mode mode,
+                                   idx_dtype dtype, float *out, long long ld, void *ws, size_t ws_bytes,
+                                   idx_stream_t stream) {
+    if (!out || ld < 1 || stage < 0 || stage > 2) return IDX_ERR_INVALID;
+    if (stage == 0) mode = IDX_MODE_DENSE;
+    if (stage == 2 && mode != IDX_MODE_REFINE) return IDX_ERR_INVALID;
+    if (stage == 1 && mode == IDX_MODE_DENSE) return IDX_ERR_INVALID;
+    int dummy = 0;
+    idx_status s = check_decode(q, kcache, kv_len, w, B, G, n_max, H, d, topk, c, mode, dtype, &dummy, ws, ws_bytes);
+    if (s != IDX_OK) return s;
+    Decode D{q, kcache, kv_len, w, B, G, n_max, H, d, topk, c, mode, dtype, static_cast<char *>(ws),
+             decode_ws(B, G, n_max, H, d, c, mode, dtype), reinterpret_cast<cudaStream_t>(stream)};
+    TRY_CUDA(cudaMemsetAsync(D.status(), 0, 4, D.st));
+    if (stage == 2) {
+        // member re-scores of the preceding Refine call: rows b*G+m
+        const float *msc = reinterpret_cast<const float *>(D.ws + D.L.msc);
+        for (int r = 0; r < B * G; ++r)
+            TRY_CUDA(cudaMemcpyAsync(out + (long long)r * ld, msc + (long long)r * c, (size_t)c * 4,
+                                     cudaMemcpyDeviceToDevice, D.st));
+        return IDX_OK;
+    }
+    if (stage == 1)
+        TRY_CUDA(launch_decode_proxy(q, w, B, G, H, d, (int)dtype, D.ws + D.L.qbar,
+                                     reinterpret_cast<float *>(D.ws + D.L.wbar), D.st));
+    DecodeArgs a = D.dargs(stage == 1, out);
+    a.spill = out;
+    // the scan kernels write row r at spill + r * n_max; a separate ld needs a staging copy
+    if (ld == n_max) return cuda_st(D.scan(a));
+    float *spill = reinterpret_cast<float *>(D.ws + D.L.spill);
+    a.spill = spill;
+    TRY_CUDA(D.scan(a));
+    const int rows = stage == 1 ? B : B * G;
+    for (int r = 0; r < rows; ++r)
+        TRY_CUDA(cudaMemcpyAsync(out + (long long)r * ld, spill + (long long)r * n_max, (size_t)n_max * 4,
+                                 cudaMemcpyDeviceToDevice, D.st));
+    return IDX_OK;
+}
+
+}  // extern "C"

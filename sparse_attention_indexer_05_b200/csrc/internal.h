@@ -1,0 +1,145 @@
+// internal.h -- launch-side declarations shared by the libidx sources.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace idx {
+
+constexpr int RB = 8;           // scored rows per row block (score kernels)
+constexpr int KT = 128;         // keys per key tile
+constexpr int kMaxLen = 1 << 20;  // longest supported request / cache
+
+// Plan area (int32 words at the start of a prefill workspace plan region):
+//   [0] valid flag (1 = cu_seqlens passed the device checks)
+//   [1] number of row blocks      [2] number of scored rows
+//   [3] work counter (persistent score kernels)
+//   [4 .. 4+S]          rp[b]: first scored row of request b (S = num_seqs)
+//   [5+S .. 5+2S]       bp[b]: first row block of request b
+//   [6+2S .. +maxblk)   order: row blocks, longest key range first
+//   then (maxtiles+1)   per-tile-count histogram (plan scratch)
+struct PlanLayout {
+    int S, maxblk, maxtiles;
+    __host__ __device__ size_t words() const {
+        return (size_t)6 + 2 * (size_t)S + (size_t)maxblk + (size_t)maxtiles + 1;
+    }
+    __host__ __device__ int rp() const { return 4; }
+    __host__ __device__ int bp() const { return 5 + S; }
+    __host__ __device__ int order() const { return 6 + 2 * S; }
+    __host__ __device__ int hist() const { return 6 + 2 * S + maxblk; }
+};
+
+enum Sink { SINK_FILTER = 0, SINK_SPILL = 1 };
+
+// A prefill score pass: rows of `q` (queries, or PIVOT proxies when g > 1)
+// against the keys of their request, streamed into a sink.
+struct ScoreArgs {
+    const void *q;       // [R, H, d] scored rows
+    const void *k;       // [T, d] keys
+    const float *w;      // [R, H]
+    const int *cu;       // cu_seqlens [S+1] (device)
+    int S, T, H, d, g;   // g = 1: row i of request b is query i; g > 1: proxy i
+    const int *plan;     // plan area
+    PlanLayout pl;
+    int sink;
+    // SINK_FILTER: candidate buffers [R, cap] and counts [R]
+    unsigned long long *buf;
+    unsigned cap, ksel;
+    unsigned *cnt;
+    // SINK_SPILL: out[slot * ld + s] for rows with slot_of_row[row] >= 0
+    float *spill;
+    long long ld;
+    const int *slot_of_row;
+    unsigned *status;
+};
+
+// decode score pass (one row block = the G queries of one request, or its proxy)
+struct DecodeArgs {
+    const void *q;       // [B, Gq, H, d] rows scored (Gq = G queries, or 1 proxy)
+    const void *kc;      // [B, n_max, d]
+    const float *w;      // [B, Gq, H]
+    const int *kv_len;   // [B]
+    int B, G, Gq, n_max, H, d;
+    int chunk_tiles;     // key tiles per work item
+    float *spill;        // [B*Gq, n_max]
+    unsigned *status;
+    unsigned *work;
+};
+
+// Refine re-score pass: member rows against the gathered candidate keys.
+struct GatherArgs {
+    const void *q;       // [rows, H, d] member queries
+    const void *k;       // [*, d] keys (prefill: packed keys; decode: cache)
+    const float *w;      // [rows, H]
+    const int *cand;     // [P, c] candidate positions (ascending, -1 padded)
+    int c, H, d;
+    int nitems;          // work items (one per group, members <= RB)
+    // mapping of a work item -> (first member row, members, candidate row, key base)
+    int mode;            // 0: prefill (cu, g, plan rp of proxies), 1: decode (B, G, n_max)
+    const int *cu;
+    int S, g;
+    const int *plan;
+    PlanLayout pl;
+    int G, n_max;
+    const int *kv_len;
+    float *out;          // [rows, c] member scores
+    unsigned *status;
+};
+
+// select pass descriptors
+enum SelKind {
+    SEL_DENSE_CAND = 0,     // out row = query row; candidates of that row
+    SEL_REUSE_CAND = 1,     // out row = member; candidates of its group's proxy row
+    SEL_PROXY_TO_C = 2,     // out = candidate set of proxy row (k = c), positions only
+    SEL_MEMBER_SCORES = 3,  // out row = member; scores over its group's candidate set
+    SEL_DEC_DENSE = 4,      // decode: spill row (b, m)
+    SEL_DEC_REUSE = 5,      // decode: proxy spill row b restricted to member m
+    SEL_DEC_PROXY_TO_C = 6, // decode: candidate set of request b
+    SEL_DEC_MEMBER = 7      // decode: member scores over the candidate set
+};
+
+struct SelectArgs {
+    int kind;
+    int nrows;               // CTAs / output rows
+    int k;                   // entries selected per row
+    int *out_idx;            // [nrows, k]
+    float *out_score;        // [nrows, k] or NULL
+    // prefill context
+    const int *cu;
+    int S, g;
+    const int *plan;
+    PlanLayout pl;
+    const unsigned long long *buf;
+    unsigned cap;
+    const unsigned *cnt;
+    // score-row sources
+    const float *scores;     // spill or member scores
+    long long ld;
+    const int *cand;         // candidate sets [P, c]
+    int c;
+    // decode context
+    const int *kv_len;
+    int G, n_max;
+    int bitmap_words;        // shared bitmap capacity (words)
+    unsigned *status;
+};
+
+// ---- launchers (each returns cudaSuccess or the launch error)
+cudaError_t launch_plan(const int *cu, int S, int T, int g, int *plan, const PlanLayout &pl,
+                        unsigned *status, cudaStream_t st);
+cudaError_t launch_score_simt(const ScoreArgs &a, int dtype, cudaStream_t st);
+cudaError_t launch_score_tc(const ScoreArgs &a, cudaStream_t st);
+cudaError_t launch_decode_simt(const DecodeArgs &a, int dtype, cudaStream_t st);
+cudaError_t launch_decode_tc(const DecodeArgs &a, cudaStream_t st);
+cudaError_t launch_gather_simt(const GatherArgs &a, int dtype, cudaStream_t st);
+cudaError_t launch_gather_tc(const GatherArgs &a, cudaStream_t st);
+cudaError_t launch_select(const SelectArgs &a, cudaStream_t st);
+cudaError_t launch_proxy(const void *q, const float *w, const int *cu, int S, int T, int H, int d,
+                         int g, int dtype, const int *plan, const PlanLayout &pl, void *qbar,
+                         float *wbar, int max_proxies, cudaStream_t st);
+cudaError_t launch_decode_proxy(const void *q, const float *w, int B, int G, int H, int d, int dtype,
+                                void *qbar, float *wbar, cudaStream_t st);
+size_t simt_smem_bytes(int H, int d, int dtype);
+bool tc_supported(int H, int d, int dtype);
+
+}  // namespace idx

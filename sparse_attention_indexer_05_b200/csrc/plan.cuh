@@ -1,0 +1,62 @@
+// plan.cuh -- device helpers that map row blocks and rows to requests.
+#pragma once
+
+#include "internal.h"
+
+namespace idx {
+
+// first index i in a[0..n] (sorted, non-decreasing) with a[i] > v, minus 1:
+// the last i with a[i] <= v (callers guarantee a[0] <= v < a[n]).
+__device__ __forceinline__ int find_seg(const int *a, int n, long long v) {
+    int lo = 0, hi = n;  // answer in [0, n-1]
+    while (hi - lo > 1) {
+        int mid = (lo + hi) >> 1;
+        if ((long long)a[mid] <= v) lo = mid; else hi = mid;
+    }
+    return lo;
+}
+
+// Number of scored rows of a request of n tokens: queries (g = 1) or proxies.
+__device__ __forceinline__ int rows_of(int n, int g) { return g == 1 ? n : (n + g - 1) / g; }
+
+// Causal bound (request-local, inclusive) of scored row i of a request of n
+// tokens: a query sees s <= i; proxy i (group [i*g, min((i+1)*g, n)))
+// sees the prefix of its last member.
+__device__ __forceinline__ int row_bound(int i, int n, int g) {
+    if (g == 1) return i;
+    long long e = (long long)(i + 1) * g;
+    return (int)((e < n ? e : n) - 1);
+}
+
+struct BlockInfo {
+    int b;        // request
+    int row0;     // first scored row (global index into the scored tensor)
+    int nrows;    // valid rows in the block (<= RB)
+    long long key0;  // first key row of the request
+    int n;        // request length
+    int i0;       // request-local index of the first scored row
+    int maxbound; // bound of the last valid row
+    int ntiles;   // key tiles covering 0..maxbound
+};
+
+__device__ __forceinline__ BlockInfo block_info(const int *plan, const PlanLayout &pl, const int *cu,
+                                                int g, int blk) {
+    BlockInfo bi;
+    const int *rp = plan + pl.rp();
+    const int *bp = plan + pl.bp();
+    bi.b = find_seg(bp, pl.S, blk);
+    const int j = blk - bp[bi.b];
+    bi.n = cu[bi.b + 1] - cu[bi.b];
+    const int R = rows_of(bi.n, g);
+    bi.i0 = j * RB;
+    bi.row0 = rp[bi.b] + bi.i0;
+    int e = bi.i0 + RB;
+    if (e > R) e = R;
+    bi.nrows = e - bi.i0;
+    bi.key0 = cu[bi.b];
+    bi.maxbound = row_bound(e - 1, bi.n, g);
+    bi.ntiles = bi.maxbound / KT + 1;
+    return bi;
+}
+
+}  // namespace idx

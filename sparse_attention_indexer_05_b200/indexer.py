@@ -1,0 +1,189 @@
+"""Python binding of libidx: the lightning indexer + per-query top-k.
+
+Argument marshalling only: tensors are checked and their device pointers
+passed to the C ABI (include/idx.h); every step of the computation runs in
+the library's CUDA kernels.  torch provides device memory and streams.
+
+Entry points (names follow the C ABI):
+    dense_topk(q, k, w, cu_seqlens, topk)               -> idx [T, topk]
+    pivot_topk(q, k, w, cu_seqlens, topk, g, c, mode)   -> idx [T, topk]
+    decode_topk(q, kcache, kv_len, w, topk, c, mode)    -> idx [B, G, topk]
+Each accepts out_idx / out_score / workspace to reuse buffers, and
+return_scores=True to also get the selected scores.
+"""
+from __future__ import annotations
+
+import ctypes
+from typing import Optional
+
+import torch
+
+from . import _native as N
+
+MODES = {"dense": N.MODE_DENSE, "reuse": N.MODE_REUSE, "refine": N.MODE_REFINE}
+
+
+def _mode(m) -> int:
+    if isinstance(m, str):
+        return MODES[m.lower()]
+    return int(m)
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return N.BF16
+    if t.dtype == torch.float32:
+        return N.F32
+    raise TypeError(f"q/k must be bfloat16 or float32, got {t.dtype}")
+
+
+def _dev(t: torch.Tensor, name: str, dtype=None) -> int:
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor (the library has no CPU path)")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    return t.data_ptr()
+
+
+def _stream(stream) -> int:
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return s.cuda_stream
+
+
+def _ws(workspace: Optional[torch.Tensor], need: int, device) -> torch.Tensor:
+    if need == 0:
+        raise ValueError("invalid arguments (workspace size 0)")
+    if workspace is None or workspace.numel() * workspace.element_size() < need:
+        workspace = torch.empty(need, dtype=torch.uint8, device=device)
+    return workspace
+
+
+def dense_workspace_size(T, H, d, topk, num_seqs, dtype=torch.bfloat16) -> int:
+    dt = N.BF16 if dtype == torch.bfloat16 else N.F32
+    return int(N.lib().idx_dense_workspace_size(T, H, d, topk, num_seqs, dt))
+
+
+def pivot_workspace_size(T, H, d, topk, num_seqs, g, c, mode, dtype=torch.bfloat16) -> int:
+    dt = N.BF16 if dtype == torch.bfloat16 else N.F32
+    return int(N.lib().idx_pivot_workspace_size(T, H, d, topk, num_seqs, dt, g, c, _mode(mode)))
+
+
+def decode_workspace_size(B, G, n_max, H, d, topk, c, mode, dtype=torch.bfloat16) -> int:
+    dt = N.BF16 if dtype == torch.bfloat16 else N.F32
+    return int(N.lib().idx_decode_workspace_size(B, G, n_max, H, d, topk, c, _mode(mode), dt))
+
+
+def _outs(rows_shape, topk, device, out_idx, out_score, return_scores):
+    if out_idx is None:
+        out_idx = torch.empty(*rows_shape, topk, dtype=torch.int32, device=device)
+    if out_score is None and return_scores:
+        out_score = torch.empty(*rows_shape, topk, dtype=torch.float32, device=device)
+    return out_idx, out_score
+
+
+def dense_topk(q, k, w, cu_seqlens, topk: int, out_idx=None, out_score=None, workspace=None, stream=None,
+               return_scores=False):
+    """Dense indexer + top-k; q [T,H,d], k [T,d], w [T,H] fp32, cu_seqlens int32 [S+1]."""
+    T, H, d = q.shape
+    S = cu_seqlens.numel() - 1
+    dt = _dtype_code(q)
+    ws = _ws(workspace, dense_workspace_size(T, H, d, topk, S, q.dtype), q.device)
+    out_idx, out_score = _outs((T,), topk, q.device, out_idx, out_score, return_scores)
+    N.check(N.lib().idx_dense_topk(
+        _dev(q, "q"), _dev(k, "k", q.dtype), _dev(w, "w", torch.float32), _dev(cu_seqlens, "cu_seqlens", torch.int32),
+        S, T, H, d, topk, dt, _dev(out_idx, "out_idx", torch.int32),
+        _dev(out_score, "out_score", torch.float32) if out_score is not None else None,
+        ws.data_ptr(), ws.numel(), _stream(stream)), "idx_dense_topk")
+    return (out_idx, out_score) if return_scores else out_idx
+
+
+def pivot_topk(q, k, w, cu_seqlens, topk: int, g: int, c: int, mode="refine", out_idx=None, out_score=None,
+               workspace=None, stream=None, return_scores=False):
+    """PIVOT Reuse / Refine indexer + top-k over groups of g queries."""
+    T, H, d = q.shape
+    S = cu_seqlens.numel() - 1
+    dt = _dtype_code(q)
+    m = _mode(mode)
+    ws = _ws(workspace, pivot_workspace_size(T, H, d, topk, S, g, c, m, q.dtype), q.device)
+    out_idx, out_score = _outs((T,), topk, q.device, out_idx, out_score, return_scores)
+    N.check(N.lib().idx_pivot_topk(
+        _dev(q, "q"), _dev(k, "k", q.dtype), _dev(w, "w", torch.float32), _dev(cu_seqlens, "cu_seqlens", torch.int32),
+        S, T, H, d, topk, dt, g, c, m, _dev(out_idx, "out_idx", torch.int32),
+        _dev(out_score, "out_score", torch.float32) if out_score is not None else None,
+        ws.data_ptr(), ws.numel(), _stream(stream)), "idx_pivot_topk")
+    return (out_idx, out_score) if return_scores else out_idx
+
+
+def decode_topk(q, kcache, kv_len, w, topk: int, c: int = 0, mode="dense", out_idx=None, out_score=None,
+                workspace=None, stream=None, return_scores=False):
+    """One decode step: q [B,G,H,d], kcache [B,n_max,d], kv_len int32 [B], w [B,G,H]."""
+    B, G, H, d = q.shape
+    n_max = kcache.shape[1]
+    dt = _dtype_code(q)
+    m = _mode(mode)
+    ws = _ws(workspace, decode_workspace_size(B, G, n_max, H, d, topk, c, m, q.dtype), q.device)
+    out_idx, out_score = _outs((B, G), topk, q.device, out_idx, out_score, return_scores)
+    N.check(N.lib().idx_decode_topk(
+        _dev(q, "q"), _dev(kcache, "kcache", q.dtype), _dev(kv_len, "kv_len", torch.int32),
+        _dev(w, "w", torch.float32), B, G, n_max, H, d, topk, c, m, dt, _dev(out_idx, "out_idx", torch.int32),
+        _dev(out_score, "out_score", torch.float32) if out_score is not None else None,
+        ws.data_ptr(), ws.numel(), _stream(stream)), "idx_decode_topk")
+    return (out_idx, out_score) if return_scores else out_idx
+
+
+def device_status(workspace: torch.Tensor, stream=None) -> str:
+    """Synchronise the stream and return the status name recorded in the workspace."""
+    code = N.lib().idx_device_status(workspace.data_ptr(), _stream(stream))
+    return N.STATUS.get(code, str(code))
+
+
+def uses_tensor_cores(H: int, d: int, dtype=torch.bfloat16) -> bool:
+    dt = N.BF16 if dtype == torch.bfloat16 else N.F32
+    return bool(N.lib().idx_uses_tensor_cores(H, d, dt))
+
+
+def debug_scores(stage: int, q, k, w, cu_seqlens, topk, rows, g=1, c=0, workspace=None, ld=None, stream=None):
+    """Scores the selection used (test hook): stage 0 dense rows, 1 proxies, 2 Refine members.
+    `workspace` must be the one the matching top-k call used (required for stage 2)."""
+    T, H, d = q.shape
+    S = cu_seqlens.numel() - 1
+    dt = _dtype_code(q)
+    rows = rows.to(device=q.device, dtype=torch.int32).contiguous()
+    width = ld or (c if stage == 2 else T)
+    out = torch.full((rows.numel(), width), float("nan"), dtype=torch.float32, device=q.device)
+    if workspace is None:
+        if stage == 0:
+            need = dense_workspace_size(T, H, d, topk, S, q.dtype)
+        else:
+            need = pivot_workspace_size(T, H, d, topk, S, g, c if c > 0 else topk, "refine" if c > 0 else "reuse",
+                                        q.dtype)
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    N.check(N.lib().idx_debug_scores(
+        stage, _dev(q, "q"), _dev(k, "k", q.dtype), _dev(w, "w", torch.float32),
+        _dev(cu_seqlens, "cu_seqlens", torch.int32), S, T, H, d, dt, g, c, topk, rows.data_ptr(), rows.numel(),
+        out.data_ptr(), width, workspace.data_ptr(), workspace.numel(), _stream(stream)), "idx_debug_scores")
+    return out
+
+
+def debug_decode_scores(stage: int, q, kcache, kv_len, w, topk, c=0, mode="dense", workspace=None, stream=None):
+    """Decode scores the selection used (test hook): stage 0 dense queries, 1 proxies, 2 Refine members."""
+    B, G, H, d = q.shape
+    n_max = kcache.shape[1]
+    dt = _dtype_code(q)
+    m = _mode(mode)
+    rows = B if stage == 1 else B * G
+    width = c if stage == 2 else n_max
+    out = torch.full((rows, width), float("nan"), dtype=torch.float32, device=q.device)
+    if workspace is None:
+        need = max(decode_workspace_size(B, G, n_max, H, d, topk, c, mm, q.dtype)
+                   for mm in ((0, m) if m != 0 else (0,)))
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    N.check(N.lib().idx_debug_decode_scores(
+        stage, _dev(q, "q"), _dev(kcache, "kcache", q.dtype), _dev(kv_len, "kv_len", torch.int32),
+        _dev(w, "w", torch.float32), B, G, n_max, H, d, topk, c, m, dt, out.data_ptr(), width,
+        workspace.data_ptr(), workspace.numel(), _stream(stream)), "idx_debug_decode_scores")
+    return out

@@ -1,0 +1,87 @@
+"""The C ABI library loads, exports every declared entry point, and rejects
+bad arguments on the host (no GPU needed: nothing is launched)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from sparse_attention_indexer_05_b200 import _native as N
+from sparse_attention_indexer_05_b200 import build as B
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    B.build()
+    return N.lib()
+
+
+def declared_functions():
+    src = open(os.path.join(ROOT, "include", "idx.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(idx_[a-z_]+)\s*\(", src)))
+
+
+def test_exports_every_declared_symbol(lib):
+    names = declared_functions()
+    assert len(names) == 11
+    for n in names:
+        assert hasattr(lib, n), n
+        assert n in N.SIGNATURES, n
+
+
+def test_status_strings(lib):
+    for code, name in N.STATUS.items():
+        assert lib.idx_status_string(code).decode() == name
+
+
+def test_workspace_sizes(lib):
+    assert lib.idx_dense_workspace_size(16384, 64, 128, 2048, 1, 0) > 16384 * 2048 * 8
+    assert lib.idx_dense_workspace_size(0, 64, 128, 2048, 1, 0) == 0
+    assert lib.idx_dense_workspace_size(100, 64, 12, 8, 1, 0) == 0        # d % 8 != 0
+    assert lib.idx_pivot_workspace_size(65536, 64, 128, 2048, 1, 0, 4, 4096, 2) > 0
+    assert lib.idx_pivot_workspace_size(65536, 64, 128, 2048, 1, 0, 4, 1024, 2) == 0   # c < k
+    assert lib.idx_pivot_workspace_size(65536, 64, 128, 2048, 1, 0, 0, 4096, 2) == 0   # g < 1
+    assert lib.idx_pivot_workspace_size(65536, 64, 128, 2048, 1, 0, 4, 4096, 0) == 0   # dense mode
+    assert lib.idx_decode_workspace_size(64, 2, 131072, 64, 128, 2048, 4096, 2, 0) > 64 * 131072 * 4
+    assert lib.idx_decode_workspace_size(64, 2, 1, 64, 128, 2048, 4096, 2, 0) == 0     # n_max < G
+
+
+def test_invalid_arguments_return_before_launch(lib):
+    fake = ctypes.c_void_p(256)  # never dereferenced: the checks fail first
+    # null q
+    assert lib.idx_dense_topk(None, fake, fake, fake, 1, 10, 4, 64, 8, 0, fake, None, fake, 1 << 30, None) == 1
+    # bad head dim
+    assert lib.idx_dense_topk(fake, fake, fake, fake, 1, 10, 4, 60, 8, 0, fake, None, fake, 1 << 30, None) == 1
+    # workspace too small
+    assert lib.idx_dense_topk(fake, fake, fake, fake, 1, 10, 4, 64, 8, 0, fake, None, fake, 16, None) == 3
+    # misaligned workspace
+    assert lib.idx_dense_topk(fake, fake, fake, fake, 1, 10, 4, 64, 8, 0, fake, None, ctypes.c_void_p(264),
+                              1 << 30, None) == 3
+    # refine with c < k
+    assert lib.idx_pivot_topk(fake, fake, fake, fake, 1, 10, 4, 64, 8, 0, 4, 4, 2, fake, None, fake, 1 << 30,
+                              None) == 1
+    # unknown mode
+    assert lib.idx_pivot_topk(fake, fake, fake, fake, 1, 10, 4, 64, 8, 0, 4, 16, 7, fake, None, fake, 1 << 30,
+                              None) == 1
+    # decode: more MTP queries than a row block holds
+    assert lib.idx_decode_topk(fake, fake, fake, fake, 2, 9, 64, 4, 64, 8, 0, 0, 0, fake, None, fake, 1 << 30,
+                               None) == 2
+    # decode: refine with c < k
+    assert lib.idx_decode_topk(fake, fake, fake, fake, 2, 2, 64, 4, 64, 8, 4, 2, 0, fake, None, fake, 1 << 30,
+                               None) == 1
+    # shape that fits neither kernel family
+    assert lib.idx_dense_topk(fake, fake, fake, fake, 1, 10, 256, 256, 8, 1, fake, None, fake, 1 << 40,
+                              None) == 2
+
+
+def test_binding_refuses_cpu_tensors():
+    torch = pytest.importorskip("torch")
+    import sparse_attention_indexer_05_b200 as idx
+    B.build()
+    q = torch.zeros(4, 2, 8, dtype=torch.bfloat16)
+    with pytest.raises((ValueError, RuntimeError)):
+        idx.dense_topk(q, torch.zeros(4, 8, dtype=torch.bfloat16), torch.zeros(4, 2),
+                       torch.tensor([0, 4], dtype=torch.int32), 2)
