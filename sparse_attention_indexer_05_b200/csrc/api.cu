@@ -160,6 +160,7 @@ struct Prefill {
         a.cu = cu;
         a.S = S; a.T = T; a.H = H; a.d = d;
         a.g = proxies ? g : 1;
+        a.R = proxies ? L.R : T;
         a.plan = plan();
         a.pl = L.pl;
         a.sink = SINK_FILTER;
@@ -304,7 +305,8 @@ idx_status idx_pivot_topk(const void *q, const void *k, const float *w, const in
     int *cand = reinterpret_cast<int *>(P.ws + P.L.cand);
     TRY_CUDA(launch_select(P.select_args(SEL_PROXY_TO_C, (int)P.L.R, c, cand, nullptr), P.st));
     const GatherArgs ga = P.gather_args();
-    TRY_CUDA(tc_supported(H, d, (int)dtype) ? launch_gather_tc(ga, P.st) : launch_gather_simt(ga, (int)dtype, P.st));
+    TRY_CUDA(tc_gather_supported(H, d, (int)dtype, g) ? launch_gather_tc(ga, P.st)
+                                                       : launch_gather_simt(ga, (int)dtype, P.st));
     return cuda_st(launch_select(P.select_args(SEL_MEMBER_SCORES, T, topk, out_idx, out_score), P.st));
 }
 
@@ -345,8 +347,8 @@ struct Decode {
         return a;
     }
     cudaError_t scan(const DecodeArgs &a) const {
-        return tc_supported(H, d, (int)dt) && (a.Gq * H) <= 256 ? launch_decode_tc(a, st)
-                                                                : launch_decode_simt(a, (int)dt, st);
+        return tc_decode_supported(H, d, (int)dt, a.Gq) ? launch_decode_tc(a, st)
+                                                        : launch_decode_simt(a, (int)dt, st);
     }
     SelectArgs sargs(int kind, int nrows, int kk, int *oi, float *os, const float *scores, long long ld) const {
         SelectArgs s{};
@@ -410,8 +412,8 @@ idx_status idx_decode_topk(const void *q, const void *kcache, const int *kv_len,
     int *cand = reinterpret_cast<int *>(D.ws + D.L.cand);
     TRY_CUDA(launch_select(D.sargs(SEL_DEC_PROXY_TO_C, B, c, cand, nullptr, spill, n_max), D.st));
     const GatherArgs ga = D.gargs();
-    TRY_CUDA(tc_supported(H, d, (int)dtype) && G * H <= 256 ? launch_gather_tc(ga, D.st)
-                                                            : launch_gather_simt(ga, (int)dtype, D.st));
+    TRY_CUDA(tc_gather_supported(H, d, (int)dtype, G) ? launch_gather_tc(ga, D.st)
+                                                       : launch_gather_simt(ga, (int)dtype, D.st));
     const float *msc = reinterpret_cast<const float *>(D.ws + D.L.msc);
     return cuda_st(launch_select(D.sargs(SEL_DEC_MEMBER, B * G, topk, out_idx, out_score, msc, c), D.st));
 }

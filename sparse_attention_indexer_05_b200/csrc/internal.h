@@ -39,6 +39,7 @@ struct ScoreArgs {
     const float *w;      // [R, H]
     const int *cu;       // cu_seqlens [S+1] (device)
     int S, T, H, d, g;   // g = 1: row i of request b is query i; g > 1: proxy i
+    long long R;         // rows allocated in q / w
     const int *plan;     // plan area
     PlanLayout pl;
     int sink;
@@ -141,5 +142,7 @@ cudaError_t launch_decode_proxy(const void *q, const float *w, int B, int G, int
                                 void *qbar, float *wbar, cudaStream_t st);
 size_t simt_smem_bytes(int H, int d, int dtype);
 bool tc_supported(int H, int d, int dtype);
+bool tc_decode_supported(int H, int d, int dtype, int rows_per_request);
+bool tc_gather_supported(int H, int d, int dtype, int group);
 
 }  // namespace idx
