@@ -1,0 +1,379 @@
+#!/usr/bin/env python
+"""Benchmark of the lightning indexer + top-k on B200.
+
+One step = one pass of the whole hot path over the long-prefill batch
+(131072 tokens, H=64, d=128, k=2048, bf16 q/k, fp32 w): the dense
+indexer + top-k over the batch as ONE 131072-token request, and PIVOT
+Refine (g=16, c=4096) over the same tokens as TWO packed 65536-token
+requests (proxy build, proxy scan, candidate select, member re-score,
+member select).  `value` = query rows ranked per second (2 * 131072 per
+step, whole job).  The decode step (B=64 requests x 131072-token caches,
+G=2 MTP queries, dense and Refine c=4096) is timed after it and reported
+under "decode" as HBM GB/s of the cache scan.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Multi-GPU (torchrun): every rank runs its own batch (seed = rank): weak
+scaling with no collective on the data path; the time is the max over
+ranks of the device time.  --impl reference runs the CPU oracle (the
+plain double-precision restatement) on the host cores on a bounded sample
+of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+L_TOK, H, D, TOPK, G_REF, C_REF = 131072, 64, 128, 2048, 16, 4096
+DEC_B, DEC_N, DEC_G = 64, 131072, 2
+METRIC = "indexer+top-k queries/s and TFLOP/s (% bf16 TC peak); decode HBM GB/s @ L=128K"
+
+
+def parse():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=5)
+    p.add_argument("--warmup", type=int, default=3)
+    p.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--no-decode", action="store_true")
+    p.add_argument("--cpu-rows", type=int, default=64, help="oracle sample rows (dense + refine) per CPU step")
+    return p.parse_args()
+
+
+def dense_flops_single(L=L_TOK):
+    return 2.0 * H * D * L * (L + 1) / 2.0
+
+
+def proxy_pairs(n, g):
+    # sum over proxies of (t_last + 1), request of n tokens
+    tot = 0
+    for i in range((n + g - 1) // g):
+        tot += min((i + 1) * g, n)
+    return tot
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            m = json.load(f)
+        return m.get("bf16_tflops", 1590.0), m.get("bf16_tflops_sustained", 1400.0), m.get("hbm_gbs", 6650.0), "measured"
+    return 1590.0, 1400.0, 6650.0, "fallback"
+
+
+class Clocks:
+    """nvidia-smi sampling of SM clocks and throttle reasons during the timed region."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.Q}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    sm.append(float(parts[1]))
+                    smax = float(parts[2])
+                except ValueError:
+                    continue
+                for nm, v in zip(names, parts[5:9]):
+                    if v.lower() == "active":
+                        reasons.add(nm)
+        os.unlink(self.path)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def trace_report(lib):
+    import ctypes
+    buf = ctypes.create_string_buffer(1 << 16)
+    n = lib.idx_trace_report(buf, len(buf))
+    out = {}
+    for line in buf.value.decode().splitlines():
+        name, cnt, ms = line.split()
+        out[name] = (int(cnt), float(ms))
+    return n, out
+
+
+def to_dev(a, dev):
+    import torch
+    if a.dtype == np.uint16:
+        return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).to(dev)
+    return torch.from_numpy(np.ascontiguousarray(a)).to(dev)
+
+
+def pinned(a):
+    import torch
+    t = torch.from_numpy(np.ascontiguousarray(a).view(np.int16) if a.dtype == np.uint16 else np.ascontiguousarray(a))
+    return t.pin_memory()
+
+
+# ---------------------------------------------------------------- CPU oracle
+def oracle_sample(P, nrows, seed=0):
+    """Time the oracle on `nrows` rows of the step (half dense on the single
+    request, half Refine on the packed requests); returns (rows/s, seconds,
+    threads, description)."""
+    import oracle as O
+    rng = np.random.default_rng(seed)
+    nd = max(1, nrows // 2)
+    nr = max(1, nrows - nd)
+    # stratified by position so the sample's mean prefix matches the batch's
+    dense_rows = np.sort((np.arange(nd) + rng.random(nd)) * (L_TOK / nd)).astype(np.int64)
+    ref_rows = np.sort((np.arange(nr) + rng.random(nr)) * (L_TOK / nr)).astype(np.int64)
+    cu1 = np.array([0, L_TOK], np.int32)
+    cu2 = np.array([0, L_TOK // 2, L_TOK], np.int32)
+    threads = os.cpu_count() or 1
+    t0 = time.perf_counter()
+    O.dense_topk(P.q, P.k, P.w, cu1, TOPK, rows=dense_rows, threads=threads)
+    O.pivot_topk(P.q, P.k, P.w, cu2, TOPK, G_REF, C_REF, O.REFINE, rows=ref_rows, threads=threads)
+    dt = time.perf_counter() - t0
+    desc = (f"{nd} dense rows (single 131072-token request) + {nr} Refine g=16 c=4096 member rows "
+            f"(2x65536 packed), stratified by position, seed {seed}")
+    return (nd + nr) / dt, dt, threads, desc
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    from sparse_attention_indexer_05_b200 import workloads as W
+    P = W.cfg_long_single(seed=0)
+    times, rows = [], 0
+    for i in range(args.warmup + args.steps):
+        v, dt, threads, desc = oracle_sample(P, max(2, args.cpu_rows // 3), seed=i)
+        if i >= args.warmup:
+            times.append(dt)
+            rows += max(2, args.cpu_rows // 3)
+    val = rows / sum(times)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": val, "unit": "queries/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000 * sum(times) / len(times),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic",
+        "config": {"workload": "long_prefill_131072_dense+refine_g16_c4096", "tokens": L_TOK, "H": H, "d": D,
+                   "topk": TOPK},
+        "cpu_baseline": {"value": val, "unit": "queries/s", "cores": threads, "kind": "oracle",
+                         "sample": f"per step: {desc}"},
+        "e2e": {"value": val, "unit": "queries/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line))
+    return 0
+
+
+# --------------------------------------------------------------- GPU bench
+def main():
+    args = parse()
+    if args.impl == "reference":
+        return run_reference(args)
+    import torch
+    import torch.distributed as dist
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+
+    import sparse_attention_indexer_05_b200 as idx
+    from sparse_attention_indexer_05_b200 import _native as N
+    from sparse_attention_indexer_05_b200 import workloads as W
+    lib = N.lib()
+
+    def barrier():
+        if world > 1:
+            dist.barrier(device_ids=[local])
+
+    def max_over_ranks(x):
+        if world == 1:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    P = W.cfg_long_single(seed=rank)
+    cu1_h = np.array([0, L_TOK], np.int32)
+    cu2_h = np.array([0, L_TOK // 2, L_TOK], np.int32)
+    q, k, w = to_dev(P.q, dev), to_dev(P.k, dev), to_dev(P.w, dev)
+    cu1, cu2 = to_dev(cu1_h, dev), to_dev(cu2_h, dev)
+    ws1 = torch.empty(idx.dense_workspace_size(L_TOK, H, D, TOPK, 1), dtype=torch.uint8, device=dev)
+    ws2 = torch.empty(idx.pivot_workspace_size(L_TOK, H, D, TOPK, 2, G_REF, C_REF, "refine"), dtype=torch.uint8,
+                      device=dev)
+    o1 = torch.empty(L_TOK, TOPK, dtype=torch.int32, device=dev)
+    o2 = torch.empty(L_TOK, TOPK, dtype=torch.int32, device=dev)
+
+    def step(qq=q, kk=k, ww=w, c1=cu1, c2=cu2):
+        idx.dense_topk(qq, kk, ww, c1, TOPK, out_idx=o1, workspace=ws1)
+        idx.pivot_topk(qq, kk, ww, c2, TOPK, G_REF, C_REF, "refine", out_idx=o2, workspace=ws2)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    assert idx.device_status(ws1) == "IDX_OK" and idx.device_status(ws2) == "IDX_OK"
+
+    stream = torch.cuda.current_stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = Clocks(local)
+    barrier()
+    torch.cuda.synchronize()
+    lib.idx_trace_enable(1)
+    clocks.start()
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    lib.idx_trace_enable(0)
+    barrier()
+    ms = max_over_ranks(e0.elapsed_time(e1) / args.steps)
+    nlaunch, tr = trace_report(lib)
+    rows_per_step = 2 * L_TOK
+    value = world * rows_per_step / (ms / 1000.0)
+
+    bf16_peak, bf16_sus, hbm_peak, peak_src = peaks()
+    n_dense, ms_dense = tr.get("dense/score_tc", (0, 0.0))
+    dense_ms = ms_dense / max(1, n_dense)
+    achieved = dense_flops_single() / (dense_ms / 1000.0) / 1e12 if dense_ms > 0 else None
+    roof = {"kernel": "score_tc (dense pass)", "bound": "tensor", "achieved": achieved,
+            "peak": bf16_sus, "unit": "TFLOP/s", "frac": (achieved / bf16_sus) if achieved else None,
+            "traffic": None, "peak_kind": f"{peak_src} bf16 sustained (kernel timed inside a long step)",
+            "flops_per_launch": dense_flops_single(), "ms_per_launch": dense_ms}
+
+    per_kernel = {name: {"launches": c, "ms_total": t, "ms_per_step": t / args.steps} for name, (c, t) in tr.items()}
+
+    # ---------------------------------------------------------------- e2e
+    e2e = None
+    if not args.no_e2e:
+        hq, hk, hw, h1, h2 = pinned(P.q), pinned(P.k), pinned(P.w), pinned(cu1_h), pinned(cu2_h)
+        ho1 = torch.empty(o1.shape, dtype=torch.int32).pin_memory()
+        ho2 = torch.empty(o2.shape, dtype=torch.int32).pin_memory()
+        dq, dk, dw = torch.empty_like(q), torch.empty_like(k), torch.empty_like(w)
+        dc1, dc2 = torch.empty_like(cu1), torch.empty_like(cu2)
+
+        def e2e_step():
+            dq.view(torch.int16).copy_(hq, non_blocking=True)
+            dk.view(torch.int16).copy_(hk, non_blocking=True)
+            dw.copy_(hw, non_blocking=True)
+            dc1.copy_(h1, non_blocking=True)
+            dc2.copy_(h2, non_blocking=True)
+            step(dq, dk, dw, dc1, dc2)
+            ho1.copy_(o1, non_blocking=True)
+            ho2.copy_(o2, non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize()
+        barrier()
+        e0.record(stream)
+        for _ in range(args.steps):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        ems = max_over_ranks(e0.elapsed_time(e1) / args.steps)
+        h2d = hq.numel() * 2 + hk.numel() * 2 + hw.numel() * 4 + h1.numel() * 4 + h2.numel() * 4
+        d2h = (ho1.numel() + ho2.numel()) * 4
+        e2e = {"value": world * rows_per_step / (ems / 1000.0), "unit": "queries/s", "ms_per_step": ems,
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+        del dq, dk, dw
+
+    # ------------------------------------------------------------- decode
+    dec = None
+    if not args.no_decode:
+        Dd = W.cfg_decode(seed=rank)
+        dq_, dkc, dw_, dkv = to_dev(Dd.q, dev), to_dev(Dd.kcache, dev), to_dev(Dd.w, dev), to_dev(Dd.kv_len, dev)
+        wsd = torch.empty(max(idx.decode_workspace_size(DEC_B, DEC_G, DEC_N, H, D, TOPK, C_REF, m)
+                              for m in ("dense", "refine")), dtype=torch.uint8, device=dev)
+        od = torch.empty(DEC_B, DEC_G, TOPK, dtype=torch.int32, device=dev)
+        dec = {"workload": "decode_B64_n131072_G2_H64_d128_k2048", "kcache_bytes": Dd.kcache.nbytes}
+        for mode in ("dense", "refine"):
+            for _ in range(args.warmup):
+                idx.decode_topk(dq_, dkc, dkv, dw_, TOPK, C_REF, mode, out_idx=od, workspace=wsd)
+            torch.cuda.synchronize()
+            assert idx.device_status(wsd) == "IDX_OK"
+            lib.idx_trace_enable(1)
+            e0.record(stream)
+            for _ in range(args.steps):
+                idx.decode_topk(dq_, dkc, dkv, dw_, TOPK, C_REF, mode, out_idx=od, workspace=wsd)
+            e1.record(stream)
+            torch.cuda.synchronize()
+            lib.idx_trace_enable(0)
+            _, trd = trace_report(lib)
+            step_ms = max_over_ranks(e0.elapsed_time(e1) / args.steps)
+            scan = [(n, c, t) for n, (c, t) in trd.items() if "decode_" in n.split("/")[-1]]
+            scan_ms = sum(t for _, _, t in scan) / args.steps
+            gbs = Dd.kcache.nbytes / (scan_ms / 1000.0) / 1e9 if scan_ms > 0 else None
+            dec[mode] = {"ms_per_step": step_ms, "scan_kernel_ms": scan_ms,
+                         "scan_GBps": gbs, "scan_frac_hbm": (gbs / hbm_peak) if gbs else None,
+                         "kernels": {n: {"launches": c, "ms_per_step": t / args.steps} for n, (c, t) in trd.items()}}
+        dec["hbm_peak_GBps"] = hbm_peak
+
+    # -------------------------------------------------------- CPU baseline
+    cpu = None
+    if rank == 0 and world == 1:
+        v, dt, threads, desc = oracle_sample(P, args.cpu_rows)
+        cpu = {"value": v, "unit": "queries/s", "cores": threads, "kind": "oracle", "sample": desc,
+               "seconds": dt}
+
+    line = {
+        "metric": METRIC, "value": value, "unit": "queries/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": "long_prefill_131072_dense+refine_g16_c4096", "tokens": L_TOK, "H": H, "d": D,
+                   "topk": TOPK, "dense_requests": [L_TOK], "refine_requests": [L_TOK // 2, L_TOK // 2],
+                   "g": G_REF, "c": C_REF, "parallelism": f"dp{world} (independent batches)",
+                   "l2": "inputs larger than L2 (q is 2 GiB)"},
+        "tflops_dense": achieved, "roofline": roof, "cpu_baseline": cpu, "e2e": e2e, "clocks": clk,
+        "gpu_launches": nlaunch, "kernels": per_kernel, "decode": dec,
+    }
+    if rank == 0:
+        print(json.dumps(line))
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

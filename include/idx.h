@@ -164,6 +164,17 @@ idx_status idx_debug_decode_scores(int stage, const void *q, const void *kcache,
                                    int c, idx_mode mode, idx_dtype dtype, float *out, long long ld,
                                    void *ws, size_t ws_bytes, idx_stream_t stream);
 
+/* Per-kernel device timing.  idx_trace_enable(1) clears the record and
+ * starts bracketing every kernel launch of the library with two CUDA events
+ * on its stream; idx_trace_enable(0) stops (the record is kept).
+ * idx_trace_report() waits for the recorded events and writes one line per
+ * kernel, "<phase>/<kernel> <launches> <total milliseconds>", into buf
+ * (NUL-terminated, truncated to len); it returns the number of launches
+ * recorded, or -1 if an event could not be read.  Host-side state shared by
+ * all threads; meant for benchmarks, off by default. */
+int idx_trace_enable(int on);
+long long idx_trace_report(char *buf, size_t len);
+
 /* Which score kernel serves a shape: 1 = tcgen05 tensor-core kernel,
  * 0 = SIMT kernel.  (bf16 with H = 64 and d = 128 uses the tensor cores.) */
 int idx_uses_tensor_cores(int H, int d, idx_dtype dtype);

@@ -30,6 +30,8 @@ SIGNATURES = {
     "idx_debug_decode_scores": (_i, [_i, _vp, _vp, _ip, _fp, _i, _i, _i, _i, _i, _i, _i, _i, _i, _fp, _ll,
                                      _vp, _sz, _vp]),
     "idx_uses_tensor_cores": (_i, [_i, _i, _i]),
+    "idx_trace_enable": (_i, [_i]),
+    "idx_trace_report": (_ll, [ctypes.c_char_p, _sz]),
 }
 
 _lib = None

@@ -221,7 +221,7 @@ struct Prefill {
         a.c = c; a.H = H; a.d = d;
         a.nitems = (int)L.R;
         a.mode = 0;
-        a.cu = cu; a.S = S; a.g = g;
+        a.cu = cu; a.S = S; a.g = g; a.cu_T = T;
         a.plan = plan(); a.pl = L.pl;
         a.out = reinterpret_cast<float *>(ws + L.msc);
         a.status = status();
@@ -270,6 +270,7 @@ idx_status idx_dense_topk(const void *q, const void *k, const float *w, const in
     idx_status s = check_prefill(q, k, w, cu_seqlens, num_seqs, T, H, d, topk, dtype, out_idx, ws, ws_bytes,
                                  need);
     if (s != IDX_OK) return s;
+    TracePhase phase("dense");
     Prefill P{q, k, w, cu_seqlens, num_seqs, T, H, d, topk, dtype, 1, topk, IDX_MODE_DENSE,
               static_cast<char *>(ws), prefill_ws(T, H, d, topk, num_seqs, dtype, 1, topk, IDX_MODE_DENSE),
               reinterpret_cast<cudaStream_t>(stream)};
@@ -296,6 +297,7 @@ idx_status idx_pivot_topk(const void *q, const void *k, const float *w, const in
     idx_status s = check_prefill(q, k, w, cu_seqlens, num_seqs, T, H, d, topk, dtype, out_idx, ws, ws_bytes,
                                  need);
     if (s != IDX_OK) return s;
+    TracePhase phase(mode == IDX_MODE_REUSE ? "reuse" : "refine");
     Prefill P{q, k, w, cu_seqlens, num_seqs, T, H, d, topk, dtype, g, c, mode, static_cast<char *>(ws),
               prefill_ws(T, H, d, topk, num_seqs, dtype, g, c, mode), reinterpret_cast<cudaStream_t>(stream)};
     TRY_CUDA(P.prepare());
@@ -396,6 +398,7 @@ idx_status idx_decode_topk(const void *q, const void *kcache, const int *kv_len,
     idx_status s = check_decode(q, kcache, kv_len, w, B, G, n_max, H, d, topk, c, mode, dtype, out_idx, ws,
                                 ws_bytes);
     if (s != IDX_OK) return s;
+    TracePhase phase(mode == IDX_MODE_DENSE ? "decode_dense" : mode == IDX_MODE_REUSE ? "decode_reuse" : "decode_refine");
     Decode D{q, kcache, kv_len, w, B, G, n_max, H, d, topk, c, mode, dtype, static_cast<char *>(ws),
              decode_ws(B, G, n_max, H, d, c, mode, dtype), reinterpret_cast<cudaStream_t>(stream)};
     TRY_CUDA(cudaMemsetAsync(D.status(), 0, 4, D.st));

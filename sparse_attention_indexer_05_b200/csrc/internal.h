@@ -79,6 +79,7 @@ struct GatherArgs {
     int mode;            // 0: prefill (cu, g, plan rp of proxies), 1: decode (B, G, n_max)
     const int *cu;
     int S, g;
+    int cu_T;            // prefill: rows of q and k (total tokens)
     const int *plan;
     PlanLayout pl;
     int G, n_max;
@@ -123,6 +124,21 @@ struct SelectArgs {
     int G, n_max;
     int bitmap_words;        // shared bitmap capacity (words)
     unsigned *status;
+};
+
+// ---- tracing (trace.cu): a TraceScope around a launch records two events
+// on its stream while tracing is enabled; TracePhase names the entry-point
+// phase that prefixes the kernel names in the report.
+struct TracePhase {
+    explicit TracePhase(const char *p);
+    ~TracePhase();
+    const char *prev;
+};
+struct TraceScope {
+    TraceScope(const char *name, cudaStream_t st);
+    ~TraceScope();
+    cudaStream_t st_;
+    int idx_;
 };
 
 // ---- launchers (each returns cudaSuccess or the launch error)

@@ -113,6 +113,7 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const int *cu, int S
 
 cudaError_t launch_plan(const int *cu, int S, int T, int g, int *plan, const PlanLayout &pl,
                         unsigned *status, cudaStream_t st) {
+    TraceScope ts("plan", st);
     plan_kernel<<<1, kPlanThreads, 0, st>>>(cu, S, T, g, plan, pl, status);
     return cudaGetLastError();
 }

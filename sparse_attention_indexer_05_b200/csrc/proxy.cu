@@ -109,6 +109,7 @@ cudaError_t launch_proxy(const void *q, const float *w, const int *cu, int S, in
                          int max_proxies, cudaStream_t st) {
     (void)T;
     if (max_proxies <= 0) return cudaSuccess;
+    TraceScope ts("proxy", st);
     if (dtype == 1)
         proxy_kernel<float><<<max_proxies, kProxyThreads, 0, st>>>(
             (const float *)q, w, cu, S, H, d, g, plan, pl, (float *)qbar, wbar);
@@ -120,6 +121,7 @@ cudaError_t launch_proxy(const void *q, const float *w, const int *cu, int S, in
 
 cudaError_t launch_decode_proxy(const void *q, const float *w, int B, int G, int H, int d, int dtype,
                                 void *qbar, float *wbar, cudaStream_t st) {
+    TraceScope ts("proxy", st);
     if (dtype == 1)
         decode_proxy_kernel<float><<<B, kProxyThreads, 0, st>>>((const float *)q, w, G, H, d, (float *)qbar,
                                                                 wbar);

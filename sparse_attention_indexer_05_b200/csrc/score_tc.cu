@@ -214,10 +214,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                         tc::tmem_ld32(taddr + 32, v1);
                         tc::tmem_ld32(taddr + 64, v2);
                         tc::tmem_ld32(taddr + 96, v3);
-                        tc::tmem_wait_ld(v0);
-                        tc::tmem_wait_ld(v1);
-                        tc::tmem_wait_ld(v2);
-                        tc::tmem_wait_ld(v3);
+                        tc::tmem_wait_ld_all();
+                        tc::reg_fence(v0);
+                        tc::reg_fence(v1);
+                        tc::reg_fence(v2);
+                        tc::reg_fence(v3);
                         tc::fence_before_sync();
                         __syncwarp();
                         if (lane == 0) tc::mbar_arrive(&sh.tempty[h]);
@@ -313,8 +314,6 @@ int num_sms() {
 }  // namespace
 
 bool tc_supported(int H, int d, int dtype) { return H == TC_H && d == TC_D && dtype == 0; }
-bool tc_decode_supported(int, int, int, int) { return false; }
-bool tc_gather_supported(int, int, int, int) { return false; }
 
 cudaError_t launch_score_tc(const ScoreArgs &a, cudaStream_t st) {
     // the scored tensor [R, 64, 128] viewed as [R*64, 128]; keys [T, 128]
@@ -323,11 +322,10 @@ cudaError_t launch_score_tc(const ScoreArgs &a, cudaStream_t st) {
         return cudaErrorInvalidValue;
     cudaError_t e = cudaFuncSetAttribute(score_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
     if (e != cudaSuccess) return e;
+    TraceScope ts("score_tc", st);
     score_tc_kernel<<<num_sms(), kThreads, kSmemBytes, st>>>(mq, mk, a);
     return cudaGetLastError();
 }
 
-cudaError_t launch_decode_tc(const DecodeArgs &, cudaStream_t) { return cudaErrorNotSupported; }
-cudaError_t launch_gather_tc(const GatherArgs &, cudaStream_t) { return cudaErrorNotSupported; }
 
 }  // namespace idx

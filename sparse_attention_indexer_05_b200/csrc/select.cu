@@ -251,6 +251,7 @@ cudaError_t launch_select(const SelectArgs &a, cudaStream_t st) {
     cudaError_t e = cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)smem);
     if (e != cudaSuccess) return e;
+    TraceScope ts("select", st);
     select_kernel<<<a.nrows, kSelThreads, smem, st>>>(a);
     return cudaGetLastError();
 }

@@ -269,6 +269,7 @@ cudaError_t launch_score_simt(const ScoreArgs &a, int dtype, cudaStream_t st) {
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     const size_t smem = simt_smem_bytes(a.H, a.d, dtype);
     cudaError_t e;
+    TraceScope ts("score_simt", st);
     if (dtype == 1) {
         if ((e = set_smem(score_simt_kernel<float>, smem)) != cudaSuccess) return e;
         score_simt_kernel<float><<<sms * 2, kSimtThreads, smem, st>>>(a);
@@ -285,6 +286,7 @@ cudaError_t launch_decode_simt(const DecodeArgs &a, int dtype, cudaStream_t st) 
     const size_t smem = simt_smem_bytes(a.H, a.d, dtype);
     const long long ld = a.n_max;
     cudaError_t e;
+    TraceScope ts("decode_simt", st);
     if (dtype == 1) {
         if ((e = set_smem(decode_simt_kernel<float>, smem)) != cudaSuccess) return e;
         decode_simt_kernel<float><<<a.B * nchunks, kSimtThreads, smem, st>>>(a, nchunks, ld);
@@ -301,6 +303,7 @@ cudaError_t launch_gather_simt(const GatherArgs &a, int dtype, cudaStream_t st) 
     const size_t smem = simt_smem_bytes(a.H, a.d, dtype);
     cudaError_t e;
     if (a.nitems <= 0) return cudaSuccess;
+    TraceScope ts("gather_simt", st);
     if (dtype == 1) {
         if ((e = set_smem(gather_simt_kernel<float>, smem)) != cudaSuccess) return e;
         gather_simt_kernel<float><<<a.nitems * mchunks, kSimtThreads, smem, st>>>(a, mchunks);

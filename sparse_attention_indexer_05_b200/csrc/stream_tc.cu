@@ -1,0 +1,393 @@
+// stream_tc.cu -- tensor-core kernels that score up to 4 query rows (N =
+// 64*m <= 256 columns) against a stream of key tiles and write every score:
+//   * decode scan: the keys are the request's cache, streamed once by TMA
+//     in 128-key tiles; rows = the request's G MTP queries (or its proxy);
+//   * Refine re-score: the keys are a group's candidate set C, gathered row
+//     by row with TMA gather4; rows = up to 4 members of the group.
+// Same MMA shape as the prefill score kernel (keys on M, (row, head) on N,
+// bf16 -> fp32 in TMEM, fused ReLU + w-weighted head sum), with the two
+// 256-column TMEM buffers used alternately by consecutive key tiles.
+#include <cudaTypedefs.h>
+#include <string.h>
+
+#include "common.cuh"
+#include "internal.h"
+#include "plan.cuh"
+#include "tc.cuh"
+
+namespace idx {
+
+namespace {
+
+constexpr int S_H = 64;
+constexpr int S_D = 128;
+constexpr int kThreads = 320;
+constexpr int kEpiWarps = 8;
+constexpr int kStages = 4;
+constexpr uint32_t kQSlice = 256 * 128;          // 256 rows x 64 bf16 (32 KB)
+constexpr uint32_t kQBytes = 2 * kQSlice;        // 2 K slices
+constexpr uint32_t kASlice = KT * 128;           // 128 keys x 64 bf16 (16 KB)
+constexpr uint32_t kAStage = 2 * kASlice;        // one key tile (32 KB)
+constexpr int kDecodeChunkTiles = 64;            // decode: key tiles per work item
+
+struct __align__(8) StShared {
+    uint64_t afull[kStages], aempty[kStages], qfull, tfull[2], tempty[2], drain;
+    uint32_t tmem_base;
+    int abort;
+};
+
+constexpr size_t kOffQ = 0;
+constexpr size_t kOffA = kOffQ + kQBytes;
+constexpr size_t kOffW = kOffA + (size_t)kStages * kAStage;
+constexpr size_t kOffCtl = kOffW + 4 * S_H * 4;
+constexpr size_t kSmemBytes = kOffCtl + sizeof(StShared) + 1024;
+
+struct Item {
+    bool valid;
+    int m;              // rows scored (<= 4)
+    long long qrow0;    // first query row (rows of [*, 64, 128])
+    long long key0;     // first key row of the request
+    int t0, nt;         // key tiles [t0, t0 + nt) of the item
+    // outputs
+    long long out_row0; // output row of scored row 0
+    int bound[4];       // decode: causal bound per row (inclusive)
+    const int *cand;    // gather: candidate positions of the group
+};
+
+template <bool GATHER>
+__device__ __forceinline__ Item item_info(const GatherArgs &g, const DecodeArgs &dd, int item) {
+    Item it{};
+    it.valid = false;
+    if (GATHER) {
+        const int mchunks = ((g.mode == 0 ? g.g : g.G) + 3) / 4;
+        const int grp = item / mchunks, mc = item % mchunks;
+        long long m0, key0;
+        int cnt;
+        if (g.mode == 0) {
+            if (!g.plan[0] || grp >= g.plan[2]) return it;
+            const int *rp = g.plan + g.pl.rp();
+            const int b = find_seg(rp, g.S, grp);
+            const int i = grp - rp[b];
+            const int n = g.cu[b + 1] - g.cu[b];
+            const int lo = i * g.g;
+            cnt = (lo + g.g < n ? lo + g.g : n) - lo;
+            m0 = (long long)g.cu[b] + lo;
+            key0 = g.cu[b];
+        } else {
+            const int kv = g.kv_len[grp];
+            if (kv < g.G || kv > g.n_max) return it;
+            cnt = g.G;
+            m0 = (long long)grp * g.G;
+            key0 = (long long)grp * g.n_max;
+        }
+        const int m = cnt - mc * 4;
+        if (m <= 0) return it;
+        it.valid = true;
+        it.m = m < 4 ? m : 4;
+        it.qrow0 = m0 + mc * 4;
+        it.out_row0 = it.qrow0;
+        it.key0 = key0;
+        it.t0 = 0;
+        it.nt = (g.c + KT - 1) / KT;
+        it.cand = g.cand + (long long)grp * g.c;
+    } else {
+        const int ntiles_max = (dd.n_max + KT - 1) / KT;
+        const int nch = (ntiles_max + kDecodeChunkTiles - 1) / kDecodeChunkTiles;
+        const int b = item / nch, ch = item % nch;
+        const int kv = dd.kv_len[b];
+        if (kv < dd.G || kv > dd.n_max) return it;
+        const int ntiles = (kv - 1) / KT + 1;
+        const int t0 = ch * kDecodeChunkTiles;
+        if (t0 >= ntiles) return it;
+        it.valid = true;
+        it.m = dd.Gq;
+        it.qrow0 = (long long)b * dd.Gq;
+        it.out_row0 = it.qrow0;
+        it.key0 = (long long)b * dd.n_max;
+        it.t0 = t0;
+        it.nt = (t0 + kDecodeChunkTiles < ntiles ? t0 + kDecodeChunkTiles : ntiles) - t0;
+        for (int r = 0; r < 4; ++r) it.bound[r] = dd.Gq == 1 ? kv - 1 : kv - dd.G + r;
+    }
+    return it;
+}
+
+__device__ __forceinline__ float reduce64(const uint32_t (&v0)[32], const uint32_t (&v1)[32], const float *w) {
+    float a[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) a[i] = 0.0f;
+#pragma unroll
+    for (int j = 0; j < 32; ++j) a[j & 7] = fmaf(w[j], fmaxf(__uint_as_float(v0[j]), 0.0f), a[j & 7]);
+#pragma unroll
+    for (int j = 0; j < 32; ++j) a[j & 7] = fmaf(w[32 + j], fmaxf(__uint_as_float(v1[j]), 0.0f), a[j & 7]);
+    return ((a[0] + a[1]) + (a[2] + a[3])) + ((a[4] + a[5]) + (a[6] + a[7]));
+}
+
+__device__ __forceinline__ void gather4(void *dst, const CUtensorMap *map, int x, int r0, int r1, int r2, int r3,
+                                        uint64_t *bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4, %5, %6, %7}], [%2];" ::"r"(tc::smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(tc::smem_u32(bar)), "r"(x), "r"(r0), "r"(r1), "r"(r2), "r"(r3)
+        : "memory");
+}
+
+template <bool GATHER>
+__global__ void __launch_bounds__(kThreads, 1)
+    stream_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_k,
+                     GatherArgs g, DecodeArgs dd, int nitems) {
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw = tc::smem_u32(smem_raw);
+    uint8_t *smem = smem_raw + (((raw + 1023u) & ~1023u) - raw);
+    uint8_t *qs = smem + kOffQ;
+    uint8_t *as = smem + kOffA;
+    float *wsm = reinterpret_cast<float *>(smem + kOffW);
+    StShared &sh = *reinterpret_cast<StShared *>(smem + kOffCtl);
+    volatile int *abort = &sh.abort;
+    unsigned *status = GATHER ? g.status : dd.status;
+    const float *wsrc = GATHER ? g.w : dd.w;
+    float *out = GATHER ? g.out : dd.spill;
+    const long long ld = GATHER ? (long long)g.c : (long long)dd.n_max;
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kStages; ++s) {
+            tc::mbar_init(&sh.afull[s], 1);
+            tc::mbar_init(&sh.aempty[s], 1);
+        }
+        tc::mbar_init(&sh.qfull, 1);
+        for (int b = 0; b < 2; ++b) {
+            tc::mbar_init(&sh.tfull[b], 1);
+            tc::mbar_init(&sh.tempty[b], kEpiWarps);
+        }
+        tc::mbar_init(&sh.drain, 1);
+        sh.abort = 0;
+        tc::fence_mbar_init();
+        tc::prefetch_tmap(&tmap_q);
+        tc::prefetch_tmap(&tmap_k);
+    }
+    if (warp == 1) {
+        tc::tmem_alloc(&sh.tmem_base, 512);
+        tc::tmem_relinquish();
+    }
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    const uint32_t tmem = sh.tmem_base;
+
+    uint32_t t = 0;     // key tiles consumed by this CTA (all roles agree)
+    uint32_t nq = 0;    // query loads so far
+    uint32_t mma_issued = 0;
+
+    for (int item = blockIdx.x; item < nitems; item += gridDim.x) {
+        const Item it = item_info<GATHER>(g, dd, item);
+        if (!it.valid) continue;
+        __syncthreads();
+        for (int i = threadIdx.x; i < 4 * S_H; i += kThreads)
+            wsm[i] = (i / S_H) < it.m ? wsrc[it.qrow0 * S_H + i] : 0.0f;
+        __syncthreads();
+        const uint32_t idesc = tc::idesc_bf16_f32(128, 64 * it.m);
+
+        if (warp == 0) {
+            bool ok = !*abort;
+            if (lane == 0 && ok) {
+                tc::mbar_arrive_expect_tx(&sh.qfull, kQBytes);
+                for (int kh = 0; kh < 2; ++kh)
+                    tc::tma_load_2d(qs + kh * kQSlice, &tmap_q, kh * 64, (int)(it.qrow0 * S_H), &sh.qfull);
+            }
+            for (int j = 0; j < it.nt && ok; ++j) {
+                const uint32_t tt = t + j, st = tt % kStages, ph = (tt / kStages) & 1u;
+                if (lane == 0) ok = tc::mbar_wait(&sh.aempty[st], ph ^ 1u, abort, status);
+                ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
+                if (!ok) break;
+                uint8_t *dst = as + st * kAStage;
+                if (GATHER) {
+                    if (lane == 0) tc::mbar_arrive_expect_tx(&sh.afull[st], kAStage);
+                    __syncwarp();
+                    int r[4];
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const int jj = j * KT + lane * 4 + i;
+                        const int pos = jj < g.c ? it.cand[jj] : -1;
+                        r[i] = (int)(it.key0 + (pos >= 0 ? pos : 0));
+                    }
+                    for (int kh = 0; kh < 2; ++kh)
+                        gather4(dst + kh * kASlice + lane * 4 * 128, &tmap_k, kh * 64, r[0], r[1], r[2], r[3],
+                                &sh.afull[st]);
+                } else if (lane == 0) {
+                    tc::mbar_arrive_expect_tx(&sh.afull[st], kAStage);
+                    const int row = (int)(it.key0 + (long long)(it.t0 + j) * KT);
+                    for (int kh = 0; kh < 2; ++kh) tc::tma_load_2d(dst + kh * kASlice, &tmap_k, kh * 64, row, &sh.afull[st]);
+                }
+            }
+        } else if (warp == 1) {
+            if (lane == 0) {
+                bool ok = tc::mbar_wait(&sh.qfull, nq & 1u, abort, status);
+                const uint32_t qbase = tc::smem_u32(qs);
+                for (int j = 0; j < it.nt && ok; ++j) {
+                    const uint32_t tt = t + j, st = tt % kStages, ph = (tt / kStages) & 1u, buf = tt & 1u;
+                    if (!(ok = tc::mbar_wait(&sh.afull[st], ph, abort, status))) break;
+                    if (!(ok = tc::mbar_wait(&sh.tempty[buf], ((tt >> 1) & 1u) ^ 1u, abort, status))) break;
+                    tc::fence_after_sync();
+                    const uint32_t abase = tc::smem_u32(as + st * kAStage);
+#pragma unroll
+                    for (int kk = 0; kk < 8; ++kk) {
+                        const uint32_t off_a = (kk >> 2) * kASlice + (kk & 3) * 32;
+                        const uint32_t off_q = (kk >> 2) * kQSlice + (kk & 3) * 32;
+                        tc::mma_bf16(tmem + buf * 256, tc::sw128_desc(abase + off_a), tc::sw128_desc(qbase + off_q),
+                                     idesc, kk > 0 ? 1u : 0u);
+                    }
+                    ++mma_issued;
+                    tc::mma_commit(&sh.tfull[buf]);
+                    tc::mma_commit(&sh.aempty[st]);
+                }
+            }
+        } else {
+            const int quarter = warp & 3;
+            const int qp = (warp - 2) >> 2;
+            bool ok = true;
+            for (int j = 0; j < it.nt; ++j) {
+                const uint32_t tt = t + j, buf = tt & 1u;
+                if (ok) ok = tc::mbar_wait(&sh.tfull[buf], (tt >> 1) & 1u, abort, status);
+                float sc[2] = {0.0f, 0.0f};
+                if (ok) {
+                    tc::fence_after_sync();
+                    const uint32_t taddr = tmem + ((uint32_t)(quarter * 32) << 16) + buf * 256 + qp * 128;
+                    uint32_t v0[32], v1[32], v2[32], v3[32];
+                    const bool r0 = 2 * qp < it.m, r1 = 2 * qp + 1 < it.m;
+                    if (r0) {
+                        tc::tmem_ld32(taddr, v0);
+                        tc::tmem_ld32(taddr + 32, v1);
+                    }
+                    if (r1) {
+                        tc::tmem_ld32(taddr + 64, v2);
+                        tc::tmem_ld32(taddr + 96, v3);
+                    }
+                    tc::tmem_wait_ld_all();
+                    if (r0) { tc::reg_fence(v0); tc::reg_fence(v1); }
+                    if (r1) { tc::reg_fence(v2); tc::reg_fence(v3); }
+                    tc::fence_before_sync();
+                    __syncwarp();
+                    if (lane == 0) tc::mbar_arrive(&sh.tempty[buf]);
+                    if (r0) sc[0] = reduce64(v0, v1, wsm + (2 * qp) * S_H);
+                    if (r1) sc[1] = reduce64(v2, v3, wsm + (2 * qp + 1) * S_H);
+                    const int kidx = quarter * 32 + lane;
+#pragma unroll
+                    for (int rr = 0; rr < 2; ++rr) {
+                        const int r = 2 * qp + rr;
+                        if (r >= it.m) continue;
+                        if (GATHER) {
+                            const int jj = j * KT + kidx;
+                            if (jj < g.c) out[(it.out_row0 + r) * ld + jj] = sc[rr];
+                        } else {
+                            const int s = (it.t0 + j) * KT + kidx;
+                            if (s <= it.bound[r]) out[(it.out_row0 + r) * ld + s] = sc[rr];
+                        }
+                    }
+                }
+            }
+        }
+        t += it.nt;
+        ++nq;
+    }
+
+    __syncthreads();
+    if (*abort) {
+        if (warp == 1 && lane == 0 && mma_issued) {
+            tc::mma_commit(&sh.drain);
+            tc::mbar_wait_drain(&sh.drain, 0);
+        }
+        if (warp == 0 && lane == 0) {
+            for (uint32_t tt = t > kStages ? t - kStages : 0; tt < t; ++tt)
+                tc::mbar_wait_drain(&sh.afull[tt % kStages], (tt / kStages) & 1u);
+            if (nq) tc::mbar_wait_drain(&sh.qfull, (nq - 1) & 1u);
+        }
+    }
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    if (warp == 1) tc::tmem_dealloc(tmem, 512);
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn2() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    if (!fn) {
+        cudaDriverEntryPointQueryResult q;
+        void *p = nullptr;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    }
+    return fn;
+}
+
+bool map2d(CUtensorMap *m, const void *base, unsigned long long rows, unsigned box_rows) {
+    PFN_cuTensorMapEncodeTiled_v12000 fn = encode_fn2();
+    if (!fn) return false;
+    memset(m, 0, sizeof(*m));
+    cuuint64_t dims[2] = {(cuuint64_t)S_D, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)S_D * 2};
+    cuuint32_t box[2] = {64u, box_rows};
+    cuuint32_t estr[2] = {1u, 1u};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+int sm_count() {
+    static int sms = 0;
+    if (!sms) {
+        int dev = 0;
+        cudaGetDevice(&dev);
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    }
+    return sms;
+}
+
+}  // namespace
+
+bool tc_decode_supported(int H, int d, int dtype, int rows_per_request) {
+    return H == S_H && d == S_D && dtype == 0 && rows_per_request >= 1 && rows_per_request <= 4;
+}
+bool tc_gather_supported(int H, int d, int dtype, int group) {
+    (void)group;
+    return H == S_H && d == S_D && dtype == 0;
+}
+
+cudaError_t launch_decode_tc(const DecodeArgs &a, cudaStream_t st) {
+    CUtensorMap mq, mk;
+    if (!map2d(&mq, a.q, (unsigned long long)a.B * a.Gq * S_H, 256) ||
+        !map2d(&mk, a.kc, (unsigned long long)a.B * a.n_max, KT))
+        return cudaErrorInvalidValue;
+    const int ntiles_max = (a.n_max + KT - 1) / KT;
+    const int nitems = a.B * ((ntiles_max + kDecodeChunkTiles - 1) / kDecodeChunkTiles);
+    cudaError_t e = cudaFuncSetAttribute(stream_tc_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)kSmemBytes);
+    if (e != cudaSuccess) return e;
+    GatherArgs g{};
+    TraceScope ts("decode_tc", st);
+    const int grid = nitems < sm_count() ? nitems : sm_count();
+    stream_tc_kernel<false><<<grid, kThreads, kSmemBytes, st>>>(mq, mk, g, a, nitems);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_gather_tc(const GatherArgs &a, cudaStream_t st) {
+    const long long qrows = a.mode == 0 ? (long long)a.cu_T : (long long)a.G * a.nitems;
+    const long long krows = a.mode == 0 ? (long long)a.cu_T : (long long)a.nitems * a.n_max;
+    CUtensorMap mq, mk;
+    if (!map2d(&mq, a.q, (unsigned long long)qrows * S_H, 256) || !map2d(&mk, a.k, (unsigned long long)krows, 1))
+        return cudaErrorInvalidValue;
+    const int mchunks = ((a.mode == 0 ? a.g : a.G) + 3) / 4;
+    const int nitems = a.nitems * mchunks;
+    cudaError_t e = cudaFuncSetAttribute(stream_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)kSmemBytes);
+    if (e != cudaSuccess) return e;
+    DecodeArgs dd{};
+    TraceScope ts("gather_tc", st);
+    const int grid = nitems < sm_count() ? nitems : sm_count();
+    if (grid <= 0) return cudaSuccess;
+    stream_tc_kernel<true><<<grid, kThreads, kSmemBytes, st>>>(mq, mk, a, dd, nitems);
+    return cudaGetLastError();
+}
+
+}  // namespace idx

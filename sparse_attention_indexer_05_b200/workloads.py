@@ -60,24 +60,29 @@ def keys(L: int, d: int, planted_frac: float, seed: int, sub: int = 0, scale: fl
 
 
 def queries_ar1(L: int, H: int, d: int, rho: float, seed: int, sub: int = 0, bf16: bool = True,
-                chunk: int = 4096) -> np.ndarray:
-    """[L, H, d] AR(1) queries along positions (rows generated in chunks)."""
-    g = rng_for(seed, _Q, sub)
-    out = np.empty((L, H * d), np.uint16 if bf16 else np.float32)
-    s = np.float32(np.sqrt(1.0 - rho * rho))
-    r = np.float32(rho)
-    prev = None
-    for c0 in range(0, L, chunk):
-        c1 = min(L, c0 + chunk)
-        e = g.standard_normal((c1 - c0, H * d), dtype=np.float32)
-        for i in range(c1 - c0):
-            if prev is None:
-                prev = e[i].copy()
-            else:
-                prev *= r
-                prev += s * e[i]
-            e[i] = prev
-        out[c0:c1] = bf16_bits(e) if bf16 else e
+                col_block: int = 512, threads: int = 8) -> np.ndarray:
+    """[L, H, d] AR(1) queries along positions.  The H*d columns are drawn in
+    blocks of `col_block`, each block from its own stream (seed, sub, block),
+    so blocks are generated in parallel; within a block the recurrence runs
+    along positions."""
+    from concurrent.futures import ThreadPoolExecutor
+    from scipy.signal import lfilter
+
+    HD = H * d
+    out = np.empty((L, HD), np.uint16 if bf16 else np.float32)
+    s = float(np.sqrt(1.0 - rho * rho))
+
+    def block(c0):
+        c1 = min(HD, c0 + col_block)
+        # drawn as [columns, positions] so the recurrence runs along contiguous memory
+        e = rng_for(seed, _Q, sub * 1000003 + c0 // col_block).standard_normal((c1 - c0, L), dtype=np.float32)
+        e[:, 0] /= np.float32(s)  # so that q[0] = e[0]
+        y = lfilter(np.array([s], np.float32), np.array([1.0, -rho], np.float32), e, axis=1)
+        y = np.ascontiguousarray(y.T, dtype=np.float32)
+        out[:, c0:c1] = bf16_bits(y) if bf16 else y
+
+    with ThreadPoolExecutor(max_workers=max(1, threads)) as ex:
+        list(ex.map(block, range(0, HD, col_block)))
     return out.reshape(L, H, d)
 
 
@@ -163,10 +168,16 @@ def decode(B=64, n=131072, G=2, H=64, d=128, topk=2048, c=4096, rho=0.95, plante
            kv_len=None, n_max=None, name="decode") -> Decode:
     """Decode step over a contiguous cache [B, n_max, d]; request b's keys use
     the key recipe with sub-stream b; queries are AR(1) across the G positions."""
+    from concurrent.futures import ThreadPoolExecutor
+
     n_max = int(n_max or n)
     kc = np.zeros((B, n_max, d), np.uint16)
-    for b in range(B):
+
+    def fill(b):
         kc[b] = keys(n_max, d, planted, seed, sub=1000 + b)
+
+    with ThreadPoolExecutor(max_workers=8) as ex:
+        list(ex.map(fill, range(B)))
     e = rng_for(seed, _DEC_Q).standard_normal((B, G, H, d), dtype=np.float32)
     s = np.float32(np.sqrt(1.0 - rho * rho))
     qf = np.empty_like(e)
