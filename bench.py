@@ -22,7 +22,6 @@ of the same workload.
 from __future__ import annotations
 
 import argparse
-import datetime
 import json
 import math
 import os
@@ -51,6 +50,11 @@ def parse():
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-decode", action="store_true")
     p.add_argument("--cpu-rows", type=int, default=64, help="oracle sample rows (dense + refine) per CPU step")
+    p.add_argument("--no-cpu", action="store_true", help="skip the CPU-oracle baseline")
+    p.add_argument("--tokens", type=int, default=L_TOK,
+                   help="batch length (profiling runs use a smaller case; the bench line uses 131072)")
+    p.add_argument("--only", default="all", choices=["all", "dense", "refine"],
+                   help="profiling runs: time one half of the step only")
     return p.parse_args()
 
 
@@ -207,51 +211,49 @@ def main():
     if args.impl == "reference":
         return run_reference(args)
     import torch
-    import torch.distributed as dist
-
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    if world > 1:
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
-    torch.cuda.set_device(local)
-    dev = torch.device("cuda", local)
 
     import sparse_attention_indexer_05_b200 as idx
     from sparse_attention_indexer_05_b200 import _native as N
+    from sparse_attention_indexer_05_b200 import multirank as M
     from sparse_attention_indexer_05_b200 import workloads as W
+
+    rank, world, local = M.init("nccl")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
     lib = N.lib()
 
     def barrier():
-        if world > 1:
-            dist.barrier(device_ids=[local])
+        M.barrier(dev)
 
     def max_over_ranks(x):
-        if world == 1:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+        return M.max_over_ranks(x, dev)
 
-    P = W.cfg_long_single(seed=rank)
-    cu1_h = np.array([0, L_TOK], np.int32)
-    cu2_h = np.array([0, L_TOK // 2, L_TOK], np.int32)
+    L = args.tokens
+    P = W.cfg_long_single(seed=M.rank_seed(rank), L=L)
+    cu1_h = np.array([0, L], np.int32)
+    cu2_h = np.array([0, L // 2, L], np.int32)
     q, k, w = to_dev(P.q, dev), to_dev(P.k, dev), to_dev(P.w, dev)
     cu1, cu2 = to_dev(cu1_h, dev), to_dev(cu2_h, dev)
-    ws1 = torch.empty(idx.dense_workspace_size(L_TOK, H, D, TOPK, 1), dtype=torch.uint8, device=dev)
-    ws2 = torch.empty(idx.pivot_workspace_size(L_TOK, H, D, TOPK, 2, G_REF, C_REF, "refine"), dtype=torch.uint8,
+    do_dense = args.only in ("all", "dense")
+    do_refine = args.only in ("all", "refine")
+    ws1 = torch.empty(idx.dense_workspace_size(L, H, D, TOPK, 1) if do_dense else 256, dtype=torch.uint8,
                       device=dev)
-    o1 = torch.empty(L_TOK, TOPK, dtype=torch.int32, device=dev)
-    o2 = torch.empty(L_TOK, TOPK, dtype=torch.int32, device=dev)
+    ws2 = torch.empty(idx.pivot_workspace_size(L, H, D, TOPK, 2, G_REF, C_REF, "refine") if do_refine else 256,
+                      dtype=torch.uint8, device=dev)
+    o1 = torch.empty(L, TOPK, dtype=torch.int32, device=dev)
+    o2 = torch.empty(L, TOPK, dtype=torch.int32, device=dev)
 
     def step(qq=q, kk=k, ww=w, c1=cu1, c2=cu2):
-        idx.dense_topk(qq, kk, ww, c1, TOPK, out_idx=o1, workspace=ws1)
-        idx.pivot_topk(qq, kk, ww, c2, TOPK, G_REF, C_REF, "refine", out_idx=o2, workspace=ws2)
+        if do_dense:
+            idx.dense_topk(qq, kk, ww, c1, TOPK, out_idx=o1, workspace=ws1)
+        if do_refine:
+            idx.pivot_topk(qq, kk, ww, c2, TOPK, G_REF, C_REF, "refine", out_idx=o2, workspace=ws2)
 
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize()
-    assert idx.device_status(ws1) == "IDX_OK" and idx.device_status(ws2) == "IDX_OK"
+    assert (not do_dense or idx.device_status(ws1) == "IDX_OK") and \
+        (not do_refine or idx.device_status(ws2) == "IDX_OK")
 
     stream = torch.cuda.current_stream()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -270,17 +272,17 @@ def main():
     barrier()
     ms = max_over_ranks(e0.elapsed_time(e1) / args.steps)
     nlaunch, tr = trace_report(lib)
-    rows_per_step = 2 * L_TOK
+    rows_per_step = L * (int(do_dense) + int(do_refine))
     value = world * rows_per_step / (ms / 1000.0)
 
     bf16_peak, bf16_sus, hbm_peak, peak_src = peaks()
     n_dense, ms_dense = tr.get("dense/score_tc", (0, 0.0))
     dense_ms = ms_dense / max(1, n_dense)
-    achieved = dense_flops_single() / (dense_ms / 1000.0) / 1e12 if dense_ms > 0 else None
+    achieved = dense_flops_single(L) / (dense_ms / 1000.0) / 1e12 if dense_ms > 0 else None
     roof = {"kernel": "score_tc (dense pass)", "bound": "tensor", "achieved": achieved,
             "peak": bf16_sus, "unit": "TFLOP/s", "frac": (achieved / bf16_sus) if achieved else None,
             "traffic": None, "peak_kind": f"{peak_src} bf16 sustained (kernel timed inside a long step)",
-            "flops_per_launch": dense_flops_single(), "ms_per_launch": dense_ms}
+            "flops_per_launch": dense_flops_single(L), "ms_per_launch": dense_ms}
 
     per_kernel = {name: {"launches": c, "ms_total": t, "ms_per_step": t / args.steps} for name, (c, t) in tr.items()}
 
@@ -322,7 +324,7 @@ def main():
     # ------------------------------------------------------------- decode
     dec = None
     if not args.no_decode:
-        Dd = W.cfg_decode(seed=rank)
+        Dd = W.cfg_decode(seed=M.rank_seed(rank))
         dq_, dkc, dw_, dkv = to_dev(Dd.q, dev), to_dev(Dd.kcache, dev), to_dev(Dd.w, dev), to_dev(Dd.kv_len, dev)
         wsd = torch.empty(max(idx.decode_workspace_size(DEC_B, DEC_G, DEC_N, H, D, TOPK, C_REF, m)
                               for m in ("dense", "refine")), dtype=torch.uint8, device=dev)
@@ -352,7 +354,7 @@ def main():
 
     # -------------------------------------------------------- CPU baseline
     cpu = None
-    if rank == 0 and world == 1:
+    if rank == 0 and world == 1 and not args.no_cpu and L == L_TOK:
         v, dt, threads, desc = oracle_sample(P, args.cpu_rows)
         cpu = {"value": v, "unit": "queries/s", "cores": threads, "kind": "oracle", "sample": desc,
                "seconds": dt}
@@ -361,8 +363,10 @@ def main():
         "metric": METRIC, "value": value, "unit": "queries/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": "long_prefill_131072_dense+refine_g16_c4096", "tokens": L_TOK, "H": H, "d": D,
-                   "topk": TOPK, "dense_requests": [L_TOK], "refine_requests": [L_TOK // 2, L_TOK // 2],
+        "config": {"workload": f"long_prefill_{L}_" + {"all": "dense+refine", "dense": "dense",
+                                                          "refine": "refine"}[args.only] + "_g16_c4096",
+                   "tokens": L, "H": H, "d": D,
+                   "topk": TOPK, "dense_requests": [L], "refine_requests": [L // 2, L // 2],
                    "g": G_REF, "c": C_REF, "parallelism": f"dp{world} (independent batches)",
                    "l2": "inputs larger than L2 (q is 2 GiB)"},
         "tflops_dense": achieved, "roofline": roof, "cpu_baseline": cpu, "e2e": e2e, "clocks": clk,
@@ -370,8 +374,7 @@ def main():
     }
     if rank == 0:
         print(json.dumps(line))
-    if world > 1:
-        dist.destroy_process_group()
+    M.finish()
     return 0
 
 

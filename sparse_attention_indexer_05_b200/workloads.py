@@ -70,6 +70,8 @@ def queries_ar1(L: int, H: int, d: int, rho: float, seed: int, sub: int = 0, bf1
 
     HD = H * d
     out = np.empty((L, HD), np.uint16 if bf16 else np.float32)
+    if L == 0:
+        return out.reshape(0, H, d)
     s = float(np.sqrt(1.0 - rho * rho))
 
     def block(c0):

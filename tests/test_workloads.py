@@ -45,3 +45,8 @@ def test_weights_range_and_configs_shapes():
     S = W.small_fp32()
     assert S.q.dtype == np.float32 and S.q.shape == (2048, 4, 64)
     assert abs(S.q.std() - 1 / 8) < 0.005
+
+
+def test_empty_request_in_a_pack():
+    P = W.prefill([5, 0, 3], H=2, d=8, topk=2)
+    assert P.q.shape == (8, 2, 8) and P.cu_seqlens.tolist() == [0, 5, 5, 8]
