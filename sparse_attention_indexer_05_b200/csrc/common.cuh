@@ -122,18 +122,20 @@ __device__ __forceinline__ void sel_offer(RowSel &st, unsigned *hist, unsigned l
     }
 }
 
-// Warp-level suffix search over a 256-entry histogram h (lane l owns bins
-// 8l..8l+7): returns the largest bin b with sum(h[b..255]) >= need (or -1
+// Warp-level suffix search over a 256-entry histogram h (16-byte aligned;
+// lane l owns bins 8l..8l+7): returns the largest bin b with sum(h[b..255]) >= need (or -1
 // if the total is below need) and, through *above, sum(h[b+1..255]).
 __device__ __forceinline__ int warp_find_bin(const unsigned *h, unsigned need, unsigned *above) {
     const int lane = threadIdx.x & 31;
     unsigned loc[8];
+    // two 16-byte loads per lane: 4 wavefronts each, no bank conflicts
+    const uint4 *h4 = reinterpret_cast<const uint4 *>(h) + lane * 2;
+    const uint4 x0 = h4[0], x1 = h4[1];
+    loc[0] = x0.x; loc[1] = x0.y; loc[2] = x0.z; loc[3] = x0.w;
+    loc[4] = x1.x; loc[5] = x1.y; loc[6] = x1.z; loc[7] = x1.w;
     unsigned sum = 0;
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-        loc[i] = h[lane * 8 + i];
-        sum += loc[i];
-    }
+    for (int i = 0; i < 8; ++i) sum += loc[i];
     // inclusive suffix sum over lanes: suf(l) = sum of lanes >= l
     unsigned suf = sum;
 #pragma unroll
@@ -257,8 +259,9 @@ __device__ __forceinline__ void sel_compact(RowSel &st, unsigned long long *buf_
 // ksel keys have been appended (from the largest appended ord, 12 octaves
 // below it to 4 above), cut the buffer when it is close to full, and raise
 // the admission threshold.  Called only between tiles, when no warp offers.
+// `slack` = the most keys one row can be offered before the next upkeep.
 __device__ __forceinline__ void sel_maintain(RowSel &st, unsigned *hist, unsigned long long *buf_row,
-                                             unsigned cap, unsigned ksel, unsigned *scratch) {
+                                             unsigned cap, unsigned ksel, unsigned *scratch, int slack) {
     const int lane = threadIdx.x & 31;
     __syncwarp();  // the warp's appends (buffer, counts) are visible to all its lanes
     if (st.base == kBaseUnset && st.cnt >= ksel) {
@@ -279,7 +282,7 @@ __device__ __forceinline__ void sel_maintain(RowSel &st, unsigned *hist, unsigne
         if (lane == 0) st.base = base;
         __syncwarp();
     }
-    if ((int)st.cnt > (int)cap - 128) sel_compact(st, buf_row, cap, ksel, scratch);
+    if ((int)st.cnt > (int)cap - slack) sel_compact(st, buf_row, cap, ksel, scratch);
     if (st.base != kBaseUnset) sel_update_threshold(st, hist, ksel);
 }
 

@@ -32,8 +32,9 @@ namespace {
 
 constexpr int TC_H = 64;
 constexpr int TC_D = 128;
-constexpr int kThreads = 320;
-constexpr int kEpiWarps = 8;
+constexpr int kEpiWarps = 16;                         // 4 per TMEM lane quarter, one query each per half
+constexpr int kThreads = 64 + 32 * kEpiWarps;         // + TMA warp + MMA warp
+constexpr int kMaintEvery = 2;                        // tiles between candidate-filter upkeeps
 constexpr int kStages = 2;                            // key-tile stages
 constexpr uint32_t kQHalfBytes = 256 * 128;           // one half, one 64-column K slice (32 KB)
 constexpr uint32_t kQBytes = 4 * kQHalfBytes;         // 2 halves x 2 K slices (128 KB)
@@ -58,18 +59,32 @@ constexpr size_t kOffK = kOffQ + kQBytes;
 constexpr size_t kOffW = kOffK + (size_t)kStages * kKStageBytes;
 constexpr size_t kOffHist = kOffW + (size_t)RB * TC_H * 4;
 constexpr size_t kOffScr = kOffHist + (size_t)RB * kBins * 4;
-constexpr size_t kOffCtl = kOffScr + (size_t)kEpiWarps * 256 * 4;
+constexpr size_t kOffCtl = kOffScr + (size_t)RB * 256 * 4;
 constexpr size_t kSmemBytes = kOffCtl + sizeof(TcShared) + 1024;  // + alignment slack
 
-// sum_j w[j] * max(v[j], 0) over 64 heads held in four 32-register groups
+// sum_j w[j] * max(v[j], 0) over 64 heads held in two 32-register groups;
+// w read as float4 (16-byte aligned); 8 independent partial sums.
 __device__ __forceinline__ float head_reduce(const uint32_t (&v0)[32], const uint32_t (&v1)[32], const float *w) {
+    const float4 *w4 = reinterpret_cast<const float4 *>(w);
     float a[8];
 #pragma unroll
     for (int i = 0; i < 8; ++i) a[i] = 0.0f;
 #pragma unroll
-    for (int j = 0; j < 32; ++j) a[j & 7] = fmaf(w[j], fmaxf(__uint_as_float(v0[j]), 0.0f), a[j & 7]);
+    for (int j4 = 0; j4 < 8; ++j4) {
+        const float4 wv = w4[j4];
+        a[(4 * j4 + 0) & 7] = fmaf(wv.x, fmaxf(__uint_as_float(v0[4 * j4 + 0]), 0.0f), a[(4 * j4 + 0) & 7]);
+        a[(4 * j4 + 1) & 7] = fmaf(wv.y, fmaxf(__uint_as_float(v0[4 * j4 + 1]), 0.0f), a[(4 * j4 + 1) & 7]);
+        a[(4 * j4 + 2) & 7] = fmaf(wv.z, fmaxf(__uint_as_float(v0[4 * j4 + 2]), 0.0f), a[(4 * j4 + 2) & 7]);
+        a[(4 * j4 + 3) & 7] = fmaf(wv.w, fmaxf(__uint_as_float(v0[4 * j4 + 3]), 0.0f), a[(4 * j4 + 3) & 7]);
+    }
 #pragma unroll
-    for (int j = 0; j < 32; ++j) a[j & 7] = fmaf(w[32 + j], fmaxf(__uint_as_float(v1[j]), 0.0f), a[j & 7]);
+    for (int j4 = 0; j4 < 8; ++j4) {
+        const float4 wv = w4[8 + j4];
+        a[(4 * j4 + 0) & 7] = fmaf(wv.x, fmaxf(__uint_as_float(v1[4 * j4 + 0]), 0.0f), a[(4 * j4 + 0) & 7]);
+        a[(4 * j4 + 1) & 7] = fmaf(wv.y, fmaxf(__uint_as_float(v1[4 * j4 + 1]), 0.0f), a[(4 * j4 + 1) & 7]);
+        a[(4 * j4 + 2) & 7] = fmaf(wv.z, fmaxf(__uint_as_float(v1[4 * j4 + 2]), 0.0f), a[(4 * j4 + 2) & 7]);
+        a[(4 * j4 + 3) & 7] = fmaf(wv.w, fmaxf(__uint_as_float(v1[4 * j4 + 3]), 0.0f), a[(4 * j4 + 3) & 7]);
+    }
     return ((a[0] + a[1]) + (a[2] + a[3])) + ((a[4] + a[5]) + (a[6] + a[7]));
 }
 
@@ -140,12 +155,15 @@ __global__ void __launch_bounds__(kThreads, 1)
             // head weights of the block's rows, zero for rows past the request
             for (int i = threadIdx.x - 64; i < RB * TC_H; i += kEpiWarps * 32)
                 wsm[i] = (i / TC_H) < bi.nrows ? a.w[(long long)bi.row0 * TC_H + i] : 0.0f;
-            if (lane == 0) {
-                sh.bound[e] = e < bi.nrows ? row_bound(bi.i0 + e, bi.n, a.g) : -1;
-                sh.slot[e] = -1;
-                if (a.sink == SINK_SPILL && e < bi.nrows && a.slot_of_row) sh.slot[e] = a.slot_of_row[bi.row0 + e];
+            if (e < RB) {
+                if (lane == 0) {
+                    sh.bound[e] = e < bi.nrows ? row_bound(bi.i0 + e, bi.n, a.g) : -1;
+                    sh.slot[e] = -1;
+                    if (a.sink == SINK_SPILL && e < bi.nrows && a.slot_of_row)
+                        sh.slot[e] = a.slot_of_row[bi.row0 + e];
+                }
+                if (a.sink == SINK_FILTER) sel_init(sh.sel[e], hist + e * kBins);
             }
-            if (a.sink == SINK_FILTER) sel_init(sh.sel[e], hist + e * kBins);
         }
         __syncthreads();
 
@@ -196,53 +214,43 @@ __global__ void __launch_bounds__(kThreads, 1)
         } else {
             const int e = warp - 2;
             const int quarter = warp & 3;
-            const int qp = e >> 2;
+            const int qi = e >> 2;  // query of each half handled by this warp
             const int key_in_tile = quarter * 32 + lane;
             bool ok = true;
             for (int j = 0; j < ntiles; ++j) {
                 const uint32_t t = kt + j;
                 const int s = j * KT + key_in_tile;
                 for (int h = 0; h < 2; ++h) {
-                    float score[2] = {0.0f, 0.0f};
+                    float score = 0.0f;
+                    const int r = h * 4 + qi;
                     if (ok) ok = tc::mbar_wait(&sh.tfull[h], t & 1u, abort, a.status);
                     if (ok) {
                         tc::fence_after_sync();
-                        const uint32_t col = h * 256 + qp * 128;
-                        const uint32_t taddr = tmem + ((uint32_t)(quarter * 32) << 16) + col;
-                        uint32_t v0[32], v1[32], v2[32], v3[32];
+                        const uint32_t taddr = tmem + ((uint32_t)(quarter * 32) << 16) + h * 256 + qi * 64;
+                        uint32_t v0[32], v1[32];
                         tc::tmem_ld32(taddr, v0);
                         tc::tmem_ld32(taddr + 32, v1);
-                        tc::tmem_ld32(taddr + 64, v2);
-                        tc::tmem_ld32(taddr + 96, v3);
                         tc::tmem_wait_ld_all();
                         tc::reg_fence(v0);
                         tc::reg_fence(v1);
-                        tc::reg_fence(v2);
-                        tc::reg_fence(v3);
                         tc::fence_before_sync();
                         __syncwarp();
                         if (lane == 0) tc::mbar_arrive(&sh.tempty[h]);
-                        const int qa = h * 4 + qp * 2;
-                        score[0] = head_reduce(v0, v1, wsm + qa * TC_H);
-                        score[1] = head_reduce(v2, v3, wsm + (qa + 1) * TC_H);
+                        score = head_reduce(v0, v1, wsm + r * TC_H);
                     }
-#pragma unroll
-                    for (int qq = 0; qq < 2; ++qq) {
-                        const int r = h * 4 + qp * 2 + qq;
-                        const bool valid = ok && s <= sh.bound[r];
-                        if (a.sink == SINK_FILTER) {
-                            sel_offer(sh.sel[r], hist + r * kBins, a.buf + ((long long)bi.row0 + r) * a.cap, a.cap,
-                                      valid, score[qq], s, a.status);
-                        } else if (valid && sh.slot[r] >= 0) {
-                            a.spill[(long long)sh.slot[r] * a.ld + s] = score[qq];
-                        }
+                    const bool valid = ok && s <= sh.bound[r];
+                    if (a.sink == SINK_FILTER) {
+                        sel_offer(sh.sel[r], hist + r * kBins, a.buf + ((long long)bi.row0 + r) * a.cap, a.cap, valid,
+                                  score, s, a.status);
+                    } else if (valid && sh.slot[r] >= 0) {
+                        a.spill[(long long)sh.slot[r] * a.ld + s] = score;
                     }
                 }
-                if (a.sink == SINK_FILTER) {
+                if (a.sink == SINK_FILTER && ((j % kMaintEvery) == kMaintEvery - 1 || j == ntiles - 1)) {
                     tc::named_bar_sync(1, kEpiWarps * 32);
                     if (e < bi.nrows)
                         sel_maintain(sh.sel[e], hist + e * kBins, a.buf + ((long long)bi.row0 + e) * a.cap, a.cap,
-                                     a.ksel, scr + e * 256);
+                                     a.ksel, scr + e * 256, KT * kMaintEvery);
                     tc::named_bar_sync(1, kEpiWarps * 32);
                 }
             }

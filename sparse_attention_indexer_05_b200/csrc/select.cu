@@ -53,54 +53,108 @@ __device__ unsigned block_sum(unsigned v, unsigned *red) {
     return t;
 }
 
+constexpr int kMaxBins = 4096;  // widest radix digit: 12 bits
+
 struct SelShared {
-    unsigned hist[256];
+    unsigned hist[kMaxBins];
     unsigned red[32];
+    unsigned red2[32];
     int dgt;
     unsigned above;
     unsigned inbin;
 };
 
+// Digits of the 64-bit key, most significant first: 12 + 12 + 8 bits of the
+// score's ord (the first digit separates exponents, so the k-th key's bin is
+// already narrow), then 12 + 12 + 8 bits of the position part (ties only).
+__device__ __forceinline__ int digit_bits(int pass) { return (pass % 3 == 2) ? 8 : 12; }
+
+// Block-wide: the largest bin b of hist[0..nbins) with sum(hist[b..]) >= need;
+// writes b, sum(hist[b+1..]) and hist[b] to sh.  nbins is a multiple of 8
+// and at most 8 * blockDim.x.
+__device__ void block_find_bin(SelShared &sh, int nbins, unsigned need) {
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nw = blockDim.x >> 5;
+    const int per = 8;
+    const bool own = tid * per < nbins;
+    unsigned loc[per];
+    unsigned sum = 0;
+#pragma unroll
+    for (int i = 0; i < per; ++i) {
+        loc[i] = own ? sh.hist[tid * per + i] : 0u;
+        sum += loc[i];
+    }
+    // inclusive suffix sum over threads: suf(t) = sum of threads >= t
+    unsigned suf = sum;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const unsigned v = __shfl_down_sync(0xFFFFFFFFu, suf, o);
+        if (lane + o < 32) suf += v;
+    }
+    if (lane == 0) sh.red2[warp] = suf;  // warp total
+    __syncthreads();
+    unsigned after = 0;  // totals of the warps above this one
+    for (int w2 = warp + 1; w2 < nw; ++w2) after += sh.red2[w2];
+    suf += after;
+    if (suf >= need && suf - sum < need) {
+        unsigned run = suf - sum;
+        for (int i = per - 1; i >= 0; --i) {
+            if (run + loc[i] >= need) {
+                sh.dgt = tid * per + i;
+                sh.above = run;
+                sh.inbin = loc[i];
+                break;
+            }
+            run += loc[i];
+        }
+    }
+    __syncthreads();
+}
+
 template <class Src>
 __device__ void block_select(const Src &src, int k, int *out_idx, float *out_score, SelShared &sh,
                              unsigned *bm, unsigned *gpre, int wcap, unsigned *status) {
-    const int tid = threadIdx.x, nt = blockDim.x;
-    unsigned nvl = 0;
-    for (int i = tid; i < src.n; i += nt) nvl += src.key(i) != 0ull;
-    const unsigned nv = block_sum(nvl, sh.red);
+    const int tid = threadIdx.x, nt = blockDim.x, lane = tid & 31;
     unsigned long long K = 1ull;
-    if (nv > (unsigned)k) {
+    unsigned nv = 0;
+    {
         unsigned long long prefix = 0ull, mask = 0ull;
         unsigned need = (unsigned)k;
-        for (int shift = 56; shift >= 0; shift -= 8) {
-            for (int i = tid; i < 256; i += nt) sh.hist[i] = 0u;
+        int shift = 64;
+        for (int pass = 0; pass < 6; ++pass) {
+            const int bits = digit_bits(pass);
+            shift -= bits;
+            const unsigned dmask = (1u << bits) - 1u;
+            for (int i = tid; i < (1 << bits); i += nt) sh.hist[i] = 0u;
+            if (tid == 0) sh.dgt = -1;
             __syncthreads();
-            for (int i = tid; i < src.n; i += nt) {
-                const unsigned long long key = src.key(i);
-                if (key != 0ull && (key & mask) == prefix)
-                    atomicAdd(&sh.hist[(unsigned)(key >> shift) & 255u], 1u);
+            unsigned nvl = 0;
+            for (int base = 0; base < src.n; base += nt) {
+                const int i = base + tid;
+                unsigned long long key = i < src.n ? src.key(i) : 0ull;
+                const bool act = key != 0ull && (key & mask) == prefix;
+                nvl += key != 0ull;
+                const unsigned dg = act ? (unsigned)(key >> shift) & dmask : 0xFFFFFFFFu;
+                const unsigned m = __match_any_sync(0xFFFFFFFFu, dg);
+                if (act && lane == __ffs(m) - 1) atomicAdd(&sh.hist[dg], (unsigned)__popc(m));
             }
-            __syncthreads();
-            if (tid < 32) {
-                unsigned above;
-                const int d = warp_find_bin(sh.hist, need, &above);
-                if (tid == 0) {
-                    sh.dgt = d;
-                    sh.above = above;
-                    sh.inbin = d >= 0 ? sh.hist[d] : 0u;
-                }
+            if (pass == 0) {
+                nv = block_sum(nvl, sh.red);  // also orders the histogram updates
+                if (nv <= (unsigned)k) break;  // every valid entry is selected
+            } else {
+                __syncthreads();
             }
-            __syncthreads();
+            block_find_bin(sh, 1 << bits, need);
             const int d = sh.dgt;
             const unsigned above = sh.above, inbin = sh.inbin;
             __syncthreads();
             if (d < 0) break;  // unreachable when nv > k
             need -= above;
             prefix |= (unsigned long long)d << shift;
-            mask |= 0xFFull << shift;
-            if (inbin == need) break;
+            mask |= (unsigned long long)dmask << shift;
+            K = prefix;
+            if (inbin == need) break;  // the whole bin is selected
         }
-        K = prefix;
+        if (nv <= (unsigned)k) K = 1ull;
     }
     const int nsel = (int)(nv < (unsigned)k ? nv : (unsigned)k);
     if (nsel > 0) {
