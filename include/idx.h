@@ -129,6 +129,32 @@ idx_status idx_decode_topk(const void *q, const void *kcache, const int *kv_len,
                            idx_dtype dtype, int *out_idx, float *out_score, void *ws,
                            size_t ws_bytes, idx_stream_t stream);
 
+/* ----------------------------------------------- no-allocation variant */
+
+/* The pages have no counterpart of this entry point; it exists for callers
+ * that cannot allocate device memory, such as a plugin inside another
+ * runtime that owns all device memory and hands out no workspace, or a
+ * serving loop that must not allocate once decoding runs.
+ *
+ * Same result as idx_decode_topk with mode IDX_MODE_DENSE (c unused), same
+ * tensors and layouts, but no workspace argument: the scratch is a fixed
+ * 32 MiB device array inside the library, reserved on every GPU that loads
+ * the library until the process exits.  Nothing is allocated by the call.
+ *   - Limit: 256 + 4*B*G*n_max bytes must fit in 32 MiB (B*G*n_max <=
+ *     8388544, e.g. 32 requests x 2 queries x 131071 tokens); larger calls
+ *     return IDX_ERR_UNSUPPORTED with a message on stderr and launch nothing.
+ *   - The first call on a device looks up the array's device address
+ *     (cudaGetSymbolAddress); make that first call before any stream capture.
+ *   - Every call uses the same array, which keeps the last call's contents
+ *     (the status word is cleared at the start of each call): calls whose
+ *     kernels overlap on the GPU -- other streams, other host threads --
+ *     race and corrupt each other's results.  Order them on one stream.
+ *   - The device status word lives in the shared array and is not
+ *     returned; requests whose kv_len is out of range come back as rows of -1. */
+idx_status idx_decode_topk_noalloc(const void *q, const void *kcache, const int *kv_len, const float *w,
+                                   int B, int G, int n_max, int H, int d, int topk, idx_dtype dtype,
+                                   int *out_idx, float *out_score, idx_stream_t stream);
+
 /* ------------------------------------------------------ status, debug */
 
 /* Synchronises `stream`, returns the device status recorded in `ws` by the

@@ -1,0 +1,56 @@
+"""The decode entry point that allocates nothing (idx_decode_topk_noalloc).
+
+It is for callers that cannot allocate device memory (a plugin that only
+receives input and output buffers, a serving loop that must not allocate):
+its scratch is a fixed device array inside the library.  The test calls it
+through the C ABI twice in a row, on different inputs, and checks each
+result against the workspace-taking idx_decode_topk (dense mode): the same
+indices, and scores within the tolerance of the other parity tests.  It
+also checks that a call too large for the fixed scratch is refused.  This
+file is collected last so that a failure here leaves every other test run.
+"""
+import numpy as np
+import pytest
+
+from sparse_attention_indexer_05_b200 import workloads as W
+from tests._util import to_dev
+
+pytestmark = pytest.mark.gpu
+torch = pytest.importorskip("torch")
+
+
+def _close(a, b, rtol=1e-3):
+    fa, fb = np.isfinite(a), np.isfinite(b)
+    assert np.array_equal(fa, fb)
+    assert np.array_equal(a[~fa], b[~fb])              # -inf pads
+    m = np.abs(b[fb]).max() if fb.any() else 0.0
+    assert (np.abs(a[fa] - b[fb]) <= rtol * np.maximum(np.abs(b[fb]), 1e-3 * m)).all()
+
+
+def test_noalloc_decode_matches_workspace_entry_point_twice():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    import sparse_attention_indexer_05_b200 as idx
+    from sparse_attention_indexer_05_b200 import _native as N
+    f = N.lib().idx_decode_topk_noalloc
+    topk = 128
+    for seed, kv in ((1, [2500, 1999, 130]), (2, [2500, 2, 2400])):
+        D = W.decode(B=3, n=2500, G=2, H=64, d=128, topk=topk, seed=seed, kv_len=kv)
+        q, kc, w, kvl = to_dev(D.q), to_dev(D.kcache), to_dev(D.w), to_dev(D.kv_len)
+        ref_idx, ref_sc = idx.decode_topk(q, kc, kvl, w, topk, 0, "dense", return_scores=True)
+        out_idx = torch.full((3, 2, topk), 7, dtype=torch.int32, device="cuda")
+        out_sc = torch.zeros((3, 2, topk), dtype=torch.float32, device="cuda")
+        rc = f(q.data_ptr(), kc.data_ptr(), kvl.data_ptr(), w.data_ptr(), 3, 2, 2500, 64, 128, topk, N.BF16,
+               out_idx.data_ptr(), out_sc.data_ptr(), torch.cuda.current_stream().cuda_stream)
+        assert rc == 0, N.STATUS.get(rc, rc)
+        torch.cuda.synchronize()
+        assert torch.equal(out_idx, ref_idx)
+        _close(out_sc.cpu().numpy(), ref_sc.cpu().numpy())
+
+
+def test_noalloc_refuses_calls_beyond_its_scratch():
+    from sparse_attention_indexer_05_b200 import _native as N
+    f = N.lib().idx_decode_topk_noalloc
+    fake = 256  # never dereferenced: the size check fails before any launch
+    rc = f(fake, fake, fake, fake, 64, 2, 131072, 64, 128, 2048, N.BF16, fake, None, None)
+    assert rc == 2  # IDX_ERR_UNSUPPORTED
