@@ -51,7 +51,7 @@ struct PrefillWs {
     PlanLayout pl;
     long long R;          // scored rows (queries or proxies, upper bound)
     unsigned cap, ksel;
-    size_t status, plan, slot, qbar, wbar, cnt, buf, cand, msc, total;
+    size_t status, plan, slot, qbar, wbar, cnt, floor, buf, cand, msc, total;
 };
 
 PrefillWs prefill_ws(int T, int H, int d, int topk, int S, idx_dtype dt, int g, int c, idx_mode mode) {
@@ -71,6 +71,7 @@ PrefillWs prefill_ws(int T, int H, int d, int topk, int S, idx_dtype dt, int g, 
     L.qbar = pivot ? cv.take((size_t)L.R * H * d * esize(dt)) : 0;
     L.wbar = pivot ? cv.take((size_t)L.R * H * 4) : 0;
     L.cnt = cv.take((size_t)L.R * 4);
+    L.floor = cv.take((size_t)L.R * 4);
     L.buf = cv.take((size_t)L.R * L.cap * 8);
     L.cand = mode == IDX_MODE_REFINE ? cv.take((size_t)L.R * c * 4) : 0;
     L.msc = mode == IDX_MODE_REFINE ? cv.take((size_t)T * c * 4) : 0;
@@ -168,6 +169,7 @@ struct Prefill {
         a.cap = L.cap;
         a.ksel = L.ksel;
         a.cnt = reinterpret_cast<unsigned *>(ws + L.cnt);
+        a.floor_out = reinterpret_cast<unsigned *>(ws + L.floor);
         a.status = status();
         return a;
     }
@@ -205,6 +207,7 @@ struct Prefill {
         s.buf = reinterpret_cast<const unsigned long long *>(ws + L.buf);
         s.cap = L.cap;
         s.cnt = reinterpret_cast<const unsigned *>(ws + L.cnt);
+        s.floor = reinterpret_cast<const unsigned *>(ws + L.floor);
         s.c = c;
         s.cand = reinterpret_cast<const int *>(ws + L.cand);
         s.scores = reinterpret_cast<const float *>(ws + L.msc);

@@ -85,6 +85,7 @@ struct RowSel {
     unsigned thr;
     int base;           // histogram window base, in units of ord >> kBinShift
     unsigned last_cnt;  // cnt at the last histogram threshold update
+    unsigned floor;     // an ord that >= ksel offered keys reach: keys below it are out
 };
 
 __device__ __forceinline__ int sel_bin(unsigned ord, int base) {
@@ -181,6 +182,7 @@ __device__ __forceinline__ void sel_update_threshold(RowSel &st, const unsigned 
         if (b >= 0) {
             const unsigned e = sel_bin_edge(b, st.base);
             if (e > st.thr) st.thr = e;
+            if (e > st.floor) st.floor = e;
         }
     }
     __syncwarp();
@@ -251,6 +253,7 @@ __device__ __forceinline__ void sel_compact(RowSel &st, unsigned long long *buf_
         st.cnt = wpos;
         const unsigned t = minord + 1u;
         if (t > st.thr) st.thr = t;
+        if (minord > st.floor) st.floor = minord;
     }
     __syncwarp();
 }
@@ -294,6 +297,7 @@ __device__ __forceinline__ void sel_init(RowSel &st, unsigned *hist) {
         st.thr = 0u;
         st.base = kBaseUnset;
         st.last_cnt = 0u;
+        st.floor = 0u;
     }
     __syncwarp();
 }

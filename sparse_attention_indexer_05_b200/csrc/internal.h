@@ -47,6 +47,7 @@ struct ScoreArgs {
     unsigned long long *buf;
     unsigned cap, ksel;
     unsigned *cnt;
+    unsigned *floor_out;  // per row: keys with a lower ord cannot be selected
     // SINK_SPILL: out[slot * ld + s] for rows with slot_of_row[row] >= 0
     float *spill;
     long long ld;
@@ -114,6 +115,8 @@ struct SelectArgs {
     const unsigned long long *buf;
     unsigned cap;
     const unsigned *cnt;
+    const unsigned *floor;   // per candidate row (NULL: no floor)
+    int stage_cap;           // set by launch_select
     // score-row sources
     const float *scores;     // spill or member scores
     long long ld;

@@ -254,7 +254,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                     tc::named_bar_sync(1, kEpiWarps * 32);
                 }
             }
-            if (a.sink == SINK_FILTER && e < bi.nrows && lane == 0) a.cnt[bi.row0 + e] = sh.sel[e].cnt;
+            if (a.sink == SINK_FILTER && e < bi.nrows && lane == 0) {
+                a.cnt[bi.row0 + e] = sh.sel[e].cnt;
+                if (a.floor_out) a.floor_out[bi.row0 + e] = sh.sel[e].floor;
+            }
         }
         kt += ntiles;
         ++nb;

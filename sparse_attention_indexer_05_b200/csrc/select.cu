@@ -2,11 +2,22 @@
 //
 // The entries of a row (candidate keys from a score pass, or dense fp32
 // scores) are ranked by key = (ord(score) << 32) | (0xFFFFFFFF - s), so the
-// top-k is "highest score first, ties to the lower position".  An MSB-first
-// radix select with 8-bit digits finds the k-th largest key K; the selected
-// positions (key >= K) are marked in a shared bitmap over 0..bound, and
-// each selected entry writes itself at its rank among the marked bits,
-// which lists the top-k in ascending position without a sort.
+// top-k is "highest score first, ties to the lower position".
+//
+// 1. One pass over the row in global memory counts the valid entries and
+//    builds a histogram of the key's top 12 bits (1/16-octave score bins);
+//    the bin D holding the k-th largest key follows.
+// 2. A second global pass copies every entry whose top bits are >= D into
+//    shared memory: the k-th key and everything above it, a few thousand
+//    entries at most for the workloads here.
+// 3. An MSB-first radix select (12/12/8-bit digits over the score part, the
+//    position part only for ties) over the staged keys finds the exact k-th
+//    largest key K.
+// 4. The selected positions (key >= K) are marked in a shared bitmap over
+//    0..bound; each selected entry writes itself at its rank among the
+//    marked bits, which lists the top-k in ascending position without a sort.
+// When the staged set would not fit, steps 3-4 read the row from global
+// memory instead (same arithmetic).
 #include <math.h>
 
 #include "common.cuh"
@@ -17,20 +28,25 @@ namespace idx {
 namespace {
 
 constexpr int kSelThreads = 512;
+constexpr int kMaxBins = 4096;  // widest radix digit: 12 bits
 
+// candidate keys of a score pass; entries below the row's floor (a score
+// that at least ksel appended keys reach) can no longer be selected
 struct CandSrc {
     const unsigned long long *buf;
     int n;
     int bound;
+    unsigned floor_ord;
     __device__ unsigned long long key(int i) const {
         const unsigned long long kk = buf[i];
-        return key_pos(kk) <= bound ? kk : 0ull;
+        return (key_pos(kk) <= bound && key_ord(kk) >= floor_ord) ? kk : 0ull;
     }
 };
 
+// dense fp32 scores with their positions (NULL: position = index)
 struct ScoreSrc {
     const float *sc;
-    const int *pos;  // NULL: position = i
+    const int *pos;
     int n;
     int bound;
     __device__ unsigned long long key(int i) const {
@@ -38,6 +54,24 @@ struct ScoreSrc {
         if (p < 0 || p > bound) return 0ull;
         return make_key(score_ord(sc[i]), p);
     }
+};
+
+// keys staged in shared memory (all valid)
+struct StageSrc {
+    const unsigned long long *st;
+    int n;
+    int bound;
+    __device__ unsigned long long key(int i) const { return st[i]; }
+};
+
+struct SelShared {
+    unsigned hist[kMaxBins];
+    unsigned red[32];
+    unsigned red2[32];
+    int dgt;
+    unsigned above;
+    unsigned inbin;
+    unsigned nstage;
 };
 
 __device__ unsigned block_sum(unsigned v, unsigned *red) {
@@ -53,28 +87,16 @@ __device__ unsigned block_sum(unsigned v, unsigned *red) {
     return t;
 }
 
-constexpr int kMaxBins = 4096;  // widest radix digit: 12 bits
-
-struct SelShared {
-    unsigned hist[kMaxBins];
-    unsigned red[32];
-    unsigned red2[32];
-    int dgt;
-    unsigned above;
-    unsigned inbin;
-};
-
 // Digits of the 64-bit key, most significant first: 12 + 12 + 8 bits of the
-// score's ord (the first digit separates exponents, so the k-th key's bin is
-// already narrow), then 12 + 12 + 8 bits of the position part (ties only).
+// score's ord, then 12 + 12 + 8 bits of the position part (ties only).
 __device__ __forceinline__ int digit_bits(int pass) { return (pass % 3 == 2) ? 8 : 12; }
 
 // Block-wide: the largest bin b of hist[0..nbins) with sum(hist[b..]) >= need;
-// writes b, sum(hist[b+1..]) and hist[b] to sh.  nbins is a multiple of 8
-// and at most 8 * blockDim.x.
+// writes b, sum(hist[b+1..]) and hist[b] to sh (sh.dgt stays -1 if none).
+// nbins is a multiple of 8 and at most 8 * blockDim.x.
 __device__ void block_find_bin(SelShared &sh, int nbins, unsigned need) {
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nw = blockDim.x >> 5;
-    const int per = 8;
+    constexpr int per = 8;
     const bool own = tid * per < nbins;
     unsigned loc[per];
     unsigned sum = 0;
@@ -83,16 +105,15 @@ __device__ void block_find_bin(SelShared &sh, int nbins, unsigned need) {
         loc[i] = own ? sh.hist[tid * per + i] : 0u;
         sum += loc[i];
     }
-    // inclusive suffix sum over threads: suf(t) = sum of threads >= t
-    unsigned suf = sum;
+    unsigned suf = sum;  // inclusive suffix sum over the warp's threads
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
         const unsigned v = __shfl_down_sync(0xFFFFFFFFu, suf, o);
         if (lane + o < 32) suf += v;
     }
-    if (lane == 0) sh.red2[warp] = suf;  // warp total
+    if (lane == 0) sh.red2[warp] = suf;
     __syncthreads();
-    unsigned after = 0;  // totals of the warps above this one
+    unsigned after = 0;
     for (int w2 = warp + 1; w2 < nw; ++w2) after += sh.red2[w2];
     suf += after;
     if (suf >= need && suf - sum < need) {
@@ -110,101 +131,126 @@ __device__ void block_find_bin(SelShared &sh, int nbins, unsigned need) {
     __syncthreads();
 }
 
+// Histogram of digit (key >> shift) & dmask over entries matching `prefix`
+// under `mask`; warp-aggregated increments (equal digits add once per warp).
+// Returns the number of valid entries seen by this thread.
+// Entries are read kUnroll at a time per thread, all loads issued before any
+// is used, so that a warp keeps several memory requests in flight.
+constexpr int kUnroll = 8;
+
 template <class Src>
-__device__ void block_select(const Src &src, int k, int *out_idx, float *out_score, SelShared &sh,
-                             unsigned *bm, unsigned *gpre, int wcap, unsigned *status) {
+__device__ unsigned hist_pass(const Src &src, SelShared &sh, int shift, unsigned dmask, unsigned long long prefix,
+                              unsigned long long mask) {
     const int tid = threadIdx.x, nt = blockDim.x, lane = tid & 31;
-    unsigned long long K = 1ull;
-    unsigned nv = 0;
-    {
-        unsigned long long prefix = 0ull, mask = 0ull;
-        unsigned need = (unsigned)k;
-        int shift = 64;
-        for (int pass = 0; pass < 6; ++pass) {
-            const int bits = digit_bits(pass);
-            shift -= bits;
-            const unsigned dmask = (1u << bits) - 1u;
-            for (int i = tid; i < (1 << bits); i += nt) sh.hist[i] = 0u;
-            if (tid == 0) sh.dgt = -1;
-            __syncthreads();
-            unsigned nvl = 0;
-            for (int base = 0; base < src.n; base += nt) {
-                const int i = base + tid;
-                unsigned long long key = i < src.n ? src.key(i) : 0ull;
-                const bool act = key != 0ull && (key & mask) == prefix;
-                nvl += key != 0ull;
-                const unsigned dg = act ? (unsigned)(key >> shift) & dmask : 0xFFFFFFFFu;
-                const unsigned m = __match_any_sync(0xFFFFFFFFu, dg);
-                if (act && lane == __ffs(m) - 1) atomicAdd(&sh.hist[dg], (unsigned)__popc(m));
-            }
-            if (pass == 0) {
-                nv = block_sum(nvl, sh.red);  // also orders the histogram updates
-                if (nv <= (unsigned)k) break;  // every valid entry is selected
-            } else {
-                __syncthreads();
-            }
-            block_find_bin(sh, 1 << bits, need);
-            const int d = sh.dgt;
-            const unsigned above = sh.above, inbin = sh.inbin;
-            __syncthreads();
-            if (d < 0) break;  // unreachable when nv > k
-            need -= above;
-            prefix |= (unsigned long long)d << shift;
-            mask |= (unsigned long long)dmask << shift;
-            K = prefix;
-            if (inbin == need) break;  // the whole bin is selected
+    unsigned nvl = 0;
+    for (int base = 0; base < src.n; base += nt * kUnroll) {
+        unsigned long long key[kUnroll];
+#pragma unroll
+        for (int u = 0; u < kUnroll; ++u) {
+            const int i = base + u * nt + tid;
+            key[u] = i < src.n ? src.key(i) : 0ull;
         }
-        if (nv <= (unsigned)k) K = 1ull;
+#pragma unroll
+        for (int u = 0; u < kUnroll; ++u) {
+            nvl += key[u] != 0ull;
+            const bool act = key[u] != 0ull && (key[u] & mask) == prefix;
+            const unsigned dg = act ? (unsigned)(key[u] >> shift) & dmask : 0xFFFFFFFFu;
+            const unsigned m = __match_any_sync(0xFFFFFFFFu, dg);
+            if (act && lane == __ffs(m) - 1) atomicAdd(&sh.hist[dg], (unsigned)__popc(m));
+        }
     }
-    const int nsel = (int)(nv < (unsigned)k ? nv : (unsigned)k);
+    return nvl;
+}
+
+// Exact k-th largest valid key of src, refining a known prefix from digit
+// pass `pass0` on; `need` = how many keys matching the prefix to select.
+template <class Src>
+__device__ unsigned long long radix_kth(const Src &src, SelShared &sh, unsigned need, int pass0,
+                                        unsigned long long prefix, unsigned long long mask) {
+    const int tid = threadIdx.x, nt = blockDim.x;
+    int shift = 64;
+    for (int p = 0; p < pass0; ++p) shift -= digit_bits(p);
+    unsigned long long K = prefix;
+    for (int pass = pass0; pass < 6; ++pass) {
+        const int bits = digit_bits(pass);
+        shift -= bits;
+        const unsigned dmask = (1u << bits) - 1u;
+        for (int i = tid; i < (1 << bits); i += nt) sh.hist[i] = 0u;
+        if (tid == 0) sh.dgt = -1;
+        __syncthreads();
+        hist_pass(src, sh, shift, dmask, prefix, mask);
+        __syncthreads();
+        block_find_bin(sh, 1 << bits, need);
+        const int d = sh.dgt;
+        const unsigned above = sh.above, inbin = sh.inbin;
+        __syncthreads();
+        if (d < 0) break;  // unreachable when more than `need` keys match
+        need -= above;
+        prefix |= (unsigned long long)d << shift;
+        mask |= (unsigned long long)dmask << shift;
+        K = prefix;
+        if (inbin == need) break;  // the whole bin is selected
+    }
+    return K;
+}
+
+// write the nsel keys >= K of src in ascending position, then pad to k
+template <class Src>
+__device__ void emit(const Src &src, unsigned long long K, int nsel, int k, int *out_idx, float *out_score,
+                     unsigned *bm, unsigned *gpre, int wcap, unsigned *status) {
+    const int tid = threadIdx.x, nt = blockDim.x;
     if (nsel > 0) {
         const int W = src.bound / 32 + 1;
         if (W > wcap) {
             raise_status(status, ST_INVALID);
-            for (int r = tid; r < k; r += nt) {
-                out_idx[r] = -1;
-                if (out_score) out_score[r] = -INFINITY;
+            nsel = 0;
+        } else {
+            for (int i = tid; i < W; i += nt) bm[i] = 0u;
+            __syncthreads();
+            for (int i = tid; i < src.n; i += nt) {
+                const unsigned long long key = src.key(i);
+                if (key != 0ull && key >= K) {
+                    const int p = key_pos(key);
+                    atomicOr(&bm[p >> 5], 1u << (p & 31));
+                }
             }
-            return;
-        }
-        for (int i = tid; i < W; i += nt) bm[i] = 0u;
-        __syncthreads();
-        for (int i = tid; i < src.n; i += nt) {
-            const unsigned long long key = src.key(i);
-            if (key != 0ull && key >= K) {
-                const int p = key_pos(key);
-                atomicOr(&bm[p >> 5], 1u << (p & 31));
+            __syncthreads();
+            // per group of 32 words: exclusive prefix of the set bits
+            const int NG = (W + 31) / 32;
+            for (int gi = tid; gi < NG; gi += nt) {
+                unsigned s = 0;
+                const int e = (gi + 1) * 32 < W ? (gi + 1) * 32 : W;
+                for (int w = gi * 32; w < e; ++w) s += __popc(bm[w]);
+                gpre[gi] = s;
             }
-        }
-        __syncthreads();
-        // per group of 32 words: exclusive prefix of the set bits
-        const int NG = (W + 31) / 32;
-        for (int gi = tid; gi < NG; gi += nt) {
-            unsigned s = 0;
-            const int e = (gi + 1) * 32 < W ? (gi + 1) * 32 : W;
-            for (int w = gi * 32; w < e; ++w) s += __popc(bm[w]);
-            gpre[gi] = s;
-        }
-        __syncthreads();
-        if (tid == 0) {
-            unsigned run = 0;
-            for (int gi = 0; gi < NG; ++gi) {
-                const unsigned s = gpre[gi];
-                gpre[gi] = run;
-                run += s;
+            __syncthreads();
+            if (tid < 32) {  // warp-level exclusive scan over the groups
+                unsigned carry = 0;
+                for (int g0 = 0; g0 < NG; g0 += 32) {
+                    const int gi = g0 + tid;
+                    const unsigned s = gi < NG ? gpre[gi] : 0u;
+                    unsigned inc = s;
+#pragma unroll
+                    for (int o = 1; o < 32; o <<= 1) {
+                        const unsigned v = __shfl_up_sync(0xFFFFFFFFu, inc, o);
+                        if (tid >= o) inc += v;
+                    }
+                    if (gi < NG) gpre[gi] = carry + inc - s;
+                    carry += __shfl_sync(0xFFFFFFFFu, inc, 31);
+                }
             }
-        }
-        __syncthreads();
-        for (int i = tid; i < src.n; i += nt) {
-            const unsigned long long key = src.key(i);
-            if (key != 0ull && key >= K) {
-                const int p = key_pos(key);
-                const int w = p >> 5;
-                unsigned r = gpre[w >> 5];
-                for (int w2 = w & ~31; w2 < w; ++w2) r += __popc(bm[w2]);
-                r += __popc(bm[w] & ((1u << (p & 31)) - 1u));
-                out_idx[r] = p;
-                if (out_score) out_score[r] = ord_score(key_ord(key));
+            __syncthreads();
+            for (int i = tid; i < src.n; i += nt) {
+                const unsigned long long key = src.key(i);
+                if (key != 0ull && key >= K) {
+                    const int p = key_pos(key);
+                    const int w = p >> 5;
+                    unsigned r = gpre[w >> 5];
+                    for (int w2 = w & ~31; w2 < w; ++w2) r += __popc(bm[w2]);
+                    r += __popc(bm[w] & ((1u << (p & 31)) - 1u));
+                    out_idx[r] = p;
+                    if (out_score) out_score[r] = ord_score(key_ord(key));
+                }
             }
         }
     }
@@ -214,13 +260,72 @@ __device__ void block_select(const Src &src, int k, int *out_idx, float *out_sco
     }
 }
 
+template <class Src>
+__device__ void block_select(const Src &src, int k, int *out_idx, float *out_score, SelShared &sh,
+                             unsigned long long *stage, int stage_cap, unsigned *bm, unsigned *gpre, int wcap,
+                             unsigned *status) {
+    const int tid = threadIdx.x, nt = blockDim.x, lane = tid & 31;
+    // pass 1: valid count and the top-12-bit histogram
+    for (int i = tid; i < kMaxBins; i += nt) sh.hist[i] = 0u;
+    if (tid == 0) {
+        sh.dgt = -1;
+        sh.nstage = 0;
+    }
+    __syncthreads();
+    const unsigned nv = block_sum(hist_pass(src, sh, 52, 0xFFFu, 0ull, 0ull), sh.red);
+    if (nv <= (unsigned)k) {  // every valid entry is selected
+        emit(src, 1ull, (int)nv, k, out_idx, out_score, bm, gpre, wcap, status);
+        return;
+    }
+    block_find_bin(sh, kMaxBins, (unsigned)k);
+    const int d0 = sh.dgt;
+    const unsigned above0 = sh.above, inbin0 = sh.inbin;
+    __syncthreads();
+    const unsigned long long pre0 = (unsigned long long)d0 << 52, mask0 = 0xFFFull << 52;
+    const unsigned need = (unsigned)k - above0;
+    if (inbin0 == need) {  // the k-th key closes its bin: select everything >= the bin
+        emit(src, pre0, k, k, out_idx, out_score, bm, gpre, wcap, status);
+        return;
+    }
+    if (above0 + inbin0 <= (unsigned)stage_cap) {
+        // pass 2: stage the keys of bin d0 and above
+        for (int base = 0; base < src.n; base += nt * kUnroll) {
+            unsigned long long key[kUnroll];
+#pragma unroll
+            for (int u = 0; u < kUnroll; ++u) {
+                const int i = base + u * nt + tid;
+                key[u] = i < src.n ? src.key(i) : 0ull;
+            }
+#pragma unroll
+            for (int u = 0; u < kUnroll; ++u) {
+                const bool keep = key[u] != 0ull && key[u] >= pre0;
+                const unsigned m = __ballot_sync(0xFFFFFFFFu, keep);
+                if (m) {
+                    unsigned b = 0;
+                    if (lane == __ffs(m) - 1) b = atomicAdd(&sh.nstage, (unsigned)__popc(m));
+                    b = __shfl_sync(0xFFFFFFFFu, b, __ffs(m) - 1);
+                    if (keep) stage[b + __popc(m & lanemask_lt())] = key[u];
+                }
+            }
+        }
+        __syncthreads();
+        const StageSrc ss{stage, (int)sh.nstage, src.bound};
+        const unsigned long long K = radix_kth(ss, sh, need, 1, pre0, mask0);
+        emit(ss, K, k, k, out_idx, out_score, bm, gpre, wcap, status);
+        return;
+    }
+    const unsigned long long K = radix_kth(src, sh, need, 1, pre0, mask0);
+    emit(src, K, k, k, out_idx, out_score, bm, gpre, wcap, status);
+}
+
 __global__ void __launch_bounds__(kSelThreads) select_kernel(SelectArgs a) {
-    extern __shared__ unsigned sel_smem[];
+    extern __shared__ __align__(16) unsigned long long sel_smem[];
     __shared__ SelShared sh;
     const int row = blockIdx.x;
     const int wcap = a.bitmap_words;
-    unsigned *bm = sel_smem;
-    unsigned *gpre = sel_smem + wcap;
+    unsigned long long *stage = sel_smem;
+    unsigned *bm = reinterpret_cast<unsigned *>(sel_smem + a.stage_cap);
+    unsigned *gpre = bm + wcap;
     int *oi = a.out_idx + (long long)row * a.k;
     float *os = a.out_score ? a.out_score + (long long)row * a.k : nullptr;
     auto pad_all = [&]() {
@@ -228,6 +333,10 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(SelectArgs a) {
             oi[r] = -1;
             if (os) os[r] = -INFINITY;
         }
+    };
+    auto cand = [&](long long r, int bound) {
+        const unsigned n = a.cnt[r];
+        return CandSrc{a.buf + r * a.cap, (int)(n < a.cap ? n : a.cap), bound, a.floor ? a.floor[r] : 0u};
     };
     switch (a.kind) {
     case SEL_DENSE_CAND:
@@ -237,18 +346,14 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(SelectArgs a) {
         const int b = find_seg(a.cu, a.S, row);
         const int t = row - a.cu[b];
         if (a.kind == SEL_DENSE_CAND) {
-            unsigned n = a.cnt[row];
-            CandSrc src{a.buf + (long long)row * a.cap, (int)(n < a.cap ? n : a.cap), t};
-            block_select(src, a.k, oi, os, sh, bm, gpre, wcap, a.status);
+            block_select(cand(row, t), a.k, oi, os, sh, stage, a.stage_cap, bm, gpre, wcap, a.status);
         } else {
             const int p = a.plan[a.pl.rp() + b] + t / a.g;
             if (a.kind == SEL_REUSE_CAND) {
-                unsigned n = a.cnt[p];
-                CandSrc src{a.buf + (long long)p * a.cap, (int)(n < a.cap ? n : a.cap), t};
-                block_select(src, a.k, oi, os, sh, bm, gpre, wcap, a.status);
+                block_select(cand(p, t), a.k, oi, os, sh, stage, a.stage_cap, bm, gpre, wcap, a.status);
             } else {
                 ScoreSrc src{a.scores + (long long)row * a.ld, a.cand + (long long)p * a.c, a.c, t};
-                block_select(src, a.k, oi, os, sh, bm, gpre, wcap, a.status);
+                block_select(src, a.k, oi, os, sh, stage, a.stage_cap, bm, gpre, wcap, a.status);
             }
         }
         return;
@@ -260,10 +365,8 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(SelectArgs a) {
         const int b = find_seg(rp, a.S, row);
         const int i = row - rp[b];
         const int n = a.cu[b + 1] - a.cu[b];
-        const int bound = row_bound(i, n, a.g);
-        unsigned cn = a.cnt[row];
-        CandSrc src{a.buf + (long long)row * a.cap, (int)(cn < a.cap ? cn : a.cap), bound};
-        block_select(src, a.k, oi, nullptr, sh, bm, gpre, wcap, a.status);
+        block_select(cand(row, row_bound(i, n, a.g)), a.k, oi, nullptr, sh, stage, a.stage_cap, bm, gpre, wcap,
+                     a.status);
         return;
     }
     default: {  // decode kinds
@@ -279,18 +382,18 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(SelectArgs a) {
         if (a.kind == SEL_DEC_DENSE) {
             const int bound = kv - a.G + m;
             ScoreSrc src{a.scores + (long long)row * a.ld, nullptr, bound + 1, bound};
-            block_select(src, a.k, oi, os, sh, bm, gpre, wcap, a.status);
+            block_select(src, a.k, oi, os, sh, stage, a.stage_cap, bm, gpre, wcap, a.status);
         } else if (a.kind == SEL_DEC_REUSE) {
             const int bound = kv - a.G + m;
             ScoreSrc src{a.scores + (long long)b * a.ld, nullptr, bound + 1, bound};
-            block_select(src, a.k, oi, os, sh, bm, gpre, wcap, a.status);
+            block_select(src, a.k, oi, os, sh, stage, a.stage_cap, bm, gpre, wcap, a.status);
         } else if (a.kind == SEL_DEC_PROXY_TO_C) {
             ScoreSrc src{a.scores + (long long)b * a.ld, nullptr, kv, kv - 1};
-            block_select(src, a.k, oi, nullptr, sh, bm, gpre, wcap, a.status);
+            block_select(src, a.k, oi, nullptr, sh, stage, a.stage_cap, bm, gpre, wcap, a.status);
         } else {  // SEL_DEC_MEMBER
             const int bound = kv - a.G + m;
             ScoreSrc src{a.scores + (long long)row * a.ld, a.cand + (long long)b * a.c, a.c, bound};
-            block_select(src, a.k, oi, os, sh, bm, gpre, wcap, a.status);
+            block_select(src, a.k, oi, os, sh, stage, a.stage_cap, bm, gpre, wcap, a.status);
         }
         return;
     }
@@ -301,12 +404,19 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(SelectArgs a) {
 
 cudaError_t launch_select(const SelectArgs &a, cudaStream_t st) {
     if (a.nrows <= 0) return cudaSuccess;
-    const size_t smem = ((size_t)a.bitmap_words + (size_t)(a.bitmap_words + 31) / 32 + 1) * 4;
-    cudaError_t e = cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)smem);
+    SelectArgs b = a;
+    const size_t tail = ((size_t)a.bitmap_words + (size_t)(a.bitmap_words + 31) / 32 + 1) * 4;
+    const size_t limit = 232448 - sizeof(SelShared) - 1024;
+    // staging room: the k-th key's 1/16-octave bin and everything above it
+    long long cap = 2LL * a.k + 2048;
+    if ((size_t)cap * 8 + tail > limit) cap = ((long long)limit - (long long)tail) / 8;
+    if (cap < 0) cap = 0;
+    b.stage_cap = (int)cap;
+    const size_t smem = (size_t)cap * 8 + tail;
+    cudaError_t e = cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     TraceScope ts("select", st);
-    select_kernel<<<a.nrows, kSelThreads, smem, st>>>(a);
+    select_kernel<<<a.nrows, kSelThreads, smem, st>>>(b);
     return cudaGetLastError();
 }
 

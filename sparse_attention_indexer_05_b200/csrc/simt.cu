@@ -140,7 +140,10 @@ __global__ void __launch_bounds__(kSimtThreads) score_simt_kernel(ScoreArgs a) {
             if (a.sink == SINK_FILTER && row_ok)
                 sel_maintain(sel[r], hist + r * kBins, a.buf + grow * a.cap, a.cap, a.ksel, scr + warp * 256, KT);
         }
-        if (a.sink == SINK_FILTER && row_ok && (threadIdx.x & 31) == 0) a.cnt[grow] = sel[r].cnt;
+        if (a.sink == SINK_FILTER && row_ok && (threadIdx.x & 31) == 0) {
+            a.cnt[grow] = sel[r].cnt;
+            if (a.floor_out) a.floor_out[grow] = sel[r].floor;
+        }
     }
 }
 

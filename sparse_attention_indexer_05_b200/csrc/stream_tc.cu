@@ -21,8 +21,8 @@ namespace {
 
 constexpr int S_H = 64;
 constexpr int S_D = 128;
-constexpr int kThreads = 320;
-constexpr int kEpiWarps = 8;
+constexpr int kEpiWarps = 16;                    // 4 per TMEM lane quarter, one scored row each
+constexpr int kThreads = 64 + 32 * kEpiWarps;    // + producer warp + MMA warp
 constexpr int kStages = 4;
 constexpr uint32_t kQSlice = 256 * 128;          // 256 rows x 64 bf16 (32 KB)
 constexpr uint32_t kQBytes = 2 * kQSlice;        // 2 K slices
@@ -50,7 +50,7 @@ struct Item {
     int t0, nt;         // key tiles [t0, t0 + nt) of the item
     // outputs
     long long out_row0; // output row of scored row 0
-    int bound[4];       // decode: causal bound per row (inclusive)
+    int bound0, bstep;  // decode: causal bound of row r = bound0 + bstep * r (inclusive)
     const int *cand;    // gather: candidate positions of the group
 };
 
@@ -106,19 +106,51 @@ __device__ __forceinline__ Item item_info(const GatherArgs &g, const DecodeArgs 
         it.key0 = (long long)b * dd.n_max;
         it.t0 = t0;
         it.nt = (t0 + kDecodeChunkTiles < ntiles ? t0 + kDecodeChunkTiles : ntiles) - t0;
-        for (int r = 0; r < 4; ++r) it.bound[r] = dd.Gq == 1 ? kv - 1 : kv - dd.G + r;
+        it.bound0 = dd.Gq == 1 ? kv - 1 : kv - dd.G;
+        it.bstep = dd.Gq == 1 ? 0 : 1;
     }
     return it;
 }
 
-__device__ __forceinline__ float reduce64(const uint32_t (&v0)[32], const uint32_t (&v1)[32], const float *w) {
+// sum_j w[j] * max(v[j], 0) over 32 heads; w 16-byte aligned, read as float4
+__device__ __forceinline__ float reduce32(const uint32_t (&v)[32], const float *w) {
+    const float4 *w4 = reinterpret_cast<const float4 *>(w);
     float a[8];
 #pragma unroll
     for (int i = 0; i < 8; ++i) a[i] = 0.0f;
 #pragma unroll
-    for (int j = 0; j < 32; ++j) a[j & 7] = fmaf(w[j], fmaxf(__uint_as_float(v0[j]), 0.0f), a[j & 7]);
+    for (int j4 = 0; j4 < 8; ++j4) {
+        const float4 wv = w4[j4];
+        a[(4 * j4 + 0) & 7] = fmaf(wv.x, fmaxf(__uint_as_float(v[4 * j4 + 0]), 0.0f), a[(4 * j4 + 0) & 7]);
+        a[(4 * j4 + 1) & 7] = fmaf(wv.y, fmaxf(__uint_as_float(v[4 * j4 + 1]), 0.0f), a[(4 * j4 + 1) & 7]);
+        a[(4 * j4 + 2) & 7] = fmaf(wv.z, fmaxf(__uint_as_float(v[4 * j4 + 2]), 0.0f), a[(4 * j4 + 2) & 7]);
+        a[(4 * j4 + 3) & 7] = fmaf(wv.w, fmaxf(__uint_as_float(v[4 * j4 + 3]), 0.0f), a[(4 * j4 + 3) & 7]);
+    }
+    return ((a[0] + a[1]) + (a[2] + a[3])) + ((a[4] + a[5]) + (a[6] + a[7]));
+}
+
+// sum_j w[j] * max(v[j], 0) over 64 heads; w 16-byte aligned, read as float4
+__device__ __forceinline__ float reduce64(const uint32_t (&v0)[32], const uint32_t (&v1)[32], const float *w) {
+    const float4 *w4 = reinterpret_cast<const float4 *>(w);
+    float a[8];
 #pragma unroll
-    for (int j = 0; j < 32; ++j) a[j & 7] = fmaf(w[32 + j], fmaxf(__uint_as_float(v1[j]), 0.0f), a[j & 7]);
+    for (int i = 0; i < 8; ++i) a[i] = 0.0f;
+#pragma unroll
+    for (int j4 = 0; j4 < 8; ++j4) {
+        const float4 wv = w4[j4];
+        a[(4 * j4 + 0) & 7] = fmaf(wv.x, fmaxf(__uint_as_float(v0[4 * j4 + 0]), 0.0f), a[(4 * j4 + 0) & 7]);
+        a[(4 * j4 + 1) & 7] = fmaf(wv.y, fmaxf(__uint_as_float(v0[4 * j4 + 1]), 0.0f), a[(4 * j4 + 1) & 7]);
+        a[(4 * j4 + 2) & 7] = fmaf(wv.z, fmaxf(__uint_as_float(v0[4 * j4 + 2]), 0.0f), a[(4 * j4 + 2) & 7]);
+        a[(4 * j4 + 3) & 7] = fmaf(wv.w, fmaxf(__uint_as_float(v0[4 * j4 + 3]), 0.0f), a[(4 * j4 + 3) & 7]);
+    }
+#pragma unroll
+    for (int j4 = 0; j4 < 8; ++j4) {
+        const float4 wv = w4[8 + j4];
+        a[(4 * j4 + 0) & 7] = fmaf(wv.x, fmaxf(__uint_as_float(v1[4 * j4 + 0]), 0.0f), a[(4 * j4 + 0) & 7]);
+        a[(4 * j4 + 1) & 7] = fmaf(wv.y, fmaxf(__uint_as_float(v1[4 * j4 + 1]), 0.0f), a[(4 * j4 + 1) & 7]);
+        a[(4 * j4 + 2) & 7] = fmaf(wv.z, fmaxf(__uint_as_float(v1[4 * j4 + 2]), 0.0f), a[(4 * j4 + 2) & 7]);
+        a[(4 * j4 + 3) & 7] = fmaf(wv.w, fmaxf(__uint_as_float(v1[4 * j4 + 3]), 0.0f), a[(4 * j4 + 3) & 7]);
+    }
     return ((a[0] + a[1]) + (a[2] + a[3])) + ((a[4] + a[5]) + (a[6] + a[7]));
 }
 
@@ -244,44 +276,39 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
         } else {
             const int quarter = warp & 3;
-            const int qp = (warp - 2) >> 2;
+            const int r = (warp - 2) >> 2;  // the scored row of this warp
+            const bool mine = r < it.m;
             bool ok = true;
             for (int j = 0; j < it.nt; ++j) {
                 const uint32_t tt = t + j, buf = tt & 1u;
                 if (ok) ok = tc::mbar_wait(&sh.tfull[buf], (tt >> 1) & 1u, abort, status);
-                float sc[2] = {0.0f, 0.0f};
                 if (ok) {
                     tc::fence_after_sync();
-                    const uint32_t taddr = tmem + ((uint32_t)(quarter * 32) << 16) + buf * 256 + qp * 128;
-                    uint32_t v0[32], v1[32], v2[32], v3[32];
-                    const bool r0 = 2 * qp < it.m, r1 = 2 * qp + 1 < it.m;
-                    if (r0) {
-                        tc::tmem_ld32(taddr, v0);
-                        tc::tmem_ld32(taddr + 32, v1);
+                    const uint32_t taddr = tmem + ((uint32_t)(quarter * 32) << 16) + buf * 256 + r * 64;
+                    // two 32-column halves, to keep the register footprint small
+                    float part[2] = {0.0f, 0.0f};
+                    if (mine) {
+#pragma unroll
+                        for (int hh = 0; hh < 2; ++hh) {
+                            uint32_t v[32];
+                            tc::tmem_ld32(taddr + hh * 32, v);
+                            tc::tmem_wait_ld_all();
+                            tc::reg_fence(v);
+                            part[hh] = reduce32(v, wsm + r * S_H + hh * 32);
+                        }
                     }
-                    if (r1) {
-                        tc::tmem_ld32(taddr + 64, v2);
-                        tc::tmem_ld32(taddr + 96, v3);
-                    }
-                    tc::tmem_wait_ld_all();
-                    if (r0) { tc::reg_fence(v0); tc::reg_fence(v1); }
-                    if (r1) { tc::reg_fence(v2); tc::reg_fence(v3); }
                     tc::fence_before_sync();
                     __syncwarp();
                     if (lane == 0) tc::mbar_arrive(&sh.tempty[buf]);
-                    if (r0) sc[0] = reduce64(v0, v1, wsm + (2 * qp) * S_H);
-                    if (r1) sc[1] = reduce64(v2, v3, wsm + (2 * qp + 1) * S_H);
-                    const int kidx = quarter * 32 + lane;
-#pragma unroll
-                    for (int rr = 0; rr < 2; ++rr) {
-                        const int r = 2 * qp + rr;
-                        if (r >= it.m) continue;
+                    if (mine) {
+                        const float sc = part[0] + part[1];
+                        const int kidx = quarter * 32 + lane;
                         if (GATHER) {
                             const int jj = j * KT + kidx;
-                            if (jj < g.c) out[(it.out_row0 + r) * ld + jj] = sc[rr];
+                            if (jj < g.c) out[(it.out_row0 + r) * ld + jj] = sc;
                         } else {
                             const int s = (it.t0 + j) * KT + kidx;
-                            if (s <= it.bound[r]) out[(it.out_row0 + r) * ld + s] = sc[rr];
+                            if (s <= it.bound0 + it.bstep * r) out[(it.out_row0 + r) * ld + s] = sc;
                         }
                     }
                 }
