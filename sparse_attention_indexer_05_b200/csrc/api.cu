@@ -310,7 +310,7 @@ idx_status idx_pivot_topk(const void *q, const void *k, const float *w, const in
     int *cand = reinterpret_cast<int *>(P.ws + P.L.cand);
     TRY_CUDA(launch_select(P.select_args(SEL_PROXY_TO_C, (int)P.L.R, c, cand, nullptr), P.st));
     const GatherArgs ga = P.gather_args();
-    TRY_CUDA(tc_gather_supported(H, d, (int)dtype, g) ? launch_gather_tc(ga, P.st)
+    TRY_CUDA(tc_gather_supported(H, d, (int)dtype, g, c) ? launch_gather_tc(ga, P.st)
                                                        : launch_gather_simt(ga, (int)dtype, P.st));
     return cuda_st(launch_select(P.select_args(SEL_MEMBER_SCORES, T, topk, out_idx, out_score), P.st));
 }
@@ -418,7 +418,7 @@ idx_status idx_decode_topk(const void *q, const void *kcache, const int *kv_len,
     int *cand = reinterpret_cast<int *>(D.ws + D.L.cand);
     TRY_CUDA(launch_select(D.sargs(SEL_DEC_PROXY_TO_C, B, c, cand, nullptr, spill, n_max), D.st));
     const GatherArgs ga = D.gargs();
-    TRY_CUDA(tc_gather_supported(H, d, (int)dtype, G) ? launch_gather_tc(ga, D.st)
+    TRY_CUDA(tc_gather_supported(H, d, (int)dtype, G, c) ? launch_gather_tc(ga, D.st)
                                                        : launch_gather_simt(ga, (int)dtype, D.st));
     const float *msc = reinterpret_cast<const float *>(D.ws + D.L.msc);
     return cuda_st(launch_select(D.sargs(SEL_DEC_MEMBER, B * G, topk, out_idx, out_score, msc, c), D.st));

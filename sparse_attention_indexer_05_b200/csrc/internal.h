@@ -162,6 +162,6 @@ cudaError_t launch_decode_proxy(const void *q, const float *w, int B, int G, int
 size_t simt_smem_bytes(int H, int d, int dtype);
 bool tc_supported(int H, int d, int dtype);
 bool tc_decode_supported(int H, int d, int dtype, int rows_per_request);
-bool tc_gather_supported(int H, int d, int dtype, int group);
+bool tc_gather_supported(int H, int d, int dtype, int group, int c);
 
 }  // namespace idx

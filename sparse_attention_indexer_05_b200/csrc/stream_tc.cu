@@ -40,7 +40,9 @@ constexpr size_t kOffQ = 0;
 constexpr size_t kOffA = kOffQ + kQBytes;
 constexpr size_t kOffW = kOffA + (size_t)kStages * kAStage;
 constexpr size_t kOffCtl = kOffW + 4 * S_H * 4;
-constexpr size_t kSmemBytes = kOffCtl + sizeof(StShared) + 1024;
+constexpr size_t kOffCand = (kOffCtl + sizeof(StShared) + 15) / 16 * 16;  // gather: key rows of C
+constexpr int kMaxCand = 8192;
+__host__ __device__ constexpr size_t smem_bytes(int cand_slots) { return kOffCand + (size_t)cand_slots * 4 + 1024; }
 
 struct Item {
     bool valid;
@@ -174,6 +176,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint8_t *as = smem + kOffA;
     float *wsm = reinterpret_cast<float *>(smem + kOffW);
     StShared &sh = *reinterpret_cast<StShared *>(smem + kOffCtl);
+    int *crow = reinterpret_cast<int *>(smem + kOffCand);
     volatile int *abort = &sh.abort;
     unsigned *status = GATHER ? g.status : dd.status;
     const float *wsrc = GATHER ? g.w : dd.w;
@@ -217,6 +220,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         __syncthreads();
         for (int i = threadIdx.x; i < 4 * S_H; i += kThreads)
             wsm[i] = (i / S_H) < it.m ? wsrc[it.qrow0 * S_H + i] : 0.0f;
+        if (GATHER) {
+            // key rows of the group's candidates (padding slots read row key0; their
+            // scores are written but the select pass ignores position -1)
+            for (int i = threadIdx.x; i < it.nt * KT; i += kThreads) {
+                const int pos = i < g.c ? it.cand[i] : -1;
+                crow[i] = (int)(it.key0 + (pos >= 0 ? pos : 0));
+            }
+        }
         __syncthreads();
         const uint32_t idesc = tc::idesc_bf16_f32(128, 64 * it.m);
 
@@ -236,15 +247,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (GATHER) {
                     if (lane == 0) tc::mbar_arrive_expect_tx(&sh.afull[st], kAStage);
                     __syncwarp();
-                    int r[4];
-#pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        const int jj = j * KT + lane * 4 + i;
-                        const int pos = jj < g.c ? it.cand[jj] : -1;
-                        r[i] = (int)(it.key0 + (pos >= 0 ? pos : 0));
-                    }
+                    const int4 r = reinterpret_cast<const int4 *>(crow)[j * (KT / 4) + lane];
                     for (int kh = 0; kh < 2; ++kh)
-                        gather4(dst + kh * kASlice + lane * 4 * 128, &tmap_k, kh * 64, r[0], r[1], r[2], r[3],
+                        gather4(dst + kh * kASlice + lane * 4 * 128, &tmap_k, kh * 64, r.x, r.y, r.z, r.w,
                                 &sh.afull[st]);
                 } else if (lane == 0) {
                     tc::mbar_arrive_expect_tx(&sh.afull[st], kAStage);
@@ -376,9 +381,9 @@ int sm_count() {
 bool tc_decode_supported(int H, int d, int dtype, int rows_per_request) {
     return H == S_H && d == S_D && dtype == 0 && rows_per_request >= 1 && rows_per_request <= 4;
 }
-bool tc_gather_supported(int H, int d, int dtype, int group) {
+bool tc_gather_supported(int H, int d, int dtype, int group, int c) {
     (void)group;
-    return H == S_H && d == S_D && dtype == 0;
+    return H == S_H && d == S_D && dtype == 0 && c >= 1 && c <= kMaxCand;
 }
 
 cudaError_t launch_decode_tc(const DecodeArgs &a, cudaStream_t st) {
@@ -388,13 +393,14 @@ cudaError_t launch_decode_tc(const DecodeArgs &a, cudaStream_t st) {
         return cudaErrorInvalidValue;
     const int ntiles_max = (a.n_max + KT - 1) / KT;
     const int nitems = a.B * ((ntiles_max + kDecodeChunkTiles - 1) / kDecodeChunkTiles);
+    const size_t smem = smem_bytes(0);
     cudaError_t e = cudaFuncSetAttribute(stream_tc_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)kSmemBytes);
+                                         (int)smem);
     if (e != cudaSuccess) return e;
     GatherArgs g{};
     TraceScope ts("decode_tc", st);
     const int grid = nitems < sm_count() ? nitems : sm_count();
-    stream_tc_kernel<false><<<grid, kThreads, kSmemBytes, st>>>(mq, mk, g, a, nitems);
+    stream_tc_kernel<false><<<grid, kThreads, smem, st>>>(mq, mk, g, a, nitems);
     return cudaGetLastError();
 }
 
@@ -406,14 +412,15 @@ cudaError_t launch_gather_tc(const GatherArgs &a, cudaStream_t st) {
         return cudaErrorInvalidValue;
     const int mchunks = ((a.mode == 0 ? a.g : a.G) + 3) / 4;
     const int nitems = a.nitems * mchunks;
+    const size_t smem = smem_bytes((a.c + KT - 1) / KT * KT);
     cudaError_t e = cudaFuncSetAttribute(stream_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)kSmemBytes);
+                                         (int)smem);
     if (e != cudaSuccess) return e;
     DecodeArgs dd{};
     TraceScope ts("gather_tc", st);
     const int grid = nitems < sm_count() ? nitems : sm_count();
     if (grid <= 0) return cudaSuccess;
-    stream_tc_kernel<true><<<grid, kThreads, kSmemBytes, st>>>(mq, mk, a, dd, nitems);
+    stream_tc_kernel<true><<<grid, kThreads, smem, st>>>(mq, mk, a, dd, nitems);
     return cudaGetLastError();
 }
 
