@@ -45,13 +45,15 @@ struct Carve {
 
 size_t esize(idx_dtype dt) { return dt == IDX_F32 ? 4 : 2; }
 
+int c_pad_of(int c) { return (c + KT - 1) / KT * KT; }
+
 long long nbound(int T) { return T < kMaxLen ? T : kMaxLen; }
 
 struct PrefillWs {
     PlanLayout pl;
     long long R;          // scored rows (queries or proxies, upper bound)
     unsigned cap, ksel;
-    size_t status, plan, slot, qbar, wbar, cnt, floor, buf, cand, msc, total;
+    size_t status, plan, slot, qbar, wbar, cnt, floor, buf, cand, msc, ckeys, total;
 };
 
 PrefillWs prefill_ws(int T, int H, int d, int topk, int S, idx_dtype dt, int g, int c, idx_mode mode) {
@@ -75,12 +77,15 @@ PrefillWs prefill_ws(int T, int H, int d, int topk, int S, idx_dtype dt, int g, 
     L.buf = cv.take((size_t)L.R * L.cap * 8);
     L.cand = mode == IDX_MODE_REFINE ? cv.take((size_t)L.R * c * 4) : 0;
     L.msc = mode == IDX_MODE_REFINE ? cv.take((size_t)T * c * 4) : 0;
+    L.ckeys = (mode == IDX_MODE_REFINE && tc_gather_supported(H, d, (int)dt, g, c))
+                  ? cv.take((size_t)L.R * c_pad_of(c) * d * esize(dt))
+                  : 0;
     L.total = cv.off;
     return L;
 }
 
 struct DecodeWs {
-    size_t status, qbar, wbar, spill, cand, msc, total;
+    size_t status, qbar, wbar, spill, cand, msc, ckeys, total;
 };
 
 DecodeWs decode_ws(int B, int G, int n_max, int H, int d, int c, idx_mode mode, idx_dtype dt) {
@@ -93,6 +98,9 @@ DecodeWs decode_ws(int B, int G, int n_max, int H, int d, int c, idx_mode mode, 
     L.spill = cv.take((size_t)rows * n_max * 4);
     L.cand = mode == IDX_MODE_REFINE ? cv.take((size_t)B * c * 4) : 0;
     L.msc = mode == IDX_MODE_REFINE ? cv.take((size_t)B * G * c * 4) : 0;
+    L.ckeys = (mode == IDX_MODE_REFINE && tc_gather_supported(H, d, (int)dt, G, c))
+                  ? cv.take((size_t)B * c_pad_of(c) * d * esize(dt))
+                  : 0;
     L.total = cv.off;
     return L;
 }
@@ -227,6 +235,8 @@ struct Prefill {
         a.cu = cu; a.S = S; a.g = g; a.cu_T = T;
         a.plan = plan(); a.pl = L.pl;
         a.out = reinterpret_cast<float *>(ws + L.msc);
+        a.ckeys = ws + L.ckeys;
+        a.c_pad = c_pad_of(c);
         a.status = status();
         return a;
     }
@@ -375,6 +385,8 @@ struct Decode {
         a.mode = 1;
         a.G = G; a.n_max = n_max; a.kv_len = kv;
         a.out = reinterpret_cast<float *>(ws + L.msc);
+        a.ckeys = ws + L.ckeys;
+        a.c_pad = c_pad_of(c);
         a.status = status();
         return a;
     }

@@ -86,6 +86,8 @@ struct GatherArgs {
     int G, n_max;
     const int *kv_len;
     float *out;          // [rows, c] member scores
+    void *ckeys;         // [groups, c_pad, d] packed candidate keys (tensor-core path)
+    int c_pad;           // c rounded up to a multiple of 128
     unsigned *status;
 };
 

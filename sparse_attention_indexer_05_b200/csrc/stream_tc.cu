@@ -2,8 +2,10 @@
 // 64*m <= 256 columns) against a stream of key tiles and write every score:
 //   * decode scan: the keys are the request's cache, streamed once by TMA
 //     in 128-key tiles; rows = the request's G MTP queries (or its proxy);
-//   * Refine re-score: the keys are a group's candidate set C, gathered row
-//     by row with TMA gather4; rows = up to 4 members of the group.
+//   * Refine re-score: the keys are a group's candidate set C, first packed
+//     into a contiguous [c_pad, d] block per group by compact_keys_kernel
+//     (coalesced 16-byte copies), then streamed by TMA like the decode
+//     cache; rows = up to 4 members of the group.
 // Same MMA shape as the prefill score kernel (keys on M, (row, head) on N,
 // bf16 -> fp32 in TMEM, fused ReLU + w-weighted head sum), with the two
 // 256-column TMEM buffers used alternately by consecutive key tiles.
@@ -40,9 +42,7 @@ constexpr size_t kOffQ = 0;
 constexpr size_t kOffA = kOffQ + kQBytes;
 constexpr size_t kOffW = kOffA + (size_t)kStages * kAStage;
 constexpr size_t kOffCtl = kOffW + 4 * S_H * 4;
-constexpr size_t kOffCand = (kOffCtl + sizeof(StShared) + 15) / 16 * 16;  // gather: key rows of C
-constexpr int kMaxCand = 8192;
-__host__ __device__ constexpr size_t smem_bytes(int cand_slots) { return kOffCand + (size_t)cand_slots * 4 + 1024; }
+constexpr size_t kSmemBytes = kOffCtl + sizeof(StShared) + 1024;
 
 struct Item {
     bool valid;
@@ -53,7 +53,6 @@ struct Item {
     // outputs
     long long out_row0; // output row of scored row 0
     int bound0, bstep;  // decode: causal bound of row r = bound0 + bstep * r (inclusive)
-    const int *cand;    // gather: candidate positions of the group
 };
 
 template <bool GATHER>
@@ -84,14 +83,14 @@ __device__ __forceinline__ Item item_info(const GatherArgs &g, const DecodeArgs 
         }
         const int m = cnt - mc * 4;
         if (m <= 0) return it;
+        (void)key0;
         it.valid = true;
         it.m = m < 4 ? m : 4;
         it.qrow0 = m0 + mc * 4;
         it.out_row0 = it.qrow0;
-        it.key0 = key0;
+        it.key0 = (long long)grp * g.c_pad;  // the group's block of packed candidate keys
         it.t0 = 0;
-        it.nt = (g.c + KT - 1) / KT;
-        it.cand = g.cand + (long long)grp * g.c;
+        it.nt = g.c_pad / KT;
     } else {
         const int ntiles_max = (dd.n_max + KT - 1) / KT;
         const int nch = (ntiles_max + kDecodeChunkTiles - 1) / kDecodeChunkTiles;
@@ -156,15 +155,6 @@ __device__ __forceinline__ float reduce64(const uint32_t (&v0)[32], const uint32
     return ((a[0] + a[1]) + (a[2] + a[3])) + ((a[4] + a[5]) + (a[6] + a[7]));
 }
 
-__device__ __forceinline__ void gather4(void *dst, const CUtensorMap *map, int x, int r0, int r1, int r2, int r3,
-                                        uint64_t *bar) {
-    asm volatile(
-        "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
-        " [%0], [%1, {%3, %4, %5, %6, %7}], [%2];" ::"r"(tc::smem_u32(dst)),
-        "l"(reinterpret_cast<uint64_t>(map)), "r"(tc::smem_u32(bar)), "r"(x), "r"(r0), "r"(r1), "r"(r2), "r"(r3)
-        : "memory");
-}
-
 template <bool GATHER>
 __global__ void __launch_bounds__(kThreads, 1)
     stream_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_k,
@@ -176,7 +166,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint8_t *as = smem + kOffA;
     float *wsm = reinterpret_cast<float *>(smem + kOffW);
     StShared &sh = *reinterpret_cast<StShared *>(smem + kOffCtl);
-    int *crow = reinterpret_cast<int *>(smem + kOffCand);
     volatile int *abort = &sh.abort;
     unsigned *status = GATHER ? g.status : dd.status;
     const float *wsrc = GATHER ? g.w : dd.w;
@@ -220,14 +209,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         __syncthreads();
         for (int i = threadIdx.x; i < 4 * S_H; i += kThreads)
             wsm[i] = (i / S_H) < it.m ? wsrc[it.qrow0 * S_H + i] : 0.0f;
-        if (GATHER) {
-            // key rows of the group's candidates (padding slots read row key0; their
-            // scores are written but the select pass ignores position -1)
-            for (int i = threadIdx.x; i < it.nt * KT; i += kThreads) {
-                const int pos = i < g.c ? it.cand[i] : -1;
-                crow[i] = (int)(it.key0 + (pos >= 0 ? pos : 0));
-            }
-        }
         __syncthreads();
         const uint32_t idesc = tc::idesc_bf16_f32(128, 64 * it.m);
 
@@ -244,14 +225,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
                 if (!ok) break;
                 uint8_t *dst = as + st * kAStage;
-                if (GATHER) {
-                    if (lane == 0) tc::mbar_arrive_expect_tx(&sh.afull[st], kAStage);
-                    __syncwarp();
-                    const int4 r = reinterpret_cast<const int4 *>(crow)[j * (KT / 4) + lane];
-                    for (int kh = 0; kh < 2; ++kh)
-                        gather4(dst + kh * kASlice + lane * 4 * 128, &tmap_k, kh * 64, r.x, r.y, r.z, r.w,
-                                &sh.afull[st]);
-                } else if (lane == 0) {
+                if (lane == 0) {
                     tc::mbar_arrive_expect_tx(&sh.afull[st], kAStage);
                     const int row = (int)(it.key0 + (long long)(it.t0 + j) * KT);
                     for (int kh = 0; kh < 2; ++kh) tc::tma_load_2d(dst + kh * kASlice, &tmap_k, kh * 64, row, &sh.afull[st]);
@@ -341,6 +315,35 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (warp == 1) tc::tmem_dealloc(tmem, 512);
 }
 
+// Packs the key rows of every group's candidate set into a contiguous block
+// of c_pad rows (padding slots and the -1 pads of short sets copy the
+// request's row 0; their scores are written but never selected).
+// Grid (groups, c_pad / 128); each CTA copies 128 rows of d bf16.
+__global__ void __launch_bounds__(256) compact_keys_kernel(GatherArgs a) {
+    const int grp = blockIdx.x;
+    const int j0 = blockIdx.y * KT;
+    long long key0;
+    if (a.mode == 0) {
+        if (!a.plan[0] || grp >= a.plan[2]) return;
+        const int *rp = a.plan + a.pl.rp();
+        key0 = a.cu[find_seg(rp, a.S, grp)];
+    } else {
+        const int kv = a.kv_len[grp];
+        if (kv < a.G || kv > a.n_max) return;
+        key0 = (long long)grp * a.n_max;
+    }
+    const int *cand = a.cand + (long long)grp * a.c;
+    const int per_row = a.d * 2 / 16;  // 16-byte chunks per key row
+    const uint4 *src = reinterpret_cast<const uint4 *>(a.k);
+    uint4 *dst = reinterpret_cast<uint4 *>(a.ckeys) + ((long long)grp * a.c_pad + j0) * per_row;
+    for (int u = threadIdx.x; u < KT * per_row; u += blockDim.x) {
+        const int r = u / per_row, part = u - r * per_row;
+        const int j = j0 + r;
+        const int pos = j < a.c ? cand[j] : -1;
+        dst[u] = src[(key0 + (pos >= 0 ? pos : 0)) * per_row + part];
+    }
+}
+
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn2() {
     static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
     if (!fn) {
@@ -383,7 +386,7 @@ bool tc_decode_supported(int H, int d, int dtype, int rows_per_request) {
 }
 bool tc_gather_supported(int H, int d, int dtype, int group, int c) {
     (void)group;
-    return H == S_H && d == S_D && dtype == 0 && c >= 1 && c <= kMaxCand;
+    return H == S_H && d == S_D && dtype == 0 && c >= 1;
 }
 
 cudaError_t launch_decode_tc(const DecodeArgs &a, cudaStream_t st) {
@@ -393,7 +396,7 @@ cudaError_t launch_decode_tc(const DecodeArgs &a, cudaStream_t st) {
         return cudaErrorInvalidValue;
     const int ntiles_max = (a.n_max + KT - 1) / KT;
     const int nitems = a.B * ((ntiles_max + kDecodeChunkTiles - 1) / kDecodeChunkTiles);
-    const size_t smem = smem_bytes(0);
+    const size_t smem = kSmemBytes;
     cudaError_t e = cudaFuncSetAttribute(stream_tc_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)smem);
     if (e != cudaSuccess) return e;
@@ -406,13 +409,20 @@ cudaError_t launch_decode_tc(const DecodeArgs &a, cudaStream_t st) {
 
 cudaError_t launch_gather_tc(const GatherArgs &a, cudaStream_t st) {
     const long long qrows = a.mode == 0 ? (long long)a.cu_T : (long long)a.G * a.nitems;
-    const long long krows = a.mode == 0 ? (long long)a.cu_T : (long long)a.nitems * a.n_max;
+    const long long krows = (long long)a.nitems * a.c_pad;  // packed candidate keys
     CUtensorMap mq, mk;
-    if (!map2d(&mq, a.q, (unsigned long long)qrows * S_H, 256) || !map2d(&mk, a.k, (unsigned long long)krows, 1))
+    if (!map2d(&mq, a.q, (unsigned long long)qrows * S_H, 256) || !map2d(&mk, a.ckeys, (unsigned long long)krows, KT))
         return cudaErrorInvalidValue;
+    {
+        TraceScope tsc("pack_keys", st);
+        dim3 cgrid(a.nitems, a.c_pad / KT);
+        compact_keys_kernel<<<cgrid, 256, 0, st>>>(a);
+        cudaError_t ce = cudaGetLastError();
+        if (ce != cudaSuccess) return ce;
+    }
     const int mchunks = ((a.mode == 0 ? a.g : a.G) + 3) / 4;
     const int nitems = a.nitems * mchunks;
-    const size_t smem = smem_bytes((a.c + KT - 1) / KT * KT);
+    const size_t smem = kSmemBytes;
     cudaError_t e = cudaFuncSetAttribute(stream_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)smem);
     if (e != cudaSuccess) return e;
