@@ -34,7 +34,7 @@ constexpr int TC_H = 64;
 constexpr int TC_D = 128;
 constexpr int kEpiWarps = 16;                         // 4 per TMEM lane quarter, one query each per half
 constexpr int kThreads = 64 + 32 * kEpiWarps;         // + TMA warp + MMA warp
-constexpr int kMaintEvery = 2;                        // tiles between candidate-filter upkeeps
+constexpr int kMaintEvery = 4;                        // tiles between candidate-filter upkeeps
 constexpr int kStages = 2;                            // key-tile stages
 constexpr uint32_t kQHalfBytes = 256 * 128;           // one half, one 64-column K slice (32 KB)
 constexpr uint32_t kQBytes = 4 * kQHalfBytes;         // 2 halves x 2 K slices (128 KB)
@@ -62,9 +62,47 @@ constexpr size_t kOffScr = kOffHist + (size_t)RB * kBins * 4;
 constexpr size_t kOffCtl = kOffScr + (size_t)RB * 256 * 4;
 constexpr size_t kSmemBytes = kOffCtl + sizeof(TcShared) + 1024;  // + alignment slack
 
+// Packed (2 x fp32) fused multiply-add: acc.{x,y} = w.{x,y} * r.{x,y} + acc.{x,y},
+// each lane of the pair rounded separately (the sm_100 fma.rn.f32x2).
+__device__ __forceinline__ unsigned long long ffma2(unsigned long long acc, float w0, float w1, float r0, float r1) {
+    unsigned long long wp, rp;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(wp) : "f"(w0), "f"(w1));
+    asm("mov.b64 %0, {%1, %2};" : "=l"(rp) : "f"(r0), "f"(r1));
+    asm("fma.rn.f32x2 %0, %1, %2, %0;" : "+l"(acc) : "l"(wp), "l"(rp));
+    return acc;
+}
+
 // sum_j w[j] * max(v[j], 0) over 64 heads held in two 32-register groups;
-// w read as float4 (16-byte aligned); 8 independent partial sums.
+// w read as float4 (16-byte aligned); 8 independent partial sums kept as 4
+// packed pairs, so each two heads cost two max and one packed fma.
 __device__ __forceinline__ float head_reduce(const uint32_t (&v0)[32], const uint32_t (&v1)[32], const float *w) {
+    const float4 *w4 = reinterpret_cast<const float4 *>(w);
+    unsigned long long a[4] = {0ull, 0ull, 0ull, 0ull};
+#pragma unroll
+    for (int j4 = 0; j4 < 8; ++j4) {
+        const float4 wv = w4[j4];
+        a[(2 * j4) & 3] = ffma2(a[(2 * j4) & 3], wv.x, wv.y, fmaxf(__uint_as_float(v0[4 * j4 + 0]), 0.0f),
+                                fmaxf(__uint_as_float(v0[4 * j4 + 1]), 0.0f));
+        a[(2 * j4 + 1) & 3] = ffma2(a[(2 * j4 + 1) & 3], wv.z, wv.w, fmaxf(__uint_as_float(v0[4 * j4 + 2]), 0.0f),
+                                    fmaxf(__uint_as_float(v0[4 * j4 + 3]), 0.0f));
+    }
+#pragma unroll
+    for (int j4 = 0; j4 < 8; ++j4) {
+        const float4 wv = w4[8 + j4];
+        a[(2 * j4) & 3] = ffma2(a[(2 * j4) & 3], wv.x, wv.y, fmaxf(__uint_as_float(v1[4 * j4 + 0]), 0.0f),
+                                fmaxf(__uint_as_float(v1[4 * j4 + 1]), 0.0f));
+        a[(2 * j4 + 1) & 3] = ffma2(a[(2 * j4 + 1) & 3], wv.z, wv.w, fmaxf(__uint_as_float(v1[4 * j4 + 2]), 0.0f),
+                                    fmaxf(__uint_as_float(v1[4 * j4 + 3]), 0.0f));
+    }
+    float s[8];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) asm("mov.b64 {%0, %1}, %2;" : "=f"(s[2 * i]), "=f"(s[2 * i + 1]) : "l"(a[i]));
+    return ((s[0] + s[1]) + (s[2] + s[3])) + ((s[4] + s[5]) + (s[6] + s[7]));
+}
+
+// The same sum with scalar fma (reference form, unused by the kernel).
+__device__ __forceinline__ float head_reduce_scalar(const uint32_t (&v0)[32], const uint32_t (&v1)[32],
+                                                    const float *w) {
     const float4 *w4 = reinterpret_cast<const float4 *>(w);
     float a[8];
 #pragma unroll
