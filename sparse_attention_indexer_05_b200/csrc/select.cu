@@ -33,6 +33,7 @@ constexpr int kMaxBins = 4096;  // widest radix digit: 12 bits
 // candidate keys of a score pass; entries below the row's floor (a score
 // that at least ksel appended keys reach) can no longer be selected
 struct CandSrc {
+    static constexpr bool kFloor = true;  // valid entries are few: stage them directly
     const unsigned long long *buf;
     int n;
     int bound;
@@ -45,6 +46,7 @@ struct CandSrc {
 
 // dense fp32 scores with their positions (NULL: position = index)
 struct ScoreSrc {
+    static constexpr bool kFloor = false;
     const float *sc;
     const int *pos;
     int n;
@@ -260,11 +262,59 @@ __device__ void emit(const Src &src, unsigned long long K, int nsel, int k, int 
     }
 }
 
+// Append the keys of src that are valid and >= lo to the shared stage
+// (order not kept); returns how many there were (the stage holds the first
+// stage_cap of them).
+template <class Src>
+__device__ unsigned stage_keys(const Src &src, SelShared &sh, unsigned long long lo, unsigned long long *stage,
+                               int stage_cap) {
+    const int tid = threadIdx.x, nt = blockDim.x, lane = tid & 31;
+    if (tid == 0) sh.nstage = 0;
+    __syncthreads();
+    for (int base = 0; base < src.n; base += nt * kUnroll) {
+        unsigned long long key[kUnroll];
+#pragma unroll
+        for (int u = 0; u < kUnroll; ++u) {
+            const int i = base + u * nt + tid;
+            key[u] = i < src.n ? src.key(i) : 0ull;
+        }
+#pragma unroll
+        for (int u = 0; u < kUnroll; ++u) {
+            const bool keep = key[u] != 0ull && key[u] >= lo;
+            const unsigned m = __ballot_sync(0xFFFFFFFFu, keep);
+            if (m) {
+                unsigned b = 0;
+                if (lane == __ffs(m) - 1) b = atomicAdd(&sh.nstage, (unsigned)__popc(m));
+                b = __shfl_sync(0xFFFFFFFFu, b, __ffs(m) - 1) + __popc(m & lanemask_lt());
+                if (keep && b < (unsigned)stage_cap) stage[b] = key[u];
+            }
+        }
+    }
+    __syncthreads();
+    return sh.nstage;
+}
+
 template <class Src>
 __device__ void block_select(const Src &src, int k, int *out_idx, float *out_score, SelShared &sh,
                              unsigned long long *stage, int stage_cap, unsigned *bm, unsigned *gpre, int wcap,
                              unsigned *status) {
     const int tid = threadIdx.x, nt = blockDim.x, lane = tid & 31;
+    if (Src::kFloor) {
+        // candidate rows: the entries at or above the row's floor are about
+        // k plus a bin's worth; one pass stages them all
+        const unsigned ns = stage_keys(src, sh, 1ull, stage, stage_cap);
+        if (ns <= (unsigned)stage_cap) {
+            const StageSrc ss{stage, (int)ns, src.bound};
+            if (ns <= (unsigned)k) {
+                emit(ss, 1ull, (int)ns, k, out_idx, out_score, bm, gpre, wcap, status);
+            } else {
+                const unsigned long long K = radix_kth(ss, sh, (unsigned)k, 0, 0ull, 0ull);
+                emit(ss, K, k, k, out_idx, out_score, bm, gpre, wcap, status);
+            }
+            return;
+        }
+        __syncthreads();  // too many: select over the row in global memory
+    }
     // pass 1: valid count and the top-12-bit histogram
     for (int i = tid; i < kMaxBins; i += nt) sh.hist[i] = 0u;
     if (tid == 0) {
