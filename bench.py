@@ -70,6 +70,33 @@ def proxy_pairs(n, g):
     return tot
 
 
+SCORE_SOURCES = ["score_tc.cu", "tc.cuh", "common.cuh", "internal.h", "plan.cuh"]
+
+
+def score_sources_sha():
+    """sha256 over the sources of the dense score kernel (to tell whether a
+    recorded ncu traffic figure still describes the kernel that runs)."""
+    import hashlib
+    h = hashlib.sha256()
+    for f in SCORE_SOURCES:
+        with open(os.path.join(ROOT, "sparse_attention_indexer_05_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()
+
+
+def recorded_traffic(L):
+    """DRAM bytes (read + write) of one dense score launch from the committed
+    ncu capture, or None when the kernel changed since or the size differs."""
+    path = os.path.join(ROOT, "profiles", "score_tc_dense_L131072_traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        rec = json.load(f)
+    if rec.get("sources_sha256") != score_sources_sha() or rec.get("tokens") != L:
+        return None
+    return rec["dram_bytes_read"] + rec["dram_bytes_write"]
+
+
 def peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
@@ -281,7 +308,7 @@ def main():
     achieved = dense_flops_single(L) / (dense_ms / 1000.0) / 1e12 if dense_ms > 0 else None
     roof = {"kernel": "score_tc (dense pass)", "bound": "tensor", "achieved": achieved,
             "peak": bf16_sus, "unit": "TFLOP/s", "frac": (achieved / bf16_sus) if achieved else None,
-            "traffic": None, "peak_kind": f"{peak_src} bf16 sustained (kernel timed inside a long step)",
+            "traffic": recorded_traffic(L), "peak_kind": f"{peak_src} bf16 sustained (kernel timed inside a long step)",
             "flops_per_launch": dense_flops_single(L), "ms_per_launch": dense_ms}
 
     per_kernel = {name: {"launches": c, "ms_total": t, "ms_per_step": t / args.steps} for name, (c, t) in tr.items()}

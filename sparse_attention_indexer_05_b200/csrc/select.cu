@@ -34,6 +34,7 @@ constexpr int kMaxBins = 4096;  // widest radix digit: 12 bits
 // that at least ksel appended keys reach) can no longer be selected
 struct CandSrc {
     static constexpr bool kFloor = true;  // valid entries are few: stage them directly
+    static constexpr bool kShared = false;
     const unsigned long long *buf;
     int n;
     int bound;
@@ -47,6 +48,7 @@ struct CandSrc {
 // dense fp32 scores with their positions (NULL: position = index)
 struct ScoreSrc {
     static constexpr bool kFloor = false;
+    static constexpr bool kShared = false;
     const float *sc;
     const int *pos;
     int n;
@@ -60,6 +62,8 @@ struct ScoreSrc {
 
 // keys staged in shared memory (all valid)
 struct StageSrc {
+    static constexpr bool kFloor = false;
+    static constexpr bool kShared = true;  // cheap to read: no unrolled prefetch needed
     const unsigned long long *st;
     int n;
     int bound;
@@ -145,20 +149,32 @@ __device__ unsigned hist_pass(const Src &src, SelShared &sh, int shift, unsigned
                               unsigned long long mask) {
     const int tid = threadIdx.x, nt = blockDim.x, lane = tid & 31;
     unsigned nvl = 0;
-    for (int base = 0; base < src.n; base += nt * kUnroll) {
-        unsigned long long key[kUnroll];
-#pragma unroll
-        for (int u = 0; u < kUnroll; ++u) {
-            const int i = base + u * nt + tid;
-            key[u] = i < src.n ? src.key(i) : 0ull;
-        }
-#pragma unroll
-        for (int u = 0; u < kUnroll; ++u) {
-            nvl += key[u] != 0ull;
-            const bool act = key[u] != 0ull && (key[u] & mask) == prefix;
-            const unsigned dg = act ? (unsigned)(key[u] >> shift) & dmask : 0xFFFFFFFFu;
+    if constexpr (Src::kShared) {
+        for (int base = 0; base < src.n; base += nt) {
+            const int i = base + tid;
+            const unsigned long long key = i < src.n ? src.key(i) : 0ull;
+            nvl += key != 0ull;
+            const bool act = key != 0ull && (key & mask) == prefix;
+            const unsigned dg = act ? (unsigned)(key >> shift) & dmask : 0xFFFFFFFFu;
             const unsigned m = __match_any_sync(0xFFFFFFFFu, dg);
             if (act && lane == __ffs(m) - 1) atomicAdd(&sh.hist[dg], (unsigned)__popc(m));
+        }
+    } else {
+        for (int base = 0; base < src.n; base += nt * kUnroll) {
+            unsigned long long key[kUnroll];
+#pragma unroll
+            for (int u = 0; u < kUnroll; ++u) {
+                const int i = base + u * nt + tid;
+                key[u] = i < src.n ? src.key(i) : 0ull;
+            }
+#pragma unroll
+            for (int u = 0; u < kUnroll; ++u) {
+                nvl += key[u] != 0ull;
+                const bool act = key[u] != 0ull && (key[u] & mask) == prefix;
+                const unsigned dg = act ? (unsigned)(key[u] >> shift) & dmask : 0xFFFFFFFFu;
+                const unsigned m = __match_any_sync(0xFFFFFFFFu, dg);
+                if (act && lane == __ffs(m) - 1) atomicAdd(&sh.hist[dg], (unsigned)__popc(m));
+            }
         }
     }
     return nvl;
@@ -217,29 +233,27 @@ __device__ void emit(const Src &src, unsigned long long K, int nsel, int k, int 
                 }
             }
             __syncthreads();
-            // per group of 32 words: exclusive prefix of the set bits
-            const int NG = (W + 31) / 32;
-            for (int gi = tid; gi < NG; gi += nt) {
-                unsigned s = 0;
-                const int e = (gi + 1) * 32 < W ? (gi + 1) * 32 : W;
-                for (int w = gi * 32; w < e; ++w) s += __popc(bm[w]);
-                gpre[gi] = s;
-            }
-            __syncthreads();
-            if (tid < 32) {  // warp-level exclusive scan over the groups
-                unsigned carry = 0;
-                for (int g0 = 0; g0 < NG; g0 += 32) {
-                    const int gi = g0 + tid;
-                    const unsigned s = gi < NG ? gpre[gi] : 0u;
-                    unsigned inc = s;
+            // exclusive prefix of the set bits per word: each thread owns a
+            // contiguous run of words; a block scan of the runs' totals
+            const int per = (W + nt - 1) / nt;
+            const int w0 = tid * per, w1 = w0 + per < W ? w0 + per : W;
+            unsigned run = 0;
+            for (int w = w0; w < w1; ++w) run += __popc(bm[w]);
+            unsigned inc = run;
 #pragma unroll
-                    for (int o = 1; o < 32; o <<= 1) {
-                        const unsigned v = __shfl_up_sync(0xFFFFFFFFu, inc, o);
-                        if (tid >= o) inc += v;
-                    }
-                    if (gi < NG) gpre[gi] = carry + inc - s;
-                    carry += __shfl_sync(0xFFFFFFFFu, inc, 31);
-                }
+            for (int o = 1; o < 32; o <<= 1) {
+                const unsigned v = __shfl_up_sync(0xFFFFFFFFu, inc, o);
+                if ((tid & 31) >= o) inc += v;
+            }
+            if ((tid & 31) == 31) gpre[W + (tid >> 5)] = inc;  // warp totals after the words
+            __syncthreads();
+            unsigned before = 0;
+            for (int w2 = 0; w2 < (tid >> 5); ++w2) before += gpre[W + w2];
+            unsigned acc = before + inc - run;
+            for (int w = w0; w < w1; ++w) {
+                const unsigned c = __popc(bm[w]);
+                gpre[w] = acc;
+                acc += c;
             }
             __syncthreads();
             for (int i = tid; i < src.n; i += nt) {
@@ -247,9 +261,7 @@ __device__ void emit(const Src &src, unsigned long long K, int nsel, int k, int 
                 if (key != 0ull && key >= K) {
                     const int p = key_pos(key);
                     const int w = p >> 5;
-                    unsigned r = gpre[w >> 5];
-                    for (int w2 = w & ~31; w2 < w; ++w2) r += __popc(bm[w2]);
-                    r += __popc(bm[w] & ((1u << (p & 31)) - 1u));
+                    const unsigned r = gpre[w] + __popc(bm[w] & ((1u << (p & 31)) - 1u));
                     out_idx[r] = p;
                     if (out_score) out_score[r] = ord_score(key_ord(key));
                 }
@@ -278,15 +290,27 @@ __device__ unsigned stage_keys(const Src &src, SelShared &sh, unsigned long long
             const int i = base + u * nt + tid;
             key[u] = i < src.n ? src.key(i) : 0ull;
         }
+        // one reservation per warp for all kept keys of the round
+        unsigned cnt = 0;
 #pragma unroll
-        for (int u = 0; u < kUnroll; ++u) {
-            const bool keep = key[u] != 0ull && key[u] >= lo;
-            const unsigned m = __ballot_sync(0xFFFFFFFFu, keep);
-            if (m) {
-                unsigned b = 0;
-                if (lane == __ffs(m) - 1) b = atomicAdd(&sh.nstage, (unsigned)__popc(m));
-                b = __shfl_sync(0xFFFFFFFFu, b, __ffs(m) - 1) + __popc(m & lanemask_lt());
-                if (keep && b < (unsigned)stage_cap) stage[b] = key[u];
+        for (int u = 0; u < kUnroll; ++u) cnt += (key[u] != 0ull && key[u] >= lo) ? 1u : 0u;
+        unsigned inc = cnt;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const unsigned v = __shfl_up_sync(0xFFFFFFFFu, inc, o);
+            if (lane >= o) inc += v;
+        }
+        const unsigned total = __shfl_sync(0xFFFFFFFFu, inc, 31);
+        if (total) {
+            unsigned b = 0;
+            if (lane == 31) b = atomicAdd(&sh.nstage, total);
+            b = __shfl_sync(0xFFFFFFFFu, b, 31) + inc - cnt;
+#pragma unroll
+            for (int u = 0; u < kUnroll; ++u) {
+                if (key[u] != 0ull && key[u] >= lo) {
+                    if (b < (unsigned)stage_cap) stage[b] = key[u];
+                    ++b;
+                }
             }
         }
     }
@@ -299,7 +323,7 @@ __device__ void block_select(const Src &src, int k, int *out_idx, float *out_sco
                              unsigned long long *stage, int stage_cap, unsigned *bm, unsigned *gpre, int wcap,
                              unsigned *status) {
     const int tid = threadIdx.x, nt = blockDim.x, lane = tid & 31;
-    if (Src::kFloor) {
+    if constexpr (Src::kFloor) {
         // candidate rows: the entries at or above the row's floor are about
         // k plus a bin's worth; one pass stages them all
         const unsigned ns = stage_keys(src, sh, 1ull, stage, stage_cap);
@@ -339,27 +363,8 @@ __device__ void block_select(const Src &src, int k, int *out_idx, float *out_sco
     }
     if (above0 + inbin0 <= (unsigned)stage_cap) {
         // pass 2: stage the keys of bin d0 and above
-        for (int base = 0; base < src.n; base += nt * kUnroll) {
-            unsigned long long key[kUnroll];
-#pragma unroll
-            for (int u = 0; u < kUnroll; ++u) {
-                const int i = base + u * nt + tid;
-                key[u] = i < src.n ? src.key(i) : 0ull;
-            }
-#pragma unroll
-            for (int u = 0; u < kUnroll; ++u) {
-                const bool keep = key[u] != 0ull && key[u] >= pre0;
-                const unsigned m = __ballot_sync(0xFFFFFFFFu, keep);
-                if (m) {
-                    unsigned b = 0;
-                    if (lane == __ffs(m) - 1) b = atomicAdd(&sh.nstage, (unsigned)__popc(m));
-                    b = __shfl_sync(0xFFFFFFFFu, b, __ffs(m) - 1);
-                    if (keep) stage[b + __popc(m & lanemask_lt())] = key[u];
-                }
-            }
-        }
-        __syncthreads();
-        const StageSrc ss{stage, (int)sh.nstage, src.bound};
+        const unsigned ns = stage_keys(src, sh, pre0, stage, stage_cap);
+        const StageSrc ss{stage, (int)ns, src.bound};
         const unsigned long long K = radix_kth(ss, sh, need, 1, pre0, mask0);
         emit(ss, K, k, k, out_idx, out_score, bm, gpre, wcap, status);
         return;
@@ -455,7 +460,7 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(SelectArgs a) {
 cudaError_t launch_select(const SelectArgs &a, cudaStream_t st) {
     if (a.nrows <= 0) return cudaSuccess;
     SelectArgs b = a;
-    const size_t tail = ((size_t)a.bitmap_words + (size_t)(a.bitmap_words + 31) / 32 + 1) * 4;
+    const size_t tail = ((size_t)a.bitmap_words * 2 + 32) * 4;  // bitmap + per-word prefix + warp totals
     const size_t limit = 232448 - sizeof(SelShared) - 1024;
     // staging room: the k-th key's 1/16-octave bin and everything above it
     long long cap = 2LL * a.k + 2048;
