@@ -190,6 +190,13 @@ idx_status idx_debug_decode_scores(int stage, const void *q, const void *kcache,
                                    int c, idx_mode mode, idx_dtype dtype, float *out, long long ld,
                                    void *ws, size_t ws_bytes, idx_stream_t stream);
 
+/* Test hook for failure detection: launches one thread that waits, with the
+ * bounded wait every tensor-core kernel uses, on a barrier nothing completes.
+ * After limit_ms milliseconds (1..10000) the wait gives up and records
+ * IDX_ERR_TIMEOUT in the status word of `ws` (at least 4 bytes); read it
+ * with idx_device_status().  Nothing faults and the context stays usable. */
+idx_status idx_debug_wait_probe(void *ws, unsigned limit_ms, idx_stream_t stream);
+
 /* Per-kernel device timing.  idx_trace_enable(1) clears the record and
  * starts bracketing every kernel launch of the library with two CUDA events
  * on its stream; idx_trace_enable(0) stops (the record is kept).

@@ -46,13 +46,13 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
 // (or at once when another role already gave up): records ST_TIMEOUT, sets
 // *abort and returns false, so that the CTA unwinds instead of hanging.
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort,
-                                          unsigned *status) {
+                                          unsigned *status, unsigned long long limit_ns = kWaitNs) {
     if (mbar_try_wait(bar, parity)) return true;
     const unsigned long long t0 = globaltimer_ns();
     for (unsigned it = 1;; ++it) {
         if (mbar_try_wait(bar, parity)) return true;
         if (*abort) return false;
-        if ((it & 31u) == 0u && globaltimer_ns() - t0 > kWaitNs) {
+        if ((it & 31u) == 0u && globaltimer_ns() - t0 > limit_ns) {
             *abort = 1;
             raise_status(status, ST_TIMEOUT);
             return false;

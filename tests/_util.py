@@ -46,6 +46,14 @@ def check_scores(gpu: np.ndarray, ora: np.ndarray, rtol=1e-3):
     assert not bad.any(), f"{bad.sum()} scores off, worst {np.max(np.abs(gpu - ora) - tol)}"
 
 
+def score_rows(jobs, threads=16):
+    """Oracle score rows for a list of (q, k, w, q_row, key0, n) jobs, in parallel
+    (the oracle call releases the interpreter lock)."""
+    from concurrent.futures import ThreadPoolExecutor
+    with ThreadPoolExecutor(max_workers=threads) as ex:
+        return list(ex.map(lambda j: O.score_row(*j), jobs))
+
+
 def reselect(scores_f32: np.ndarray, k: int, pos=None) -> np.ndarray:
     """The oracle's selection rule applied to scores the GPU exported."""
     return O.select(np.asarray(scores_f32, np.float32).astype(np.float64), k, pos)
