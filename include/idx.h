@@ -175,7 +175,8 @@ const char *idx_status_string(idx_status s);
  *   2: PIVOT Refine member re-scores over the candidate set (rows[] = global
  *      member rows; out[i * ld + j] is the score of candidate j of the
  *      member's group, j < c; requires that idx_pivot_topk ran on `ws`).
- * rows is a DEVICE int32 array.  The scores come from the same kernels and
+ * rows is a DEVICE int32 array of DISTINCT rows (a row listed twice gets one
+ * of its output rows written).  The scores come from the same kernels and
  * arithmetic as the selection, so re-selecting on them reproduces out_idx. */
 idx_status idx_debug_scores(int stage, const void *q, const void *k, const float *w,
                             const int *cu_seqlens, int num_seqs, int T, int H, int d, idx_dtype dtype,

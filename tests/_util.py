@@ -40,6 +40,7 @@ def check_scores(gpu: np.ndarray, ora: np.ndarray, rtol=1e-3):
     bf16/fp32 inputs with fp32 accumulation against the double oracle."""
     gpu = np.asarray(gpu, np.float64)
     ora = np.asarray(ora, np.float64)
+    assert np.isfinite(gpu).all(), "non-finite GPU score (an entry was not written)"
     m = np.abs(ora).max() if ora.size else 0.0
     tol = rtol * np.maximum(np.abs(ora), 1e-3 * m)
     bad = np.abs(gpu - ora) > tol

@@ -77,8 +77,10 @@ def _check_pivot_rows(idx, P, dev, got, rows, topk, g, c, mode, ws):
         lo = (t // g) * g
         plist.append(req_first_proxy[b] + t // g)
         geo.append((b, t, lo, min(lo + g, n)))
-    psc = idx.debug_scores(1, q, k, w, cu, topk, torch.tensor(plist, dtype=torch.int32), g=g,
-                           c=c if mode == "refine" else 0).cpu().numpy()
+    # export each proxy once (members of one group share it)
+    uniq, slot = np.unique(np.asarray(plist), return_inverse=True)
+    psc = idx.debug_scores(1, q, k, w, cu, topk, torch.from_numpy(uniq.astype(np.int32)), g=g,
+                           c=c if mode == "refine" else 0).cpu().numpy()[slot]
     msc = None
     if mode == "refine":
         msc = idx.debug_scores(2, q, k, w, cu, topk, torch.from_numpy(rows.astype(np.int32)), g=g, c=c,
