@@ -8,8 +8,9 @@ Refine (g=16, c=4096) over the same tokens as TWO packed 65536-token
 requests (proxy build, proxy scan, candidate select, member re-score,
 member select).  `value` = query rows ranked per second (2 * 131072 per
 step, whole job).  The decode step (B=64 requests x 131072-token caches,
-G=2 MTP queries, dense and Refine c=4096) is timed after it and reported
-under "decode" as HBM GB/s of the cache scan.
+G=2 MTP queries, dense and Refine c=4096, and dense over the same cache
+scattered into 64-key pages behind a block table) is timed after it and
+reported under "decode" as HBM GB/s of the cache scan.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
@@ -357,15 +358,28 @@ def main():
                               for m in ("dense", "refine")), dtype=torch.uint8, device=dev)
         od = torch.empty(DEC_B, DEC_G, TOPK, dtype=torch.int32, device=dev)
         dec = {"workload": "decode_B64_n131072_G2_H64_d128_k2048", "kcache_bytes": Dd.kcache.nbytes}
-        for mode in ("dense", "refine"):
+        # the same cache scattered over a shuffled pool of 64-key pages (block-table layout)
+        PAGE = 64
+        npg = DEC_N // PAGE
+        gen = torch.Generator(device=dev)
+        gen.manual_seed(1234 + rank)
+        perm = torch.randperm(DEC_B * npg, device=dev, generator=gen)
+        dpool = torch.empty(DEC_B * npg, PAGE, D, dtype=dkc.dtype, device=dev)
+        dpool[perm] = dkc.reshape(DEC_B * npg, PAGE, D)
+        dbt = perm.to(torch.int32).reshape(DEC_B, npg)
+        runs = {"dense": lambda m: idx.decode_topk(dq_, dkc, dkv, dw_, TOPK, C_REF, m, out_idx=od, workspace=wsd),
+                "refine": lambda m: idx.decode_topk(dq_, dkc, dkv, dw_, TOPK, C_REF, m, out_idx=od, workspace=wsd),
+                "paged64_dense": lambda m: idx.decode_paged_topk(dq_, dpool, dbt, dkv, dw_, TOPK, C_REF, "dense",
+                                                                  out_idx=od, workspace=wsd)}
+        for mode, fn in runs.items():
             for _ in range(args.warmup):
-                idx.decode_topk(dq_, dkc, dkv, dw_, TOPK, C_REF, mode, out_idx=od, workspace=wsd)
+                fn(mode)
             torch.cuda.synchronize()
             assert idx.device_status(wsd) == "IDX_OK"
             lib.idx_trace_enable(1)
             e0.record(stream)
             for _ in range(args.steps):
-                idx.decode_topk(dq_, dkc, dkv, dw_, TOPK, C_REF, mode, out_idx=od, workspace=wsd)
+                fn(mode)
             e1.record(stream)
             torch.cuda.synchronize()
             lib.idx_trace_enable(0)
@@ -378,6 +392,7 @@ def main():
                          "scan_GBps": gbs, "scan_frac_hbm": (gbs / hbm_peak) if gbs else None,
                          "kernels": {n: {"launches": c, "ms_per_step": t / args.steps} for n, (c, t) in trd.items()}}
         dec["hbm_peak_GBps"] = hbm_peak
+        del dpool, dbt, perm
 
     # -------------------------------------------------------- CPU baseline
     cpu = None

@@ -129,6 +129,29 @@ idx_status idx_decode_topk(const void *q, const void *kcache, const int *kv_len,
                            idx_dtype dtype, int *out_idx, float *out_score, void *ws,
                            size_t ws_bytes, idx_stream_t stream);
 
+/* idx_decode_topk over a paged key cache (the block-table layout of
+ * paged-attention serving engines; the pages describe a contiguous cache
+ * and leave its storage open).  Same queries, weights, modes, outputs and
+ * status as idx_decode_topk; only the key addressing differs:
+ *   kpool        [num_pages, page, d] dtype   device pages of keys
+ *   block_table  [B, max_pages] int32          device; position s of request
+ *                b is row s % page of page block_table[b, s / page].
+ *                Entries covering only positions >= kv_len[b] may hold any
+ *                value and never change a result.  An entry outside
+ *                [0, num_pages) is read as page 0.
+ *   page         keys per page: a divisor of 128 (1, 2, 4, ..., 128) or a
+ *                multiple of 128, else IDX_ERR_UNSUPPORTED.  Pages of 8 keys
+ *                or more use the tensor-core scan; smaller ones the CUDA-core
+ *                scan.
+ *   kv_len[b] <= max_pages * page <= 2^20; num_pages * page < 2^31.
+ * Workspace: idx_decode_workspace_size(B, G, max_pages * page, ...).
+ * Returns IDX_ERR_INVALID for a NULL block_table or a non-positive size. */
+idx_status idx_decode_paged_topk(const void *q, const void *kpool, const int *block_table,
+                                 const int *kv_len, const float *w, int B, int G, int max_pages,
+                                 int page, long long num_pages, int H, int d, int topk, int c,
+                                 idx_mode mode, idx_dtype dtype, int *out_idx, float *out_score,
+                                 void *ws, size_t ws_bytes, idx_stream_t stream);
+
 /* ----------------------------------------------- no-allocation variant */
 
 /* The pages have no counterpart of this entry point; it exists for callers

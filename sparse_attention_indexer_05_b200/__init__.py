@@ -3,8 +3,9 @@
 The computation lives in libidx.so (CUDA, sm_100a) behind the C ABI of
 include/idx.h; `indexer` is its thin Python binding.
 """
-from .indexer import (debug_decode_scores, debug_scores, decode_topk, decode_workspace_size, dense_topk,
+from .indexer import (debug_decode_scores, debug_scores, decode_paged_topk, decode_topk, decode_workspace_size,
+                      dense_topk,
                       dense_workspace_size, device_status, pivot_topk, pivot_workspace_size, uses_tensor_cores)
 
-__all__ = ["dense_topk", "pivot_topk", "decode_topk", "dense_workspace_size", "pivot_workspace_size",
+__all__ = ["dense_topk", "pivot_topk", "decode_topk", "decode_paged_topk", "dense_workspace_size", "pivot_workspace_size",
            "decode_workspace_size", "device_status", "uses_tensor_cores", "debug_scores", "debug_decode_scores"]

@@ -23,6 +23,8 @@ SIGNATURES = {
     "idx_decode_workspace_size": (_sz, [_i, _i, _i, _i, _i, _i, _i, _i, _i]),
     "idx_decode_topk": (_i, [_vp, _vp, _ip, _fp, _i, _i, _i, _i, _i, _i, _i, _i, _i, _ip, _fp, _vp, _sz,
                              _vp]),
+    "idx_decode_paged_topk": (_i, [_vp, _vp, _ip, _ip, _fp, _i, _i, _i, _i, _ll, _i, _i, _i, _i, _i, _i, _ip,
+                                   _fp, _vp, _sz, _vp]),
     "idx_device_status": (_i, [_vp, _vp]),
     "idx_status_string": (ctypes.c_char_p, [_i]),
     "idx_debug_scores": (_i, [_i, _vp, _vp, _fp, _ip, _i, _i, _i, _i, _i, _i, _i, _i, _ip, _i, _fp, _ll,

@@ -346,6 +346,9 @@ struct Decode {
     char *ws;
     DecodeWs L;
     cudaStream_t st;
+    const int *bt = nullptr;  // paged cache: block table [B, max_pages], else NULL
+    int page = 0, max_pages = 0;
+    long long num_pages = 0;
 
     unsigned *status() const { return reinterpret_cast<unsigned *>(ws + L.status); }
 
@@ -359,11 +362,14 @@ struct Decode {
         a.chunk_tiles = 64;
         a.spill = spill;
         a.status = status();
+        a.bt = bt; a.page = page; a.max_pages = max_pages; a.num_pages = num_pages;
         return a;
     }
     cudaError_t scan(const DecodeArgs &a) const {
-        return tc_decode_supported(H, d, (int)dt, a.Gq) ? launch_decode_tc(a, st)
-                                                        : launch_decode_simt(a, (int)dt, st);
+        // the tensor-core scan loads a paged tile as 128 / page boxes; a box of
+        // fewer than 8 rows would break the 1 KB alignment of its swizzled slice
+        const bool tc = tc_decode_supported(H, d, (int)dt, a.Gq) && (!bt || page >= 8);
+        return tc ? launch_decode_tc(a, st) : launch_decode_simt(a, (int)dt, st);
     }
     SelectArgs sargs(int kind, int nrows, int kk, int *oi, float *os, const float *scores, long long ld) const {
         SelectArgs s{};
@@ -388,9 +394,31 @@ struct Decode {
         a.ckeys = ws + L.ckeys;
         a.c_pad = c_pad_of(c);
         a.status = status();
+        a.bt = bt; a.page = page; a.max_pages = max_pages; a.num_pages = num_pages;
         return a;
     }
+    idx_status run(int *out_idx, float *out_score) const;
 };
+
+idx_status Decode::run(int *out_idx, float *out_score) const {
+    TRY_CUDA(cudaMemsetAsync(status(), 0, 4, st));
+    float *spill = reinterpret_cast<float *>(ws + L.spill);
+    if (mode == IDX_MODE_DENSE) {
+        TRY_CUDA(scan(dargs(false, spill)));
+        return cuda_st(launch_select(sargs(SEL_DEC_DENSE, B * G, topk, out_idx, out_score, spill, n_max), st));
+    }
+    TRY_CUDA(launch_decode_proxy(q, w, B, G, H, d, (int)dt, ws + L.qbar, reinterpret_cast<float *>(ws + L.wbar), st));
+    TRY_CUDA(scan(dargs(true, spill)));
+    if (mode == IDX_MODE_REUSE)
+        return cuda_st(launch_select(sargs(SEL_DEC_REUSE, B * G, topk, out_idx, out_score, spill, n_max), st));
+    int *cand = reinterpret_cast<int *>(ws + L.cand);
+    TRY_CUDA(launch_select(sargs(SEL_DEC_PROXY_TO_C, B, c, cand, nullptr, spill, n_max), st));
+    const GatherArgs ga = gargs();
+    TRY_CUDA(tc_gather_supported(H, d, (int)dt, G, c) ? launch_gather_tc(ga, st)
+                                                     : launch_gather_simt(ga, (int)dt, st));
+    const float *msc = reinterpret_cast<const float *>(ws + L.msc);
+    return cuda_st(launch_select(sargs(SEL_DEC_MEMBER, B * G, topk, out_idx, out_score, msc, c), st));
+}
 
 idx_status check_decode(const void *q, const void *kc, const int *kv, const float *w, int B, int G, int n_max,
                         int H, int d, int topk, int c, idx_mode mode, idx_dtype dt, const int *out_idx,
@@ -416,24 +444,31 @@ idx_status idx_decode_topk(const void *q, const void *kcache, const int *kv_len,
     TracePhase phase(mode == IDX_MODE_DENSE ? "decode_dense" : mode == IDX_MODE_REUSE ? "decode_reuse" : "decode_refine");
     Decode D{q, kcache, kv_len, w, B, G, n_max, H, d, topk, c, mode, dtype, static_cast<char *>(ws),
              decode_ws(B, G, n_max, H, d, c, mode, dtype), reinterpret_cast<cudaStream_t>(stream)};
-    TRY_CUDA(cudaMemsetAsync(D.status(), 0, 4, D.st));
-    float *spill = reinterpret_cast<float *>(D.ws + D.L.spill);
-    if (mode == IDX_MODE_DENSE) {
-        TRY_CUDA(D.scan(D.dargs(false, spill)));
-        return cuda_st(launch_select(D.sargs(SEL_DEC_DENSE, B * G, topk, out_idx, out_score, spill, n_max), D.st));
-    }
-    TRY_CUDA(launch_decode_proxy(q, w, B, G, H, d, (int)dtype, D.ws + D.L.qbar,
-                                 reinterpret_cast<float *>(D.ws + D.L.wbar), D.st));
-    TRY_CUDA(D.scan(D.dargs(true, spill)));
-    if (mode == IDX_MODE_REUSE)
-        return cuda_st(launch_select(D.sargs(SEL_DEC_REUSE, B * G, topk, out_idx, out_score, spill, n_max), D.st));
-    int *cand = reinterpret_cast<int *>(D.ws + D.L.cand);
-    TRY_CUDA(launch_select(D.sargs(SEL_DEC_PROXY_TO_C, B, c, cand, nullptr, spill, n_max), D.st));
-    const GatherArgs ga = D.gargs();
-    TRY_CUDA(tc_gather_supported(H, d, (int)dtype, G, c) ? launch_gather_tc(ga, D.st)
-                                                       : launch_gather_simt(ga, (int)dtype, D.st));
-    const float *msc = reinterpret_cast<const float *>(D.ws + D.L.msc);
-    return cuda_st(launch_select(D.sargs(SEL_DEC_MEMBER, B * G, topk, out_idx, out_score, msc, c), D.st));
+    return D.run(out_idx, out_score);
+}
+
+idx_status idx_decode_paged_topk(const void *q, const void *kpool, const int *block_table, const int *kv_len,
+                                 const float *w, int B, int G, int max_pages, int page, long long num_pages, int H,
+                                 int d, int topk, int c, idx_mode mode, idx_dtype dtype, int *out_idx,
+                                 float *out_score, void *ws, size_t ws_bytes, idx_stream_t stream) {
+    if (!block_table || max_pages < 1 || page < 1 || num_pages < 1) return IDX_ERR_INVALID;
+    if ((long long)max_pages * page > kMaxLen) return IDX_ERR_UNSUPPORTED;
+    if (KT % page != 0 && page % KT != 0) return IDX_ERR_UNSUPPORTED;
+    if (num_pages > (long long)0x7FFFFFFF / page) return IDX_ERR_UNSUPPORTED;
+    const int n_max = max_pages * page;
+    idx_status s = check_decode(q, kpool, kv_len, w, B, G, n_max, H, d, topk, c, mode, dtype, out_idx, ws,
+                                ws_bytes);
+    if (s != IDX_OK) return s;
+    TracePhase phase(mode == IDX_MODE_DENSE ? "decode_paged_dense"
+                     : mode == IDX_MODE_REUSE ? "decode_paged_reuse"
+                                              : "decode_paged_refine");
+    Decode D{q, kpool, kv_len, w, B, G, n_max, H, d, topk, c, mode, dtype, static_cast<char *>(ws),
+             decode_ws(B, G, n_max, H, d, c, mode, dtype), reinterpret_cast<cudaStream_t>(stream)};
+    D.bt = block_table;
+    D.page = page;
+    D.max_pages = max_pages;
+    D.num_pages = num_pages;
+    return D.run(out_idx, out_score);
 }
 
 idx_status idx_device_status(const void *ws, idx_stream_t stream) {

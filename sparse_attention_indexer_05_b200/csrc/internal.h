@@ -66,6 +66,11 @@ struct DecodeArgs {
     float *spill;        // [B*Gq, n_max]
     unsigned *status;
     unsigned *work;
+    // paged cache (bt != NULL): kc is [num_pages, page, d]; position s of
+    // request b sits at row bt[b * max_pages + s / page] * page + s % page
+    const int *bt;
+    int page, max_pages;
+    long long num_pages;
 };
 
 // Refine re-score pass: member rows against the gathered candidate keys.
@@ -89,7 +94,23 @@ struct GatherArgs {
     void *ckeys;         // [groups, c_pad, d] packed candidate keys (tensor-core path)
     int c_pad;           // c rounded up to a multiple of 128
     unsigned *status;
+    const int *bt;       // decode: paged cache, as in DecodeArgs
+    int page, max_pages;
+    long long num_pages;
 };
+
+// Row of the key cache holding position s of request b: contiguous
+// [B, n_max, d] when bt is NULL, else paged through the block table (an
+// entry outside [0, num_pages) reads row 0; positions past the request are
+// masked by the callers).
+__host__ __device__ inline long long cache_row(const int *bt, int page, int max_pages, long long num_pages,
+                                               long long n_max, int b, int s) {
+    if (!bt) return (long long)b * n_max + s;
+    const int j = s / page;
+    long long pg = j < max_pages ? bt[(long long)b * max_pages + j] : 0;
+    if (pg < 0 || pg >= num_pages) pg = 0;
+    return pg * page + s % page;
+}
 
 // select pass descriptors
 enum SelKind {

@@ -323,9 +323,9 @@ __device__ void block_select(const Src &src, int k, int *out_idx, float *out_sco
                              unsigned long long *stage, int stage_cap, unsigned *bm, unsigned *gpre, int wcap,
                              unsigned *status) {
     const int tid = threadIdx.x, nt = blockDim.x, lane = tid & 31;
-    if constexpr (Src::kFloor) {
-        // candidate rows: the entries at or above the row's floor are about
-        // k plus a bin's worth; one pass stages them all
+    if (Src::kFloor || src.n <= stage_cap) {
+        // candidate rows (the entries at or above the row's floor are about
+        // k plus a bin's worth) and short rows: one pass stages them all
         const unsigned ns = stage_keys(src, sh, 1ull, stage, stage_cap);
         if (ns <= (unsigned)stage_cap) {
             const StageSrc ss{stage, (int)ns, src.bound};

@@ -161,7 +161,7 @@ __global__ void __launch_bounds__(kSimtThreads) decode_simt_kernel(DecodeArgs a,
     const int kv = a.kv_len[b];
     if (kv < a.G || kv > a.n_max) return;  // the select pass flags the request
     const T *q = reinterpret_cast<const T *>(a.q) + (long long)b * a.Gq * HD;
-    const T *kc = reinterpret_cast<const T *>(a.kc) + (long long)b * a.n_max * a.d;
+    const T *kc = reinterpret_cast<const T *>(a.kc);
     load_rows(qs, q, a.Gq, HD);
     for (int i = threadIdx.x; i < RB * a.H; i += blockDim.x)
         wsm[i] = (i / a.H) < a.Gq ? a.w[(long long)b * a.Gq * a.H + i] : 0.0f;
@@ -177,7 +177,12 @@ __global__ void __launch_bounds__(kSimtThreads) decode_simt_kernel(DecodeArgs a,
         const int s0 = tile * KT;
         int nvk = kv - s0;
         nvk = nvk > KT ? KT : nvk;
-        load_keys(ks, kc + (long long)s0 * a.d, nvk, a.d);
+        for (int idx = threadIdx.x; idx < KT * a.d; idx += blockDim.x) {
+            const int i = idx / a.d, e = idx - i * a.d;
+            ks[i * (a.d + 1) + e] =
+                i < nvk ? to_f(kc[cache_row(a.bt, a.page, a.max_pages, a.num_pages, a.n_max, b, s0 + i) * a.d + e])
+                        : 0.0f;
+        }
         __syncthreads();
         if (row_ok && s0 <= bound) {
             float sc[4];
@@ -239,7 +244,9 @@ __global__ void __launch_bounds__(kSimtThreads) gather_simt_kernel(GatherArgs a,
         for (int idx = threadIdx.x; idx < KT * a.d; idx += blockDim.x) {
             const int i = idx / a.d, e = idx - i * a.d;
             const int p = s_pos[i];
-            ks[i * (a.d + 1) + e] = p >= 0 ? to_f(k[(key0 + p) * a.d + e]) : 0.0f;
+            const long long row = a.mode == 0 ? key0 + p
+                                              : cache_row(a.bt, a.page, a.max_pages, a.num_pages, a.n_max, grp, p);
+            ks[i * (a.d + 1) + e] = p >= 0 ? to_f(k[row * a.d + e]) : 0.0f;
         }
         __syncthreads();
         if (r < nmem) {

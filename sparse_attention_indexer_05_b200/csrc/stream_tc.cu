@@ -227,8 +227,23 @@ __global__ void __launch_bounds__(kThreads, 1)
                 uint8_t *dst = as + st * kAStage;
                 if (lane == 0) {
                     tc::mbar_arrive_expect_tx(&sh.afull[st], kAStage);
-                    const int row = (int)(it.key0 + (long long)(it.t0 + j) * KT);
-                    for (int kh = 0; kh < 2; ++kh) tc::tma_load_2d(dst + kh * kASlice, &tmap_k, kh * 64, row, &sh.afull[st]);
+                    if (GATHER || !dd.bt) {
+                        const int row = (int)(it.key0 + (long long)(it.t0 + j) * KT);
+                        for (int kh = 0; kh < 2; ++kh)
+                            tc::tma_load_2d(dst + kh * kASlice, &tmap_k, kh * 64, row, &sh.afull[st]);
+                    } else {
+                        // paged cache: the tile's 128 positions span 128 / box pages (box = min(page, 128))
+                        const int box = dd.page < KT ? dd.page : KT;
+                        const int s0 = (it.t0 + j) * KT;
+                        const int b = (int)(it.qrow0 / dd.Gq);
+                        for (int i = 0; i < KT / box; ++i) {
+                            const int row =
+                                (int)cache_row(dd.bt, dd.page, dd.max_pages, dd.num_pages, dd.n_max, b, s0 + i * box);
+                            for (int kh = 0; kh < 2; ++kh)
+                                tc::tma_load_2d(dst + kh * kASlice + i * box * 128, &tmap_k, kh * 64, row,
+                                                &sh.afull[st]);
+                        }
+                    }
                 }
             }
         } else if (warp == 1) {
@@ -330,7 +345,7 @@ __global__ void __launch_bounds__(256) compact_keys_kernel(GatherArgs a) {
     } else {
         const int kv = a.kv_len[grp];
         if (kv < a.G || kv > a.n_max) return;
-        key0 = (long long)grp * a.n_max;
+        key0 = -1;  // decode: rows through cache_row
     }
     const int *cand = a.cand + (long long)grp * a.c;
     const int per_row = a.d * 2 / 16;  // 16-byte chunks per key row
@@ -340,7 +355,10 @@ __global__ void __launch_bounds__(256) compact_keys_kernel(GatherArgs a) {
         const int r = u / per_row, part = u - r * per_row;
         const int j = j0 + r;
         const int pos = j < a.c ? cand[j] : -1;
-        dst[u] = src[(key0 + (pos >= 0 ? pos : 0)) * per_row + part];
+        const int p = pos >= 0 ? pos : 0;
+        const long long row =
+            key0 >= 0 ? key0 + p : cache_row(a.bt, a.page, a.max_pages, a.num_pages, a.n_max, grp, p);
+        dst[u] = src[row * per_row + part];
     }
 }
 
@@ -391,8 +409,9 @@ bool tc_gather_supported(int H, int d, int dtype, int group, int c) {
 
 cudaError_t launch_decode_tc(const DecodeArgs &a, cudaStream_t st) {
     CUtensorMap mq, mk;
-    if (!map2d(&mq, a.q, (unsigned long long)a.B * a.Gq * S_H, 256) ||
-        !map2d(&mk, a.kc, (unsigned long long)a.B * a.n_max, KT))
+    const unsigned long long krows = a.bt ? (unsigned long long)a.num_pages * a.page : (unsigned long long)a.B * a.n_max;
+    const unsigned box = a.bt && a.page < KT ? (unsigned)a.page : (unsigned)KT;
+    if (!map2d(&mq, a.q, (unsigned long long)a.B * a.Gq * S_H, 256) || !map2d(&mk, a.kc, krows, box))
         return cudaErrorInvalidValue;
     const int ntiles_max = (a.n_max + KT - 1) / KT;
     const int nitems = a.B * ((ntiles_max + kDecodeChunkTiles - 1) / kDecodeChunkTiles);

@@ -8,6 +8,7 @@ Entry points (names follow the C ABI):
     dense_topk(q, k, w, cu_seqlens, topk)               -> idx [T, topk]
     pivot_topk(q, k, w, cu_seqlens, topk, g, c, mode)   -> idx [T, topk]
     decode_topk(q, kcache, kv_len, w, topk, c, mode)    -> idx [B, G, topk]
+    decode_paged_topk(q, kpool, block_table, kv_len, w, topk, c, mode)  -> idx [B, G, topk]
 Each accepts out_idx / out_score / workspace to reuse buffers, and
 return_scores=True to also get the selected scores.
 """
@@ -132,6 +133,28 @@ def decode_topk(q, kcache, kv_len, w, topk: int, c: int = 0, mode="dense", out_i
         _dev(w, "w", torch.float32), B, G, n_max, H, d, topk, c, m, dt, _dev(out_idx, "out_idx", torch.int32),
         _dev(out_score, "out_score", torch.float32) if out_score is not None else None,
         ws.data_ptr(), ws.numel(), _stream(stream)), "idx_decode_topk")
+    return (out_idx, out_score) if return_scores else out_idx
+
+
+def decode_paged_topk(q, kpool, block_table, kv_len, w, topk: int, c: int = 0, mode="dense", out_idx=None,
+                      out_score=None, workspace=None, stream=None, return_scores=False):
+    """One decode step over a paged cache: q [B,G,H,d], kpool [num_pages,page,d],
+    block_table int32 [B,max_pages], kv_len int32 [B], w [B,G,H]."""
+    B, G, H, d = q.shape
+    num_pages, page = kpool.shape[0], kpool.shape[1]
+    max_pages = block_table.shape[1]
+    if block_table.shape[0] != B:
+        raise ValueError("block_table must have one row per request")
+    dt = _dtype_code(q)
+    m = _mode(mode)
+    ws = _ws(workspace, decode_workspace_size(B, G, max_pages * page, H, d, topk, c, m, q.dtype), q.device)
+    out_idx, out_score = _outs((B, G), topk, q.device, out_idx, out_score, return_scores)
+    N.check(N.lib().idx_decode_paged_topk(
+        _dev(q, "q"), _dev(kpool, "kpool", q.dtype), _dev(block_table, "block_table", torch.int32),
+        _dev(kv_len, "kv_len", torch.int32), _dev(w, "w", torch.float32), B, G, max_pages, page, num_pages, H, d,
+        topk, c, m, dt, _dev(out_idx, "out_idx", torch.int32),
+        _dev(out_score, "out_score", torch.float32) if out_score is not None else None,
+        ws.data_ptr(), ws.numel(), _stream(stream)), "idx_decode_paged_topk")
     return (out_idx, out_score) if return_scores else out_idx
 
 

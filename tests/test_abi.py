@@ -26,7 +26,7 @@ def declared_functions():
 
 def test_exports_every_declared_symbol(lib):
     names = declared_functions()
-    assert len(names) == 15
+    assert len(names) == 16
     for n in names:
         assert hasattr(lib, n), n
         assert n in N.SIGNATURES, n
@@ -72,6 +72,14 @@ def test_invalid_arguments_return_before_launch(lib):
     # decode: refine with c < k
     assert lib.idx_decode_topk(fake, fake, fake, fake, 2, 2, 64, 4, 64, 8, 4, 2, 0, fake, None, fake, 1 << 30,
                                None) == 1
+    # paged decode: no block table / a page size that neither divides 128 nor is a multiple of it /
+    # a logical cache longer than 2^20
+    assert lib.idx_decode_paged_topk(fake, fake, None, fake, fake, 2, 2, 4, 16, 8, 4, 64, 8, 0, 0, 0, fake, None,
+                                     fake, 1 << 30, None) == 1
+    assert lib.idx_decode_paged_topk(fake, fake, fake, fake, fake, 2, 2, 4, 48, 8, 4, 64, 8, 0, 0, 0, fake, None,
+                                     fake, 1 << 30, None) == 2
+    assert lib.idx_decode_paged_topk(fake, fake, fake, fake, fake, 2, 2, 8193, 128, 8, 4, 64, 8, 0, 0, 0, fake,
+                                     None, fake, 1 << 30, None) == 2
     # shape that fits neither kernel family
     assert lib.idx_dense_topk(fake, fake, fake, fake, 1, 10, 256, 256, 8, 1, fake, None, fake, 1 << 40,
                               None) == 2
