@@ -19,7 +19,7 @@ import numpy as np
 from . import build as _build
 
 BF16, F32 = 0, 1
-DENSE, REUSE, REFINE = 0, 1, 2
+DENSE, REUSE, REFINE, BLOCK = 0, 1, 2, 3
 
 _libs = {}
 _active = [None]
@@ -37,9 +37,10 @@ def load(path: str) -> ctypes.CDLL:
         L.ora_select.argtypes = [dp, ip, i, i, ip]
         L.ora_group_proxy.argtypes = [vp, fp, i, i, i, ll, i, vp, fp]
         L.ora_dense_topk.argtypes = [vp, vp, fp, i, ip, i, i, i, i, llp, i, ip, i]
-        L.ora_pivot_topk.argtypes = [vp, vp, fp, i, ip, i, i, i, i, i, i, i, llp, i, ip, i]
-        L.ora_decode_topk.argtypes = [vp, vp, fp, i, ip, i, i, i, i, i, i, i, i, llp, i, ip, i]
-        for f in (L.ora_score_row, L.ora_select, L.ora_group_proxy, L.ora_dense_topk,
+        L.ora_block_mean.argtypes = [vp, i, i, ll, i, vp]
+        L.ora_pivot_topk.argtypes = [vp, vp, fp, i, ip, i, i, i, i, i, i, i, i, llp, i, ip, i]
+        L.ora_decode_topk.argtypes = [vp, vp, fp, i, ip, i, i, i, i, i, i, i, i, i, llp, i, ip, i]
+        for f in (L.ora_score_row, L.ora_select, L.ora_group_proxy, L.ora_block_mean, L.ora_dense_topk,
                   L.ora_pivot_topk, L.ora_decode_topk):
             f.restype = ctypes.c_int
         _libs[path] = L
@@ -128,6 +129,16 @@ def group_proxy(q, w, m0: int, cnt: int):
     return qbar, wbar
 
 
+def block_mean(k, r0: int, bn: int):
+    """Mean key [d] (in k's dtype) of key rows r0 .. r0+bn-1 of k [*, d]."""
+    k = np.ascontiguousarray(k)
+    dt = _dtype_code(k)
+    d = k.shape[1]
+    out = np.empty(d, k.dtype)
+    _check(lib().ora_block_mean(_ptr(k), dt, d, r0, bn, _ptr(out)), "block_mean")
+    return out
+
+
 def _rows(rows, total):
     if rows is None:
         rows = np.arange(total, dtype=np.int64)
@@ -149,8 +160,9 @@ def dense_topk(q, k, w, cu_seqlens, topk: int, rows=None, threads=None) -> np.nd
 
 
 def pivot_topk(q, k, w, cu_seqlens, topk: int, g: int, c: int, mode: int, rows=None,
-               threads=None) -> np.ndarray:
-    """PIVOT Reuse (mode=REUSE) or Refine (mode=REFINE) top-k of member rows."""
+               threads=None, bn: int = 64) -> np.ndarray:
+    """PIVOT Reuse (mode=REUSE), Refine (mode=REFINE) or Refine over block
+    pre-filter candidates (mode=BLOCK, block size bn) top-k of member rows."""
     q = np.ascontiguousarray(q); k = np.ascontiguousarray(k); w = _c(w, np.float32)
     cu = _c(cu_seqlens, np.int32)
     dt = _dtype_code(q)
@@ -158,13 +170,13 @@ def pivot_topk(q, k, w, cu_seqlens, topk: int, g: int, c: int, mode: int, rows=N
     r = _rows(rows, T)
     out = np.empty((len(r), topk), np.int32)
     _check(lib().ora_pivot_topk(_ptr(q), _ptr(k), _ptr(w, ctypes.c_float), dt, _ptr(cu, ctypes.c_int),
-                                len(cu) - 1, H, d, topk, g, c, mode, _ptr(r, ctypes.c_longlong),
+                                len(cu) - 1, H, d, topk, g, c, mode, bn, _ptr(r, ctypes.c_longlong),
                                 len(r), _ptr(out, ctypes.c_int), _threads(threads)), "pivot_topk")
     return out
 
 
 def decode_topk(q, kcache, w, kv_len, topk: int, c: int = 0, mode: int = DENSE, reqs=None,
-                threads=None) -> np.ndarray:
+                threads=None, bn: int = 64) -> np.ndarray:
     """Decode top-k: q [B,G,H,d], kcache [B,n_max,d], w [B,G,H] -> [nreqs,G,topk]."""
     q = np.ascontiguousarray(q); kc = np.ascontiguousarray(kcache); w = _c(w, np.float32)
     kv = _c(kv_len, np.int32)
@@ -174,6 +186,6 @@ def decode_topk(q, kcache, w, kv_len, topk: int, c: int = 0, mode: int = DENSE, 
     r = _rows(reqs, B)
     out = np.empty((len(r), G, topk), np.int32)
     _check(lib().ora_decode_topk(_ptr(q), _ptr(kc), _ptr(w, ctypes.c_float), dt, _ptr(kv, ctypes.c_int),
-                                 B, G, n_max, H, d, topk, c, mode, _ptr(r, ctypes.c_longlong), len(r),
+                                 B, G, n_max, H, d, topk, c, mode, bn, _ptr(r, ctypes.c_longlong), len(r),
                                  _ptr(out, ctypes.c_int), _threads(threads)), "decode_topk")
     return out

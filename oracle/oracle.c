@@ -29,6 +29,20 @@
  *        then PIVOT-Refine re-scores it with each member's own indexer.
  *      Method, decode paragraph: the decode group is the current query plus
  *        the MTP draft queries of the same step.
+ *  - Block pre-filter (mode ORA_BLOCK), a candidate generator for Refine built
+ *    from two other pages: "Not All Tokens Deserve Equal Resolution:
+ *    Score-Adaptive Indexing for Sparse Attention in Long-Context LLMs"
+ *    (abstract: coarse summaries of key chunks are scored first, then the
+ *    tokens of the chosen chunks are refined exactly) and "Uncertainty-gated
+ *    selection for block-sparse attention" (Sec. 3.1, step 1: a block is
+ *    summarised by the mean of its keys, block size 64).  Readings: the
+ *    block score is the indexer score of the group proxy against the block's
+ *    mean key; only complete blocks inside the group's prefix are scored, so
+ *    no key after the group's last member takes part; the partial block that
+ *    holds the last member is always a candidate; the candidate budget c
+ *    counts tokens (c / bn blocks, one of them the partial block if there
+ *    is one); the mean key is rounded like the proxy (fp32 sum in key order,
+ *    IEEE division, bf16 round-to-nearest-even).
  *  - Readings where the pages are silent (each also listed in the design
  *    notes): proxy of w = mean of w; proxy arithmetic = fp32 sum in member
  *    order, IEEE division, then round-to-nearest-even to bf16 for bf16
@@ -49,7 +63,7 @@
 #include <string.h>
 
 enum { ORA_BF16 = 0, ORA_F32 = 1 };
-enum { ORA_DENSE = 0, ORA_REUSE = 1, ORA_REFINE = 2 };
+enum { ORA_DENSE = 0, ORA_REUSE = 1, ORA_REFINE = 2, ORA_BLOCK = 3 };
 
 /* ---------------------------------------------------------------- inputs */
 
@@ -180,6 +194,26 @@ static void group_proxy(const void *q, const float *w, int dtype, int H, int d,
     }
 }
 
+/* Mean key of the bn keys at rows r0 .. r0+bn-1 of k [*, d]: per dimension
+ * the fp32 sum in key order, divided by bn (IEEE fp32), rounded to bf16 for
+ * bf16 keys.  kbar receives d elements in dtype format. */
+static void block_mean(const void *k, int dtype, int d, long long r0, int bn, void *kbar) {
+    for (int i = 0; i < d; ++i) {
+        float sum = 0.0f;
+        for (int r = 0; r < bn; ++r) sum = sum + (float)load_elem(k, dtype, (size_t)(r0 + r) * d + i);
+        float mean = sum / (float)bn;
+        if (dtype == ORA_BF16) ((uint16_t *)kbar)[i] = float_to_bf16_rne(mean);
+        else ((float *)kbar)[i] = mean;
+    }
+}
+
+/* Exported for tests of the block-mean step alone. */
+int ora_block_mean(const void *k, int dtype, int d, long long r0, int bn, void *kbar) {
+    if (!k || !kbar || bn <= 0 || d <= 0) return 1;
+    block_mean(k, dtype, d, r0, bn, kbar);
+    return 0;
+}
+
 /* Exported for tests of the proxy step alone. */
 int ora_group_proxy(const void *q, const float *w, int dtype, int H, int d, long long m0, int cnt,
                     void *qbar, float *wbar) {
@@ -193,11 +227,12 @@ int ora_group_proxy(const void *q, const float *w, int dtype, int H, int d, long
  *         are pos0 .. pos0+cnt-1 (request-local); the group's last member
  *         sits at t_last = pos0+cnt-1.
  *   keys: key rows key0 + s for s = 0 .. t_last.
- *   mode: ORA_REUSE or ORA_REFINE; c: candidate budget (Refine).
+ *   mode: ORA_REUSE, ORA_REFINE or ORA_BLOCK; c: candidate budget (Refine,
+ *         Block); bn: block size (Block).
  *   member: which member (0..cnt-1) to produce; out: k entries. */
 static int grouped_member_topk(const void *q, const void *k, const float *w, int dtype, int H, int d,
                                long long m0, int cnt, int pos0, long long key0, int topk, int c,
-                               int mode, int member, int *out) {
+                               int mode, int bn, int member, int *out) {
     int t_last = pos0 + cnt - 1;
     int n = t_last + 1;
     size_t esz = dtype == ORA_BF16 ? 2 : 4;
@@ -206,13 +241,54 @@ static int grouped_member_topk(const void *q, const void *k, const float *w, int
     cand_t *pc = (cand_t *)malloc(sizeof(cand_t) * (size_t)n);
     if (!qbar || !wbar || !pc) { free(qbar); free(wbar); free(pc); return 2; }
     group_proxy(q, w, dtype, H, d, m0, cnt, qbar, wbar);
+    int t = pos0 + member;
+    int rc = 0;
+    if (mode == ORA_BLOCK) {
+        /* complete blocks [j*bn, (j+1)*bn) inside the prefix, scored by the
+         * proxy against their mean keys; the partial block [part0, n) */
+        int nfull = n / bn;
+        int part0 = nfull * bn;
+        int want = c / bn - (part0 < n ? 1 : 0);
+        int take = want < nfull ? want : nfull;
+        if (take < 0) take = 0;
+        void *kbar = malloc(esz * (size_t)d);
+        /* C holds distinct positions of the prefix: at most n entries */
+        cand_t *mc = (cand_t *)malloc(sizeof(cand_t) * (size_t)n);
+        if (!kbar || !mc) { free(kbar); free(mc); rc = 2; goto done; }
+        for (int j = 0; j < nfull; ++j) {
+            block_mean(k, dtype, d, key0 + (long long)j * bn, bn, kbar);
+            pc[j].score = index_score(qbar, 0, kbar, 0, wbar, H, d, dtype);
+            pc[j].pos = j;
+        }
+        qsort(pc, (size_t)nfull, sizeof(cand_t), by_score_desc_pos_asc);
+        /* C = tokens of the top `take` blocks and of the partial block; the
+         * member re-scores those inside its own prefix */
+        int m = 0;
+        for (int i = 0; i < take; ++i)
+            for (int r = 0; r < bn; ++r) {
+                int s = pc[i].pos * bn + r;
+                if (s > t) continue;
+                mc[m].score = index_score(q, (size_t)(m0 + member) * H * d, k, (size_t)(key0 + s) * d,
+                                          w + (size_t)(m0 + member) * H, H, d, dtype);
+                mc[m].pos = s;
+                ++m;
+            }
+        for (int s = part0; s < n && s <= t; ++s) {
+            mc[m].score = index_score(q, (size_t)(m0 + member) * H * d, k, (size_t)(key0 + s) * d,
+                                      w + (size_t)(m0 + member) * H, H, d, dtype);
+            mc[m].pos = s;
+            ++m;
+        }
+        select_topk(mc, m, topk, out);
+        free(mc);
+        free(kbar);
+        goto done;
+    }
     /* one shared scan of the group's full prefix with the proxy */
     for (int s = 0; s < n; ++s) {
         pc[s].score = index_score(qbar, 0, k, (size_t)(key0 + s) * d, wbar, H, d, dtype);
         pc[s].pos = s;
     }
-    int t = pos0 + member;
-    int rc = 0;
     if (mode == ORA_REUSE) {
         /* the proxy ranking, restricted to the member's own prefix */
         select_topk(pc, t + 1, topk, out);
@@ -247,7 +323,7 @@ typedef struct {
     int kind; /* 0 dense, 1 pivot, 2 decode */
     const void *q, *k;
     const float *w;
-    int dtype, H, d, topk, g, c, mode;
+    int dtype, H, d, topk, g, c, mode, bn;
     const int *cu;
     int num_seqs;
     const long long *rows;
@@ -298,7 +374,7 @@ static void run_pivot_row(job_t *J, int i) {
     int lo = (t / J->g) * J->g;
     int hi = lo + J->g < n ? lo + J->g : n;
     set_rc(J, grouped_member_topk(J->q, J->k, J->w, J->dtype, J->H, J->d, J->cu[b] + lo, hi - lo, lo,
-                                  J->cu[b], J->topk, J->c, J->mode, t - lo,
+                                  J->cu[b], J->topk, J->c, J->mode, J->bn, t - lo,
                                   J->out + (size_t)i * J->topk));
 }
 
@@ -326,7 +402,7 @@ static void run_decode_req(job_t *J, int i) {
     } else {
         for (int m = 0; m < G; ++m)
             set_rc(J, grouped_member_topk(J->q, J->k, J->w, J->dtype, H, d, m0, G, n - G, key0,
-                                          J->topk, J->c, J->mode, m, out + (size_t)m * J->topk));
+                                          J->topk, J->c, J->mode, J->bn, m, out + (size_t)m * J->topk));
     }
 }
 
@@ -382,22 +458,24 @@ int ora_dense_topk(const void *q, const void *k, const float *w, int dtype, cons
     return run_job(&J, nthreads);
 }
 
-/* PIVOT top-k (mode ORA_REUSE or ORA_REFINE) for the given global member
- * rows; same layouts as ora_dense_topk; g >= 1; Refine needs c >= topk. */
+/* PIVOT top-k (mode ORA_REUSE, ORA_REFINE or ORA_BLOCK) for the given
+ * global member rows; same layouts as ora_dense_topk; g >= 1; Refine and
+ * Block need c >= topk; Block needs bn >= 1 (c / bn blocks). */
 int ora_pivot_topk(const void *q, const void *k, const float *w, int dtype, const int *cu_seqlens,
-                   int num_seqs, int H, int d, int topk, int g, int c, int mode,
+                   int num_seqs, int H, int d, int topk, int g, int c, int mode, int bn,
                    const long long *rows, int nrows, int *out, int nthreads) {
     if (!q || !k || !w || !out || (nrows > 0 && !rows) || H <= 0 || d <= 0 || topk <= 0 || g <= 0)
         return 1;
-    if (mode != ORA_REUSE && mode != ORA_REFINE) return 1;
-    if (mode == ORA_REFINE && c < topk) return 1;
+    if (mode != ORA_REUSE && mode != ORA_REFINE && mode != ORA_BLOCK) return 1;
+    if ((mode == ORA_REFINE || mode == ORA_BLOCK) && c < topk) return 1;
+    if (mode == ORA_BLOCK && bn < 1) return 1;
     if (check_requests(cu_seqlens, num_seqs)) return 1;
     for (int i = 0; i < nrows; ++i)
         if (rows[i] < 0 || rows[i] >= cu_seqlens[num_seqs]) return 1;
     job_t J;
     memset(&J, 0, sizeof J);
     J.kind = 1; J.q = q; J.k = k; J.w = w; J.dtype = dtype; J.H = H; J.d = d; J.topk = topk;
-    J.g = g; J.c = c; J.mode = mode; J.cu = cu_seqlens; J.num_seqs = num_seqs; J.rows = rows;
+    J.g = g; J.c = c; J.mode = mode; J.bn = bn; J.cu = cu_seqlens; J.num_seqs = num_seqs; J.rows = rows;
     J.nrows = nrows; J.out = out;
     return run_job(&J, nthreads);
 }
@@ -406,15 +484,17 @@ int ora_pivot_topk(const void *q, const void *k, const float *w, int dtype, cons
  * q [B,G,H,d], kcache [B,n_max,d], w [B,G,H]; kv_len host [B] with
  * G <= kv_len[b] <= n_max; query m of request b sits at position
  * kv_len[b]-G+m and the cache already holds the keys of the group.
- * mode ORA_DENSE, ORA_REUSE or ORA_REFINE (c >= topk); out [nreqs,G,topk]. */
+ * mode ORA_DENSE, ORA_REUSE, ORA_REFINE (c >= topk) or ORA_BLOCK (c >= topk,
+ * bn >= 1); out [nreqs,G,topk]. */
 int ora_decode_topk(const void *q, const void *kcache, const float *w, int dtype, const int *kv_len,
-                    int B, int G, int n_max, int H, int d, int topk, int c, int mode,
+                    int B, int G, int n_max, int H, int d, int topk, int c, int mode, int bn,
                     const long long *reqs, int nreqs, int *out, int nthreads) {
     if (!q || !kcache || !w || !kv_len || !out || (nreqs > 0 && !reqs) || H <= 0 || d <= 0 ||
         topk <= 0 || G <= 0)
         return 1;
-    if (mode != ORA_DENSE && mode != ORA_REUSE && mode != ORA_REFINE) return 1;
-    if (mode == ORA_REFINE && c < topk) return 1;
+    if (mode != ORA_DENSE && mode != ORA_REUSE && mode != ORA_REFINE && mode != ORA_BLOCK) return 1;
+    if ((mode == ORA_REFINE || mode == ORA_BLOCK) && c < topk) return 1;
+    if (mode == ORA_BLOCK && bn < 1) return 1;
     for (int i = 0; i < nreqs; ++i) {
         if (reqs[i] < 0 || reqs[i] >= B) return 1;
         int n = kv_len[reqs[i]];
@@ -423,7 +503,7 @@ int ora_decode_topk(const void *q, const void *kcache, const float *w, int dtype
     job_t J;
     memset(&J, 0, sizeof J);
     J.kind = 2; J.q = q; J.k = kcache; J.w = w; J.dtype = dtype; J.H = H; J.d = d; J.topk = topk;
-    J.c = c; J.mode = mode; J.kv_len = kv_len; J.G = G; J.n_max = n_max; J.rows = reqs;
+    J.c = c; J.mode = mode; J.bn = bn; J.kv_len = kv_len; J.G = G; J.n_max = n_max; J.rows = reqs;
     J.nrows = nreqs; J.out = out;
     return run_job(&J, nthreads);
 }

@@ -301,8 +301,8 @@ def pin_decode_matches_prefill():
     qd = _bf(rng.standard_normal((B, G, H, d)))
     wd = rng.random((B, G, H)).astype(np.float32)
     for mode, c, kv in ((O.DENSE, 0, np.array([40, 23, 3], np.int32)), (O.REUSE, 6, kv),
-                        (O.REFINE, 6, kv)):
-        got = O.decode_topk(qd, kc, wd, kv, 5, c, mode)
+                        (O.REFINE, 6, kv), (O.BLOCK, 8, kv)):
+        got = O.decode_topk(qd, kc, wd, kv, 5, c, mode, bn=4)
         for b in range(B):
             n = kv[b]
             # prefill request of length n whose last G rows are the decode queries;
@@ -317,8 +317,75 @@ def pin_decode_matches_prefill():
                 want = O.dense_topk(q, kc[b, :n], w, cu, 5, rows=rows)
             else:
                 assert (n - G) % G == 0
-                want = O.pivot_topk(q, kc[b, :n], w, cu, 5, G, c, mode, rows=rows)
+                want = O.pivot_topk(q, kc[b, :n], w, cu, 5, G, c, mode, rows=rows, bn=4)
             assert np.array_equal(got[b], want), (mode, b)
+
+
+def pin_block_mean_exact():
+    """The mean key of a block whose fp32 sum is exact is the exact mean rounded
+    once to bf16 (nearest, ties to even); only rows r0 .. r0+bn-1 count."""
+    rng = np.random.default_rng(29)
+    for bn in (1, 2, 4, 64):
+        vals = rng.integers(-255, 256, size=(bn + 3, 8)).astype(np.float32) / np.float32(64)
+        k = _bf(vals)
+        got = O.block_mean(k, 2, bn)
+        for i in range(8):
+            exact = sum(Fraction(float(v)) for v in vals[2:2 + bn, i]) / bn
+            assert Fraction(float(W.bf16_to_f32(got[i:i + 1])[0])) == _round_bf16(exact), (bn, i)
+    # (1 + 2^-8) / 2 lies halfway between two bf16 values: even wins -> 0.5;
+    # (1 + 3 * 2^-8) / 2 likewise -> 0.5 + 2^-7
+    k = _bf(np.array([[1.0, 1.0], [2.0 ** -8, 3 * 2.0 ** -8]], np.float32))
+    got = W.bf16_to_f32(O.block_mean(k, 0, 2))
+    assert got.tolist() == [0.5, 0.5 + 2.0 ** -7]
+
+
+def pin_block_reductions():
+    """Block pre-filter: block size 1 is Refine; a budget covering the prefix is dense."""
+    P = W.prefill([37, 20], H=4, d=32, topk=5, rho=0.9, planted=0.1, seed=31)
+    cu = P.cu_seqlens
+    for g, c in ((2, 8), (4, 6), (3, 5)):
+        a = O.pivot_topk(P.q, P.k, P.w, cu, 5, g, c, O.BLOCK, bn=1)
+        b = O.pivot_topk(P.q, P.k, P.w, cu, 5, g, c, O.REFINE)
+        assert np.array_equal(a, b), ("block size 1 must equal Refine", g, c)
+    dense = O.dense_topk(P.q, P.k, P.w, cu, 5)
+    for g, bn in ((2, 4), (4, 8), (3, 16)):
+        a = O.pivot_topk(P.q, P.k, P.w, cu, 5, g, 64, O.BLOCK, bn=bn)
+        assert np.array_equal(a, dense), ("a budget covering the prefix must equal dense", g, bn)
+
+
+def pin_block_constant_keys_equal_refine():
+    """Keys constant inside each block: a block's mean is its key, so the block
+    ranking is the token ranking; with groups ending on block boundaries the
+    block pre-filter keeps exactly Refine's candidate set (c a multiple of bn)."""
+    rng = np.random.default_rng(37)
+    L, H, d, bn = 48, 4, 16, 4
+    kb = rng.integers(-8, 9, size=(L // bn, d)).astype(np.float32)
+    k = _bf(np.repeat(kb, bn, axis=0))
+    q = _bf(rng.integers(-8, 9, size=(L, H, d)).astype(np.float32))
+    w = (rng.integers(0, 5, size=(L, H)) / 4).astype(np.float32)
+    cu = np.array([0, L], np.int32)
+    for c in (8, 12, 20):
+        a = O.pivot_topk(q, k, w, cu, 6, 4, c, O.BLOCK, bn=bn)
+        b = O.pivot_topk(q, k, w, cu, 6, 4, c, O.REFINE)
+        assert np.array_equal(a, b), c
+
+
+def pin_block_partial_closed_form():
+    """A budget of one block and a group ending inside a block: the candidate
+    set is the partial block, so member t gets positions part0 .. t."""
+    P = W.prefill([30], H=4, d=16, topk=8, rho=0.9, planted=0.1, seed=41)
+    bn, g = 8, 3
+    got = O.pivot_topk(P.q, P.k, P.w, P.cu_seqlens, 8, g, bn, O.BLOCK, bn=bn)
+    checked = 0
+    for t in range(30):
+        t_last = min((t // g) * g + g, 30) - 1
+        if (t_last + 1) % bn == 0:
+            continue
+        part0 = ((t_last + 1) // bn) * bn
+        want = list(range(part0, t + 1))
+        assert got[t].tolist() == want + [-1] * (8 - len(want)), t
+        checked += 1
+    assert checked > 20
 
 
 def pin_gaussian_mean_score():
@@ -339,7 +406,9 @@ def pin_gaussian_mean_score():
 ALL_PINS = [pin_hand_scores, pin_hand_topk, pin_hand_decode, pin_bruteforce_dense,
             pin_bruteforce_pivot, pin_exact_integer_inputs, pin_textbook_single_head,
             pin_pivot_special_cases, pin_invariants, pin_reuse_within_proxy_ranking,
-            pin_proxy_exact_mean, pin_decode_matches_prefill, pin_gaussian_mean_score]
+            pin_proxy_exact_mean, pin_decode_matches_prefill, pin_gaussian_mean_score,
+            pin_block_mean_exact, pin_block_reductions, pin_block_constant_keys_equal_refine,
+            pin_block_partial_closed_form]
 
 
 @pytest.mark.parametrize("pin", ALL_PINS, ids=[p.__name__ for p in ALL_PINS])
@@ -365,6 +434,13 @@ MUTANTS = {
     "pad_with_zero": ("for (int i = m; i < k; ++i) out[i] = -1;", "for (int i = m; i < k; ++i) out[i] = 0;"),
     "output_not_sorted": ("qsort(out, (size_t)m, sizeof(int), int_asc);", ""),
     "head_weight_dropped": ("total += (double)w_row[j] * dot;", "total += dot;"),
+    "block_mean_not_divided": ("float mean = sum / (float)bn;", "float mean = sum;"),
+    "block_partial_dropped": ("for (int s = part0; s < n && s <= t; ++s) {", "for (int s = n; s < n; ++s) {"),
+    "block_budget_ignores_partial": ("int want = c / bn - (part0 < n ? 1 : 0);", "int want = c / bn;"),
+    "block_partial_scored": ("int nfull = n / bn;", "int nfull = (n + bn - 1) / bn;"),
+    "block_rank_by_position": ("qsort(pc, (size_t)nfull, sizeof(cand_t), by_score_desc_pos_asc);", ""),
+    "block_member_mask_dropped": ("                if (s > t) continue;\n                mc[m].score", "                mc[m].score"),
+    "block_keys_from_block_start_only": ("int s = pc[i].pos * bn + r;", "int s = pc[i].pos * bn;"),
 }
 
 
