@@ -10,7 +10,9 @@ member select).  `value` = query rows ranked per second (2 * 131072 per
 step, whole job).  The decode step (B=64 requests x 131072-token caches,
 G=2 MTP queries, dense and Refine c=4096, and dense over the same cache
 scattered into 64-key pages behind a block table) is timed after it and
-reported under "decode" as HBM GB/s of the cache scan.
+reported under "decode" as HBM GB/s of the cache scan.  The block
+pre-filter variant of Refine (candidates from 64-key block means) runs on
+the same packed batch under "block_prefilter", outside the step.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
@@ -50,6 +52,7 @@ def parse():
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-decode", action="store_true")
+    p.add_argument("--no-block", action="store_true")
     p.add_argument("--cpu-rows", type=int, default=64, help="oracle sample rows (dense + refine) per CPU step")
     p.add_argument("--no-cpu", action="store_true", help="skip the CPU-oracle baseline")
     p.add_argument("--tokens", type=int, default=L_TOK,
@@ -349,6 +352,40 @@ def main():
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
         del dq, dk, dw
 
+    # ------------------------------------------- block pre-filter (Refine)
+    blk = None
+    if do_refine and not args.no_block:
+        ws3 = torch.empty(idx.pivot_workspace_size(L, H, D, TOPK, 2, G_REF, C_REF, "block"), dtype=torch.uint8,
+                          device=dev)
+        o3 = torch.empty(L, TOPK, dtype=torch.int32, device=dev)
+
+        def bstep():
+            idx.pivot_topk(q, k, w, cu2, TOPK, G_REF, C_REF, "block", out_idx=o3, workspace=ws3)
+
+        for _ in range(args.warmup):
+            bstep()
+        torch.cuda.synchronize()
+        assert idx.device_status(ws3) == "IDX_OK"
+        barrier()
+        lib.idx_trace_enable(1)
+        e0.record(stream)
+        for _ in range(args.steps):
+            bstep()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        lib.idx_trace_enable(0)
+        barrier()
+        bms = max_over_ranks(e0.elapsed_time(e1) / args.steps)
+        _, trb = trace_report(lib)
+        # overlap with the token-scan Refine output on sampled rows (o2 holds the last Refine step)
+        srows = torch.from_numpy(np.random.default_rng(5).integers(0, L, 256)).to(dev)
+        a, b_ = o2[srows].cpu().numpy(), o3[srows].cpu().numpy()
+        ov = float(np.mean([len(set(x[x >= 0]) & set(y[y >= 0])) / max(1, (x >= 0).sum()) for x, y in zip(a, b_)]))
+        blk = {"workload": f"block_prefilter_refine_2x{L // 2}_g{G_REF}_c{C_REF}_bn64", "ms_per_step": bms,
+               "queries_per_s": world * L / (bms / 1000.0), "overlap_with_refine_topk": ov,
+               "kernels": {n: {"launches": c, "ms_per_step": t / args.steps} for n, (c, t) in trb.items()}}
+        del ws3, o3
+
     # ------------------------------------------------------------- decode
     dec = None
     if not args.no_decode:
@@ -412,7 +449,7 @@ def main():
                    "g": G_REF, "c": C_REF, "parallelism": f"dp{world} (independent batches)",
                    "l2": "inputs larger than L2 (q is 2 GiB)"},
         "tflops_dense": achieved, "roofline": roof, "cpu_baseline": cpu, "e2e": e2e, "clocks": clk,
-        "gpu_launches": nlaunch, "kernels": per_kernel, "decode": dec,
+        "gpu_launches": nlaunch, "kernels": per_kernel, "block_prefilter": blk, "decode": dec,
     }
     if rank == 0:
         print(json.dumps(line))

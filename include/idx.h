@@ -23,6 +23,23 @@
  *   - IDX_MODE_REFINE: the proxy's top-c positions form the candidate set C;
  *                      each member re-scores C with its own q and w, masks
  *                      s > t_member and takes its own top-k.
+ *   - IDX_MODE_BLOCK:  Refine over a candidate set from block summaries
+ *                      instead of the token scan (pages "Not All Tokens
+ *                      Deserve Equal Resolution", abstract: chunk summaries
+ *                      first, exact token scores inside the chosen chunks;
+ *                      "Uncertainty-gated selection for block-sparse
+ *                      attention", Sec. 3.1: a 64-key block is summarised by
+ *                      its mean key).  Each complete 64-token block of the
+ *                      request that ends at or before the group's last
+ *                      member t_last gets a mean key (fp32 sum in key order,
+ *                      IEEE division, bf16 rounding for bf16 keys) and a
+ *                      proxy score (the indexer score against that key).  C
+ *                      is the tokens of the top c/64 blocks by (score desc,
+ *                      block asc), one block fewer when t_last+1 is not a
+ *                      multiple of 64, plus the partial block that holds
+ *                      t_last.  Members then re-score C as in Refine.  No
+ *                      key after t_last takes part.  c must be a multiple of
+ *                      64 and >= topk.
  *
  * Decode form (same page, Method, decode paragraph): the G queries of one
  * MTP step form one group; query m of request b sits at position
@@ -68,7 +85,7 @@ typedef enum {
 
 typedef enum { IDX_BF16 = 0, IDX_F32 = 1 } idx_dtype;
 
-typedef enum { IDX_MODE_DENSE = 0, IDX_MODE_REUSE = 1, IDX_MODE_REFINE = 2 } idx_mode;
+typedef enum { IDX_MODE_DENSE = 0, IDX_MODE_REUSE = 1, IDX_MODE_REFINE = 2, IDX_MODE_BLOCK = 3 } idx_mode;
 
 /* ------------------------------------------------------------ prefill */
 
@@ -93,15 +110,18 @@ idx_status idx_dense_topk(const void *q, const void *k, const float *w, const in
                           int *out_idx, float *out_score, void *ws, size_t ws_bytes,
                           idx_stream_t stream);
 
-/* Workspace bytes for idx_pivot_topk (mode REUSE or REFINE). */
+/* Workspace bytes for idx_pivot_topk (mode REUSE, REFINE or BLOCK); 0 for
+ * arguments idx_pivot_topk would reject. */
 size_t idx_pivot_workspace_size(int T, int H, int d, int topk, int num_seqs, idx_dtype dtype, int g,
                                 int c, idx_mode mode);
 
-/* PIVOT grouped indexer + top-k (Reuse or Refine) over a packed batch.
- * Same tensors and layouts as idx_dense_topk, plus
+/* PIVOT grouped indexer + top-k (Reuse, Refine or block pre-filter Refine)
+ * over a packed batch.  Same tensors and layouts as idx_dense_topk, plus
  *   g     group size (>= 1); groups are request-local [m*g, min((m+1)*g, n))
- *   c     candidate budget for REFINE (c >= topk); ignored for REUSE
- *   mode  IDX_MODE_REUSE or IDX_MODE_REFINE */
+ *   c     candidate budget in tokens for REFINE and BLOCK (c >= topk; BLOCK:
+ *         a multiple of 64); ignored for REUSE
+ *   mode  IDX_MODE_REUSE, IDX_MODE_REFINE or IDX_MODE_BLOCK
+ * IDX_ERR_INVALID for g < 1, an unknown mode or a c these rules reject. */
 idx_status idx_pivot_topk(const void *q, const void *k, const float *w, const int *cu_seqlens,
                           int num_seqs, int T, int H, int d, int topk, idx_dtype dtype, int g, int c,
                           idx_mode mode, int *out_idx, float *out_score, void *ws, size_t ws_bytes,
@@ -197,7 +217,13 @@ const char *idx_status_string(idx_status s);
  *      arguments as idx_pivot_topk),
  *   2: PIVOT Refine member re-scores over the candidate set (rows[] = global
  *      member rows; out[i * ld + j] is the score of candidate j of the
- *      member's group, j < c; requires that idx_pivot_topk ran on `ws`).
+ *      member's group, j < c; requires that idx_pivot_topk ran on `ws`),
+ *   3: block mode proxy rows against the block mean keys (rows[] = proxy
+ *      indices; out[i * ld + j] for blocks j = 0 .. (t_last+1)/64 - 1),
+ *   4: like 2 for a preceding idx_pivot_topk call in IDX_MODE_BLOCK; the
+ *      candidate j of a group is slot j/64, position j%64 of that slot (the
+ *      selected blocks in ascending order, -1 slots, the partial block in
+ *      the last slot).
  * rows is a DEVICE int32 array of DISTINCT rows (a row listed twice gets one
  * of its output rows written).  The scores come from the same kernels and
  * arithmetic as the selection, so re-selecting on them reproduces out_idx. */

@@ -53,8 +53,12 @@ struct PrefillWs {
     PlanLayout pl;
     long long R;          // scored rows (queries or proxies, upper bound)
     unsigned cap, ksel;
-    size_t status, plan, slot, qbar, wbar, cnt, floor, buf, cand, msc, ckeys, total;
+    size_t status, plan, slot, qbar, wbar, cnt, floor, buf, cand, msc, ckeys, kblk, cblk, total;
 };
+
+bool refines(idx_mode m) { return m == IDX_MODE_REFINE || m == IDX_MODE_BLOCK; }
+
+long long block_rows(int T) { return (T >> kBlockShift) > 0 ? (T >> kBlockShift) : 1; }
 
 PrefillWs prefill_ws(int T, int H, int d, int topk, int S, idx_dtype dt, int g, int c, idx_mode mode) {
     PrefillWs L{};
@@ -63,9 +67,11 @@ PrefillWs prefill_ws(int T, int H, int d, int topk, int S, idx_dtype dt, int g, 
     L.pl.S = S;
     L.pl.maxblk = (int)((L.R + RB - 1) / RB + S);
     L.pl.maxtiles = (int)(nbound(T) / KT + 1);
-    L.ksel = mode == IDX_MODE_REUSE ? (unsigned)(topk + g - 1) : mode == IDX_MODE_REFINE ? (unsigned)c
-                                                                                       : (unsigned)topk;
-    L.cap = cap_for(L.ksel, nbound(T));
+    L.ksel = mode == IDX_MODE_REUSE    ? (unsigned)(topk + g - 1)
+             : mode == IDX_MODE_REFINE ? (unsigned)c
+             : mode == IDX_MODE_BLOCK  ? (unsigned)(c >> kBlockShift)
+                                       : (unsigned)topk;
+    L.cap = mode == IDX_MODE_BLOCK ? cap_for(L.ksel, (nbound(T) >> kBlockShift) + 1) : cap_for(L.ksel, nbound(T));
     Carve cv;
     L.status = cv.take(16);
     L.plan = cv.take(L.pl.words() * 4);
@@ -75,11 +81,13 @@ PrefillWs prefill_ws(int T, int H, int d, int topk, int S, idx_dtype dt, int g, 
     L.cnt = cv.take((size_t)L.R * 4);
     L.floor = cv.take((size_t)L.R * 4);
     L.buf = cv.take((size_t)L.R * L.cap * 8);
-    L.cand = mode == IDX_MODE_REFINE ? cv.take((size_t)L.R * c * 4) : 0;
-    L.msc = mode == IDX_MODE_REFINE ? cv.take((size_t)T * c * 4) : 0;
-    L.ckeys = (mode == IDX_MODE_REFINE && tc_gather_supported(H, d, (int)dt, g, c))
+    L.cand = refines(mode) ? cv.take((size_t)L.R * c * 4) : 0;
+    L.msc = refines(mode) ? cv.take((size_t)T * c * 4) : 0;
+    L.ckeys = (refines(mode) && tc_gather_supported(H, d, (int)dt, g, c))
                   ? cv.take((size_t)L.R * c_pad_of(c) * d * esize(dt))
                   : 0;
+    L.kblk = mode == IDX_MODE_BLOCK ? cv.take((size_t)block_rows(T) * d * esize(dt)) : 0;
+    L.cblk = mode == IDX_MODE_BLOCK ? cv.take((size_t)L.R * (c >> kBlockShift) * 4) : 0;
     L.total = cv.off;
     return L;
 }
@@ -163,8 +171,10 @@ struct Prefill {
 
     ScoreArgs score_args(bool proxies) const {
         ScoreArgs a{};
+        const bool blocks = proxies && mode == IDX_MODE_BLOCK;
         a.q = proxies ? (const void *)(ws + L.qbar) : q;
-        a.k = k;
+        a.k = blocks ? (const void *)(ws + L.kblk) : k;
+        a.kshift = blocks ? kBlockShift : 0;
         a.w = proxies ? reinterpret_cast<const float *>(ws + L.wbar) : w;
         a.cu = cu;
         a.S = S; a.T = T; a.H = H; a.d = d;
@@ -197,6 +207,8 @@ struct Prefill {
         if (mode != IDX_MODE_DENSE)
             e = launch_proxy(q, w, cu, S, T, H, d, g, (int)dt, plan(), L.pl, ws + L.qbar,
                              reinterpret_cast<float *>(ws + L.wbar), (int)L.R, st);
+        if (e == cudaSuccess && mode == IDX_MODE_BLOCK)
+            e = launch_block_means(k, cu, S, T, d, (int)dt, ws + L.kblk, st);
         return e;
     }
 
@@ -295,22 +307,25 @@ idx_status idx_dense_topk(const void *q, const void *k, const float *w, const in
 size_t idx_pivot_workspace_size(int T, int H, int d, int topk, int num_seqs, idx_dtype dtype, int g, int c,
                                 idx_mode mode) {
     if (T < 1 || num_seqs < 1 || topk < 1 || g < 1 || !shape_ok(H, d, dtype)) return 0;
-    if (mode != IDX_MODE_REUSE && mode != IDX_MODE_REFINE) return 0;
-    if (mode == IDX_MODE_REFINE && c < topk) return 0;
+    if (mode != IDX_MODE_REUSE && mode != IDX_MODE_REFINE && mode != IDX_MODE_BLOCK) return 0;
+    if (refines(mode) && c < topk) return 0;
+    if (mode == IDX_MODE_BLOCK && (c < kBlockN || c % kBlockN != 0)) return 0;
     return prefill_ws(T, H, d, topk, num_seqs, dtype, g, c, mode).total;
 }
 
 idx_status idx_pivot_topk(const void *q, const void *k, const float *w, const int *cu_seqlens, int num_seqs,
                           int T, int H, int d, int topk, idx_dtype dtype, int g, int c, idx_mode mode,
                           int *out_idx, float *out_score, void *ws, size_t ws_bytes, idx_stream_t stream) {
-    if (g < 1 || (mode != IDX_MODE_REUSE && mode != IDX_MODE_REFINE)) return IDX_ERR_INVALID;
-    if (mode == IDX_MODE_REFINE && c < topk) return IDX_ERR_INVALID;
+    if (g < 1 || (mode != IDX_MODE_REUSE && mode != IDX_MODE_REFINE && mode != IDX_MODE_BLOCK))
+        return IDX_ERR_INVALID;
+    if (refines(mode) && c < topk) return IDX_ERR_INVALID;
+    if (mode == IDX_MODE_BLOCK && (c < kBlockN || c % kBlockN != 0)) return IDX_ERR_INVALID;
     if (mode == IDX_MODE_REUSE) c = topk;
     const size_t need = idx_pivot_workspace_size(T, H, d, topk, num_seqs, dtype, g, c, mode);
     idx_status s = check_prefill(q, k, w, cu_seqlens, num_seqs, T, H, d, topk, dtype, out_idx, ws, ws_bytes,
                                  need);
     if (s != IDX_OK) return s;
-    TracePhase phase(mode == IDX_MODE_REUSE ? "reuse" : "refine");
+    TracePhase phase(mode == IDX_MODE_REUSE ? "reuse" : mode == IDX_MODE_REFINE ? "refine" : "block");
     Prefill P{q, k, w, cu_seqlens, num_seqs, T, H, d, topk, dtype, g, c, mode, static_cast<char *>(ws),
               prefill_ws(T, H, d, topk, num_seqs, dtype, g, c, mode), reinterpret_cast<cudaStream_t>(stream)};
     TRY_CUDA(P.prepare());
@@ -318,7 +333,14 @@ idx_status idx_pivot_topk(const void *q, const void *k, const float *w, const in
     if (mode == IDX_MODE_REUSE)
         return cuda_st(launch_select(P.select_args(SEL_REUSE_CAND, T, topk, out_idx, out_score), P.st));
     int *cand = reinterpret_cast<int *>(P.ws + P.L.cand);
-    TRY_CUDA(launch_select(P.select_args(SEL_PROXY_TO_C, (int)P.L.R, c, cand, nullptr), P.st));
+    if (mode == IDX_MODE_BLOCK) {
+        int *cblk = reinterpret_cast<int *>(P.ws + P.L.cblk);
+        TRY_CUDA(launch_select(P.select_args(SEL_PROXY_TO_BLOCKS, (int)P.L.R, c >> kBlockShift, cblk, nullptr),
+                               P.st));
+        TRY_CUDA(launch_block_expand(cu_seqlens, num_seqs, g, P.plan(), P.L.pl, cblk, cand, c, (int)P.L.R, P.st));
+    } else {
+        TRY_CUDA(launch_select(P.select_args(SEL_PROXY_TO_C, (int)P.L.R, c, cand, nullptr), P.st));
+    }
     const GatherArgs ga = P.gather_args();
     TRY_CUDA(tc_gather_supported(H, d, (int)dtype, g, c) ? launch_gather_tc(ga, P.st)
                                                        : launch_gather_simt(ga, (int)dtype, P.st));
@@ -487,11 +509,14 @@ idx_status idx_debug_scores(int stage, const void *q, const void *k, const float
                             int num_seqs, int T, int H, int d, idx_dtype dtype, int g, int c, int topk,
                             const int *rows, int nrows, float *out, long long ld, void *ws, size_t ws_bytes,
                             idx_stream_t stream) {
-    if (!rows || !out || nrows < 0 || ld < 1 || stage < 0 || stage > 2) return IDX_ERR_INVALID;
-    const idx_mode mode = stage == 0 ? IDX_MODE_DENSE : (stage == 2 || c > 0 ? IDX_MODE_REFINE : IDX_MODE_REUSE);
+    if (!rows || !out || nrows < 0 || ld < 1 || stage < 0 || stage > 4) return IDX_ERR_INVALID;
+    const idx_mode mode = stage == 0   ? IDX_MODE_DENSE
+                          : stage >= 3 ? IDX_MODE_BLOCK
+                                       : (stage == 2 || c > 0 ? IDX_MODE_REFINE : IDX_MODE_REUSE);
     const int gg = stage == 0 ? 1 : g;
-    const int cc = mode == IDX_MODE_REFINE ? c : topk;
-    if (gg < 1 || (mode == IDX_MODE_REFINE && cc < topk)) return IDX_ERR_INVALID;
+    const int cc = refines(mode) ? c : topk;
+    if (gg < 1 || (refines(mode) && cc < topk)) return IDX_ERR_INVALID;
+    if (mode == IDX_MODE_BLOCK && (cc < kBlockN || cc % kBlockN != 0)) return IDX_ERR_INVALID;
     const size_t need = mode == IDX_MODE_DENSE
                             ? idx_dense_workspace_size(T, H, d, topk, num_seqs, dtype)
                             : idx_pivot_workspace_size(T, H, d, topk, num_seqs, dtype, gg, cc, mode);
@@ -501,7 +526,7 @@ idx_status idx_debug_scores(int stage, const void *q, const void *k, const float
     Prefill P{q, k, w, cu_seqlens, num_seqs, T, H, d, topk, dtype, gg, cc, mode, static_cast<char *>(ws),
               prefill_ws(T, H, d, topk, num_seqs, dtype, gg, cc, mode), reinterpret_cast<cudaStream_t>(stream)};
     if (nrows == 0) return IDX_OK;
-    if (stage == 2) {
+    if (stage == 2 || stage == 4) {
         TRY_CUDA(cudaMemsetAsync(P.status(), 0, 4, P.st));
         for (int r0 = 0; r0 < nrows; r0 += 65535) {
             const int nr = nrows - r0 < 65535 ? nrows - r0 : 65535;
@@ -518,7 +543,7 @@ idx_status idx_debug_scores(int stage, const void *q, const void *k, const float
     TRY_CUDA(cudaMemsetAsync(slot, 0xFF, (size_t)R * 4, P.st));
     scatter_slots<<<(nrows + 255) / 256, 256, 0, P.st>>>(rows, nrows, (int)R, slot, P.status());
     TRY_CUDA(cudaGetLastError());
-    ScoreArgs a = P.score_args(stage == 1);
+    ScoreArgs a = P.score_args(stage == 1 || stage == 3);
     a.sink = SINK_SPILL;
     a.spill = out;
     a.ld = ld;

@@ -33,13 +33,21 @@ enum Sink { SINK_FILTER = 0, SINK_SPILL = 1 };
 
 // A prefill score pass: rows of `q` (queries, or PIVOT proxies when g > 1)
 // against the keys of their request, streamed into a sink.
+// block pre-filter: keys summarised per complete block of kBlockN tokens
+constexpr int kBlockShift = 6;
+constexpr int kBlockN = 1 << kBlockShift;
+
 struct ScoreArgs {
     const void *q;       // [R, H, d] scored rows
-    const void *k;       // [T, d] keys
+    const void *k;       // [T, d] keys (kshift = 0), or block mean keys (kshift > 0)
     const float *w;      // [R, H]
     const int *cu;       // cu_seqlens [S+1] (device)
     int S, T, H, d, g;   // g = 1: row i of request b is query i; g > 1: proxy i
     long long R;         // rows allocated in q / w
+    // kshift > 0: keys are the complete 2^kshift-token blocks of each request,
+    // block i of request b at key row (cu[b] >> kshift) + i; a row whose token
+    // bound is t sees blocks 0 .. ((t + 1) >> kshift) - 1
+    int kshift;
     const int *plan;     // plan area
     PlanLayout pl;
     int sink;
@@ -121,7 +129,9 @@ enum SelKind {
     SEL_DEC_DENSE = 4,      // decode: spill row (b, m)
     SEL_DEC_REUSE = 5,      // decode: proxy spill row b restricted to member m
     SEL_DEC_PROXY_TO_C = 6, // decode: candidate set of request b
-    SEL_DEC_MEMBER = 7      // decode: member scores over the candidate set
+    SEL_DEC_MEMBER = 7,     // decode: member scores over the candidate set
+    SEL_PROXY_TO_BLOCKS = 8 // block pre-filter: complete blocks of a proxy row (k = c / kBlockN, one
+                            // fewer when the row's prefix ends inside a block), block indices only
 };
 
 struct SelectArgs {
@@ -180,6 +190,13 @@ cudaError_t launch_select(const SelectArgs &a, cudaStream_t st);
 cudaError_t launch_proxy(const void *q, const float *w, const int *cu, int S, int T, int H, int d,
                          int g, int dtype, const int *plan, const PlanLayout &pl, void *qbar,
                          float *wbar, int max_proxies, cudaStream_t st);
+// block pre-filter: mean keys of the complete blocks of every request
+cudaError_t launch_block_means(const void *k, const int *cu, int S, int T, int d, int dtype, void *kb,
+                               cudaStream_t st);
+// block pre-filter: candidate positions [R, c] from the selected blocks [R, c / kBlockN]
+// plus the partial block that holds each proxy's last member
+cudaError_t launch_block_expand(const int *cu, int S, int g, const int *plan, const PlanLayout &pl,
+                                const int *cblk, int *cand, int c, int R, cudaStream_t st);
 cudaError_t launch_decode_proxy(const void *q, const float *w, int B, int G, int H, int d, int dtype,
                                 void *qbar, float *wbar, cudaStream_t st);
 size_t simt_smem_bytes(int H, int d, int dtype);

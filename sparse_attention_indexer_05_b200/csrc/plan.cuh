@@ -39,8 +39,13 @@ struct BlockInfo {
     int ntiles;   // key tiles covering 0..maxbound
 };
 
+// Row bound in key units: keys are tokens (kshift = 0) or complete blocks of
+// 2^kshift tokens (a row whose token bound is t sees the blocks that end at
+// or before t); -1 when no key is visible.
+__device__ __forceinline__ int key_bound(int t, int kshift) { return ((t + 1) >> kshift) - 1; }
+
 __device__ __forceinline__ BlockInfo block_info(const int *plan, const PlanLayout &pl, const int *cu,
-                                                int g, int blk) {
+                                                int g, int blk, int kshift = 0) {
     BlockInfo bi;
     const int *rp = plan + pl.rp();
     const int *bp = plan + pl.bp();
@@ -53,9 +58,9 @@ __device__ __forceinline__ BlockInfo block_info(const int *plan, const PlanLayou
     int e = bi.i0 + RB;
     if (e > R) e = R;
     bi.nrows = e - bi.i0;
-    bi.key0 = cu[bi.b];
-    bi.maxbound = row_bound(e - 1, bi.n, g);
-    bi.ntiles = bi.maxbound / KT + 1;
+    bi.key0 = kshift ? (long long)(cu[bi.b] >> kshift) : (long long)cu[bi.b];
+    bi.maxbound = key_bound(row_bound(e - 1, bi.n, g), kshift);
+    bi.ntiles = bi.maxbound < 0 ? 1 : bi.maxbound / KT + 1;
     return bi;
 }
 

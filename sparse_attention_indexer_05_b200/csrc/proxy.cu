@@ -102,7 +102,109 @@ __global__ void __launch_bounds__(kProxyThreads) decode_proxy_kernel(const T *q,
               wbar + (long long)b * H);
 }
 
+// Block pre-filter (page "Uncertainty-gated selection for block-sparse
+// attention", Sec. 3.1: a block of 64 keys is summarised by its mean key;
+// page "Not All Tokens Deserve Equal Resolution", abstract: coarse chunk
+// summaries first, exact token scores inside the chosen chunks next).  The
+// mean of each complete block of a request: fp32 sum in key order, one IEEE
+// division by the block size, bf16 round-to-nearest-even for bf16 keys.
+// Block i of request b goes to row (cu[b] >> kBlockShift) + i; rows that
+// belong to no complete block are zero.  One thread per 8 dimensions of one
+// block row.
+template <typename T>
+__global__ void __launch_bounds__(kProxyThreads) block_mean_kernel(const T *k, const int *cu, int S, int T_,
+                                                                   int d, long long nrows, T *kb) {
+    const int per_row = d / 8;
+    const long long u = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    if (u >= nrows * per_row) return;
+    const long long x = u / per_row;
+    const int e = (int)(u - x * per_row) * 8;
+    // the request whose block rows start at or before x (last such b)
+    int lo = 0, hi = S;
+    while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if ((long long)(cu[mid] >> kBlockShift) <= x) lo = mid; else hi = mid;
+    }
+    const long long i = x - (cu[lo] >> kBlockShift);
+    // malformed cu_seqlens (the plan flags them) read nothing
+    const bool ok = cu[lo] >= 0 && cu[lo] <= cu[lo + 1] && cu[lo + 1] <= T_;
+    const int nfull = ok ? (cu[lo + 1] - cu[lo]) >> kBlockShift : 0;
+    float acc[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) acc[j] = 0.0f;
+    if (i < nfull) {
+        const T *src = k + ((long long)cu[lo] + i * kBlockN) * d + e;
+        float v[8];
+        for (int r = 0; r < kBlockN; ++r) {
+            Vec<T>::load(src + (long long)r * d, v);
+#pragma unroll
+            for (int j = 0; j < 8; ++j) acc[j] = __fadd_rn(acc[j], v[j]);
+        }
+#pragma unroll
+        for (int j = 0; j < 8; ++j) acc[j] = __fdiv_rn(acc[j], (float)kBlockN);
+    }
+    Vec<T>::store(kb + x * d + e, acc);
+}
+
+// Candidate set of each proxy row in block mode: slot j of cblk [R, nb]
+// (a selected block, or -1) expands to the 64 positions of that block; the
+// partial block that holds the proxy's last member t_last fills the last
+// slot, which the block selection leaves empty whenever such a block exists.
+__global__ void __launch_bounds__(kProxyThreads) block_expand_kernel(const int *cu, int S, int g, const int *plan,
+                                                                     PlanLayout pl, const int *cblk, int *cand,
+                                                                     int c) {
+    const int p = blockIdx.x;
+    int *out = cand + (long long)p * c;
+    const int nb = c >> kBlockShift;
+    if (!plan[0] || p >= plan[2]) {
+        for (int j = threadIdx.x; j < c; j += blockDim.x) out[j] = -1;
+        return;
+    }
+    const int *rp = plan + pl.rp();
+    const int b = find_seg(rp, S, p);
+    const int i = p - rp[b];
+    const int n = cu[b + 1] - cu[b];
+    const int tl = row_bound(i, n, g);
+    const int part0 = (tl + 1) & ~(kBlockN - 1);
+    const bool partial = part0 <= tl;
+    const int *sel = cblk + (long long)p * nb;
+    for (int j = threadIdx.x; j < c; j += blockDim.x) {
+        const int slot = j >> kBlockShift, r = j & (kBlockN - 1);
+        int v;
+        if (partial && slot == nb - 1) {
+            v = part0 + r <= tl ? part0 + r : -1;
+        } else {
+            const int blk = sel[slot];
+            v = blk >= 0 ? blk * kBlockN + r : -1;
+        }
+        out[j] = v;
+    }
+}
+
 }  // namespace
+
+cudaError_t launch_block_means(const void *k, const int *cu, int S, int T, int d, int dtype, void *kb,
+                               cudaStream_t st) {
+    const long long nrows = (T >> kBlockShift) > 0 ? (T >> kBlockShift) : 1;
+    const long long units = nrows * (d / 8);
+    TraceScope ts("block_means", st);
+    const unsigned grid = (unsigned)((units + kProxyThreads - 1) / kProxyThreads);
+    if (dtype == 1)
+        block_mean_kernel<float><<<grid, kProxyThreads, 0, st>>>((const float *)k, cu, S, T, d, nrows,
+                                                                 (float *)kb);
+    else
+        block_mean_kernel<__nv_bfloat16><<<grid, kProxyThreads, 0, st>>>(
+            (const __nv_bfloat16 *)k, cu, S, T, d, nrows, (__nv_bfloat16 *)kb);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_block_expand(const int *cu, int S, int g, const int *plan, const PlanLayout &pl,
+                                const int *cblk, int *cand, int c, int R, cudaStream_t st) {
+    if (R <= 0) return cudaSuccess;
+    TraceScope ts("block_expand", st);
+    block_expand_kernel<<<R, kProxyThreads, 0, st>>>(cu, S, g, plan, pl, cblk, cand, c);
+    return cudaGetLastError();
+}
 
 cudaError_t launch_proxy(const void *q, const float *w, const int *cu, int S, int T, int H, int d, int g,
                          int dtype, const int *plan, const PlanLayout &pl, void *qbar, float *wbar,

@@ -185,7 +185,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         __syncthreads();
         const int item = sh.item;
         if (item >= nblocks) break;
-        const BlockInfo bi = block_info(plan, a.pl, a.cu, a.g, plan[a.pl.order() + item]);
+        const BlockInfo bi = block_info(plan, a.pl, a.cu, a.g, plan[a.pl.order() + item], a.kshift);
         const int ntiles = bi.ntiles;
 
         if (warp >= 2) {
@@ -195,7 +195,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 wsm[i] = (i / TC_H) < bi.nrows ? a.w[(long long)bi.row0 * TC_H + i] : 0.0f;
             if (e < RB) {
                 if (lane == 0) {
-                    sh.bound[e] = e < bi.nrows ? row_bound(bi.i0 + e, bi.n, a.g) : -1;
+                    sh.bound[e] = e < bi.nrows ? key_bound(row_bound(bi.i0 + e, bi.n, a.g), a.kshift) : -1;
                     sh.slot[e] = -1;
                     if (a.sink == SINK_SPILL && e < bi.nrows && a.slot_of_row)
                         sh.slot[e] = a.slot_of_row[bi.row0 + e];
@@ -367,7 +367,9 @@ bool tc_supported(int H, int d, int dtype) { return H == TC_H && d == TC_D && dt
 cudaError_t launch_score_tc(const ScoreArgs &a, cudaStream_t st) {
     // the scored tensor [R, 64, 128] viewed as [R*64, 128]; keys [T, 128]
     CUtensorMap mq, mk;
-    if (!make_map(&mq, a.q, (unsigned long long)a.R * TC_H, 256) || !make_map(&mk, a.k, (unsigned long long)a.T, KT))
+    const unsigned long long krows =
+        a.kshift ? ((a.T >> a.kshift) > 0 ? (unsigned long long)(a.T >> a.kshift) : 1ull) : (unsigned long long)a.T;
+    if (!make_map(&mq, a.q, (unsigned long long)a.R * TC_H, 256) || !make_map(&mk, a.k, krows, KT))
         return cudaErrorInvalidValue;
     cudaError_t e = cudaFuncSetAttribute(score_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
     if (e != cudaSuccess) return e;

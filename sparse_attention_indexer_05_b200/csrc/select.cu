@@ -424,6 +424,22 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(SelectArgs a) {
                      a.status);
         return;
     }
+    case SEL_PROXY_TO_BLOCKS: {
+        if (!a.plan[0]) { pad_all(); return; }
+        if (row >= a.plan[2]) return;
+        const int *rp = a.plan + a.pl.rp();
+        const int b = find_seg(rp, a.S, row);
+        const int i = row - rp[b];
+        const int n = a.cu[b + 1] - a.cu[b];
+        const int tl = row_bound(i, n, a.g);
+        // the partial block holding the last member takes one slot of the budget
+        const int kr = a.k - (((tl + 1) & (kBlockN - 1)) ? 1 : 0);
+        if (kr > 0)
+            block_select(cand(row, key_bound(tl, kBlockShift)), kr, oi, nullptr, sh, stage, a.stage_cap, bm, gpre,
+                         wcap, a.status);
+        for (int r = (kr > 0 ? kr : 0) + (int)threadIdx.x; r < a.k; r += blockDim.x) oi[r] = -1;
+        return;
+    }
     default: {  // decode kinds
         const bool per_member = a.kind != SEL_DEC_PROXY_TO_C;
         const int b = per_member ? row / a.G : row;

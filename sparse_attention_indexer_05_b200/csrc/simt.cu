@@ -104,14 +104,14 @@ __global__ void __launch_bounds__(kSimtThreads) score_simt_kernel(ScoreArgs a) {
         __syncthreads();
         const int item = s_item;
         if (item >= nblocks) break;
-        const BlockInfo bi = block_info(plan, a.pl, a.cu, a.g, plan[a.pl.order() + item]);
+        const BlockInfo bi = block_info(plan, a.pl, a.cu, a.g, plan[a.pl.order() + item], a.kshift);
         load_rows(qs, q + (long long)bi.row0 * HD, bi.nrows, HD);
         for (int i = threadIdx.x; i < RB * a.H; i += blockDim.x)
             wsm[i] = (i / a.H) < bi.nrows ? a.w[(long long)bi.row0 * a.H + i] : 0.0f;
         if (a.sink == SINK_FILTER && warp < RB) sel_init(sel[warp], hist + warp * kBins);
         const int r = warp;
         const bool row_ok = r < bi.nrows;
-        const int bound = row_ok ? row_bound(bi.i0 + r, bi.n, a.g) : -1;
+        const int bound = row_ok ? key_bound(row_bound(bi.i0 + r, bi.n, a.g), a.kshift) : -1;
         const long long grow = (long long)bi.row0 + r;
         int slot = -1;
         if (a.sink == SINK_SPILL && row_ok && a.slot_of_row) slot = a.slot_of_row[grow];

@@ -40,8 +40,10 @@ struct __align__(8) StShared {
 
 constexpr size_t kOffQ = 0;
 constexpr size_t kOffA = kOffQ + kQBytes;
+constexpr int kMaxPageBoxes = kDecodeChunkTiles * (KT / 8);  // paged decode: boxes of >= 8 rows per item
 constexpr size_t kOffW = kOffA + (size_t)kStages * kAStage;
-constexpr size_t kOffCtl = kOffW + 4 * S_H * 4;
+constexpr size_t kOffPg = kOffW + 4 * S_H * 4;
+constexpr size_t kOffCtl = kOffPg + (size_t)kMaxPageBoxes * 4;
 constexpr size_t kSmemBytes = kOffCtl + sizeof(StShared) + 1024;
 
 struct Item {
@@ -165,6 +167,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint8_t *qs = smem + kOffQ;
     uint8_t *as = smem + kOffA;
     float *wsm = reinterpret_cast<float *>(smem + kOffW);
+    int *pg_rows = reinterpret_cast<int *>(smem + kOffPg);  // paged decode: first pool row of each box
     StShared &sh = *reinterpret_cast<StShared *>(smem + kOffCtl);
     volatile int *abort = &sh.abort;
     unsigned *status = GATHER ? g.status : dd.status;
@@ -214,6 +217,17 @@ __global__ void __launch_bounds__(kThreads, 1)
 
         if (warp == 0) {
             bool ok = !*abort;
+            const bool paged = !GATHER && dd.bt;
+            const int box = paged && dd.page < KT ? dd.page : KT;  // rows per TMA box
+            if (paged) {
+                // the item's block-table lookups in one coalesced pass, off the issue path
+                const int n = it.nt * (KT / box);
+                const int b = (int)(it.qrow0 / dd.Gq);
+                for (int i = lane; i < n; i += 32)
+                    pg_rows[i] = (int)cache_row(dd.bt, dd.page, dd.max_pages, dd.num_pages, dd.n_max, b,
+                                                it.t0 * KT + i * box);
+                __syncwarp();
+            }
             if (lane == 0 && ok) {
                 tc::mbar_arrive_expect_tx(&sh.qfull, kQBytes);
                 for (int kh = 0; kh < 2; ++kh)
@@ -227,22 +241,18 @@ __global__ void __launch_bounds__(kThreads, 1)
                 uint8_t *dst = as + st * kAStage;
                 if (lane == 0) {
                     tc::mbar_arrive_expect_tx(&sh.afull[st], kAStage);
-                    if (GATHER || !dd.bt) {
+                    if (!paged) {
                         const int row = (int)(it.key0 + (long long)(it.t0 + j) * KT);
                         for (int kh = 0; kh < 2; ++kh)
                             tc::tma_load_2d(dst + kh * kASlice, &tmap_k, kh * 64, row, &sh.afull[st]);
                     } else {
-                        // paged cache: the tile's 128 positions span 128 / box pages (box = min(page, 128))
-                        const int box = dd.page < KT ? dd.page : KT;
-                        const int s0 = (it.t0 + j) * KT;
-                        const int b = (int)(it.qrow0 / dd.Gq);
-                        for (int i = 0; i < KT / box; ++i) {
-                            const int row =
-                                (int)cache_row(dd.bt, dd.page, dd.max_pages, dd.num_pages, dd.n_max, b, s0 + i * box);
+                        // paged cache: the tile's 128 positions are 128 / box boxes of whole pages
+                        // (or one box inside a page); each box lands at its row offset in the stage
+                        const int per = KT / box;
+                        for (int i = 0; i < per; ++i)
                             for (int kh = 0; kh < 2; ++kh)
-                                tc::tma_load_2d(dst + kh * kASlice + i * box * 128, &tmap_k, kh * 64, row,
-                                                &sh.afull[st]);
-                        }
+                                tc::tma_load_2d(dst + kh * kASlice + i * box * 128, &tmap_k, kh * 64,
+                                                pg_rows[j * per + i], &sh.afull[st]);
                     }
                 }
             }
@@ -408,6 +418,7 @@ bool tc_gather_supported(int H, int d, int dtype, int group, int c) {
 }
 
 cudaError_t launch_decode_tc(const DecodeArgs &a, cudaStream_t st) {
+    if (a.bt && (a.page < 8 || (KT % a.page != 0 && a.page % KT != 0))) return cudaErrorInvalidValue;
     CUtensorMap mq, mk;
     const unsigned long long krows = a.bt ? (unsigned long long)a.num_pages * a.page : (unsigned long long)a.B * a.n_max;
     const unsigned box = a.bt && a.page < KT ? (unsigned)a.page : (unsigned)KT;

@@ -21,7 +21,7 @@ import torch
 
 from . import _native as N
 
-MODES = {"dense": N.MODE_DENSE, "reuse": N.MODE_REUSE, "refine": N.MODE_REFINE}
+MODES = {"dense": N.MODE_DENSE, "reuse": N.MODE_REUSE, "refine": N.MODE_REFINE, "block": N.MODE_BLOCK}
 
 
 def _mode(m) -> int:
@@ -170,17 +170,20 @@ def uses_tensor_cores(H: int, d: int, dtype=torch.bfloat16) -> bool:
 
 
 def debug_scores(stage: int, q, k, w, cu_seqlens, topk, rows, g=1, c=0, workspace=None, ld=None, stream=None):
-    """Scores the selection used (test hook): stage 0 dense rows, 1 proxies, 2 Refine members.
-    `workspace` must be the one the matching top-k call used (required for stage 2)."""
+    """Scores the selection used (test hook): stage 0 dense rows, 1 proxies, 2 Refine members,
+    3 block-mode proxies against block mean keys, 4 block-mode members.
+    `workspace` must be the one the matching top-k call used (required for stages 2 and 4)."""
     T, H, d = q.shape
     S = cu_seqlens.numel() - 1
     dt = _dtype_code(q)
     rows = rows.to(device=q.device, dtype=torch.int32).contiguous()
-    width = ld or (c if stage == 2 else T)
+    width = ld or (c if stage in (2, 4) else (max(T // 64, 1) if stage == 3 else T))
     out = torch.full((rows.numel(), width), float("nan"), dtype=torch.float32, device=q.device)
     if workspace is None:
         if stage == 0:
             need = dense_workspace_size(T, H, d, topk, S, q.dtype)
+        elif stage >= 3:
+            need = pivot_workspace_size(T, H, d, topk, S, g, c, "block", q.dtype)
         else:
             need = pivot_workspace_size(T, H, d, topk, S, g, c if c > 0 else topk, "refine" if c > 0 else "reuse",
                                         q.dtype)
