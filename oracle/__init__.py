@@ -1,8 +1,9 @@
 """ctypes front of the CPU oracle (oracle.c).
 
 TEST INFRASTRUCTURE ONLY: the plain, slow double-precision restatement of
-the lightning indexer + top-k (dense, PIVOT Reuse/Refine, decode) that the
-CUDA library is checked against.  Only the tests, ``__graft_entry__.smoke``
+the lightning indexer + top-k (dense, PIVOT Reuse/Refine/block pre-filter,
+decode) and of the token-sparse attention over the selected positions that
+the CUDA library is checked against.  Only the tests, ``__graft_entry__.smoke``
 and the benchmark's CPU-baseline leg may import this package.  It imports
 nothing from the product package and the product imports nothing from it.
 
@@ -40,8 +41,9 @@ def load(path: str) -> ctypes.CDLL:
         L.ora_block_mean.argtypes = [vp, i, i, ll, i, vp]
         L.ora_pivot_topk.argtypes = [vp, vp, fp, i, ip, i, i, i, i, i, i, i, i, llp, i, ip, i]
         L.ora_decode_topk.argtypes = [vp, vp, fp, i, ip, i, i, i, i, i, i, i, i, i, llp, i, ip, i]
+        L.ora_sparse_attn.argtypes = [vp, vp, i, ip, ip, ip, i, i, i, i, i, ctypes.c_double, llp, i, dp, dp, i]
         for f in (L.ora_score_row, L.ora_select, L.ora_group_proxy, L.ora_block_mean, L.ora_dense_topk,
-                  L.ora_pivot_topk, L.ora_decode_topk):
+                  L.ora_pivot_topk, L.ora_decode_topk, L.ora_sparse_attn):
             f.restype = ctypes.c_int
         _libs[path] = L
     return _libs[path]
@@ -189,3 +191,24 @@ def decode_topk(q, kcache, w, kv_len, topk: int, c: int = 0, mode: int = DENSE, 
                                  B, G, n_max, H, d, topk, c, mode, bn, _ptr(r, ctypes.c_longlong), len(r),
                                  _ptr(out, ctypes.c_int), _threads(threads)), "decode_topk")
     return out
+
+
+def sparse_attn(q, kv, idx, cu_q, cu_kv, Dv: int, scale: float, rows=None, threads=None):
+    """Token-sparse attention of query rows over their listed kv positions:
+    q [R, Ha, Dqk], kv [Nkv, Dqk], idx [R, topk] (-1 = none), cu_q / cu_kv the
+    request boundaries over query rows and kv rows.  Returns (o [n, Ha, Dv],
+    lse [n, Ha]) in float64."""
+    q = np.ascontiguousarray(q); kv = np.ascontiguousarray(kv)
+    ix = _c(idx, np.int32)
+    cq, ck = _c(cu_q, np.int32), _c(cu_kv, np.int32)
+    dt = _dtype_code(q)
+    R, Ha, Dqk = q.shape
+    topk = ix.shape[1]
+    r = _rows(rows, R)
+    o = np.empty((len(r), Ha, Dv), np.float64)
+    lse = np.empty((len(r), Ha), np.float64)
+    _check(lib().ora_sparse_attn(_ptr(q), _ptr(kv), dt, _ptr(ix, ctypes.c_int), _ptr(cq, ctypes.c_int),
+                                 _ptr(ck, ctypes.c_int), len(cq) - 1, Ha, Dqk, Dv, topk, float(scale),
+                                 _ptr(r, ctypes.c_longlong), len(r), _ptr(o, ctypes.c_double),
+                                 _ptr(lse, ctypes.c_double), _threads(threads)), "sparse_attn")
+    return o, lse

@@ -43,6 +43,13 @@
  *    counts tokens (c / bn blocks, one of them the partial block if there
  *    is one); the mean key is rounded like the proxy (fp32 sum in key order,
  *    IEEE division, bf16 round-to-nearest-even).
+ *  - Token-sparse attention (ora_sparse_attn), the consumer of the selected
+ *    sets: the PIVOT page's introduction says the selected set feeds sparse
+ *    MLA attention.  The pages give no formula; the reading used here is
+ *    softmax attention restricted to the selected positions, in the
+ *    absorbed MLA form of the production models that page names: one
+ *    latent row per key serves as the key (all Dqk dimensions) and its
+ *    first Dv dimensions as the value, shared by every head.
  *  - Readings where the pages are silent (each also listed in the design
  *    notes): proxy of w = mean of w; proxy arithmetic = fp32 sum in member
  *    order, IEEE division, then round-to-nearest-even to bf16 for bf16
@@ -506,4 +513,117 @@ int ora_decode_topk(const void *q, const void *kcache, const float *w, int dtype
     J.c = c; J.mode = mode; J.bn = bn; J.kv_len = kv_len; J.G = G; J.n_max = n_max; J.rows = reqs;
     J.nrows = nreqs; J.out = out;
     return run_job(&J, nthreads);
+}
+
+/* ------------------------------------------------ token-sparse attention */
+
+typedef struct {
+    const void *q, *kv;
+    int dtype, Ha, Dqk, Dv, topk;
+    const int *idx, *cu_q, *cu_kv;
+    int S;
+    double scale;
+    const long long *rows;
+    int nrows;
+    double *o, *lse;
+    int next, rc;
+    pthread_mutex_t lock;
+} attn_job_t;
+
+/* One query row r, every head:
+ *   z_j = scale * sum_i q[r,h,i] * kv[row_j, i]   for the listed j (idx >= 0),
+ *         row_j = cu_kv[b] + idx[r, j], b the request of r (cu_q);
+ *   o[h, c] = sum_j exp(z_j - m) * kv[row_j, c] / sum_j exp(z_j - m), c < Dv,
+ *   lse[h]  = m + log(sum_j exp(z_j - m)),  m = max_j z_j.
+ * A row with no listed position gets o = 0 and lse = -inf.  Each listed
+ * entry is one term (a position listed twice counts twice). */
+static int attn_row(attn_job_t *J, int i) {
+    long long r = J->rows[i];
+    int b = find_request(J->cu_q, J->S, r);
+    int nkv = J->cu_kv[b + 1] - J->cu_kv[b];
+    const int *ix = J->idx + (size_t)r * J->topk;
+    double *z = (double *)malloc(sizeof(double) * (size_t)(J->topk > 0 ? J->topk : 1));
+    if (!z) return 2;
+    for (int j = 0; j < J->topk; ++j)
+        if (ix[j] >= nkv) { free(z); return 1; }
+    for (int h = 0; h < J->Ha; ++h) {
+        double *o = J->o + ((size_t)i * J->Ha + h) * J->Dv;
+        for (int c = 0; c < J->Dv; ++c) o[c] = 0.0;
+        double m = -INFINITY;
+        for (int j = 0; j < J->topk; ++j) {
+            if (ix[j] < 0) continue;
+            size_t kr = (size_t)(J->cu_kv[b] + ix[j]) * J->Dqk;
+            size_t qr = ((size_t)r * J->Ha + h) * J->Dqk;
+            double dot = 0.0;
+            for (int e = 0; e < J->Dqk; ++e)
+                dot += load_elem(J->q, J->dtype, qr + e) * load_elem(J->kv, J->dtype, kr + e);
+            z[j] = J->scale * dot;
+            if (z[j] > m) m = z[j];
+        }
+        if (m == -INFINITY) {
+            J->lse[(size_t)i * J->Ha + h] = -INFINITY;
+            continue;
+        }
+        double l = 0.0;
+        for (int j = 0; j < J->topk; ++j) {
+            if (ix[j] < 0) continue;
+            double p = exp(z[j] - m);
+            l += p;
+            size_t kr = (size_t)(J->cu_kv[b] + ix[j]) * J->Dqk;
+            for (int c = 0; c < J->Dv; ++c) o[c] += p * load_elem(J->kv, J->dtype, kr + c);
+        }
+        for (int c = 0; c < J->Dv; ++c) o[c] /= l;
+        J->lse[(size_t)i * J->Ha + h] = m + log(l);
+    }
+    free(z);
+    return 0;
+}
+
+static void *attn_worker(void *arg) {
+    attn_job_t *J = (attn_job_t *)arg;
+    for (;;) {
+        pthread_mutex_lock(&J->lock);
+        int i = J->next++;
+        pthread_mutex_unlock(&J->lock);
+        if (i >= J->nrows) break;
+        int rc = attn_row(J, i);
+        if (rc) {
+            pthread_mutex_lock(&J->lock);
+            if (!J->rc) J->rc = rc;
+            pthread_mutex_unlock(&J->lock);
+        }
+    }
+    return NULL;
+}
+
+/* Token-sparse attention for the given query rows.
+ *   q [R, Ha, Dqk], kv [Nkv, Dqk] (bf16 bits or fp32); idx [R, topk] int32
+ *   positions inside the row's request (-1 = no entry); cu_q, cu_kv host
+ *   [S+1]: query rows cu_q[b] .. cu_q[b+1]-1 read kv rows cu_kv[b] + idx.
+ *   o [nrows, Ha, Dv] and lse [nrows, Ha] in double. */
+int ora_sparse_attn(const void *q, const void *kv, int dtype, const int *idx, const int *cu_q, const int *cu_kv,
+                    int S, int Ha, int Dqk, int Dv, int topk, double scale, const long long *rows, int nrows,
+                    double *o, double *lse, int nthreads) {
+    if (!q || !kv || !idx || !o || !lse || (nrows > 0 && !rows) || Ha <= 0 || Dqk <= 0 || Dv <= 0 ||
+        Dv > Dqk || topk <= 0)
+        return 1;
+    if (check_requests(cu_q, S) || check_requests(cu_kv, S)) return 1;
+    for (int i = 0; i < nrows; ++i)
+        if (rows[i] < 0 || rows[i] >= cu_q[S]) return 1;
+    attn_job_t J;
+    memset(&J, 0, sizeof J);
+    J.q = q; J.kv = kv; J.dtype = dtype; J.Ha = Ha; J.Dqk = Dqk; J.Dv = Dv; J.topk = topk;
+    J.idx = idx; J.cu_q = cu_q; J.cu_kv = cu_kv; J.S = S; J.scale = scale; J.rows = rows; J.nrows = nrows;
+    J.o = o; J.lse = lse;
+    if (nthreads < 1) nthreads = 1;
+    if (nthreads > 256) nthreads = 256;
+    pthread_t th[256];
+    pthread_mutex_init(&J.lock, NULL);
+    int started = 0;
+    for (int t = 0; t < nthreads; ++t)
+        if (pthread_create(&th[t], NULL, attn_worker, &J) == 0) ++started;
+    if (!started) attn_worker(&J);
+    for (int t = 0; t < started; ++t) pthread_join(th[t], NULL);
+    pthread_mutex_destroy(&J.lock);
+    return J.rc;
 }

@@ -388,6 +388,87 @@ def pin_block_partial_closed_form():
     assert checked > 20
 
 
+def pin_attn_single_entry():
+    """One listed position: the output is that key's value part exactly and lse
+    its scaled logit (integer inputs: every product and sum is exact)."""
+    rng = np.random.default_rng(43)
+    R, Ha, Dqk, Dv = 3, 4, 24, 16
+    qi = rng.integers(-4, 5, size=(R, Ha, Dqk))
+    ki = rng.integers(-4, 5, size=(10, Dqk))
+    q, kv = _bf(qi.astype(np.float32)), _bf(ki.astype(np.float32))
+    idx = np.full((R, 4), -1, np.int32)
+    idx[:, 2] = [3, 0, 9]
+    o, lse = O.sparse_attn(q, kv, idx, [0, R], [0, 10], Dv, 0.125)
+    for r in range(R):
+        j = idx[r, 2]
+        assert np.array_equal(o[r], np.repeat(ki[j, :Dv][None].astype(np.float64), Ha, 0)), r
+        for h in range(Ha):
+            assert lse[r, h] == 0.125 * int((qi[r, h] * ki[j]).sum()), (r, h)
+
+
+def pin_attn_equal_logits_mean():
+    """q = 0: every logit is 0, so o is the plain mean of the listed value rows
+    (a position listed twice counts twice) and lse = log(number listed)."""
+    rng = np.random.default_rng(47)
+    R, Ha, Dqk, Dv, N = 4, 2, 32, 24, 20
+    kv = _bf(rng.standard_normal((N, Dqk)).astype(np.float32))
+    q = np.zeros((R, Ha, Dqk), np.uint16)
+    idx = np.array([[0, 5, 5, -1, 19], [-1, -1, 7, -1, -1], [1, 2, 3, 4, 6], [19, -1, 0, 0, 0]], np.int32)
+    o, lse = O.sparse_attn(q, kv, idx, [0, R], [0, N], Dv, 0.7)
+    vf = W.bf16_to_f32(kv).astype(np.float64)[:, :Dv]
+    for r in range(R):
+        sel = idx[r][idx[r] >= 0]
+        want = vf[sel].mean(axis=0)
+        for h in range(Ha):
+            assert np.allclose(o[r, h], want, rtol=1e-14, atol=1e-15), r
+            assert abs(lse[r, h] - math.log(len(sel))) < 1e-15, r
+
+
+def pin_attn_library_sdpa():
+    """Two packed requests of random bf16 inputs: the library's scaled
+    dot-product attention (torch, float64, CPU) over the gathered rows."""
+    import torch
+    rng = np.random.default_rng(53)
+    Ha, Dqk, Dv, topk = 4, 48, 32, 12
+    cu_q = np.array([0, 5, 9], np.int32)
+    cu_kv = np.array([0, 30, 47], np.int32)
+    q = _bf(rng.standard_normal((9, Ha, Dqk)).astype(np.float32))
+    kv = _bf(rng.standard_normal((47, Dqk)).astype(np.float32))
+    idx = np.full((9, topk), -1, np.int32)
+    for r in range(9):
+        b = 0 if r < 5 else 1
+        n = cu_kv[b + 1] - cu_kv[b]
+        m = rng.integers(1, topk + 1)
+        idx[r, :m] = rng.choice(n, size=m, replace=False)
+    scale = 0.3
+    o, lse = O.sparse_attn(q, kv, idx, cu_q, cu_kv, Dv, scale)
+    qf = torch.from_numpy(W.bf16_to_f32(q).astype(np.float64))
+    kf = torch.from_numpy(W.bf16_to_f32(kv).astype(np.float64))
+    for r in range(9):
+        b = 0 if r < 5 else 1
+        rows = torch.from_numpy((cu_kv[b] + idx[r][idx[r] >= 0]).astype(np.int64))
+        K = kf[rows]
+        want = torch.nn.functional.scaled_dot_product_attention(qf[r][None], K[None], K[None, :, :Dv], scale=scale)[0]
+        assert np.allclose(o[r], want.numpy(), rtol=1e-12, atol=1e-13), r
+        wl = torch.logsumexp(scale * qf[r] @ K.T, dim=-1)
+        assert np.allclose(lse[r], wl.numpy(), rtol=1e-13, atol=1e-13), r
+
+
+def pin_attn_large_logits():
+    """Logit gaps far beyond exp's range: the dominant key's value comes out
+    exactly and lse equals its logit."""
+    Dqk, Dv = 24, 16
+    kv = np.zeros((6, Dqk), np.float32)
+    kv[4] = 8.0
+    kv[:, :Dv] += np.arange(Dv, dtype=np.float32)[None] / 4
+    kv[4, :Dv] = np.arange(Dv, dtype=np.float32) - 3
+    q = np.full((1, 1, Dqk), 8.0, np.float32)
+    q16, kv16 = _bf(q), _bf(kv)
+    o, lse = O.sparse_attn(q16, kv16, np.array([[0, 4, 1, 5]], np.int32), [0, 1], [0, 6], Dv, 1.0)
+    assert np.array_equal(o[0, 0], kv[4, :Dv].astype(np.float64))
+    assert lse[0, 0] == float((q[0, 0].astype(np.float64) * kv[4]).sum())
+
+
 def pin_gaussian_mean_score():
     """i.i.d. Gaussian q, k: E[I] = sum_j w_j * sigma / sqrt(2 pi), sigma^2 = d var_q var_k."""
     P = W.small_fp32(L=512, H=4, d=64, topk=8, seed=23)
@@ -408,7 +489,8 @@ ALL_PINS = [pin_hand_scores, pin_hand_topk, pin_hand_decode, pin_bruteforce_dens
             pin_pivot_special_cases, pin_invariants, pin_reuse_within_proxy_ranking,
             pin_proxy_exact_mean, pin_decode_matches_prefill, pin_gaussian_mean_score,
             pin_block_mean_exact, pin_block_reductions, pin_block_constant_keys_equal_refine,
-            pin_block_partial_closed_form]
+            pin_block_partial_closed_form, pin_attn_single_entry, pin_attn_equal_logits_mean,
+            pin_attn_library_sdpa, pin_attn_large_logits]
 
 
 @pytest.mark.parametrize("pin", ALL_PINS, ids=[p.__name__ for p in ALL_PINS])
@@ -441,6 +523,12 @@ MUTANTS = {
     "block_rank_by_position": ("qsort(pc, (size_t)nfull, sizeof(cand_t), by_score_desc_pos_asc);", ""),
     "block_member_mask_dropped": ("                if (s > t) continue;\n                mc[m].score", "                mc[m].score"),
     "block_keys_from_block_start_only": ("int s = pc[i].pos * bn + r;", "int s = pc[i].pos * bn;"),
+    "attn_no_max_shift": ("double p = exp(z[j] - m);", "double p = exp(z[j]);"),
+    "attn_value_from_tail": ("o[c] += p * load_elem(J->kv, J->dtype, kr + c);",
+                             "o[c] += p * load_elem(J->kv, J->dtype, kr + (J->Dqk - J->Dv) + c);"),
+    "attn_scale_dropped": ("z[j] = J->scale * dot;", "z[j] = dot;"),
+    "attn_request_lookup_dropped": ("int b = find_request(J->cu_q, J->S, r);", "int b = 0;"),
+    "attn_normaliser_dropped": ("for (int c = 0; c < J->Dv; ++c) o[c] /= l;", ""),
 }
 
 
