@@ -12,7 +12,9 @@ G=2 MTP queries, dense and Refine c=4096, and dense over the same cache
 scattered into 64-key pages behind a block table) is timed after it and
 reported under "decode" as HBM GB/s of the cache scan.  The block
 pre-filter variant of Refine (candidates from 64-key block means) runs on
-the same packed batch under "block_prefilter", outside the step.
+the same packed batch under "block_prefilter", outside the step, and the
+token-sparse attention (absorbed-MLA shapes: 128 heads, 576/512 dims) over
+the dense selections of the last 16384 query rows under "sparse_attn".
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
@@ -53,6 +55,8 @@ def parse():
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-decode", action="store_true")
     p.add_argument("--no-block", action="store_true")
+    p.add_argument("--no-attn", action="store_true")
+    p.add_argument("--attn-rows", type=int, default=16384)
     p.add_argument("--cpu-rows", type=int, default=64, help="oracle sample rows (dense + refine) per CPU step")
     p.add_argument("--no-cpu", action="store_true", help="skip the CPU-oracle baseline")
     p.add_argument("--tokens", type=int, default=L_TOK,
@@ -386,6 +390,52 @@ def main():
                "kernels": {n: {"launches": c, "ms_per_step": t / args.steps} for n, (c, t) in trb.items()}}
         del ws3, o3
 
+    # ------------------------------- token-sparse attention on the selections
+    att = None
+    if do_dense and not args.no_attn:
+        Ra = min(args.attn_rows, L)
+        gen = torch.Generator(device=dev)
+        gen.manual_seed(4321 + rank)
+        qa = torch.randn(Ra, 128, 576, generator=gen, device=dev).to(torch.bfloat16)
+        kva = torch.randn(L, 576, generator=gen, device=dev).to(torch.bfloat16)
+        sel = o1[L - Ra:]  # the dense indexer's selections of the last Ra query rows
+        cq = torch.tensor([0, Ra], dtype=torch.int32, device=dev)
+        ck = torch.tensor([0, L], dtype=torch.int32, device=dev)
+        oa = torch.empty(Ra, 128, 512, dtype=torch.bfloat16, device=dev)
+        wsa = torch.empty(256, dtype=torch.uint8, device=dev)
+        sc = 1.0 / math.sqrt(192.0)
+
+        def astep():
+            idx.sparse_attn(qa, kva, sel, cq, ck, sc, out=oa, workspace=wsa)
+
+        for _ in range(args.warmup):
+            astep()
+        torch.cuda.synchronize()
+        assert idx.device_status(wsa) == "IDX_OK"
+        nvalid = int((sel >= 0).sum().item())
+        barrier()
+        lib.idx_trace_enable(1)
+        e0.record(stream)
+        for _ in range(args.steps):
+            astep()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        lib.idx_trace_enable(0)
+        barrier()
+        ams = max_over_ranks(e0.elapsed_time(e1) / args.steps)
+        _, tra = trace_report(lib)
+        kms = sum(t for n, (c, t) in tra.items() if n.endswith("attn_tc")) / args.steps
+        useful = 2.0 * 128 * nvalid * (576 + 512)  # logits + weighted values, per listed key and head
+        issued = 2.0 * 128 * (Ra * 2048) * (2 * 576 + 512)  # each value half recomputes the logits
+        tf = useful / (kms / 1000.0) / 1e12 if kms > 0 else None
+        att = {"workload": f"sparse_mla_attn_rows{Ra}_H128_dqk576_dv512_k2048_kv{L}",
+               "indices": "dense indexer top-2048 of the last rows of the 131072-token request",
+               "ms_per_step": ams, "kernel_ms": kms, "rows_per_s": world * Ra / (ams / 1000.0),
+               "useful_flops": useful, "issued_flops": issued, "tflops_useful": tf,
+               "frac_bf16_sustained": (tf / bf16_sus) if tf else None,
+               "kernels": {n: {"launches": c, "ms_per_step": t / args.steps} for n, (c, t) in tra.items()}}
+        del qa, kva, oa
+
     # ------------------------------------------------------------- decode
     dec = None
     if not args.no_decode:
@@ -449,7 +499,7 @@ def main():
                    "g": G_REF, "c": C_REF, "parallelism": f"dp{world} (independent batches)",
                    "l2": "inputs larger than L2 (q is 2 GiB)"},
         "tflops_dense": achieved, "roofline": roof, "cpu_baseline": cpu, "e2e": e2e, "clocks": clk,
-        "gpu_launches": nlaunch, "kernels": per_kernel, "block_prefilter": blk, "decode": dec,
+        "gpu_launches": nlaunch, "kernels": per_kernel, "block_prefilter": blk, "sparse_attn": att, "decode": dec,
     }
     if rank == 0:
         print(json.dumps(line))

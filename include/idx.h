@@ -198,6 +198,41 @@ idx_status idx_decode_topk_noalloc(const void *q, const void *kcache, const int 
                                    int B, int G, int n_max, int H, int d, int topk, idx_dtype dtype,
                                    int *out_idx, float *out_score, idx_stream_t stream);
 
+/* --------------------------------------------- token-sparse attention */
+
+/* Workspace bytes for idx_sparse_attn (its status word). */
+size_t idx_sparse_attn_workspace_size(void);
+
+/* Attention of each query row restricted to its selected positions: the
+ * consumer of the top-k sets (PIVOT page, introduction: the selected set
+ * feeds sparse MLA attention).  The pages give no formula; the reading is
+ * softmax attention over the listed keys in the absorbed-MLA form of the
+ * production models that page names: one latent row per key is the key
+ * (all Dqk dims) and its first Dv dims the value, shared by all heads.
+ *   z_j      = scale * q[r,h,:] . kv[cu_kv[b] + idx[r,j], :]   (idx[r,j] >= 0)
+ *   out[r,h] = sum_j softmax_j(z) * kv[cu_kv[b] + idx[r,j], :Dv]
+ *   lse[r,h] = log sum_j exp(z_j)   (natural log; -inf for a row with no entry)
+ * where b is the request of query row r (cu_q[b] <= r < cu_q[b+1]).
+ *   q       [R, H, Dqk] bf16        query rows
+ *   kv      [Nkv, Dqk] bf16         latent rows of all requests
+ *   idx     [R, topk] int32         positions inside the row's request; -1 =
+ *                                   no entry (anywhere in the row); an entry
+ *                                   listed twice counts twice.  The output of
+ *                                   idx_dense_topk / idx_pivot_topk (cu_q =
+ *                                   cu_kv = cu_seqlens) or idx_decode_topk
+ *                                   (cu_q = [0, G, 2G, ..], cu_kv = [0, n_max,
+ *                                   2 n_max, ..]) fits as is.
+ *   cu_q, cu_kv [num_seqs+1] int32  device request boundaries
+ *   out     [R, H, Dv] bf16; lse [R, H] fp32 or NULL
+ * Supported: bf16, Dqk = 576, Dv = 512, 1 <= H <= 128 (tensor cores);
+ * other shapes return IDX_ERR_UNSUPPORTED.  Positions >= the request's kv
+ * length and malformed boundaries are skipped and flagged as
+ * IDX_ERR_INVALID in the device status word of ws. */
+idx_status idx_sparse_attn(const void *q, const void *kv, const int *idx, const int *cu_q,
+                           const int *cu_kv, int num_seqs, int R, long long Nkv, int H, int Dqk,
+                           int Dv, int topk, float scale, idx_dtype dtype, void *out, float *lse,
+                           void *ws, size_t ws_bytes, idx_stream_t stream);
+
 /* ------------------------------------------------------ status, debug */
 
 /* Synchronises `stream`, returns the device status recorded in `ws` by the

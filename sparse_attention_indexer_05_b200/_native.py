@@ -25,6 +25,9 @@ SIGNATURES = {
                              _vp]),
     "idx_decode_paged_topk": (_i, [_vp, _vp, _ip, _ip, _fp, _i, _i, _i, _i, _ll, _i, _i, _i, _i, _i, _i, _ip,
                                    _fp, _vp, _sz, _vp]),
+    "idx_sparse_attn_workspace_size": (_sz, []),
+    "idx_sparse_attn": (_i, [_vp, _vp, _ip, _ip, _ip, _i, _i, _ll, _i, _i, _i, _i, ctypes.c_float, _i, _vp, _fp,
+                             _vp, _sz, _vp]),
     "idx_device_status": (_i, [_vp, _vp]),
     "idx_status_string": (ctypes.c_char_p, [_i]),
     "idx_debug_scores": (_i, [_i, _vp, _vp, _fp, _ip, _i, _i, _i, _i, _i, _i, _i, _i, _ip, _i, _fp, _ll,

@@ -493,6 +493,29 @@ idx_status idx_decode_paged_topk(const void *q, const void *kpool, const int *bl
     return D.run(out_idx, out_score);
 }
 
+size_t idx_sparse_attn_workspace_size(void) { return kAlign; }
+
+idx_status idx_sparse_attn(const void *q, const void *kv, const int *idx, const int *cu_q, const int *cu_kv,
+                           int num_seqs, int R, long long Nkv, int H, int Dqk, int Dv, int topk, float scale,
+                           idx_dtype dtype, void *out, float *lse, void *ws, size_t ws_bytes, idx_stream_t stream) {
+    if (!q || !kv || !idx || !cu_q || !cu_kv || !out) return IDX_ERR_INVALID;
+    if (num_seqs < 1 || R < 0 || Nkv < 1 || H < 1 || Dqk < 1 || Dv < 1 || Dv > Dqk || topk < 1 || !isfinite(scale))
+        return IDX_ERR_INVALID;
+    if (dtype != IDX_BF16 && dtype != IDX_F32) return IDX_ERR_INVALID;
+    if (!attn_tc_supported(H, Dqk, Dv, (int)dtype) || (long long)R * 128 > 0x7FFFFFFFLL) return IDX_ERR_UNSUPPORTED;
+    if (!ws || (reinterpret_cast<uintptr_t>(ws) % kAlign) != 0 || ws_bytes < kAlign) return IDX_ERR_WORKSPACE;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    TracePhase phase("sparse_attn");
+    unsigned *status = static_cast<unsigned *>(ws);
+    TRY_CUDA(cudaMemsetAsync(status, 0, 4, st));
+    if (R == 0) return IDX_OK;
+    SparseAttnArgs a{};
+    a.q = q; a.kv = kv; a.idx = idx; a.cu_q = cu_q; a.cu_kv = cu_kv;
+    a.S = num_seqs; a.R = R; a.H = H; a.topk = topk; a.Nkv = Nkv; a.scale = scale;
+    a.out = out; a.lse = lse; a.status = status;
+    return cuda_st(launch_sparse_attn_tc(a, st));
+}
+
 idx_status idx_device_status(const void *ws, idx_stream_t stream) {
     if (!ws) return IDX_ERR_WORKSPACE;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);

@@ -1,0 +1,415 @@
+// attn_tc.cu -- token-sparse attention over the selected positions, the
+// consumer of the indexer's top-k sets (PIVOT page, introduction: the chosen
+// set feeds sparse MLA attention).  Absorbed-MLA form: one latent row per key
+// (Dqk = 576 dims) is the key and its first Dv = 512 dims the value, shared
+// by all heads:
+//     z_j   = scale * q[r,h] . kv[row_j],   row_j = cu_kv[b] + idx[r, j] (idx >= 0)
+//     o[r,h] = sum_j softmax_j(z) * kv[row_j, :Dv],   lse[r,h] = log sum_j exp(z_j)
+//
+// One CTA per (query row, half of the value dimensions).  The 128 heads of
+// the row are the MMA's M; the row's Q (128 x 576 bf16, 144 KB) stays in
+// shared memory for the whole row.  Per chunk of 32 selected keys:
+//   S  = Q K^T      tcgen05, M=128, N=32, K=576 (36 steps)   -> TMEM, 2 buffers
+//   P  = exp2(S*scale*log2e - m), m a running row maximum that is only moved
+//        (and O rescaled in TMEM) when it grows by more than 8, so that P <= 2^8
+//   O += P V_half   tcgen05, M=128, N=256, K=32 (2 steps)   -> TMEM, 256 cols
+// The key rows of a chunk are gathered by cp.async (16-byte pieces, rows of
+// -1 or out-of-range positions zero-filled) into the 128-byte-swizzled
+// K-major layout; the same buffer is the value operand of the second MMA
+// through an MN-major descriptor.  P goes to shared memory as bf16 in the
+// unswizzled K-major layout (8x16-byte core matrices).
+//
+// Roles (288 threads): warp 0 = MMA issuer (one lane) and TMEM owner;
+// warps 1..4 = softmax and epilogue, one head row per thread (TMEM lane
+// quarter = warp % 4); warps 5..8 = gather, two groups of two warps that
+// fill the two key stages alternately.  Every wait is bounded.
+#include <cudaTypedefs.h>
+#include <math.h>
+#include <string.h>
+
+#include "common.cuh"
+#include "internal.h"
+#include "tc.cuh"
+
+namespace idx {
+
+namespace {
+
+constexpr int A_H = 128;                    // head rows on M (fewer heads: the rest is computed, not stored)
+constexpr int A_DQK = 576;
+constexpr int A_DV = 512;
+constexpr int A_DVH = 256;                  // value dims per CTA
+constexpr int A_KC = 32;                    // keys per chunk
+constexpr int A_SLICES = A_DQK / 64;        // 64-dim slices of a 128-byte swizzled row
+constexpr int A_STAGES = 2;
+constexpr uint32_t kQSlice = A_H * 128;              // 16 KB
+constexpr uint32_t kQBytes = A_SLICES * kQSlice;     // 144 KB
+constexpr uint32_t kKSlice = A_KC * 128;             // 4 KB
+constexpr uint32_t kKStage = A_SLICES * kKSlice;     // 36 KB
+constexpr uint32_t kPBytes = A_H * A_KC * 2;         // 8 KB
+constexpr int kSoftWarps = 4;
+constexpr int kGatherWarps = 4;
+constexpr int kThreads = 32 * (1 + kSoftWarps + kGatherWarps);
+constexpr int kGroupThreads = 32 * kGatherWarps / A_STAGES;  // gather threads per stage group
+constexpr uint32_t kColS = 0;               // S buffers: columns [0, 64)
+constexpr uint32_t kColO = 256;             // O: columns [256, 512)
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kRescale = 8.0f;            // move the running max only past this growth (log2 units)
+
+struct __align__(8) AttnShared {
+    uint64_t qfull, kfull[A_STAGES], kempty[A_STAGES], sfull[2], sfree[2], pfull, pdone, drain;
+    uint32_t tmem_base;
+    int abort;
+};
+
+constexpr size_t kOffQ = 0;
+constexpr size_t kOffK = kOffQ + kQBytes;
+constexpr size_t kOffP = kOffK + (size_t)A_STAGES * kKStage;
+constexpr size_t kOffCtl = kOffP + kPBytes;
+constexpr size_t kSmemBytes = kOffCtl + sizeof(AttnShared) + 1024;
+static_assert(kSmemBytes <= 232448, "shared memory of one CTA");
+
+// K-major operand stored as 8-row x 16-byte core matrices without swizzle:
+// stride between K-adjacent core matrices `lbo`, between 8-row groups `sbo`.
+__device__ __forceinline__ uint64_t kmajor_plain_desc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+    uint64_t d = 0;
+    d |= (uint64_t)((saddr >> 4) & 0x3FFFu);
+    d |= (uint64_t)((lbo >> 4) & 0x3FFFu) << 16;
+    d |= (uint64_t)((sbo >> 4) & 0x3FFFu) << 32;
+    d |= (uint64_t)1u << 46;
+    return d;  // swizzle mode 0
+}
+
+// MN-major operand in the 128-byte swizzle: rows of 128 bytes along MN (64
+// elements), 8 K-rows per 1024-byte atom; `lbo` = stride between 64-element
+// MN blocks, 1024 B between 8-row K groups.
+__device__ __forceinline__ uint64_t mnmajor_sw128_desc(uint32_t saddr, uint32_t lbo) {
+    uint64_t d = 0;
+    d |= (uint64_t)((saddr >> 4) & 0x3FFFu);
+    d |= (uint64_t)((lbo >> 4) & 0x3FFFu) << 16;
+    d |= (uint64_t)(1024u >> 4) << 32;
+    d |= (uint64_t)1u << 46;
+    d |= (uint64_t)2u << 61;
+    return d;
+}
+
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void *src, uint32_t src_bytes) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
+__device__ __forceinline__ void fence_proxy_async() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+        "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, "
+        "%17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};" ::"r"(taddr),
+        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),
+        "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]), "r"(r[16]),
+        "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]),
+        "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
+        : "memory");
+}
+__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+__device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
+    const __nv_bfloat162 v = __floats2bfloat162_rn(a, b);
+    return *reinterpret_cast<const uint32_t *>(&v);
+}
+
+// The request of query row r and its key range; false for malformed
+// boundaries (the row is then written as zeros and flagged).
+__device__ __forceinline__ bool locate(const int *cu_q, const int *cu_kv, int S, int R, long long Nkv, int r,
+                                      long long &kv0, int &nkv) {
+    int lo = 0, hi = S;
+    while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if (cu_q[mid] <= r) lo = mid; else hi = mid;
+    }
+    const bool ok = cu_q[lo] <= r && r < cu_q[lo + 1] && cu_q[S] <= R && cu_kv[lo] >= 0 &&
+                    cu_kv[lo] <= cu_kv[lo + 1] && (long long)cu_kv[lo + 1] <= Nkv;
+    kv0 = ok ? cu_kv[lo] : 0;
+    nkv = ok ? cu_kv[lo + 1] - cu_kv[lo] : 0;
+    return ok;
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+    attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, SparseAttnArgs a) {
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw = tc::smem_u32(smem_raw);
+    uint8_t *smem = smem_raw + (((raw + 1023u) & ~1023u) - raw);
+    uint8_t *qs = smem + kOffQ;
+    uint8_t *ks = smem + kOffK;
+    uint8_t *ps = smem + kOffP;
+    AttnShared &sh = *reinterpret_cast<AttnShared *>(smem + kOffCtl);
+    volatile int *abort = &sh.abort;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int r = blockIdx.x >> 1, half = blockIdx.x & 1;
+    const int nch = (a.topk + A_KC - 1) / A_KC;
+    long long kv0;
+    int nkv;
+    const bool row_ok = locate(a.cu_q, a.cu_kv, a.S, a.R, a.Nkv, r, kv0, nkv);
+    const int *ix = a.idx + (long long)r * a.topk;
+
+    if (threadIdx.x == 0) {
+        tc::mbar_init(&sh.qfull, 1);
+        for (int s = 0; s < A_STAGES; ++s) {
+            tc::mbar_init(&sh.kfull[s], kGroupThreads);
+            tc::mbar_init(&sh.kempty[s], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            tc::mbar_init(&sh.sfull[b], 1);
+            tc::mbar_init(&sh.sfree[b], 32 * kSoftWarps);
+        }
+        tc::mbar_init(&sh.pfull, 32 * kSoftWarps);
+        tc::mbar_init(&sh.pdone, 1);
+        tc::mbar_init(&sh.drain, 1);
+        sh.abort = 0;
+        tc::fence_mbar_init();
+        if (!row_ok) raise_status(a.status, ST_INVALID);
+    }
+    if (warp == 0) {
+        tc::tmem_alloc(&sh.tmem_base, 512);
+        tc::tmem_relinquish();
+    }
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    const uint32_t tmem = sh.tmem_base;
+
+    if (warp == 0) {
+        // ------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            tc::prefetch_tmap(&tmap_q);
+            tc::mbar_arrive_expect_tx(&sh.qfull, kQBytes);
+            for (int s = 0; s < A_SLICES; ++s)
+                tc::tma_load_2d(qs + s * kQSlice, &tmap_q, s * 64, r * a.H, &sh.qfull);
+            const uint32_t idesc_s = tc::idesc_bf16_f32(A_H, A_KC);
+            const uint32_t idesc_o = tc::idesc_bf16_f32(A_H, A_DVH) | (1u << 16);  // value operand MN-major
+            const uint32_t qa = tc::smem_u32(qs), ka = tc::smem_u32(ks), pa = tc::smem_u32(ps);
+            bool ok = tc::mbar_wait(&sh.qfull, 0, abort, a.status);
+            for (int j = 0; ok && j <= nch; ++j) {
+                if (j < nch) {
+                    const int st = j % A_STAGES, sb = j & 1;
+                    if (!(ok = tc::mbar_wait(&sh.kfull[st], (j / A_STAGES) & 1u, abort, a.status))) break;
+                    if (!(ok = tc::mbar_wait(&sh.sfree[sb], ((j >> 1) & 1u) ^ 1u, abort, a.status))) break;
+                    tc::fence_after_sync();
+                    for (int kk = 0; kk < A_DQK / 16; ++kk) {
+                        const uint32_t off = (kk & 3) * 32u;  // 16-element K step inside the 128-byte row
+                        const uint64_t ad = tc::sw128_desc(qa + (kk >> 2) * kQSlice + off);
+                        const uint64_t bd = tc::sw128_desc(ka + st * kKStage + (kk >> 2) * kKSlice + off);
+                        tc::mma_bf16(tmem + kColS + sb * A_KC, ad, bd, idesc_s, kk > 0 ? 1u : 0u);
+                    }
+                    tc::mma_commit(&sh.sfull[sb]);
+                }
+                if (j >= 1) {
+                    const int jp = j - 1, st = jp % A_STAGES;
+                    if (!(ok = tc::mbar_wait(&sh.pfull, jp & 1u, abort, a.status))) break;
+                    tc::fence_after_sync();
+                    const uint32_t vbase = ka + st * kKStage + (4 * half) * kKSlice;
+                    for (int kk = 0; kk < A_KC / 16; ++kk) {
+                        const uint64_t ad = kmajor_plain_desc(pa + kk * 256u, 128u, 512u);
+                        const uint64_t bd = mnmajor_sw128_desc(vbase + kk * 16u * 128u, kKSlice);
+                        tc::mma_bf16(tmem + kColO, ad, bd, idesc_o, (jp > 0 || kk > 0) ? 1u : 0u);
+                    }
+                    tc::mma_commit(&sh.kempty[st]);
+                    tc::mma_commit(&sh.pdone);
+                }
+            }
+            // drain: every MMA issued so far has completed before TMEM is released
+            tc::mma_commit(&sh.drain);
+            tc::mbar_wait_drain(&sh.drain, 0);
+            tc::mbar_wait_drain(&sh.qfull, 0);
+        }
+        __syncwarp();
+    } else if (warp <= kSoftWarps) {
+        // ---------------------------------------- softmax and epilogue
+        const int quarter = warp & 3;
+        const int h = quarter * 32 + lane;
+        const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
+        const float sl2 = a.scale * kLog2e;
+        float m_used = -INFINITY, l = 0.0f;
+        bool ok = true;
+        uint32_t s[32];
+        for (int j = 0; j < nch; ++j) {
+            const int sb = j & 1;
+            if (lane == 0) ok = tc::mbar_wait(&sh.sfull[sb], (j >> 1) & 1u, abort, a.status);
+            ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
+            if (!ok) break;
+            tc::fence_after_sync();
+            tc::tmem_ld32(tmem + lane_off + kColS + sb * A_KC, s);
+            tc::tmem_wait_ld(s);
+            tc::fence_before_sync();
+            tc::mbar_arrive(&sh.sfree[sb]);
+            // which keys of the chunk are listed and inside the request
+            const int pos = j * A_KC + lane < a.topk ? ix[j * A_KC + lane] : -1;
+            const bool bad = pos >= nkv;
+            if (bad && half == 0 && quarter == 0) raise_status(a.status, ST_INVALID);
+            const unsigned valid = __ballot_sync(0xFFFFFFFFu, row_ok && pos >= 0 && !bad);
+            float x[32];
+            float mx = -INFINITY;
+#pragma unroll
+            for (int c = 0; c < 32; ++c) {
+                x[c] = (valid >> c) & 1u ? __uint_as_float(s[c]) * sl2 : -INFINITY;
+                mx = fmaxf(mx, x[c]);
+            }
+            if (j >= 1) {
+                if (lane == 0) ok = tc::mbar_wait(&sh.pdone, (j - 1) & 1u, abort, a.status);
+                ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
+                if (!ok) break;
+                tc::fence_after_sync();
+            }
+            const bool need = mx > m_used + kRescale;
+            const float factor = need ? exp2f(m_used - mx) : 1.0f;  // 0 while nothing was listed yet
+            if (j >= 1 && __any_sync(0xFFFFFFFFu, need)) {
+                uint32_t o[32];
+                for (int b = 0; b < A_DVH / 32; ++b) {
+                    tc::tmem_ld32(tmem + lane_off + kColO + b * 32, o);
+                    tc::tmem_wait_ld(o);
+#pragma unroll
+                    for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * factor);
+                    tmem_st32(tmem + lane_off + kColO + b * 32, o);
+                }
+                tmem_wait_st();
+            }
+            if (need) {
+                l *= factor;
+                m_used = mx;
+            }
+            float p[32];
+#pragma unroll
+            for (int c = 0; c < 32; ++c) {
+                p[c] = x[c] == -INFINITY ? 0.0f : exp2f(x[c] - m_used);
+                l += p[c];
+            }
+            // P row h: core matrix (h/8, c/8) at (h/8)*512 + (c/8)*128, row h%8 at +16*(h%8)
+            uint8_t *prow = ps + (h >> 3) * 512 + (h & 7) * 16;
+#pragma unroll
+            for (int c8 = 0; c8 < 4; ++c8) {
+                uint4 v;
+                v.x = pack_bf16(p[8 * c8 + 0], p[8 * c8 + 1]);
+                v.y = pack_bf16(p[8 * c8 + 2], p[8 * c8 + 3]);
+                v.z = pack_bf16(p[8 * c8 + 4], p[8 * c8 + 5]);
+                v.w = pack_bf16(p[8 * c8 + 6], p[8 * c8 + 7]);
+                *reinterpret_cast<uint4 *>(prow + c8 * 128) = v;
+            }
+            fence_proxy_async();
+            tc::fence_before_sync();
+            tc::mbar_arrive(&sh.pfull);
+        }
+        // epilogue: O / l for this half of the value dims, lse from half 0
+        if (ok && nch > 0) {
+            if (lane == 0) ok = tc::mbar_wait(&sh.pdone, (nch - 1) & 1u, abort, a.status);
+            ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
+        }
+        if (ok) {
+            tc::fence_after_sync();
+            const float inv = l > 0.0f ? 1.0f / l : 0.0f;
+            __nv_bfloat16 *orow = reinterpret_cast<__nv_bfloat16 *>(a.out) + ((long long)r * a.H + h) * A_DV + half * A_DVH;
+            uint32_t o[32];
+            for (int b = 0; b < A_DVH / 32; ++b) {
+                if (nch > 0) {
+                    tc::tmem_ld32(tmem + lane_off + kColO + b * 32, o);
+                    tc::tmem_wait_ld(o);
+                } else {
+#pragma unroll
+                    for (int c = 0; c < 32; ++c) o[c] = 0u;
+                }
+                if (h < a.H) {
+                    uint4 *dst = reinterpret_cast<uint4 *>(orow + b * 32);
+#pragma unroll
+                    for (int q4 = 0; q4 < 4; ++q4) {
+                        uint4 v;
+                        v.x = pack_bf16(__uint_as_float(o[8 * q4 + 0]) * inv, __uint_as_float(o[8 * q4 + 1]) * inv);
+                        v.y = pack_bf16(__uint_as_float(o[8 * q4 + 2]) * inv, __uint_as_float(o[8 * q4 + 3]) * inv);
+                        v.z = pack_bf16(__uint_as_float(o[8 * q4 + 4]) * inv, __uint_as_float(o[8 * q4 + 5]) * inv);
+                        v.w = pack_bf16(__uint_as_float(o[8 * q4 + 6]) * inv, __uint_as_float(o[8 * q4 + 7]) * inv);
+                        dst[q4] = v;
+                    }
+                }
+            }
+            if (half == 0 && h < a.H && a.lse)
+                a.lse[(long long)r * a.H + h] = l > 0.0f ? (m_used + log2f(l)) * 0.69314718055994531f : -INFINITY;
+        }
+    } else {
+        // -------------------------------------------------- gather
+        const int gt = threadIdx.x - 32 * (1 + kSoftWarps);  // 0 .. 127
+        const int grp = gt / kGroupThreads, t = gt % kGroupThreads;
+        const uint8_t *kvb = reinterpret_cast<const uint8_t *>(a.kv);
+        bool ok = true;
+        for (int j = grp; j < nch; j += A_STAGES) {
+            const int st = j % A_STAGES;  // == grp
+            if (lane == 0) ok = tc::mbar_wait(&sh.kempty[st], ((j / A_STAGES) & 1u) ^ 1u, abort, a.status);
+            ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
+            if (!ok) break;
+            const uint32_t dst0 = tc::smem_u32(ks + st * kKStage);
+            // 32 rows x 72 pieces of 16 bytes; piece u: row u / 72, piece c = u % 72 (slice c / 8)
+            for (int u = t; u < A_KC * (A_DQK / 8); u += kGroupThreads) {
+                const int row = u / (A_DQK / 8), c = u % (A_DQK / 8);
+                const int k = j * A_KC + row;
+                const int pos = k < a.topk ? ix[k] : -1;
+                const bool valid = row_ok && pos >= 0 && pos < nkv;
+                const uint8_t *src = valid ? kvb + ((kv0 + pos) * A_DQK + c * 8) * 2 : kvb;
+                const uint32_t dst = dst0 + (c >> 3) * kKSlice + row * 128 + ((((c & 7) ^ (row & 7))) << 4);
+                cp_async16(dst, src, valid ? 16u : 0u);
+            }
+            cp_async_commit();
+            cp_async_wait_all();
+            fence_proxy_async();
+            tc::mbar_arrive(&sh.kfull[st]);
+        }
+        cp_async_wait_all();
+    }
+
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    if (warp == 0) tc::tmem_dealloc(tmem, 512);
+}
+
+// ------------------------------------------------------------------ host
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn_attn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    if (!fn) {
+        cudaDriverEntryPointQueryResult q;
+        void *p = nullptr;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    }
+    return fn;
+}
+
+}  // namespace
+
+bool attn_tc_supported(int H, int Dqk, int Dv, int dtype) {
+    return H >= 1 && H <= A_H && Dqk == A_DQK && Dv == A_DV && dtype == 0;
+}
+
+cudaError_t launch_sparse_attn_tc(const SparseAttnArgs &a, cudaStream_t st) {
+    if (a.R <= 0) return cudaSuccess;
+    if (!attn_tc_supported(a.H, A_DQK, A_DV, 0)) return cudaErrorInvalidValue;
+    // q [R * H, 576] bf16 rows, boxes of 64 columns x 128 rows (one row's heads,
+    // and for H < 128 rows of the next query or the zero fill past the end)
+    PFN_cuTensorMapEncodeTiled_v12000 fn = encode_fn_attn();
+    if (!fn) return cudaErrorInvalidValue;
+    CUtensorMap mq;
+    memset(&mq, 0, sizeof(mq));
+    cuuint64_t dims[2] = {(cuuint64_t)A_DQK, (cuuint64_t)a.R * a.H};
+    cuuint64_t strides[1] = {(cuuint64_t)A_DQK * 2};
+    cuuint32_t box[2] = {64u, (cuuint32_t)A_H};
+    cuuint32_t estr[2] = {1u, 1u};
+    if (fn(&mq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(a.q), dims, strides, box, estr,
+           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+        return cudaErrorInvalidValue;
+    cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
+    if (e != cudaSuccess) return e;
+    TraceScope ts("attn_tc", st);
+    attn_tc_kernel<<<(unsigned)(2LL * a.R), kThreads, kSmemBytes, st>>>(mq, a);
+    return cudaGetLastError();
+}
+
+}  // namespace idx

@@ -190,6 +190,23 @@ cudaError_t launch_select(const SelectArgs &a, cudaStream_t st);
 cudaError_t launch_proxy(const void *q, const float *w, const int *cu, int S, int T, int H, int d,
                          int g, int dtype, const int *plan, const PlanLayout &pl, void *qbar,
                          float *wbar, int max_proxies, cudaStream_t st);
+// token-sparse attention over selected positions (absorbed-MLA shapes)
+struct SparseAttnArgs {
+    const void *q;        // [R, H, 576] bf16
+    const void *kv;       // [Nkv, 576] bf16: key = all dims, value = dims [0, 512)
+    const int *idx;       // [R, topk] positions inside the row's request, -1 = none
+    const int *cu_q;      // [S+1] request boundaries over query rows
+    const int *cu_kv;     // [S+1] request boundaries over kv rows
+    int S, R, H, topk;
+    long long Nkv;
+    float scale;          // logit = scale * q . k
+    void *out;            // [R, H, 512] bf16
+    float *lse;           // [R, H] natural-log softmax denominators, or NULL
+    unsigned *status;
+};
+bool attn_tc_supported(int H, int Dqk, int Dv, int dtype);
+cudaError_t launch_sparse_attn_tc(const SparseAttnArgs &a, cudaStream_t st);
+
 // block pre-filter: mean keys of the complete blocks of every request
 cudaError_t launch_block_means(const void *k, const int *cu, int S, int T, int d, int dtype, void *kb,
                                cudaStream_t st);

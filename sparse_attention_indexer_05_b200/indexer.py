@@ -9,6 +9,7 @@ Entry points (names follow the C ABI):
     pivot_topk(q, k, w, cu_seqlens, topk, g, c, mode)   -> idx [T, topk]
     decode_topk(q, kcache, kv_len, w, topk, c, mode)    -> idx [B, G, topk]
     decode_paged_topk(q, kpool, block_table, kv_len, w, topk, c, mode)  -> idx [B, G, topk]
+    sparse_attn(q, kv, idx, cu_q, cu_kv, scale)         -> out [R, H, 512]
 Each accepts out_idx / out_score / workspace to reuse buffers, and
 return_scores=True to also get the selected scores.
 """
@@ -156,6 +157,29 @@ def decode_paged_topk(q, kpool, block_table, kv_len, w, topk: int, c: int = 0, m
         _dev(out_score, "out_score", torch.float32) if out_score is not None else None,
         ws.data_ptr(), ws.numel(), _stream(stream)), "idx_decode_paged_topk")
     return (out_idx, out_score) if return_scores else out_idx
+
+
+def sparse_attn(q, kv, idx, cu_q, cu_kv, scale: float, out=None, lse=None, workspace=None, stream=None,
+                return_lse=False):
+    """Token-sparse attention over the selected positions: q [R,H,576] bf16,
+    kv [Nkv,576] bf16 (value = first 512 dims), idx int32 [R,topk] (-1 = none),
+    cu_q / cu_kv int32 request boundaries over query rows and kv rows."""
+    R, H, Dqk = q.shape
+    Nkv = kv.shape[0]
+    Dv = 512
+    topk = idx.shape[1]
+    dt = _dtype_code(q)
+    if out is None:
+        out = torch.empty(R, H, Dv, dtype=q.dtype, device=q.device)
+    if lse is None and return_lse:
+        lse = torch.empty(R, H, dtype=torch.float32, device=q.device)
+    ws = _ws(workspace, int(N.lib().idx_sparse_attn_workspace_size()), q.device)
+    N.check(N.lib().idx_sparse_attn(
+        _dev(q, "q"), _dev(kv, "kv", q.dtype), _dev(idx, "idx", torch.int32), _dev(cu_q, "cu_q", torch.int32),
+        _dev(cu_kv, "cu_kv", torch.int32), cu_q.numel() - 1, R, Nkv, H, Dqk, Dv, topk, float(scale), dt,
+        _dev(out, "out", q.dtype), _dev(lse, "lse", torch.float32) if lse is not None else None,
+        ws.data_ptr(), ws.numel(), _stream(stream)), "idx_sparse_attn")
+    return (out, lse) if return_lse else out
 
 
 def device_status(workspace: torch.Tensor, stream=None) -> str:
