@@ -13,16 +13,17 @@
 //   P  = exp2(S*scale*log2e - m), m a running row maximum that is only moved
 //        (and O rescaled in TMEM) when it grows by more than 8, so that P <= 2^8
 //   O += P V_half   tcgen05, M=128, N=256, K=32 (2 steps)   -> TMEM, 256 cols
-// The key rows of a chunk are gathered by cp.async (16-byte pieces, rows of
-// -1 or out-of-range positions zero-filled) into the 128-byte-swizzled
+// The key rows of a chunk are gathered by TMA (tile::gather4: four rows of one
+// 64-dim slice per request, 72 requests per chunk) into the 128-byte-swizzled
 // K-major layout; the same buffer is the value operand of the second MMA
-// through an MN-major descriptor.  P goes to shared memory as bf16 in the
+// through an MN-major descriptor.  Entries that are -1 or out of range load
+// the request's first row (finite data) and get weight 0.  P goes to shared memory as bf16 in the
 // unswizzled K-major layout (8x16-byte core matrices).
 //
-// Roles (288 threads): warp 0 = MMA issuer (one lane) and TMEM owner;
+// Roles (224 threads): warp 0 = MMA issuer (one lane) and TMEM owner;
 // warps 1..4 = softmax and epilogue, one head row per thread (TMEM lane
-// quarter = warp % 4); warps 5..8 = gather, two groups of two warps that
-// fill the two key stages alternately.  Every wait is bounded.
+// quarter = warp % 4); warps 5, 6 = gather (TMA, five and four slices).
+// Every wait is bounded.
 #include <cudaTypedefs.h>
 #include <math.h>
 #include <string.h>
@@ -48,9 +49,8 @@ constexpr uint32_t kKSlice = A_KC * 128;             // 4 KB
 constexpr uint32_t kKStage = A_SLICES * kKSlice;     // 36 KB
 constexpr uint32_t kPBytes = A_H * A_KC * 2;         // 8 KB
 constexpr int kSoftWarps = 4;
-constexpr int kGatherWarps = 4;
+constexpr int kGatherWarps = 2;  // slices [0, 5) and [5, 9)
 constexpr int kThreads = 32 * (1 + kSoftWarps + kGatherWarps);
-constexpr int kGroupThreads = 32 * kGatherWarps / A_STAGES;  // gather threads per stage group
 constexpr uint32_t kColS = 0;               // S buffers: columns [0, 64)
 constexpr uint32_t kColO = 256;             // O: columns [256, 512)
 constexpr float kLog2e = 1.4426950408889634f;
@@ -68,6 +68,7 @@ constexpr size_t kOffP = kOffK + (size_t)A_STAGES * kKStage;
 constexpr size_t kOffCtl = kOffP + kPBytes;
 constexpr size_t kSmemBytes = kOffCtl + sizeof(AttnShared) + 1024;
 static_assert(kSmemBytes <= 232448, "shared memory of one CTA");
+static_assert(A_KC == 32, "one chunk position per lane of the gather warp");
 
 // K-major operand stored as 8-row x 16-byte core matrices without swizzle:
 // stride between K-adjacent core matrices `lbo`, between 8-row groups `sbo`.
@@ -93,11 +94,28 @@ __device__ __forceinline__ uint64_t mnmajor_sw128_desc(uint32_t saddr, uint32_t 
     return d;
 }
 
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void *src, uint32_t src_bytes) {
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
+// four rows (r0..r3) of the 64-column box at column x, 128 bytes each, to
+// four consecutive 128-byte rows at dst (tensor map box: 64 x 1)
+__device__ __forceinline__ void tma_gather4(uint32_t dst, const CUtensorMap *map, int x, int r0, int r1, int r2,
+                                            int r3, uint64_t *bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4, %5, %6, %7}], [%2];" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(tc::smem_u32(bar)), "r"(x), "r"(r0), "r"(r1), "r"(r2), "r"(r3)
+        : "memory");
 }
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
+// non-blocking test of an mbarrier phase (polling two barriers in turn)
+__device__ __forceinline__ bool mbar_test(uint64_t *bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}\n"
+        : "=r"(ok)
+        : "r"(tc::smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
 __device__ __forceinline__ void fence_proxy_async() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 
 __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
@@ -135,7 +153,8 @@ __device__ __forceinline__ bool locate(const int *cu_q, const int *cu_kv, int S,
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
-    attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, SparseAttnArgs a) {
+    attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_kv,
+                   SparseAttnArgs a) {
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = tc::smem_u32(smem_raw);
     uint8_t *smem = smem_raw + (((raw + 1023u) & ~1023u) - raw);
@@ -156,7 +175,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (threadIdx.x == 0) {
         tc::mbar_init(&sh.qfull, 1);
         for (int s = 0; s < A_STAGES; ++s) {
-            tc::mbar_init(&sh.kfull[s], kGroupThreads);
+            tc::mbar_init(&sh.kfull[s], kGatherWarps);
             tc::mbar_init(&sh.kempty[s], 1);
         }
         for (int b = 0; b < 2; ++b) {
@@ -190,23 +209,32 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint32_t idesc_o = tc::idesc_bf16_f32(A_H, A_DVH) | (1u << 16);  // value operand MN-major
             const uint32_t qa = tc::smem_u32(qs), ka = tc::smem_u32(ks), pa = tc::smem_u32(ps);
             bool ok = tc::mbar_wait(&sh.qfull, 0, abort, a.status);
-            for (int j = 0; ok && j <= nch; ++j) {
-                if (j < nch) {
-                    const int st = j % A_STAGES, sb = j & 1;
-                    if (!(ok = tc::mbar_wait(&sh.kfull[st], (j / A_STAGES) & 1u, abort, a.status))) break;
-                    if (!(ok = tc::mbar_wait(&sh.sfree[sb], ((j >> 1) & 1u) ^ 1u, abort, a.status))) break;
-                    tc::fence_after_sync();
-                    for (int kk = 0; kk < A_DQK / 16; ++kk) {
-                        const uint32_t off = (kk & 3) * 32u;  // 16-element K step inside the 128-byte row
-                        const uint64_t ad = tc::sw128_desc(qa + (kk >> 2) * kQSlice + off);
-                        const uint64_t bd = tc::sw128_desc(ka + st * kKStage + (kk >> 2) * kKSlice + off);
-                        tc::mma_bf16(tmem + kColS + sb * A_KC, ad, bd, idesc_s, kk > 0 ? 1u : 0u);
+            // two independent streams: S = Q K^T of chunk jq (needs its keys and a free
+            // S buffer) and O += P V of chunk jp (needs its P); issue whichever is ready,
+            // so that a late key chunk never holds back the P V that frees a stage
+            int jq = 0, jp = 0;
+            unsigned idle = 0;
+            unsigned long long t_idle = 0;
+            while (ok && jp < nch) {
+                bool progressed = false;
+                if (jq < nch) {
+                    const int st = jq % A_STAGES, sb = jq & 1;
+                    if (mbar_test(&sh.kfull[st], (jq / A_STAGES) & 1u) &&
+                        mbar_test(&sh.sfree[sb], ((jq >> 1) & 1u) ^ 1u)) {
+                        tc::fence_after_sync();
+                        for (int kk = 0; kk < A_DQK / 16; ++kk) {
+                            const uint32_t off = (kk & 3) * 32u;  // 16-element K step inside the 128-byte row
+                            const uint64_t ad = tc::sw128_desc(qa + (kk >> 2) * kQSlice + off);
+                            const uint64_t bd = tc::sw128_desc(ka + st * kKStage + (kk >> 2) * kKSlice + off);
+                            tc::mma_bf16(tmem + kColS + sb * A_KC, ad, bd, idesc_s, kk > 0 ? 1u : 0u);
+                        }
+                        tc::mma_commit(&sh.sfull[sb]);
+                        ++jq;
+                        progressed = true;
                     }
-                    tc::mma_commit(&sh.sfull[sb]);
                 }
-                if (j >= 1) {
-                    const int jp = j - 1, st = jp % A_STAGES;
-                    if (!(ok = tc::mbar_wait(&sh.pfull, jp & 1u, abort, a.status))) break;
+                if (jp < jq && mbar_test(&sh.pfull, jp & 1u)) {
+                    const int st = jp % A_STAGES;
                     tc::fence_after_sync();
                     const uint32_t vbase = ka + st * kKStage + (4 * half) * kKSlice;
                     for (int kk = 0; kk < A_KC / 16; ++kk) {
@@ -216,6 +244,19 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                     tc::mma_commit(&sh.kempty[st]);
                     tc::mma_commit(&sh.pdone);
+                    ++jp;
+                    progressed = true;
+                }
+                if (progressed) {
+                    idle = 0;
+                } else if (*abort) {
+                    ok = false;
+                } else if (idle++ == 0) {
+                    t_idle = globaltimer_ns();
+                } else if ((idle & 63u) == 0 && globaltimer_ns() - t_idle > kWaitNs) {
+                    *abort = 1;
+                    raise_status(a.status, ST_TIMEOUT);
+                    ok = false;
                 }
             }
             // drain: every MMA issued so far has completed before TMEM is released
@@ -233,8 +274,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         float m_used = -INFINITY, l = 0.0f;
         bool ok = true;
         uint32_t s[32];
+        // the chunk's positions are loaded one chunk ahead (off the wait for S)
+        int pos_next = lane < a.topk ? ix[lane] : -1;
         for (int j = 0; j < nch; ++j) {
             const int sb = j & 1;
+            const int pos = pos_next;
+            if ((j + 1) * A_KC + lane < a.topk) pos_next = ix[(j + 1) * A_KC + lane];
+            else pos_next = -1;
             if (lane == 0) ok = tc::mbar_wait(&sh.sfull[sb], (j >> 1) & 1u, abort, a.status);
             ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
             if (!ok) break;
@@ -244,7 +290,6 @@ __global__ void __launch_bounds__(kThreads, 1)
             tc::fence_before_sync();
             tc::mbar_arrive(&sh.sfree[sb]);
             // which keys of the chunk are listed and inside the request
-            const int pos = j * A_KC + lane < a.topk ? ix[j * A_KC + lane] : -1;
             const bool bad = pos >= nkv;
             if (bad && half == 0 && quarter == 0) raise_status(a.status, ST_INVALID);
             const unsigned valid = __ballot_sync(0xFFFFFFFFu, row_ok && pos >= 0 && !bad);
@@ -255,14 +300,25 @@ __global__ void __launch_bounds__(kThreads, 1)
                 x[c] = (valid >> c) & 1u ? __uint_as_float(s[c]) * sl2 : -INFINITY;
                 mx = fmaxf(mx, x[c]);
             }
+            const bool need = mx > m_used + kRescale;
+            const float factor = need ? exp2f(m_used - mx) : 1.0f;  // 0 while nothing was listed yet
+            const float m_new = need ? mx : m_used;
+            // weights and their bf16 packing do not depend on the previous chunk's P V
+            uint32_t pk[16];
+            float psum = 0.0f;
+#pragma unroll
+            for (int c = 0; c < 32; c += 2) {
+                const float p0 = x[c] == -INFINITY ? 0.0f : exp2f(x[c] - m_new);
+                const float p1 = x[c + 1] == -INFINITY ? 0.0f : exp2f(x[c + 1] - m_new);
+                psum += p0 + p1;
+                pk[c >> 1] = pack_bf16(p0, p1);
+            }
             if (j >= 1) {
                 if (lane == 0) ok = tc::mbar_wait(&sh.pdone, (j - 1) & 1u, abort, a.status);
                 ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
                 if (!ok) break;
                 tc::fence_after_sync();
             }
-            const bool need = mx > m_used + kRescale;
-            const float factor = need ? exp2f(m_used - mx) : 1.0f;  // 0 while nothing was listed yet
             if (j >= 1 && __any_sync(0xFFFFFFFFu, need)) {
                 uint32_t o[32];
                 for (int b = 0; b < A_DVH / 32; ++b) {
@@ -274,27 +330,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 tmem_wait_st();
             }
-            if (need) {
-                l *= factor;
-                m_used = mx;
-            }
-            float p[32];
-#pragma unroll
-            for (int c = 0; c < 32; ++c) {
-                p[c] = x[c] == -INFINITY ? 0.0f : exp2f(x[c] - m_used);
-                l += p[c];
-            }
+            l = l * factor + psum;
+            m_used = m_new;
             // P row h: core matrix (h/8, c/8) at (h/8)*512 + (c/8)*128, row h%8 at +16*(h%8)
             uint8_t *prow = ps + (h >> 3) * 512 + (h & 7) * 16;
 #pragma unroll
-            for (int c8 = 0; c8 < 4; ++c8) {
-                uint4 v;
-                v.x = pack_bf16(p[8 * c8 + 0], p[8 * c8 + 1]);
-                v.y = pack_bf16(p[8 * c8 + 2], p[8 * c8 + 3]);
-                v.z = pack_bf16(p[8 * c8 + 4], p[8 * c8 + 5]);
-                v.w = pack_bf16(p[8 * c8 + 6], p[8 * c8 + 7]);
-                *reinterpret_cast<uint4 *>(prow + c8 * 128) = v;
-            }
+            for (int c8 = 0; c8 < 4; ++c8)
+                *reinterpret_cast<uint4 *>(prow + c8 * 128) =
+                    make_uint4(pk[4 * c8 + 0], pk[4 * c8 + 1], pk[4 * c8 + 2], pk[4 * c8 + 3]);
             fence_proxy_async();
             tc::fence_before_sync();
             tc::mbar_arrive(&sh.pfull);
@@ -334,33 +377,42 @@ __global__ void __launch_bounds__(kThreads, 1)
                 a.lse[(long long)r * a.H + h] = l > 0.0f ? (m_used + log2f(l)) * 0.69314718055994531f : -INFINITY;
         }
     } else {
-        // -------------------------------------------------- gather
-        const int gt = threadIdx.x - 32 * (1 + kSoftWarps);  // 0 .. 127
-        const int grp = gt / kGroupThreads, t = gt % kGroupThreads;
-        const uint8_t *kvb = reinterpret_cast<const uint8_t *>(a.kv);
+        // ------------------------------------------------- gather (TMA)
+        const int gw = warp - (1 + kSoftWarps);                 // 0 or 1
+        const int sl0 = gw == 0 ? 0 : 5, sl1 = gw == 0 ? 5 : A_SLICES;
         bool ok = true;
-        for (int j = grp; j < nch; j += A_STAGES) {
-            const int st = j % A_STAGES;  // == grp
+        int issued = 0;
+        int pos_next = lane < a.topk ? ix[lane] : -1;   // positions one chunk ahead
+        for (int j = 0; j < nch; ++j) {
+            const int st = j % A_STAGES;
+            const int pos = pos_next;
+            pos_next = (j + 1) * A_KC + lane < a.topk ? ix[(j + 1) * A_KC + lane] : -1;
             if (lane == 0) ok = tc::mbar_wait(&sh.kempty[st], ((j / A_STAGES) & 1u) ^ 1u, abort, a.status);
             ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
             if (!ok) break;
-            const uint32_t dst0 = tc::smem_u32(ks + st * kKStage);
-            // 32 rows x 72 pieces of 16 bytes; piece u: row u / 72, piece c = u % 72 (slice c / 8)
-            for (int u = t; u < A_KC * (A_DQK / 8); u += kGroupThreads) {
-                const int row = u / (A_DQK / 8), c = u % (A_DQK / 8);
-                const int k = j * A_KC + row;
-                const int pos = k < a.topk ? ix[k] : -1;
-                const bool valid = row_ok && pos >= 0 && pos < nkv;
-                const uint8_t *src = valid ? kvb + ((kv0 + pos) * A_DQK + c * 8) * 2 : kvb;
-                const uint32_t dst = dst0 + (c >> 3) * kKSlice + row * 128 + ((((c & 7) ^ (row & 7))) << 4);
-                cp_async16(dst, src, valid ? 16u : 0u);
+            // lane i: row of chunk position i (the request's first row for entries not used)
+            const bool valid = row_ok && pos >= 0 && pos < nkv;
+            const int row = (int)(valid ? kv0 + pos : kv0);
+            if (lane == 0) tc::mbar_arrive_expect_tx(&sh.kfull[st], (uint32_t)(sl1 - sl0) * kKSlice);
+            __syncwarp();
+            const int r0 = __shfl_sync(0xFFFFFFFFu, row, (lane & 7) * 4 + 0);
+            const int r1 = __shfl_sync(0xFFFFFFFFu, row, (lane & 7) * 4 + 1);
+            const int r2 = __shfl_sync(0xFFFFFFFFu, row, (lane & 7) * 4 + 2);
+            const int r3 = __shfl_sync(0xFFFFFFFFu, row, (lane & 7) * 4 + 3);
+            if (lane < 8) {
+                // rows 4*lane .. 4*lane+3 of every 64-dim slice
+                const uint32_t dst0 = tc::smem_u32(ks + st * kKStage) + lane * 4 * 128;
+                for (int sl = sl0; sl < sl1; ++sl)
+                    tma_gather4(dst0 + sl * kKSlice, &tmap_kv, sl * 64, r0, r1, r2, r3, &sh.kfull[st]);
             }
-            cp_async_commit();
-            cp_async_wait_all();
-            fence_proxy_async();
-            tc::mbar_arrive(&sh.kfull[st]);
+            issued = j + 1;
         }
-        cp_async_wait_all();
+        // teardown: the copies issued last land before shared memory is released
+        if (lane == 0) {
+            for (int j = (issued > A_STAGES ? issued - A_STAGES : 0); j < issued; ++j)
+                tc::mbar_wait_drain(&sh.kfull[j % A_STAGES], (j / A_STAGES) & 1u);
+        }
+        __syncwarp();
     }
 
     tc::fence_before_sync();
@@ -405,10 +457,19 @@ cudaError_t launch_sparse_attn_tc(const SparseAttnArgs &a, cudaStream_t st) {
            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
         return cudaErrorInvalidValue;
+    // kv [Nkv, 576] bf16 rows, gather boxes of 64 columns x 1 row
+    CUtensorMap mkv;
+    memset(&mkv, 0, sizeof(mkv));
+    cuuint64_t kdims[2] = {(cuuint64_t)A_DQK, (cuuint64_t)a.Nkv};
+    cuuint32_t kbox[2] = {64u, 1u};
+    if (fn(&mkv, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(a.kv), kdims, strides, kbox, estr,
+           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+        return cudaErrorInvalidValue;
     cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
     if (e != cudaSuccess) return e;
     TraceScope ts("attn_tc", st);
-    attn_tc_kernel<<<(unsigned)(2LL * a.R), kThreads, kSmemBytes, st>>>(mq, a);
+    attn_tc_kernel<<<(unsigned)(2LL * a.R), kThreads, kSmemBytes, st>>>(mq, mkv, a);
     return cudaGetLastError();
 }
 
