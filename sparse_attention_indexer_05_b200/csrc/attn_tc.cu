@@ -20,9 +20,10 @@
 // the request's first row (finite data) and get weight 0.  P goes to shared memory as bf16 in the
 // unswizzled K-major layout (8x16-byte core matrices).
 //
-// Roles (224 threads): warp 0 = MMA issuer (one lane) and TMEM owner;
+// Roles (288 threads): warp 0 = MMA issuer (one lane) and TMEM owner;
 // warps 1..4 = softmax and epilogue, one head row per thread (TMEM lane
-// quarter = warp % 4); warps 5, 6 = gather (TMA, five and four slices).
+// quarter = warp % 4); warps 5..8 = gather (TMA, three, two, two and two
+// slices).
 // Every wait is bounded.
 #include <cudaTypedefs.h>
 #include <math.h>
@@ -49,7 +50,7 @@ constexpr uint32_t kKSlice = A_KC * 128;             // 4 KB
 constexpr uint32_t kKStage = A_SLICES * kKSlice;     // 36 KB
 constexpr uint32_t kPBytes = A_H * A_KC * 2;         // 8 KB
 constexpr int kSoftWarps = 4;
-constexpr int kGatherWarps = 2;  // slices [0, 5) and [5, 9)
+constexpr int kGatherWarps = 4;  // slices [0, 3), [3, 5), [5, 7), [7, 9)
 constexpr int kThreads = 32 * (1 + kSoftWarps + kGatherWarps);
 constexpr uint32_t kColS = 0;               // S buffers: columns [0, 64)
 constexpr uint32_t kColO = 256;             // O: columns [256, 512)
@@ -378,8 +379,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     } else {
         // ------------------------------------------------- gather (TMA)
-        const int gw = warp - (1 + kSoftWarps);                 // 0 or 1
-        const int sl0 = gw == 0 ? 0 : 5, sl1 = gw == 0 ? 5 : A_SLICES;
+        const int gw = warp - (1 + kSoftWarps);                 // 0 .. kGatherWarps-1
+        const int sl0 = gw == 0 ? 0 : 1 + 2 * gw, sl1 = 3 + 2 * gw;
         bool ok = true;
         int issued = 0;
         int pos_next = lane < a.topk ? ix[lane] : -1;   // positions one chunk ahead
