@@ -20,10 +20,10 @@
 // the request's first row (finite data) and get weight 0.  P goes to shared memory as bf16 in the
 // unswizzled K-major layout (8x16-byte core matrices).
 //
-// Roles (288 threads): warp 0 = MMA issuer (one lane) and TMEM owner;
+// Roles (448 threads): warp 0 = MMA issuer (one lane) and TMEM owner;
 // warps 1..4 = softmax and epilogue, one head row per thread (TMEM lane
-// quarter = warp % 4); warps 5..8 = gather (TMA, three, two, two and two
-// slices).
+// quarter = warp % 4); warps 5..13 = gather (TMA, one 64-dim slice each:
+// a warp's TMA requests issue one after another, so more warps issue more).
 // Every wait is bounded.
 #include <cudaTypedefs.h>
 #include <math.h>
@@ -50,7 +50,7 @@ constexpr uint32_t kKSlice = A_KC * 128;             // 4 KB
 constexpr uint32_t kKStage = A_SLICES * kKSlice;     // 36 KB
 constexpr uint32_t kPBytes = A_H * A_KC * 2;         // 8 KB
 constexpr int kSoftWarps = 4;
-constexpr int kGatherWarps = 4;  // slices [0, 3), [3, 5), [5, 7), [7, 9)
+constexpr int kGatherWarps = A_SLICES;  // one 64-dim slice per producer warp
 constexpr int kThreads = 32 * (1 + kSoftWarps + kGatherWarps);
 constexpr uint32_t kColS = 0;               // S buffers: columns [0, 64)
 constexpr uint32_t kColO = 256;             // O: columns [256, 512)
@@ -131,6 +131,14 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32
         : "memory");
 }
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+// 2^x by the hardware approximation (ex2.approx.ftz: relative error far below
+// the bf16 rounding of P that follows; 2^-inf = 0)
+__device__ __forceinline__ float fast_exp2(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
 
 __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
     const __nv_bfloat162 v = __floats2bfloat162_rn(a, b);
@@ -302,15 +310,18 @@ __global__ void __launch_bounds__(kThreads, 1)
                 mx = fmaxf(mx, x[c]);
             }
             const bool need = mx > m_used + kRescale;
-            const float factor = need ? exp2f(m_used - mx) : 1.0f;  // 0 while nothing was listed yet
+            const float factor = need ? fast_exp2(m_used - mx) : 1.0f;  // 0 while nothing was listed yet
             const float m_new = need ? mx : m_used;
+            // masked entries are -inf and give 0; with nothing listed yet every
+            // entry is masked and any finite reference serves
+            const float m_ref = m_new == -INFINITY ? 0.0f : m_new;
             // weights and their bf16 packing do not depend on the previous chunk's P V
             uint32_t pk[16];
             float psum = 0.0f;
 #pragma unroll
             for (int c = 0; c < 32; c += 2) {
-                const float p0 = x[c] == -INFINITY ? 0.0f : exp2f(x[c] - m_new);
-                const float p1 = x[c + 1] == -INFINITY ? 0.0f : exp2f(x[c + 1] - m_new);
+                const float p0 = fast_exp2(x[c] - m_ref);
+                const float p1 = fast_exp2(x[c + 1] - m_ref);
                 psum += p0 + p1;
                 pk[c >> 1] = pack_bf16(p0, p1);
             }
@@ -380,7 +391,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else {
         // ------------------------------------------------- gather (TMA)
         const int gw = warp - (1 + kSoftWarps);                 // 0 .. kGatherWarps-1
-        const int sl0 = gw == 0 ? 0 : 1 + 2 * gw, sl1 = 3 + 2 * gw;
+        const int sl0 = gw, sl1 = gw + 1;
         bool ok = true;
         int issued = 0;
         int pos_next = lane < a.topk ? ix[lane] : -1;   // positions one chunk ahead
