@@ -6,25 +6,33 @@
 //     z_j   = scale * q[r,h] . kv[row_j],   row_j = cu_kv[b] + idx[r, j] (idx >= 0)
 //     o[r,h] = sum_j softmax_j(z) * kv[row_j, :Dv],   lse[r,h] = log sum_j exp(z_j)
 //
-// One CTA per (query row, half of the value dimensions).  The 128 heads of
-// the row are the MMA's M; the row's Q (128 x 576 bf16, 144 KB) stays in
-// shared memory for the whole row.  Per chunk of 32 selected keys:
-//   S  = Q K^T      tcgen05, M=128, N=32, K=576 (36 steps)   -> TMEM, 2 buffers
+// A cluster of two CTAs per query row.  The 128 heads of the row are the
+// MMA's M.  The 576 key dims are split between the pair: CTA 0 holds Q and
+// gathers the keys of 64-dim slices 0..4, CTA 1 holds Q of slices 5..8 and
+// gathers key slices 4..8, so that each also holds the value dims of its
+// output half (CTA c writes value dims [256c, 256c+256)).  Per chunk of 32
+// selected keys, in each CTA:
+//   S_c = Q_c K_c^T   tcgen05, M=128, N=32, K=320 or 256   -> TMEM, 2 buffers
+//   the partial S_c goes to the peer's shared memory (DSMEM) and the peer's
+//   partial comes back; both add own + peer (the same fp32 sum on both sides)
 //   P  = exp2(S*scale*log2e - m), m a running row maximum that is only moved
 //        (and O rescaled in TMEM) when it grows by more than 8, so that P <= 2^8
-//   O += P V_half   tcgen05, M=128, N=256, K=32 (2 steps)   -> TMEM, 256 cols
-// The key rows of a chunk are gathered by TMA (tile::gather4: four rows of one
-// 64-dim slice per request, 72 requests per chunk) into the 128-byte-swizzled
-// K-major layout; the same buffer is the value operand of the second MMA
-// through an MN-major descriptor.  Entries that are -1 or out of range load
-// the request's first row (finite data) and get weight 0.  P goes to shared memory as bf16 in the
-// unswizzled K-major layout (8x16-byte core matrices).
+//   O_c += P V_c      tcgen05, M=128, N=256, K=32            -> TMEM, 256 cols
+// Both CTAs run the same softmax on the same S, so m, l and P agree.
+// The key rows are gathered by TMA (tile::gather4: four rows of one 64-dim
+// slice per request, 40 requests per chunk and CTA) into the
+// 128-byte-swizzled K-major layout; the value operand is read from the same
+// buffer through an MN-major descriptor.  Entries that are -1 or out of
+// range load the request's first row (finite data) and get weight 0.  P goes
+// to shared memory as bf16 in the unswizzled K-major layout.
 //
-// Roles (448 threads): warp 0 = MMA issuer (one lane) and TMEM owner;
+// Roles (352 threads per CTA): warp 0 = MMA issuer (one lane) and TMEM owner;
 // warps 1..4 = softmax and epilogue, one head row per thread (TMEM lane
-// quarter = warp % 4); warps 5..13 = gather (TMA, one 64-dim slice each:
-// a warp's TMA requests issue one after another, so more warps issue more).
-// Every wait is bounded.
+// quarter = warp % 4); warps 5..9 = gather, one slice each; warp 10 = courier
+// (one lane): one bulk shared-to-peer copy per chunk moves the staged partial
+// S, and the buffer hand-back to the peer is one remote arrive.  Every wait
+// is bounded; a cluster barrier after set-up and another before exit keep
+// each CTA's shared memory alive while its peer may still write to it.
 #include <cudaTypedefs.h>
 #include <math.h>
 #include <string.h>
@@ -42,34 +50,43 @@ constexpr int A_DQK = 576;
 constexpr int A_DV = 512;
 constexpr int A_DVH = 256;                  // value dims per CTA
 constexpr int A_KC = 32;                    // keys per chunk
-constexpr int A_SLICES = A_DQK / 64;        // 64-dim slices of a 128-byte swizzled row
-constexpr int A_STAGES = 2;
+constexpr int A_LS = 5;                     // 64-dim key slices gathered per CTA
+constexpr int A_STAGES = 4;
 constexpr uint32_t kQSlice = A_H * 128;              // 16 KB
-constexpr uint32_t kQBytes = A_SLICES * kQSlice;     // 144 KB
+constexpr uint32_t kQBytesMax = A_LS * kQSlice;      // 80 KB (CTA 0: 5 slices, CTA 1: 4)
 constexpr uint32_t kKSlice = A_KC * 128;             // 4 KB
-constexpr uint32_t kKStage = A_SLICES * kKSlice;     // 36 KB
-constexpr uint32_t kPBytes = A_H * A_KC * 2;         // 8 KB
+constexpr uint32_t kKStage = A_LS * kKSlice;         // 20 KB
+constexpr uint32_t kPBytes = A_H * A_KC * 2;         // 8 KB per P buffer (two)
+constexpr uint32_t kXBytes = A_H * A_KC * 4;         // 16 KB: one chunk's partial S
 constexpr int kSoftWarps = 4;
-constexpr int kGatherWarps = A_SLICES;  // one 64-dim slice per producer warp
-constexpr int kThreads = 32 * (1 + kSoftWarps + kGatherWarps);
+constexpr int kGatherWarps = A_LS;
+constexpr int kCourierWarp = 1 + kSoftWarps + kGatherWarps;  // moves partial S to the peer
+constexpr int kThreads = 32 * (kCourierWarp + 1);
 constexpr uint32_t kColS = 0;               // S buffers: columns [0, 64)
 constexpr uint32_t kColO = 256;             // O: columns [256, 512)
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescale = 8.0f;            // move the running max only past this growth (log2 units)
 
 struct __align__(8) AttnShared {
-    uint64_t qfull, kfull[A_STAGES], kempty[A_STAGES], sfull[2], sfree[2], pfull, pdone, drain;
+    uint64_t qfull, kfull[A_STAGES], kempty[A_STAGES], sfull[2], sfree[2], pfull[2], pdone[2], drain;
+    // exchange: xfull[b] = the peer's partial landed in xin[b] (transaction bytes);
+    // xfree[b] = the peer read what this CTA sent into its xin[b] (remote arrive);
+    // xready = xout holds this CTA's next partial; xout_free = the copy read xout;
+    // xused[b] = this CTA's softmax threads read xin[b]
+    uint64_t xfull[2], xfree[2], xready, xout_free, xused[2];
     uint32_t tmem_base;
     int abort;
 };
 
 constexpr size_t kOffQ = 0;
-constexpr size_t kOffK = kOffQ + kQBytes;
-constexpr size_t kOffP = kOffK + (size_t)A_STAGES * kKStage;
-constexpr size_t kOffCtl = kOffP + kPBytes;
+constexpr size_t kOffK = kOffQ + kQBytesMax;
+constexpr size_t kOffX = kOffK + (size_t)A_STAGES * kKStage;   // xin[2]: partials from the peer
+constexpr size_t kOffXo = kOffX + 2 * (size_t)kXBytes;          // xout: this CTA's partial, staged
+constexpr size_t kOffP = kOffXo + kXBytes;
+constexpr size_t kOffCtl = kOffP + 2 * (size_t)kPBytes;
 constexpr size_t kSmemBytes = kOffCtl + sizeof(AttnShared) + 1024;
 static_assert(kSmemBytes <= 232448, "shared memory of one CTA");
-static_assert(A_KC == 32, "one chunk position per lane of the gather warp");
+static_assert(A_KC == 32, "one chunk position per lane of a gather warp");
 
 // K-major operand stored as 8-row x 16-byte core matrices without swizzle:
 // stride between K-adjacent core matrices `lbo`, between 8-row groups `sbo`.
@@ -145,6 +162,65 @@ __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
     return *reinterpret_cast<const uint32_t *>(&v);
 }
 
+// ------------------------------------------------ cluster (DSMEM) helpers
+__device__ __forceinline__ uint32_t cluster_rank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+// shared::cluster address of this CTA's shared address `saddr` in CTA `rank`
+__device__ __forceinline__ uint32_t peer_addr(uint32_t saddr, uint32_t rank) {
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
+    return r;
+}
+// arrive on an mbarrier of the peer CTA, releasing this thread's earlier writes at cluster scope
+__device__ __forceinline__ void mbar_arrive_remote(uint32_t caddr) {
+    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(caddr) : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t *bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}\n"
+        : "=r"(ok)
+        : "r"(tc::smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+// bounded wait for a phase completed by the peer CTA (acquire at cluster scope)
+__device__ __forceinline__ bool mbar_wait_cluster(uint64_t *bar, uint32_t parity, volatile int *abort,
+                                                  unsigned *status) {
+    if (mbar_try_wait_cluster(bar, parity)) return true;
+    const unsigned long long t0 = globaltimer_ns();
+    for (unsigned it = 1;; ++it) {
+        if (mbar_try_wait_cluster(bar, parity)) return true;
+        if (*abort) return false;
+        if ((it & 31u) == 0u && globaltimer_ns() - t0 > kWaitNs) {
+            *abort = 1;
+            raise_status(status, ST_TIMEOUT);
+            return false;
+        }
+    }
+}
+// this CTA's shared bytes [src, src+bytes) into the peer's shared memory at
+// `dst`, completing `bytes` of transaction count on the peer's barrier `bar`
+// (dst and bar are shared::cluster addresses)
+__device__ __forceinline__ void bulk_to_peer(uint32_t dst, uint32_t src, uint32_t bytes, uint32_t bar) {
+    asm volatile("cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+                 "r"(src), "r"(bytes), "r"(bar)
+                 : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// wait until the committed bulk copies have read their source
+__device__ __forceinline__ void bulk_wait_read_all() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+// wait until the committed bulk copies have completed
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+__device__ __forceinline__ void cluster_sync() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
 // The request of query row r and its key range; false for malformed
 // boundaries (the row is then written as zeros and flagged).
 __device__ __forceinline__ bool locate(const int *cu_q, const int *cu_kv, int S, int R, long long Nkv, int r,
@@ -161,20 +237,29 @@ __device__ __forceinline__ bool locate(const int *cu_q, const int *cu_kv, int S,
     return ok;
 }
 
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_kv,
                    SparseAttnArgs a) {
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = tc::smem_u32(smem_raw);
+    // the same offset in both CTAs of the pair (same kernel, same shared layout)
     uint8_t *smem = smem_raw + (((raw + 1023u) & ~1023u) - raw);
     uint8_t *qs = smem + kOffQ;
     uint8_t *ks = smem + kOffK;
+    uint8_t *xs = smem + kOffX;
     uint8_t *ps = smem + kOffP;
     AttnShared &sh = *reinterpret_cast<AttnShared *>(smem + kOffCtl);
     volatile int *abort = &sh.abort;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int r = blockIdx.x >> 1, half = blockIdx.x & 1;
+    const uint32_t crank = cluster_rank();
+    const uint32_t peer = crank ^ 1u;
+    const int r = blockIdx.x >> 1;
+    const int half = (int)crank;                 // value dims [256 * half, +256) are written here
+    const int nq = crank == 0 ? 5 : 4;           // Q slices held here = key slices in this CTA's logits
+    const int gq0 = crank == 0 ? 0 : 5;          // global slice of Q slot 0
+    const int gk0 = crank == 0 ? 0 : 4;          // global slice of local key slice 0
+    const int qk0 = crank == 0 ? 0 : 1;          // local key slice of Q slot 0
     const int nch = (a.topk + A_KC - 1) / A_KC;
     long long kv0;
     int nkv;
@@ -190,13 +275,23 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int b = 0; b < 2; ++b) {
             tc::mbar_init(&sh.sfull[b], 1);
             tc::mbar_init(&sh.sfree[b], 32 * kSoftWarps);
+            tc::mbar_init(&sh.xfull[b], 1);      // this CTA's courier (expected bytes) + the peer's copy
+            tc::mbar_init(&sh.xfree[b], 1);      // the peer's courier
+            tc::mbar_init(&sh.xused[b], 32 * kSoftWarps);
         }
-        tc::mbar_init(&sh.pfull, 32 * kSoftWarps);
-        tc::mbar_init(&sh.pdone, 1);
+        tc::mbar_init(&sh.xready, 32 * kSoftWarps);
+        tc::mbar_init(&sh.xout_free, 1);
+        for (int b = 0; b < 2; ++b) {
+            tc::mbar_init(&sh.pfull[b], 32 * kSoftWarps);
+            tc::mbar_init(&sh.pdone[b], 1);
+        }
         tc::mbar_init(&sh.drain, 1);
         sh.abort = 0;
         tc::fence_mbar_init();
-        if (!row_ok) raise_status(a.status, ST_INVALID);
+        // the first use of each receive buffer expects one partial (before the peer may send)
+        for (int b = 0; b < 2; ++b)
+            if (b < nch) tc::mbar_arrive_expect_tx(&sh.xfull[b], kXBytes);
+        if (!row_ok && crank == 0) raise_status(a.status, ST_INVALID);
     }
     if (warp == 0) {
         tc::tmem_alloc(&sh.tmem_base, 512);
@@ -204,6 +299,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     tc::fence_before_sync();
     __syncthreads();
+    cluster_sync();  // both CTAs' barriers exist before any remote arrive
     tc::fence_after_sync();
     const uint32_t tmem = sh.tmem_base;
 
@@ -211,16 +307,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         // ------------------------------------------------ MMA issuer
         if (lane == 0) {
             tc::prefetch_tmap(&tmap_q);
-            tc::mbar_arrive_expect_tx(&sh.qfull, kQBytes);
-            for (int s = 0; s < A_SLICES; ++s)
-                tc::tma_load_2d(qs + s * kQSlice, &tmap_q, s * 64, r * a.H, &sh.qfull);
+            tc::mbar_arrive_expect_tx(&sh.qfull, (uint32_t)nq * kQSlice);
+            for (int s = 0; s < nq; ++s)
+                tc::tma_load_2d(qs + s * kQSlice, &tmap_q, (gq0 + s) * 64, r * a.H, &sh.qfull);
             const uint32_t idesc_s = tc::idesc_bf16_f32(A_H, A_KC);
             const uint32_t idesc_o = tc::idesc_bf16_f32(A_H, A_DVH) | (1u << 16);  // value operand MN-major
             const uint32_t qa = tc::smem_u32(qs), ka = tc::smem_u32(ks), pa = tc::smem_u32(ps);
             bool ok = tc::mbar_wait(&sh.qfull, 0, abort, a.status);
-            // two independent streams: S = Q K^T of chunk jq (needs its keys and a free
-            // S buffer) and O += P V of chunk jp (needs its P); issue whichever is ready,
-            // so that a late key chunk never holds back the P V that frees a stage
+            // two independent streams: the partial logits of chunk jq (its keys have
+            // landed and an S buffer is free) and O += P V of chunk jp (its P is
+            // written); whichever is ready is issued
             int jq = 0, jp = 0;
             unsigned idle = 0;
             unsigned long long t_idle = 0;
@@ -231,10 +327,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                     if (mbar_test(&sh.kfull[st], (jq / A_STAGES) & 1u) &&
                         mbar_test(&sh.sfree[sb], ((jq >> 1) & 1u) ^ 1u)) {
                         tc::fence_after_sync();
-                        for (int kk = 0; kk < A_DQK / 16; ++kk) {
+                        for (int kk = 0; kk < nq * 4; ++kk) {
                             const uint32_t off = (kk & 3) * 32u;  // 16-element K step inside the 128-byte row
                             const uint64_t ad = tc::sw128_desc(qa + (kk >> 2) * kQSlice + off);
-                            const uint64_t bd = tc::sw128_desc(ka + st * kKStage + (kk >> 2) * kKSlice + off);
+                            const uint64_t bd =
+                                tc::sw128_desc(ka + st * kKStage + (qk0 + (kk >> 2)) * kKSlice + off);
                             tc::mma_bf16(tmem + kColS + sb * A_KC, ad, bd, idesc_s, kk > 0 ? 1u : 0u);
                         }
                         tc::mma_commit(&sh.sfull[sb]);
@@ -242,17 +339,18 @@ __global__ void __launch_bounds__(kThreads, 1)
                         progressed = true;
                     }
                 }
-                if (jp < jq && mbar_test(&sh.pfull, jp & 1u)) {
+                if (jp < jq && mbar_test(&sh.pfull[jp & 1], (jp >> 1) & 1u)) {
                     const int st = jp % A_STAGES;
                     tc::fence_after_sync();
-                    const uint32_t vbase = ka + st * kKStage + (4 * half) * kKSlice;
+                    const uint32_t vbase = ka + st * kKStage;  // local key slices 0..3 = this CTA's value dims
+                    const uint32_t pbase = pa + (jp & 1) * kPBytes;
                     for (int kk = 0; kk < A_KC / 16; ++kk) {
-                        const uint64_t ad = kmajor_plain_desc(pa + kk * 256u, 128u, 512u);
+                        const uint64_t ad = kmajor_plain_desc(pbase + kk * 256u, 128u, 512u);
                         const uint64_t bd = mnmajor_sw128_desc(vbase + kk * 16u * 128u, kKSlice);
                         tc::mma_bf16(tmem + kColO, ad, bd, idesc_o, (jp > 0 || kk > 0) ? 1u : 0u);
                     }
                     tc::mma_commit(&sh.kempty[st]);
-                    tc::mma_commit(&sh.pdone);
+                    tc::mma_commit(&sh.pdone[jp & 1]);
                     ++jp;
                     progressed = true;
                 }
@@ -275,38 +373,83 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         __syncwarp();
     } else if (warp <= kSoftWarps) {
-        // ---------------------------------------- softmax and epilogue
+        // ------------------------------ exchange, softmax and epilogue
         const int quarter = warp & 3;
         const int h = quarter * 32 + lane;
         const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
         const float sl2 = a.scale * kLog2e;
+        // this thread's row of the staging and receive buffers (16-byte piece c
+        // of row h stored at piece c ^ (h & 7): conflict-free row-per-thread access)
+        uint8_t *xo_row = smem + kOffXo + h * 128;
         float m_used = -INFINITY, l = 0.0f;
         bool ok = true;
-        uint32_t s[32];
+        // send(jj, own): this CTA's partial logits of chunk jj from TMEM into
+        // `own` and into the staging buffer, from which the courier copies them
+        // to the peer
+        auto send = [&](int jj, uint32_t (&own)[32]) -> bool {
+            const int b = jj & 1;
+            const uint32_t u = (uint32_t)(jj >> 1);
+            bool good = true;
+            if (lane == 0) good = tc::mbar_wait(&sh.sfull[b], u & 1u, abort, a.status);
+            good = __shfl_sync(0xFFFFFFFFu, good, 0);
+            if (!good) return false;
+            tc::fence_after_sync();
+            tc::tmem_ld32(tmem + lane_off + kColS + b * A_KC, own);
+            tc::tmem_wait_ld(own);
+            tc::fence_before_sync();
+            tc::mbar_arrive(&sh.sfree[b]);
+            (void)u;
+            // the staging buffer is free once the copy of chunk jj-1 has read it
+            if (lane == 0) good = tc::mbar_wait(&sh.xout_free, (jj & 1) ^ 1u, abort, a.status);
+            good = __shfl_sync(0xFFFFFFFFu, good, 0);
+            if (!good) return false;
+#pragma unroll
+            for (int c = 0; c < 8; ++c)
+                *reinterpret_cast<uint4 *>(xo_row + ((c ^ (h & 7)) << 4)) =
+                    make_uint4(own[4 * c], own[4 * c + 1], own[4 * c + 2], own[4 * c + 3]);
+            fence_proxy_async();  // the copy reads the staging buffer through the async proxy
+            tc::mbar_arrive(&sh.xready);
+            return true;
+        };
+        uint32_t own[32], nxt[32];
+        // the exchange runs one chunk ahead: chunk j+1's partial is on its way
+        // while chunk j's softmax is computed
+        ok = nch > 0 && send(0, own);
         // the chunk's positions are loaded one chunk ahead (off the wait for S)
         int pos_next = lane < a.topk ? ix[lane] : -1;
-        for (int j = 0; j < nch; ++j) {
-            const int sb = j & 1;
+        for (int j = 0; ok && j < nch; ++j) {
+            const int xb = j & 1;
+            const uint32_t use = (uint32_t)(j >> 1);  // use of exchange buffer xb
             const int pos = pos_next;
             if ((j + 1) * A_KC + lane < a.topk) pos_next = ix[(j + 1) * A_KC + lane];
             else pos_next = -1;
-            if (lane == 0) ok = tc::mbar_wait(&sh.sfull[sb], (j >> 1) & 1u, abort, a.status);
+            if (j + 1 < nch && !(ok = send(j + 1, nxt))) break;
+            // the peer's partial of chunk j; the sum is the same fp32 addition on both sides
+            if (lane == 0) ok = tc::mbar_wait(&sh.xfull[xb], use & 1u, abort, a.status);
             ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
             if (!ok) break;
-            tc::fence_after_sync();
-            tc::tmem_ld32(tmem + lane_off + kColS + sb * A_KC, s);
-            tc::tmem_wait_ld(s);
-            tc::fence_before_sync();
-            tc::mbar_arrive(&sh.sfree[sb]);
+            const uint4 *xr = reinterpret_cast<const uint4 *>(xs + xb * kXBytes + h * 128);
+            float st_[32];
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+                const uint4 v = xr[c ^ (h & 7)];
+                st_[4 * c + 0] = __uint_as_float(own[4 * c + 0]) + __uint_as_float(v.x);
+                st_[4 * c + 1] = __uint_as_float(own[4 * c + 1]) + __uint_as_float(v.y);
+                st_[4 * c + 2] = __uint_as_float(own[4 * c + 2]) + __uint_as_float(v.z);
+                st_[4 * c + 3] = __uint_as_float(own[4 * c + 3]) + __uint_as_float(v.w);
+            }
+            tc::mbar_arrive(&sh.xused[xb]);  // the courier tells the peer this buffer is free
+#pragma unroll
+            for (int c = 0; c < 32; ++c) own[c] = nxt[c];
             // which keys of the chunk are listed and inside the request
             const bool bad = pos >= nkv;
-            if (bad && half == 0 && quarter == 0) raise_status(a.status, ST_INVALID);
+            if (bad && crank == 0 && quarter == 0) raise_status(a.status, ST_INVALID);
             const unsigned valid = __ballot_sync(0xFFFFFFFFu, row_ok && pos >= 0 && !bad);
             float x[32];
             float mx = -INFINITY;
 #pragma unroll
             for (int c = 0; c < 32; ++c) {
-                x[c] = (valid >> c) & 1u ? __uint_as_float(s[c]) * sl2 : -INFINITY;
+                x[c] = (valid >> c) & 1u ? st_[c] * sl2 : -INFINITY;
                 mx = fmaxf(mx, x[c]);
             }
             const bool need = mx > m_used + kRescale;
@@ -325,13 +468,21 @@ __global__ void __launch_bounds__(kThreads, 1)
                 psum += p0 + p1;
                 pk[c >> 1] = pack_bf16(p0, p1);
             }
-            if (j >= 1) {
-                if (lane == 0) ok = tc::mbar_wait(&sh.pdone, (j - 1) & 1u, abort, a.status);
+            // P buffer j&1 is free once P V of chunk j-2 completed
+            if (j >= 2) {
+                if (lane == 0) ok = tc::mbar_wait(&sh.pdone[j & 1], ((j - 2) >> 1) & 1u, abort, a.status);
                 ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
                 if (!ok) break;
-                tc::fence_after_sync();
             }
-            if (j >= 1 && __any_sync(0xFFFFFFFFu, need)) {
+            const bool resc = j >= 1 && __any_sync(0xFFFFFFFFu, need);
+            if (resc) {
+                // O is rescaled only after every earlier P V completed (that of chunk j-1 last)
+                if (lane == 0) ok = tc::mbar_wait(&sh.pdone[(j - 1) & 1], ((j - 1) >> 1) & 1u, abort, a.status);
+                ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
+                if (!ok) break;
+            }
+            tc::fence_after_sync();
+            if (resc) {
                 uint32_t o[32];
                 for (int b = 0; b < A_DVH / 32; ++b) {
                     tc::tmem_ld32(tmem + lane_off + kColO + b * 32, o);
@@ -345,33 +496,29 @@ __global__ void __launch_bounds__(kThreads, 1)
             l = l * factor + psum;
             m_used = m_new;
             // P row h: core matrix (h/8, c/8) at (h/8)*512 + (c/8)*128, row h%8 at +16*(h%8)
-            uint8_t *prow = ps + (h >> 3) * 512 + (h & 7) * 16;
+            uint8_t *prow = ps + (j & 1) * kPBytes + (h >> 3) * 512 + (h & 7) * 16;
 #pragma unroll
             for (int c8 = 0; c8 < 4; ++c8)
                 *reinterpret_cast<uint4 *>(prow + c8 * 128) =
                     make_uint4(pk[4 * c8 + 0], pk[4 * c8 + 1], pk[4 * c8 + 2], pk[4 * c8 + 3]);
             fence_proxy_async();
             tc::fence_before_sync();
-            tc::mbar_arrive(&sh.pfull);
+            tc::mbar_arrive(&sh.pfull[j & 1]);
         }
-        // epilogue: O / l for this half of the value dims, lse from half 0
+        // epilogue: O / l for this half of the value dims, lse from CTA 0
         if (ok && nch > 0) {
-            if (lane == 0) ok = tc::mbar_wait(&sh.pdone, (nch - 1) & 1u, abort, a.status);
+            if (lane == 0) ok = tc::mbar_wait(&sh.pdone[(nch - 1) & 1], ((nch - 1) >> 1) & 1u, abort, a.status);
             ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
         }
         if (ok) {
             tc::fence_after_sync();
             const float inv = l > 0.0f ? 1.0f / l : 0.0f;
-            __nv_bfloat16 *orow = reinterpret_cast<__nv_bfloat16 *>(a.out) + ((long long)r * a.H + h) * A_DV + half * A_DVH;
+            __nv_bfloat16 *orow =
+                reinterpret_cast<__nv_bfloat16 *>(a.out) + ((long long)r * a.H + h) * A_DV + half * A_DVH;
             uint32_t o[32];
             for (int b = 0; b < A_DVH / 32; ++b) {
-                if (nch > 0) {
-                    tc::tmem_ld32(tmem + lane_off + kColO + b * 32, o);
-                    tc::tmem_wait_ld(o);
-                } else {
-#pragma unroll
-                    for (int c = 0; c < 32; ++c) o[c] = 0u;
-                }
+                tc::tmem_ld32(tmem + lane_off + kColO + b * 32, o);
+                tc::tmem_wait_ld(o);
                 if (h < a.H) {
                     uint4 *dst = reinterpret_cast<uint4 *>(orow + b * 32);
 #pragma unroll
@@ -385,16 +532,16 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                 }
             }
-            if (half == 0 && h < a.H && a.lse)
+            if (crank == 0 && h < a.H && a.lse)
                 a.lse[(long long)r * a.H + h] = l > 0.0f ? (m_used + log2f(l)) * 0.69314718055994531f : -INFINITY;
         }
-    } else {
-        // ------------------------------------------------- gather (TMA)
-        const int gw = warp - (1 + kSoftWarps);                 // 0 .. kGatherWarps-1
-        const int sl0 = gw, sl1 = gw + 1;
+    } else if (warp < kCourierWarp) {
+        // --------------------------------------- gather (TMA), one slice per warp
+        const int gw = warp - (1 + kSoftWarps);  // local key slice
+        const int xcol = (gk0 + gw) * 64;         // its first column in the latent rows
         bool ok = true;
         int issued = 0;
-        int pos_next = lane < a.topk ? ix[lane] : -1;   // positions one chunk ahead
+        int pos_next = lane < a.topk ? ix[lane] : -1;  // positions one chunk ahead
         for (int j = 0; j < nch; ++j) {
             const int st = j % A_STAGES;
             const int pos = pos_next;
@@ -405,18 +552,15 @@ __global__ void __launch_bounds__(kThreads, 1)
             // lane i: row of chunk position i (the request's first row for entries not used)
             const bool valid = row_ok && pos >= 0 && pos < nkv;
             const int row = (int)(valid ? kv0 + pos : kv0);
-            if (lane == 0) tc::mbar_arrive_expect_tx(&sh.kfull[st], (uint32_t)(sl1 - sl0) * kKSlice);
+            if (lane == 0) tc::mbar_arrive_expect_tx(&sh.kfull[st], kKSlice);
             __syncwarp();
             const int r0 = __shfl_sync(0xFFFFFFFFu, row, (lane & 7) * 4 + 0);
             const int r1 = __shfl_sync(0xFFFFFFFFu, row, (lane & 7) * 4 + 1);
             const int r2 = __shfl_sync(0xFFFFFFFFu, row, (lane & 7) * 4 + 2);
             const int r3 = __shfl_sync(0xFFFFFFFFu, row, (lane & 7) * 4 + 3);
-            if (lane < 8) {
-                // rows 4*lane .. 4*lane+3 of every 64-dim slice
-                const uint32_t dst0 = tc::smem_u32(ks + st * kKStage) + lane * 4 * 128;
-                for (int sl = sl0; sl < sl1; ++sl)
-                    tma_gather4(dst0 + sl * kKSlice, &tmap_kv, sl * 64, r0, r1, r2, r3, &sh.kfull[st]);
-            }
+            if (lane < 8)  // rows 4*lane .. 4*lane+3 of this slice
+                tma_gather4(tc::smem_u32(ks + st * kKStage + gw * kKSlice) + lane * 4 * 128, &tmap_kv, xcol, r0, r1,
+                            r2, r3, &sh.kfull[st]);
             issued = j + 1;
         }
         // teardown: the copies issued last land before shared memory is released
@@ -425,10 +569,51 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tc::mbar_wait_drain(&sh.kfull[j % A_STAGES], (j / A_STAGES) & 1u);
         }
         __syncwarp();
+    } else {
+        // ------------------------------------------------ courier (one lane)
+        // copies each staged partial to the peer in one bulk DSMEM transfer and
+        // returns the peer's receive buffers once this CTA's threads read them
+        if (lane == 0) {
+            uint32_t xin_peer[2], xfull_peer[2], xfree_peer[2];
+            for (int b = 0; b < 2; ++b) {
+                xin_peer[b] = peer_addr(tc::smem_u32(xs + b * kXBytes), peer);
+                xfull_peer[b] = peer_addr(tc::smem_u32(&sh.xfull[b]), peer);
+                xfree_peer[b] = peer_addr(tc::smem_u32(&sh.xfree[b]), peer);
+            }
+            const uint32_t xo = tc::smem_u32(smem + kOffXo);
+            auto send = [&](int jj) -> bool {
+                const int b = jj & 1;
+                const uint32_t u = (uint32_t)(jj >> 1);
+                if (!tc::mbar_wait(&sh.xready, jj & 1u, abort, a.status)) return false;
+                // the peer read what was sent into its buffer b two chunks ago
+                if (!mbar_wait_cluster(&sh.xfree[b], (u & 1u) ^ 1u, abort, a.status)) return false;
+                bulk_to_peer(xin_peer[b], xo, kXBytes, xfull_peer[b]);
+                bulk_commit();
+                bulk_wait_read_all();
+                tc::mbar_arrive(&sh.xout_free);
+                return true;
+            };
+            auto returned = [&](int j) -> bool {
+                const int b = j & 1;
+                if (!tc::mbar_wait(&sh.xused[b], (j >> 1) & 1u, abort, a.status)) return false;
+                // announce the buffer's next partial (chunk j+2) before the peer may send it
+                if (j + 2 < nch) tc::mbar_arrive_expect_tx(&sh.xfull[b], kXBytes);
+                mbar_arrive_remote(xfree_peer[b]);
+                return true;
+            };
+            bool ok = nch > 0 && send(0);
+            for (int j = 0; ok && j < nch; ++j) {
+                if (j + 1 < nch && !(ok = send(j + 1))) break;
+                ok = returned(j);
+            }
+            bulk_wait_all();  // this CTA's copies have landed in the peer
+        }
+        __syncwarp();
     }
 
     tc::fence_before_sync();
     __syncthreads();
+    cluster_sync();  // the peer no longer writes into this CTA's shared memory
     tc::fence_after_sync();
     if (warp == 0) tc::tmem_dealloc(tmem, 512);
 }
@@ -455,10 +640,10 @@ bool attn_tc_supported(int H, int Dqk, int Dv, int dtype) {
 cudaError_t launch_sparse_attn_tc(const SparseAttnArgs &a, cudaStream_t st) {
     if (a.R <= 0) return cudaSuccess;
     if (!attn_tc_supported(a.H, A_DQK, A_DV, 0)) return cudaErrorInvalidValue;
-    // q [R * H, 576] bf16 rows, boxes of 64 columns x 128 rows (one row's heads,
-    // and for H < 128 rows of the next query or the zero fill past the end)
     PFN_cuTensorMapEncodeTiled_v12000 fn = encode_fn_attn();
     if (!fn) return cudaErrorInvalidValue;
+    // q [R * H, 576] bf16 rows, boxes of 64 columns x 128 rows (one row's heads,
+    // and for H < 128 rows of the next query or the zero fill past the end)
     CUtensorMap mq;
     memset(&mq, 0, sizeof(mq));
     cuuint64_t dims[2] = {(cuuint64_t)A_DQK, (cuuint64_t)a.R * a.H};
@@ -481,6 +666,7 @@ cudaError_t launch_sparse_attn_tc(const SparseAttnArgs &a, cudaStream_t st) {
     cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
     if (e != cudaSuccess) return e;
     TraceScope ts("attn_tc", st);
+    // a cluster of two CTAs per query row (compile-time cluster shape)
     attn_tc_kernel<<<(unsigned)(2LL * a.R), kThreads, kSmemBytes, st>>>(mq, mkv, a);
     return cudaGetLastError();
 }
