@@ -426,7 +426,7 @@ def main():
         _, tra = trace_report(lib)
         kms = sum(t for n, (c, t) in tra.items() if n.endswith("attn_tc")) / args.steps
         useful = 2.0 * 128 * nvalid * (576 + 512)  # logits + weighted values, per listed key and head
-        issued = 2.0 * 128 * (Ra * 2048) * (2 * 576 + 512)  # each value half recomputes the logits
+        issued = 2.0 * 128 * (Ra * 2048) * (576 + 512)  # every slot of the 2048 is computed (-1 slots too)
         tf = useful / (kms / 1000.0) / 1e12 if kms > 0 else None
         att = {"workload": f"sparse_mla_attn_rows{Ra}_H128_dqk576_dv512_k2048_kv{L}",
                "indices": "dense indexer top-2048 of the last rows of the 131072-token request",
