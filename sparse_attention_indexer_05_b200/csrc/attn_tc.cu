@@ -26,9 +26,11 @@
 // range load the request's first row (finite data) and get weight 0.  P goes
 // to shared memory as bf16 in the unswizzled K-major layout.
 //
-// Roles (352 threads per CTA): warp 0 = MMA issuer (one lane) and TMEM owner;
-// warps 1..4 = softmax and epilogue, one head row per thread (TMEM lane
-// quarter = warp % 4); warps 5..9 = gather, one slice each; warp 10 = courier
+// Roles (480 threads per CTA): warp 0 = MMA issuer (one lane) and TMEM owner;
+// warps 1..4 = receive, softmax and epilogue, one head row per thread (TMEM
+// lane quarter = warp % 4); warps 5..8 = send (this CTA's partial S from TMEM
+// to the staging buffer, ahead of the softmax); warps 9..13 = gather, one
+// slice each; warp 14 = courier
 // (one lane): one bulk shared-to-peer copy per chunk moves the staged partial
 // S, and the buffer hand-back to the peer is one remote arrive.  Every wait
 // is bounded; a cluster barrier after set-up and another before exit keep
@@ -58,9 +60,10 @@ constexpr uint32_t kKSlice = A_KC * 128;             // 4 KB
 constexpr uint32_t kKStage = A_LS * kKSlice;         // 20 KB
 constexpr uint32_t kPBytes = A_H * A_KC * 2;         // 8 KB per P buffer (two)
 constexpr uint32_t kXBytes = A_H * A_KC * 4;         // 16 KB: one chunk's partial S
-constexpr int kSoftWarps = 4;
+constexpr int kSoftWarps = 4;   // receive, softmax, epilogue
+constexpr int kSendWarps = 4;   // this CTA's partial S: TMEM -> staging buffer
 constexpr int kGatherWarps = A_LS;
-constexpr int kCourierWarp = 1 + kSoftWarps + kGatherWarps;  // moves partial S to the peer
+constexpr int kCourierWarp = 1 + kSoftWarps + kSendWarps + kGatherWarps;  // moves partial S to the peer
 constexpr int kThreads = 32 * (kCourierWarp + 1);
 constexpr uint32_t kColS = 0;               // S buffers: columns [0, 64)
 constexpr uint32_t kColO = 256;             // O: columns [256, 512)
@@ -274,12 +277,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         }
         for (int b = 0; b < 2; ++b) {
             tc::mbar_init(&sh.sfull[b], 1);
-            tc::mbar_init(&sh.sfree[b], 32 * kSoftWarps);
+            tc::mbar_init(&sh.sfree[b], 32 * (kSoftWarps + kSendWarps));  // both read S
             tc::mbar_init(&sh.xfull[b], 1);      // this CTA's courier (expected bytes) + the peer's copy
             tc::mbar_init(&sh.xfree[b], 1);      // the peer's courier
             tc::mbar_init(&sh.xused[b], 32 * kSoftWarps);
         }
-        tc::mbar_init(&sh.xready, 32 * kSoftWarps);
+        tc::mbar_init(&sh.xready, 32 * kSendWarps);
         tc::mbar_init(&sh.xout_free, 1);
         for (int b = 0; b < 2; ++b) {
             tc::mbar_init(&sh.pfull[b], 32 * kSoftWarps);
@@ -378,43 +381,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         const int h = quarter * 32 + lane;
         const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
         const float sl2 = a.scale * kLog2e;
-        // this thread's row of the staging and receive buffers (16-byte piece c
-        // of row h stored at piece c ^ (h & 7): conflict-free row-per-thread access)
-        uint8_t *xo_row = smem + kOffXo + h * 128;
         float m_used = -INFINITY, l = 0.0f;
         bool ok = true;
-        // send(jj, own): this CTA's partial logits of chunk jj from TMEM into
-        // `own` and into the staging buffer, from which the courier copies them
-        // to the peer
-        auto send = [&](int jj, uint32_t (&own)[32]) -> bool {
-            const int b = jj & 1;
-            const uint32_t u = (uint32_t)(jj >> 1);
-            bool good = true;
-            if (lane == 0) good = tc::mbar_wait(&sh.sfull[b], u & 1u, abort, a.status);
-            good = __shfl_sync(0xFFFFFFFFu, good, 0);
-            if (!good) return false;
-            tc::fence_after_sync();
-            tc::tmem_ld32(tmem + lane_off + kColS + b * A_KC, own);
-            tc::tmem_wait_ld(own);
-            tc::fence_before_sync();
-            tc::mbar_arrive(&sh.sfree[b]);
-            (void)u;
-            // the staging buffer is free once the copy of chunk jj-1 has read it
-            if (lane == 0) good = tc::mbar_wait(&sh.xout_free, (jj & 1) ^ 1u, abort, a.status);
-            good = __shfl_sync(0xFFFFFFFFu, good, 0);
-            if (!good) return false;
-#pragma unroll
-            for (int c = 0; c < 8; ++c)
-                *reinterpret_cast<uint4 *>(xo_row + ((c ^ (h & 7)) << 4)) =
-                    make_uint4(own[4 * c], own[4 * c + 1], own[4 * c + 2], own[4 * c + 3]);
-            fence_proxy_async();  // the copy reads the staging buffer through the async proxy
-            tc::mbar_arrive(&sh.xready);
-            return true;
-        };
-        uint32_t own[32], nxt[32];
-        // the exchange runs one chunk ahead: chunk j+1's partial is on its way
-        // while chunk j's softmax is computed
-        ok = nch > 0 && send(0, own);
+        uint32_t own[32];
         // the chunk's positions are loaded one chunk ahead (off the wait for S)
         int pos_next = lane < a.topk ? ix[lane] : -1;
         for (int j = 0; ok && j < nch; ++j) {
@@ -423,11 +392,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             const int pos = pos_next;
             if ((j + 1) * A_KC + lane < a.topk) pos_next = ix[(j + 1) * A_KC + lane];
             else pos_next = -1;
-            if (j + 1 < nch && !(ok = send(j + 1, nxt))) break;
-            // the peer's partial of chunk j; the sum is the same fp32 addition on both sides
-            if (lane == 0) ok = tc::mbar_wait(&sh.xfull[xb], use & 1u, abort, a.status);
+            // the peer's partial of chunk j and this CTA's own (read again from TMEM);
+            // the sum is the same fp32 addition on both sides
+            if (lane == 0)
+                ok = tc::mbar_wait(&sh.xfull[xb], use & 1u, abort, a.status) &&
+                     tc::mbar_wait(&sh.sfull[xb], use & 1u, abort, a.status);
             ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
             if (!ok) break;
+            tc::fence_after_sync();
+            tc::tmem_ld32(tmem + lane_off + kColS + xb * A_KC, own);
+            tc::tmem_wait_ld(own);
+            tc::fence_before_sync();
+            tc::mbar_arrive(&sh.sfree[xb]);
             const uint4 *xr = reinterpret_cast<const uint4 *>(xs + xb * kXBytes + h * 128);
             float st_[32];
 #pragma unroll
@@ -439,8 +415,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                 st_[4 * c + 3] = __uint_as_float(own[4 * c + 3]) + __uint_as_float(v.w);
             }
             tc::mbar_arrive(&sh.xused[xb]);  // the courier tells the peer this buffer is free
-#pragma unroll
-            for (int c = 0; c < 32; ++c) own[c] = nxt[c];
             // which keys of the chunk are listed and inside the request
             const bool bad = pos >= nkv;
             if (bad && crank == 0 && quarter == 0) raise_status(a.status, ST_INVALID);
@@ -535,9 +509,40 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             if (crank == 0 && h < a.H && a.lse)
                 a.lse[(long long)r * a.H + h] = l > 0.0f ? (m_used + log2f(l)) * 0.69314718055994531f : -INFINITY;
         }
+    } else if (warp <= kSoftWarps + kSendWarps) {
+        // --------------------- send: this CTA's partial S into the staging buffer
+        // (runs ahead of the softmax, bounded by the two S buffers)
+        const int quarter = warp & 3;
+        const int h = quarter * 32 + lane;
+        const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
+        // 16-byte piece c of row h stored at piece c ^ (h & 7): conflict-free row-per-thread access
+        uint8_t *xo_row = smem + kOffXo + h * 128;
+        bool ok = true;
+        uint32_t own[32];
+        for (int j = 0; ok && j < nch; ++j) {
+            const int b = j & 1;
+            if (lane == 0) ok = tc::mbar_wait(&sh.sfull[b], (j >> 1) & 1u, abort, a.status);
+            ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
+            if (!ok) break;
+            tc::fence_after_sync();
+            tc::tmem_ld32(tmem + lane_off + kColS + b * A_KC, own);
+            tc::tmem_wait_ld(own);
+            tc::fence_before_sync();
+            tc::mbar_arrive(&sh.sfree[b]);
+            // the staging buffer is free once the copy of chunk j-1 has read it
+            if (lane == 0) ok = tc::mbar_wait(&sh.xout_free, (j & 1) ^ 1u, abort, a.status);
+            ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
+            if (!ok) break;
+#pragma unroll
+            for (int c = 0; c < 8; ++c)
+                *reinterpret_cast<uint4 *>(xo_row + ((c ^ (h & 7)) << 4)) =
+                    make_uint4(own[4 * c], own[4 * c + 1], own[4 * c + 2], own[4 * c + 3]);
+            fence_proxy_async();  // the copy reads the staging buffer through the async proxy
+            tc::mbar_arrive(&sh.xready);
+        }
     } else if (warp < kCourierWarp) {
         // --------------------------------------- gather (TMA), one slice per warp
-        const int gw = warp - (1 + kSoftWarps);  // local key slice
+        const int gw = warp - (1 + kSoftWarps + kSendWarps);  // local key slice
         const int xcol = (gk0 + gw) * 64;         // its first column in the latent rows
         bool ok = true;
         int issued = 0;
