@@ -24,13 +24,13 @@
 // 128-byte-swizzled K-major layout; the value operand is read from the same
 // buffer through an MN-major descriptor.  Entries that are -1 or out of
 // range load the request's first row (finite data) and get weight 0.  P goes
-// to shared memory as bf16 in the unswizzled K-major layout.
+// to tensor memory as bf16 pairs and is the A operand of the second MMA there.
 //
-// Roles (480 threads per CTA): warp 0 = MMA issuer (one lane) and TMEM owner;
+// Roles (512 threads per CTA): warp 0 = MMA issuer (one lane) and TMEM owner;
 // warps 1..4 = receive, softmax and epilogue, one head row per thread (TMEM
 // lane quarter = warp % 4); warps 5..8 = send (this CTA's partial S from TMEM
 // to the staging buffer, ahead of the softmax); warps 9..13 = gather, one
-// slice each; warp 14 = courier
+// slice each; warp 14 = courier (send), warp 15 = courier (hand back)
 // (one lane): one bulk shared-to-peer copy per chunk moves the staged partial
 // S, and the buffer hand-back to the peer is one remote arrive.  Every wait
 // is bounded; a cluster barrier after set-up and another before exit keep
@@ -58,14 +58,15 @@ constexpr uint32_t kQSlice = A_H * 128;              // 16 KB
 constexpr uint32_t kQBytesMax = A_LS * kQSlice;      // 80 KB (CTA 0: 5 slices, CTA 1: 4)
 constexpr uint32_t kKSlice = A_KC * 128;             // 4 KB
 constexpr uint32_t kKStage = A_LS * kKSlice;         // 20 KB
-constexpr uint32_t kPBytes = A_H * A_KC * 2;         // 8 KB per P buffer (two)
 constexpr uint32_t kXBytes = A_H * A_KC * 4;         // 16 KB: one chunk's partial S
 constexpr int kSoftWarps = 4;   // receive, softmax, epilogue
 constexpr int kSendWarps = 4;   // this CTA's partial S: TMEM -> staging buffer
 constexpr int kGatherWarps = A_LS;
-constexpr int kCourierWarp = 1 + kSoftWarps + kSendWarps + kGatherWarps;  // moves partial S to the peer
-constexpr int kThreads = 32 * (kCourierWarp + 1);
+constexpr int kCourierWarp = 1 + kSoftWarps + kSendWarps + kGatherWarps;  // copies partial S to the peer
+constexpr int kReturnWarp = kCourierWarp + 1;                                // hands receive buffers back
+constexpr int kThreads = 32 * (kReturnWarp + 1);
 constexpr uint32_t kColS = 0;               // S buffers: columns [0, 64)
+constexpr uint32_t kColP = 64;              // P buffers (bf16 pairs): columns [64, 96)
 constexpr uint32_t kColO = 256;             // O: columns [256, 512)
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescale = 8.0f;            // move the running max only past this growth (log2 units)
@@ -74,9 +75,9 @@ struct __align__(8) AttnShared {
     uint64_t qfull, kfull[A_STAGES], kempty[A_STAGES], sfull[2], sfree[2], pfull[2], pdone[2], drain;
     // exchange: xfull[b] = the peer's partial landed in xin[b] (transaction bytes);
     // xfree[b] = the peer read what this CTA sent into its xin[b] (remote arrive);
-    // xready = xout holds this CTA's next partial; xout_free = the copy read xout;
-    // xused[b] = this CTA's softmax threads read xin[b]
-    uint64_t xfull[2], xfree[2], xready, xout_free, xused[2];
+    // xready[b] = xout[b] holds this CTA's next partial; xout_free[b] = the copy
+    // read xout[b]; xused[b] = this CTA's softmax threads read xin[b]
+    uint64_t xfull[2], xfree[2], xready[2], xout_free[2], xused[2];
     uint32_t tmem_base;
     int abort;
 };
@@ -84,23 +85,11 @@ struct __align__(8) AttnShared {
 constexpr size_t kOffQ = 0;
 constexpr size_t kOffK = kOffQ + kQBytesMax;
 constexpr size_t kOffX = kOffK + (size_t)A_STAGES * kKStage;   // xin[2]: partials from the peer
-constexpr size_t kOffXo = kOffX + 2 * (size_t)kXBytes;          // xout: this CTA's partial, staged
-constexpr size_t kOffP = kOffXo + kXBytes;
-constexpr size_t kOffCtl = kOffP + 2 * (size_t)kPBytes;
+constexpr size_t kOffXo = kOffX + 2 * (size_t)kXBytes;          // xout[2]: this CTA's partials, staged
+constexpr size_t kOffCtl = kOffXo + 2 * (size_t)kXBytes;
 constexpr size_t kSmemBytes = kOffCtl + sizeof(AttnShared) + 1024;
 static_assert(kSmemBytes <= 232448, "shared memory of one CTA");
 static_assert(A_KC == 32, "one chunk position per lane of a gather warp");
-
-// K-major operand stored as 8-row x 16-byte core matrices without swizzle:
-// stride between K-adjacent core matrices `lbo`, between 8-row groups `sbo`.
-__device__ __forceinline__ uint64_t kmajor_plain_desc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
-    uint64_t d = 0;
-    d |= (uint64_t)((saddr >> 4) & 0x3FFFu);
-    d |= (uint64_t)((lbo >> 4) & 0x3FFFu) << 16;
-    d |= (uint64_t)((sbo >> 4) & 0x3FFFu) << 32;
-    d |= (uint64_t)1u << 46;
-    return d;  // swizzle mode 0
-}
 
 // MN-major operand in the 128-byte swizzle: rows of 128 bytes along MN (64
 // elements), 8 K-rows per 1024-byte atom; `lbo` = stride between 64-element
@@ -148,6 +137,26 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32
         "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]), "r"(r[16]),
         "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]),
         "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
+        : "memory");
+}
+// 16 consecutive 32-bit columns of the warp's 32 TMEM lanes (one lane per thread)
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+        "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16};" ::"r"(taddr),
+        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),
+        "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+        : "memory");
+}
+// D[tmem] (+)= A[tmem] * B: A (M x 16, bf16 pairs per 32-bit column, row = lane)
+// in tensor memory, B by a shared-memory descriptor
+__device__ __forceinline__ void mma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                            uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+        "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
         : "memory");
 }
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
@@ -250,7 +259,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     uint8_t *qs = smem + kOffQ;
     uint8_t *ks = smem + kOffK;
     uint8_t *xs = smem + kOffX;
-    uint8_t *ps = smem + kOffP;
     AttnShared &sh = *reinterpret_cast<AttnShared *>(smem + kOffCtl);
     volatile int *abort = &sh.abort;
 
@@ -281,9 +289,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             tc::mbar_init(&sh.xfull[b], 1);      // this CTA's courier (expected bytes) + the peer's copy
             tc::mbar_init(&sh.xfree[b], 1);      // the peer's courier
             tc::mbar_init(&sh.xused[b], 32 * kSoftWarps);
+            tc::mbar_init(&sh.xready[b], 32 * kSendWarps);
+            tc::mbar_init(&sh.xout_free[b], 1);
         }
-        tc::mbar_init(&sh.xready, 32 * kSendWarps);
-        tc::mbar_init(&sh.xout_free, 1);
         for (int b = 0; b < 2; ++b) {
             tc::mbar_init(&sh.pfull[b], 32 * kSoftWarps);
             tc::mbar_init(&sh.pdone[b], 1);
@@ -315,7 +323,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                 tc::tma_load_2d(qs + s * kQSlice, &tmap_q, (gq0 + s) * 64, r * a.H, &sh.qfull);
             const uint32_t idesc_s = tc::idesc_bf16_f32(A_H, A_KC);
             const uint32_t idesc_o = tc::idesc_bf16_f32(A_H, A_DVH) | (1u << 16);  // value operand MN-major
-            const uint32_t qa = tc::smem_u32(qs), ka = tc::smem_u32(ks), pa = tc::smem_u32(ps);
+            const uint32_t qa = tc::smem_u32(qs), ka = tc::smem_u32(ks);
             bool ok = tc::mbar_wait(&sh.qfull, 0, abort, a.status);
             // two independent streams: the partial logits of chunk jq (its keys have
             // landed and an S buffer is free) and O += P V of chunk jp (its P is
@@ -346,11 +354,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                     const int st = jp % A_STAGES;
                     tc::fence_after_sync();
                     const uint32_t vbase = ka + st * kKStage;  // local key slices 0..3 = this CTA's value dims
-                    const uint32_t pbase = pa + (jp & 1) * kPBytes;
                     for (int kk = 0; kk < A_KC / 16; ++kk) {
-                        const uint64_t ad = kmajor_plain_desc(pbase + kk * 256u, 128u, 512u);
+                        // P (keys 16kk .. 16kk+15) = 8 columns of bf16 pairs in TMEM
+                        const uint32_t at = tmem + kColP + (jp & 1) * (A_KC / 2) + kk * 8;
                         const uint64_t bd = mnmajor_sw128_desc(vbase + kk * 16u * 128u, kKSlice);
-                        tc::mma_bf16(tmem + kColO, ad, bd, idesc_o, (jp > 0 || kk > 0) ? 1u : 0u);
+                        mma_bf16_ts(tmem + kColO, at, bd, idesc_o, (jp > 0 || kk > 0) ? 1u : 0u);
                     }
                     tc::mma_commit(&sh.kempty[st]);
                     tc::mma_commit(&sh.pdone[jp & 1]);
@@ -469,13 +477,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             }
             l = l * factor + psum;
             m_used = m_new;
-            // P row h: core matrix (h/8, c/8) at (h/8)*512 + (c/8)*128, row h%8 at +16*(h%8)
-            uint8_t *prow = ps + (j & 1) * kPBytes + (h >> 3) * 512 + (h & 7) * 16;
-#pragma unroll
-            for (int c8 = 0; c8 < 4; ++c8)
-                *reinterpret_cast<uint4 *>(prow + c8 * 128) =
-                    make_uint4(pk[4 * c8 + 0], pk[4 * c8 + 1], pk[4 * c8 + 2], pk[4 * c8 + 3]);
-            fence_proxy_async();
+            // P row h into TMEM lane h: column i holds keys 2i, 2i+1 (bf16 pair)
+            tmem_st16(tmem + lane_off + kColP + (j & 1) * (A_KC / 2), pk);
+            tmem_wait_st();
             tc::fence_before_sync();
             tc::mbar_arrive(&sh.pfull[j & 1]);
         }
@@ -516,7 +520,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         const int h = quarter * 32 + lane;
         const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
         // 16-byte piece c of row h stored at piece c ^ (h & 7): conflict-free row-per-thread access
-        uint8_t *xo_row = smem + kOffXo + h * 128;
+        uint8_t *xo_row = smem + kOffXo + h * 128;  // + b * kXBytes
         bool ok = true;
         uint32_t own[32];
         for (int j = 0; ok && j < nch; ++j) {
@@ -529,16 +533,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             tc::tmem_wait_ld(own);
             tc::fence_before_sync();
             tc::mbar_arrive(&sh.sfree[b]);
-            // the staging buffer is free once the copy of chunk j-1 has read it
-            if (lane == 0) ok = tc::mbar_wait(&sh.xout_free, (j & 1) ^ 1u, abort, a.status);
+            // staging buffer b is free once the copy of chunk j-2 has read it
+            if (lane == 0) ok = tc::mbar_wait(&sh.xout_free[b], ((j >> 1) & 1u) ^ 1u, abort, a.status);
             ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
             if (!ok) break;
 #pragma unroll
             for (int c = 0; c < 8; ++c)
-                *reinterpret_cast<uint4 *>(xo_row + ((c ^ (h & 7)) << 4)) =
+                *reinterpret_cast<uint4 *>(xo_row + b * kXBytes + ((c ^ (h & 7)) << 4)) =
                     make_uint4(own[4 * c], own[4 * c + 1], own[4 * c + 2], own[4 * c + 3]);
             fence_proxy_async();  // the copy reads the staging buffer through the async proxy
-            tc::mbar_arrive(&sh.xready);
+            tc::mbar_arrive(&sh.xready[b]);
         }
     } else if (warp < kCourierWarp) {
         // --------------------------------------- gather (TMA), one slice per warp
@@ -574,44 +578,38 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                 tc::mbar_wait_drain(&sh.kfull[j % A_STAGES], (j / A_STAGES) & 1u);
         }
         __syncwarp();
-    } else {
-        // ------------------------------------------------ courier (one lane)
-        // copies each staged partial to the peer in one bulk DSMEM transfer and
-        // returns the peer's receive buffers once this CTA's threads read them
+    } else if (warp == kCourierWarp) {
+        // ------------------------------------------- courier (one lane): send
+        // each staged partial goes to the peer in one bulk DSMEM transfer
         if (lane == 0) {
-            uint32_t xin_peer[2], xfull_peer[2], xfree_peer[2];
-            for (int b = 0; b < 2; ++b) {
-                xin_peer[b] = peer_addr(tc::smem_u32(xs + b * kXBytes), peer);
-                xfull_peer[b] = peer_addr(tc::smem_u32(&sh.xfull[b]), peer);
-                xfree_peer[b] = peer_addr(tc::smem_u32(&sh.xfree[b]), peer);
-            }
-            const uint32_t xo = tc::smem_u32(smem + kOffXo);
-            auto send = [&](int jj) -> bool {
-                const int b = jj & 1;
-                const uint32_t u = (uint32_t)(jj >> 1);
-                if (!tc::mbar_wait(&sh.xready, jj & 1u, abort, a.status)) return false;
+            bool ok = true;
+            for (int j = 0; ok && j < nch; ++j) {
+                const int b = j & 1;
+                const uint32_t u = (uint32_t)(j >> 1);
+                if (!(ok = tc::mbar_wait(&sh.xready[b], u & 1u, abort, a.status))) break;
                 // the peer read what was sent into its buffer b two chunks ago
-                if (!mbar_wait_cluster(&sh.xfree[b], (u & 1u) ^ 1u, abort, a.status)) return false;
-                bulk_to_peer(xin_peer[b], xo, kXBytes, xfull_peer[b]);
+                if (!(ok = mbar_wait_cluster(&sh.xfree[b], (u & 1u) ^ 1u, abort, a.status))) break;
+                bulk_to_peer(peer_addr(tc::smem_u32(xs + b * kXBytes), peer), tc::smem_u32(smem + kOffXo + b * kXBytes),
+                             kXBytes, peer_addr(tc::smem_u32(&sh.xfull[b]), peer));
                 bulk_commit();
                 bulk_wait_read_all();
-                tc::mbar_arrive(&sh.xout_free);
-                return true;
-            };
-            auto returned = [&](int j) -> bool {
-                const int b = j & 1;
-                if (!tc::mbar_wait(&sh.xused[b], (j >> 1) & 1u, abort, a.status)) return false;
-                // announce the buffer's next partial (chunk j+2) before the peer may send it
-                if (j + 2 < nch) tc::mbar_arrive_expect_tx(&sh.xfull[b], kXBytes);
-                mbar_arrive_remote(xfree_peer[b]);
-                return true;
-            };
-            bool ok = nch > 0 && send(0);
-            for (int j = 0; ok && j < nch; ++j) {
-                if (j + 1 < nch && !(ok = send(j + 1))) break;
-                ok = returned(j);
+                tc::mbar_arrive(&sh.xout_free[b]);
             }
             bulk_wait_all();  // this CTA's copies have landed in the peer
+        }
+        __syncwarp();
+    } else {
+        // ------------------------------------- courier (one lane): hand back
+        // once this CTA's threads read a receive buffer, its next partial is
+        // announced and the peer may send into it again
+        if (lane == 0) {
+            bool ok = true;
+            for (int j = 0; ok && j < nch; ++j) {
+                const int b = j & 1;
+                if (!(ok = tc::mbar_wait(&sh.xused[b], (j >> 1) & 1u, abort, a.status))) break;
+                if (j + 2 < nch) tc::mbar_arrive_expect_tx(&sh.xfull[b], kXBytes);
+                mbar_arrive_remote(peer_addr(tc::smem_u32(&sh.xfree[b]), peer));
+            }
         }
         __syncwarp();
     }
