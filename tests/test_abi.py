@@ -93,3 +93,21 @@ def test_binding_refuses_cpu_tensors():
     with pytest.raises((ValueError, RuntimeError)):
         idx.dense_topk(q, torch.zeros(4, 8, dtype=torch.bfloat16), torch.zeros(4, 2),
                        torch.tensor([0, 4], dtype=torch.int32), 2)
+
+
+def test_sparse_attn_argument_checks(lib):
+    """Host-side checks of idx_sparse_attn return before any launch."""
+    fake = ctypes.c_void_p(256)  # never dereferenced: the checks fail first
+    assert lib.idx_sparse_attn_workspace_size() == 256
+
+    def call(q=fake, kv=fake, H=128, Dqk=576, Dv=512, scale=0.07, ws=fake, ws_bytes=256):
+        return lib.idx_sparse_attn(q, kv, fake, fake, fake, 1, 4, 100, H, Dqk, Dv, 64, scale, 0, fake, None,
+                                   ws, ws_bytes, None)
+
+    assert call(kv=None) == 1                      # null latent rows
+    assert call(Dv=600) == 1                       # value wider than the key
+    assert call(scale=float("nan")) == 1           # non-finite scale
+    assert call(Dqk=512) == 2                      # shape without a kernel
+    assert call(H=256) == 2                        # more heads than the MMA's M
+    assert call(ws_bytes=16) == 3                  # workspace too small
+    assert call(ws=ctypes.c_void_p(264)) == 3      # misaligned workspace
