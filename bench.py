@@ -278,11 +278,11 @@ def main():
     o1 = torch.empty(L, TOPK, dtype=torch.int32, device=dev)
     o2 = torch.empty(L, TOPK, dtype=torch.int32, device=dev)
 
-    def step(qq=q, kk=k, ww=w, c1=cu1, c2=cu2):
+    def step(qq=q, kk=k, ww=w, c1=cu1, c2=cu2, oo1=o1, oo2=o2, st=None):
         if do_dense:
-            idx.dense_topk(qq, kk, ww, c1, TOPK, out_idx=o1, workspace=ws1)
+            idx.dense_topk(qq, kk, ww, c1, TOPK, out_idx=oo1, workspace=ws1, stream=st)
         if do_refine:
-            idx.pivot_topk(qq, kk, ww, c2, TOPK, G_REF, C_REF, "refine", out_idx=o2, workspace=ws2)
+            idx.pivot_topk(qq, kk, ww, c2, TOPK, G_REF, C_REF, "refine", out_idx=oo2, workspace=ws2, stream=st)
 
     for _ in range(args.warmup):
         step()
@@ -322,39 +322,65 @@ def main():
     per_kernel = {name: {"launches": c, "ms_total": t, "ms_per_step": t / args.steps} for name, (c, t) in tr.items()}
 
     # ---------------------------------------------------------------- e2e
+    # Every step copies its inputs in from pinned host memory and reads its
+    # results back, as a serving loop does: the copies of step i+1's inputs
+    # and step i-1's results run on their own streams while step i computes
+    # (two input sets and two output sets on the device).
     e2e = None
     if not args.no_e2e:
         hq, hk, hw, h1, h2 = pinned(P.q), pinned(P.k), pinned(P.w), pinned(cu1_h), pinned(cu2_h)
-        ho1 = torch.empty(o1.shape, dtype=torch.int32).pin_memory()
-        ho2 = torch.empty(o2.shape, dtype=torch.int32).pin_memory()
-        dq, dk, dw = torch.empty_like(q), torch.empty_like(k), torch.empty_like(w)
-        dc1, dc2 = torch.empty_like(cu1), torch.empty_like(cu2)
+        hos = [(torch.empty(o1.shape, dtype=torch.int32).pin_memory(),
+                torch.empty(o2.shape, dtype=torch.int32).pin_memory()) for _ in range(2)]
+        sets = [(torch.empty_like(q), torch.empty_like(k), torch.empty_like(w), torch.empty_like(cu1),
+                 torch.empty_like(cu2)) for _ in range(2)]
+        outs = [(torch.empty_like(o1), torch.empty_like(o2)) for _ in range(2)]
+        s_in, s_cmp, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+        ev_in = [torch.cuda.Event() for _ in range(2)]
+        ev_cmp = [torch.cuda.Event() for _ in range(2)]
+        ev_out = [torch.cuda.Event() for _ in range(2)]
 
-        def e2e_step():
-            dq.view(torch.int16).copy_(hq, non_blocking=True)
-            dk.view(torch.int16).copy_(hk, non_blocking=True)
-            dw.copy_(hw, non_blocking=True)
-            dc1.copy_(h1, non_blocking=True)
-            dc2.copy_(h2, non_blocking=True)
-            step(dq, dk, dw, dc1, dc2)
-            ho1.copy_(o1, non_blocking=True)
-            ho2.copy_(o2, non_blocking=True)
+        def e2e_run(nsteps):
+            for i in range(nsteps):
+                b = i % 2
+                dq, dk, dw, dc1, dc2 = sets[b]
+                with torch.cuda.stream(s_in):
+                    if i >= 2:
+                        s_in.wait_event(ev_cmp[b])  # step i-2 finished reading input set b
+                    dq.view(torch.int16).copy_(hq, non_blocking=True)
+                    dk.view(torch.int16).copy_(hk, non_blocking=True)
+                    dw.copy_(hw, non_blocking=True)
+                    dc1.copy_(h1, non_blocking=True)
+                    dc2.copy_(h2, non_blocking=True)
+                    ev_in[b].record(s_in)
+                with torch.cuda.stream(s_cmp):
+                    s_cmp.wait_event(ev_in[b])
+                    if i >= 2:
+                        s_cmp.wait_event(ev_out[b])  # step i-2's results were read back
+                    step(dq, dk, dw, dc1, dc2, outs[b][0], outs[b][1], st=s_cmp)
+                    ev_cmp[b].record(s_cmp)
+                with torch.cuda.stream(s_out):
+                    s_out.wait_event(ev_cmp[b])
+                    hos[b][0].copy_(outs[b][0], non_blocking=True)
+                    hos[b][1].copy_(outs[b][1], non_blocking=True)
+                    ev_out[b].record(s_out)
 
-        e2e_step()
+        e2e_run(2)
         torch.cuda.synchronize()
         barrier()
-        e0.record(stream)
-        for _ in range(args.steps):
-            e2e_step()
-        e1.record(stream)
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        t0.record(s_in)
+        e2e_run(args.steps)
+        s_out.wait_event(ev_cmp[(args.steps - 1) % 2])
+        t1.record(s_out)  # after the last read-back, which follows every earlier step
         torch.cuda.synchronize()
         barrier()
-        ems = max_over_ranks(e0.elapsed_time(e1) / args.steps)
+        ems = max_over_ranks(t0.elapsed_time(t1) / args.steps)
         h2d = hq.numel() * 2 + hk.numel() * 2 + hw.numel() * 4 + h1.numel() * 4 + h2.numel() * 4
-        d2h = (ho1.numel() + ho2.numel()) * 4
+        d2h = (hos[0][0].numel() + hos[0][1].numel()) * 4
         e2e = {"value": world * rows_per_step / (ems / 1000.0), "unit": "queries/s", "ms_per_step": ems,
-               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
-        del dq, dk, dw
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+               "overlap": "inputs of step i+1 and results of step i-1 copied while step i computes"}
+        del sets, outs
 
     # ------------------------------------------- block pre-filter (Refine)
     blk = None
