@@ -20,16 +20,16 @@ size_t up(size_t x, size_t a = kAlign) { return (x + a - 1) / a * a; }
 // Candidate buffer capacity per scored row for a streaming top-ksel over
 // rows of at most n keys.  A random key order appends about
 // ksel * (1 + ln(n / ksel)) keys; 1.5x that leaves room for the histogram's
-// coarse threshold.  At least 2*ksel + 512 so that a compaction (cut to
+// coarse threshold.  At least 2*ksel + 1024 so that a compaction (cut to
 // ksel) always frees more than the appends that can arrive between two
-// upkeeps (4 tiles of 128 keys); never more than n, which cannot overflow.
+// upkeeps (8 tiles of 128 keys); never more than n, which cannot overflow.
 unsigned cap_for(long long ksel, long long n) {
     if (n < 1) n = 1;
     const long long nn = (long long)up((size_t)n, 32);
     if (n <= ksel) return (unsigned)nn;
     const double est = 1.5 * (double)ksel * (1.0 + log((double)n / (double)ksel));
     long long cap = (long long)up((size_t)ceil(est), 256);
-    if (cap < 2 * ksel + 512) cap = 2 * ksel + 512;
+    if (cap < 2 * ksel + 1024) cap = 2 * ksel + 1024;
     if (cap > nn) cap = nn;
     return (unsigned)cap;
 }

@@ -10,12 +10,17 @@
 // share every key tile that TMA brings in, so each key byte fetched feeds
 // 8 queries.  The epilogue of one half overlaps the MMA of the other.
 //
-// Roles (320 threads): warp 0 = TMA producer (one lane), warp 1 = MMA issuer
-// (one lane; the whole warp allocates TMEM), warps 2..9 = epilogue.  Epilogue
-// warp e reads TMEM lane quarter (e % 4) -- keys 32*(e%4) .. +31 of the tile --
-// for the two queries 2*((e-2)/4), +1 of each half.  Each thread then holds the
-// 64 head dot products of its key for a query and reduces them in registers:
-//     I = sum_j w_j * max(dot_j, 0)      (8 partial sums, fixed order).
+// Roles (576 threads): warp 0 = TMA producer (one lane), warp 1 = MMA issuer
+// (one lane; the whole warp allocates TMEM), warps 2..17 = epilogue in four
+// roles of four warps, one warp per TMEM lane quarter (warp % 4: keys
+// 32*(warp%4) .. +31 of the tile).  Role p owns rows 2p, 2p+1, two queries
+// of half p/2, so half-0 and half-1 roles run offset by one MMA half and
+// their ALU-heavy reductions interleave with the other half's waits and
+// loads.  Each thread reduces, per row, the 64 head dot products of its key:
+//     I = sum_j w_j * max(dot_j, 0)      (8 partial sums, fixed order),
+// computed as (w_j / 2) * (dot_j + |dot_j|), the same value bit for bit
+// (dot + |dot| is 2 max(dot, 0) exactly; halving w is exact), which keeps the
+// max off the ALU pipe.
 // The scores go to the same sinks as the CUDA-core kernel: the streaming
 // candidate filter (common.cuh) or a spill of full score rows (debug export).
 #include <cudaTypedefs.h>
@@ -34,7 +39,7 @@ constexpr int TC_H = 64;
 constexpr int TC_D = 128;
 constexpr int kEpiWarps = 16;                         // 4 per TMEM lane quarter, one query each per half
 constexpr int kThreads = 64 + 32 * kEpiWarps;         // + TMA warp + MMA warp
-constexpr int kMaintEvery = 4;                        // tiles between candidate-filter upkeeps
+constexpr int kMaintEvery = 8;                        // tiles between candidate-filter upkeeps
 constexpr int kStages = 2;                            // key-tile stages
 constexpr uint32_t kQHalfBytes = 256 * 128;           // one half, one 64-column K slice (32 KB)
 constexpr uint32_t kQBytes = 4 * kQHalfBytes;         // 2 halves x 2 K slices (128 KB)
@@ -72,58 +77,38 @@ __device__ __forceinline__ unsigned long long ffma2(unsigned long long acc, floa
     return acc;
 }
 
-// sum_j w[j] * max(v[j], 0) over 64 heads held in two 32-register groups;
-// w read as float4 (16-byte aligned); 8 independent partial sums kept as 4
-// packed pairs, so each two heads cost two max and one packed fma.
-__device__ __forceinline__ float head_reduce(const uint32_t (&v0)[32], const uint32_t (&v1)[32], const float *w) {
-    const float4 *w4 = reinterpret_cast<const float4 *>(w);
+// v + |v| = 2 max(v, 0), exactly for every finite v below FLT_MAX / 2; an
+// fp32 add on the FMA pipe instead of a max on the half-rate ALU pipe.
+__device__ __forceinline__ float twice_relu(uint32_t x) {
+    const float f = __uint_as_float(x);
+    return f + fabsf(f);
+}
+
+// sum_j w[j] * max(v[j], 0) over 64 heads held in two 32-register groups,
+// given w2 = w / 2 (read as float4, 16-byte aligned): each term is
+// w2[j] * (v[j] + |v[j]|), the same fp32 product.  8 independent partial sums
+// kept as 4 packed pairs, so each two heads cost two adds and one packed fma.
+__device__ __forceinline__ float head_reduce(const uint32_t (&v0)[32], const uint32_t (&v1)[32], const float *w2) {
+    const float4 *w4 = reinterpret_cast<const float4 *>(w2);
     unsigned long long a[4] = {0ull, 0ull, 0ull, 0ull};
 #pragma unroll
     for (int j4 = 0; j4 < 8; ++j4) {
         const float4 wv = w4[j4];
-        a[(2 * j4) & 3] = ffma2(a[(2 * j4) & 3], wv.x, wv.y, fmaxf(__uint_as_float(v0[4 * j4 + 0]), 0.0f),
-                                fmaxf(__uint_as_float(v0[4 * j4 + 1]), 0.0f));
-        a[(2 * j4 + 1) & 3] = ffma2(a[(2 * j4 + 1) & 3], wv.z, wv.w, fmaxf(__uint_as_float(v0[4 * j4 + 2]), 0.0f),
-                                    fmaxf(__uint_as_float(v0[4 * j4 + 3]), 0.0f));
+        a[(2 * j4) & 3] = ffma2(a[(2 * j4) & 3], wv.x, wv.y, twice_relu(v0[4 * j4 + 0]), twice_relu(v0[4 * j4 + 1]));
+        a[(2 * j4 + 1) & 3] =
+            ffma2(a[(2 * j4 + 1) & 3], wv.z, wv.w, twice_relu(v0[4 * j4 + 2]), twice_relu(v0[4 * j4 + 3]));
     }
 #pragma unroll
     for (int j4 = 0; j4 < 8; ++j4) {
         const float4 wv = w4[8 + j4];
-        a[(2 * j4) & 3] = ffma2(a[(2 * j4) & 3], wv.x, wv.y, fmaxf(__uint_as_float(v1[4 * j4 + 0]), 0.0f),
-                                fmaxf(__uint_as_float(v1[4 * j4 + 1]), 0.0f));
-        a[(2 * j4 + 1) & 3] = ffma2(a[(2 * j4 + 1) & 3], wv.z, wv.w, fmaxf(__uint_as_float(v1[4 * j4 + 2]), 0.0f),
-                                    fmaxf(__uint_as_float(v1[4 * j4 + 3]), 0.0f));
+        a[(2 * j4) & 3] = ffma2(a[(2 * j4) & 3], wv.x, wv.y, twice_relu(v1[4 * j4 + 0]), twice_relu(v1[4 * j4 + 1]));
+        a[(2 * j4 + 1) & 3] =
+            ffma2(a[(2 * j4 + 1) & 3], wv.z, wv.w, twice_relu(v1[4 * j4 + 2]), twice_relu(v1[4 * j4 + 3]));
     }
     float s[8];
 #pragma unroll
     for (int i = 0; i < 4; ++i) asm("mov.b64 {%0, %1}, %2;" : "=f"(s[2 * i]), "=f"(s[2 * i + 1]) : "l"(a[i]));
     return ((s[0] + s[1]) + (s[2] + s[3])) + ((s[4] + s[5]) + (s[6] + s[7]));
-}
-
-// The same sum with scalar fma (reference form, unused by the kernel).
-__device__ __forceinline__ float head_reduce_scalar(const uint32_t (&v0)[32], const uint32_t (&v1)[32],
-                                                    const float *w) {
-    const float4 *w4 = reinterpret_cast<const float4 *>(w);
-    float a[8];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) a[i] = 0.0f;
-#pragma unroll
-    for (int j4 = 0; j4 < 8; ++j4) {
-        const float4 wv = w4[j4];
-        a[(4 * j4 + 0) & 7] = fmaf(wv.x, fmaxf(__uint_as_float(v0[4 * j4 + 0]), 0.0f), a[(4 * j4 + 0) & 7]);
-        a[(4 * j4 + 1) & 7] = fmaf(wv.y, fmaxf(__uint_as_float(v0[4 * j4 + 1]), 0.0f), a[(4 * j4 + 1) & 7]);
-        a[(4 * j4 + 2) & 7] = fmaf(wv.z, fmaxf(__uint_as_float(v0[4 * j4 + 2]), 0.0f), a[(4 * j4 + 2) & 7]);
-        a[(4 * j4 + 3) & 7] = fmaf(wv.w, fmaxf(__uint_as_float(v0[4 * j4 + 3]), 0.0f), a[(4 * j4 + 3) & 7]);
-    }
-#pragma unroll
-    for (int j4 = 0; j4 < 8; ++j4) {
-        const float4 wv = w4[8 + j4];
-        a[(4 * j4 + 0) & 7] = fmaf(wv.x, fmaxf(__uint_as_float(v1[4 * j4 + 0]), 0.0f), a[(4 * j4 + 0) & 7]);
-        a[(4 * j4 + 1) & 7] = fmaf(wv.y, fmaxf(__uint_as_float(v1[4 * j4 + 1]), 0.0f), a[(4 * j4 + 1) & 7]);
-        a[(4 * j4 + 2) & 7] = fmaf(wv.z, fmaxf(__uint_as_float(v1[4 * j4 + 2]), 0.0f), a[(4 * j4 + 2) & 7]);
-        a[(4 * j4 + 3) & 7] = fmaf(wv.w, fmaxf(__uint_as_float(v1[4 * j4 + 3]), 0.0f), a[(4 * j4 + 3) & 7]);
-    }
-    return ((a[0] + a[1]) + (a[2] + a[3])) + ((a[4] + a[5]) + (a[6] + a[7]));
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -152,7 +137,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc::mbar_init(&sh.qfull, 1);
         for (int h = 0; h < 2; ++h) {
             tc::mbar_init(&sh.tfull[h], 1);
-            tc::mbar_init(&sh.tempty[h], kEpiWarps);
+            tc::mbar_init(&sh.tempty[h], kEpiWarps / 2);
         }
         tc::mbar_init(&sh.drain, 1);
         sh.abort = 0;
@@ -190,9 +175,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 
         if (warp >= 2) {
             const int e = warp - 2;
-            // head weights of the block's rows, zero for rows past the request
+            // halved head weights of the block's rows, zero for rows past the request
             for (int i = threadIdx.x - 64; i < RB * TC_H; i += kEpiWarps * 32)
-                wsm[i] = (i / TC_H) < bi.nrows ? a.w[(long long)bi.row0 * TC_H + i] : 0.0f;
+                wsm[i] = (i / TC_H) < bi.nrows ? 0.5f * a.w[(long long)bi.row0 * TC_H + i] : 0.0f;
             if (e < RB) {
                 if (lane == 0) {
                     sh.bound[e] = e < bi.nrows ? key_bound(row_bound(bi.i0 + e, bi.n, a.g), a.kshift) : -1;
@@ -250,51 +235,61 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
             }
         } else {
+            // epilogue role: warps 2+4*role .. 5+4*role (one per TMEM lane
+            // quarter) own rows 2*role, 2*role+1 -- two queries of half role/2
             const int e = warp - 2;
+            const int role = e >> 2;
+            const int h = role >> 1;
+            const int ra = 2 * role;             // first of the role's two rows (h*4 + query)
             const int quarter = warp & 3;
-            const int qi = e >> 2;  // query of each half handled by this warp
             const int key_in_tile = quarter * 32 + lane;
+            const uint32_t tbase = tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(ra * 64);
+            const bool filter = a.sink == SINK_FILTER;
+            const int mrow = ra + (e & 1);       // row this warp maintains (warps with e & 3 < 2)
+            const bool maint = (e & 3) < 2 && mrow < bi.nrows;
             bool ok = true;
             for (int j = 0; j < ntiles; ++j) {
                 const uint32_t t = kt + j;
                 const int s = j * KT + key_in_tile;
-                for (int h = 0; h < 2; ++h) {
+                if (ok) ok = tc::mbar_wait(&sh.tfull[h], t & 1u, abort, a.status);
+                if (ok) tc::fence_after_sync();
+#pragma unroll
+                for (int q = 0; q < 2; ++q) {
                     float score = 0.0f;
-                    const int r = h * 4 + qi;
-                    if (ok) ok = tc::mbar_wait(&sh.tfull[h], t & 1u, abort, a.status);
+                    const int r = ra + q;
                     if (ok) {
-                        tc::fence_after_sync();
-                        const uint32_t taddr = tmem + ((uint32_t)(quarter * 32) << 16) + h * 256 + qi * 64;
                         uint32_t v0[32], v1[32];
-                        tc::tmem_ld32(taddr, v0);
-                        tc::tmem_ld32(taddr + 32, v1);
+                        tc::tmem_ld32(tbase + q * 64, v0);
+                        tc::tmem_ld32(tbase + q * 64 + 32, v1);
                         tc::tmem_wait_ld_all();
                         tc::reg_fence(v0);
                         tc::reg_fence(v1);
-                        tc::fence_before_sync();
-                        __syncwarp();
-                        if (lane == 0) tc::mbar_arrive(&sh.tempty[h]);
+                        if (q == 1) {
+                            tc::fence_before_sync();
+                            __syncwarp();
+                            tc::mbar_arrive_if(&sh.tempty[h], lane == 0);
+                        }
                         score = head_reduce(v0, v1, wsm + r * TC_H);
                     }
                     const bool valid = ok && s <= sh.bound[r];
-                    if (a.sink == SINK_FILTER) {
+                    if (filter) {
                         sel_offer(sh.sel[r], hist + r * kBins, a.buf + ((long long)bi.row0 + r) * a.cap, a.cap, valid,
                                   score, s, a.status);
                     } else if (valid && sh.slot[r] >= 0) {
                         a.spill[(long long)sh.slot[r] * a.ld + s] = score;
                     }
                 }
-                if (a.sink == SINK_FILTER && ((j % kMaintEvery) == kMaintEvery - 1 || j == ntiles - 1)) {
-                    tc::named_bar_sync(1, kEpiWarps * 32);
-                    if (e < bi.nrows)
-                        sel_maintain(sh.sel[e], hist + e * kBins, a.buf + ((long long)bi.row0 + e) * a.cap, a.cap,
-                                     a.ksel, scr + e * 256, KT * kMaintEvery);
-                    tc::named_bar_sync(1, kEpiWarps * 32);
+                if (filter && ((j % kMaintEvery) == kMaintEvery - 1 || j == ntiles - 1)) {
+                    tc::named_bar_sync(1 + role, 128);
+                    if (maint)
+                        sel_maintain(sh.sel[mrow], hist + mrow * kBins, a.buf + ((long long)bi.row0 + mrow) * a.cap,
+                                     a.cap, a.ksel, scr + mrow * 256, KT * kMaintEvery);
+                    tc::named_bar_sync(1 + role, 128);
                 }
             }
-            if (a.sink == SINK_FILTER && e < bi.nrows && lane == 0) {
-                a.cnt[bi.row0 + e] = sh.sel[e].cnt;
-                if (a.floor_out) a.floor_out[bi.row0 + e] = sh.sel[e].floor;
+            if (filter && maint && lane == 0) {
+                a.cnt[bi.row0 + mrow] = sh.sel[mrow].cnt;
+                if (a.floor_out) a.floor_out[bi.row0 + mrow] = sh.sel[mrow].floor;
             }
         }
         kt += ntiles;
