@@ -3,7 +3,8 @@
 TEST INFRASTRUCTURE ONLY: the plain, slow double-precision restatement of
 the lightning indexer + top-k (dense, PIVOT Reuse/Refine/block pre-filter,
 decode) and of the token-sparse attention over the selected positions that
-the CUDA library is checked against.  Only the tests, ``__graft_entry__.smoke``
+the CUDA library is checked against.  ``oracle.adaptive`` restates the
+adaptive top-k budget from the cutoff margin in numpy.  Only the tests, ``__graft_entry__.smoke``
 and the benchmark's CPU-baseline leg may import this package.  It imports
 nothing from the product package and the product imports nothing from it.
 
