@@ -15,6 +15,9 @@ pre-filter variant of Refine (candidates from 64-key block means) runs on
 the same packed batch under "block_prefilter", outside the step, and the
 token-sparse attention (absorbed-MLA shapes: 128 heads, 576/512 dims) over
 the dense selections of the last 16384 query rows under "sparse_attn".
+The dense pass with the cutoff-margin adaptive budget (rho = 2, q = 0.4:
+rows whose margin is in the bottom 40% keep 4096 positions, the others
+2048) runs on the single request under "adaptive".
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
@@ -56,6 +59,7 @@ def parse():
     p.add_argument("--no-decode", action="store_true")
     p.add_argument("--no-block", action="store_true")
     p.add_argument("--no-attn", action="store_true")
+    p.add_argument("--no-adaptive", action="store_true")
     p.add_argument("--attn-rows", type=int, default=16384)
     p.add_argument("--cpu-rows", type=int, default=64, help="oracle sample rows (dense + refine) per CPU step")
     p.add_argument("--no-cpu", action="store_true", help="skip the CPU-oracle baseline")
@@ -462,6 +466,46 @@ def main():
                "kernels": {n: {"launches": c, "ms_per_step": t / args.steps} for n, (c, t) in tra.items()}}
         del qa, kva, oa
 
+    # -------------------- adaptive budget from the cutoff margin (dense)
+    ada = None
+    if do_dense and not args.no_adaptive:
+        RHO_A, Q_A = 2, 0.4  # the router page's working values
+        wsad = torch.empty(idx.adaptive_workspace_size(L, H, D, TOPK, RHO_A, 1), dtype=torch.uint8, device=dev)
+        ai = torch.empty(L, RHO_A * TOPK, dtype=torch.int32, device=dev)
+        asc = torch.empty(L, RHO_A * TOPK, dtype=torch.float32, device=dev)
+        asg = torch.empty(L, dtype=torch.float32, device=dev)
+        atr = torch.empty(L, dtype=torch.uint8, device=dev)
+
+        def adstep():
+            idx.adaptive_topk(q, k, w, cu1, TOPK, RHO_A, Q_A, out_idx=ai, out_score=asc, out_sigma=asg,
+                              out_trigger=atr, workspace=wsad)
+
+        for _ in range(args.warmup):
+            adstep()
+        torch.cuda.synchronize()
+        assert idx.device_status(wsad) == "IDX_OK"
+        barrier()
+        lib.idx_trace_enable(1)
+        e0.record(stream)
+        for _ in range(args.steps):
+            adstep()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        lib.idx_trace_enable(0)
+        barrier()
+        adms = max_over_ranks(e0.elapsed_time(e1) / args.steps)
+        _, trd = trace_report(lib)
+        dense_ms = sum(v["ms_per_step"] for n, v in per_kernel.items() if n.startswith("dense/"))
+        ndef = int((~torch.isnan(asg)).sum().item())
+        ada = {"workload": f"adaptive_dense_{L}_k{TOPK}_rho{RHO_A}_q{Q_A}",
+               "ms_per_step": adms, "queries_per_s": world * L / (adms / 1000.0),
+               "ratio_to_dense_topk": adms / dense_ms if dense_ms > 0 else None,
+               "rows_with_margin": ndef, "triggered_rows": int(atr.sum().item()),
+               "mean_kept_per_row": float((ai >= 0).sum().item()) / L,
+               "page_accounting_kept": TOPK * (1 + Q_A * (RHO_A - 1)),
+               "kernels": {n: {"launches": c, "ms_per_step": t / args.steps} for n, (c, t) in trd.items()}}
+        del wsad, ai, asc, asg, atr
+
     # ------------------------------------------------------------- decode
     dec = None
     if not args.no_decode:
@@ -525,7 +569,8 @@ def main():
                    "g": G_REF, "c": C_REF, "parallelism": f"dp{world} (independent batches)",
                    "l2": "inputs larger than L2 (q is 2 GiB)"},
         "tflops_dense": achieved, "roofline": roof, "cpu_baseline": cpu, "e2e": e2e, "clocks": clk,
-        "gpu_launches": nlaunch, "kernels": per_kernel, "block_prefilter": blk, "sparse_attn": att, "decode": dec,
+        "gpu_launches": nlaunch, "kernels": per_kernel, "block_prefilter": blk, "sparse_attn": att,
+        "adaptive": ada, "decode": dec,
     }
     if rank == 0:
         print(json.dumps(line))

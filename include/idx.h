@@ -110,6 +110,36 @@ idx_status idx_dense_topk(const void *q, const void *k, const float *w, const in
                           int *out_idx, float *out_score, void *ws, size_t ws_bytes,
                           idx_stream_t stream);
 
+/* Workspace bytes for idx_adaptive_topk; 0 for arguments it would reject. */
+size_t idx_adaptive_workspace_size(int T, int H, int d, int topk, int rho, int num_seqs, idx_dtype dtype);
+
+/* Dense indexer + top-k with an adaptive budget ("Read the Cutoff", the
+ * sparse-attention router page: Section 3, steps 3-5, and Appendix A,
+ * steps (A.5)-(A.9)), on the indexer's per-query scores:
+ *   sigma[t] = (s_(k-1) - s_(k)) / (s_(0) - s_(k))   (fp32; s_(i) = the row's
+ *              i-th largest score; 0 when the first k+1 scores are equal;
+ *              NaN when the row has at most k positions);
+ *   tau      = the ceil(q n)-th smallest defined sigma over all T rows
+ *              (n = rows with a defined sigma, q n formed in fp64; no row
+ *              triggers when ceil(q n) = 0);
+ *   trigger  = sigma[t] <= tau;
+ * a triggered row lists its top-(rho topk); any other row its top-topk,
+ * padded with -1 to rho*topk entries.  Positions ascending, ties to the lower
+ * position, as in idx_dense_topk.
+ *   q, k, w, cu_seqlens  as in idx_dense_topk
+ *   rho          budget expansion, >= 2 (the page uses 2)
+ *   qfrac        trigger quantile in [0, 1] (the page uses 0.4)
+ *   out_idx      [T, rho*topk] int32
+ *   out_score    [T, rho*topk] fp32 or NULL (-inf on padding)
+ *   out_sigma    [T] fp32 or NULL
+ *   out_trigger  [T] uint8 or NULL (1 = the row kept rho*topk)
+ * Errors: rho < 2, qfrac outside [0, 1] or NaN, rho*topk overflowing int ->
+ * IDX_ERR_INVALID; otherwise as idx_dense_topk. */
+idx_status idx_adaptive_topk(const void *q, const void *k, const float *w, const int *cu_seqlens,
+                             int num_seqs, int T, int H, int d, int topk, int rho, double qfrac,
+                             idx_dtype dtype, int *out_idx, float *out_score, float *out_sigma,
+                             uint8_t *out_trigger, void *ws, size_t ws_bytes, idx_stream_t stream);
+
 /* Workspace bytes for idx_pivot_topk (mode REUSE, REFINE or BLOCK); 0 for
  * arguments idx_pivot_topk would reject. */
 size_t idx_pivot_workspace_size(int T, int H, int d, int topk, int num_seqs, idx_dtype dtype, int g,

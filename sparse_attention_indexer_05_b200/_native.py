@@ -18,6 +18,9 @@ _i, _sz, _ll = ctypes.c_int, ctypes.c_size_t, ctypes.c_longlong
 SIGNATURES = {
     "idx_dense_workspace_size": (_sz, [_i, _i, _i, _i, _i, _i]),
     "idx_dense_topk": (_i, [_vp, _vp, _fp, _ip, _i, _i, _i, _i, _i, _i, _ip, _fp, _vp, _sz, _vp]),
+    "idx_adaptive_workspace_size": (_sz, [_i, _i, _i, _i, _i, _i, _i]),
+    "idx_adaptive_topk": (_i, [_vp, _vp, _fp, _ip, _i, _i, _i, _i, _i, _i, ctypes.c_double, _i, _ip, _fp, _fp,
+                               _vp, _vp, _sz, _vp]),
     "idx_pivot_workspace_size": (_sz, [_i, _i, _i, _i, _i, _i, _i, _i, _i]),
     "idx_pivot_topk": (_i, [_vp, _vp, _fp, _ip, _i, _i, _i, _i, _i, _i, _i, _i, _i, _ip, _fp, _vp, _sz, _vp]),
     "idx_decode_workspace_size": (_sz, [_i, _i, _i, _i, _i, _i, _i, _i, _i]),

@@ -92,6 +92,26 @@ PrefillWs prefill_ws(int T, int H, int d, int topk, int S, idx_dtype dt, int g, 
     return L;
 }
 
+struct AdaptiveWs {
+    PrefillWs P;   // the dense top-(rho k) pass
+    size_t score, sigma, vk, need, tau, total;
+};
+
+AdaptiveWs adaptive_ws(int T, int H, int d, int topk, int rho, int S, idx_dtype dt) {
+    AdaptiveWs L{};
+    const int width = topk * rho;
+    L.P = prefill_ws(T, H, d, width, S, dt, 1, width, IDX_MODE_DENSE);
+    Carve cv;
+    cv.off = L.P.total;
+    L.score = cv.take((size_t)T * width * 4);
+    L.sigma = cv.take((size_t)T * 4);
+    L.vk = cv.take((size_t)T * 4);
+    L.need = cv.take((size_t)T * 4);
+    L.tau = cv.take(16);
+    L.total = cv.off;
+    return L;
+}
+
 struct DecodeWs {
     size_t status, qbar, wbar, spill, cand, msc, ckeys, total;
 };
@@ -302,6 +322,48 @@ idx_status idx_dense_topk(const void *q, const void *k, const float *w, const in
     TRY_CUDA(P.prepare());
     TRY_CUDA(P.score(P.score_args(false)));
     return cuda_st(launch_select(P.select_args(SEL_DENSE_CAND, T, topk, out_idx, out_score), P.st));
+}
+
+size_t idx_adaptive_workspace_size(int T, int H, int d, int topk, int rho, int num_seqs, idx_dtype dtype) {
+    if (T < 1 || num_seqs < 1 || topk < 1 || rho < 2 || !shape_ok(H, d, dtype)) return 0;
+    if ((long long)topk * rho > 0x7FFFFFFFLL) return 0;
+    return adaptive_ws(T, H, d, topk, rho, num_seqs, dtype).total;
+}
+
+idx_status idx_adaptive_topk(const void *q, const void *k, const float *w, const int *cu_seqlens, int num_seqs,
+                             int T, int H, int d, int topk, int rho, double qfrac, idx_dtype dtype, int *out_idx,
+                             float *out_score, float *out_sigma, uint8_t *out_trigger, void *ws, size_t ws_bytes,
+                             idx_stream_t stream) {
+    if (rho < 2 || !(qfrac >= 0.0 && qfrac <= 1.0) || topk < 1 || (long long)topk * rho > 0x7FFFFFFFLL)
+        return IDX_ERR_INVALID;
+    const int width = topk * rho;
+    const size_t need = idx_adaptive_workspace_size(T, H, d, topk, rho, num_seqs, dtype);
+    idx_status s = check_prefill(q, k, w, cu_seqlens, num_seqs, T, H, d, width, dtype, out_idx, ws, ws_bytes,
+                                 need);
+    if (s != IDX_OK) return s;
+    TracePhase phase("adaptive");
+    const AdaptiveWs L = adaptive_ws(T, H, d, topk, rho, num_seqs, dtype);
+    char *base = static_cast<char *>(ws);
+    Prefill P{q, k, w, cu_seqlens, num_seqs, T, H, d, width, dtype, 1, width, IDX_MODE_DENSE, base, L.P,
+              reinterpret_cast<cudaStream_t>(stream)};
+    TRY_CUDA(P.prepare());
+    TRY_CUDA(P.score(P.score_args(false)));
+    float *sc = out_score ? out_score : reinterpret_cast<float *>(base + L.score);
+    TRY_CUDA(launch_select(P.select_args(SEL_DENSE_CAND, T, width, out_idx, sc), P.st));
+    AdaptiveArgs a{};
+    a.T = T;
+    a.k = topk;
+    a.width = width;
+    a.idx = out_idx;
+    a.score = sc;
+    a.sigma = out_sigma ? out_sigma : reinterpret_cast<float *>(base + L.sigma);
+    a.vk = reinterpret_cast<unsigned *>(base + L.vk);
+    a.need = reinterpret_cast<int *>(base + L.need);
+    a.trigger = out_trigger;
+    a.tau = reinterpret_cast<unsigned *>(base + L.tau);
+    a.q = qfrac;
+    a.status = P.status();
+    return cuda_st(launch_adaptive(a, P.st));
 }
 
 size_t idx_pivot_workspace_size(int T, int H, int d, int topk, int num_seqs, idx_dtype dtype, int g, int c,

@@ -162,6 +162,22 @@ struct SelectArgs {
     unsigned *status;
 };
 
+// adaptive.cu: the adaptive budget from the cutoff margin over the rows of a
+// top-(rho k) result (in place).
+struct AdaptiveArgs {
+    long long T;
+    int k, width;             // width = rho * k
+    int *idx;                 // [T, width] ascending positions, -1 padded (in/out)
+    float *score;             // [T, width] their scores (in/out)
+    float *sigma;             // [T] cutoff margins (out)
+    unsigned *vk;             // [T] ord of s_(k-1) (scratch)
+    int *need;                // [T] ties of s_(k-1) the top-k keeps (scratch)
+    unsigned char *trigger;   // [T] or null (out)
+    unsigned *tau;            // [2] {tau defined, ord of tau} (scratch)
+    double q;                 // trigger quantile
+    unsigned *status;
+};
+
 // ---- tracing (trace.cu): a TraceScope around a launch records two events
 // on its stream while tracing is enabled; TracePhase names the entry-point
 // phase that prefixes the kernel names in the report.
@@ -187,6 +203,7 @@ cudaError_t launch_decode_tc(const DecodeArgs &a, cudaStream_t st);
 cudaError_t launch_gather_simt(const GatherArgs &a, int dtype, cudaStream_t st);
 cudaError_t launch_gather_tc(const GatherArgs &a, cudaStream_t st);
 cudaError_t launch_select(const SelectArgs &a, cudaStream_t st);
+cudaError_t launch_adaptive(const AdaptiveArgs &a, cudaStream_t st);
 cudaError_t launch_proxy(const void *q, const float *w, const int *cu, int S, int T, int H, int d,
                          int g, int dtype, const int *plan, const PlanLayout &pl, void *qbar,
                          float *wbar, int max_proxies, cudaStream_t st);

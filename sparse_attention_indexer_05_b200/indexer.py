@@ -69,6 +69,11 @@ def dense_workspace_size(T, H, d, topk, num_seqs, dtype=torch.bfloat16) -> int:
     return int(N.lib().idx_dense_workspace_size(T, H, d, topk, num_seqs, dt))
 
 
+def adaptive_workspace_size(T, H, d, topk, rho, num_seqs, dtype=torch.bfloat16) -> int:
+    dt = N.BF16 if dtype == torch.bfloat16 else N.F32
+    return int(N.lib().idx_adaptive_workspace_size(T, H, d, topk, rho, num_seqs, dt))
+
+
 def pivot_workspace_size(T, H, d, topk, num_seqs, g, c, mode, dtype=torch.bfloat16) -> int:
     dt = N.BF16 if dtype == torch.bfloat16 else N.F32
     return int(N.lib().idx_pivot_workspace_size(T, H, d, topk, num_seqs, dt, g, c, _mode(mode)))
@@ -101,6 +106,33 @@ def dense_topk(q, k, w, cu_seqlens, topk: int, out_idx=None, out_score=None, wor
         _dev(out_score, "out_score", torch.float32) if out_score is not None else None,
         ws.data_ptr(), ws.numel(), _stream(stream)), "idx_dense_topk")
     return (out_idx, out_score) if return_scores else out_idx
+
+
+def adaptive_topk(q, k, w, cu_seqlens, topk: int, rho: int = 2, qfrac: float = 0.4, out_idx=None, out_score=None,
+                  out_sigma=None, out_trigger=None, workspace=None, stream=None):
+    """Dense top-k with the cutoff-margin budget: rows whose margin sigma is in
+    the bottom qfrac of the call keep rho*topk positions, the others topk
+    (padded with -1).  Returns (idx [T, rho*topk], scores, sigma [T], trigger [T] uint8)."""
+    T, H, d = q.shape
+    S = cu_seqlens.numel() - 1
+    dt = _dtype_code(q)
+    width = rho * topk
+    ws = _ws(workspace, adaptive_workspace_size(T, H, d, topk, rho, S, q.dtype), q.device)
+    if out_idx is None:
+        out_idx = torch.empty(T, width, dtype=torch.int32, device=q.device)
+    if out_score is None:
+        out_score = torch.empty(T, width, dtype=torch.float32, device=q.device)
+    if out_sigma is None:
+        out_sigma = torch.empty(T, dtype=torch.float32, device=q.device)
+    if out_trigger is None:
+        out_trigger = torch.empty(T, dtype=torch.uint8, device=q.device)
+    N.check(N.lib().idx_adaptive_topk(
+        _dev(q, "q"), _dev(k, "k", q.dtype), _dev(w, "w", torch.float32), _dev(cu_seqlens, "cu_seqlens", torch.int32),
+        S, T, H, d, topk, rho, float(qfrac), dt, _dev(out_idx, "out_idx", torch.int32),
+        _dev(out_score, "out_score", torch.float32), _dev(out_sigma, "out_sigma", torch.float32),
+        _dev(out_trigger, "out_trigger", torch.uint8), ws.data_ptr(), ws.numel(), _stream(stream)),
+        "idx_adaptive_topk")
+    return out_idx, out_score, out_sigma, out_trigger
 
 
 def pivot_topk(q, k, w, cu_seqlens, topk: int, g: int, c: int, mode="refine", out_idx=None, out_score=None,

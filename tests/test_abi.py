@@ -26,7 +26,7 @@ def declared_functions():
 
 def test_exports_every_declared_symbol(lib):
     names = declared_functions()
-    assert len(names) == 18
+    assert len(names) == 20
     for n in names:
         assert hasattr(lib, n), n
         assert n in N.SIGNATURES, n
@@ -47,6 +47,21 @@ def test_workspace_sizes(lib):
     assert lib.idx_pivot_workspace_size(65536, 64, 128, 2048, 1, 0, 4, 4096, 0) == 0   # dense mode
     assert lib.idx_decode_workspace_size(64, 2, 131072, 64, 128, 2048, 4096, 2, 0) > 64 * 131072 * 4
     assert lib.idx_decode_workspace_size(64, 2, 1, 64, 128, 2048, 4096, 2, 0) == 0     # n_max < G
+
+
+def test_adaptive_workspace_and_argument_checks(lib):
+    assert lib.idx_adaptive_workspace_size(4096, 64, 128, 256, 2, 1, 0) > lib.idx_dense_workspace_size(
+        4096, 64, 128, 512, 1, 0)
+    assert lib.idx_adaptive_workspace_size(4096, 64, 128, 256, 1, 1, 0) == 0     # rho < 2
+    assert lib.idx_adaptive_workspace_size(4096, 64, 128, 1 << 30, 4, 1, 0) == 0  # rho*topk overflows
+    fake = ctypes.c_void_p(256)  # never dereferenced: the checks fail first
+    f = lib.idx_adaptive_topk
+    assert f(fake, fake, fake, fake, 1, 10, 4, 64, 8, 1, 0.4, 0, fake, None, None, None, fake, 1 << 30, None) == 1
+    assert f(fake, fake, fake, fake, 1, 10, 4, 64, 8, 2, 1.5, 0, fake, None, None, None, fake, 1 << 30, None) == 1
+    assert f(fake, fake, fake, fake, 1, 10, 4, 64, 8, 2, float("nan"), 0, fake, None, None, None, fake, 1 << 30,
+             None) == 1
+    assert f(None, fake, fake, fake, 1, 10, 4, 64, 8, 2, 0.4, 0, fake, None, None, None, fake, 1 << 30, None) == 1
+    assert f(fake, fake, fake, fake, 1, 10, 4, 64, 8, 2, 0.4, 0, fake, None, None, None, fake, 16, None) == 3
 
 
 def test_invalid_arguments_return_before_launch(lib):
