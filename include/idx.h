@@ -110,7 +110,8 @@ idx_status idx_dense_topk(const void *q, const void *k, const float *w, const in
                           int *out_idx, float *out_score, void *ws, size_t ws_bytes,
                           idx_stream_t stream);
 
-/* Workspace bytes for idx_adaptive_topk; 0 for arguments it would reject. */
+/* Workspace bytes for idx_adaptive_topk; 0 for arguments it would reject
+ * (including rho*topk above 8192). */
 size_t idx_adaptive_workspace_size(int T, int H, int d, int topk, int rho, int num_seqs, idx_dtype dtype);
 
 /* Dense indexer + top-k with an adaptive budget ("Read the Cutoff", the
@@ -133,8 +134,8 @@ size_t idx_adaptive_workspace_size(int T, int H, int d, int topk, int rho, int n
  *   out_score    [T, rho*topk] fp32 or NULL (-inf on padding)
  *   out_sigma    [T] fp32 or NULL
  *   out_trigger  [T] uint8 or NULL (1 = the row kept rho*topk)
- * Errors: rho < 2, qfrac outside [0, 1] or NaN, rho*topk overflowing int ->
- * IDX_ERR_INVALID; otherwise as idx_dense_topk. */
+ * Errors: rho < 2, qfrac outside [0, 1] or NaN -> IDX_ERR_INVALID;
+ * rho*topk above 8192 -> IDX_ERR_UNSUPPORTED; otherwise as idx_dense_topk. */
 idx_status idx_adaptive_topk(const void *q, const void *k, const float *w, const int *cu_seqlens,
                              int num_seqs, int T, int H, int d, int topk, int rho, double qfrac,
                              idx_dtype dtype, int *out_idx, float *out_score, float *out_sigma,

@@ -326,7 +326,7 @@ idx_status idx_dense_topk(const void *q, const void *k, const float *w, const in
 
 size_t idx_adaptive_workspace_size(int T, int H, int d, int topk, int rho, int num_seqs, idx_dtype dtype) {
     if (T < 1 || num_seqs < 1 || topk < 1 || rho < 2 || !shape_ok(H, d, dtype)) return 0;
-    if ((long long)topk * rho > 0x7FFFFFFFLL) return 0;
+    if ((long long)topk * rho > kAdaptiveMaxWidth) return 0;
     return adaptive_ws(T, H, d, topk, rho, num_seqs, dtype).total;
 }
 
@@ -336,6 +336,7 @@ idx_status idx_adaptive_topk(const void *q, const void *k, const float *w, const
                              idx_stream_t stream) {
     if (rho < 2 || !(qfrac >= 0.0 && qfrac <= 1.0) || topk < 1 || (long long)topk * rho > 0x7FFFFFFFLL)
         return IDX_ERR_INVALID;
+    if ((long long)topk * rho > kAdaptiveMaxWidth) return IDX_ERR_UNSUPPORTED;
     const int width = topk * rho;
     const size_t need = idx_adaptive_workspace_size(T, H, d, topk, rho, num_seqs, dtype);
     idx_status s = check_prefill(q, k, w, cu_seqlens, num_seqs, T, H, d, width, dtype, out_idx, ws, ws_bytes,

@@ -164,6 +164,7 @@ struct SelectArgs {
 
 // adaptive.cu: the adaptive budget from the cutoff margin over the rows of a
 // top-(rho k) result (in place).
+constexpr int kAdaptiveMaxWidth = 8192;  // rho * k held in registers by the margin kernel
 struct AdaptiveArgs {
     long long T;
     int k, width;             // width = rho * k

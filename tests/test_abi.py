@@ -54,6 +54,7 @@ def test_adaptive_workspace_and_argument_checks(lib):
         4096, 64, 128, 512, 1, 0)
     assert lib.idx_adaptive_workspace_size(4096, 64, 128, 256, 1, 1, 0) == 0     # rho < 2
     assert lib.idx_adaptive_workspace_size(4096, 64, 128, 1 << 30, 4, 1, 0) == 0  # rho*topk overflows
+    assert lib.idx_adaptive_workspace_size(4096, 64, 128, 4097, 2, 1, 0) == 0     # rho*topk above 8192
     fake = ctypes.c_void_p(256)  # never dereferenced: the checks fail first
     f = lib.idx_adaptive_topk
     assert f(fake, fake, fake, fake, 1, 10, 4, 64, 8, 1, 0.4, 0, fake, None, None, None, fake, 1 << 30, None) == 1
@@ -62,6 +63,8 @@ def test_adaptive_workspace_and_argument_checks(lib):
              None) == 1
     assert f(None, fake, fake, fake, 1, 10, 4, 64, 8, 2, 0.4, 0, fake, None, None, None, fake, 1 << 30, None) == 1
     assert f(fake, fake, fake, fake, 1, 10, 4, 64, 8, 2, 0.4, 0, fake, None, None, None, fake, 16, None) == 3
+    assert f(fake, fake, fake, fake, 1, 10, 4, 64, 4097, 2, 0.4, 0, fake, None, None, None, fake, 1 << 30,
+             None) == 2
 
 
 def test_invalid_arguments_return_before_launch(lib):
