@@ -469,7 +469,7 @@ def main():
     # -------------------- adaptive budget from the cutoff margin (dense)
     ada = None
     if do_dense and not args.no_adaptive:
-        RHO_A, Q_A = 2, 0.4  # the router page's working values
+        RHO_A, Q_A = 2, 0.4  # the working values of the uncertainty-gated selection page (Sec. 3.4, 3.5)
         wsad = torch.empty(idx.adaptive_workspace_size(L, H, D, TOPK, RHO_A, 1), dtype=torch.uint8, device=dev)
         ai = torch.empty(L, RHO_A * TOPK, dtype=torch.int32, device=dev)
         asc = torch.empty(L, RHO_A * TOPK, dtype=torch.float32, device=dev)

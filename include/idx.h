@@ -114,9 +114,9 @@ idx_status idx_dense_topk(const void *q, const void *k, const float *w, const in
  * (including rho*topk above 8192). */
 size_t idx_adaptive_workspace_size(int T, int H, int d, int topk, int rho, int num_seqs, idx_dtype dtype);
 
-/* Dense indexer + top-k with an adaptive budget ("Read the Cutoff", the
- * sparse-attention router page: Section 3, steps 3-5, and Appendix A,
- * steps (A.5)-(A.9)), on the indexer's per-query scores:
+/* Dense indexer + top-k with an adaptive budget ("Uncertainty-gated
+ * selection for block-sparse attention", Section 3 Method, steps 3-5, and
+ * Appendix A, steps (A.5)-(A.9)), on the indexer's per-query scores:
  *   sigma[t] = (s_(k-1) - s_(k)) / (s_(0) - s_(k))   (fp32; s_(i) = the row's
  *              i-th largest score; 0 when the first k+1 scores are equal;
  *              NaN when the row has at most k positions);

@@ -2,8 +2,8 @@
 
 TEST INFRASTRUCTURE ONLY (part of the oracle package; see ``oracle/__init__``).
 
-Follows "Read the Cutoff" (the sparse-attention router page), Section 3,
-steps 3-5, and its Appendix A, steps (A.5)-(A.9), applied to the lightning
+Follows "Uncertainty-gated selection for block-sparse attention", Section 3
+(Method), steps 3-5, and its Appendix A, steps (A.5)-(A.9), applied to the lightning
 indexer's per-query scores instead of per-tile block scores:
 
 * (A.5) sort the row's candidates by (score desc, position asc) and keep the

@@ -1,6 +1,7 @@
-// adaptive.cu -- adaptive top-k budget from the cutoff margin ("Read the
-// Cutoff", the sparse-attention router page: Section 3, steps 3-5, and
-// Appendix A, steps (A.5)-(A.9)), applied to the indexer's per-query scores.
+// adaptive.cu -- adaptive top-k budget from the cutoff margin
+// ("Uncertainty-gated selection for block-sparse attention", Section 3
+// Method, steps 3-5, and Appendix A, steps (A.5)-(A.9)), applied to the
+// indexer's per-query scores.
 //
 // Input: the dense top-(rho k) of every row (ascending positions, -1 padded)
 // with its fp32 scores.  Three launches:
