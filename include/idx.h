@@ -219,15 +219,27 @@ idx_status idx_decode_paged_topk(const void *q, const void *kpool, const int *bl
  *     return IDX_ERR_UNSUPPORTED with a message on stderr and launch nothing.
  *   - The first call on a device looks up the array's device address
  *     (cudaGetSymbolAddress); make that first call before any stream capture.
+ *     The address is kept per device together with the id of the context it
+ *     came from, and looked up again when the current context differs (after
+ *     cudaDeviceReset the module, and with it the array, is loaded anew).
  *   - Every call uses the same array, which keeps the last call's contents
  *     (the status word is cleared at the start of each call): calls whose
  *     kernels overlap on the GPU -- other streams, other host threads --
  *     race and corrupt each other's results.  Order them on one stream.
- *   - The device status word lives in the shared array and is not
- *     returned; requests whose kv_len is out of range come back as rows of -1. */
+ *   - Arguments idx_decode_topk rejects are rejected with the same code.
+ *   - The device status word lives in the shared array; read it with
+ *     idx_decode_noalloc_status() after the call (requests whose kv_len is
+ *     out of range come back as rows of -1 and IDX_ERR_INVALID there; a
+ *     bounded wait that ran out gives IDX_ERR_TIMEOUT and invalid rows). */
 idx_status idx_decode_topk_noalloc(const void *q, const void *kcache, const int *kv_len, const float *w,
                                    int B, int G, int n_max, int H, int d, int topk, idx_dtype dtype,
                                    int *out_idx, float *out_score, idx_stream_t stream);
+
+/* Device status of the last idx_decode_topk_noalloc call on the current
+ * device, as idx_device_status() reports it for a workspace: synchronises
+ * `stream` (the stream of that call), then reads the status word out of the
+ * library's fixed array.  Allocates nothing. */
+idx_status idx_decode_noalloc_status(idx_stream_t stream);
 
 /* --------------------------------------------- token-sparse attention */
 

@@ -41,14 +41,42 @@ def stale() -> bool:
     return any(os.path.getmtime(p) > t for p in deps())
 
 
+OBJ_DIR = os.path.join(os.path.dirname(HERE), "_build")
+
+
 def build(force: bool = False, verbose: bool = False) -> str:
+    """Compile every source to an object in parallel (each .cu holds its own
+    kernels and launchers: whole-program compilation per file), then link."""
     if not force and not stale():
         return LIB
+    from concurrent.futures import ThreadPoolExecutor
     nvcc = os.environ.get("NVCC", "nvcc")
-    cmd = [nvcc, *NVCC_FLAGS, "-o", LIB, *sources()]
+    os.makedirs(OBJ_DIR, exist_ok=True)
+    cflags = [f for f in NVCC_FLAGS if f != "-shared"]
+    objs, cmds = [], []
+    for src in sources():
+        obj = os.path.join(OBJ_DIR, os.path.basename(src)[:-3] + ".o")
+        objs.append(obj)
+        cmds.append([nvcc, *cflags, "-c", "-o", obj, src])
+
+    def run(cmd):
+        if verbose:
+            print(" ".join(cmd))
+        return subprocess.run(cmd, capture_output=True, text=True)
+
+    with ThreadPoolExecutor(max_workers=min(len(cmds), os.cpu_count() or 1)) as ex:
+        results = list(ex.map(run, cmds))
+    for cmd, r in zip(cmds, results):
+        if r.stdout or r.stderr:
+            sys.stdout.write(r.stdout)
+            sys.stderr.write(r.stderr)
+        if r.returncode != 0:
+            raise subprocess.CalledProcessError(r.returncode, cmd)
+    link = [nvcc, "-gencode", "arch=compute_100a,code=sm_100a", "-shared", "-Xcompiler", "-fPIC", "-o", LIB,
+            *objs]
     if verbose:
-        print(" ".join(cmd))
-    subprocess.run(cmd, check=True)
+        print(" ".join(link))
+    subprocess.run(link, check=True)
     return LIB
 
 

@@ -6,8 +6,11 @@ its scratch is a fixed device array inside the library.  The test calls it
 through the C ABI twice in a row, on different inputs, and checks each
 result against the workspace-taking idx_decode_topk (dense mode): the same
 indices, and scores within the tolerance of the other parity tests.  It
-also checks that a call too large for the fixed scratch is refused.  This
-file is collected last so that a failure here leaves every other test run.
+also checks that a call too large for the fixed scratch is refused, that
+arguments the workspace entry point rejects are rejected with the same
+code, and that the device status word of the fixed scratch is reported by
+idx_decode_noalloc_status.  This file is collected last so that a failure
+here leaves every other test run.
 """
 import numpy as np
 import pytest
@@ -54,3 +57,47 @@ def test_noalloc_refuses_calls_beyond_its_scratch():
     fake = 256  # never dereferenced: the size check fails before any launch
     rc = f(fake, fake, fake, fake, 64, 2, 131072, 64, 128, 2048, N.BF16, fake, None, None)
     assert rc == 2  # IDX_ERR_UNSUPPORTED
+
+
+def test_noalloc_rejects_what_the_workspace_entry_point_rejects():
+    from sparse_attention_indexer_05_b200 import _native as N
+    L = N.lib()
+    fake = 256  # never dereferenced: the argument checks fail before any launch
+    cases = [
+        (0, 2, 4096),     # no request
+        (4, 9, 4096),     # more MTP queries than one row block holds
+        (4, 2, 1),        # cache shorter than the query group
+        (4, 2, 1 << 21),  # cache longer than the supported maximum
+    ]
+    for B, G, n in cases:
+        a = L.idx_decode_topk_noalloc(fake, fake, fake, fake, B, G, n, 64, 128, 64, N.BF16, fake, None, None)
+        b = L.idx_decode_topk(fake, fake, fake, fake, B, G, n, 64, 128, 64, 0, N.MODE_DENSE, N.BF16, fake, None,
+                              fake, 1 << 40, None)
+        assert a == b and a != 0, (B, G, n, a, b)
+
+
+def test_noalloc_status_word_is_reported():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from sparse_attention_indexer_05_b200 import _native as N
+    L = N.lib()
+    topk = 64
+    D = W.decode(B=2, n=600, G=2, H=64, d=128, topk=topk, seed=3, kv_len=[600, 300])
+    q, kc, w = to_dev(D.q), to_dev(D.kcache), to_dev(D.w)
+    out_idx = torch.empty((2, 2, topk), dtype=torch.int32, device="cuda")
+    st = torch.cuda.current_stream().cuda_stream
+
+    def call(kv):
+        kvl = torch.tensor(kv, dtype=torch.int32, device="cuda")
+        rc = L.idx_decode_topk_noalloc(q.data_ptr(), kc.data_ptr(), kvl.data_ptr(), w.data_ptr(), 2, 2, 600, 64,
+                                       128, topk, N.BF16, out_idx.data_ptr(), None, st)
+        assert rc == 0, N.STATUS.get(rc, rc)
+        return L.idx_decode_noalloc_status(st)
+
+    assert call([600, 300]) == 0
+    # request 1 claims more keys than the cache holds: caught on the device,
+    # its rows come back as -1 and the status word says IDX_ERR_INVALID
+    assert call([600, 601]) == 1
+    assert (out_idx[1] == -1).all()
+    # the next call clears the status word again
+    assert call([600, 300]) == 0
