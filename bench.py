@@ -61,7 +61,13 @@ def parse():
     p.add_argument("--no-attn", action="store_true")
     p.add_argument("--no-adaptive", action="store_true")
     p.add_argument("--attn-rows", type=int, default=16384)
-    p.add_argument("--cpu-rows", type=int, default=64, help="oracle sample rows (dense + refine) per CPU step")
+    p.add_argument("--cpu-rows", type=int, default=512, help="oracle sample rows (dense + refine) per CPU step")
+    p.add_argument("--no-configs", action="store_true",
+                   help="skip the 16384-token dense and 65536-token PIVOT (g=4, c=4096) legs")
+    p.add_argument("--crossover", action="store_true",
+                   help="only time dense, Reuse and Refine on single requests of 1K..64K tokens (g=4, 16)")
+    p.add_argument("--dense-below", type=int, default=0,
+                   help="--crossover: also time PIVOT with this guardrail threshold (0 = without)")
     p.add_argument("--no-cpu", action="store_true", help="skip the CPU-oracle baseline")
     p.add_argument("--tokens", type=int, default=L_TOK,
                    help="batch length (profiling runs use a smaller case; the bench line uses 131072)")
@@ -72,6 +78,10 @@ def parse():
 
 def dense_flops_single(L=L_TOK):
     return 2.0 * H * D * L * (L + 1) / 2.0
+
+
+def causal_flops(lengths):
+    return sum(2.0 * H * D * n * (n + 1) / 2.0 for n in lengths)
 
 
 def proxy_pairs(n, g):
@@ -192,6 +202,139 @@ def pinned(a):
     return t.pin_memory()
 
 
+
+def timed_calls(fn, warmup, steps, lib, barrier, max_over_ranks):
+    """Run fn warmup times, then time `steps` calls with CUDA events on the
+    current stream (library tracer on); returns (ms per call, max over ranks,
+    and the per-kernel split {name: (launches, ms per call)})."""
+    import torch
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    lib.idx_trace_enable(1)
+    e0.record(stream)
+    for _ in range(steps):
+        fn()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    lib.idx_trace_enable(0)
+    barrier()
+    ms = max_over_ranks(e0.elapsed_time(e1) / steps)
+    _, tr = trace_report(lib)
+    return ms, {n: (c, t / steps) for n, (c, t) in tr.items()}
+
+
+def kernel_ms(split, suffix, prefix=None):
+    return sum(t for n, (c, t) in split.items()
+               if n.endswith(suffix) and (prefix is None or n.startswith(prefix + "/")))
+
+
+def run_configs(args, dev, lib, barrier, max_over_ranks, rank, bf16_sus):
+    """The 16384-token dense case and the 65536-token PIVOT case (g=4,
+    c=4096: dense, Reuse and Refine on the same inputs), each with the
+    score kernel's rate against the sustained bf16 peak."""
+    import torch
+
+    import sparse_attention_indexer_05_b200 as idx
+    from sparse_attention_indexer_05_b200 import multirank as M
+    from sparse_attention_indexer_05_b200 import workloads as W
+    out = {}
+
+    def dense_leg(P, label):
+        T = P.T
+        q, k, w = to_dev(P.q, dev), to_dev(P.k, dev), to_dev(P.w, dev)
+        cu = to_dev(P.cu_seqlens, dev)
+        S = len(P.cu_seqlens) - 1
+        o = torch.empty(T, TOPK, dtype=torch.int32, device=dev)
+        ws = torch.empty(idx.dense_workspace_size(T, H, D, TOPK, S), dtype=torch.uint8, device=dev)
+        ms, sp = timed_calls(lambda: idx.dense_topk(q, k, w, cu, TOPK, out_idx=o, workspace=ws), args.warmup,
+                             args.steps, lib, barrier, max_over_ranks)
+        assert idx.device_status(ws) == "IDX_OK"
+        sms = kernel_ms(sp, "score_tc", "dense")
+        fl = causal_flops(P.meta["lengths"])
+        tf = fl / (sms / 1000.0) / 1e12 if sms > 0 else None
+        del ws
+        return {"workload": label, "ms_per_call": ms, "queries_per_s": T / (ms / 1000.0),
+                "score_tc": {"ms": sms, "flops": fl, "tflops": tf, "frac_bf16_sustained": (tf / bf16_sus) if tf else None},
+                "kernels_ms": {n: t for n, (c, t) in sp.items()}}, (q, k, w, cu, o)
+
+    # dense L = 16384 (rho 0.95, 1% planted keys)
+    P2 = W.cfg_dense_16k(seed=M.rank_seed(rank))
+    out["dense_16384"], _ = dense_leg(P2, "dense_L16384_H64_d128_k2048")
+    del P2
+    # PIVOT L = 65536, g = 4, c = 4096 against dense on the same inputs
+    P3 = W.cfg_pivot_64k(seed=M.rank_seed(rank))
+    res, (q, k, w, cu, o) = dense_leg(P3, "dense_L65536_H64_d128_k2048")
+    leg = {"dense": res}
+    T = P3.T
+    for mode in ("reuse", "refine"):
+        ws = torch.empty(idx.pivot_workspace_size(T, H, D, TOPK, 1, 4, 4096, mode), dtype=torch.uint8, device=dev)
+        ms, sp = timed_calls(lambda: idx.pivot_topk(q, k, w, cu, TOPK, 4, 4096, mode, out_idx=o, workspace=ws),
+                             args.warmup, args.steps, lib, barrier, max_over_ranks)
+        assert idx.device_status(ws) == "IDX_OK"
+        sms = kernel_ms(sp, "score_tc", mode)
+        fl = 2.0 * H * D * proxy_pairs(T, 4)
+        tf = fl / (sms / 1000.0) / 1e12 if sms > 0 else None
+        leg[mode] = {"ms_per_call": ms, "queries_per_s": T / (ms / 1000.0),
+                     "speedup_vs_dense": res["ms_per_call"] / ms,
+                     "proxy_scan": {"ms": sms, "flops": fl, "tflops": tf,
+                                    "frac_bf16_sustained": (tf / bf16_sus) if tf else None},
+                     "kernels_ms": {n: t for n, (c, t) in sp.items()}}
+        del ws
+    leg["workload"] = "pivot_L65536_g4_c4096_H64_d128_k2048 (dense, Reuse and Refine on the same inputs)"
+    out["pivot_65536_g4_c4096"] = leg
+    del q, k, w, cu, o, P3
+    torch.cuda.empty_cache()
+    return out
+
+
+def run_crossover(args):
+    """Dense against PIVOT Reuse and Refine (c = 4096) on one request of
+    L tokens, L = 1K .. 64K, g = 4 and 16: the inputs of the 65536-token
+    recipe cut to their first L tokens (a prefix of a request is a request)."""
+    import torch
+
+    import sparse_attention_indexer_05_b200 as idx
+    from sparse_attention_indexer_05_b200 import _native as N
+    from sparse_attention_indexer_05_b200 import workloads as W
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    lib = N.lib()
+    P = W.cfg_pivot_64k(seed=0)
+    qa, ka, wa = to_dev(P.q, dev), to_dev(P.k, dev), to_dev(P.w, dev)
+    guard = args.dense_below
+    rows = []
+    for L in (1024, 2048, 4096, 8192, 12288, 16384, 24576, 32768, 49152, 65536):
+        q, k, w = qa[:L].contiguous(), ka[:L].contiguous(), wa[:L].contiguous()
+        cu = torch.tensor([0, L], dtype=torch.int32, device=dev)
+        o = torch.empty(L, TOPK, dtype=torch.int32, device=dev)
+        ws = torch.empty(idx.dense_workspace_size(L, H, D, TOPK, 1), dtype=torch.uint8, device=dev)
+        dms, _ = timed_calls(lambda: idx.dense_topk(q, k, w, cu, TOPK, out_idx=o, workspace=ws), 2, 5, lib,
+                             lambda: None, float)
+        row = {"L": L, "dense_ms": dms}
+        del ws
+        for g in (4, 16):
+            for mode in ("reuse", "refine"):
+                for db in ((0, guard) if guard else (0,)):
+                    kw = {"dense_below": db} if db else {}
+                    ws = torch.empty(idx.pivot_workspace_size(L, H, D, TOPK, 1, g, 4096, mode, **kw),
+                                     dtype=torch.uint8, device=dev)
+                    ms, _ = timed_calls(lambda: idx.pivot_topk(q, k, w, cu, TOPK, g, 4096, mode, out_idx=o,
+                                                               workspace=ws, **kw),
+                                        2, 5, lib, lambda: None, float)
+                    key = f"{mode}_g{g}" + (f"_guard{db}" if db else "")
+                    row[key + "_ms"] = ms
+                    row[key + "_speedup"] = dms / ms
+                    del ws
+        rows.append(row)
+        print(json.dumps(row), flush=True)
+    print(json.dumps({"crossover": rows, "c": 4096, "topk": TOPK,
+                      "workload": "prefixes of the 65536-token recipe (rho 0.95, 1% planted keys), one request"}))
+    return 0
+
 # ---------------------------------------------------------------- CPU oracle
 def oracle_sample(P, nrows, seed=0):
     """Time the oracle on `nrows` rows of the step (half dense on the single
@@ -212,7 +355,8 @@ def oracle_sample(P, nrows, seed=0):
     O.pivot_topk(P.q, P.k, P.w, cu2, TOPK, G_REF, C_REF, O.REFINE, rows=ref_rows, threads=threads)
     dt = time.perf_counter() - t0
     desc = (f"{nd} dense rows (single 131072-token request) + {nr} Refine g=16 c=4096 member rows "
-            f"(2x65536 packed), stratified by position, seed {seed}")
+            f"(2x65536 packed), stratified by position, seed {seed}; the rate is extrapolated to the "
+            f"step's {2 * L_TOK} rows (a stratified sample has the batch's mean prefix)")
     return (nd + nr) / dt, dt, threads, desc
 
 
@@ -249,6 +393,8 @@ def main():
     args = parse()
     if args.impl == "reference":
         return run_reference(args)
+    if args.crossover:
+        return run_crossover(args)
     import torch
 
     import sparse_attention_indexer_05_b200 as idx
@@ -324,6 +470,22 @@ def main():
             "flops_per_launch": dense_flops_single(L), "ms_per_launch": dense_ms}
 
     per_kernel = {name: {"launches": c, "ms_total": t, "ms_per_step": t / args.steps} for name, (c, t) in tr.items()}
+
+    # ----------- Refine g=16 against dense on the same 2 x 65536 packing
+    packed = None
+    if args.only == "all" and not args.no_configs:
+        wsp = torch.empty(idx.dense_workspace_size(L, H, D, TOPK, 2), dtype=torch.uint8, device=dev)
+        pd_ms, pd_sp = timed_calls(lambda: idx.dense_topk(q, k, w, cu2, TOPK, out_idx=o1, workspace=wsp),
+                                   args.warmup, args.steps, lib, barrier, max_over_ranks)
+        assert idx.device_status(wsp) == "IDX_OK"
+        del wsp
+        pr_ms, pr_sp = timed_calls(lambda: idx.pivot_topk(q, k, w, cu2, TOPK, G_REF, C_REF, "refine", out_idx=o2,
+                                                          workspace=ws2), args.warmup, args.steps, lib, barrier,
+                                   max_over_ranks)
+        packed = {"workload": f"packed_2x{L // 2}_g{G_REF}_c{C_REF} (dense and Refine on the same inputs)",
+                  "dense_ms": pd_ms, "refine_ms": pr_ms, "speedup_refine_vs_dense": pd_ms / pr_ms,
+                  "dense_score_tc_ms": kernel_ms(pd_sp, "score_tc"),
+                  "refine_kernels_ms": {n: t for n, (c, t) in pr_sp.items()}}
 
     # ---------------------------------------------------------------- e2e
     # Every step copies its inputs in from pinned host memory and reads its
@@ -506,6 +668,11 @@ def main():
                "kernels": {n: {"launches": c, "ms_per_step": t / args.steps} for n, (c, t) in trd.items()}}
         del wsad, ai, asc, asg, atr
 
+    # ---------------------------- the 16384 dense and 65536 PIVOT configs
+    cfgs = None
+    if args.only == "all" and not args.no_configs and L == L_TOK:
+        cfgs = run_configs(args, dev, lib, barrier, max_over_ranks, rank, bf16_sus)
+
     # ------------------------------------------------------------- decode
     dec = None
     if not args.no_decode:
@@ -570,7 +737,8 @@ def main():
                    "l2": "inputs larger than L2 (q is 2 GiB)"},
         "tflops_dense": achieved, "roofline": roof, "cpu_baseline": cpu, "e2e": e2e, "clocks": clk,
         "gpu_launches": nlaunch, "kernels": per_kernel, "block_prefilter": blk, "sparse_attn": att,
-        "adaptive": ada, "decode": dec,
+        "adaptive": ada, "decode": dec, "configs": cfgs,
+        "packed_refine_vs_dense": packed,
     }
     if rank == 0:
         print(json.dumps(line))

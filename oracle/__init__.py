@@ -40,7 +40,7 @@ def load(path: str) -> ctypes.CDLL:
         L.ora_group_proxy.argtypes = [vp, fp, i, i, i, ll, i, vp, fp]
         L.ora_dense_topk.argtypes = [vp, vp, fp, i, ip, i, i, i, i, llp, i, ip, i]
         L.ora_block_mean.argtypes = [vp, i, i, ll, i, vp]
-        L.ora_pivot_topk.argtypes = [vp, vp, fp, i, ip, i, i, i, i, i, i, i, i, llp, i, ip, i]
+        L.ora_pivot_topk.argtypes = [vp, vp, fp, i, ip, i, i, i, i, i, i, i, i, i, llp, i, ip, i]
         L.ora_decode_topk.argtypes = [vp, vp, fp, i, ip, i, i, i, i, i, i, i, i, i, llp, i, ip, i]
         L.ora_sparse_attn.argtypes = [vp, vp, i, ip, ip, ip, i, i, i, i, i, ctypes.c_double, llp, i, dp, dp, i]
         for f in (L.ora_score_row, L.ora_select, L.ora_group_proxy, L.ora_block_mean, L.ora_dense_topk,
@@ -163,9 +163,11 @@ def dense_topk(q, k, w, cu_seqlens, topk: int, rows=None, threads=None) -> np.nd
 
 
 def pivot_topk(q, k, w, cu_seqlens, topk: int, g: int, c: int, mode: int, rows=None,
-               threads=None, bn: int = 64) -> np.ndarray:
+               threads=None, bn: int = 64, dense_below: int = 0) -> np.ndarray:
     """PIVOT Reuse (mode=REUSE), Refine (mode=REFINE) or Refine over block
-    pre-filter candidates (mode=BLOCK, block size bn) top-k of member rows."""
+    pre-filter candidates (mode=BLOCK, block size bn) top-k of member rows.
+    Groups whose last member's prefix holds at most dense_below keys take the
+    dense top-k (the guardrail; 0 = off)."""
     q = np.ascontiguousarray(q); k = np.ascontiguousarray(k); w = _c(w, np.float32)
     cu = _c(cu_seqlens, np.int32)
     dt = _dtype_code(q)
@@ -173,7 +175,8 @@ def pivot_topk(q, k, w, cu_seqlens, topk: int, g: int, c: int, mode: int, rows=N
     r = _rows(rows, T)
     out = np.empty((len(r), topk), np.int32)
     _check(lib().ora_pivot_topk(_ptr(q), _ptr(k), _ptr(w, ctypes.c_float), dt, _ptr(cu, ctypes.c_int),
-                                len(cu) - 1, H, d, topk, g, c, mode, bn, _ptr(r, ctypes.c_longlong),
+                                len(cu) - 1, H, d, topk, g, c, mode, bn, int(dense_below),
+                                _ptr(r, ctypes.c_longlong),
                                 len(r), _ptr(out, ctypes.c_int), _threads(threads)), "pivot_topk")
     return out
 

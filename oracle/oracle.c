@@ -29,6 +29,12 @@
  *        then PIVOT-Refine re-scores it with each member's own indexer.
  *      Method, decode paragraph: the decode group is the current query plus
  *        the MTP draft queries of the same step.
+ *      Results, indexer speed: PIVOT falls back to a dense scan for short
+ *        groups, so it is never slower than the dense indexer.  The
+ *        threshold is not given; here it is an argument, dense_below: a
+ *        group whose shared scan would cover at most dense_below keys
+ *        (t_last + 1 <= dense_below) is not grouped, every member scores its
+ *        own prefix and takes its own top-k.  dense_below = 0 turns it off.
  *  - Block pre-filter (mode ORA_BLOCK), a candidate generator for Refine built
  *    from two other pages: "Not All Tokens Deserve Equal Resolution:
  *    Score-Adaptive Indexing for Sparse Attention in Long-Context LLMs"
@@ -330,7 +336,7 @@ typedef struct {
     int kind; /* 0 dense, 1 pivot, 2 decode */
     const void *q, *k;
     const float *w;
-    int dtype, H, d, topk, g, c, mode, bn;
+    int dtype, H, d, topk, g, c, mode, bn, dense_below;
     const int *cu;
     int num_seqs;
     const long long *rows;
@@ -380,6 +386,12 @@ static void run_pivot_row(job_t *J, int i) {
     int t = (int)(r - J->cu[b]);
     int lo = (t / J->g) * J->g;
     int hi = lo + J->g < n ? lo + J->g : n;
+    /* a short group (its last member's prefix holds at most dense_below
+     * keys) falls back to the dense top-k of each member */
+    if (J->dense_below > 0 && hi <= J->dense_below) {
+        run_dense_row(J, i);
+        return;
+    }
     set_rc(J, grouped_member_topk(J->q, J->k, J->w, J->dtype, J->H, J->d, J->cu[b] + lo, hi - lo, lo,
                                   J->cu[b], J->topk, J->c, J->mode, J->bn, t - lo,
                                   J->out + (size_t)i * J->topk));
@@ -467,11 +479,14 @@ int ora_dense_topk(const void *q, const void *k, const float *w, int dtype, cons
 
 /* PIVOT top-k (mode ORA_REUSE, ORA_REFINE or ORA_BLOCK) for the given
  * global member rows; same layouts as ora_dense_topk; g >= 1; Refine and
- * Block need c >= topk; Block needs bn >= 1 (c / bn blocks). */
+ * Block need c >= topk; Block needs bn >= 1 (c / bn blocks).  Groups whose
+ * last member's prefix holds at most dense_below keys (0 = none) take the
+ * dense top-k instead. */
 int ora_pivot_topk(const void *q, const void *k, const float *w, int dtype, const int *cu_seqlens,
-                   int num_seqs, int H, int d, int topk, int g, int c, int mode, int bn,
+                   int num_seqs, int H, int d, int topk, int g, int c, int mode, int bn, int dense_below,
                    const long long *rows, int nrows, int *out, int nthreads) {
-    if (!q || !k || !w || !out || (nrows > 0 && !rows) || H <= 0 || d <= 0 || topk <= 0 || g <= 0)
+    if (!q || !k || !w || !out || (nrows > 0 && !rows) || H <= 0 || d <= 0 || topk <= 0 || g <= 0 ||
+        dense_below < 0)
         return 1;
     if (mode != ORA_REUSE && mode != ORA_REFINE && mode != ORA_BLOCK) return 1;
     if ((mode == ORA_REFINE || mode == ORA_BLOCK) && c < topk) return 1;
@@ -482,7 +497,8 @@ int ora_pivot_topk(const void *q, const void *k, const float *w, int dtype, cons
     job_t J;
     memset(&J, 0, sizeof J);
     J.kind = 1; J.q = q; J.k = k; J.w = w; J.dtype = dtype; J.H = H; J.d = d; J.topk = topk;
-    J.g = g; J.c = c; J.mode = mode; J.bn = bn; J.cu = cu_seqlens; J.num_seqs = num_seqs; J.rows = rows;
+    J.g = g; J.c = c; J.mode = mode; J.bn = bn; J.dense_below = dense_below;
+    J.cu = cu_seqlens; J.num_seqs = num_seqs; J.rows = rows;
     J.nrows = nrows; J.out = out;
     return run_job(&J, nthreads);
 }

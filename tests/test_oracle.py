@@ -69,6 +69,44 @@ def pin_hand_topk():
         assert got.tolist() == want, ("refine", tag, got.tolist(), want)
 
 
+def pin_hand_guardrail():
+    """The guardrail on the hand example: dense rows for short groups, PIVOT rows otherwise."""
+    G, q, k, w = _hand()
+    cu = np.array([0, 4], np.int32)
+    Gd = G["guarded_g2"]
+    for db, want in Gd["reuse_k1"].items():
+        got = O.pivot_topk(q, k, w, cu, 1, 2, 1, O.REUSE, dense_below=int(db))
+        assert got.tolist() == want, ("reuse k1", db, got.tolist(), want)
+    for db, want in Gd["refine_k1_c1"].items():
+        got = O.pivot_topk(q, k, w, cu, 1, 2, 1, O.REFINE, dense_below=int(db))
+        assert got.tolist() == want, ("refine k1 c1", db, got.tolist(), want)
+    for db, want in Gd["reuse_k2"].items():
+        got = O.pivot_topk(q, k, w, cu, 2, 2, 2, O.REUSE, dense_below=int(db))
+        assert got.tolist() == want, ("reuse k2", db, got.tolist(), want)
+
+
+def pin_guardrail_reductions():
+    """dense_below >= every request length gives dense for every mode and g;
+    dense_below below the first group's prefix gives plain PIVOT; in between,
+    exactly the groups whose prefix fits take the dense rows."""
+    P = W.prefill([37, 20, 5], H=4, d=32, topk=5, rho=0.9, planted=0.1, seed=17)
+    cu = P.cu_seqlens
+    dense = O.dense_topk(P.q, P.k, P.w, cu, 5)
+    for mode, c in ((O.REUSE, 5), (O.REFINE, 8)):
+        for g in (2, 3, 8):
+            plain = O.pivot_topk(P.q, P.k, P.w, cu, 5, g, c, mode)
+            assert np.array_equal(O.pivot_topk(P.q, P.k, P.w, cu, 5, g, c, mode, dense_below=37), dense)
+            assert np.array_equal(O.pivot_topk(P.q, P.k, P.w, cu, 5, g, c, mode, dense_below=0), plain)
+            for db in (1, 9, 16):
+                got = O.pivot_topk(P.q, P.k, P.w, cu, 5, g, c, mode, dense_below=db)
+                for b in range(3):
+                    n = cu[b + 1] - cu[b]
+                    for t in range(n):
+                        t_last = min((t // g + 1) * g, n) - 1
+                        want = dense if t_last + 1 <= db else plain
+                        assert np.array_equal(got[cu[b] + t], want[cu[b] + t]), (mode, g, db, b, t)
+
+
 def pin_hand_decode():
     G, q, k, w = _hand()
     qd = q[2:4][None]          # the decode queries are rows 2 and 3
@@ -484,7 +522,7 @@ def pin_gaussian_mean_score():
     assert abs(tot / pred - 1.0) < 0.05, tot / pred
 
 
-ALL_PINS = [pin_hand_scores, pin_hand_topk, pin_hand_decode, pin_bruteforce_dense,
+ALL_PINS = [pin_hand_scores, pin_hand_topk, pin_hand_guardrail, pin_guardrail_reductions, pin_hand_decode, pin_bruteforce_dense,
             pin_bruteforce_pivot, pin_exact_integer_inputs, pin_textbook_single_head,
             pin_pivot_special_cases, pin_invariants, pin_reuse_within_proxy_ranking,
             pin_proxy_exact_mean, pin_decode_matches_prefill, pin_gaussian_mean_score,
@@ -529,6 +567,12 @@ MUTANTS = {
     "attn_scale_dropped": ("z[j] = J->scale * dot;", "z[j] = dot;"),
     "attn_request_lookup_dropped": ("int b = find_request(J->cu_q, J->S, r);", "int b = 0;"),
     "attn_normaliser_dropped": ("for (int c = 0; c < J->Dv; ++c) o[c] /= l;", ""),
+    "guard_strict_bound": ("if (J->dense_below > 0 && hi <= J->dense_below) {",
+                           "if (J->dense_below > 0 && hi < J->dense_below) {"),
+    "guard_by_first_member": ("if (J->dense_below > 0 && hi <= J->dense_below) {",
+                              "if (J->dense_below > 0 && lo + 1 <= J->dense_below) {"),
+    "guard_by_own_position": ("if (J->dense_below > 0 && hi <= J->dense_below) {",
+                              "if (J->dense_below > 0 && t + 1 <= J->dense_below) {"),
 }
 
 
