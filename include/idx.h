@@ -141,10 +141,10 @@ idx_status idx_adaptive_topk(const void *q, const void *k, const float *w, const
                              idx_dtype dtype, int *out_idx, float *out_score, float *out_sigma,
                              uint8_t *out_trigger, void *ws, size_t ws_bytes, idx_stream_t stream);
 
-/* Workspace bytes for idx_pivot_topk (mode REUSE, REFINE or BLOCK); 0 for
- * arguments idx_pivot_topk would reject. */
+/* Workspace bytes for idx_pivot_topk (mode REUSE, REFINE or BLOCK) with the
+ * same dense_below; 0 for arguments idx_pivot_topk would reject. */
 size_t idx_pivot_workspace_size(int T, int H, int d, int topk, int num_seqs, idx_dtype dtype, int g,
-                                int c, idx_mode mode);
+                                int c, idx_mode mode, int dense_below);
 
 /* PIVOT grouped indexer + top-k (Reuse, Refine or block pre-filter Refine)
  * over a packed batch.  Same tensors and layouts as idx_dense_topk, plus
@@ -152,11 +152,23 @@ size_t idx_pivot_workspace_size(int T, int H, int d, int topk, int num_seqs, idx
  *   c     candidate budget in tokens for REFINE and BLOCK (c >= topk; BLOCK:
  *         a multiple of 64); ignored for REUSE
  *   mode  IDX_MODE_REUSE, IDX_MODE_REFINE or IDX_MODE_BLOCK
- * IDX_ERR_INVALID for g < 1, an unknown mode or a c these rules reject. */
+ *   dense_below  the guardrail (PIVOT page, Results, indexer speed: PIVOT
+ *         falls back to a dense scan for short groups, so that it is never
+ *         slower than the dense indexer; the page gives no threshold).  A
+ *         group whose last member's prefix holds at most dense_below keys
+ *         (t_last + 1 <= dense_below) is not grouped: each member takes its
+ *         dense top-k, exactly as idx_dense_topk would.  Those groups are
+ *         the first min(n, floor(dense_below / g) * g) tokens of a request
+ *         (all n when n <= dense_below); the other groups are unchanged.
+ *         0 turns it off.  REUSE and REFINE only (BLOCK: IDX_ERR_UNSUPPORTED
+ *         for dense_below > 0).  For REFINE a threshold of at most c changes
+ *         no result: such a group's candidate set is its whole prefix.
+ * IDX_ERR_INVALID for g < 1, dense_below < 0, an unknown mode or a c these
+ * rules reject. */
 idx_status idx_pivot_topk(const void *q, const void *k, const float *w, const int *cu_seqlens,
                           int num_seqs, int T, int H, int d, int topk, idx_dtype dtype, int g, int c,
-                          idx_mode mode, int *out_idx, float *out_score, void *ws, size_t ws_bytes,
-                          idx_stream_t stream);
+                          idx_mode mode, int dense_below, int *out_idx, float *out_score, void *ws,
+                          size_t ws_bytes, idx_stream_t stream);
 
 /* ------------------------------------------------------------- decode */
 

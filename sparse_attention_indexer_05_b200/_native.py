@@ -21,8 +21,9 @@ SIGNATURES = {
     "idx_adaptive_workspace_size": (_sz, [_i, _i, _i, _i, _i, _i, _i]),
     "idx_adaptive_topk": (_i, [_vp, _vp, _fp, _ip, _i, _i, _i, _i, _i, _i, ctypes.c_double, _i, _ip, _fp, _fp,
                                _vp, _vp, _sz, _vp]),
-    "idx_pivot_workspace_size": (_sz, [_i, _i, _i, _i, _i, _i, _i, _i, _i]),
-    "idx_pivot_topk": (_i, [_vp, _vp, _fp, _ip, _i, _i, _i, _i, _i, _i, _i, _i, _i, _ip, _fp, _vp, _sz, _vp]),
+    "idx_pivot_workspace_size": (_sz, [_i, _i, _i, _i, _i, _i, _i, _i, _i, _i]),
+    "idx_pivot_topk": (_i, [_vp, _vp, _fp, _ip, _i, _i, _i, _i, _i, _i, _i, _i, _i, _i, _ip, _fp, _vp, _sz,
+                            _vp]),
     "idx_decode_workspace_size": (_sz, [_i, _i, _i, _i, _i, _i, _i, _i, _i]),
     "idx_decode_topk": (_i, [_vp, _vp, _ip, _fp, _i, _i, _i, _i, _i, _i, _i, _i, _i, _ip, _fp, _vp, _sz,
                              _vp]),

@@ -60,10 +60,17 @@ bool refines(idx_mode m) { return m == IDX_MODE_REFINE || m == IDX_MODE_BLOCK; }
 
 long long block_rows(int T) { return (T >> kBlockShift) > 0 ? (T >> kBlockShift) : 1; }
 
-PrefillWs prefill_ws(int T, int H, int d, int topk, int S, idx_dtype dt, int g, int c, idx_mode mode) {
+PrefillWs prefill_ws(int T, int H, int d, int topk, int S, idx_dtype dt, int g, int c, idx_mode mode,
+                     int db = 0) {
     PrefillWs L{};
     const bool pivot = mode != IDX_MODE_DENSE;
     L.R = pivot ? ((long long)T + (long long)S * (g - 1)) / g : T;
+    if (pivot && db > 0 && g > 1) {
+        // members of short groups are scored rows of their own: at most
+        // min(n, db) per request
+        const long long extra = (long long)S * db < T ? (long long)S * db : T;
+        L.R = L.R + extra < T ? L.R + extra : T;
+    }
     L.pl.S = S;
     L.pl.maxblk = (int)((L.R + RB - 1) / RB + S);
     L.pl.maxtiles = (int)(nbound(T) / KT + 1);
@@ -185,6 +192,7 @@ struct Prefill {
     char *ws;
     PrefillWs L;
     cudaStream_t st;
+    int db = 0;  // guardrail threshold (PIVOT modes)
 
     unsigned *status() const { return reinterpret_cast<unsigned *>(ws + L.status); }
     int *plan() const { return reinterpret_cast<int *>(ws + L.plan); }
@@ -199,6 +207,7 @@ struct Prefill {
         a.cu = cu;
         a.S = S; a.T = T; a.H = H; a.d = d;
         a.g = proxies ? g : 1;
+        a.db = proxies ? db : 0;
         a.R = proxies ? L.R : T;
         a.plan = plan();
         a.pl = L.pl;
@@ -222,10 +231,11 @@ struct Prefill {
     cudaError_t prepare() const {
         cudaError_t e = cudaMemsetAsync(status(), 0, 4, st);
         if (e != cudaSuccess) return e;
-        e = launch_plan(cu, S, T, mode == IDX_MODE_DENSE ? 1 : g, plan(), L.pl, status(), st);
+        e = launch_plan(cu, S, T, mode == IDX_MODE_DENSE ? 1 : g, mode == IDX_MODE_DENSE ? 0 : db, plan(), L.pl,
+                        status(), st);
         if (e != cudaSuccess) return e;
         if (mode != IDX_MODE_DENSE)
-            e = launch_proxy(q, w, cu, S, T, H, d, g, (int)dt, plan(), L.pl, ws + L.qbar,
+            e = launch_proxy(q, w, cu, S, T, H, d, g, db, (int)dt, plan(), L.pl, ws + L.qbar,
                              reinterpret_cast<float *>(ws + L.wbar), (int)L.R, st);
         if (e == cudaSuccess && mode == IDX_MODE_BLOCK)
             e = launch_block_means(k, cu, S, T, d, (int)dt, ws + L.kblk, st);
@@ -242,6 +252,7 @@ struct Prefill {
         s.cu = cu;
         s.S = S;
         s.g = mode == IDX_MODE_DENSE ? 1 : g;
+        s.db = mode == IDX_MODE_DENSE ? 0 : db;
         s.plan = plan();
         s.pl = L.pl;
         s.buf = reinterpret_cast<const unsigned long long *>(ws + L.buf);
@@ -264,7 +275,7 @@ struct Prefill {
         a.c = c; a.H = H; a.d = d;
         a.nitems = (int)L.R;
         a.mode = 0;
-        a.cu = cu; a.S = S; a.g = g; a.cu_T = T;
+        a.cu = cu; a.S = S; a.g = g; a.db = db; a.cu_T = T;
         a.plan = plan(); a.pl = L.pl;
         a.out = reinterpret_cast<float *>(ws + L.msc);
         a.ckeys = ws + L.ckeys;
@@ -368,29 +379,33 @@ idx_status idx_adaptive_topk(const void *q, const void *k, const float *w, const
 }
 
 size_t idx_pivot_workspace_size(int T, int H, int d, int topk, int num_seqs, idx_dtype dtype, int g, int c,
-                                idx_mode mode) {
-    if (T < 1 || num_seqs < 1 || topk < 1 || g < 1 || !shape_ok(H, d, dtype)) return 0;
+                                idx_mode mode, int dense_below) {
+    if (T < 1 || num_seqs < 1 || topk < 1 || g < 1 || dense_below < 0 || !shape_ok(H, d, dtype)) return 0;
     if (mode != IDX_MODE_REUSE && mode != IDX_MODE_REFINE && mode != IDX_MODE_BLOCK) return 0;
     if (refines(mode) && c < topk) return 0;
-    if (mode == IDX_MODE_BLOCK && (c < kBlockN || c % kBlockN != 0)) return 0;
-    return prefill_ws(T, H, d, topk, num_seqs, dtype, g, c, mode).total;
+    if (mode == IDX_MODE_BLOCK && (c < kBlockN || c % kBlockN != 0 || dense_below > 0)) return 0;
+    return prefill_ws(T, H, d, topk, num_seqs, dtype, g, c, mode, dense_below).total;
 }
 
 idx_status idx_pivot_topk(const void *q, const void *k, const float *w, const int *cu_seqlens, int num_seqs,
                           int T, int H, int d, int topk, idx_dtype dtype, int g, int c, idx_mode mode,
-                          int *out_idx, float *out_score, void *ws, size_t ws_bytes, idx_stream_t stream) {
-    if (g < 1 || (mode != IDX_MODE_REUSE && mode != IDX_MODE_REFINE && mode != IDX_MODE_BLOCK))
+                          int dense_below, int *out_idx, float *out_score, void *ws, size_t ws_bytes,
+                          idx_stream_t stream) {
+    if (g < 1 || dense_below < 0 || (mode != IDX_MODE_REUSE && mode != IDX_MODE_REFINE && mode != IDX_MODE_BLOCK))
         return IDX_ERR_INVALID;
     if (refines(mode) && c < topk) return IDX_ERR_INVALID;
     if (mode == IDX_MODE_BLOCK && (c < kBlockN || c % kBlockN != 0)) return IDX_ERR_INVALID;
+    if (mode == IDX_MODE_BLOCK && dense_below > 0) return IDX_ERR_UNSUPPORTED;
     if (mode == IDX_MODE_REUSE) c = topk;
-    const size_t need = idx_pivot_workspace_size(T, H, d, topk, num_seqs, dtype, g, c, mode);
+    const size_t need = idx_pivot_workspace_size(T, H, d, topk, num_seqs, dtype, g, c, mode, dense_below);
     idx_status s = check_prefill(q, k, w, cu_seqlens, num_seqs, T, H, d, topk, dtype, out_idx, ws, ws_bytes,
                                  need);
     if (s != IDX_OK) return s;
     TracePhase phase(mode == IDX_MODE_REUSE ? "reuse" : mode == IDX_MODE_REFINE ? "refine" : "block");
     Prefill P{q, k, w, cu_seqlens, num_seqs, T, H, d, topk, dtype, g, c, mode, static_cast<char *>(ws),
-              prefill_ws(T, H, d, topk, num_seqs, dtype, g, c, mode), reinterpret_cast<cudaStream_t>(stream)};
+              prefill_ws(T, H, d, topk, num_seqs, dtype, g, c, mode, dense_below),
+              reinterpret_cast<cudaStream_t>(stream)};
+    P.db = g > 1 ? dense_below : 0;
     TRY_CUDA(P.prepare());
     TRY_CUDA(P.score(P.score_args(true)));
     if (mode == IDX_MODE_REUSE)
@@ -605,7 +620,7 @@ idx_status idx_debug_scores(int stage, const void *q, const void *k, const float
     if (mode == IDX_MODE_BLOCK && (cc < kBlockN || cc % kBlockN != 0)) return IDX_ERR_INVALID;
     const size_t need = mode == IDX_MODE_DENSE
                             ? idx_dense_workspace_size(T, H, d, topk, num_seqs, dtype)
-                            : idx_pivot_workspace_size(T, H, d, topk, num_seqs, dtype, gg, cc, mode);
+                            : idx_pivot_workspace_size(T, H, d, topk, num_seqs, dtype, gg, cc, mode, 0);
     int dummy = 0;
     idx_status s = check_prefill(q, k, w, cu_seqlens, num_seqs, T, H, d, topk, dtype, &dummy, ws, ws_bytes, need);
     if (s != IDX_OK) return s;

@@ -43,6 +43,7 @@ struct ScoreArgs {
     const float *w;      // [R, H]
     const int *cu;       // cu_seqlens [S+1] (device)
     int S, T, H, d, g;   // g = 1: row i of request b is query i; g > 1: proxy i
+    int db;              // guardrail: short groups scored member by member (plan.cuh)
     long long R;         // rows allocated in q / w
     // kshift > 0: keys are the complete 2^kshift-token blocks of each request,
     // block i of request b at key row (cu[b] >> kshift) + i; a row whose token
@@ -92,7 +93,7 @@ struct GatherArgs {
     // mapping of a work item -> (first member row, members, candidate row, key base)
     int mode;            // 0: prefill (cu, g, plan rp of proxies), 1: decode (B, G, n_max)
     const int *cu;
-    int S, g;
+    int S, g, db;
     int cu_T;            // prefill: rows of q and k (total tokens)
     const int *plan;
     PlanLayout pl;
@@ -142,7 +143,7 @@ struct SelectArgs {
     float *out_score;        // [nrows, k] or NULL
     // prefill context
     const int *cu;
-    int S, g;
+    int S, g, db;
     const int *plan;
     PlanLayout pl;
     const unsigned long long *buf;
@@ -195,7 +196,7 @@ struct TraceScope {
 };
 
 // ---- launchers (each returns cudaSuccess or the launch error)
-cudaError_t launch_plan(const int *cu, int S, int T, int g, int *plan, const PlanLayout &pl,
+cudaError_t launch_plan(const int *cu, int S, int T, int g, int db, int *plan, const PlanLayout &pl,
                         unsigned *status, cudaStream_t st);
 cudaError_t launch_score_simt(const ScoreArgs &a, int dtype, cudaStream_t st);
 cudaError_t launch_score_tc(const ScoreArgs &a, cudaStream_t st);
@@ -206,7 +207,7 @@ cudaError_t launch_gather_tc(const GatherArgs &a, cudaStream_t st);
 cudaError_t launch_select(const SelectArgs &a, cudaStream_t st);
 cudaError_t launch_adaptive(const AdaptiveArgs &a, cudaStream_t st);
 cudaError_t launch_proxy(const void *q, const float *w, const int *cu, int S, int T, int H, int d,
-                         int g, int dtype, const int *plan, const PlanLayout &pl, void *qbar,
+                         int g, int db, int dtype, const int *plan, const PlanLayout &pl, void *qbar,
                          float *wbar, int max_proxies, cudaStream_t st);
 // token-sparse attention over selected positions (absorbed-MLA shapes)
 struct SparseAttnArgs {

@@ -36,8 +36,8 @@ __device__ int block_incl_scan(int v, int *warp_tot, int *total) {
     return v;
 }
 
-__global__ void __launch_bounds__(kPlanThreads) plan_kernel(const int *cu, int S, int T, int g, int *plan,
-                                                            PlanLayout pl, unsigned *status) {
+__global__ void __launch_bounds__(kPlanThreads) plan_kernel(const int *cu, int S, int T, int g, int db,
+                                                            int *plan, PlanLayout pl, unsigned *status) {
     __shared__ int s_bad;
     __shared__ int warp_tot[32];
     __shared__ int warp_tot2[32];
@@ -61,7 +61,7 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const int *cu, int S
     int carry_r = 0, carry_b = 0;
     for (int base = 0; base < S; base += kPlanThreads) {
         const int b = base + tid;
-        const int r = b < S ? rows_of(cu[b + 1] - cu[b], g) : 0;
+        const int r = b < S ? rows_of(cu[b + 1] - cu[b], g, db) : 0;
         const int nb = (r + RB - 1) / RB;
         int tot_r, tot_b;
         const int ir = block_incl_scan(r, warp_tot, &tot_r);
@@ -85,7 +85,7 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const int *cu, int S
     for (int i = tid; i <= pl.maxtiles; i += kPlanThreads) hist[i] = 0;
     __syncthreads();
     for (int blk = tid; blk < nblocks; blk += kPlanThreads) {
-        const BlockInfo bi = block_info(plan, pl, cu, g, blk);
+        const BlockInfo bi = block_info(plan, pl, cu, g, blk, 0, db);
         const int t = bi.ntiles < pl.maxtiles ? bi.ntiles : pl.maxtiles;
         atomicAdd(&hist[t], 1);
     }
@@ -102,7 +102,7 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const int *cu, int S
     __syncthreads();
     int *order = plan + pl.order();
     for (int blk = tid; blk < nblocks; blk += kPlanThreads) {
-        const BlockInfo bi = block_info(plan, pl, cu, g, blk);
+        const BlockInfo bi = block_info(plan, pl, cu, g, blk, 0, db);
         const int t = bi.ntiles < pl.maxtiles ? bi.ntiles : pl.maxtiles;
         order[atomicAdd(&hist[t], 1)] = blk;
     }
@@ -111,10 +111,10 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const int *cu, int S
 
 }  // namespace
 
-cudaError_t launch_plan(const int *cu, int S, int T, int g, int *plan, const PlanLayout &pl,
+cudaError_t launch_plan(const int *cu, int S, int T, int g, int db, int *plan, const PlanLayout &pl,
                         unsigned *status, cudaStream_t st) {
     TraceScope ts("plan", st);
-    plan_kernel<<<1, kPlanThreads, 0, st>>>(cu, S, T, g, plan, pl, status);
+    plan_kernel<<<1, kPlanThreads, 0, st>>>(cu, S, T, g, db, plan, pl, status);
     return cudaGetLastError();
 }
 

@@ -16,15 +16,50 @@ __device__ __forceinline__ int find_seg(const int *a, int n, long long v) {
     return lo;
 }
 
+// Grouping of a request of n tokens into scored rows.  Groups are the
+// request-local [m*g, min((m+1)*g, n)).  Under the guardrail (db > 0, the
+// PIVOT page's dense fallback for short groups) every group whose last
+// member's prefix holds at most db keys is not grouped: each of its members
+// is a scored row of its own.  Those groups form a prefix of the request,
+// its first dense_rows() tokens; the groups after it are unchanged, so
+// scored row i is member i for i < nd and proxy i - nd of the rest.
+__device__ __forceinline__ int dense_rows(int n, int g, int db) {
+    if (db <= 0 || g == 1) return 0;
+    return n <= db ? n : (db / g) * g;
+}
+
 // Number of scored rows of a request of n tokens: queries (g = 1) or proxies.
-__device__ __forceinline__ int rows_of(int n, int g) { return g == 1 ? n : (n + g - 1) / g; }
+__device__ __forceinline__ int rows_of(int n, int g, int db = 0) {
+    if (g == 1) return n;
+    const int nd = dense_rows(n, g, db);
+    return nd + (n - nd + g - 1) / g;
+}
+
+// First member (request-local) and member count of scored row i.
+__device__ __forceinline__ int group_start(int i, int n, int g, int db = 0) {
+    const int nd = dense_rows(n, g, db);
+    return i < nd ? i : nd + (i - nd) * g;
+}
+__device__ __forceinline__ int group_size(int i, int n, int g, int db = 0) {
+    const int nd = dense_rows(n, g, db);
+    if (i < nd) return 1;
+    const int lo = nd + (i - nd) * g;
+    return (lo + g < n ? lo + g : n) - lo;
+}
+
+// Scored row that holds member t.
+__device__ __forceinline__ int group_of(int t, int n, int g, int db = 0) {
+    const int nd = dense_rows(n, g, db);
+    return t < nd ? t : nd + (t - nd) / g;
+}
 
 // Causal bound (request-local, inclusive) of scored row i of a request of n
-// tokens: a query sees s <= i; proxy i (group [i*g, min((i+1)*g, n)))
-// sees the prefix of its last member.
-__device__ __forceinline__ int row_bound(int i, int n, int g) {
+// tokens: a query sees s <= i; a proxy sees the prefix of its last member.
+__device__ __forceinline__ int row_bound(int i, int n, int g, int db = 0) {
     if (g == 1) return i;
-    long long e = (long long)(i + 1) * g;
+    const int nd = dense_rows(n, g, db);
+    if (i < nd) return i;
+    const long long e = nd + (long long)(i - nd + 1) * g;
     return (int)((e < n ? e : n) - 1);
 }
 
@@ -45,21 +80,21 @@ struct BlockInfo {
 __device__ __forceinline__ int key_bound(int t, int kshift) { return ((t + 1) >> kshift) - 1; }
 
 __device__ __forceinline__ BlockInfo block_info(const int *plan, const PlanLayout &pl, const int *cu,
-                                                int g, int blk, int kshift = 0) {
+                                                int g, int blk, int kshift = 0, int db = 0) {
     BlockInfo bi;
     const int *rp = plan + pl.rp();
     const int *bp = plan + pl.bp();
     bi.b = find_seg(bp, pl.S, blk);
     const int j = blk - bp[bi.b];
     bi.n = cu[bi.b + 1] - cu[bi.b];
-    const int R = rows_of(bi.n, g);
+    const int R = rows_of(bi.n, g, db);
     bi.i0 = j * RB;
     bi.row0 = rp[bi.b] + bi.i0;
     int e = bi.i0 + RB;
     if (e > R) e = R;
     bi.nrows = e - bi.i0;
     bi.key0 = kshift ? (long long)(cu[bi.b] >> kshift) : (long long)cu[bi.b];
-    bi.maxbound = key_bound(row_bound(e - 1, bi.n, g), kshift);
+    bi.maxbound = key_bound(row_bound(e - 1, bi.n, g, db), kshift);
     bi.ntiles = bi.maxbound < 0 ? 1 : bi.maxbound / KT + 1;
     return bi;
 }

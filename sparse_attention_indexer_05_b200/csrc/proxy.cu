@@ -78,7 +78,7 @@ __device__ void mean_rows(const T *src, const float *wsrc, int cnt, int HD, int 
 
 template <typename T>
 __global__ void __launch_bounds__(kProxyThreads) proxy_kernel(const T *q, const float *w, const int *cu, int S,
-                                                              int H, int d, int g, const int *plan,
+                                                              int H, int d, int g, int db, const int *plan,
                                                               PlanLayout pl, T *qbar, float *wbar) {
     const int p = blockIdx.x;
     if (!plan[0] || p >= plan[2]) return;
@@ -86,8 +86,10 @@ __global__ void __launch_bounds__(kProxyThreads) proxy_kernel(const T *q, const 
     const int b = find_seg(rp, S, p);
     const int i = p - rp[b];
     const int n = cu[b + 1] - cu[b];
-    const int lo = i * g;
-    const int cnt = (lo + g < n ? lo + g : n) - lo;
+    // a member scored on its own (guardrail) is a group of one: its mean is
+    // the member itself, bit for bit
+    const int lo = group_start(i, n, g, db);
+    const int cnt = group_size(i, n, g, db);
     const int HD = H * d;
     const long long m0 = (long long)cu[b] + lo;
     mean_rows(q + m0 * HD, w + m0 * H, cnt, HD, H, qbar + (long long)p * HD, wbar + (long long)p * H);
@@ -207,17 +209,17 @@ cudaError_t launch_block_expand(const int *cu, int S, int g, const int *plan, co
 }
 
 cudaError_t launch_proxy(const void *q, const float *w, const int *cu, int S, int T, int H, int d, int g,
-                         int dtype, const int *plan, const PlanLayout &pl, void *qbar, float *wbar,
+                         int db, int dtype, const int *plan, const PlanLayout &pl, void *qbar, float *wbar,
                          int max_proxies, cudaStream_t st) {
     (void)T;
     if (max_proxies <= 0) return cudaSuccess;
     TraceScope ts("proxy", st);
     if (dtype == 1)
         proxy_kernel<float><<<max_proxies, kProxyThreads, 0, st>>>(
-            (const float *)q, w, cu, S, H, d, g, plan, pl, (float *)qbar, wbar);
+            (const float *)q, w, cu, S, H, d, g, db, plan, pl, (float *)qbar, wbar);
     else
         proxy_kernel<__nv_bfloat16><<<max_proxies, kProxyThreads, 0, st>>>(
-            (const __nv_bfloat16 *)q, w, cu, S, H, d, g, plan, pl, (__nv_bfloat16 *)qbar, wbar);
+            (const __nv_bfloat16 *)q, w, cu, S, H, d, g, db, plan, pl, (__nv_bfloat16 *)qbar, wbar);
     return cudaGetLastError();
 }
 

@@ -170,7 +170,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         __syncthreads();
         const int item = sh.item;
         if (item >= nblocks) break;
-        const BlockInfo bi = block_info(plan, a.pl, a.cu, a.g, plan[a.pl.order() + item], a.kshift);
+        const BlockInfo bi = block_info(plan, a.pl, a.cu, a.g, plan[a.pl.order() + item], a.kshift, a.db);
         const int ntiles = bi.ntiles;
 
         if (warp >= 2) {
@@ -180,7 +180,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 wsm[i] = (i / TC_H) < bi.nrows ? 0.5f * a.w[(long long)bi.row0 * TC_H + i] : 0.0f;
             if (e < RB) {
                 if (lane == 0) {
-                    sh.bound[e] = e < bi.nrows ? key_bound(row_bound(bi.i0 + e, bi.n, a.g), a.kshift) : -1;
+                    sh.bound[e] = e < bi.nrows ? key_bound(row_bound(bi.i0 + e, bi.n, a.g, a.db), a.kshift) : -1;
                     sh.slot[e] = -1;
                     if (a.sink == SINK_SPILL && e < bi.nrows && a.slot_of_row)
                         sh.slot[e] = a.slot_of_row[bi.row0 + e];

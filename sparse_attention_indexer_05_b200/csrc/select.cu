@@ -1,9 +1,17 @@
 // select.cu -- exact final top-k of one row per CTA.
 //
-// The entries of a row (candidate keys from a score pass, or dense fp32
-// scores) are ranked by key = (ord(score) << 32) | (0xFFFFFFFF - s), so the
-// top-k is "highest score first, ties to the lower position".
+// The entries of a row (candidate keys from a score pass, or fp32 scores)
+// are ranked by key = (ord(score) << 32) | (0xFFFFFFFF - s), so the top-k is
+// "highest score first, ties to the lower position".
 //
+// Two kernels:
+//  - select_kernel: decode score rows (a full fp32 score row per query or
+//    proxy over its whole cache, up to 2^20 entries, few rows), below;
+//  - select_fast_kernel: candidate buffers with a floor (dense, Reuse,
+//    proxy -> C, proxy -> blocks) and Refine member rows over a candidate
+//    set, further down.
+//
+// select_kernel:
 // 1. One pass over the row in global memory counts the valid entries and
 //    builds a histogram of the key's top 12 bits (1/16-octave score bins);
 //    the bin D holding the k-th largest key follows.
@@ -30,24 +38,8 @@ namespace {
 constexpr int kSelThreads = 512;
 constexpr int kMaxBins = 4096;  // widest radix digit: 12 bits
 
-// candidate keys of a score pass; entries below the row's floor (a score
-// that at least ksel appended keys reach) can no longer be selected
-struct CandSrc {
-    static constexpr bool kFloor = true;  // valid entries are few: stage them directly
-    static constexpr bool kShared = false;
-    const unsigned long long *buf;
-    int n;
-    int bound;
-    unsigned floor_ord;
-    __device__ unsigned long long key(int i) const {
-        const unsigned long long kk = buf[i];
-        return (key_pos(kk) <= bound && key_ord(kk) >= floor_ord) ? kk : 0ull;
-    }
-};
-
 // dense fp32 scores with their positions (NULL: position = index)
 struct ScoreSrc {
-    static constexpr bool kFloor = false;
     static constexpr bool kShared = false;
     const float *sc;
     const int *pos;
@@ -62,7 +54,6 @@ struct ScoreSrc {
 
 // keys staged in shared memory (all valid)
 struct StageSrc {
-    static constexpr bool kFloor = false;
     static constexpr bool kShared = true;  // cheap to read: no unrolled prefetch needed
     const unsigned long long *st;
     int n;
@@ -323,9 +314,8 @@ __device__ void block_select(const Src &src, int k, int *out_idx, float *out_sco
                              unsigned long long *stage, int stage_cap, unsigned *bm, unsigned *gpre, int wcap,
                              unsigned *status) {
     const int tid = threadIdx.x, nt = blockDim.x, lane = tid & 31;
-    if (Src::kFloor || src.n <= stage_cap) {
-        // candidate rows (the entries at or above the row's floor are about
-        // k plus a bin's worth) and short rows: one pass stages them all
+    if (src.n <= stage_cap) {
+        // short rows: one pass stages them all
         const unsigned ns = stage_keys(src, sh, 1ull, stage, stage_cap);
         if (ns <= (unsigned)stage_cap) {
             const StageSrc ss{stage, (int)ns, src.bound};
@@ -389,58 +379,10 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(SelectArgs a) {
             if (os) os[r] = -INFINITY;
         }
     };
-    auto cand = [&](long long r, int bound) {
-        const unsigned n = a.cnt[r];
-        return CandSrc{a.buf + r * a.cap, (int)(n < a.cap ? n : a.cap), bound, a.floor ? a.floor[r] : 0u};
-    };
     switch (a.kind) {
-    case SEL_DENSE_CAND:
-    case SEL_REUSE_CAND:
-    case SEL_MEMBER_SCORES: {
-        if (!a.plan[0]) { pad_all(); return; }
-        const int b = find_seg(a.cu, a.S, row);
-        const int t = row - a.cu[b];
-        if (a.kind == SEL_DENSE_CAND) {
-            block_select(cand(row, t), a.k, oi, os, sh, stage, a.stage_cap, bm, gpre, wcap, a.status);
-        } else {
-            const int p = a.plan[a.pl.rp() + b] + t / a.g;
-            if (a.kind == SEL_REUSE_CAND) {
-                block_select(cand(p, t), a.k, oi, os, sh, stage, a.stage_cap, bm, gpre, wcap, a.status);
-            } else {
-                ScoreSrc src{a.scores + (long long)row * a.ld, a.cand + (long long)p * a.c, a.c, t};
-                block_select(src, a.k, oi, os, sh, stage, a.stage_cap, bm, gpre, wcap, a.status);
-            }
-        }
-        return;
-    }
-    case SEL_PROXY_TO_C: {
-        if (!a.plan[0]) { pad_all(); return; }
-        if (row >= a.plan[2]) return;
-        const int *rp = a.plan + a.pl.rp();
-        const int b = find_seg(rp, a.S, row);
-        const int i = row - rp[b];
-        const int n = a.cu[b + 1] - a.cu[b];
-        block_select(cand(row, row_bound(i, n, a.g)), a.k, oi, nullptr, sh, stage, a.stage_cap, bm, gpre, wcap,
-                     a.status);
-        return;
-    }
-    case SEL_PROXY_TO_BLOCKS: {
-        if (!a.plan[0]) { pad_all(); return; }
-        if (row >= a.plan[2]) return;
-        const int *rp = a.plan + a.pl.rp();
-        const int b = find_seg(rp, a.S, row);
-        const int i = row - rp[b];
-        const int n = a.cu[b + 1] - a.cu[b];
-        const int tl = row_bound(i, n, a.g);
-        // the partial block holding the last member takes one slot of the budget
-        const int kr = a.k - (((tl + 1) & (kBlockN - 1)) ? 1 : 0);
-        if (kr > 0)
-            block_select(cand(row, key_bound(tl, kBlockShift)), kr, oi, nullptr, sh, stage, a.stage_cap, bm, gpre,
-                         wcap, a.status);
-        for (int r = (kr > 0 ? kr : 0) + (int)threadIdx.x; r < a.k; r += blockDim.x) oi[r] = -1;
-        return;
-    }
-    default: {  // decode kinds
+    case SEL_DEC_DENSE:
+    case SEL_DEC_REUSE:
+    case SEL_DEC_PROXY_TO_C: {
         const bool per_member = a.kind != SEL_DEC_PROXY_TO_C;
         const int b = per_member ? row / a.G : row;
         const int m = per_member ? row % a.G : 0;
@@ -458,23 +400,525 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(SelectArgs a) {
             const int bound = kv - a.G + m;
             ScoreSrc src{a.scores + (long long)b * a.ld, nullptr, bound + 1, bound};
             block_select(src, a.k, oi, os, sh, stage, a.stage_cap, bm, gpre, wcap, a.status);
-        } else if (a.kind == SEL_DEC_PROXY_TO_C) {
+        } else {  // SEL_DEC_PROXY_TO_C
             ScoreSrc src{a.scores + (long long)b * a.ld, nullptr, kv, kv - 1};
             block_select(src, a.k, oi, nullptr, sh, stage, a.stage_cap, bm, gpre, wcap, a.status);
-        } else {  // SEL_DEC_MEMBER
-            const int bound = kv - a.G + m;
-            ScoreSrc src{a.scores + (long long)row * a.ld, a.cand + (long long)b * a.c, a.c, bound};
-            block_select(src, a.k, oi, os, sh, stage, a.stage_cap, bm, gpre, wcap, a.status);
         }
         return;
     }
+    default:  // the other kinds run in select_fast_kernel
+        return;
     }
+}
+
+// ===================================================================
+// select_fast_kernel: the final top-k of rows whose entries are few or
+// filtered -- candidate buffers with a floor (dense, Reuse, proxy -> C,
+// proxy -> blocks) and Refine member score rows over a candidate set.
+//
+// One CTA of 256 threads per row, several CTAs per SM (the row's work is a
+// chain of short, barrier-separated steps, so rows in flight hide each
+// other's latency):
+// 1. one global pass stages every valid entry at or above the row's floor
+//    into shared memory (16-byte loads, one reservation per warp and round);
+//    member rows stage entry i at slot i, which keeps their order;
+// 2. an MSB-first radix select with 8-bit digits over the staged keys finds
+//    the exact k-th largest key K, starting right below the leading bits all
+//    staged scores share (they lie between the floor and the largest staged
+//    score), two barriers per digit (double-buffered histograms);
+// 3. the selected entries (key >= K) are listed in ascending position:
+//    member rows by an ordered compaction of the stage (their candidate
+//    positions ascend), candidate rows by a bitmap over the prefix, in
+//    chunks of 131072 positions (16 KB), walked word by word.
+// A row whose floor admits more entries than the stage holds takes the same
+// steps reading its entries from global memory instead.
+// ===================================================================
+constexpr int kFT = 256;                          // threads of select_fast_kernel
+constexpr int kFWarps = kFT / 32;
+constexpr int kChunkBits = 1 << 17;               // positions per bitmap chunk
+constexpr int kChunkWords = kChunkBits / 32;      // 4096 words = 16 KB
+constexpr int kWordsPer = kChunkWords / kFT;      // 16 words per thread
+
+struct __align__(16) FastShared {
+    unsigned hist[2][256];
+    unsigned wtot[kFWarps];
+    unsigned tpre[kFT];
+    unsigned nstage;
+    unsigned maxord;
+    unsigned minord;
+    int dgt;
+    unsigned above;
+    unsigned inbin;
+};
+
+// Block-wide exclusive prefix of one value per thread; *total = the sum.
+__device__ __forceinline__ unsigned fast_excl_scan(unsigned v, unsigned *wtot, unsigned *total) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    unsigned inc = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const unsigned u = __shfl_up_sync(0xFFFFFFFFu, inc, o);
+        if (lane >= o) inc += u;
+    }
+    if (lane == 31) wtot[warp] = inc;
+    __syncthreads();
+    unsigned before = 0, all = 0;
+#pragma unroll
+    for (int w = 0; w < kFWarps; ++w) {
+        const unsigned t = wtot[w];
+        before += w < warp ? t : 0u;
+        all += t;
+    }
+    __syncthreads();  // wtot may be reused right after
+    *total = all;
+    return before + inc - v;
+}
+
+// Source: candidate keys in global memory, filtered by floor and bound.
+struct GCand {
+    const unsigned long long *buf;
+    int n;
+    unsigned long long lo;  // keys below lo (ord < floor) are out
+    unsigned pmin;          // low word >= pmin <=> position <= bound
+    __device__ __forceinline__ unsigned long long key(int i) const {
+        const unsigned long long kk = buf[i];
+        return (kk >= lo && (unsigned)kk >= pmin) ? kk : 0ull;
+    }
+};
+// Source: score row over a list of positions (NULL: position = index).
+struct GScore {
+    const float *sc;
+    const int *pos;
+    int n;
+    int bound;
+    __device__ __forceinline__ unsigned long long key(int i) const {
+        const int p = pos ? pos[i] : i;
+        if (p < 0 || p > bound) return 0ull;
+        return make_key(score_ord(sc[i]), p);
+    }
+};
+// Source: keys staged in shared memory (0 = empty slot).
+struct SStage {
+    const unsigned long long *st;
+    int n;
+    __device__ __forceinline__ unsigned long long key(int i) const { return st[i]; }
+};
+
+// Exact k-th largest nonzero key of src (more than `need` nonzero keys,
+// all with ords in [lo_ord, hi_ord]).  MSB-first radix with 8-bit digits
+// from the first bit where lo_ord and hi_ord differ; sh.hist[0] is clear
+// on entry (and sh.hist[1] is cleared here).
+template <class Src>
+__device__ unsigned long long fast_kth(const Src &src, FastShared &sh, unsigned need, unsigned lo_ord,
+                                       unsigned hi_ord) {
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const unsigned diff = lo_ord ^ hi_ord;
+    const int lead = diff ? __clz(diff) : 32;  // leading ord bits every key shares
+    int shift = 64 - lead;
+    unsigned long long mask = lead ? (~0ull << (64 - lead)) : 0ull;
+    unsigned long long prefix = ((unsigned long long)hi_ord << 32) & mask;
+    int p = 0;
+    while (shift > 0) {
+        const int bits = shift >= 8 ? 8 : shift;
+        shift -= bits;
+        const unsigned dmask = (1u << bits) - 1u;
+        unsigned *h = sh.hist[p & 1];
+        sh.hist[(p + 1) & 1][tid] = 0u;  // the next digit's histogram
+        for (int i = tid; i < src.n; i += kFT) {
+            const unsigned long long kk = src.key(i);
+            if (kk != 0ull && (kk & mask) == prefix) atomicAdd(&h[(unsigned)(kk >> shift) & dmask], 1u);
+        }
+        __syncthreads();
+        if (warp == 0) {
+            unsigned above;
+            const int b = warp_find_bin(h, need, &above);
+            if (lane == 0) {
+                sh.dgt = b;
+                sh.above = above;
+                sh.inbin = b >= 0 ? h[b] : 0u;
+            }
+        }
+        __syncthreads();
+        const int d = sh.dgt;
+        const unsigned above = sh.above, inbin = sh.inbin;
+        ++p;
+        if (d < 0) break;  // unreachable: more than `need` keys match the prefix
+        need -= above;
+        prefix |= (unsigned long long)d << shift;
+        mask |= (unsigned long long)dmask << shift;
+        if (inbin == need) break;  // the whole bin is selected
+    }
+    // leave hist[0] clear for the next user
+    sh.hist[0][tid] = 0u;
+    __syncthreads();
+    return prefix;
+}
+
+// List the nonzero keys >= K of src in ascending position through a bitmap
+// (chunks of kChunkBits positions over 0..bound); returns how many.
+template <class Src>
+__device__ int fast_emit_bitmap(const Src &src, unsigned long long K, int bound, int *out_idx, float *out_score,
+                                FastShared &sh, unsigned *bm) {
+    const int tid = threadIdx.x;
+    int base = 0;
+    for (int c0 = 0; c0 <= bound; c0 += kChunkBits) {
+        const int nwords = (bound - c0) / 32 + 1 < kChunkWords ? (bound - c0) / 32 + 1 : kChunkWords;
+#pragma unroll
+        for (int j = 0; j < kWordsPer; ++j) bm[tid * kWordsPer + j] = 0u;
+        __syncthreads();
+        for (int i = tid; i < src.n; i += kFT) {
+            const unsigned long long kk = src.key(i);
+            if (kk != 0ull && kk >= K) {
+                const int p = key_pos(kk) - c0;
+                if (p >= 0 && p < kChunkBits) atomicOr(&bm[p >> 5], 1u << (p & 31));
+            }
+        }
+        __syncthreads();
+        // thread tid owns words [tid * kWordsPer, +kWordsPer)
+        const int w0 = tid * kWordsPer;
+        unsigned words[kWordsPer];
+        unsigned cnt = 0;
+        const uint4 *b4 = reinterpret_cast<const uint4 *>(bm + w0);
+#pragma unroll
+        for (int j = 0; j < kWordsPer / 4; ++j) {
+            const uint4 v = b4[j];
+            words[4 * j + 0] = v.x;
+            words[4 * j + 1] = v.y;
+            words[4 * j + 2] = v.z;
+            words[4 * j + 3] = v.w;
+        }
+#pragma unroll
+        for (int j = 0; j < kWordsPer; ++j) cnt += __popc(words[j]);
+        unsigned total;
+        const unsigned pre = fast_excl_scan(cnt, sh.wtot, &total);
+        sh.tpre[tid] = pre;
+        unsigned r = base + pre;
+#pragma unroll
+        for (int j = 0; j < kWordsPer; ++j) {
+            unsigned x = words[j];
+            while (x) {
+                const int bit = __ffs(x) - 1;
+                x &= x - 1u;
+                out_idx[r++] = c0 + (w0 + j) * 32 + bit;
+            }
+        }
+        if (out_score) {
+            __syncthreads();  // tpre complete
+            for (int i = tid; i < src.n; i += kFT) {
+                const unsigned long long kk = src.key(i);
+                if (kk != 0ull && kk >= K) {
+                    const int p = key_pos(kk) - c0;
+                    if (p >= 0 && p < kChunkBits) {
+                        const int w = p >> 5, owner = w / kWordsPer;
+                        unsigned rk = sh.tpre[owner] + __popc(bm[w] & ((1u << (p & 31)) - 1u));
+                        for (int x = owner * kWordsPer; x < w; ++x) rk += __popc(bm[x]);
+                        out_score[base + rk] = ord_score(key_ord(kk));
+                    }
+                }
+            }
+        }
+        (void)nwords;
+        base += (int)total;
+        __syncthreads();  // the bitmap is cleared again by the next chunk
+    }
+    return base;
+}
+
+// Member rows: the staged entries are in candidate order (ascending
+// position); list the nonzero keys >= K in that order.
+__device__ int fast_emit_ordered(const unsigned long long *st, int n, unsigned long long K, int *out_idx,
+                                 float *out_score, FastShared &sh) {
+    const int tid = threadIdx.x;
+    const int per = (n + kFT - 1) / kFT;
+    const int i0 = tid * per, i1 = i0 + per < n ? i0 + per : n;
+    unsigned cnt = 0;
+    for (int i = i0; i < i1; ++i) {
+        const unsigned long long kk = st[i];
+        cnt += (kk != 0ull && kk >= K) ? 1u : 0u;
+    }
+    unsigned total;
+    unsigned r = fast_excl_scan(cnt, sh.wtot, &total);
+    for (int i = i0; i < i1; ++i) {
+        const unsigned long long kk = st[i];
+        if (kk != 0ull && kk >= K) {
+            out_idx[r] = key_pos(kk);
+            if (out_score) out_score[r] = ord_score(key_ord(kk));
+            ++r;
+        }
+    }
+    return (int)total;
+}
+
+__device__ __forceinline__ void fast_pad(int nsel, int k, int *out_idx, float *out_score) {
+    for (int r = nsel + (int)threadIdx.x; r < k; r += kFT) {
+        out_idx[r] = -1;
+        if (out_score) out_score[r] = -INFINITY;
+    }
+}
+
+__device__ __forceinline__ unsigned warp_max_u(unsigned v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        const unsigned u = __shfl_xor_sync(0xFFFFFFFFu, v, o);
+        v = u > v ? u : v;
+    }
+    return v;
+}
+__device__ __forceinline__ unsigned warp_min_u(unsigned v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        const unsigned u = __shfl_xor_sync(0xFFFFFFFFu, v, o);
+        v = u < v ? u : v;
+    }
+    return v;
+}
+
+// Top-k of a candidate row (keys at or above `floor_ord`, positions <= bound).
+__device__ void fast_cand_row(const unsigned long long *buf, int n, unsigned floor_ord, int bound, int k,
+                              int *out_idx, float *out_score, FastShared &sh, unsigned long long *stage,
+                              int stage_cap, unsigned *bm) {
+    const int tid = threadIdx.x, lane = tid & 31;
+    const GCand g{buf, n, (unsigned long long)floor_ord << 32, 0xFFFFFFFFu - (unsigned)bound};
+    if (tid == 0) {
+        sh.nstage = 0u;
+        sh.maxord = 0u;
+    }
+    sh.hist[0][tid] = 0u;
+    __syncthreads();
+    unsigned mx = 0u;
+    // 8 keys per thread and round, as four 16-byte loads (rows start 2 KB aligned)
+    const ulonglong2 *b2 = reinterpret_cast<const ulonglong2 *>(buf);
+    for (int base = 0; base < n; base += kFT * 8) {
+        unsigned long long kv[8];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int i = base + u * (kFT * 2) + tid * 2;
+            ulonglong2 v = make_ulonglong2(0ull, 0ull);
+            if (i < n) v = b2[i >> 1];
+            kv[2 * u] = v.x;
+            kv[2 * u + 1] = (i + 1 < n) ? v.y : 0ull;
+        }
+        unsigned cnt = 0;
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            const bool ok = kv[u] >= g.lo && (unsigned)kv[u] >= g.pmin && kv[u] != 0ull;
+            if (!ok) kv[u] = 0ull;
+            cnt += ok ? 1u : 0u;
+            const unsigned o = key_ord(kv[u]);
+            mx = ok && o > mx ? o : mx;
+        }
+        unsigned inc = cnt;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const unsigned v = __shfl_up_sync(0xFFFFFFFFu, inc, o);
+            if (lane >= o) inc += v;
+        }
+        const unsigned wt = __shfl_sync(0xFFFFFFFFu, inc, 31);
+        if (wt) {
+            unsigned b = 0;
+            if (lane == 31) b = atomicAdd(&sh.nstage, wt);
+            b = __shfl_sync(0xFFFFFFFFu, b, 31) + inc - cnt;
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                if (kv[u] != 0ull) {
+                    if (b < (unsigned)stage_cap) stage[b] = kv[u];
+                    ++b;
+                }
+            }
+        }
+    }
+    mx = warp_max_u(mx);
+    if (lane == 0 && mx) atomicMax(&sh.maxord, mx);
+    __syncthreads();
+    const int ns = (int)sh.nstage;
+    const unsigned hi = sh.maxord;
+    int nsel;
+    if (ns <= k) {
+        const SStage s{stage, ns};
+        nsel = fast_emit_bitmap(s, 1ull, bound, out_idx, out_score, sh, bm);
+    } else if (ns <= stage_cap) {
+        const SStage s{stage, ns};
+        const unsigned long long K = fast_kth(s, sh, (unsigned)k, floor_ord, hi);
+        nsel = fast_emit_bitmap(s, K, bound, out_idx, out_score, sh, bm);
+    } else {
+        // more entries at or above the floor than the stage holds: the same
+        // steps over the row in global memory
+        const unsigned long long K = fast_kth(g, sh, (unsigned)k, floor_ord, hi);
+        nsel = fast_emit_bitmap(g, K, bound, out_idx, out_score, sh, bm);
+    }
+    fast_pad(nsel, k, out_idx, out_score);
+}
+
+// Top-k of a member score row over its candidate list (positions ascending,
+// -1 = none), masked to positions <= bound.
+__device__ void fast_member_row(const float *sc, const int *pos, int n, int bound, int k, int *out_idx,
+                                float *out_score, FastShared &sh, unsigned long long *stage, int stage_cap,
+                                unsigned *bm) {
+    const int tid = threadIdx.x, lane = tid & 31;
+    const GScore g{sc, pos, n, bound};
+    if (tid == 0) {
+        sh.nstage = 0u;
+        sh.maxord = 0u;
+        sh.minord = 0xFFFFFFFFu;
+    }
+    sh.hist[0][tid] = 0u;
+    __syncthreads();
+    unsigned mx = 0u, mn = 0xFFFFFFFFu, cnt = 0;
+    const bool staged = n <= stage_cap;
+    for (int i = tid; i < n; i += kFT) {
+        const unsigned long long kk = g.key(i);
+        if (staged) stage[i] = kk;
+        if (kk != 0ull) {
+            const unsigned o = key_ord(kk);
+            mx = o > mx ? o : mx;
+            mn = o < mn ? o : mn;
+            ++cnt;
+        }
+    }
+    mx = warp_max_u(mx);
+    mn = warp_min_u(mn);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) cnt += __shfl_xor_sync(0xFFFFFFFFu, cnt, o);
+    if (lane == 0) {
+        if (cnt) {
+            atomicMax(&sh.maxord, mx);
+            atomicMin(&sh.minord, mn);
+        }
+        atomicAdd(&sh.nstage, cnt);
+    }
+    __syncthreads();
+    const unsigned nv = sh.nstage, hi = sh.maxord, lo = sh.minord;
+    int nsel;
+    if (staged) {
+        const SStage s{stage, n};
+        const unsigned long long K = nv <= (unsigned)k ? 1ull : fast_kth(s, sh, (unsigned)k, lo, hi);
+        nsel = fast_emit_ordered(stage, n, K, out_idx, out_score, sh);
+    } else {
+        const unsigned long long K = nv <= (unsigned)k ? 1ull : fast_kth(g, sh, (unsigned)k, lo, hi);
+        nsel = fast_emit_bitmap(g, K, bound, out_idx, out_score, sh, bm);
+    }
+    fast_pad(nsel, k, out_idx, out_score);
+}
+
+__global__ void __launch_bounds__(kFT, 4) select_fast_kernel(SelectArgs a) {
+    extern __shared__ __align__(16) unsigned long long fast_smem[];
+    __shared__ FastShared sh;
+    const int row = blockIdx.x;
+    unsigned *bm = reinterpret_cast<unsigned *>(fast_smem);
+    unsigned long long *stage = fast_smem + kChunkWords / 2;
+    const int scap = a.stage_cap;
+    int *oi = a.out_idx + (long long)row * a.k;
+    float *os = a.out_score ? a.out_score + (long long)row * a.k : nullptr;
+    auto cand = [&](long long r, int bound, int k) {
+        const unsigned n = a.cnt[r];
+        fast_cand_row(a.buf + r * a.cap, (int)(n < a.cap ? n : a.cap), a.floor ? a.floor[r] : 0u, bound, k, oi, os,
+                      sh, stage, scap, bm);
+    };
+    switch (a.kind) {
+    case SEL_DENSE_CAND:
+    case SEL_REUSE_CAND:
+    case SEL_MEMBER_SCORES: {
+        if (!a.plan[0]) { fast_pad(0, a.k, oi, os); return; }
+        const int b = find_seg(a.cu, a.S, row);
+        const int t = row - a.cu[b];
+        if (a.kind == SEL_DENSE_CAND) {
+            cand(row, t, a.k);
+        } else {
+            const int n = a.cu[b + 1] - a.cu[b];
+            const int p = a.plan[a.pl.rp() + b] + group_of(t, n, a.g, a.db);
+            // Reuse, and members scored on their own (guardrail): the top-k of
+            // the scored row's candidates inside the member's prefix
+            if (a.kind == SEL_REUSE_CAND || t < dense_rows(n, a.g, a.db))
+                cand(p, t, a.k);
+            else
+                fast_member_row(a.scores + (long long)row * a.ld, a.cand + (long long)p * a.c, a.c, t, a.k, oi, os,
+                                sh, stage, scap, bm);
+        }
+        return;
+    }
+    case SEL_PROXY_TO_C: {
+        if (!a.plan[0]) { fast_pad(0, a.k, oi, os); return; }
+        if (row >= a.plan[2]) return;
+        const int *rp = a.plan + a.pl.rp();
+        const int b = find_seg(rp, a.S, row);
+        const int i = row - rp[b];
+        const int n = a.cu[b + 1] - a.cu[b];
+        if (i < dense_rows(n, a.g, a.db)) {  // a member scored on its own needs no candidate set
+            fast_pad(0, a.k, oi, nullptr);
+            return;
+        }
+        cand(row, row_bound(i, n, a.g, a.db), a.k);
+        return;
+    }
+    case SEL_PROXY_TO_BLOCKS: {
+        if (!a.plan[0]) { fast_pad(0, a.k, oi, os); return; }
+        if (row >= a.plan[2]) return;
+        const int *rp = a.plan + a.pl.rp();
+        const int b = find_seg(rp, a.S, row);
+        const int i = row - rp[b];
+        const int n = a.cu[b + 1] - a.cu[b];
+        const int tl = row_bound(i, n, a.g);
+        // the partial block holding the last member takes one slot of the budget
+        const int kr = a.k - (((tl + 1) & (kBlockN - 1)) ? 1 : 0);
+        if (kr > 0) {
+            const unsigned cn = a.cnt[row];
+            fast_cand_row(a.buf + (long long)row * a.cap, (int)(cn < a.cap ? cn : a.cap), a.floor ? a.floor[row] : 0u,
+                          key_bound(tl, kBlockShift), kr, oi, nullptr, sh, stage, scap, bm);
+        }
+        for (int r = (kr > 0 ? kr : 0) + (int)threadIdx.x; r < a.k; r += kFT) oi[r] = -1;
+        return;
+    }
+    case SEL_DEC_MEMBER: {
+        const int b = row / a.G, m = row % a.G;
+        const int kv = a.kv_len[b];
+        if (kv < a.G || kv > a.n_max) {
+            if (threadIdx.x == 0) raise_status(a.status, ST_INVALID);
+            fast_pad(0, a.k, oi, os);
+            return;
+        }
+        fast_member_row(a.scores + (long long)row * a.ld, a.cand + (long long)b * a.c, a.c, kv - a.G + m, a.k, oi,
+                        os, sh, stage, scap, bm);
+        return;
+    }
+    default:
+        return;
+    }
+}
+
+
+// Staging room (keys) of select_fast_kernel: room for the top-k plus the
+// entries the floor lets through beyond it, and for every entry of a member
+// row (c); at least the room that still fits four CTAs per SM.
+constexpr int kFastMinRoom = 4608;
+
+bool fast_kind(int kind) {
+    return kind == SEL_DENSE_CAND || kind == SEL_REUSE_CAND || kind == SEL_PROXY_TO_C ||
+           kind == SEL_PROXY_TO_BLOCKS || kind == SEL_MEMBER_SCORES || kind == SEL_DEC_MEMBER;
+}
+
+cudaError_t launch_select_fast(const SelectArgs &a, cudaStream_t st) {
+    SelectArgs b = a;
+    const bool member = a.kind == SEL_MEMBER_SCORES || a.kind == SEL_DEC_MEMBER;
+    long long room = 2LL * a.k;
+    if (member && a.c > room) room = a.c;
+    if (room < kFastMinRoom) room = kFastMinRoom;
+    room = (room + 255) / 256 * 256;
+    const size_t limit = 232448 - sizeof(FastShared) - 1024 - (size_t)kChunkWords * 4;
+    if ((size_t)room * 8 > limit) room = (long long)(limit / 8);
+    b.stage_cap = (int)room;
+    const size_t smem = (size_t)kChunkWords * 4 + (size_t)room * 8;
+    cudaError_t e = cudaFuncSetAttribute(select_fast_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    TraceScope ts("select", st);
+    select_fast_kernel<<<a.nrows, kFT, smem, st>>>(b);
+    return cudaGetLastError();
 }
 
 }  // namespace
 
 cudaError_t launch_select(const SelectArgs &a, cudaStream_t st) {
     if (a.nrows <= 0) return cudaSuccess;
+    if (fast_kind(a.kind)) return launch_select_fast(a, st);
     SelectArgs b = a;
     const size_t tail = ((size_t)a.bitmap_words * 2 + 32) * 4;  // bitmap + per-word prefix + warp totals
     const size_t limit = 232448 - sizeof(SelShared) - 1024;
@@ -492,3 +936,4 @@ cudaError_t launch_select(const SelectArgs &a, cudaStream_t st) {
 }
 
 }  // namespace idx
+

@@ -104,14 +104,14 @@ __global__ void __launch_bounds__(kSimtThreads) score_simt_kernel(ScoreArgs a) {
         __syncthreads();
         const int item = s_item;
         if (item >= nblocks) break;
-        const BlockInfo bi = block_info(plan, a.pl, a.cu, a.g, plan[a.pl.order() + item], a.kshift);
+        const BlockInfo bi = block_info(plan, a.pl, a.cu, a.g, plan[a.pl.order() + item], a.kshift, a.db);
         load_rows(qs, q + (long long)bi.row0 * HD, bi.nrows, HD);
         for (int i = threadIdx.x; i < RB * a.H; i += blockDim.x)
             wsm[i] = (i / a.H) < bi.nrows ? a.w[(long long)bi.row0 * a.H + i] : 0.0f;
         if (a.sink == SINK_FILTER && warp < RB) sel_init(sel[warp], hist + warp * kBins);
         const int r = warp;
         const bool row_ok = r < bi.nrows;
-        const int bound = row_ok ? key_bound(row_bound(bi.i0 + r, bi.n, a.g), a.kshift) : -1;
+        const int bound = row_ok ? key_bound(row_bound(bi.i0 + r, bi.n, a.g, a.db), a.kshift) : -1;
         const long long grow = (long long)bi.row0 + r;
         int slot = -1;
         if (a.sink == SINK_SPILL && row_ok && a.slot_of_row) slot = a.slot_of_row[grow];
@@ -216,8 +216,9 @@ __global__ void __launch_bounds__(kSimtThreads) gather_simt_kernel(GatherArgs a,
         const int b = find_seg(rp, a.S, grp);
         const int i = grp - rp[b];
         const int n = a.cu[b + 1] - a.cu[b];
-        const int lo = i * a.g;
-        const int cnt = (lo + a.g < n ? lo + a.g : n) - lo;
+        if (i < dense_rows(n, a.g, a.db)) return;  // a member scored on its own: no re-score
+        const int lo = group_start(i, n, a.g, a.db);
+        const int cnt = group_size(i, n, a.g, a.db);
         mrow0 = (long long)a.cu[b] + lo + mc * RB;
         nmem = cnt - mc * RB;
         key0 = a.cu[b];

@@ -72,8 +72,9 @@ __device__ __forceinline__ Item item_info(const GatherArgs &g, const DecodeArgs 
             const int b = find_seg(rp, g.S, grp);
             const int i = grp - rp[b];
             const int n = g.cu[b + 1] - g.cu[b];
-            const int lo = i * g.g;
-            cnt = (lo + g.g < n ? lo + g.g : n) - lo;
+            if (i < dense_rows(n, g.g, g.db)) return it;  // a member scored on its own: no re-score
+            const int lo = group_start(i, n, g.g, g.db);
+            cnt = group_size(i, n, g.g, g.db);
             m0 = (long long)g.cu[b] + lo;
             key0 = g.cu[b];
         } else {
@@ -351,7 +352,9 @@ __global__ void __launch_bounds__(256) compact_keys_kernel(GatherArgs a) {
     if (a.mode == 0) {
         if (!a.plan[0] || grp >= a.plan[2]) return;
         const int *rp = a.plan + a.pl.rp();
-        key0 = a.cu[find_seg(rp, a.S, grp)];
+        const int b = find_seg(rp, a.S, grp);
+        if (grp - rp[b] < dense_rows(a.cu[b + 1] - a.cu[b], a.g, a.db)) return;  // no candidate set
+        key0 = a.cu[b];
     } else {
         const int kv = a.kv_len[grp];
         if (kv < a.G || kv > a.n_max) return;

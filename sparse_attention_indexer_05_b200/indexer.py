@@ -74,9 +74,9 @@ def adaptive_workspace_size(T, H, d, topk, rho, num_seqs, dtype=torch.bfloat16) 
     return int(N.lib().idx_adaptive_workspace_size(T, H, d, topk, rho, num_seqs, dt))
 
 
-def pivot_workspace_size(T, H, d, topk, num_seqs, g, c, mode, dtype=torch.bfloat16) -> int:
+def pivot_workspace_size(T, H, d, topk, num_seqs, g, c, mode, dtype=torch.bfloat16, dense_below=0) -> int:
     dt = N.BF16 if dtype == torch.bfloat16 else N.F32
-    return int(N.lib().idx_pivot_workspace_size(T, H, d, topk, num_seqs, dt, g, c, _mode(mode)))
+    return int(N.lib().idx_pivot_workspace_size(T, H, d, topk, num_seqs, dt, g, c, _mode(mode), int(dense_below)))
 
 
 def decode_workspace_size(B, G, n_max, H, d, topk, c, mode, dtype=torch.bfloat16) -> int:
@@ -136,17 +136,19 @@ def adaptive_topk(q, k, w, cu_seqlens, topk: int, rho: int = 2, qfrac: float = 0
 
 
 def pivot_topk(q, k, w, cu_seqlens, topk: int, g: int, c: int, mode="refine", out_idx=None, out_score=None,
-               workspace=None, stream=None, return_scores=False):
-    """PIVOT Reuse / Refine indexer + top-k over groups of g queries."""
+               workspace=None, stream=None, return_scores=False, dense_below: int = 0):
+    """PIVOT Reuse / Refine indexer + top-k over groups of g queries.
+    dense_below > 0: groups whose last member's prefix holds at most that many
+    keys take the dense top-k (the guardrail)."""
     T, H, d = q.shape
     S = cu_seqlens.numel() - 1
     dt = _dtype_code(q)
     m = _mode(mode)
-    ws = _ws(workspace, pivot_workspace_size(T, H, d, topk, S, g, c, m, q.dtype), q.device)
+    ws = _ws(workspace, pivot_workspace_size(T, H, d, topk, S, g, c, m, q.dtype, dense_below), q.device)
     out_idx, out_score = _outs((T,), topk, q.device, out_idx, out_score, return_scores)
     N.check(N.lib().idx_pivot_topk(
         _dev(q, "q"), _dev(k, "k", q.dtype), _dev(w, "w", torch.float32), _dev(cu_seqlens, "cu_seqlens", torch.int32),
-        S, T, H, d, topk, dt, g, c, m, _dev(out_idx, "out_idx", torch.int32),
+        S, T, H, d, topk, dt, g, c, m, int(dense_below), _dev(out_idx, "out_idx", torch.int32),
         _dev(out_score, "out_score", torch.float32) if out_score is not None else None,
         ws.data_ptr(), ws.numel(), _stream(stream)), "idx_pivot_topk")
     return (out_idx, out_score) if return_scores else out_idx

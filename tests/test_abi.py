@@ -41,10 +41,18 @@ def test_workspace_sizes(lib):
     assert lib.idx_dense_workspace_size(16384, 64, 128, 2048, 1, 0) > 16384 * 2048 * 8
     assert lib.idx_dense_workspace_size(0, 64, 128, 2048, 1, 0) == 0
     assert lib.idx_dense_workspace_size(100, 64, 12, 8, 1, 0) == 0        # d % 8 != 0
-    assert lib.idx_pivot_workspace_size(65536, 64, 128, 2048, 1, 0, 4, 4096, 2) > 0
-    assert lib.idx_pivot_workspace_size(65536, 64, 128, 2048, 1, 0, 4, 1024, 2) == 0   # c < k
-    assert lib.idx_pivot_workspace_size(65536, 64, 128, 2048, 1, 0, 0, 4096, 2) == 0   # g < 1
-    assert lib.idx_pivot_workspace_size(65536, 64, 128, 2048, 1, 0, 4, 4096, 0) == 0   # dense mode
+    assert lib.idx_pivot_workspace_size(65536, 64, 128, 2048, 1, 0, 4, 4096, 2, 0) > 0
+    assert lib.idx_pivot_workspace_size(65536, 64, 128, 2048, 1, 0, 4, 1024, 2, 0) == 0   # c < k
+    assert lib.idx_pivot_workspace_size(65536, 64, 128, 2048, 1, 0, 0, 4096, 2, 0) == 0   # g < 1
+    assert lib.idx_pivot_workspace_size(65536, 64, 128, 2048, 1, 0, 4, 4096, 0, 0) == 0   # dense mode
+    # the guardrail: members of short groups are scored rows of their own, so
+    # the workspace grows with the threshold, up to one row per token
+    plain = lib.idx_pivot_workspace_size(65536, 64, 128, 2048, 1, 0, 4, 4096, 2, 0)
+    guard = lib.idx_pivot_workspace_size(65536, 64, 128, 2048, 1, 0, 4, 4096, 2, 8192)
+    assert guard > plain
+    assert lib.idx_pivot_workspace_size(65536, 64, 128, 2048, 1, 0, 4, 4096, 2, 1 << 20) >= guard
+    assert lib.idx_pivot_workspace_size(65536, 64, 128, 2048, 1, 0, 4, 4096, 2, -1) == 0  # negative threshold
+    assert lib.idx_pivot_workspace_size(65536, 64, 128, 2048, 1, 0, 4, 4096, 3, 64) == 0  # block mode
     assert lib.idx_decode_workspace_size(64, 2, 131072, 64, 128, 2048, 4096, 2, 0) > 64 * 131072 * 4
     assert lib.idx_decode_workspace_size(64, 2, 1, 64, 128, 2048, 4096, 2, 0) == 0     # n_max < G
 
@@ -79,11 +87,17 @@ def test_invalid_arguments_return_before_launch(lib):
     assert lib.idx_dense_topk(fake, fake, fake, fake, 1, 10, 4, 64, 8, 0, fake, None, ctypes.c_void_p(264),
                               1 << 30, None) == 3
     # refine with c < k
-    assert lib.idx_pivot_topk(fake, fake, fake, fake, 1, 10, 4, 64, 8, 0, 4, 4, 2, fake, None, fake, 1 << 30,
+    assert lib.idx_pivot_topk(fake, fake, fake, fake, 1, 10, 4, 64, 8, 0, 4, 4, 2, 0, fake, None, fake, 1 << 30,
                               None) == 1
     # unknown mode
-    assert lib.idx_pivot_topk(fake, fake, fake, fake, 1, 10, 4, 64, 8, 0, 4, 16, 7, fake, None, fake, 1 << 30,
+    assert lib.idx_pivot_topk(fake, fake, fake, fake, 1, 10, 4, 64, 8, 0, 4, 16, 7, 0, fake, None, fake, 1 << 30,
                               None) == 1
+    # negative guardrail threshold
+    assert lib.idx_pivot_topk(fake, fake, fake, fake, 1, 10, 4, 64, 8, 0, 4, 16, 2, -1, fake, None, fake, 1 << 30,
+                              None) == 1
+    # the guardrail is not offered for the block pre-filter
+    assert lib.idx_pivot_topk(fake, fake, fake, fake, 1, 10, 4, 64, 8, 0, 4, 64, 3, 64, fake, None, fake, 1 << 30,
+                              None) == 2
     # decode: more MTP queries than a row block holds
     assert lib.idx_decode_topk(fake, fake, fake, fake, 2, 9, 64, 4, 64, 8, 0, 0, 0, fake, None, fake, 1 << 30,
                                None) == 2
