@@ -66,6 +66,8 @@ def parse():
                    help="skip the 16384-token dense and 65536-token PIVOT (g=4, c=4096) legs")
     p.add_argument("--crossover", action="store_true",
                    help="only time dense, Reuse and Refine on single requests of 1K..64K tokens (g=4, 16)")
+    p.add_argument("--skip-study", action="store_true",
+                   help="CPU only: fraction of (row block, key tile) pairs a per-tile score bound could skip")
     p.add_argument("--dense-below", type=int, default=0,
                    help="--crossover: also time PIVOT with this guardrail threshold (0 = without)")
     p.add_argument("--no-cpu", action="store_true", help="skip the CPU-oracle baseline")
@@ -291,6 +293,83 @@ def run_configs(args, dev, lib, barrier, max_over_ranks, rank, bf16_sus):
     return out
 
 
+
+def run_skip_study(args):
+    """Could the score kernel skip whole key tiles?  For sampled row blocks
+    (8 consecutive queries, the kernel's unit) of the 16384-, 65536- and
+    131072-token workloads, walk the key tiles (128 keys) in the kernel's
+    ascending order and keep each row's exact running k-th best score tau
+    (the best threshold any one-pass filter can hold; the kernel's is lower).
+    A tile can be skipped only if, for all 8 rows, an upper bound on every
+    score in the tile is below tau.  Two bounds are measured:
+      box:  per head, max over the tile of q . k <= sum_i max(q_i kmin_i,
+            q_i kmax_i) from the tile's per-dimension key range; then
+            sum_j w_j max(0, bound_j);
+      max:  the tile's true largest score per row (the tightest bound there
+            is; no kernel can compute it without doing the work it would
+            skip).
+    Scores are computed here in fp32 from the bf16 inputs (a study, not a
+    parity reference)."""
+    from sparse_attention_indexer_05_b200 import workloads as W
+    rng = np.random.default_rng(11)
+    out = {}
+    cases = [("dense_L16384_rho0.95_planted1%", lambda: W.cfg_dense_16k(seed=0)),
+             ("pivot_L65536_rho0.95_planted1%", lambda: W.cfg_pivot_64k(seed=0)),
+             ("long_L131072_rho0.98_planted0.5%", lambda: W.cfg_long_single(seed=0))]
+    for name, make in cases:
+        P = make()
+        L = P.T
+        q = W.bf16_to_f32(P.q)
+        kk = W.bf16_to_f32(P.k)
+        w = P.w.astype(np.float32)
+        nblk = 24
+        starts = np.sort(rng.choice(np.arange(TOPK // 8 + 1, L // 8), size=nblk, replace=False)) * 8
+        pairs = skip_box = skip_max = row_pairs = row_skip_max = 0
+        ratios = []
+        for t0 in starts:
+            rows = np.arange(t0, t0 + 8)
+            t_hi = int(rows[-1])
+            ntiles = t_hi // 128 + 1
+            Kp = kk[:(ntiles * 128)]
+            sc = np.zeros((8, ntiles * 128), np.float32)
+            for c0 in range(0, ntiles * 128, 16384):
+                dots = np.einsum("rhd,sd->rhs", q[rows], Kp[c0:c0 + 16384], optimize=True)
+                sc[:, c0:c0 + 16384] = np.einsum("rh,rhs->rs", w[rows], np.maximum(dots, 0.0))
+            pos = np.arange(ntiles * 128)
+            sc = np.where(pos[None, :] <= rows[:, None], sc, -np.inf)
+            kt = Kp.reshape(ntiles, 128, D)
+            kmin, kmax = kt.min(axis=1), kt.max(axis=1)           # [ntiles, D]
+            qr = q[rows]                                          # [8, H, D]
+            hb = np.maximum(np.einsum("rhd,td->rht", np.maximum(qr, 0), kmax) +
+                            np.einsum("rhd,td->rht", np.minimum(qr, 0), kmin), 0.0)
+            box = np.einsum("rh,rht->rt", w[rows], hb)            # [8, ntiles]
+            tmax = sc.reshape(8, ntiles, 128).max(axis=2)         # [8, ntiles]
+            # exact running k-th best before each tile (the top-k kept as a set)
+            tau = np.full((8, ntiles), -np.inf, np.float32)
+            for r in range(8):
+                top = sc[r, :TOPK].copy()
+                for j in range(TOPK // 128, ntiles):
+                    tau[r, j] = np.partition(top, 0)[0] if np.isfinite(top).all() else -np.inf
+                    both = np.concatenate([top, sc[r, j * 128:(j + 1) * 128]])
+                    top = np.partition(both, len(both) - TOPK)[len(both) - TOPK:]
+            j0 = TOPK // 128
+            pairs += ntiles - j0
+            skip_box += int(np.all(box[:, j0:] < tau[:, j0:], axis=0).sum())
+            skip_max += int(np.all(tmax[:, j0:] < tau[:, j0:], axis=0).sum())
+            row_pairs += tmax[:, j0:].size
+            row_skip_max += int((tmax[:, j0:] < tau[:, j0:]).sum())
+            ok = np.isfinite(tmax[:, j0:]) & (tmax[:, j0:] > 0)
+            ratios.append((box[:, j0:][ok] / tmax[:, j0:][ok]))
+        out[name] = {"row_blocks": nblk, "tile_pairs": pairs, "skippable_box_bound": skip_box / pairs,
+                     "skippable_exact_tile_max": skip_max / pairs,
+                     "row_tile_pairs_below_tau_exact_tile_max": row_skip_max / row_pairs,
+                     "box_bound_over_true_tile_max_median": float(np.median(np.concatenate(ratios)))}
+        print(json.dumps({name: out[name]}), flush=True)
+        del P, q, kk
+    print(json.dumps({"skip_study": out, "unit": "fraction of causal (row block of 8, key tile of 128) pairs "
+                      "after the first k keys", "topk": TOPK}))
+    return 0
+
 def run_crossover(args):
     """Dense against PIVOT Reuse and Refine (c = 4096) on one request of
     L tokens, L = 1K .. 64K, g = 4 and 16: the inputs of the 65536-token
@@ -395,6 +474,8 @@ def main():
         return run_reference(args)
     if args.crossover:
         return run_crossover(args)
+    if args.skip_study:
+        return run_skip_study(args)
     import torch
 
     import sparse_attention_indexer_05_b200 as idx

@@ -170,6 +170,27 @@ idx_status idx_pivot_topk(const void *q, const void *k, const float *w, const in
                           idx_mode mode, int dense_below, int *out_idx, float *out_score, void *ws,
                           size_t ws_bytes, idx_stream_t stream);
 
+/* Output rows [row_lo, row_hi) only (packed token rows, 0 <= row_lo <= row_hi
+ * <= T): the same result as idx_dense_topk / idx_pivot_topk for those rows,
+ * computed without the work of the others; the other rows of out_idx and
+ * out_score are left as they are.  Every key of each request is still read
+ * (a row needs its whole prefix), so q, k and w are passed whole.  This is
+ * how one request is split across GPUs: each rank passes the ranges it owns
+ * (zig-zag chunks of equal causal work, groups whole; see the multi-GPU
+ * partition in the Python package) and writes disjoint rows.  PIVOT rows:
+ * a group is computed when one of its members is in the range, so a range
+ * that cuts a group recomputes that group on both sides.  Same workspace
+ * sizes and errors as the full calls, plus IDX_ERR_INVALID for a bad range;
+ * an empty range launches nothing. */
+idx_status idx_dense_topk_rows(const void *q, const void *k, const float *w, const int *cu_seqlens,
+                               int num_seqs, int T, int H, int d, int topk, idx_dtype dtype, int row_lo,
+                               int row_hi, int *out_idx, float *out_score, void *ws, size_t ws_bytes,
+                               idx_stream_t stream);
+idx_status idx_pivot_topk_rows(const void *q, const void *k, const float *w, const int *cu_seqlens,
+                               int num_seqs, int T, int H, int d, int topk, idx_dtype dtype, int g, int c,
+                               idx_mode mode, int dense_below, int row_lo, int row_hi, int *out_idx,
+                               float *out_score, void *ws, size_t ws_bytes, idx_stream_t stream);
+
 /* ------------------------------------------------------------- decode */
 
 /* Workspace bytes for idx_decode_topk. */

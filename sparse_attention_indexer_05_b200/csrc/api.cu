@@ -193,6 +193,7 @@ struct Prefill {
     PrefillWs L;
     cudaStream_t st;
     int db = 0;  // guardrail threshold (PIVOT modes)
+    int row_lo = 0, row_hi = -1;  // output rows of the call (-1: up to T)
 
     unsigned *status() const { return reinterpret_cast<unsigned *>(ws + L.status); }
     int *plan() const { return reinterpret_cast<int *>(ws + L.plan); }
@@ -231,8 +232,8 @@ struct Prefill {
     cudaError_t prepare() const {
         cudaError_t e = cudaMemsetAsync(status(), 0, 4, st);
         if (e != cudaSuccess) return e;
-        e = launch_plan(cu, S, T, mode == IDX_MODE_DENSE ? 1 : g, mode == IDX_MODE_DENSE ? 0 : db, plan(), L.pl,
-                        status(), st);
+        e = launch_plan(cu, S, T, mode == IDX_MODE_DENSE ? 1 : g, mode == IDX_MODE_DENSE ? 0 : db, row_lo,
+                        row_hi < 0 ? T : row_hi, plan(), L.pl, status(), st);
         if (e != cudaSuccess) return e;
         if (mode != IDX_MODE_DENSE)
             e = launch_proxy(q, w, cu, S, T, H, d, g, db, (int)dt, plan(), L.pl, ws + L.qbar,
@@ -319,20 +320,31 @@ size_t idx_dense_workspace_size(int T, int H, int d, int topk, int num_seqs, idx
     return prefill_ws(T, H, d, topk, num_seqs, dtype, 1, topk, IDX_MODE_DENSE).total;
 }
 
-idx_status idx_dense_topk(const void *q, const void *k, const float *w, const int *cu_seqlens, int num_seqs,
-                          int T, int H, int d, int topk, idx_dtype dtype, int *out_idx, float *out_score,
-                          void *ws, size_t ws_bytes, idx_stream_t stream) {
+idx_status idx_dense_topk_rows(const void *q, const void *k, const float *w, const int *cu_seqlens, int num_seqs,
+                               int T, int H, int d, int topk, idx_dtype dtype, int row_lo, int row_hi, int *out_idx,
+                               float *out_score, void *ws, size_t ws_bytes, idx_stream_t stream) {
+    if (row_lo < 0 || row_hi < row_lo || row_hi > T) return IDX_ERR_INVALID;
     const size_t need = idx_dense_workspace_size(T, H, d, topk, num_seqs, dtype);
     idx_status s = check_prefill(q, k, w, cu_seqlens, num_seqs, T, H, d, topk, dtype, out_idx, ws, ws_bytes,
                                  need);
     if (s != IDX_OK) return s;
+    if (row_lo == row_hi) return IDX_OK;
     TracePhase phase("dense");
     Prefill P{q, k, w, cu_seqlens, num_seqs, T, H, d, topk, dtype, 1, topk, IDX_MODE_DENSE,
               static_cast<char *>(ws), prefill_ws(T, H, d, topk, num_seqs, dtype, 1, topk, IDX_MODE_DENSE),
               reinterpret_cast<cudaStream_t>(stream)};
+    P.row_lo = row_lo;
+    P.row_hi = row_hi;
     TRY_CUDA(P.prepare());
     TRY_CUDA(P.score(P.score_args(false)));
     return cuda_st(launch_select(P.select_args(SEL_DENSE_CAND, T, topk, out_idx, out_score), P.st));
+}
+
+idx_status idx_dense_topk(const void *q, const void *k, const float *w, const int *cu_seqlens, int num_seqs,
+                          int T, int H, int d, int topk, idx_dtype dtype, int *out_idx, float *out_score,
+                          void *ws, size_t ws_bytes, idx_stream_t stream) {
+    return idx_dense_topk_rows(q, k, w, cu_seqlens, num_seqs, T, H, d, topk, dtype, 0, T > 0 ? T : 0, out_idx,
+                               out_score, ws, ws_bytes, stream);
 }
 
 size_t idx_adaptive_workspace_size(int T, int H, int d, int topk, int rho, int num_seqs, idx_dtype dtype) {
@@ -387,12 +399,13 @@ size_t idx_pivot_workspace_size(int T, int H, int d, int topk, int num_seqs, idx
     return prefill_ws(T, H, d, topk, num_seqs, dtype, g, c, mode, dense_below).total;
 }
 
-idx_status idx_pivot_topk(const void *q, const void *k, const float *w, const int *cu_seqlens, int num_seqs,
-                          int T, int H, int d, int topk, idx_dtype dtype, int g, int c, idx_mode mode,
-                          int dense_below, int *out_idx, float *out_score, void *ws, size_t ws_bytes,
-                          idx_stream_t stream) {
+idx_status idx_pivot_topk_rows(const void *q, const void *k, const float *w, const int *cu_seqlens, int num_seqs,
+                               int T, int H, int d, int topk, idx_dtype dtype, int g, int c, idx_mode mode,
+                               int dense_below, int row_lo, int row_hi, int *out_idx, float *out_score, void *ws,
+                               size_t ws_bytes, idx_stream_t stream) {
     if (g < 1 || dense_below < 0 || (mode != IDX_MODE_REUSE && mode != IDX_MODE_REFINE && mode != IDX_MODE_BLOCK))
         return IDX_ERR_INVALID;
+    if (row_lo < 0 || row_hi < row_lo || row_hi > T) return IDX_ERR_INVALID;
     if (refines(mode) && c < topk) return IDX_ERR_INVALID;
     if (mode == IDX_MODE_BLOCK && (c < kBlockN || c % kBlockN != 0)) return IDX_ERR_INVALID;
     if (mode == IDX_MODE_BLOCK && dense_below > 0) return IDX_ERR_UNSUPPORTED;
@@ -401,11 +414,14 @@ idx_status idx_pivot_topk(const void *q, const void *k, const float *w, const in
     idx_status s = check_prefill(q, k, w, cu_seqlens, num_seqs, T, H, d, topk, dtype, out_idx, ws, ws_bytes,
                                  need);
     if (s != IDX_OK) return s;
+    if (row_lo == row_hi) return IDX_OK;
     TracePhase phase(mode == IDX_MODE_REUSE ? "reuse" : mode == IDX_MODE_REFINE ? "refine" : "block");
     Prefill P{q, k, w, cu_seqlens, num_seqs, T, H, d, topk, dtype, g, c, mode, static_cast<char *>(ws),
               prefill_ws(T, H, d, topk, num_seqs, dtype, g, c, mode, dense_below),
               reinterpret_cast<cudaStream_t>(stream)};
     P.db = g > 1 ? dense_below : 0;
+    P.row_lo = row_lo;
+    P.row_hi = row_hi;
     TRY_CUDA(P.prepare());
     TRY_CUDA(P.score(P.score_args(true)));
     if (mode == IDX_MODE_REUSE)
@@ -423,6 +439,14 @@ idx_status idx_pivot_topk(const void *q, const void *k, const float *w, const in
     TRY_CUDA(tc_gather_supported(H, d, (int)dtype, g, c) ? launch_gather_tc(ga, P.st)
                                                        : launch_gather_simt(ga, (int)dtype, P.st));
     return cuda_st(launch_select(P.select_args(SEL_MEMBER_SCORES, T, topk, out_idx, out_score), P.st));
+}
+
+idx_status idx_pivot_topk(const void *q, const void *k, const float *w, const int *cu_seqlens, int num_seqs,
+                          int T, int H, int d, int topk, idx_dtype dtype, int g, int c, idx_mode mode,
+                          int dense_below, int *out_idx, float *out_score, void *ws, size_t ws_bytes,
+                          idx_stream_t stream) {
+    return idx_pivot_topk_rows(q, k, w, cu_seqlens, num_seqs, T, H, d, topk, dtype, g, c, mode, dense_below, 0,
+                               T > 0 ? T : 0, out_idx, out_score, ws, ws_bytes, stream);
 }
 
 size_t idx_decode_workspace_size(int B, int G, int n_max, int H, int d, int topk, int c, idx_mode mode,

@@ -12,21 +12,23 @@ constexpr int kMaxLen = 1 << 20;  // longest supported request / cache
 
 // Plan area (int32 words at the start of a prefill workspace plan region):
 //   [0] valid flag (1 = cu_seqlens passed the device checks)
-//   [1] number of row blocks      [2] number of scored rows
+//   [1] number of row blocks scheduled (those with a member in [row_lo, row_hi))
+//   [2] number of scored rows
 //   [3] work counter (persistent score kernels)
-//   [4 .. 4+S]          rp[b]: first scored row of request b (S = num_seqs)
-//   [5+S .. 5+2S]       bp[b]: first row block of request b
-//   [6+2S .. +maxblk)   order: row blocks, longest key range first
+//   [4] row_lo  [5] row_hi: the output rows (packed token rows) of the call
+//   [6 .. 6+S]          rp[b]: first scored row of request b (S = num_seqs)
+//   [7+S .. 7+2S]       bp[b]: first row block of request b
+//   [8+2S .. +maxblk)   order: scheduled row blocks, longest key range first
 //   then (maxtiles+1)   per-tile-count histogram (plan scratch)
 struct PlanLayout {
     int S, maxblk, maxtiles;
     __host__ __device__ size_t words() const {
-        return (size_t)6 + 2 * (size_t)S + (size_t)maxblk + (size_t)maxtiles + 1;
+        return (size_t)8 + 2 * (size_t)S + (size_t)maxblk + (size_t)maxtiles + 1;
     }
-    __host__ __device__ int rp() const { return 4; }
-    __host__ __device__ int bp() const { return 5 + S; }
-    __host__ __device__ int order() const { return 6 + 2 * S; }
-    __host__ __device__ int hist() const { return 6 + 2 * S + maxblk; }
+    __host__ __device__ int rp() const { return 6; }
+    __host__ __device__ int bp() const { return 7 + S; }
+    __host__ __device__ int order() const { return 8 + 2 * S; }
+    __host__ __device__ int hist() const { return 8 + 2 * S + maxblk; }
 };
 
 enum Sink { SINK_FILTER = 0, SINK_SPILL = 1 };
@@ -196,8 +198,8 @@ struct TraceScope {
 };
 
 // ---- launchers (each returns cudaSuccess or the launch error)
-cudaError_t launch_plan(const int *cu, int S, int T, int g, int db, int *plan, const PlanLayout &pl,
-                        unsigned *status, cudaStream_t st);
+cudaError_t launch_plan(const int *cu, int S, int T, int g, int db, int row_lo, int row_hi, int *plan,
+                        const PlanLayout &pl, unsigned *status, cudaStream_t st);
 cudaError_t launch_score_simt(const ScoreArgs &a, int dtype, cudaStream_t st);
 cudaError_t launch_score_tc(const ScoreArgs &a, cudaStream_t st);
 cudaError_t launch_decode_simt(const DecodeArgs &a, int dtype, cudaStream_t st);

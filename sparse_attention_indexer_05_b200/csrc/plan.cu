@@ -37,7 +37,8 @@ __device__ int block_incl_scan(int v, int *warp_tot, int *total) {
 }
 
 __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const int *cu, int S, int T, int g, int db,
-                                                            int *plan, PlanLayout pl, unsigned *status) {
+                                                            int row_lo, int row_hi, int *plan, PlanLayout pl,
+                                                            unsigned *status) {
     __shared__ int s_bad;
     __shared__ int warp_tot[32];
     __shared__ int warp_tot2[32];
@@ -51,10 +52,14 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const int *cu, int S
     __syncthreads();
     if (s_bad) {
         if (tid == 0) {
-            plan[0] = 0; plan[1] = 0; plan[2] = 0; plan[3] = 0;
+            plan[0] = 0; plan[1] = 0; plan[2] = 0; plan[3] = 0; plan[4] = 0; plan[5] = 0;
             raise_status(status, ST_INVALID);
         }
         return;
+    }
+    if (tid == 0) {
+        plan[4] = row_lo;
+        plan[5] = row_hi;
     }
     int *rp = plan + pl.rp();
     int *bp = plan + pl.bp();
@@ -77,15 +82,23 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const int *cu, int S
     if (tid == 0) {
         rp[S] = carry_r;
         bp[S] = carry_b;
-        plan[1] = nblocks;
         plan[2] = carry_r;
         plan[3] = 0;
     }
     int *hist = plan + pl.hist();
     for (int i = tid; i <= pl.maxtiles; i += kPlanThreads) hist[i] = 0;
     __syncthreads();
+    // a row block is scheduled when the members of its scored rows (a
+    // contiguous run of tokens) meet [row_lo, row_hi)
+    auto scheduled = [&](const BlockInfo &bi) {
+        const int il = bi.i0 + bi.nrows - 1;
+        const long long lo = (long long)cu[bi.b] + group_start(bi.i0, bi.n, g, db);
+        const long long hi = (long long)cu[bi.b] + group_start(il, bi.n, g, db) + group_size(il, bi.n, g, db);
+        return bi.nrows > 0 && hi > row_lo && lo < row_hi;
+    };
     for (int blk = tid; blk < nblocks; blk += kPlanThreads) {
         const BlockInfo bi = block_info(plan, pl, cu, g, blk, 0, db);
+        if (!scheduled(bi)) continue;
         const int t = bi.ntiles < pl.maxtiles ? bi.ntiles : pl.maxtiles;
         atomicAdd(&hist[t], 1);
     }
@@ -98,11 +111,13 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const int *cu, int S
             hist[t] = run;
             run += h;
         }
+        plan[1] = run;
     }
     __syncthreads();
     int *order = plan + pl.order();
     for (int blk = tid; blk < nblocks; blk += kPlanThreads) {
         const BlockInfo bi = block_info(plan, pl, cu, g, blk, 0, db);
+        if (!scheduled(bi)) continue;
         const int t = bi.ntiles < pl.maxtiles ? bi.ntiles : pl.maxtiles;
         order[atomicAdd(&hist[t], 1)] = blk;
     }
@@ -111,10 +126,10 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const int *cu, int S
 
 }  // namespace
 
-cudaError_t launch_plan(const int *cu, int S, int T, int g, int db, int *plan, const PlanLayout &pl,
-                        unsigned *status, cudaStream_t st) {
+cudaError_t launch_plan(const int *cu, int S, int T, int g, int db, int row_lo, int row_hi, int *plan,
+                        const PlanLayout &pl, unsigned *status, cudaStream_t st) {
     TraceScope ts("plan", st);
-    plan_kernel<<<1, kPlanThreads, 0, st>>>(cu, S, T, g, db, plan, pl, status);
+    plan_kernel<<<1, kPlanThreads, 0, st>>>(cu, S, T, g, db, row_lo, row_hi, plan, pl, status);
     return cudaGetLastError();
 }
 

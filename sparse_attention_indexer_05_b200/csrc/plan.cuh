@@ -63,6 +63,16 @@ __device__ __forceinline__ int row_bound(int i, int n, int g, int db = 0) {
     return (int)((e < n ? e : n) - 1);
 }
 
+// Does scored row i of request b (n tokens) have a member among the call's
+// output rows [plan[4], plan[5]) (packed token rows)?  Rows without one are
+// neither scored (unless their row block is) nor selected.
+__device__ __forceinline__ bool row_in_range(const int *plan, const int *cu, int b, int i, int n, int g,
+                                             int db = 0) {
+    const long long lo = (long long)cu[b] + group_start(i, n, g, db);
+    const long long hi = lo + group_size(i, n, g, db);
+    return hi > plan[4] && lo < plan[5];
+}
+
 struct BlockInfo {
     int b;        // request
     int row0;     // first scored row (global index into the scored tensor)

@@ -166,6 +166,10 @@ __global__ void __launch_bounds__(kProxyThreads) block_expand_kernel(const int *
     const int b = find_seg(rp, S, p);
     const int i = p - rp[b];
     const int n = cu[b + 1] - cu[b];
+    if (!row_in_range(plan, cu, b, i, n, g)) {  // a proxy with no output member: no candidates
+        for (int j = threadIdx.x; j < c; j += blockDim.x) out[j] = -1;
+        return;
+    }
     const int tl = row_bound(i, n, g);
     const int part0 = (tl + 1) & ~(kBlockN - 1);
     const bool partial = part0 <= tl;

@@ -819,6 +819,7 @@ __global__ void __launch_bounds__(kFT, 4) select_fast_kernel(SelectArgs a) {
     case SEL_REUSE_CAND:
     case SEL_MEMBER_SCORES: {
         if (!a.plan[0]) { fast_pad(0, a.k, oi, os); return; }
+        if (row < a.plan[4] || row >= a.plan[5]) return;  // not an output row of this call
         const int b = find_seg(a.cu, a.S, row);
         const int t = row - a.cu[b];
         if (a.kind == SEL_DENSE_CAND) {
@@ -843,7 +844,9 @@ __global__ void __launch_bounds__(kFT, 4) select_fast_kernel(SelectArgs a) {
         const int b = find_seg(rp, a.S, row);
         const int i = row - rp[b];
         const int n = a.cu[b + 1] - a.cu[b];
-        if (i < dense_rows(n, a.g, a.db)) {  // a member scored on its own needs no candidate set
+        // a member scored on its own needs no candidate set; a proxy with no
+        // output member was not scored
+        if (i < dense_rows(n, a.g, a.db) || !row_in_range(a.plan, a.cu, b, i, n, a.g, a.db)) {
             fast_pad(0, a.k, oi, nullptr);
             return;
         }
@@ -857,6 +860,10 @@ __global__ void __launch_bounds__(kFT, 4) select_fast_kernel(SelectArgs a) {
         const int b = find_seg(rp, a.S, row);
         const int i = row - rp[b];
         const int n = a.cu[b + 1] - a.cu[b];
+        if (!row_in_range(a.plan, a.cu, b, i, n, a.g)) {  // a proxy with no output member was not scored
+            fast_pad(0, a.k, oi, nullptr);
+            return;
+        }
         const int tl = row_bound(i, n, a.g);
         // the partial block holding the last member takes one slot of the budget
         const int kr = a.k - (((tl + 1) & (kBlockN - 1)) ? 1 : 0);

@@ -216,7 +216,9 @@ __global__ void __launch_bounds__(kSimtThreads) gather_simt_kernel(GatherArgs a,
         const int b = find_seg(rp, a.S, grp);
         const int i = grp - rp[b];
         const int n = a.cu[b + 1] - a.cu[b];
-        if (i < dense_rows(n, a.g, a.db)) return;  // a member scored on its own: no re-score
+        // a member scored on its own needs no re-score; a group with no
+        // output member has no candidate set
+        if (i < dense_rows(n, a.g, a.db) || !row_in_range(a.plan, a.cu, b, i, n, a.g, a.db)) return;
         const int lo = group_start(i, n, a.g, a.db);
         const int cnt = group_size(i, n, a.g, a.db);
         mrow0 = (long long)a.cu[b] + lo + mc * RB;

@@ -72,7 +72,9 @@ __device__ __forceinline__ Item item_info(const GatherArgs &g, const DecodeArgs 
             const int b = find_seg(rp, g.S, grp);
             const int i = grp - rp[b];
             const int n = g.cu[b + 1] - g.cu[b];
-            if (i < dense_rows(n, g.g, g.db)) return it;  // a member scored on its own: no re-score
+            // a member scored on its own needs no re-score; a group with no
+            // output member has no candidate set
+            if (i < dense_rows(n, g.g, g.db) || !row_in_range(g.plan, g.cu, b, i, n, g.g, g.db)) return it;
             const int lo = group_start(i, n, g.g, g.db);
             cnt = group_size(i, n, g.g, g.db);
             m0 = (long long)g.cu[b] + lo;
@@ -353,7 +355,8 @@ __global__ void __launch_bounds__(256) compact_keys_kernel(GatherArgs a) {
         if (!a.plan[0] || grp >= a.plan[2]) return;
         const int *rp = a.plan + a.pl.rp();
         const int b = find_seg(rp, a.S, grp);
-        if (grp - rp[b] < dense_rows(a.cu[b + 1] - a.cu[b], a.g, a.db)) return;  // no candidate set
+        const int i = grp - rp[b], n = a.cu[b + 1] - a.cu[b];
+        if (i < dense_rows(n, a.g, a.db) || !row_in_range(a.plan, a.cu, b, i, n, a.g, a.db)) return;  // no set
         key0 = a.cu[b];
     } else {
         const int kv = a.kv_len[grp];

@@ -93,18 +93,20 @@ def _outs(rows_shape, topk, device, out_idx, out_score, return_scores):
 
 
 def dense_topk(q, k, w, cu_seqlens, topk: int, out_idx=None, out_score=None, workspace=None, stream=None,
-               return_scores=False):
-    """Dense indexer + top-k; q [T,H,d], k [T,d], w [T,H] fp32, cu_seqlens int32 [S+1]."""
+               return_scores=False, rows=None):
+    """Dense indexer + top-k; q [T,H,d], k [T,d], w [T,H] fp32, cu_seqlens int32 [S+1].
+    rows=(lo, hi): compute output rows lo..hi-1 only (the others are left as they are)."""
     T, H, d = q.shape
     S = cu_seqlens.numel() - 1
     dt = _dtype_code(q)
     ws = _ws(workspace, dense_workspace_size(T, H, d, topk, S, q.dtype), q.device)
     out_idx, out_score = _outs((T,), topk, q.device, out_idx, out_score, return_scores)
-    N.check(N.lib().idx_dense_topk(
+    lo, hi = (0, T) if rows is None else (int(rows[0]), int(rows[1]))
+    N.check(N.lib().idx_dense_topk_rows(
         _dev(q, "q"), _dev(k, "k", q.dtype), _dev(w, "w", torch.float32), _dev(cu_seqlens, "cu_seqlens", torch.int32),
-        S, T, H, d, topk, dt, _dev(out_idx, "out_idx", torch.int32),
+        S, T, H, d, topk, dt, lo, hi, _dev(out_idx, "out_idx", torch.int32),
         _dev(out_score, "out_score", torch.float32) if out_score is not None else None,
-        ws.data_ptr(), ws.numel(), _stream(stream)), "idx_dense_topk")
+        ws.data_ptr(), ws.numel(), _stream(stream)), "idx_dense_topk_rows")
     return (out_idx, out_score) if return_scores else out_idx
 
 
@@ -136,21 +138,23 @@ def adaptive_topk(q, k, w, cu_seqlens, topk: int, rho: int = 2, qfrac: float = 0
 
 
 def pivot_topk(q, k, w, cu_seqlens, topk: int, g: int, c: int, mode="refine", out_idx=None, out_score=None,
-               workspace=None, stream=None, return_scores=False, dense_below: int = 0):
+               workspace=None, stream=None, return_scores=False, dense_below: int = 0, rows=None):
     """PIVOT Reuse / Refine indexer + top-k over groups of g queries.
     dense_below > 0: groups whose last member's prefix holds at most that many
-    keys take the dense top-k (the guardrail)."""
+    keys take the dense top-k (the guardrail).  rows=(lo, hi): output rows
+    lo..hi-1 only."""
     T, H, d = q.shape
     S = cu_seqlens.numel() - 1
     dt = _dtype_code(q)
     m = _mode(mode)
     ws = _ws(workspace, pivot_workspace_size(T, H, d, topk, S, g, c, m, q.dtype, dense_below), q.device)
     out_idx, out_score = _outs((T,), topk, q.device, out_idx, out_score, return_scores)
-    N.check(N.lib().idx_pivot_topk(
+    lo, hi = (0, T) if rows is None else (int(rows[0]), int(rows[1]))
+    N.check(N.lib().idx_pivot_topk_rows(
         _dev(q, "q"), _dev(k, "k", q.dtype), _dev(w, "w", torch.float32), _dev(cu_seqlens, "cu_seqlens", torch.int32),
-        S, T, H, d, topk, dt, g, c, m, int(dense_below), _dev(out_idx, "out_idx", torch.int32),
+        S, T, H, d, topk, dt, g, c, m, int(dense_below), lo, hi, _dev(out_idx, "out_idx", torch.int32),
         _dev(out_score, "out_score", torch.float32) if out_score is not None else None,
-        ws.data_ptr(), ws.numel(), _stream(stream)), "idx_pivot_topk")
+        ws.data_ptr(), ws.numel(), _stream(stream)), "idx_pivot_topk_rows")
     return (out_idx, out_score) if return_scores else out_idx
 
 

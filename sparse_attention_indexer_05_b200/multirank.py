@@ -1,8 +1,15 @@
 """Host plumbing of a multi-GPU run: one process per GPU, launched by
 torchrun.  The indexer shards without an exchange step (prefill rows are
-independent given the keys, decode requests are independent), so each rank
-works on its own batch and the only collectives are the barrier around the
-timed region and the max over ranks of the measured time."""
+independent given the keys, decode requests are independent), so the only
+collectives are the barrier around the timed region and the max over ranks
+of the measured time.  Two ways to use N GPUs:
+  * independent batches: each rank works on its own batch (weak scaling);
+  * one request split across ranks (strong scaling): every rank holds the
+    request's keys, queries and weights (the keys are what every row needs;
+    here each rank generates or copies them whole, no collective), and
+    computes the top-k of the rows zigzag_ranges() gives it, through the
+    library's row-range entry points; the ranks' rows are disjoint and
+    together cover the request."""
 from __future__ import annotations
 
 import datetime
@@ -50,3 +57,29 @@ def rank_seed(rank: int, base: int = 0) -> int:
 def finish():
     if dist.is_initialized():
         dist.destroy_process_group()
+
+
+def zigzag_ranges(n: int, world: int, rank: int, align: int = 1):
+    """Rows of one request of n tokens that `rank` owns when the request is
+    split over `world` ranks: the request is cut into 2*world chunks of equal
+    length, at multiples of `align` (a multiple of the PIVOT group size keeps
+    every group on one rank), and rank r owns chunks r and 2*world-1-r.  Under
+    the causal mask a chunk's work grows with its position, so each rank's
+    early chunk and late chunk add up to the same work on every rank, up to
+    the alignment.  Returns the rank's non-empty request-local ranges
+    [(lo, hi), ...] in ascending order."""
+    if world < 1 or not 0 <= rank < world or align < 1 or n < 0:
+        raise ValueError("bad split arguments")
+    nch = 2 * world
+    bounds = [min(n, int(round(c * n / nch / align)) * align) for c in range(nch)] + [n]
+    out = []
+    for c in sorted((rank, nch - 1 - rank)):
+        lo, hi = bounds[c], bounds[c + 1]
+        if hi > lo:
+            out.append((lo, hi))
+    return out
+
+
+def causal_pairs(ranges) -> int:
+    """(query, key) pairs under the causal mask of the rows in `ranges`."""
+    return sum((hi * (hi + 1) - lo * (lo + 1)) // 2 for lo, hi in ranges)

@@ -84,9 +84,10 @@ def test_paged_equals_contiguous(idx, page):
         assert np.array_equal(gs.view(np.uint32), rs.view(np.uint32)), (page, mode)
 
 
-@pytest.mark.parametrize("page", [1, 4])
+@pytest.mark.parametrize("page", [1, 4, 8, 64])
 def test_small_pages_against_oracle(idx, page):
-    # pages under 8 keys take the CUDA-core scan: compare with the oracle
+    # pages under 8 keys take the CUDA-core scan, 8 and more the tensor-core
+    # scan (64: the serving page size the bench uses): compare with the oracle
     topk, c = 64, 128
     D = W.decode(B=3, n=700, G=2, H=64, d=128, topk=topk, c=c, seed=5, kv_len=[700, 300, 3], n_max=700)
     bounds = [int(n) - 2 + m for n in D.kv_len for m in range(2)]
