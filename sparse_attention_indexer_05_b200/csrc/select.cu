@@ -557,8 +557,8 @@ __device__ unsigned long long fast_kth(const Src &src, FastShared &sh, unsigned 
 // List the nonzero keys >= K of src in ascending position through a bitmap
 // (chunks of kChunkBits positions over 0..bound); returns how many.
 template <class Src>
-__device__ int fast_emit_bitmap(const Src &src, unsigned long long K, int bound, int *out_idx, float *out_score,
-                                FastShared &sh, unsigned *bm) {
+__device__ int fast_emit_bitmap(const Src &src, unsigned long long K, int bound, int k, int *out_idx,
+                                float *out_score, FastShared &sh, unsigned *bm) {
     const int tid = threadIdx.x;
     int base = 0;
     for (int c0 = 0; c0 <= bound; c0 += kChunkBits) {
@@ -599,7 +599,8 @@ __device__ int fast_emit_bitmap(const Src &src, unsigned long long K, int bound,
             while (x) {
                 const int bit = __ffs(x) - 1;
                 x &= x - 1u;
-                out_idx[r++] = c0 + (w0 + j) * 32 + bit;
+                if (r < (unsigned)k) out_idx[r] = c0 + (w0 + j) * 32 + bit;  // never past the row
+                ++r;
             }
         }
         if (out_score) {
@@ -612,13 +613,14 @@ __device__ int fast_emit_bitmap(const Src &src, unsigned long long K, int bound,
                         const int w = p >> 5, owner = w / kWordsPer;
                         unsigned rk = sh.tpre[owner] + __popc(bm[w] & ((1u << (p & 31)) - 1u));
                         for (int x = owner * kWordsPer; x < w; ++x) rk += __popc(bm[x]);
-                        out_score[base + rk] = ord_score(key_ord(kk));
+                        if (base + (int)rk < k) out_score[base + rk] = ord_score(key_ord(kk));
                     }
                 }
             }
         }
         (void)nwords;
         base += (int)total;
+        if (base > k) base = k;
         __syncthreads();  // the bitmap is cleared again by the next chunk
     }
     return base;
@@ -626,7 +628,7 @@ __device__ int fast_emit_bitmap(const Src &src, unsigned long long K, int bound,
 
 // Member rows: the staged entries are in candidate order (ascending
 // position); list the nonzero keys >= K in that order.
-__device__ int fast_emit_ordered(const unsigned long long *st, int n, unsigned long long K, int *out_idx,
+__device__ int fast_emit_ordered(const unsigned long long *st, int n, unsigned long long K, int k, int *out_idx,
                                  float *out_score, FastShared &sh) {
     const int tid = threadIdx.x;
     const int per = (n + kFT - 1) / kFT;
@@ -641,12 +643,14 @@ __device__ int fast_emit_ordered(const unsigned long long *st, int n, unsigned l
     for (int i = i0; i < i1; ++i) {
         const unsigned long long kk = st[i];
         if (kk != 0ull && kk >= K) {
-            out_idx[r] = key_pos(kk);
-            if (out_score) out_score[r] = ord_score(key_ord(kk));
+            if (r < (unsigned)k) {  // never past the row
+                out_idx[r] = key_pos(kk);
+                if (out_score) out_score[r] = ord_score(key_ord(kk));
+            }
             ++r;
         }
     }
-    return (int)total;
+    return (int)total < k ? (int)total : k;
 }
 
 __device__ __forceinline__ void fast_pad(int nsel, int k, int *out_idx, float *out_score) {
@@ -735,16 +739,16 @@ __device__ void fast_cand_row(const unsigned long long *buf, int n, unsigned flo
     int nsel;
     if (ns <= k) {
         const SStage s{stage, ns};
-        nsel = fast_emit_bitmap(s, 1ull, bound, out_idx, out_score, sh, bm);
+        nsel = fast_emit_bitmap(s, 1ull, bound, k, out_idx, out_score, sh, bm);
     } else if (ns <= stage_cap) {
         const SStage s{stage, ns};
         const unsigned long long K = fast_kth(s, sh, (unsigned)k, floor_ord, hi);
-        nsel = fast_emit_bitmap(s, K, bound, out_idx, out_score, sh, bm);
+        nsel = fast_emit_bitmap(s, K, bound, k, out_idx, out_score, sh, bm);
     } else {
         // more entries at or above the floor than the stage holds: the same
         // steps over the row in global memory
         const unsigned long long K = fast_kth(g, sh, (unsigned)k, floor_ord, hi);
-        nsel = fast_emit_bitmap(g, K, bound, out_idx, out_score, sh, bm);
+        nsel = fast_emit_bitmap(g, K, bound, k, out_idx, out_score, sh, bm);
     }
     fast_pad(nsel, k, out_idx, out_score);
 }
@@ -792,10 +796,10 @@ __device__ void fast_member_row(const float *sc, const int *pos, int n, int boun
     if (staged) {
         const SStage s{stage, n};
         const unsigned long long K = nv <= (unsigned)k ? 1ull : fast_kth(s, sh, (unsigned)k, lo, hi);
-        nsel = fast_emit_ordered(stage, n, K, out_idx, out_score, sh);
+        nsel = fast_emit_ordered(stage, n, K, k, out_idx, out_score, sh);
     } else {
         const unsigned long long K = nv <= (unsigned)k ? 1ull : fast_kth(g, sh, (unsigned)k, lo, hi);
-        nsel = fast_emit_bitmap(g, K, bound, out_idx, out_score, sh, bm);
+        nsel = fast_emit_bitmap(g, K, bound, k, out_idx, out_score, sh, bm);
     }
     fast_pad(nsel, k, out_idx, out_score);
 }
