@@ -495,7 +495,9 @@ def main():
         return M.max_over_ranks(x, dev)
 
     L = args.tokens
-    P = W.cfg_long_single(seed=M.rank_seed(rank), L=L)
+    split = args.split and world > 1
+    # split: every rank holds the same request (seed 0) and ranks only its rows
+    P = W.cfg_long_single(seed=0 if split else M.rank_seed(rank), L=L)
     cu1_h = np.array([0, L], np.int32)
     cu2_h = np.array([0, L // 2, L], np.int32)
     q, k, w = to_dev(P.q, dev), to_dev(P.k, dev), to_dev(P.w, dev)
@@ -509,11 +511,23 @@ def main():
     o1 = torch.empty(L, TOPK, dtype=torch.int32, device=dev)
     o2 = torch.empty(L, TOPK, dtype=torch.int32, device=dev)
 
+    if split:
+        # the rows this rank owns: zig-zag chunks of the dense request, and of
+        # each packed request with whole groups
+        r1 = M.zigzag_ranges(L, world, rank, align=8)
+        r2 = [(lo + off, hi + off) for off in (0, L // 2)
+              for lo, hi in M.zigzag_ranges(L // 2, world, rank, align=G_REF)]
+    else:
+        r1, r2 = [(0, L)], [(0, L)]
+
     def step(qq=q, kk=k, ww=w, c1=cu1, c2=cu2, oo1=o1, oo2=o2, st=None):
         if do_dense:
-            idx.dense_topk(qq, kk, ww, c1, TOPK, out_idx=oo1, workspace=ws1, stream=st)
+            for rg in r1:
+                idx.dense_topk(qq, kk, ww, c1, TOPK, out_idx=oo1, workspace=ws1, stream=st, rows=rg)
         if do_refine:
-            idx.pivot_topk(qq, kk, ww, c2, TOPK, G_REF, C_REF, "refine", out_idx=oo2, workspace=ws2, stream=st)
+            for rg in r2:
+                idx.pivot_topk(qq, kk, ww, c2, TOPK, G_REF, C_REF, "refine", out_idx=oo2, workspace=ws2, stream=st,
+                               rows=rg)
 
     for _ in range(args.warmup):
         step()
@@ -539,7 +553,11 @@ def main():
     ms = max_over_ranks(e0.elapsed_time(e1) / args.steps)
     nlaunch, tr = trace_report(lib)
     rows_per_step = L * (int(do_dense) + int(do_refine))
-    value = world * rows_per_step / (ms / 1000.0)
+    # whole job: every rank ranks its own batch, or the ranks share one
+    rows_job = rows_per_step if split else world * rows_per_step
+    value = rows_job / (ms / 1000.0)
+    if split:  # the extra legs time independent work; the split run times the step only
+        args.no_block = args.no_attn = args.no_adaptive = args.no_decode = args.no_configs = True
 
     bf16_peak, bf16_sus, hbm_peak, peak_src = peaks()
     n_dense, ms_dense = tr.get("dense/score_tc", (0, 0.0))
@@ -624,7 +642,7 @@ def main():
         ems = max_over_ranks(t0.elapsed_time(t1) / args.steps)
         h2d = hq.numel() * 2 + hk.numel() * 2 + hw.numel() * 4 + h1.numel() * 4 + h2.numel() * 4
         d2h = (hos[0][0].numel() + hos[0][1].numel()) * 4
-        e2e = {"value": world * rows_per_step / (ems / 1000.0), "unit": "queries/s", "ms_per_step": ems,
+        e2e = {"value": rows_job / (ems / 1000.0), "unit": "queries/s", "ms_per_step": ems,
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                "overlap": "inputs of step i+1 and results of step i-1 copied while step i computes"}
         del sets, outs
@@ -808,13 +826,16 @@ def main():
 
     line = {
         "metric": METRIC, "value": value, "unit": "queries/s", "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+        "scaling": "strong" if split else "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": {"workload": f"long_prefill_{L}_" + {"all": "dense+refine", "dense": "dense",
                                                           "refine": "refine"}[args.only] + "_g16_c4096",
                    "tokens": L, "H": H, "d": D,
                    "topk": TOPK, "dense_requests": [L], "refine_requests": [L // 2, L // 2],
-                   "g": G_REF, "c": C_REF, "parallelism": f"dp{world} (independent batches)",
+                   "g": G_REF, "c": C_REF,
+                   "parallelism": (f"split{world} (one request, zig-zag rows per rank)" if split
+                                   else f"dp{world} (independent batches)"),
                    "l2": "inputs larger than L2 (q is 2 GiB)"},
         "tflops_dense": achieved, "roofline": roof, "cpu_baseline": cpu, "e2e": e2e, "clocks": clk,
         "gpu_launches": nlaunch, "kernels": per_kernel, "block_prefilter": blk, "sparse_attn": att,

@@ -174,14 +174,23 @@ idx_status idx_pivot_topk(const void *q, const void *k, const float *w, const in
  * <= T): the same result as idx_dense_topk / idx_pivot_topk for those rows,
  * computed without the work of the others; the other rows of out_idx and
  * out_score are left as they are.  Every key of each request is still read
- * (a row needs its whole prefix), so q, k and w are passed whole.  This is
- * how one request is split across GPUs: each rank passes the ranges it owns
- * (zig-zag chunks of equal causal work, groups whole; see the multi-GPU
- * partition in the Python package) and writes disjoint rows.  PIVOT rows:
- * a group is computed when one of its members is in the range, so a range
- * that cuts a group recomputes that group on both sides.  Same workspace
- * sizes and errors as the full calls, plus IDX_ERR_INVALID for a bad range;
- * an empty range launches nothing. */
+ * (a row needs its whole prefix), so q, k and w are passed whole.  Uses:
+ *   - one request split across GPUs: each rank passes the ranges it owns
+ *     (zig-zag chunks of equal causal work, groups whole; see the multi-GPU
+ *     partition in the Python package) and writes disjoint rows;
+ *   - a long prefill in row chunks with a bounded workspace: the per-row
+ *     scratch covers the call's rows only, so a call whose range spans at
+ *     most max_rows rows needs *_workspace_size_rows(..., max_rows) bytes.
+ * PIVOT rows: a group is computed when one of its members is in the range,
+ * so a range that cuts a group recomputes that group on both sides.  Same
+ * errors as the full calls, plus IDX_ERR_INVALID for a bad range and
+ * IDX_ERR_WORKSPACE for a workspace smaller than the size for the range's
+ * length; an empty range launches nothing.  (The debug score export reads
+ * the member scores of full calls only.) */
+size_t idx_dense_workspace_size_rows(int T, int H, int d, int topk, int num_seqs, idx_dtype dtype,
+                                     int max_rows);
+size_t idx_pivot_workspace_size_rows(int T, int H, int d, int topk, int num_seqs, idx_dtype dtype, int g,
+                                     int c, idx_mode mode, int dense_below, int max_rows);
 idx_status idx_dense_topk_rows(const void *q, const void *k, const float *w, const int *cu_seqlens,
                                int num_seqs, int T, int H, int d, int topk, idx_dtype dtype, int row_lo,
                                int row_hi, int *out_idx, float *out_score, void *ws, size_t ws_bytes,

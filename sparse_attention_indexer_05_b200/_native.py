@@ -24,6 +24,8 @@ SIGNATURES = {
     "idx_pivot_workspace_size": (_sz, [_i, _i, _i, _i, _i, _i, _i, _i, _i, _i]),
     "idx_pivot_topk": (_i, [_vp, _vp, _fp, _ip, _i, _i, _i, _i, _i, _i, _i, _i, _i, _i, _ip, _fp, _vp, _sz,
                             _vp]),
+    "idx_dense_workspace_size_rows": (_sz, [_i, _i, _i, _i, _i, _i, _i]),
+    "idx_pivot_workspace_size_rows": (_sz, [_i, _i, _i, _i, _i, _i, _i, _i, _i, _i, _i]),
     "idx_dense_topk_rows": (_i, [_vp, _vp, _fp, _ip, _i, _i, _i, _i, _i, _i, _i, _i, _ip, _fp, _vp, _sz, _vp]),
     "idx_pivot_topk_rows": (_i, [_vp, _vp, _fp, _ip, _i, _i, _i, _i, _i, _i, _i, _i, _i, _i, _i, _i, _ip, _fp,
                                  _vp, _sz, _vp]),

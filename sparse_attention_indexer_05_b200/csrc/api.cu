@@ -52,6 +52,8 @@ long long nbound(int T) { return T < kMaxLen ? T : kMaxLen; }
 struct PrefillWs {
     PlanLayout pl;
     long long R;          // scored rows (queries or proxies, upper bound)
+    long long Rb;         // scored rows of one call's output rows (per-row scratch)
+    long long Mb;         // members of one call's groups (member scores)
     unsigned cap, ksel;
     size_t status, plan, slot, qbar, wbar, cnt, floor, buf, cand, msc, ckeys, kblk, cblk, total;
 };
@@ -60,16 +62,33 @@ bool refines(idx_mode m) { return m == IDX_MODE_REFINE || m == IDX_MODE_BLOCK; }
 
 long long block_rows(int T) { return (T >> kBlockShift) > 0 ? (T >> kBlockShift) : 1; }
 
+// Workspace of a prefill call whose output rows span at most max_rows rows
+// (max_rows <= 0 or >= T: any call).  The plan, proxies and the debug slot
+// map cover the whole batch; the per-row scratch only the call's rows.
 PrefillWs prefill_ws(int T, int H, int d, int topk, int S, idx_dtype dt, int g, int c, idx_mode mode,
-                     int db = 0) {
+                     int db = 0, long long max_rows = 0) {
     PrefillWs L{};
     const bool pivot = mode != IDX_MODE_DENSE;
+    const long long m = (max_rows <= 0 || max_rows >= T) ? T : max_rows;
     L.R = pivot ? ((long long)T + (long long)S * (g - 1)) / g : T;
+    long long extra = 0;
     if (pivot && db > 0 && g > 1) {
         // members of short groups are scored rows of their own: at most
         // min(n, db) per request
-        const long long extra = (long long)S * db < T ? (long long)S * db : T;
+        extra = (long long)S * db < T ? (long long)S * db : T;
         L.R = L.R + extra < T ? L.R + extra : T;
+    }
+    L.Rb = L.R;
+    L.Mb = T;
+    if (m < T) {
+        // a run of m output rows meets at most m / g + 2 groups per request it
+        // touches (partial groups at both ends), plus the short groups'
+        // members; those groups hold at most m + 2 (g - 1) members per request
+        long long rb = pivot ? m / g + 2LL * S + (extra < m ? extra : m) : m;
+        if (rb > m) rb = m;
+        L.Rb = rb < L.R ? rb : L.R;
+        const long long mb = pivot ? m + 2LL * (g - 1) * S : m;
+        L.Mb = mb < T ? mb : T;
     }
     L.pl.S = S;
     L.pl.maxblk = (int)((L.R + RB - 1) / RB + S);
@@ -85,16 +104,16 @@ PrefillWs prefill_ws(int T, int H, int d, int topk, int S, idx_dtype dt, int g, 
     L.slot = cv.take((size_t)(L.R > T ? L.R : T) * 4);
     L.qbar = pivot ? cv.take((size_t)L.R * H * d * esize(dt)) : 0;
     L.wbar = pivot ? cv.take((size_t)L.R * H * 4) : 0;
-    L.cnt = cv.take((size_t)L.R * 4);
-    L.floor = cv.take((size_t)L.R * 4);
-    L.buf = cv.take((size_t)L.R * L.cap * 8);
-    L.cand = refines(mode) ? cv.take((size_t)L.R * c * 4) : 0;
-    L.msc = refines(mode) ? cv.take((size_t)T * c * 4) : 0;
+    L.cnt = cv.take((size_t)L.Rb * 4);
+    L.floor = cv.take((size_t)L.Rb * 4);
+    L.buf = cv.take((size_t)L.Rb * L.cap * 8);
+    L.cand = refines(mode) ? cv.take((size_t)L.Rb * c * 4) : 0;
+    L.msc = refines(mode) ? cv.take((size_t)L.Mb * c * 4) : 0;
     L.ckeys = (refines(mode) && tc_gather_supported(H, d, (int)dt, g, c))
-                  ? cv.take((size_t)L.R * c_pad_of(c) * d * esize(dt))
+                  ? cv.take((size_t)L.Rb * c_pad_of(c) * d * esize(dt))
                   : 0;
     L.kblk = mode == IDX_MODE_BLOCK ? cv.take((size_t)block_rows(T) * d * esize(dt)) : 0;
-    L.cblk = mode == IDX_MODE_BLOCK ? cv.take((size_t)L.R * (c >> kBlockShift) * 4) : 0;
+    L.cblk = mode == IDX_MODE_BLOCK ? cv.take((size_t)L.Rb * (c >> kBlockShift) * 4) : 0;
     L.total = cv.off;
     return L;
 }
@@ -280,6 +299,7 @@ struct Prefill {
         a.plan = plan(); a.pl = L.pl;
         a.out = reinterpret_cast<float *>(ws + L.msc);
         a.ckeys = ws + L.ckeys;
+        a.ckey_groups = L.Rb;
         a.c_pad = c_pad_of(c);
         a.status = status();
         return a;
@@ -315,23 +335,28 @@ const char *idx_status_string(idx_status s) {
 
 int idx_uses_tensor_cores(int H, int d, idx_dtype dtype) { return tc_supported(H, d, (int)dtype) ? 1 : 0; }
 
+size_t idx_dense_workspace_size_rows(int T, int H, int d, int topk, int num_seqs, idx_dtype dtype, int max_rows) {
+    if (T < 1 || num_seqs < 1 || topk < 1 || max_rows < 0 || !shape_ok(H, d, dtype)) return 0;
+    return prefill_ws(T, H, d, topk, num_seqs, dtype, 1, topk, IDX_MODE_DENSE, 0, max_rows).total;
+}
+
 size_t idx_dense_workspace_size(int T, int H, int d, int topk, int num_seqs, idx_dtype dtype) {
-    if (T < 1 || num_seqs < 1 || topk < 1 || !shape_ok(H, d, dtype)) return 0;
-    return prefill_ws(T, H, d, topk, num_seqs, dtype, 1, topk, IDX_MODE_DENSE).total;
+    return idx_dense_workspace_size_rows(T, H, d, topk, num_seqs, dtype, 0);
 }
 
 idx_status idx_dense_topk_rows(const void *q, const void *k, const float *w, const int *cu_seqlens, int num_seqs,
                                int T, int H, int d, int topk, idx_dtype dtype, int row_lo, int row_hi, int *out_idx,
                                float *out_score, void *ws, size_t ws_bytes, idx_stream_t stream) {
     if (row_lo < 0 || row_hi < row_lo || row_hi > T) return IDX_ERR_INVALID;
-    const size_t need = idx_dense_workspace_size(T, H, d, topk, num_seqs, dtype);
+    const int m = row_hi - row_lo > 0 ? row_hi - row_lo : 1;
+    const size_t need = idx_dense_workspace_size_rows(T, H, d, topk, num_seqs, dtype, m);
     idx_status s = check_prefill(q, k, w, cu_seqlens, num_seqs, T, H, d, topk, dtype, out_idx, ws, ws_bytes,
                                  need);
     if (s != IDX_OK) return s;
     if (row_lo == row_hi) return IDX_OK;
     TracePhase phase("dense");
     Prefill P{q, k, w, cu_seqlens, num_seqs, T, H, d, topk, dtype, 1, topk, IDX_MODE_DENSE,
-              static_cast<char *>(ws), prefill_ws(T, H, d, topk, num_seqs, dtype, 1, topk, IDX_MODE_DENSE),
+              static_cast<char *>(ws), prefill_ws(T, H, d, topk, num_seqs, dtype, 1, topk, IDX_MODE_DENSE, 0, m),
               reinterpret_cast<cudaStream_t>(stream)};
     P.row_lo = row_lo;
     P.row_hi = row_hi;
@@ -390,13 +415,20 @@ idx_status idx_adaptive_topk(const void *q, const void *k, const float *w, const
     return cuda_st(launch_adaptive(a, P.st));
 }
 
-size_t idx_pivot_workspace_size(int T, int H, int d, int topk, int num_seqs, idx_dtype dtype, int g, int c,
-                                idx_mode mode, int dense_below) {
-    if (T < 1 || num_seqs < 1 || topk < 1 || g < 1 || dense_below < 0 || !shape_ok(H, d, dtype)) return 0;
+size_t idx_pivot_workspace_size_rows(int T, int H, int d, int topk, int num_seqs, idx_dtype dtype, int g, int c,
+                                     idx_mode mode, int dense_below, int max_rows) {
+    if (T < 1 || num_seqs < 1 || topk < 1 || g < 1 || dense_below < 0 || max_rows < 0 || !shape_ok(H, d, dtype))
+        return 0;
     if (mode != IDX_MODE_REUSE && mode != IDX_MODE_REFINE && mode != IDX_MODE_BLOCK) return 0;
+    if (mode == IDX_MODE_REUSE) c = topk;
     if (refines(mode) && c < topk) return 0;
     if (mode == IDX_MODE_BLOCK && (c < kBlockN || c % kBlockN != 0 || dense_below > 0)) return 0;
-    return prefill_ws(T, H, d, topk, num_seqs, dtype, g, c, mode, dense_below).total;
+    return prefill_ws(T, H, d, topk, num_seqs, dtype, g, c, mode, dense_below, max_rows).total;
+}
+
+size_t idx_pivot_workspace_size(int T, int H, int d, int topk, int num_seqs, idx_dtype dtype, int g, int c,
+                                idx_mode mode, int dense_below) {
+    return idx_pivot_workspace_size_rows(T, H, d, topk, num_seqs, dtype, g, c, mode, dense_below, 0);
 }
 
 idx_status idx_pivot_topk_rows(const void *q, const void *k, const float *w, const int *cu_seqlens, int num_seqs,
@@ -410,14 +442,15 @@ idx_status idx_pivot_topk_rows(const void *q, const void *k, const float *w, con
     if (mode == IDX_MODE_BLOCK && (c < kBlockN || c % kBlockN != 0)) return IDX_ERR_INVALID;
     if (mode == IDX_MODE_BLOCK && dense_below > 0) return IDX_ERR_UNSUPPORTED;
     if (mode == IDX_MODE_REUSE) c = topk;
-    const size_t need = idx_pivot_workspace_size(T, H, d, topk, num_seqs, dtype, g, c, mode, dense_below);
+    const int m = row_hi - row_lo > 0 ? row_hi - row_lo : 1;
+    const size_t need = idx_pivot_workspace_size_rows(T, H, d, topk, num_seqs, dtype, g, c, mode, dense_below, m);
     idx_status s = check_prefill(q, k, w, cu_seqlens, num_seqs, T, H, d, topk, dtype, out_idx, ws, ws_bytes,
                                  need);
     if (s != IDX_OK) return s;
     if (row_lo == row_hi) return IDX_OK;
     TracePhase phase(mode == IDX_MODE_REUSE ? "reuse" : mode == IDX_MODE_REFINE ? "refine" : "block");
     Prefill P{q, k, w, cu_seqlens, num_seqs, T, H, d, topk, dtype, g, c, mode, static_cast<char *>(ws),
-              prefill_ws(T, H, d, topk, num_seqs, dtype, g, c, mode, dense_below),
+              prefill_ws(T, H, d, topk, num_seqs, dtype, g, c, mode, dense_below, m),
               reinterpret_cast<cudaStream_t>(stream)};
     P.db = g > 1 ? dense_below : 0;
     P.row_lo = row_lo;
@@ -516,6 +549,7 @@ struct Decode {
         a.G = G; a.n_max = n_max; a.kv_len = kv;
         a.out = reinterpret_cast<float *>(ws + L.msc);
         a.ckeys = ws + L.ckeys;
+        a.ckey_groups = B;
         a.c_pad = c_pad_of(c);
         a.status = status();
         a.bt = bt; a.page = page; a.max_pages = max_pages; a.num_pages = num_pages;

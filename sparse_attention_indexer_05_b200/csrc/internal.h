@@ -16,19 +16,24 @@ constexpr int kMaxLen = 1 << 20;  // longest supported request / cache
 //   [2] number of scored rows
 //   [3] work counter (persistent score kernels)
 //   [4] row_lo  [5] row_hi: the output rows (packed token rows) of the call
-//   [6 .. 6+S]          rp[b]: first scored row of request b (S = num_seqs)
-//   [7+S .. 7+2S]       bp[b]: first row block of request b
-//   [8+2S .. +maxblk)   order: scheduled row blocks, longest key range first
+//   [6] p_lo    [7] p_hi: the scored rows with a member in [row_lo, row_hi);
+//       per-row scratch (candidate buffers, counts, floors, candidate sets,
+//       packed keys) is indexed from p_lo
+//   [8] m_lo: the first member of scored row p_lo; member scores (every
+//       member of the call's groups) are indexed from it
+//   [9 .. 9+S]          rp[b]: first scored row of request b (S = num_seqs)
+//   [10+S .. 10+2S]     bp[b]: first row block of request b
+//   [11+2S .. +maxblk)  order: scheduled row blocks, longest key range first
 //   then (maxtiles+1)   per-tile-count histogram (plan scratch)
 struct PlanLayout {
     int S, maxblk, maxtiles;
     __host__ __device__ size_t words() const {
-        return (size_t)8 + 2 * (size_t)S + (size_t)maxblk + (size_t)maxtiles + 1;
+        return (size_t)11 + 2 * (size_t)S + (size_t)maxblk + (size_t)maxtiles + 1;
     }
-    __host__ __device__ int rp() const { return 6; }
-    __host__ __device__ int bp() const { return 7 + S; }
-    __host__ __device__ int order() const { return 8 + 2 * S; }
-    __host__ __device__ int hist() const { return 8 + 2 * S + maxblk; }
+    __host__ __device__ int rp() const { return 9; }
+    __host__ __device__ int bp() const { return 10 + S; }
+    __host__ __device__ int order() const { return 11 + 2 * S; }
+    __host__ __device__ int hist() const { return 11 + 2 * S + maxblk; }
 };
 
 enum Sink { SINK_FILTER = 0, SINK_SPILL = 1 };
@@ -101,8 +106,10 @@ struct GatherArgs {
     PlanLayout pl;
     int G, n_max;
     const int *kv_len;
-    float *out;          // [rows, c] member scores
-    void *ckeys;         // [groups, c_pad, d] packed candidate keys (tensor-core path)
+    float *out;          // [rows, c] member scores (prefill: rows from the call's first member)
+    void *ckeys;         // [groups, c_pad, d] packed candidate keys (tensor-core path; prefill: groups
+                         // from the call's first scored row)
+    long long ckey_groups;  // groups the packed-key area holds
     int c_pad;           // c rounded up to a multiple of 128
     unsigned *status;
     const int *bt;       // decode: paged cache, as in DecodeArgs

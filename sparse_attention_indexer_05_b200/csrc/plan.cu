@@ -53,6 +53,7 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const int *cu, int S
     if (s_bad) {
         if (tid == 0) {
             plan[0] = 0; plan[1] = 0; plan[2] = 0; plan[3] = 0; plan[4] = 0; plan[5] = 0;
+            plan[6] = 0; plan[7] = 0; plan[8] = 0;
             raise_status(status, ST_INVALID);
         }
         return;
@@ -79,11 +80,25 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const int *cu, int S
         carry_b += tot_b;
     }
     const int nblocks = carry_b;
+    __syncthreads();  // every rp[b] is written
     if (tid == 0) {
         rp[S] = carry_r;
         bp[S] = carry_b;
         plan[2] = carry_r;
         plan[3] = 0;
+        // the scored rows holding the first and the last output row
+        int plo = 0, phi = 0, mlo = 0;
+        if (row_lo < row_hi) {
+            const int b0 = find_seg(cu, S, row_lo), b1 = find_seg(cu, S, row_hi - 1);
+            const int n0 = cu[b0 + 1] - cu[b0];
+            const int i0 = group_of(row_lo - cu[b0], n0, g, db);
+            plo = rp[b0] + i0;
+            mlo = cu[b0] + group_start(i0, n0, g, db);
+            phi = rp[b1] + group_of(row_hi - 1 - cu[b1], cu[b1 + 1] - cu[b1], g, db) + 1;
+        }
+        plan[6] = plo;
+        plan[7] = phi;
+        plan[8] = mlo;
     }
     int *hist = plan + pl.hist();
     for (int i = tid; i <= pl.maxtiles; i += kPlanThreads) hist[i] = 0;

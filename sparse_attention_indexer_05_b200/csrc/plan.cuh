@@ -73,6 +73,12 @@ __device__ __forceinline__ bool row_in_range(const int *plan, const int *cu, int
     return hi > plan[4] && lo < plan[5];
 }
 
+// Is scored row p one of the call's (a member in [row_lo, row_hi))?  Its
+// per-row scratch then sits at row p - plan[6].
+__device__ __forceinline__ bool scored_in_range(const int *plan, long long p) {
+    return p >= plan[6] && p < plan[7];
+}
+
 struct BlockInfo {
     int b;        // request
     int row0;     // first scored row (global index into the scored tensor)

@@ -156,24 +156,20 @@ __global__ void __launch_bounds__(kProxyThreads) block_expand_kernel(const int *
                                                                      PlanLayout pl, const int *cblk, int *cand,
                                                                      int c) {
     const int p = blockIdx.x;
-    int *out = cand + (long long)p * c;
+    // scratch rows (selected blocks, candidate sets) start at the call's
+    // first scored row; a proxy with no output member has none
+    if (!plan[0] || p >= plan[2] || !scored_in_range(plan, p)) return;
+    const long long sp = (long long)p - plan[6];
+    int *out = cand + sp * c;
     const int nb = c >> kBlockShift;
-    if (!plan[0] || p >= plan[2]) {
-        for (int j = threadIdx.x; j < c; j += blockDim.x) out[j] = -1;
-        return;
-    }
     const int *rp = plan + pl.rp();
     const int b = find_seg(rp, S, p);
     const int i = p - rp[b];
     const int n = cu[b + 1] - cu[b];
-    if (!row_in_range(plan, cu, b, i, n, g)) {  // a proxy with no output member: no candidates
-        for (int j = threadIdx.x; j < c; j += blockDim.x) out[j] = -1;
-        return;
-    }
     const int tl = row_bound(i, n, g);
     const int part0 = (tl + 1) & ~(kBlockN - 1);
     const bool partial = part0 <= tl;
-    const int *sel = cblk + (long long)p * nb;
+    const int *sel = cblk + sp * nb;
     for (int j = threadIdx.x; j < c; j += blockDim.x) {
         const int slot = j >> kBlockShift, r = j & (kBlockN - 1);
         int v;

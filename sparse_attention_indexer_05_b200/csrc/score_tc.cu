@@ -180,7 +180,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                 wsm[i] = (i / TC_H) < bi.nrows ? 0.5f * a.w[(long long)bi.row0 * TC_H + i] : 0.0f;
             if (e < RB) {
                 if (lane == 0) {
-                    sh.bound[e] = e < bi.nrows ? key_bound(row_bound(bi.i0 + e, bi.n, a.g, a.db), a.kshift) : -1;
+                    // a filtered row whose members are all outside the call's
+                    // output rows is not ranked (it has no scratch row)
+                    const bool act = e < bi.nrows && (a.sink != SINK_FILTER || scored_in_range(plan, bi.row0 + e));
+                    sh.bound[e] = act ? key_bound(row_bound(bi.i0 + e, bi.n, a.g, a.db), a.kshift) : -1;
                     sh.slot[e] = -1;
                     if (a.sink == SINK_SPILL && e < bi.nrows && a.slot_of_row)
                         sh.slot[e] = a.slot_of_row[bi.row0 + e];
@@ -246,7 +249,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint32_t tbase = tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(ra * 64);
             const bool filter = a.sink == SINK_FILTER;
             const int mrow = ra + (e & 1);       // row this warp maintains (warps with e & 3 < 2)
-            const bool maint = (e & 3) < 2 && mrow < bi.nrows;
+            const bool maint = (e & 3) < 2 && mrow < bi.nrows && (!filter || scored_in_range(plan, bi.row0 + mrow));
+            // scratch rows start at the call's first scored row
+            unsigned long long *buf0 = filter ? a.buf + ((long long)bi.row0 - plan[6]) * a.cap : nullptr;
+            const long long srow0 = (long long)bi.row0 - plan[6];
             bool ok = true;
             for (int j = 0; j < ntiles; ++j) {
                 const uint32_t t = kt + j;
@@ -273,8 +279,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                     const bool valid = ok && s <= sh.bound[r];
                     if (filter) {
-                        sel_offer(sh.sel[r], hist + r * kBins, a.buf + ((long long)bi.row0 + r) * a.cap, a.cap, valid,
-                                  score, s, a.status);
+                        sel_offer(sh.sel[r], hist + r * kBins, buf0 + (long long)r * a.cap, a.cap, valid, score, s,
+                                  a.status);
                     } else if (valid && sh.slot[r] >= 0) {
                         a.spill[(long long)sh.slot[r] * a.ld + s] = score;
                     }
@@ -282,14 +288,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (filter && ((j % kMaintEvery) == kMaintEvery - 1 || j == ntiles - 1)) {
                     tc::named_bar_sync(1 + role, 128);
                     if (maint)
-                        sel_maintain(sh.sel[mrow], hist + mrow * kBins, a.buf + ((long long)bi.row0 + mrow) * a.cap,
-                                     a.cap, a.ksel, scr + mrow * 256, KT * kMaintEvery);
+                        sel_maintain(sh.sel[mrow], hist + mrow * kBins, buf0 + (long long)mrow * a.cap, a.cap, a.ksel,
+                                     scr + mrow * 256, KT * kMaintEvery);
                     tc::named_bar_sync(1 + role, 128);
                 }
             }
             if (filter && maint && lane == 0) {
-                a.cnt[bi.row0 + mrow] = sh.sel[mrow].cnt;
-                if (a.floor_out) a.floor_out[bi.row0 + mrow] = sh.sel[mrow].floor;
+                a.cnt[srow0 + mrow] = sh.sel[mrow].cnt;
+                if (a.floor_out) a.floor_out[srow0 + mrow] = sh.sel[mrow].floor;
             }
         }
         kt += ntiles;

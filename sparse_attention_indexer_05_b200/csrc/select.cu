@@ -813,9 +813,13 @@ __global__ void __launch_bounds__(kFT, 4) select_fast_kernel(SelectArgs a) {
     const int scap = a.stage_cap;
     int *oi = a.out_idx + (long long)row * a.k;
     float *os = a.out_score ? a.out_score + (long long)row * a.k : nullptr;
+    // per-row scratch of prefill calls starts at the call's first scored row
+    // (plan[6]); member scores at the first member of that row (plan[8])
+    const long long p0 = a.kind == SEL_DEC_MEMBER ? 0 : a.plan[6];
     auto cand = [&](long long r, int bound, int k) {
-        const unsigned n = a.cnt[r];
-        fast_cand_row(a.buf + r * a.cap, (int)(n < a.cap ? n : a.cap), a.floor ? a.floor[r] : 0u, bound, k, oi, os,
+        const long long sr = r - p0;
+        const unsigned n = a.cnt[sr];
+        fast_cand_row(a.buf + sr * a.cap, (int)(n < a.cap ? n : a.cap), a.floor ? a.floor[sr] : 0u, bound, k, oi, os,
                       sh, stage, scap, bm);
     };
     switch (a.kind) {
@@ -836,47 +840,40 @@ __global__ void __launch_bounds__(kFT, 4) select_fast_kernel(SelectArgs a) {
             if (a.kind == SEL_REUSE_CAND || t < dense_rows(n, a.g, a.db))
                 cand(p, t, a.k);
             else
-                fast_member_row(a.scores + (long long)row * a.ld, a.cand + (long long)p * a.c, a.c, t, a.k, oi, os,
-                                sh, stage, scap, bm);
+                fast_member_row(a.scores + ((long long)row - a.plan[8]) * a.ld, a.cand + (p - p0) * a.c, a.c, t,
+                                a.k, oi, os, sh, stage, scap, bm);
         }
         return;
     }
-    case SEL_PROXY_TO_C: {
-        if (!a.plan[0]) { fast_pad(0, a.k, oi, os); return; }
-        if (row >= a.plan[2]) return;
-        const int *rp = a.plan + a.pl.rp();
-        const int b = find_seg(rp, a.S, row);
-        const int i = row - rp[b];
-        const int n = a.cu[b + 1] - a.cu[b];
-        // a member scored on its own needs no candidate set; a proxy with no
-        // output member was not scored
-        if (i < dense_rows(n, a.g, a.db) || !row_in_range(a.plan, a.cu, b, i, n, a.g, a.db)) {
-            fast_pad(0, a.k, oi, nullptr);
-            return;
-        }
-        cand(row, row_bound(i, n, a.g, a.db), a.k);
-        return;
-    }
+    case SEL_PROXY_TO_C:
     case SEL_PROXY_TO_BLOCKS: {
-        if (!a.plan[0]) { fast_pad(0, a.k, oi, os); return; }
-        if (row >= a.plan[2]) return;
+        // output: the proxy's scratch row (candidate set, or selected blocks);
+        // a proxy with no output member has none
+        if (!a.plan[0] || row >= a.plan[2] || !scored_in_range(a.plan, row)) return;
         const int *rp = a.plan + a.pl.rp();
         const int b = find_seg(rp, a.S, row);
         const int i = row - rp[b];
         const int n = a.cu[b + 1] - a.cu[b];
-        if (!row_in_range(a.plan, a.cu, b, i, n, a.g)) {  // a proxy with no output member was not scored
-            fast_pad(0, a.k, oi, nullptr);
+        int *po = a.out_idx + ((long long)row - p0) * a.k;
+        if (a.kind == SEL_PROXY_TO_C) {
+            if (i < dense_rows(n, a.g, a.db)) {  // a member scored on its own needs no candidate set
+                fast_pad(0, a.k, po, nullptr);
+                return;
+            }
+            oi = po;
+            os = nullptr;
+            cand(row, row_bound(i, n, a.g, a.db), a.k);
             return;
         }
         const int tl = row_bound(i, n, a.g);
         // the partial block holding the last member takes one slot of the budget
         const int kr = a.k - (((tl + 1) & (kBlockN - 1)) ? 1 : 0);
         if (kr > 0) {
-            const unsigned cn = a.cnt[row];
-            fast_cand_row(a.buf + (long long)row * a.cap, (int)(cn < a.cap ? cn : a.cap), a.floor ? a.floor[row] : 0u,
-                          key_bound(tl, kBlockShift), kr, oi, nullptr, sh, stage, scap, bm);
+            oi = po;
+            os = nullptr;
+            cand(row, key_bound(tl, kBlockShift), kr);
         }
-        for (int r = (kr > 0 ? kr : 0) + (int)threadIdx.x; r < a.k; r += kFT) oi[r] = -1;
+        for (int r = (kr > 0 ? kr : 0) + (int)threadIdx.x; r < a.k; r += kFT) po[r] = -1;
         return;
     }
     case SEL_DEC_MEMBER: {

@@ -110,9 +110,12 @@ __global__ void __launch_bounds__(kSimtThreads) score_simt_kernel(ScoreArgs a) {
             wsm[i] = (i / a.H) < bi.nrows ? a.w[(long long)bi.row0 * a.H + i] : 0.0f;
         if (a.sink == SINK_FILTER && warp < RB) sel_init(sel[warp], hist + warp * kBins);
         const int r = warp;
-        const bool row_ok = r < bi.nrows;
-        const int bound = row_ok ? key_bound(row_bound(bi.i0 + r, bi.n, a.g, a.db), a.kshift) : -1;
         const long long grow = (long long)bi.row0 + r;
+        // a filtered row whose members are all outside the call's output rows
+        // is not ranked (it has no scratch row)
+        const bool row_ok = r < bi.nrows && (a.sink != SINK_FILTER || scored_in_range(plan, grow));
+        const int bound = row_ok ? key_bound(row_bound(bi.i0 + r, bi.n, a.g, a.db), a.kshift) : -1;
+        const long long srow = grow - plan[6];  // scratch row
         int slot = -1;
         if (a.sink == SINK_SPILL && row_ok && a.slot_of_row) slot = a.slot_of_row[grow];
         for (int tile = 0; tile < bi.ntiles; ++tile) {
@@ -130,7 +133,7 @@ __global__ void __launch_bounds__(kSimtThreads) score_simt_kernel(ScoreArgs a) {
                     const int s = s0 + kb * 32 + (threadIdx.x & 31);
                     const bool valid = s <= bound;
                     if (a.sink == SINK_FILTER) {
-                        sel_offer(sel[r], hist + r * kBins, a.buf + grow * a.cap, a.cap, valid, sc[kb], s,
+                        sel_offer(sel[r], hist + r * kBins, a.buf + srow * a.cap, a.cap, valid, sc[kb], s,
                                   a.status);
                     } else if (slot >= 0 && valid) {
                         a.spill[(long long)slot * a.ld + s] = sc[kb];
@@ -138,11 +141,11 @@ __global__ void __launch_bounds__(kSimtThreads) score_simt_kernel(ScoreArgs a) {
                 }
             }
             if (a.sink == SINK_FILTER && row_ok)
-                sel_maintain(sel[r], hist + r * kBins, a.buf + grow * a.cap, a.cap, a.ksel, scr + warp * 256, KT);
+                sel_maintain(sel[r], hist + r * kBins, a.buf + srow * a.cap, a.cap, a.ksel, scr + warp * 256, KT);
         }
         if (a.sink == SINK_FILTER && row_ok && (threadIdx.x & 31) == 0) {
-            a.cnt[grow] = sel[r].cnt;
-            if (a.floor_out) a.floor_out[grow] = sel[r].floor;
+            a.cnt[srow] = sel[r].cnt;
+            if (a.floor_out) a.floor_out[srow] = sel[r].floor;
         }
     }
 }
@@ -208,7 +211,7 @@ __global__ void __launch_bounds__(kSimtThreads) gather_simt_kernel(GatherArgs a,
     __shared__ int s_pos[KT];
     const int HD = a.H * a.d;
     const int grp = blockIdx.x / mchunks, mc = blockIdx.x % mchunks;
-    long long mrow0, key0;
+    long long mrow0, key0, sgrp, orow0;
     int nmem;
     if (a.mode == 0) {
         if (!a.plan[0] || grp >= a.plan[2]) return;
@@ -224,12 +227,16 @@ __global__ void __launch_bounds__(kSimtThreads) gather_simt_kernel(GatherArgs a,
         mrow0 = (long long)a.cu[b] + lo + mc * RB;
         nmem = cnt - mc * RB;
         key0 = a.cu[b];
+        sgrp = (long long)grp - a.plan[6];   // scratch rows of the call
+        orow0 = mrow0 - a.plan[8];
     } else {
         const int kv = a.kv_len[grp];
         if (kv < a.G || kv > a.n_max) return;
         mrow0 = (long long)grp * a.G + mc * RB;
         nmem = a.G - mc * RB;
         key0 = (long long)grp * a.n_max;
+        sgrp = grp;
+        orow0 = mrow0;
     }
     if (nmem <= 0) return;
     if (nmem > RB) nmem = RB;
@@ -238,7 +245,7 @@ __global__ void __launch_bounds__(kSimtThreads) gather_simt_kernel(GatherArgs a,
     load_rows(qs, q, nmem, HD);
     for (int i = threadIdx.x; i < RB * a.H; i += blockDim.x)
         wsm[i] = (i / a.H) < nmem ? a.w[mrow0 * a.H + i] : 0.0f;
-    const int *cand = a.cand + (long long)grp * a.c;
+    const int *cand = a.cand + sgrp * a.c;
     const int r = threadIdx.x >> 5;
     for (int j0 = 0; j0 < a.c; j0 += KT) {
         __syncthreads();
@@ -255,7 +262,7 @@ __global__ void __launch_bounds__(kSimtThreads) gather_simt_kernel(GatherArgs a,
         if (r < nmem) {
             float sc[4];
             tile_scores(qs + r * HD, wsm + r * a.H, ks, a.H, a.d, sc);
-            float *out = a.out + (mrow0 + r) * a.c;
+            float *out = a.out + (orow0 + r) * a.c;
 #pragma unroll
             for (int kb = 0; kb < 4; ++kb) {
                 const int j = j0 + kb * 32 + (threadIdx.x & 31);

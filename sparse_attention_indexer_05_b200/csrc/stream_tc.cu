@@ -92,8 +92,10 @@ __device__ __forceinline__ Item item_info(const GatherArgs &g, const DecodeArgs 
         it.valid = true;
         it.m = m < 4 ? m : 4;
         it.qrow0 = m0 + mc * 4;
-        it.out_row0 = it.qrow0;
-        it.key0 = (long long)grp * g.c_pad;  // the group's block of packed candidate keys
+        // prefill scratch: member scores from the call's first member,
+        // packed keys from its first scored row
+        it.out_row0 = it.qrow0 - (g.mode == 0 ? g.plan[8] : 0);
+        it.key0 = ((long long)grp - (g.mode == 0 ? g.plan[6] : 0)) * g.c_pad;  // the group's packed keys
         it.t0 = 0;
         it.nt = g.c_pad / KT;
     } else {
@@ -363,10 +365,11 @@ __global__ void __launch_bounds__(256) compact_keys_kernel(GatherArgs a) {
         if (kv < a.G || kv > a.n_max) return;
         key0 = -1;  // decode: rows through cache_row
     }
-    const int *cand = a.cand + (long long)grp * a.c;
+    const long long sg = (long long)grp - (a.mode == 0 ? a.plan[6] : 0);  // the group's scratch row
+    const int *cand = a.cand + sg * a.c;
     const int per_row = a.d * 2 / 16;  // 16-byte chunks per key row
     const uint4 *src = reinterpret_cast<const uint4 *>(a.k);
-    uint4 *dst = reinterpret_cast<uint4 *>(a.ckeys) + ((long long)grp * a.c_pad + j0) * per_row;
+    uint4 *dst = reinterpret_cast<uint4 *>(a.ckeys) + (sg * a.c_pad + j0) * per_row;
     for (int u = threadIdx.x; u < KT * per_row; u += blockDim.x) {
         const int r = u / per_row, part = u - r * per_row;
         const int j = j0 + r;
@@ -445,7 +448,7 @@ cudaError_t launch_decode_tc(const DecodeArgs &a, cudaStream_t st) {
 
 cudaError_t launch_gather_tc(const GatherArgs &a, cudaStream_t st) {
     const long long qrows = a.mode == 0 ? (long long)a.cu_T : (long long)a.G * a.nitems;
-    const long long krows = (long long)a.nitems * a.c_pad;  // packed candidate keys
+    const long long krows = a.ckey_groups * a.c_pad;  // packed candidate keys
     CUtensorMap mq, mk;
     if (!map2d(&mq, a.q, (unsigned long long)qrows * S_H, 256) || !map2d(&mk, a.ckeys, (unsigned long long)krows, KT))
         return cudaErrorInvalidValue;

@@ -64,9 +64,10 @@ def _ws(workspace: Optional[torch.Tensor], need: int, device) -> torch.Tensor:
     return workspace
 
 
-def dense_workspace_size(T, H, d, topk, num_seqs, dtype=torch.bfloat16) -> int:
+def dense_workspace_size(T, H, d, topk, num_seqs, dtype=torch.bfloat16, max_rows=0) -> int:
+    """Workspace bytes; max_rows > 0: for calls whose rows= range spans at most max_rows rows."""
     dt = N.BF16 if dtype == torch.bfloat16 else N.F32
-    return int(N.lib().idx_dense_workspace_size(T, H, d, topk, num_seqs, dt))
+    return int(N.lib().idx_dense_workspace_size_rows(T, H, d, topk, num_seqs, dt, int(max_rows)))
 
 
 def adaptive_workspace_size(T, H, d, topk, rho, num_seqs, dtype=torch.bfloat16) -> int:
@@ -74,9 +75,12 @@ def adaptive_workspace_size(T, H, d, topk, rho, num_seqs, dtype=torch.bfloat16) 
     return int(N.lib().idx_adaptive_workspace_size(T, H, d, topk, rho, num_seqs, dt))
 
 
-def pivot_workspace_size(T, H, d, topk, num_seqs, g, c, mode, dtype=torch.bfloat16, dense_below=0) -> int:
+def pivot_workspace_size(T, H, d, topk, num_seqs, g, c, mode, dtype=torch.bfloat16, dense_below=0,
+                         max_rows=0) -> int:
+    """Workspace bytes; max_rows > 0: for calls whose rows= range spans at most max_rows rows."""
     dt = N.BF16 if dtype == torch.bfloat16 else N.F32
-    return int(N.lib().idx_pivot_workspace_size(T, H, d, topk, num_seqs, dt, g, c, _mode(mode), int(dense_below)))
+    return int(N.lib().idx_pivot_workspace_size_rows(T, H, d, topk, num_seqs, dt, g, c, _mode(mode),
+                                                     int(dense_below), int(max_rows)))
 
 
 def decode_workspace_size(B, G, n_max, H, d, topk, c, mode, dtype=torch.bfloat16) -> int:
@@ -99,9 +103,9 @@ def dense_topk(q, k, w, cu_seqlens, topk: int, out_idx=None, out_score=None, wor
     T, H, d = q.shape
     S = cu_seqlens.numel() - 1
     dt = _dtype_code(q)
-    ws = _ws(workspace, dense_workspace_size(T, H, d, topk, S, q.dtype), q.device)
-    out_idx, out_score = _outs((T,), topk, q.device, out_idx, out_score, return_scores)
     lo, hi = (0, T) if rows is None else (int(rows[0]), int(rows[1]))
+    ws = _ws(workspace, dense_workspace_size(T, H, d, topk, S, q.dtype, max(1, hi - lo)), q.device)
+    out_idx, out_score = _outs((T,), topk, q.device, out_idx, out_score, return_scores)
     N.check(N.lib().idx_dense_topk_rows(
         _dev(q, "q"), _dev(k, "k", q.dtype), _dev(w, "w", torch.float32), _dev(cu_seqlens, "cu_seqlens", torch.int32),
         S, T, H, d, topk, dt, lo, hi, _dev(out_idx, "out_idx", torch.int32),
@@ -147,9 +151,10 @@ def pivot_topk(q, k, w, cu_seqlens, topk: int, g: int, c: int, mode="refine", ou
     S = cu_seqlens.numel() - 1
     dt = _dtype_code(q)
     m = _mode(mode)
-    ws = _ws(workspace, pivot_workspace_size(T, H, d, topk, S, g, c, m, q.dtype, dense_below), q.device)
-    out_idx, out_score = _outs((T,), topk, q.device, out_idx, out_score, return_scores)
     lo, hi = (0, T) if rows is None else (int(rows[0]), int(rows[1]))
+    ws = _ws(workspace, pivot_workspace_size(T, H, d, topk, S, g, c, m, q.dtype, dense_below, max(1, hi - lo)),
+             q.device)
+    out_idx, out_score = _outs((T,), topk, q.device, out_idx, out_score, return_scores)
     N.check(N.lib().idx_pivot_topk_rows(
         _dev(q, "q"), _dev(k, "k", q.dtype), _dev(w, "w", torch.float32), _dev(cu_seqlens, "cu_seqlens", torch.int32),
         S, T, H, d, topk, dt, g, c, m, int(dense_below), lo, hi, _dev(out_idx, "out_idx", torch.int32),

@@ -26,7 +26,7 @@ def declared_functions():
 
 def test_exports_every_declared_symbol(lib):
     names = declared_functions()
-    assert len(names) == 23
+    assert len(names) == 25
     for n in names:
         assert hasattr(lib, n), n
         assert n in N.SIGNATURES, n
@@ -53,6 +53,14 @@ def test_workspace_sizes(lib):
     assert lib.idx_pivot_workspace_size(65536, 64, 128, 2048, 1, 0, 4, 4096, 2, 1 << 20) >= guard
     assert lib.idx_pivot_workspace_size(65536, 64, 128, 2048, 1, 0, 4, 4096, 2, -1) == 0  # negative threshold
     assert lib.idx_pivot_workspace_size(65536, 64, 128, 2048, 1, 0, 4, 4096, 3, 64) == 0  # block mode
+    # row-range calls: the per-row scratch covers the call's rows only
+    full = lib.idx_dense_workspace_size(131072, 64, 128, 2048, 1, 0)
+    assert lib.idx_dense_workspace_size_rows(131072, 64, 128, 2048, 1, 0, 0) == full
+    assert lib.idx_dense_workspace_size_rows(131072, 64, 128, 2048, 1, 0, 131072) == full
+    assert lib.idx_dense_workspace_size_rows(131072, 64, 128, 2048, 1, 0, 16384) < full / 7
+    assert lib.idx_dense_workspace_size_rows(131072, 64, 128, 2048, 1, 0, -1) == 0
+    pf = lib.idx_pivot_workspace_size(131072, 64, 128, 2048, 2, 0, 16, 4096, 2, 0)
+    assert lib.idx_pivot_workspace_size_rows(131072, 64, 128, 2048, 2, 0, 16, 4096, 2, 0, 16384) < pf / 5
     assert lib.idx_decode_workspace_size(64, 2, 131072, 64, 128, 2048, 4096, 2, 0) > 64 * 131072 * 4
     assert lib.idx_decode_workspace_size(64, 2, 1, 64, 128, 2048, 4096, 2, 0) == 0     # n_max < G
 

@@ -1,9 +1,12 @@
-"""One request split across ranks, on one GPU: the row-range entry points
-(idx_dense_topk_rows, idx_pivot_topk_rows) called once per range of every
-rank's zig-zag share must stitch together into exactly the full call's
-result, indices and scores bit for bit, and leave rows outside the range
-untouched.  The ranks run one after another here (independent calls, nothing
-waits on another rank), which is what each GPU of a split run does.
+"""Row-range calls (idx_dense_topk_rows, idx_pivot_topk_rows), on one GPU:
+  * one request split across ranks: the calls for every rank's zig-zag share
+    must stitch together into exactly the full call's result, indices and
+    scores bit for bit, and leave rows outside the range untouched.  The
+    ranks run one after another here (independent calls, nothing waits on
+    another rank), which is what each GPU of a split run does;
+  * a long prefill in row chunks with a workspace sized for one chunk
+    (*_workspace_size_rows): the same result, with the per-row scratch a
+    fraction of the full call's.
 """
 from __future__ import annotations
 
@@ -103,3 +106,47 @@ def test_bad_ranges_are_rejected(idx):
             idx.dense_topk(q, k, w, cu, 8, rows=rows)
         with pytest.raises(N.IdxError):
             idx.pivot_topk(q, k, w, cu, 8, 4, 16, "refine", rows=rows)
+
+
+@pytest.mark.parametrize("mode,g,db", [("dense", 1, 0), ("reuse", 4, 0), ("refine", 16, 0), ("refine", 4, 700)])
+def test_chunked_prefill_with_bounded_workspace(idx, mode, g, db):
+    topk, c, chunk = 64, 128, 750
+    P = W.prefill([3000, 333], H=64, d=128, topk=topk, rho=0.95, planted=0.01, seed=21)
+    q, k, w, cu = to_dev(P.q), to_dev(P.k), to_dev(P.w), to_dev(P.cu_seqlens)
+    T, S = P.T, 2
+    if mode == "dense":
+        full_ws = idx.dense_workspace_size(T, 64, 128, topk, S)
+        ws_size = idx.dense_workspace_size(T, 64, 128, topk, S, max_rows=chunk)
+        full_i, full_s = idx.dense_topk(q, k, w, cu, topk, return_scores=True)
+    else:
+        full_ws = idx.pivot_workspace_size(T, 64, 128, topk, S, g, c, mode, dense_below=db)
+        ws_size = idx.pivot_workspace_size(T, 64, 128, topk, S, g, c, mode, dense_below=db, max_rows=chunk)
+        full_i, full_s = idx.pivot_topk(q, k, w, cu, topk, g, c, mode, return_scores=True, dense_below=db)
+    assert ws_size < full_ws
+    ws = torch.empty(ws_size, dtype=torch.uint8, device="cuda")
+
+    def call(oi, os_, rows):
+        if mode == "dense":
+            idx.dense_topk(q, k, w, cu, topk, out_idx=oi, out_score=os_, rows=rows, workspace=ws)
+        else:
+            idx.pivot_topk(q, k, w, cu, topk, g, c, mode, out_idx=oi, out_score=os_, rows=rows, workspace=ws,
+                           dense_below=db)
+    # chunks that do not line up with groups or requests
+    ranges = [(lo, min(lo + chunk, T)) for lo in range(0, T, chunk)]
+    gi, gs = _stitch(call, T, topk, ranges)
+    assert np.array_equal(gi, full_i.cpu().numpy()), mode
+    assert np.array_equal(gs.view(np.uint32), full_s.cpu().numpy().view(np.uint32)), mode
+    # through the C ABI, a range longer than the workspace was sized for is
+    # refused (IDX_ERR_WORKSPACE) before anything runs
+    from sparse_attention_indexer_05_b200 import _native as N
+    oi = torch.empty(T, topk, dtype=torch.int32, device="cuda")
+    st = torch.cuda.current_stream().cuda_stream
+    if mode == "dense":
+        rc = N.lib().idx_dense_topk_rows(q.data_ptr(), k.data_ptr(), w.data_ptr(), cu.data_ptr(), S, T, 64, 128,
+                                         topk, N.BF16, 0, 2 * chunk, oi.data_ptr(), None, ws.data_ptr(), ws.numel(),
+                                         st)
+    else:
+        rc = N.lib().idx_pivot_topk_rows(q.data_ptr(), k.data_ptr(), w.data_ptr(), cu.data_ptr(), S, T, 64, 128,
+                                         topk, N.BF16, g, c, N.MODE_REUSE if mode == "reuse" else N.MODE_REFINE, db,
+                                         0, 2 * chunk, oi.data_ptr(), None, ws.data_ptr(), ws.numel(), st)
+    assert rc == 3, N.STATUS.get(rc, rc)
