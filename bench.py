@@ -69,7 +69,8 @@ def parse():
     p.add_argument("--skip-study", action="store_true",
                    help="CPU only: fraction of (row block, key tile) pairs a per-tile score bound could skip")
     p.add_argument("--dense-below", type=int, default=0,
-                   help="--crossover: also time PIVOT with this guardrail threshold (0 = without)")
+                   help="--crossover: also time PIVOT with this guardrail threshold (0 = without; -1 = the "
+                        "per-mode thresholds of GUARD_BELOW)")
     p.add_argument("--no-cpu", action="store_true", help="skip the CPU-oracle baseline")
     p.add_argument("--tokens", type=int, default=L_TOK,
                    help="batch length (profiling runs use a smaller case; the bench line uses 131072)")
@@ -370,6 +371,14 @@ def run_skip_study(args):
                       "after the first k keys", "topk": TOPK}))
     return 0
 
+# Guardrail thresholds (dense_below) for this build on B200, from the
+# crossover sweep (bench.py --crossover): the prefix length below which a
+# group's PIVOT work costs more than its members' dense work.  Reuse only pays
+# its fixed per-call costs at short lengths; Refine pays the candidate
+# select, the key pack and the re-score per member.
+GUARD_BELOW = {("reuse", 4): 4096, ("reuse", 16): 4096, ("refine", 4): 16384, ("refine", 16): 8192}
+
+
 def run_crossover(args):
     """Dense against PIVOT Reuse and Refine (c = 4096) on one request of
     L tokens, L = 1K .. 64K, g = 4 and 16: the inputs of the 65536-token
@@ -397,7 +406,8 @@ def run_crossover(args):
         del ws
         for g in (4, 16):
             for mode in ("reuse", "refine"):
-                for db in ((0, guard) if guard else (0,)):
+                gd = GUARD_BELOW[(mode, g)] if guard < 0 else guard
+                for db in ((0, gd) if gd else (0,)):
                     kw = {"dense_below": db} if db else {}
                     ws = torch.empty(idx.pivot_workspace_size(L, H, D, TOPK, 1, g, 4096, mode, **kw),
                                      dtype=torch.uint8, device=dev)

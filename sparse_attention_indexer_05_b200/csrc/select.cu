@@ -554,13 +554,33 @@ __device__ unsigned long long fast_kth(const Src &src, FastShared &sh, unsigned 
     return prefix;
 }
 
+// Copy n entries from shared memory to a row in global memory with 16-byte
+// accesses when both sides are 16-byte aligned.
+template <typename T>
+__device__ __forceinline__ void fast_copy_out(const T *src, T *dst, int n) {
+    if (((reinterpret_cast<uintptr_t>(dst) | reinterpret_cast<uintptr_t>(src)) & 15u) == 0) {
+        const int n4 = n >> 2;
+        const uint4 *s4 = reinterpret_cast<const uint4 *>(src);
+        uint4 *d4 = reinterpret_cast<uint4 *>(dst);
+        for (int i = threadIdx.x; i < n4; i += kFT) d4[i] = s4[i];
+        for (int i = (n4 << 2) + threadIdx.x; i < n; i += kFT) dst[i] = src[i];
+    } else {
+        for (int i = threadIdx.x; i < n; i += kFT) dst[i] = src[i];
+    }
+}
+
 // List the nonzero keys >= K of src in ascending position through a bitmap
 // (chunks of kChunkBits positions over 0..bound); returns how many.
 template <class Src>
 __device__ int fast_emit_bitmap(const Src &src, unsigned long long K, int bound, int k, int *out_idx,
-                                float *out_score, FastShared &sh, unsigned *bm) {
+                                float *out_score, FastShared &sh, unsigned *bm, unsigned *buf, int buf_words) {
     const int tid = threadIdx.x;
     int base = 0;
+    // the list is built in shared memory (buf: free stage room) and copied
+    // out with coalesced stores; without room it is written directly
+    const bool via_smem = buf_words >= (out_score ? 2 * k : k);
+    int *pi = via_smem ? reinterpret_cast<int *>(buf) : out_idx;
+    float *ps = via_smem ? reinterpret_cast<float *>(buf + k) : out_score;
     for (int c0 = 0; c0 <= bound; c0 += kChunkBits) {
         const int nwords = (bound - c0) / 32 + 1 < kChunkWords ? (bound - c0) / 32 + 1 : kChunkWords;
 #pragma unroll
@@ -599,7 +619,7 @@ __device__ int fast_emit_bitmap(const Src &src, unsigned long long K, int bound,
             while (x) {
                 const int bit = __ffs(x) - 1;
                 x &= x - 1u;
-                if (r < (unsigned)k) out_idx[r] = c0 + (w0 + j) * 32 + bit;  // never past the row
+                if (r < (unsigned)k) pi[r] = c0 + (w0 + j) * 32 + bit;  // never past the row
                 ++r;
             }
         }
@@ -613,7 +633,7 @@ __device__ int fast_emit_bitmap(const Src &src, unsigned long long K, int bound,
                         const int w = p >> 5, owner = w / kWordsPer;
                         unsigned rk = sh.tpre[owner] + __popc(bm[w] & ((1u << (p & 31)) - 1u));
                         for (int x = owner * kWordsPer; x < w; ++x) rk += __popc(bm[x]);
-                        if (base + (int)rk < k) out_score[base + rk] = ord_score(key_ord(kk));
+                        if (base + (int)rk < k) ps[base + rk] = ord_score(key_ord(kk));
                     }
                 }
             }
@@ -623,13 +643,19 @@ __device__ int fast_emit_bitmap(const Src &src, unsigned long long K, int bound,
         if (base > k) base = k;
         __syncthreads();  // the bitmap is cleared again by the next chunk
     }
+    if (via_smem) {
+        fast_copy_out(pi, out_idx, base);
+        if (out_score) fast_copy_out(ps, out_score, base);
+    }
     return base;
 }
 
 // Member rows: the staged entries are in candidate order (ascending
-// position); list the nonzero keys >= K in that order.
+// position); list the nonzero keys >= K in that order.  The list is built in
+// shared memory (`buf`, room for 2 * k words) and then copied out with
+// coalesced stores; without room it is written directly.
 __device__ int fast_emit_ordered(const unsigned long long *st, int n, unsigned long long K, int k, int *out_idx,
-                                 float *out_score, FastShared &sh) {
+                                 float *out_score, FastShared &sh, unsigned *buf, int buf_words) {
     const int tid = threadIdx.x;
     const int per = (n + kFT - 1) / kFT;
     const int i0 = tid * per, i1 = i0 + per < n ? i0 + per : n;
@@ -640,17 +666,26 @@ __device__ int fast_emit_ordered(const unsigned long long *st, int n, unsigned l
     }
     unsigned total;
     unsigned r = fast_excl_scan(cnt, sh.wtot, &total);
+    const bool via_smem = 2 * k <= buf_words;
+    int *pi = via_smem ? reinterpret_cast<int *>(buf) : out_idx;
+    float *ps = via_smem ? reinterpret_cast<float *>(buf + k) : out_score;
     for (int i = i0; i < i1; ++i) {
         const unsigned long long kk = st[i];
         if (kk != 0ull && kk >= K) {
             if (r < (unsigned)k) {  // never past the row
-                out_idx[r] = key_pos(kk);
-                if (out_score) out_score[r] = ord_score(key_ord(kk));
+                pi[r] = key_pos(kk);
+                if (out_score) ps[r] = ord_score(key_ord(kk));
             }
             ++r;
         }
     }
-    return (int)total < k ? (int)total : k;
+    const int nsel = (int)total < k ? (int)total : k;
+    if (via_smem) {
+        __syncthreads();
+        fast_copy_out(pi, out_idx, nsel);
+        if (out_score) fast_copy_out(ps, out_score, nsel);
+    }
+    return nsel;
 }
 
 __device__ __forceinline__ void fast_pad(int nsel, int k, int *out_idx, float *out_score) {
@@ -737,18 +772,23 @@ __device__ void fast_cand_row(const unsigned long long *buf, int n, unsigned flo
     const int ns = (int)sh.nstage;
     const unsigned hi = sh.maxord;
     int nsel;
+    // free stage room after the staged keys, from a 16-byte boundary
+    const int used = ((ns < stage_cap ? ns : stage_cap) + 1) & ~1;
+    unsigned *tail = reinterpret_cast<unsigned *>(stage + used);
+    const int tail_words = used < stage_cap ? 2 * (stage_cap - used) : 0;
     if (ns <= k) {
         const SStage s{stage, ns};
-        nsel = fast_emit_bitmap(s, 1ull, bound, k, out_idx, out_score, sh, bm);
+        nsel = fast_emit_bitmap(s, 1ull, bound, k, out_idx, out_score, sh, bm, tail, tail_words);
     } else if (ns <= stage_cap) {
         const SStage s{stage, ns};
         const unsigned long long K = fast_kth(s, sh, (unsigned)k, floor_ord, hi);
-        nsel = fast_emit_bitmap(s, K, bound, k, out_idx, out_score, sh, bm);
+        nsel = fast_emit_bitmap(s, K, bound, k, out_idx, out_score, sh, bm, tail, tail_words);
     } else {
         // more entries at or above the floor than the stage holds: the same
-        // steps over the row in global memory
+        // steps over the row in global memory (the whole stage is free)
         const unsigned long long K = fast_kth(g, sh, (unsigned)k, floor_ord, hi);
-        nsel = fast_emit_bitmap(g, K, bound, k, out_idx, out_score, sh, bm);
+        nsel = fast_emit_bitmap(g, K, bound, k, out_idx, out_score, sh, bm, reinterpret_cast<unsigned *>(stage),
+                                2 * stage_cap);
     }
     fast_pad(nsel, k, out_idx, out_score);
 }
@@ -769,14 +809,28 @@ __device__ void fast_member_row(const float *sc, const int *pos, int n, int boun
     __syncthreads();
     unsigned mx = 0u, mn = 0xFFFFFFFFu, cnt = 0;
     const bool staged = n <= stage_cap;
-    for (int i = tid; i < n; i += kFT) {
-        const unsigned long long kk = g.key(i);
-        if (staged) stage[i] = kk;
-        if (kk != 0ull) {
-            const unsigned o = key_ord(kk);
-            mx = o > mx ? o : mx;
-            mn = o < mn ? o : mn;
-            ++cnt;
+    // 8 entries per thread and round, every load issued before any is used
+    for (int base = 0; base < n; base += kFT * 8) {
+        int pv[8];
+        float sv[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            const int i = base + u * kFT + tid;
+            pv[u] = i < n ? (pos ? pos[i] : i) : -1;
+            sv[u] = i < n ? sc[i] : 0.0f;
+        }
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            const int i = base + u * kFT + tid;
+            const unsigned long long kk =
+                (pv[u] >= 0 && pv[u] <= bound) ? make_key(score_ord(sv[u]), pv[u]) : 0ull;
+            if (staged && i < n) stage[i] = kk;
+            if (kk != 0ull) {
+                const unsigned o = key_ord(kk);
+                mx = o > mx ? o : mx;
+                mn = o < mn ? o : mn;
+                ++cnt;
+            }
         }
     }
     mx = warp_max_u(mx);
@@ -796,10 +850,11 @@ __device__ void fast_member_row(const float *sc, const int *pos, int n, int boun
     if (staged) {
         const SStage s{stage, n};
         const unsigned long long K = nv <= (unsigned)k ? 1ull : fast_kth(s, sh, (unsigned)k, lo, hi);
-        nsel = fast_emit_ordered(stage, n, K, k, out_idx, out_score, sh);
+        nsel = fast_emit_ordered(stage, n, K, k, out_idx, out_score, sh, bm, kChunkWords);
     } else {
         const unsigned long long K = nv <= (unsigned)k ? 1ull : fast_kth(g, sh, (unsigned)k, lo, hi);
-        nsel = fast_emit_bitmap(g, K, bound, k, out_idx, out_score, sh, bm);
+        nsel = fast_emit_bitmap(g, K, bound, k, out_idx, out_score, sh, bm, reinterpret_cast<unsigned *>(stage),
+                                2 * stage_cap);
     }
     fast_pad(nsel, k, out_idx, out_score);
 }
