@@ -66,6 +66,9 @@ def parse():
                    help="skip the 16384-token dense and 65536-token PIVOT (g=4, c=4096) legs")
     p.add_argument("--crossover", action="store_true",
                    help="only time dense, Reuse and Refine on single requests of 1K..64K tokens (g=4, 16)")
+    p.add_argument("--split", action="store_true",
+                   help="N>1: split the one request across the ranks (zig-zag rows, strong scaling) instead of "
+                        "giving each rank its own batch; times the main step only")
     p.add_argument("--skip-study", action="store_true",
                    help="CPU only: fraction of (row block, key tile) pairs a per-tile score bound could skip")
     p.add_argument("--dense-below", type=int, default=0,
@@ -376,7 +379,7 @@ def run_skip_study(args):
 # group's PIVOT work costs more than its members' dense work.  Reuse only pays
 # its fixed per-call costs at short lengths; Refine pays the candidate
 # select, the key pack and the re-score per member.
-GUARD_BELOW = {("reuse", 4): 4096, ("reuse", 16): 4096, ("refine", 4): 16384, ("refine", 16): 8192}
+GUARD_BELOW = {("reuse", 4): 2048, ("reuse", 16): 2048, ("refine", 4): 24576, ("refine", 16): 12288}
 
 
 def run_crossover(args):

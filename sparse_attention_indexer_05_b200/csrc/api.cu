@@ -235,6 +235,7 @@ struct Prefill {
         a.buf = reinterpret_cast<unsigned long long *>(ws + L.buf);
         a.cap = L.cap;
         a.ksel = L.ksel;
+        a.ksel_dense = (unsigned)topk < L.ksel ? (unsigned)topk : L.ksel;
         a.cnt = reinterpret_cast<unsigned *>(ws + L.cnt);
         a.floor_out = reinterpret_cast<unsigned *>(ws + L.floor);
         a.status = status();
@@ -441,6 +442,17 @@ idx_status idx_pivot_topk_rows(const void *q, const void *k, const float *w, con
     if (refines(mode) && c < topk) return IDX_ERR_INVALID;
     if (mode == IDX_MODE_BLOCK && (c < kBlockN || c % kBlockN != 0)) return IDX_ERR_INVALID;
     if (mode == IDX_MODE_BLOCK && dense_below > 0) return IDX_ERR_UNSUPPORTED;
+    // every request is at most T tokens long: with dense_below >= T every
+    // group is short and the call is the dense call (the same rows, without
+    // the grouped pipeline's extra work)
+    if (g > 1 && dense_below >= T && T > 0) {
+        if (!ws || ws_bytes < idx_pivot_workspace_size_rows(T, H, d, topk, num_seqs, dtype, g,
+                                                             mode == IDX_MODE_REUSE ? topk : c, mode, dense_below,
+                                                             row_hi - row_lo > 0 ? row_hi - row_lo : 1))
+            return IDX_ERR_WORKSPACE;
+        return idx_dense_topk_rows(q, k, w, cu_seqlens, num_seqs, T, H, d, topk, dtype, row_lo, row_hi, out_idx,
+                                   out_score, ws, ws_bytes, stream);
+    }
     if (mode == IDX_MODE_REUSE) c = topk;
     const int m = row_hi - row_lo > 0 ? row_hi - row_lo : 1;
     const size_t need = idx_pivot_workspace_size_rows(T, H, d, topk, num_seqs, dtype, g, c, mode, dense_below, m);

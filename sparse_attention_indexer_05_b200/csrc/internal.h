@@ -62,6 +62,7 @@ struct ScoreArgs {
     // SINK_FILTER: candidate buffers [R, cap] and counts [R]
     unsigned long long *buf;
     unsigned cap, ksel;
+    unsigned ksel_dense;  // guardrail: rows of short-group members keep their top-k only
     unsigned *cnt;
     unsigned *floor_out;  // per row: keys with a lower ord cannot be selected
     // SINK_SPILL: out[slot * ld + s] for rows with slot_of_row[row] >= 0

@@ -288,7 +288,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (filter && ((j % kMaintEvery) == kMaintEvery - 1 || j == ntiles - 1)) {
                     tc::named_bar_sync(1 + role, 128);
                     if (maint)
-                        sel_maintain(sh.sel[mrow], hist + mrow * kBins, buf0 + (long long)mrow * a.cap, a.cap, a.ksel,
+                        sel_maintain(sh.sel[mrow], hist + mrow * kBins, buf0 + (long long)mrow * a.cap, a.cap,
+                                     bi.i0 + mrow < dense_rows(bi.n, a.g, a.db) ? a.ksel_dense : a.ksel,
                                      scr + mrow * 256, KT * kMaintEvery);
                     tc::named_bar_sync(1 + role, 128);
                 }

@@ -911,10 +911,8 @@ __global__ void __launch_bounds__(kFT, 4) select_fast_kernel(SelectArgs a) {
         const int n = a.cu[b + 1] - a.cu[b];
         int *po = a.out_idx + ((long long)row - p0) * a.k;
         if (a.kind == SEL_PROXY_TO_C) {
-            if (i < dense_rows(n, a.g, a.db)) {  // a member scored on its own needs no candidate set
-                fast_pad(0, a.k, po, nullptr);
-                return;
-            }
+            // a member scored on its own needs no candidate set (nothing reads its row)
+            if (i < dense_rows(n, a.g, a.db)) return;
             oi = po;
             os = nullptr;
             cand(row, row_bound(i, n, a.g, a.db), a.k);

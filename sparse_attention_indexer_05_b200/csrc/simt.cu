@@ -141,7 +141,8 @@ __global__ void __launch_bounds__(kSimtThreads) score_simt_kernel(ScoreArgs a) {
                 }
             }
             if (a.sink == SINK_FILTER && row_ok)
-                sel_maintain(sel[r], hist + r * kBins, a.buf + srow * a.cap, a.cap, a.ksel, scr + warp * 256, KT);
+                sel_maintain(sel[r], hist + r * kBins, a.buf + srow * a.cap, a.cap,
+                             bi.i0 + r < dense_rows(bi.n, a.g, a.db) ? a.ksel_dense : a.ksel, scr + warp * 256, KT);
         }
         if (a.sink == SINK_FILTER && row_ok && (threadIdx.x & 31) == 0) {
             a.cnt[srow] = sel[r].cnt;
