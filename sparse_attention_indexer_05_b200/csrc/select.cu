@@ -442,7 +442,6 @@ constexpr int kWordsPer = kChunkWords / kFT;      // 16 words per thread
 struct __align__(16) FastShared {
     unsigned hist[2][256];
     unsigned wtot[kFWarps];
-    unsigned tpre[kFT];
     unsigned nstage;
     unsigned maxord;
     unsigned minord;
@@ -573,7 +572,8 @@ __device__ __forceinline__ void fast_copy_out(const T *src, T *dst, int n) {
 // (chunks of kChunkBits positions over 0..bound); returns how many.
 template <class Src>
 __device__ int fast_emit_bitmap(const Src &src, unsigned long long K, int bound, int k, int *out_idx,
-                                float *out_score, FastShared &sh, unsigned *bm, unsigned *buf, int buf_words) {
+                                float *out_score, FastShared &sh, unsigned *bm, unsigned *buf, int buf_words,
+                                unsigned *wpre, bool bm_clear = false) {
     const int tid = threadIdx.x;
     int base = 0;
     // the list is built in shared memory (buf: free stage room) and copied
@@ -583,9 +583,11 @@ __device__ int fast_emit_bitmap(const Src &src, unsigned long long K, int bound,
     float *ps = via_smem ? reinterpret_cast<float *>(buf + k) : out_score;
     for (int c0 = 0; c0 <= bound; c0 += kChunkBits) {
         const int nwords = (bound - c0) / 32 + 1 < kChunkWords ? (bound - c0) / 32 + 1 : kChunkWords;
+        if (!(bm_clear && c0 == 0)) {  // the caller may have cleared it for the first chunk
 #pragma unroll
-        for (int j = 0; j < kWordsPer; ++j) bm[tid * kWordsPer + j] = 0u;
-        __syncthreads();
+            for (int j = 0; j < kWordsPer; ++j) bm[tid * kWordsPer + j] = 0u;
+            __syncthreads();
+        }
         for (int i = tid; i < src.n; i += kFT) {
             const unsigned long long kk = src.key(i);
             if (kk != 0ull && kk >= K) {
@@ -594,45 +596,55 @@ __device__ int fast_emit_bitmap(const Src &src, unsigned long long K, int bound,
             }
         }
         __syncthreads();
-        // thread tid owns words [tid * kWordsPer, +kWordsPer)
-        const int w0 = tid * kWordsPer;
-        unsigned words[kWordsPer];
+        // warp w owns words [w * kWordsW, +kWordsW) and walks them 32 at a
+        // time (lane i reads word base + i: conflict-free); a warp prefix of
+        // the words' bit counts places each word's positions, in order
+        constexpr int kWordsW = kChunkWords / kFWarps;  // 512
+        const int lane = tid & 31, warp = tid >> 5;
+        const int wb = warp * kWordsW;
         unsigned cnt = 0;
-        const uint4 *b4 = reinterpret_cast<const uint4 *>(bm + w0);
+#pragma unroll 4
+        for (int j = 0; j < kWordsW; j += 32) cnt += __popc(bm[wb + j + lane]);
+        cnt = __reduce_add_sync(0xFFFFFFFFu, cnt);
+        if (lane == 0) sh.wtot[warp] = cnt;
+        __syncthreads();
+        unsigned before = 0, total = 0;
 #pragma unroll
-        for (int j = 0; j < kWordsPer / 4; ++j) {
-            const uint4 v = b4[j];
-            words[4 * j + 0] = v.x;
-            words[4 * j + 1] = v.y;
-            words[4 * j + 2] = v.z;
-            words[4 * j + 3] = v.w;
+        for (int w = 0; w < kFWarps; ++w) {
+            const unsigned t = sh.wtot[w];
+            before += w < warp ? t : 0u;
+            total += t;
         }
+        unsigned r = base + before;
+        for (int j = 0; j < kWordsW; j += 32) {
+            const int w = wb + j + lane;
+            unsigned x = bm[w];
+            const unsigned c = __popc(x);
+            unsigned inc = c;  // inclusive warp prefix of the words' counts
 #pragma unroll
-        for (int j = 0; j < kWordsPer; ++j) cnt += __popc(words[j]);
-        unsigned total;
-        const unsigned pre = fast_excl_scan(cnt, sh.wtot, &total);
-        sh.tpre[tid] = pre;
-        unsigned r = base + pre;
-#pragma unroll
-        for (int j = 0; j < kWordsPer; ++j) {
-            unsigned x = words[j];
+            for (int o = 1; o < 32; o <<= 1) {
+                const unsigned v = __shfl_up_sync(0xFFFFFFFFu, inc, o);
+                if (lane >= o) inc += v;
+            }
+            unsigned at = r + inc - c;
+            if (wpre) wpre[w] = at - base;  // chunk-local rank of the word's first bit
             while (x) {
                 const int bit = __ffs(x) - 1;
                 x &= x - 1u;
-                if (r < (unsigned)k) pi[r] = c0 + (w0 + j) * 32 + bit;  // never past the row
-                ++r;
+                if (at < (unsigned)k) pi[at] = c0 + w * 32 + bit;  // never past the row
+                ++at;
             }
+            r += __shfl_sync(0xFFFFFFFFu, inc, 31);
         }
         if (out_score) {
-            __syncthreads();  // tpre complete
+            __syncthreads();  // every word's rank is recorded; the bitmap is intact
             for (int i = tid; i < src.n; i += kFT) {
                 const unsigned long long kk = src.key(i);
                 if (kk != 0ull && kk >= K) {
                     const int p = key_pos(kk) - c0;
                     if (p >= 0 && p < kChunkBits) {
-                        const int w = p >> 5, owner = w / kWordsPer;
-                        unsigned rk = sh.tpre[owner] + __popc(bm[w] & ((1u << (p & 31)) - 1u));
-                        for (int x = owner * kWordsPer; x < w; ++x) rk += __popc(bm[x]);
+                        const int w = p >> 5;
+                        const unsigned rk = wpre[w] + __popc(bm[w] & ((1u << (p & 31)) - 1u));
                         if (base + (int)rk < k) ps[base + rk] = ord_score(key_ord(kk));
                     }
                 }
@@ -651,33 +663,50 @@ __device__ int fast_emit_bitmap(const Src &src, unsigned long long K, int bound,
 }
 
 // Member rows: the staged entries are in candidate order (ascending
-// position); list the nonzero keys >= K in that order.  The list is built in
-// shared memory (`buf`, room for 2 * k words) and then copied out with
-// coalesced stores; without room it is written directly.
+// position); list the nonzero keys >= K in that order.  Warp w owns a
+// contiguous segment of the stage and walks it 32 entries at a time (lane i
+// reads entry base + i: conflict-free), placing its selected entries by a
+// ballot prefix; a block scan of the warps' counts gives each segment's
+// offset.  The list is built in shared memory (`buf`, room for 2 * k words)
+// and then copied out with coalesced stores; without room it is written
+// directly.
 __device__ int fast_emit_ordered(const unsigned long long *st, int n, unsigned long long K, int k, int *out_idx,
                                  float *out_score, FastShared &sh, unsigned *buf, int buf_words) {
-    const int tid = threadIdx.x;
-    const int per = (n + kFT - 1) / kFT;
-    const int i0 = tid * per, i1 = i0 + per < n ? i0 + per : n;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int seg = ((n + kFWarps - 1) / kFWarps + 31) & ~31;
+    const int i0 = warp * seg, i1 = i0 + seg < n ? i0 + seg : n;
     unsigned cnt = 0;
-    for (int i = i0; i < i1; ++i) {
-        const unsigned long long kk = st[i];
-        cnt += (kk != 0ull && kk >= K) ? 1u : 0u;
+    for (int b = i0; b < i1; b += 32) {
+        const int i = b + lane;
+        const unsigned long long kk = i < i1 ? st[i] : 0ull;
+        cnt += __popc(__ballot_sync(0xFFFFFFFFu, kk != 0ull && kk >= K));
     }
-    unsigned total;
-    unsigned r = fast_excl_scan(cnt, sh.wtot, &total);
+    // exclusive prefix over warps (lane 0 holds each warp's count)
+    if (lane == 0) sh.wtot[warp] = cnt;
+    __syncthreads();
+    unsigned before = 0, total = 0;
+#pragma unroll
+    for (int w = 0; w < kFWarps; ++w) {
+        const unsigned t = sh.wtot[w];
+        before += w < warp ? t : 0u;
+        total += t;
+    }
+    __syncthreads();  // wtot may be reused right after
     const bool via_smem = 2 * k <= buf_words;
     int *pi = via_smem ? reinterpret_cast<int *>(buf) : out_idx;
     float *ps = via_smem ? reinterpret_cast<float *>(buf + k) : out_score;
-    for (int i = i0; i < i1; ++i) {
-        const unsigned long long kk = st[i];
-        if (kk != 0ull && kk >= K) {
-            if (r < (unsigned)k) {  // never past the row
-                pi[r] = key_pos(kk);
-                if (out_score) ps[r] = ord_score(key_ord(kk));
-            }
-            ++r;
+    unsigned r = before;
+    for (int b = i0; b < i1; b += 32) {
+        const int i = b + lane;
+        const unsigned long long kk = i < i1 ? st[i] : 0ull;
+        const bool sel = kk != 0ull && kk >= K;
+        const unsigned m = __ballot_sync(0xFFFFFFFFu, sel);
+        const unsigned at = r + __popc(m & lanemask_lt());
+        if (sel && at < (unsigned)k) {  // never past the row
+            pi[at] = key_pos(kk);
+            if (out_score) ps[at] = ord_score(key_ord(kk));
         }
+        r += __popc(m);
     }
     const int nsel = (int)total < k ? (int)total : k;
     if (via_smem) {
@@ -715,7 +744,7 @@ __device__ __forceinline__ unsigned warp_min_u(unsigned v) {
 // Top-k of a candidate row (keys at or above `floor_ord`, positions <= bound).
 __device__ void fast_cand_row(const unsigned long long *buf, int n, unsigned floor_ord, int bound, int k,
                               int *out_idx, float *out_score, FastShared &sh, unsigned long long *stage,
-                              int stage_cap, unsigned *bm) {
+                              int stage_cap, unsigned *bm, unsigned *wpre) {
     const int tid = threadIdx.x, lane = tid & 31;
     const GCand g{buf, n, (unsigned long long)floor_ord << 32, 0xFFFFFFFFu - (unsigned)bound};
     if (tid == 0) {
@@ -724,6 +753,9 @@ __device__ void fast_cand_row(const unsigned long long *buf, int n, unsigned flo
     }
     sh.hist[0][tid] = 0u;
     __syncthreads();
+    // the emit's bitmap, cleared here (ordered before it by the barrier below)
+#pragma unroll
+    for (int j = 0; j < kWordsPer; ++j) bm[tid * kWordsPer + j] = 0u;
     unsigned mx = 0u;
     // 8 keys per thread and round, as four 16-byte loads (rows start 2 KB aligned)
     const ulonglong2 *b2 = reinterpret_cast<const ulonglong2 *>(buf);
@@ -778,17 +810,17 @@ __device__ void fast_cand_row(const unsigned long long *buf, int n, unsigned flo
     const int tail_words = used < stage_cap ? 2 * (stage_cap - used) : 0;
     if (ns <= k) {
         const SStage s{stage, ns};
-        nsel = fast_emit_bitmap(s, 1ull, bound, k, out_idx, out_score, sh, bm, tail, tail_words);
+        nsel = fast_emit_bitmap(s, 1ull, bound, k, out_idx, out_score, sh, bm, tail, tail_words, wpre, true);
     } else if (ns <= stage_cap) {
         const SStage s{stage, ns};
         const unsigned long long K = fast_kth(s, sh, (unsigned)k, floor_ord, hi);
-        nsel = fast_emit_bitmap(s, K, bound, k, out_idx, out_score, sh, bm, tail, tail_words);
+        nsel = fast_emit_bitmap(s, K, bound, k, out_idx, out_score, sh, bm, tail, tail_words, wpre, true);
     } else {
         // more entries at or above the floor than the stage holds: the same
         // steps over the row in global memory (the whole stage is free)
         const unsigned long long K = fast_kth(g, sh, (unsigned)k, floor_ord, hi);
         nsel = fast_emit_bitmap(g, K, bound, k, out_idx, out_score, sh, bm, reinterpret_cast<unsigned *>(stage),
-                                2 * stage_cap);
+                                2 * stage_cap, wpre);
     }
     fast_pad(nsel, k, out_idx, out_score);
 }
@@ -797,7 +829,7 @@ __device__ void fast_cand_row(const unsigned long long *buf, int n, unsigned flo
 // -1 = none), masked to positions <= bound.
 __device__ void fast_member_row(const float *sc, const int *pos, int n, int bound, int k, int *out_idx,
                                 float *out_score, FastShared &sh, unsigned long long *stage, int stage_cap,
-                                unsigned *bm) {
+                                unsigned *bm, unsigned *wpre) {
     const int tid = threadIdx.x, lane = tid & 31;
     const GScore g{sc, pos, n, bound};
     if (tid == 0) {
@@ -854,7 +886,7 @@ __device__ void fast_member_row(const float *sc, const int *pos, int n, int boun
     } else {
         const unsigned long long K = nv <= (unsigned)k ? 1ull : fast_kth(g, sh, (unsigned)k, lo, hi);
         nsel = fast_emit_bitmap(g, K, bound, k, out_idx, out_score, sh, bm, reinterpret_cast<unsigned *>(stage),
-                                2 * stage_cap);
+                                2 * stage_cap, wpre);
     }
     fast_pad(nsel, k, out_idx, out_score);
 }
@@ -866,6 +898,8 @@ __global__ void __launch_bounds__(kFT, 4) select_fast_kernel(SelectArgs a) {
     unsigned *bm = reinterpret_cast<unsigned *>(fast_smem);
     unsigned long long *stage = fast_smem + kChunkWords / 2;
     const int scap = a.stage_cap;
+    // per-word ranks of the bitmap walk, for the scores (when they are output)
+    unsigned *wpre = a.out_score ? reinterpret_cast<unsigned *>(stage + scap) : nullptr;
     int *oi = a.out_idx + (long long)row * a.k;
     float *os = a.out_score ? a.out_score + (long long)row * a.k : nullptr;
     // per-row scratch of prefill calls starts at the call's first scored row
@@ -875,7 +909,7 @@ __global__ void __launch_bounds__(kFT, 4) select_fast_kernel(SelectArgs a) {
         const long long sr = r - p0;
         const unsigned n = a.cnt[sr];
         fast_cand_row(a.buf + sr * a.cap, (int)(n < a.cap ? n : a.cap), a.floor ? a.floor[sr] : 0u, bound, k, oi, os,
-                      sh, stage, scap, bm);
+                      sh, stage, scap, bm, os ? wpre : nullptr);
     };
     switch (a.kind) {
     case SEL_DENSE_CAND:
@@ -896,7 +930,7 @@ __global__ void __launch_bounds__(kFT, 4) select_fast_kernel(SelectArgs a) {
                 cand(p, t, a.k);
             else
                 fast_member_row(a.scores + ((long long)row - a.plan[8]) * a.ld, a.cand + (p - p0) * a.c, a.c, t,
-                                a.k, oi, os, sh, stage, scap, bm);
+                                a.k, oi, os, sh, stage, scap, bm, os ? wpre : nullptr);
         }
         return;
     }
@@ -938,7 +972,7 @@ __global__ void __launch_bounds__(kFT, 4) select_fast_kernel(SelectArgs a) {
             return;
         }
         fast_member_row(a.scores + (long long)row * a.ld, a.cand + (long long)b * a.c, a.c, kv - a.G + m, a.k, oi,
-                        os, sh, stage, scap, bm);
+                        os, sh, stage, scap, bm, os ? wpre : nullptr);
         return;
     }
     default:
@@ -960,14 +994,16 @@ bool fast_kind(int kind) {
 cudaError_t launch_select_fast(const SelectArgs &a, cudaStream_t st) {
     SelectArgs b = a;
     const bool member = a.kind == SEL_MEMBER_SCORES || a.kind == SEL_DEC_MEMBER;
-    long long room = 2LL * a.k;
+    // candidate rows stage about 1.2 k keys (at most 1.7 k measured): 1.5 k + 512
+    long long room = a.k + a.k / 2 + 512;
     if (member && a.c > room) room = a.c;
     if (room < kFastMinRoom) room = kFastMinRoom;
     room = (room + 255) / 256 * 256;
-    const size_t limit = 232448 - sizeof(FastShared) - 1024 - (size_t)kChunkWords * 4;
-    if ((size_t)room * 8 > limit) room = (long long)(limit / 8);
+    const size_t wpre_bytes = a.out_score ? (size_t)kChunkWords * 4 : 0;  // per-word ranks
+    const size_t limit = 232448 - sizeof(FastShared) - 1024 - (size_t)kChunkWords * 4 - wpre_bytes;
+    if ((size_t)room * 8 > limit) room = (long long)(limit / 8) & ~1LL;
     b.stage_cap = (int)room;
-    const size_t smem = (size_t)kChunkWords * 4 + (size_t)room * 8;
+    const size_t smem = (size_t)kChunkWords * 4 + (size_t)room * 8 + wpre_bytes;
     cudaError_t e = cudaFuncSetAttribute(select_fast_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     TraceScope ts("select", st);
