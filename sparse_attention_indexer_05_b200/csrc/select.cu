@@ -437,7 +437,6 @@ constexpr int kFT = 256;                          // threads of select_fast_kern
 constexpr int kFWarps = kFT / 32;
 constexpr int kChunkBits = 1 << 17;               // positions per bitmap chunk
 constexpr int kChunkWords = kChunkBits / 32;      // 4096 words = 16 KB
-constexpr int kWordsPer = kChunkWords / kFT;      // 16 words per thread
 
 struct __align__(16) FastShared {
     unsigned hist[2][256];
@@ -583,9 +582,11 @@ __device__ int fast_emit_bitmap(const Src &src, unsigned long long K, int bound,
     float *ps = via_smem ? reinterpret_cast<float *>(buf + k) : out_score;
     for (int c0 = 0; c0 <= bound; c0 += kChunkBits) {
         const int nwords = (bound - c0) / 32 + 1 < kChunkWords ? (bound - c0) / 32 + 1 : kChunkWords;
+        // words walked: the chunk's positions up to bound, a multiple of
+        // 32 per warp (per warp: kWordsW of them)
+        const int kWordsW = ((nwords + kFWarps * 32 - 1) / (kFWarps * 32)) * 32;
         if (!(bm_clear && c0 == 0)) {  // the caller may have cleared it for the first chunk
-#pragma unroll
-            for (int j = 0; j < kWordsPer; ++j) bm[tid * kWordsPer + j] = 0u;
+            for (int j = tid; j < kFWarps * kWordsW; j += kFT) bm[j] = 0u;
             __syncthreads();
         }
         for (int i = tid; i < src.n; i += kFT) {
@@ -599,7 +600,6 @@ __device__ int fast_emit_bitmap(const Src &src, unsigned long long K, int bound,
         // warp w owns words [w * kWordsW, +kWordsW) and walks them 32 at a
         // time (lane i reads word base + i: conflict-free); a warp prefix of
         // the words' bit counts places each word's positions, in order
-        constexpr int kWordsW = kChunkWords / kFWarps;  // 512
         const int lane = tid & 31, warp = tid >> 5;
         const int wb = warp * kWordsW;
         unsigned cnt = 0;
@@ -650,7 +650,6 @@ __device__ int fast_emit_bitmap(const Src &src, unsigned long long K, int bound,
                 }
             }
         }
-        (void)nwords;
         base += (int)total;
         if (base > k) base = k;
         __syncthreads();  // the bitmap is cleared again by the next chunk
@@ -753,9 +752,13 @@ __device__ void fast_cand_row(const unsigned long long *buf, int n, unsigned flo
     }
     sh.hist[0][tid] = 0u;
     __syncthreads();
-    // the emit's bitmap, cleared here (ordered before it by the barrier below)
-#pragma unroll
-    for (int j = 0; j < kWordsPer; ++j) bm[tid * kWordsPer + j] = 0u;
+    // the emit's bitmap (first chunk, the words the walk reads), cleared here
+    // (ordered before it by the barrier below)
+    {
+        const int nw = bound / 32 + 1 < kChunkWords ? bound / 32 + 1 : kChunkWords;
+        const int nclr = ((nw + kFWarps * 32 - 1) / (kFWarps * 32)) * 32 * kFWarps;
+        for (int j = tid; j < nclr; j += kFT) bm[j] = 0u;
+    }
     unsigned mx = 0u;
     // 8 keys per thread and round, as four 16-byte loads (rows start 2 KB aligned)
     const ulonglong2 *b2 = reinterpret_cast<const ulonglong2 *>(buf);
