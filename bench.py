@@ -379,7 +379,7 @@ def run_skip_study(args):
 # group's PIVOT work costs more than its members' dense work.  Reuse only pays
 # its fixed per-call costs at short lengths; Refine pays the candidate
 # select, the key pack and the re-score per member.
-GUARD_BELOW = {("reuse", 4): 2048, ("reuse", 16): 2048, ("refine", 4): 24576, ("refine", 16): 8192}
+GUARD_BELOW = {("reuse", 4): 2048, ("reuse", 16): 2048, ("refine", 4): 24576, ("refine", 16): 16384}
 
 
 def run_crossover(args):
