@@ -502,20 +502,16 @@ struct SStage {
     __device__ __forceinline__ unsigned long long key(int i) const { return st[i]; }
 };
 
-// Exact k-th largest nonzero key of src (more than `need` nonzero keys,
-// all with ords in [lo_ord, hi_ord]).  MSB-first radix with 8-bit digits
-// from the first bit where lo_ord and hi_ord differ; sh.hist[0] is clear
-// on entry (and sh.hist[1] is cleared here).
+// MSB-first radix with 8-bit digits below a known prefix: the `need`-th
+// largest of the nonzero keys of src matching `prefix` under `mask`, the
+// digits below bit `shift`.  Pass p builds its histogram in sh.hist[p & 1],
+// which is clear on entry (p = p0), and clears the other one for the next
+// pass.  Returns the key K with exactly `need` matching keys >= K (plus the
+// keys above the prefix the caller already counted).
 template <class Src>
-__device__ unsigned long long fast_kth(const Src &src, FastShared &sh, unsigned need, unsigned lo_ord,
-                                       unsigned hi_ord) {
+__device__ unsigned long long fast_kth_run(const Src &src, FastShared &sh, unsigned need,
+                                           unsigned long long prefix, unsigned long long mask, int shift, int p) {
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const unsigned diff = lo_ord ^ hi_ord;
-    const int lead = diff ? __clz(diff) : 32;  // leading ord bits every key shares
-    int shift = 64 - lead;
-    unsigned long long mask = lead ? (~0ull << (64 - lead)) : 0ull;
-    unsigned long long prefix = ((unsigned long long)hi_ord << 32) & mask;
-    int p = 0;
     while (shift > 0) {
         const int bits = shift >= 8 ? 8 : shift;
         shift -= bits;
@@ -550,6 +546,38 @@ __device__ unsigned long long fast_kth(const Src &src, FastShared &sh, unsigned 
     sh.hist[0][tid] = 0u;
     __syncthreads();
     return prefix;
+}
+
+// Exact k-th largest nonzero key of src (more than `need` nonzero keys,
+// all with ords in [lo_ord, hi_ord]): the radix from the first bit where
+// lo_ord and hi_ord differ; sh.hist[0] is clear on entry (and sh.hist[1] is
+// cleared here).
+template <class Src>
+__device__ unsigned long long fast_kth(const Src &src, FastShared &sh, unsigned need, unsigned lo_ord,
+                                       unsigned hi_ord) {
+    const unsigned diff = lo_ord ^ hi_ord;
+    const int lead = diff ? __clz(diff) : 32;  // leading ord bits every key shares
+    const unsigned long long mask = lead ? (~0ull << (64 - lead)) : 0ull;
+    const unsigned long long prefix = ((unsigned long long)hi_ord << 32) & mask;
+    return fast_kth_run(src, sh, need, prefix, mask, 64 - lead, 0);
+}
+
+// Keys staged in shared memory, read relative to a floor ord: key - floor << 32
+// (all staged keys have ord >= floor; the result is never 0).
+struct SStageOff {
+    const unsigned long long *st;
+    int n;
+    unsigned long long base;
+    __device__ __forceinline__ unsigned long long key(int i) const { return st[i] - base; }
+};
+
+// First digit of a staged candidate key, built while staging: its ord above
+// the floor in 1/128-octave steps (2^16 ord units; the scores near the k-th
+// of these rows put about a hundred keys in a step), 255 = that far or more.
+constexpr int kFirstShift = 16;
+__device__ __forceinline__ unsigned first_digit(unsigned ord, unsigned floor_ord) {
+    const unsigned x = (ord - floor_ord) >> kFirstShift;
+    return x < 255u ? x : 255u;
 }
 
 // Copy n entries from shared memory to a row in global memory with 16-byte
@@ -744,13 +772,14 @@ __device__ __forceinline__ unsigned warp_min_u(unsigned v) {
 __device__ void fast_cand_row(const unsigned long long *buf, int n, unsigned floor_ord, int bound, int k,
                               int *out_idx, float *out_score, FastShared &sh, unsigned long long *stage,
                               int stage_cap, unsigned *bm, unsigned *wpre) {
-    const int tid = threadIdx.x, lane = tid & 31;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const GCand g{buf, n, (unsigned long long)floor_ord << 32, 0xFFFFFFFFu - (unsigned)bound};
     if (tid == 0) {
         sh.nstage = 0u;
         sh.maxord = 0u;
     }
     sh.hist[0][tid] = 0u;
+    sh.hist[1][tid] = 0u;
     __syncthreads();
     // the emit's bitmap (first chunk, the words the walk reads), cleared here
     // (ordered before it by the barrier below)
@@ -797,6 +826,8 @@ __device__ void fast_cand_row(const unsigned long long *buf, int n, unsigned flo
                 if (kv[u] != 0ull) {
                     if (b < (unsigned)stage_cap) stage[b] = kv[u];
                     ++b;
+                    // the radix's first digit, counted here
+                    atomicAdd(&sh.hist[0][first_digit(key_ord(kv[u]), floor_ord)], 1u);
                 }
             }
         }
@@ -816,11 +847,43 @@ __device__ void fast_cand_row(const unsigned long long *buf, int n, unsigned flo
         nsel = fast_emit_bitmap(s, 1ull, bound, k, out_idx, out_score, sh, bm, tail, tail_words, wpre, true);
     } else if (ns <= stage_cap) {
         const SStage s{stage, ns};
-        const unsigned long long K = fast_kth(s, sh, (unsigned)k, floor_ord, hi);
+        // the first digit's histogram is in hist[0]: find its bin, then refine
+        // inside it relative to the floor (keys - floor << 32)
+        if (warp == 0) {
+            unsigned above;
+            const int b = warp_find_bin(sh.hist[0], (unsigned)k, &above);
+            if (lane == 0) {
+                sh.dgt = b;
+                sh.above = above;
+                sh.inbin = b >= 0 ? sh.hist[0][b] : 0u;
+            }
+        }
+        __syncthreads();
+        const int b1 = sh.dgt;
+        const unsigned above1 = sh.above, inbin1 = sh.inbin;
+        const unsigned long long fl = (unsigned long long)floor_ord << 32;
+        const unsigned long long edge = (unsigned long long)floor_ord + ((unsigned long long)(b1 > 0 ? b1 : 0) << kFirstShift);
+        unsigned long long K;
+        if (b1 >= 0 && inbin1 == (unsigned)k - above1 && edge <= 0xFFFFFFFFull) {
+            K = edge << 32;  // everything from the bin's lower edge up
+            sh.hist[0][tid] = 0u;
+            __syncthreads();
+        } else if (b1 >= 0 && b1 < 255) {
+            // x = ord - floor has its top 16 bits = b1 (bits 48..63 of key - fl)
+            const SStageOff so{stage, ns, fl};
+            K = fast_kth_run(so, sh, (unsigned)k - above1, (unsigned long long)b1 << 48, 0xFFFFull << 48, 48, 1) + fl;
+        } else {  // the k-th key is far above the floor: the plain radix
+            sh.hist[0][tid] = 0u;
+            sh.hist[1][tid] = 0u;
+            __syncthreads();
+            K = fast_kth(s, sh, (unsigned)k, floor_ord, hi);
+        }
         nsel = fast_emit_bitmap(s, K, bound, k, out_idx, out_score, sh, bm, tail, tail_words, wpre, true);
     } else {
         // more entries at or above the floor than the stage holds: the same
         // steps over the row in global memory (the whole stage is free)
+        sh.hist[0][tid] = 0u;
+        __syncthreads();
         const unsigned long long K = fast_kth(g, sh, (unsigned)k, floor_ord, hi);
         nsel = fast_emit_bitmap(g, K, bound, k, out_idx, out_score, sh, bm, reinterpret_cast<unsigned *>(stage),
                                 2 * stage_cap, wpre);
