@@ -32,6 +32,7 @@ constexpr int kGatherWarps = 2;                  // Refine: cp.async producers o
 constexpr int kGatherWarp0 = 2 + kEpiWarps;      // their first warp
 constexpr int kThreadsG = kThreads + 32 * kGatherWarps;
 constexpr int kGatherThreads = 32 * kGatherWarps;
+constexpr int kGatherInFlight = 2;               // cp.async tile groups a producer keeps in flight
 constexpr int kStages = 4;
 constexpr uint32_t kQSlice = 256 * 128;          // 256 rows x 64 bf16 (32 KB)
 constexpr uint32_t kQBytes = 2 * kQSlice;        // 2 K slices
@@ -151,13 +152,9 @@ __device__ __forceinline__ float reduce32(const uint32_t (&v)[32], const float *
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void *src) {
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
 }
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 template <int N>
 __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
-// arrive on `bar` once every earlier cp.async of this thread has landed (the
-// barrier's expected count includes this arrival)
-__device__ __forceinline__ void cp_async_arrive(uint64_t *bar) {
-    asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(tc::smem_u32(bar)) : "memory");
-}
 // the executing thread's generic-proxy writes to shared memory become
 // visible to the async proxy (the tensor cores read the stage through it)
 __device__ __forceinline__ void fence_proxy_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
@@ -271,9 +268,6 @@ __global__ void __launch_bounds__(GATHER ? kThreadsG : kThreads, 1)
                     const uint32_t tt = t + j, st = tt % kStages, ph = (tt / kStages) & 1u, buf = tt & 1u;
                     if (!(ok = tc::mbar_wait(&sh.afull[st], ph, abort, status))) break;
                     if (!(ok = tc::mbar_wait(&sh.tempty[buf], ((tt >> 1) & 1u) ^ 1u, abort, status))) break;
-                    // Refine: the stage was written by cp.async (generic proxy) and
-                    // is read by the tensor cores (async proxy)
-                    if (GATHER) fence_proxy_async_smem();
                     tc::fence_after_sync();
                     const uint32_t abase = tc::smem_u32(as + st * kAStage);
 #pragma unroll
@@ -294,14 +288,10 @@ __global__ void __launch_bounds__(GATHER ? kThreadsG : kThreads, 1)
             // key row flat / 16, 16-byte chunk flat % 16 (chunks 0-7: dims
             // 0-63, slice 0; 8-15: dims 64-127, slice 1), to the swizzled
             // position TMA would give it (chunk ^ (row & 7) within the row).
-            // A tile's arrival is tracked by the hardware (each thread's
-            // copies arrive on the stage's barrier when they land), so the
-            // producers never wait for their copies.  The tiles' key rows come
-            // from a 4-slot ring in shared memory (the area the paged decode
-            // uses for its block table): the rows of tile j + 3 are loaded at
-            // iteration j and stored at iteration j + 1, so no load is waited
-            // for.
-            constexpr int kPosSlots = 4;
+            // The tiles' key rows come from a 4-slot ring in shared memory
+            // (the area the paged decode uses for its block table), filled
+            // kPosAhead tiles ahead so the copies never wait on a load.
+            constexpr int kPosAhead = 2, kPosSlots = 4;
             const int gt = threadIdx.x - kGatherWarp0 * 32;
             const int ch = gt & 15;
             const uint8_t *kbytes = reinterpret_cast<const uint8_t *>(g.k);
@@ -313,26 +303,24 @@ __global__ void __launch_bounds__(GATHER ? kThreadsG : kThreads, 1)
                 return (int)(it.key0 >= 0 ? it.key0 + p
                                           : cache_row(g.bt, g.page, g.max_pages, g.num_pages, g.n_max, it.req, p));
             };
-            for (int j = 0; j < 2 && j < it.nt; ++j) {
-                ring[j * KT + gt] = key_row(j * KT + gt);
-                ring[j * KT + gt + 64] = key_row(j * KT + gt + 64);
-            }
-            int b0 = 0, b1 = 0;  // rows of tile j + 2, stored at iteration j
-            if (2 < it.nt) {
-                b0 = key_row(2 * KT + gt);
-                b1 = key_row(2 * KT + gt + 64);
+            for (int j = 0; j < kPosAhead && j < it.nt; ++j) {
+                ring[(j % kPosSlots) * KT + gt] = key_row(j * KT + gt);
+                ring[(j % kPosSlots) * KT + gt + 64] = key_row(j * KT + gt + 64);
             }
             tc::named_bar_sync(1, kGatherThreads);
             // Both warps run every iteration and reach every barrier, even
             // after a wait ran out (then they only skip the copies): the
             // barrier between them never waits for a warp that has left.
             bool ok = true;
+            int done = 0;  // tiles of this item whose arrival was signalled
             for (int j = 0; j < it.nt; ++j) {
                 const uint32_t tt = t + j, st = tt % kStages, ph = (tt / kStages) & 1u;
-                int a0 = 0, a1 = 0;  // rows of tile j + 3, loaded now
-                if (j + 3 < it.nt) {
-                    a0 = key_row((j + 3) * KT + gt);
-                    a1 = key_row((j + 3) * KT + gt + 64);
+                // the key rows of tile j + kPosAhead, loaded now, stored after the copies
+                const int ja = j + kPosAhead;
+                int ka = 0, kb = 0;
+                if (ja < it.nt) {
+                    ka = key_row(ja * KT + gt);
+                    kb = key_row(ja * KT + gt + 64);
                 }
                 bool go = ok && !*abort;
                 if (go && lane == 0) go = tc::mbar_wait(&sh.aempty[st], ph ^ 1u, abort, status);
@@ -346,21 +334,29 @@ __global__ void __launch_bounds__(GATHER ? kThreadsG : kThreads, 1)
                         cp_async16(dst0 + row * 128 + ((((uint32_t)ch & 7u) ^ ((uint32_t)row & 7u)) << 4),
                                    kbytes + (long long)rows[row] * (S_D * 2) + ch * 16);
                     }
-                    cp_async_arrive(&sh.afull[st]);
-                } else {
-                    ok = false;
                 }
-                if (j + 2 < it.nt) {
-                    ring[((j + 2) % kPosSlots) * KT + gt] = b0;
-                    ring[((j + 2) % kPosSlots) * KT + gt + 64] = b1;
+                cp_async_commit();  // one group per tile, empty when skipped
+                if (ja < it.nt) {
+                    ring[(ja % kPosSlots) * KT + gt] = ka;
+                    ring[(ja % kPosSlots) * KT + gt + 64] = kb;
                 }
-                b0 = a0;
-                b1 = a1;
-                // slot (j + 2) is written before any thread reads it, and
-                // slot j is read by all before it is written again
+                // slot (j + kPosAhead) is written before any thread reads it,
+                // and slot j is read by all before it is written again
                 tc::named_bar_sync(1, kGatherThreads);
+                if (!go) ok = false;
+                if (ok && j >= kGatherInFlight) {
+                    // tile j - kGatherInFlight has landed: publish it
+                    cp_async_wait<kGatherInFlight>();
+                    fence_proxy_async_smem();
+                    tc::mbar_arrive(&sh.afull[(t + done) % kStages]);
+                    ++done;
+                }
             }
-            cp_async_wait<0>();  // this thread's copies have landed before shared memory is left
+            cp_async_wait<0>();
+            fence_proxy_async_smem();
+            // publish the tiles still pending (all of them when the item ran out early)
+            if (ok)
+                for (; done < it.nt; ++done) tc::mbar_arrive(&sh.afull[(t + done) % kStages]);
         } else {
             const int quarter = warp & 3;
             const int r = (warp - 2) >> 2;  // the scored row of this warp
