@@ -287,64 +287,32 @@ __global__ void __launch_bounds__(GATHER ? kThreadsG : kThreads, 1)
             // thread gt copies, per tile, chunks flat = u * 64 + gt (u < 32):
             // key row flat / 16, 16-byte chunk flat % 16 (chunks 0-7: dims
             // 0-63, slice 0; 8-15: dims 64-127, slice 1), to the swizzled
-            // position TMA would give it (chunk ^ (row & 7) within the row).
-            // The tiles' key rows come from a 4-slot ring in shared memory
-            // (the area the paged decode uses for its block table), filled
-            // kPosAhead tiles ahead so the copies never wait on a load.
-            constexpr int kPosAhead = 2, kPosSlots = 4;
+            // position TMA would give it (chunk ^ (row & 7) within the row)
             const int gt = threadIdx.x - kGatherWarp0 * 32;
             const int ch = gt & 15;
             const uint8_t *kbytes = reinterpret_cast<const uint8_t *>(g.k);
-            int *ring = pg_rows;  // [kPosSlots][KT] key rows
-            // key row of candidate slot jj (-1 and unused slots: the request's first row)
-            auto key_row = [&](int jj) -> int {
-                const int pos = jj < g.c ? it.cand[jj] : -1;
-                const int p = pos >= 0 ? pos : 0;
-                return (int)(it.key0 >= 0 ? it.key0 + p
-                                          : cache_row(g.bt, g.page, g.max_pages, g.num_pages, g.n_max, it.req, p));
-            };
-            for (int j = 0; j < kPosAhead && j < it.nt; ++j) {
-                ring[(j % kPosSlots) * KT + gt] = key_row(j * KT + gt);
-                ring[(j % kPosSlots) * KT + gt + 64] = key_row(j * KT + gt + 64);
-            }
-            tc::named_bar_sync(1, kGatherThreads);
-            // Both warps run every iteration and reach every barrier, even
-            // after a wait ran out (then they only skip the copies): the
-            // barrier between them never waits for a warp that has left.
-            bool ok = true;
+            bool ok = !*abort;
             int done = 0;  // tiles of this item whose arrival was signalled
-            for (int j = 0; j < it.nt; ++j) {
+            for (int j = 0; j < it.nt && ok; ++j) {
                 const uint32_t tt = t + j, st = tt % kStages, ph = (tt / kStages) & 1u;
-                // the key rows of tile j + kPosAhead, loaded now, stored after the copies
-                const int ja = j + kPosAhead;
-                int ka = 0, kb = 0;
-                if (ja < it.nt) {
-                    ka = key_row(ja * KT + gt);
-                    kb = key_row(ja * KT + gt + 64);
+                if (lane == 0) ok = tc::mbar_wait(&sh.aempty[st], ph ^ 1u, abort, status);
+                ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
+                if (!ok) break;
+                const uint32_t dst0 = tc::smem_u32(as + st * kAStage) + (uint32_t)(ch >> 3) * kASlice;
+#pragma unroll 4
+                for (int u = 0; u < 32; ++u) {
+                    const int row = u * 4 + (gt >> 4);
+                    const int jj = j * KT + row;
+                    const int pos = jj < g.c ? it.cand[jj] : -1;
+                    const int p = pos >= 0 ? pos : 0;  // unused slots read the request's first row
+                    const long long krow = it.key0 >= 0 ? it.key0 + p
+                                                        : cache_row(g.bt, g.page, g.max_pages, g.num_pages, g.n_max,
+                                                                    it.req, p);
+                    cp_async16(dst0 + row * 128 + ((((uint32_t)ch & 7u) ^ ((uint32_t)row & 7u)) << 4),
+                               kbytes + krow * (S_D * 2) + ch * 16);
                 }
-                bool go = ok && !*abort;
-                if (go && lane == 0) go = tc::mbar_wait(&sh.aempty[st], ph ^ 1u, abort, status);
-                go = __shfl_sync(0xFFFFFFFFu, go, 0);
-                if (go) {
-                    const uint32_t dst0 = tc::smem_u32(as + st * kAStage) + (uint32_t)(ch >> 3) * kASlice;
-                    const int *rows = ring + (j % kPosSlots) * KT;
-#pragma unroll 8
-                    for (int u = 0; u < 32; ++u) {
-                        const int row = u * 4 + (gt >> 4);
-                        cp_async16(dst0 + row * 128 + ((((uint32_t)ch & 7u) ^ ((uint32_t)row & 7u)) << 4),
-                                   kbytes + (long long)rows[row] * (S_D * 2) + ch * 16);
-                    }
-                }
-                cp_async_commit();  // one group per tile, empty when skipped
-                if (ja < it.nt) {
-                    ring[(ja % kPosSlots) * KT + gt] = ka;
-                    ring[(ja % kPosSlots) * KT + gt + 64] = kb;
-                }
-                // slot (j + kPosAhead) is written before any thread reads it,
-                // and slot j is read by all before it is written again
-                tc::named_bar_sync(1, kGatherThreads);
-                if (!go) ok = false;
-                if (ok && j >= kGatherInFlight) {
+                cp_async_commit();
+                if (j >= kGatherInFlight) {
                     // tile j - kGatherInFlight has landed: publish it
                     cp_async_wait<kGatherInFlight>();
                     fence_proxy_async_smem();
