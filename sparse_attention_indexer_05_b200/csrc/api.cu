@@ -55,7 +55,7 @@ struct PrefillWs {
     long long Rb;         // scored rows of one call's output rows (per-row scratch)
     long long Mb;         // members of one call's groups (member scores)
     unsigned cap, ksel;
-    size_t status, plan, slot, qbar, wbar, cnt, floor, buf, cand, msc, kblk, cblk, total;
+    size_t status, plan, slot, qbar, wbar, cnt, floor, buf, cand, msc, ckeys, kblk, cblk, total;
 };
 
 bool refines(idx_mode m) { return m == IDX_MODE_REFINE || m == IDX_MODE_BLOCK; }
@@ -109,6 +109,9 @@ PrefillWs prefill_ws(int T, int H, int d, int topk, int S, idx_dtype dt, int g, 
     L.buf = cv.take((size_t)L.Rb * L.cap * 8);
     L.cand = refines(mode) ? cv.take((size_t)L.Rb * c * 4) : 0;
     L.msc = refines(mode) ? cv.take((size_t)L.Mb * c * 4) : 0;
+    L.ckeys = (refines(mode) && tc_gather_supported(H, d, (int)dt, g, c))
+                  ? cv.take((size_t)L.Rb * c_pad_of(c) * d * esize(dt))
+                  : 0;
     L.kblk = mode == IDX_MODE_BLOCK ? cv.take((size_t)block_rows(T) * d * esize(dt)) : 0;
     L.cblk = mode == IDX_MODE_BLOCK ? cv.take((size_t)L.Rb * (c >> kBlockShift) * 4) : 0;
     L.total = cv.off;
@@ -136,7 +139,7 @@ AdaptiveWs adaptive_ws(int T, int H, int d, int topk, int rho, int S, idx_dtype 
 }
 
 struct DecodeWs {
-    size_t status, qbar, wbar, spill, cand, msc, total;
+    size_t status, qbar, wbar, spill, cand, msc, ckeys, total;
 };
 
 DecodeWs decode_ws(int B, int G, int n_max, int H, int d, int c, idx_mode mode, idx_dtype dt) {
@@ -149,6 +152,9 @@ DecodeWs decode_ws(int B, int G, int n_max, int H, int d, int c, idx_mode mode, 
     L.spill = cv.take((size_t)rows * n_max * 4);
     L.cand = mode == IDX_MODE_REFINE ? cv.take((size_t)B * c * 4) : 0;
     L.msc = mode == IDX_MODE_REFINE ? cv.take((size_t)B * G * c * 4) : 0;
+    L.ckeys = (mode == IDX_MODE_REFINE && tc_gather_supported(H, d, (int)dt, G, c))
+                  ? cv.take((size_t)B * c_pad_of(c) * d * esize(dt))
+                  : 0;
     L.total = cv.off;
     return L;
 }
@@ -293,6 +299,8 @@ struct Prefill {
         a.cu = cu; a.S = S; a.g = g; a.db = db; a.cu_T = T;
         a.plan = plan(); a.pl = L.pl;
         a.out = reinterpret_cast<float *>(ws + L.msc);
+        a.ckeys = ws + L.ckeys;
+        a.ckey_groups = L.Rb;
         a.c_pad = c_pad_of(c);
         a.status = status();
         return a;
@@ -552,6 +560,8 @@ struct Decode {
         a.mode = 1;
         a.G = G; a.n_max = n_max; a.kv_len = kv;
         a.out = reinterpret_cast<float *>(ws + L.msc);
+        a.ckeys = ws + L.ckeys;
+        a.ckey_groups = B;
         a.c_pad = c_pad_of(c);
         a.status = status();
         a.bt = bt; a.page = page; a.max_pages = max_pages; a.num_pages = num_pages;

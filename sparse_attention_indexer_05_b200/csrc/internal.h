@@ -108,6 +108,9 @@ struct GatherArgs {
     int G, n_max;
     const int *kv_len;
     float *out;          // [rows, c] member scores (prefill: rows from the call's first member)
+    void *ckeys;         // [groups, c_pad, d] packed candidate keys (tensor-core path; prefill: groups
+                         // from the call's first scored row)
+    long long ckey_groups;  // groups the packed-key area holds
     int c_pad;           // c rounded up to a multiple of 128
     unsigned *status;
     const int *bt;       // decode: paged cache, as in DecodeArgs

@@ -2,13 +2,10 @@
 // 64*m <= 256 columns) against a stream of key tiles and write every score:
 //   * decode scan: the keys are the request's cache, streamed once by TMA
 //     in 128-key tiles; rows = the request's G MTP queries (or its proxy);
-//   * Refine re-score: the keys are a group's candidate set C, gathered
-//     straight from the key rows (which sit in L2: 256 B per token) by two
-//     producer warps with 16-byte cp.async copies into the same
-//     128-byte-swizzled stage layout TMA writes; rows = up to 4 members of
-//     the group.  Each tile is 2048 copies of 16 B, 16 lanes per key row.
-//     (TMA tile::gather4 moves 4 rows per request, 64 requests per tile, more
-//     than one SM's TMA issue rate keeps up with at the MMA's pace.)
+//   * Refine re-score: the keys are a group's candidate set C, first packed
+//     into a contiguous [c_pad, d] block per group by compact_keys_kernel
+//     (coalesced 16-byte copies), then streamed by TMA like the decode
+//     cache; rows = up to 4 members of the group.
 // Same MMA shape as the prefill score kernel (keys on M, (row, head) on N,
 // bf16 -> fp32 in TMEM, fused ReLU + w-weighted head sum), with the two
 // 256-column TMEM buffers used alternately by consecutive key tiles.
@@ -28,11 +25,6 @@ constexpr int S_H = 64;
 constexpr int S_D = 128;
 constexpr int kEpiWarps = 16;                    // 4 per TMEM lane quarter, one scored row each
 constexpr int kThreads = 64 + 32 * kEpiWarps;    // + producer warp + MMA warp
-constexpr int kGatherWarps = 2;                  // Refine: cp.async producers of the candidate keys
-constexpr int kGatherWarp0 = 2 + kEpiWarps;      // their first warp
-constexpr int kThreadsG = kThreads + 32 * kGatherWarps;
-constexpr int kGatherThreads = 32 * kGatherWarps;
-constexpr int kGatherInFlight = 2;               // cp.async tile groups a producer keeps in flight
 constexpr int kStages = 4;
 constexpr uint32_t kQSlice = 256 * 128;          // 256 rows x 64 bf16 (32 KB)
 constexpr uint32_t kQBytes = 2 * kQSlice;        // 2 K slices
@@ -59,8 +51,6 @@ struct Item {
     int m;              // rows scored (<= 4)
     long long qrow0;    // first query row (rows of [*, 64, 128])
     long long key0;     // first key row of the request
-    const int *cand;    // Refine: the group's candidate positions [c]
-    int req;            // Refine decode: the request (key rows through cache_row)
     int t0, nt;         // key tiles [t0, t0 + nt) of the item
     // outputs
     long long out_row0; // output row of scored row 0
@@ -94,19 +84,18 @@ __device__ __forceinline__ Item item_info(const GatherArgs &g, const DecodeArgs 
             if (kv < g.G || kv > g.n_max) return it;
             cnt = g.G;
             m0 = (long long)grp * g.G;
-            key0 = -1;  // rows through cache_row
+            key0 = (long long)grp * g.n_max;
         }
         const int m = cnt - mc * 4;
         if (m <= 0) return it;
+        (void)key0;
         it.valid = true;
         it.m = m < 4 ? m : 4;
         it.qrow0 = m0 + mc * 4;
         // prefill scratch: member scores from the call's first member,
-        // candidate sets from its first scored row
+        // packed keys from its first scored row
         it.out_row0 = it.qrow0 - (g.mode == 0 ? g.plan[8] : 0);
-        it.key0 = key0;  // prefill: the request's first key row; decode: -1 (cache_row)
-        it.cand = g.cand + ((long long)grp - (g.mode == 0 ? g.plan[6] : 0)) * g.c;
-        it.req = grp;
+        it.key0 = ((long long)grp - (g.mode == 0 ? g.plan[6] : 0)) * g.c_pad;  // the group's packed keys
         it.t0 = 0;
         it.nt = g.c_pad / KT;
     } else {
@@ -148,22 +137,35 @@ __device__ __forceinline__ float reduce32(const uint32_t (&v)[32], const float *
     return ((a[0] + a[1]) + (a[2] + a[3])) + ((a[4] + a[5]) + (a[6] + a[7]));
 }
 
-// 16-byte global -> shared copy, cached in L2 only
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void *src) {
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+// sum_j w[j] * max(v[j], 0) over 64 heads; w 16-byte aligned, read as float4
+__device__ __forceinline__ float reduce64(const uint32_t (&v0)[32], const uint32_t (&v1)[32], const float *w) {
+    const float4 *w4 = reinterpret_cast<const float4 *>(w);
+    float a[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) a[i] = 0.0f;
+#pragma unroll
+    for (int j4 = 0; j4 < 8; ++j4) {
+        const float4 wv = w4[j4];
+        a[(4 * j4 + 0) & 7] = fmaf(wv.x, fmaxf(__uint_as_float(v0[4 * j4 + 0]), 0.0f), a[(4 * j4 + 0) & 7]);
+        a[(4 * j4 + 1) & 7] = fmaf(wv.y, fmaxf(__uint_as_float(v0[4 * j4 + 1]), 0.0f), a[(4 * j4 + 1) & 7]);
+        a[(4 * j4 + 2) & 7] = fmaf(wv.z, fmaxf(__uint_as_float(v0[4 * j4 + 2]), 0.0f), a[(4 * j4 + 2) & 7]);
+        a[(4 * j4 + 3) & 7] = fmaf(wv.w, fmaxf(__uint_as_float(v0[4 * j4 + 3]), 0.0f), a[(4 * j4 + 3) & 7]);
+    }
+#pragma unroll
+    for (int j4 = 0; j4 < 8; ++j4) {
+        const float4 wv = w4[8 + j4];
+        a[(4 * j4 + 0) & 7] = fmaf(wv.x, fmaxf(__uint_as_float(v1[4 * j4 + 0]), 0.0f), a[(4 * j4 + 0) & 7]);
+        a[(4 * j4 + 1) & 7] = fmaf(wv.y, fmaxf(__uint_as_float(v1[4 * j4 + 1]), 0.0f), a[(4 * j4 + 1) & 7]);
+        a[(4 * j4 + 2) & 7] = fmaf(wv.z, fmaxf(__uint_as_float(v1[4 * j4 + 2]), 0.0f), a[(4 * j4 + 2) & 7]);
+        a[(4 * j4 + 3) & 7] = fmaf(wv.w, fmaxf(__uint_as_float(v1[4 * j4 + 3]), 0.0f), a[(4 * j4 + 3) & 7]);
+    }
+    return ((a[0] + a[1]) + (a[2] + a[3])) + ((a[4] + a[5]) + (a[6] + a[7]));
 }
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-template <int N>
-__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
-// the executing thread's generic-proxy writes to shared memory become
-// visible to the async proxy (the tensor cores read the stage through it)
-__device__ __forceinline__ void fence_proxy_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 
 template <bool GATHER>
-__global__ void __launch_bounds__(GATHER ? kThreadsG : kThreads, 1)
+__global__ void __launch_bounds__(kThreads, 1)
     stream_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_k,
                      GatherArgs g, DecodeArgs dd, int nitems) {
-    constexpr int NT = GATHER ? kThreadsG : kThreads;
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = tc::smem_u32(smem_raw);
     uint8_t *smem = smem_raw + (((raw + 1023u) & ~1023u) - raw);
@@ -182,8 +184,7 @@ __global__ void __launch_bounds__(GATHER ? kThreadsG : kThreads, 1)
     const int lane = threadIdx.x & 31;
     if (threadIdx.x == 0) {
         for (int s = 0; s < kStages; ++s) {
-            // Refine: every producer thread arrives once its copies of the tile landed
-            tc::mbar_init(&sh.afull[s], GATHER ? kGatherThreads : 1);
+            tc::mbar_init(&sh.afull[s], 1);
             tc::mbar_init(&sh.aempty[s], 1);
         }
         tc::mbar_init(&sh.qfull, 1);
@@ -214,7 +215,7 @@ __global__ void __launch_bounds__(GATHER ? kThreadsG : kThreads, 1)
         const Item it = item_info<GATHER>(g, dd, item);
         if (!it.valid) continue;
         __syncthreads();
-        for (int i = threadIdx.x; i < 4 * S_H; i += NT)
+        for (int i = threadIdx.x; i < 4 * S_H; i += kThreads)
             wsm[i] = (i / S_H) < it.m ? wsrc[it.qrow0 * S_H + i] : 0.0f;
         __syncthreads();
         const uint32_t idesc = tc::idesc_bf16_f32(128, 64 * it.m);
@@ -237,7 +238,7 @@ __global__ void __launch_bounds__(GATHER ? kThreadsG : kThreads, 1)
                 for (int kh = 0; kh < 2; ++kh)
                     tc::tma_load_2d(qs + kh * kQSlice, &tmap_q, kh * 64, (int)(it.qrow0 * S_H), &sh.qfull);
             }
-            for (int j = 0; j < it.nt && ok && !GATHER; ++j) {
+            for (int j = 0; j < it.nt && ok; ++j) {
                 const uint32_t tt = t + j, st = tt % kStages, ph = (tt / kStages) & 1u;
                 if (lane == 0) ok = tc::mbar_wait(&sh.aempty[st], ph ^ 1u, abort, status);
                 ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
@@ -282,49 +283,6 @@ __global__ void __launch_bounds__(GATHER ? kThreadsG : kThreads, 1)
                     tc::mma_commit(&sh.aempty[st]);
                 }
             }
-        } else if (GATHER && warp >= kGatherWarp0) {
-            // ------------------------------ Refine: candidate keys by cp.async
-            // thread gt copies, per tile, chunks flat = u * 64 + gt (u < 32):
-            // key row flat / 16, 16-byte chunk flat % 16 (chunks 0-7: dims
-            // 0-63, slice 0; 8-15: dims 64-127, slice 1), to the swizzled
-            // position TMA would give it (chunk ^ (row & 7) within the row)
-            const int gt = threadIdx.x - kGatherWarp0 * 32;
-            const int ch = gt & 15;
-            const uint8_t *kbytes = reinterpret_cast<const uint8_t *>(g.k);
-            bool ok = !*abort;
-            int done = 0;  // tiles of this item whose arrival was signalled
-            for (int j = 0; j < it.nt && ok; ++j) {
-                const uint32_t tt = t + j, st = tt % kStages, ph = (tt / kStages) & 1u;
-                if (lane == 0) ok = tc::mbar_wait(&sh.aempty[st], ph ^ 1u, abort, status);
-                ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
-                if (!ok) break;
-                const uint32_t dst0 = tc::smem_u32(as + st * kAStage) + (uint32_t)(ch >> 3) * kASlice;
-#pragma unroll 4
-                for (int u = 0; u < 32; ++u) {
-                    const int row = u * 4 + (gt >> 4);
-                    const int jj = j * KT + row;
-                    const int pos = jj < g.c ? it.cand[jj] : -1;
-                    const int p = pos >= 0 ? pos : 0;  // unused slots read the request's first row
-                    const long long krow = it.key0 >= 0 ? it.key0 + p
-                                                        : cache_row(g.bt, g.page, g.max_pages, g.num_pages, g.n_max,
-                                                                    it.req, p);
-                    cp_async16(dst0 + row * 128 + ((((uint32_t)ch & 7u) ^ ((uint32_t)row & 7u)) << 4),
-                               kbytes + krow * (S_D * 2) + ch * 16);
-                }
-                cp_async_commit();
-                if (j >= kGatherInFlight) {
-                    // tile j - kGatherInFlight has landed: publish it
-                    cp_async_wait<kGatherInFlight>();
-                    fence_proxy_async_smem();
-                    tc::mbar_arrive(&sh.afull[(t + done) % kStages]);
-                    ++done;
-                }
-            }
-            cp_async_wait<0>();
-            fence_proxy_async_smem();
-            // publish the tiles still pending (all of them when the item ran out early)
-            if (ok)
-                for (; done < it.nt; ++done) tc::mbar_arrive(&sh.afull[(t + done) % kStages]);
         } else {
             const int quarter = warp & 3;
             const int r = (warp - 2) >> 2;  // the scored row of this warp
@@ -376,9 +334,8 @@ __global__ void __launch_bounds__(GATHER ? kThreadsG : kThreads, 1)
             tc::mbar_wait_drain(&sh.drain, 0);
         }
         if (warp == 0 && lane == 0) {
-            if (!GATHER)  // TMA key tiles in flight (the gather warps waited for their own copies)
-                for (uint32_t tt = t > kStages ? t - kStages : 0; tt < t; ++tt)
-                    tc::mbar_wait_drain(&sh.afull[tt % kStages], (tt / kStages) & 1u);
+            for (uint32_t tt = t > kStages ? t - kStages : 0; tt < t; ++tt)
+                tc::mbar_wait_drain(&sh.afull[tt % kStages], (tt / kStages) & 1u);
             if (nq) tc::mbar_wait_drain(&sh.qfull, (nq - 1) & 1u);
         }
     }
@@ -386,6 +343,42 @@ __global__ void __launch_bounds__(GATHER ? kThreadsG : kThreads, 1)
     __syncthreads();
     tc::fence_after_sync();
     if (warp == 1) tc::tmem_dealloc(tmem, 512);
+}
+
+// Packs the key rows of every group's candidate set into a contiguous block
+// of c_pad rows (padding slots and the -1 pads of short sets copy the
+// request's row 0; their scores are written but never selected).
+// Grid (groups, c_pad / 128); each CTA copies 128 rows of d bf16.
+__global__ void __launch_bounds__(256) compact_keys_kernel(GatherArgs a) {
+    const int grp = blockIdx.x;
+    const int j0 = blockIdx.y * KT;
+    long long key0;
+    if (a.mode == 0) {
+        if (!a.plan[0] || grp >= a.plan[2]) return;
+        const int *rp = a.plan + a.pl.rp();
+        const int b = find_seg(rp, a.S, grp);
+        const int i = grp - rp[b], n = a.cu[b + 1] - a.cu[b];
+        if (i < dense_rows(n, a.g, a.db) || !row_in_range(a.plan, a.cu, b, i, n, a.g, a.db)) return;  // no set
+        key0 = a.cu[b];
+    } else {
+        const int kv = a.kv_len[grp];
+        if (kv < a.G || kv > a.n_max) return;
+        key0 = -1;  // decode: rows through cache_row
+    }
+    const long long sg = (long long)grp - (a.mode == 0 ? a.plan[6] : 0);  // the group's scratch row
+    const int *cand = a.cand + sg * a.c;
+    const int per_row = a.d * 2 / 16;  // 16-byte chunks per key row
+    const uint4 *src = reinterpret_cast<const uint4 *>(a.k);
+    uint4 *dst = reinterpret_cast<uint4 *>(a.ckeys) + (sg * a.c_pad + j0) * per_row;
+    for (int u = threadIdx.x; u < KT * per_row; u += blockDim.x) {
+        const int r = u / per_row, part = u - r * per_row;
+        const int j = j0 + r;
+        const int pos = j < a.c ? cand[j] : -1;
+        const int p = pos >= 0 ? pos : 0;
+        const long long row =
+            key0 >= 0 ? key0 + p : cache_row(a.bt, a.page, a.max_pages, a.num_pages, a.n_max, grp, p);
+        dst[u] = src[row * per_row + part];
+    }
 }
 
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn2() {
@@ -454,11 +447,18 @@ cudaError_t launch_decode_tc(const DecodeArgs &a, cudaStream_t st) {
 }
 
 cudaError_t launch_gather_tc(const GatherArgs &a, cudaStream_t st) {
-    // the gather copies 16-byte pieces of key rows: the key base must be 16-byte aligned
-    if ((reinterpret_cast<uintptr_t>(a.k) & 15u) != 0) return cudaErrorInvalidValue;
     const long long qrows = a.mode == 0 ? (long long)a.cu_T : (long long)a.G * a.nitems;
-    CUtensorMap mq;
-    if (!map2d(&mq, a.q, (unsigned long long)qrows * S_H, 256)) return cudaErrorInvalidValue;
+    const long long krows = a.ckey_groups * a.c_pad;  // packed candidate keys
+    CUtensorMap mq, mk;
+    if (!map2d(&mq, a.q, (unsigned long long)qrows * S_H, 256) || !map2d(&mk, a.ckeys, (unsigned long long)krows, KT))
+        return cudaErrorInvalidValue;
+    {
+        TraceScope tsc("pack_keys", st);
+        dim3 cgrid(a.nitems, a.c_pad / KT);
+        compact_keys_kernel<<<cgrid, 256, 0, st>>>(a);
+        cudaError_t ce = cudaGetLastError();
+        if (ce != cudaSuccess) return ce;
+    }
     const int mchunks = ((a.mode == 0 ? a.g : a.G) + 3) / 4;
     const int nitems = a.nitems * mchunks;
     const size_t smem = kSmemBytes;
@@ -469,8 +469,7 @@ cudaError_t launch_gather_tc(const GatherArgs &a, cudaStream_t st) {
     TraceScope ts("gather_tc", st);
     const int grid = nitems < sm_count() ? nitems : sm_count();
     if (grid <= 0) return cudaSuccess;
-    // the key stage is filled by cp.async: the second tensor map is not used
-    stream_tc_kernel<true><<<grid, kThreadsG, smem, st>>>(mq, mq, a, dd, nitems);
+    stream_tc_kernel<true><<<grid, kThreads, smem, st>>>(mq, mk, a, dd, nitems);
     return cudaGetLastError();
 }
 
