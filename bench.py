@@ -77,8 +77,9 @@ def parse():
     p.add_argument("--no-cpu", action="store_true", help="skip the CPU-oracle baseline")
     p.add_argument("--tokens", type=int, default=L_TOK,
                    help="batch length (profiling runs use a smaller case; the bench line uses 131072)")
-    p.add_argument("--only", default="all", choices=["all", "dense", "refine"],
-                   help="profiling runs: time one half of the step only")
+    p.add_argument("--only", default="all", choices=["all", "dense", "refine", "attn"],
+                   help="profiling runs: time one half of the step only, or only the sparse attention leg "
+                        "(its selections then come from an untimed dense call)")
     return p.parse_args()
 
 
@@ -267,6 +268,22 @@ def run_configs(args, dev, lib, barrier, max_over_ranks, rank, bf16_sus):
                 "score_tc": {"ms": sms, "flops": fl, "tflops": tf, "frac_bf16_sustained": (tf / bf16_sus) if tf else None},
                 "kernels_ms": {n: t for n, (c, t) in sp.items()}}, (q, k, w, cu, o)
 
+    # the small fp32 case (L = 2048, H = 4, d = 64, k = 64): the CUDA-core path
+    P1 = W.cfg_fp32_small(seed=M.rank_seed(rank))
+    q1, k1, w1, c1 = (to_dev(P1.q, dev), to_dev(P1.k, dev), to_dev(P1.w, dev), to_dev(P1.cu_seqlens, dev))
+    o1s = torch.empty(P1.T, P1.topk, dtype=torch.int32, device=dev)
+    ws1s = torch.empty(idx.dense_workspace_size(P1.T, P1.H, P1.d, P1.topk, 1, torch.float32), dtype=torch.uint8,
+                       device=dev)
+    ms1, sp1 = timed_calls(lambda: idx.dense_topk(q1, k1, w1, c1, P1.topk, out_idx=o1s, workspace=ws1s), args.warmup,
+                           max(args.steps, 20), lib, barrier, max_over_ranks)
+    assert idx.device_status(ws1s) == "IDX_OK"
+    fl1 = 2.0 * P1.H * P1.d * P1.T * (P1.T + 1) / 2.0
+    s1 = kernel_ms(sp1, "score_simt", "dense")
+    out["dense_fp32_2048"] = {"workload": "dense_L2048_H4_d64_k64_fp32 (CUDA-core path)", "ms_per_call": ms1,
+                              "queries_per_s": P1.T / (ms1 / 1000.0), "score_simt_ms": s1,
+                              "score_simt_tflops_fp32": fl1 / (s1 / 1000.0) / 1e12 if s1 > 0 else None,
+                              "kernels_ms": {n: t for n, (c, t) in sp1.items()}}
+    del P1, q1, k1, w1, c1, o1s, ws1s
     # dense L = 16384 (rho 0.95, 1% planted keys)
     P2 = W.cfg_dense_16k(seed=M.rank_seed(rank))
     out["dense_16384"], _ = dense_leg(P2, "dense_L16384_H64_d128_k2048")
@@ -517,6 +534,7 @@ def main():
     cu1, cu2 = to_dev(cu1_h, dev), to_dev(cu2_h, dev)
     do_dense = args.only in ("all", "dense")
     do_refine = args.only in ("all", "refine")
+    attn_only = args.only == "attn"
     ws1 = torch.empty(idx.dense_workspace_size(L, H, D, TOPK, 1) if do_dense else 256, dtype=torch.uint8,
                       device=dev)
     ws2 = torch.empty(idx.pivot_workspace_size(L, H, D, TOPK, 2, G_REF, C_REF, "refine") if do_refine else 256,
@@ -696,7 +714,12 @@ def main():
 
     # ------------------------------- token-sparse attention on the selections
     att = None
-    if do_dense and not args.no_attn:
+    if attn_only:  # the selections the attention leg consumes, from one untimed dense call
+        wsx = torch.empty(idx.dense_workspace_size(L, H, D, TOPK, 1), dtype=torch.uint8, device=dev)
+        idx.dense_topk(q, k, w, cu1, TOPK, out_idx=o1, workspace=wsx)
+        torch.cuda.synchronize()
+        del wsx
+    if (do_dense or attn_only) and not args.no_attn:
         Ra = min(args.attn_rows, L)
         gen = torch.Generator(device=dev)
         gen.manual_seed(4321 + rank)
