@@ -866,7 +866,7 @@ def main():
         "scaling": "strong" if split else "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": {"workload": f"long_prefill_{L}_" + {"all": "dense+refine", "dense": "dense",
-                                                          "refine": "refine"}[args.only] + "_g16_c4096",
+                                                          "refine": "refine", "attn": "none"}[args.only] + "_g16_c4096",
                    "tokens": L, "H": H, "d": D,
                    "topk": TOPK, "dense_requests": [L], "refine_requests": [L // 2, L // 2],
                    "g": G_REF, "c": C_REF,
