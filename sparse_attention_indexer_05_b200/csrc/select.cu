@@ -595,6 +595,23 @@ __device__ __forceinline__ void fast_copy_out(const T *src, T *dst, int n) {
     }
 }
 
+// Bitmap layout of the emit.  The chunk's words (word L covers positions
+// 32L .. 32L+31) are split between the warps in contiguous ranges of
+// 32 * per words, and within a warp's range between the lanes in contiguous
+// blocks of `per` words (per a power of two), so that each lane ranks its
+// block in order with one warp scan.  Word L is stored transposed: the j-th
+// word of lane i's block at (warp range) + 32 j + i, so that a warp reading
+// the j-th word of every lane's block touches 32 consecutive words.
+__device__ __forceinline__ int emit_per(int nwords) {
+    const int per = (nwords + kFWarps * 32 - 1) / (kFWarps * 32);  // 1 .. kChunkWords / kFT
+    return per <= 1 ? 1 : 1 << (32 - __clz(per - 1));
+}
+__device__ __forceinline__ int emit_word(int L, int per) {
+    const int range = 32 * per;
+    const int m = L & (range - 1);
+    return (L - m) + ((m & (per - 1)) << 5) + (m >> (31 - __clz(per)));
+}
+
 // List the nonzero keys >= K of src in ascending position through a bitmap
 // (chunks of kChunkBits positions over 0..bound); returns how many.
 template <class Src>
@@ -610,31 +627,32 @@ __device__ int fast_emit_bitmap(const Src &src, unsigned long long K, int bound,
     float *ps = via_smem ? reinterpret_cast<float *>(buf + k) : out_score;
     for (int c0 = 0; c0 <= bound; c0 += kChunkBits) {
         const int nwords = (bound - c0) / 32 + 1 < kChunkWords ? (bound - c0) / 32 + 1 : kChunkWords;
-        // words walked: the chunk's positions up to bound, a multiple of
-        // 32 per warp (per warp: kWordsW of them)
-        const int kWordsW = ((nwords + kFWarps * 32 - 1) / (kFWarps * 32)) * 32;
+        const int per = emit_per(nwords);
         if (!(bm_clear && c0 == 0)) {  // the caller may have cleared it for the first chunk
-            for (int j = tid; j < kFWarps * kWordsW; j += kFT) bm[j] = 0u;
+            for (int j = tid; j < kFT * per; j += kFT) bm[j] = 0u;
             __syncthreads();
         }
         for (int i = tid; i < src.n; i += kFT) {
             const unsigned long long kk = src.key(i);
             if (kk != 0ull && kk >= K) {
                 const int p = key_pos(kk) - c0;
-                if (p >= 0 && p < kChunkBits) atomicOr(&bm[p >> 5], 1u << (p & 31));
+                if (p >= 0 && p < kChunkBits) atomicOr(&bm[emit_word(p >> 5, per)], 1u << (p & 31));
             }
         }
         __syncthreads();
-        // warp w owns words [w * kWordsW, +kWordsW) and walks them 32 at a
-        // time (lane i reads word base + i: conflict-free); a warp prefix of
-        // the words' bit counts places each word's positions, in order
+        // lane `lane` of warp `warp` owns logical words wb + lane * per .. + per - 1,
+        // stored at wb + 32 j + lane
         const int lane = tid & 31, warp = tid >> 5;
-        const int wb = warp * kWordsW;
+        const int wb = warp * 32 * per;
         unsigned cnt = 0;
-#pragma unroll 4
-        for (int j = 0; j < kWordsW; j += 32) cnt += __popc(bm[wb + j + lane]);
-        cnt = __reduce_add_sync(0xFFFFFFFFu, cnt);
-        if (lane == 0) sh.wtot[warp] = cnt;
+        for (int j = 0; j < per; ++j) cnt += __popc(bm[wb + 32 * j + lane]);
+        unsigned inc = cnt;  // inclusive warp prefix of the lanes' counts
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const unsigned v = __shfl_up_sync(0xFFFFFFFFu, inc, o);
+            if (lane >= o) inc += v;
+        }
+        if (lane == 31) sh.wtot[warp] = inc;
         __syncthreads();
         unsigned before = 0, total = 0;
 #pragma unroll
@@ -643,26 +661,18 @@ __device__ int fast_emit_bitmap(const Src &src, unsigned long long K, int bound,
             before += w < warp ? t : 0u;
             total += t;
         }
-        unsigned r = base + before;
-        for (int j = 0; j < kWordsW; j += 32) {
-            const int w = wb + j + lane;
+        unsigned at = base + before + inc - cnt;
+        const int pos0 = c0 + (wb + lane * per) * 32;  // first position of the lane's block
+        for (int j = 0; j < per; ++j) {
+            const int w = wb + 32 * j + lane;
             unsigned x = bm[w];
-            const unsigned c = __popc(x);
-            unsigned inc = c;  // inclusive warp prefix of the words' counts
-#pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const unsigned v = __shfl_up_sync(0xFFFFFFFFu, inc, o);
-                if (lane >= o) inc += v;
-            }
-            unsigned at = r + inc - c;
             if (wpre) wpre[w] = at - base;  // chunk-local rank of the word's first bit
             while (x) {
                 const int bit = __ffs(x) - 1;
                 x &= x - 1u;
-                if (at < (unsigned)k) pi[at] = c0 + w * 32 + bit;  // never past the row
+                if (at < (unsigned)k) pi[at] = pos0 + 32 * j + bit;  // never past the row
                 ++at;
             }
-            r += __shfl_sync(0xFFFFFFFFu, inc, 31);
         }
         if (out_score) {
             __syncthreads();  // every word's rank is recorded; the bitmap is intact
@@ -671,7 +681,7 @@ __device__ int fast_emit_bitmap(const Src &src, unsigned long long K, int bound,
                 if (kk != 0ull && kk >= K) {
                     const int p = key_pos(kk) - c0;
                     if (p >= 0 && p < kChunkBits) {
-                        const int w = p >> 5;
+                        const int w = emit_word(p >> 5, per);
                         const unsigned rk = wpre[w] + __popc(bm[w] & ((1u << (p & 31)) - 1u));
                         if (base + (int)rk < k) ps[base + rk] = ord_score(key_ord(kk));
                     }
@@ -785,21 +795,32 @@ __device__ void fast_cand_row(const unsigned long long *buf, int n, unsigned flo
     // (ordered before it by the barrier below)
     {
         const int nw = bound / 32 + 1 < kChunkWords ? bound / 32 + 1 : kChunkWords;
-        const int nclr = ((nw + kFWarps * 32 - 1) / (kFWarps * 32)) * 32 * kFWarps;
+        const int nclr = kFT * emit_per(nw);
         for (int j = tid; j < nclr; j += kFT) bm[j] = 0u;
     }
     unsigned mx = 0u;
-    // 8 keys per thread and round, as four 16-byte loads (rows start 2 KB aligned)
+    // 8 keys per thread and round, as four 16-byte loads (rows start 2 KB
+    // aligned); the next round's loads are issued before this round's keys
+    // are filtered, so their latency overlaps the work
     const ulonglong2 *b2 = reinterpret_cast<const ulonglong2 *>(buf);
+    ulonglong2 nx[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+        const int i = u * (kFT * 2) + tid * 2;
+        nx[u] = i < n ? b2[i >> 1] : make_ulonglong2(0ull, 0ull);
+    }
     for (int base = 0; base < n; base += kFT * 8) {
         unsigned long long kv[8];
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
             const int i = base + u * (kFT * 2) + tid * 2;
-            ulonglong2 v = make_ulonglong2(0ull, 0ull);
-            if (i < n) v = b2[i >> 1];
-            kv[2 * u] = v.x;
-            kv[2 * u + 1] = (i + 1 < n) ? v.y : 0ull;
+            kv[2 * u] = i < n ? nx[u].x : 0ull;
+            kv[2 * u + 1] = (i + 1 < n) ? nx[u].y : 0ull;
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int i = base + kFT * 8 + u * (kFT * 2) + tid * 2;
+            if (i < n) nx[u] = b2[i >> 1];
         }
         unsigned cnt = 0;
 #pragma unroll

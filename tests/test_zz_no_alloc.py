@@ -5,7 +5,9 @@ receives input and output buffers, a serving loop that must not allocate):
 its scratch is a fixed device array inside the library.  The test calls it
 through the C ABI twice in a row, on different inputs, and checks each
 result against the workspace-taking idx_decode_topk (dense mode): the same
-indices, and scores within the tolerance of the other parity tests.  It
+indices, and scores within the tolerance of the other parity tests; and
+against the oracle's dense decode top-k (well-formed rows, recall >= 0.999,
+the bar of the other bf16 decode parity tests).  It
 also checks that a call too large for the fixed scratch is refused, that
 arguments the workspace entry point rejects are rejected with the same
 code, and that the device status word of the fixed scratch is reported by
@@ -15,8 +17,9 @@ here leaves every other test run.
 import numpy as np
 import pytest
 
+import oracle as O
 from sparse_attention_indexer_05_b200 import workloads as W
-from tests._util import to_dev
+from tests._util import check_rows_wellformed, recall, to_dev
 
 pytestmark = pytest.mark.gpu
 torch = pytest.importorskip("torch")
@@ -49,6 +52,10 @@ def test_noalloc_decode_matches_workspace_entry_point_twice():
         torch.cuda.synchronize()
         assert torch.equal(out_idx, ref_idx)
         _close(out_sc.cpu().numpy(), ref_sc.cpu().numpy())
+        got = out_idx.cpu().numpy()
+        check_rows_wellformed(got, [int(n) - 2 + m for n in kv for m in range(2)], topk)
+        want = O.decode_topk(D.q, D.kcache, D.w, D.kv_len, topk, 0, O.DENSE)
+        assert recall(got, want) >= 0.999, seed
 
 
 def test_noalloc_refuses_calls_beyond_its_scratch():
