@@ -399,7 +399,6 @@ idx_status idx_adaptive_topk(const void *q, const void *k, const float *w, const
     TRY_CUDA(P.prepare());
     TRY_CUDA(P.score(P.score_args(false)));
     float *sc = out_score ? out_score : reinterpret_cast<float *>(base + L.score);
-    TRY_CUDA(launch_select(P.select_args(SEL_DENSE_CAND, T, width, out_idx, sc), P.st));
     AdaptiveArgs a{};
     a.T = T;
     a.k = topk;
@@ -409,6 +408,14 @@ idx_status idx_adaptive_topk(const void *q, const void *k, const float *w, const
     a.sigma = out_sigma ? out_sigma : reinterpret_cast<float *>(base + L.sigma);
     a.vk = reinterpret_cast<unsigned *>(base + L.vk);
     a.need = reinterpret_cast<int *>(base + L.need);
+    // the final select ranks each row's top-(rho k) and, from the same staged
+    // keys, its cutoff margin at k (sigma, the ord of s_(k-1), its ties kept)
+    SelectArgs sa = P.select_args(SEL_DENSE_CAND, T, width, out_idx, sc);
+    sa.kmargin = topk;
+    sa.m_sigma = a.sigma;
+    sa.m_vk = a.vk;
+    sa.m_need = a.need;
+    TRY_CUDA(launch_select(sa, P.st));
     a.trigger = out_trigger;
     a.tau = reinterpret_cast<unsigned *>(base + L.tau);
     a.q = qfrac;

@@ -171,11 +171,17 @@ struct SelectArgs {
     int G, n_max;
     int bitmap_words;        // shared bitmap capacity (words)
     unsigned *status;
+    // dense candidate rows only: the cutoff margin of the top-kmargin inside
+    // the row's top-k (adaptive budget), per output row; kmargin = 0: none
+    int kmargin;
+    float *m_sigma;
+    unsigned *m_vk;
+    int *m_need;
 };
 
 // adaptive.cu: the adaptive budget from the cutoff margin over the rows of a
 // top-(rho k) result (in place).
-constexpr int kAdaptiveMaxWidth = 8192;  // rho * k held in registers by the margin kernel
+constexpr int kAdaptiveMaxWidth = 8192;  // rho * k: the final select's staging room stays in shared memory
 struct AdaptiveArgs {
     long long T;
     int k, width;             // width = rho * k

@@ -441,6 +441,7 @@ constexpr int kChunkWords = kChunkBits / 32;      // 4096 words = 16 KB
 struct __align__(16) FastShared {
     unsigned hist[2][256];
     unsigned wtot[kFWarps];
+    unsigned blkpre[kFT];  // emit: chunk-local rank of each lane block's first bit
     unsigned nstage;
     unsigned maxord;
     unsigned minord;
@@ -617,7 +618,7 @@ __device__ __forceinline__ int emit_word(int L, int per) {
 template <class Src>
 __device__ int fast_emit_bitmap(const Src &src, unsigned long long K, int bound, int k, int *out_idx,
                                 float *out_score, FastShared &sh, unsigned *bm, unsigned *buf, int buf_words,
-                                unsigned *wpre, bool bm_clear = false) {
+                                bool bm_clear = false) {
     const int tid = threadIdx.x;
     int base = 0;
     // the list is built in shared memory (buf: free stage room) and copied
@@ -662,11 +663,11 @@ __device__ int fast_emit_bitmap(const Src &src, unsigned long long K, int bound,
             total += t;
         }
         unsigned at = base + before + inc - cnt;
+        sh.blkpre[tid] = at - base;
         const int pos0 = c0 + (wb + lane * per) * 32;  // first position of the lane's block
         for (int j = 0; j < per; ++j) {
             const int w = wb + 32 * j + lane;
             unsigned x = bm[w];
-            if (wpre) wpre[w] = at - base;  // chunk-local rank of the word's first bit
             while (x) {
                 const int bit = __ffs(x) - 1;
                 x &= x - 1u;
@@ -675,14 +676,18 @@ __device__ int fast_emit_bitmap(const Src &src, unsigned long long K, int bound,
             }
         }
         if (out_score) {
-            __syncthreads();  // every word's rank is recorded; the bitmap is intact
+            __syncthreads();  // every block's rank is recorded; the bitmap is intact
+            const int lg = 31 - __clz(per);
             for (int i = tid; i < src.n; i += kFT) {
                 const unsigned long long kk = src.key(i);
                 if (kk != 0ull && kk >= K) {
                     const int p = key_pos(kk) - c0;
                     if (p >= 0 && p < kChunkBits) {
-                        const int w = emit_word(p >> 5, per);
-                        const unsigned rk = wpre[w] + __popc(bm[w] & ((1u << (p & 31)) - 1u));
+                        // rank = the block's first rank + the bits before p in its block:
+                        // the block's earlier words sit 32, 64, .. words below
+                        const int L = p >> 5, w = emit_word(L, per);
+                        unsigned rk = sh.blkpre[L >> lg] + __popc(bm[w] & ((1u << (p & 31)) - 1u));
+                        for (int t = 1; t <= (L & (per - 1)); ++t) rk += __popc(bm[w - 32 * t]);
                         if (base + (int)rk < k) ps[base + rk] = ord_score(key_ord(kk));
                     }
                 }
@@ -778,10 +783,90 @@ __device__ __forceinline__ unsigned warp_min_u(unsigned v) {
     return v;
 }
 
-// Top-k of a candidate row (keys at or above `floor_ord`, positions <= bound).
+// Outputs of the cutoff margin of a row (adaptive budget), or km = 0.
+struct MarginOut {
+    int km;          // the budget k whose margin is taken (< the row's k_sel)
+    float *sigma;    // this row's sigma
+    unsigned *vk;    // ord of s_(km-1)
+    int *need;       // ties of s_(km-1) the top-km keeps
+};
+
+// Cutoff margin over the row's top-k_sel (the nsel keys >= K of src, every
+// key of src at or above lo_ord, the largest hi_ord) ("Uncertainty-gated
+// selection for block-sparse attention", Section 3 Method, steps 3-4):
+// s_(0) = the largest score, s_(km-1) = the km-th largest, s_(km) = the
+// (km+1)-th; sigma = (s_(km-1) - s_(km)) / (s_(0) - s_(km)) in fp32, 0 when
+// the denominator is 0, NaN when the row has at most km entries.  Also the
+// ord of s_(km-1) and how many of its ties the top-km keeps (the lowest
+// positions, as the top-k rule ranks them).
+template <class Src>
+__device__ void fast_margin(const Src &src, unsigned long long K, int nsel, unsigned lo_ord, unsigned hi_ord,
+                            const MarginOut &m, FastShared &sh) {
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    if (nsel < m.km + 1) {
+        if (tid == 0) {
+            *m.sigma = __uint_as_float(0x7FC00000u);  // quiet NaN: no (km+1)-th score
+            *m.vk = 0u;
+            *m.need = 0;
+        }
+        return;
+    }
+    sh.hist[0][tid] = 0u;
+    __syncthreads();
+    // the key with exactly km keys >= it (a bin edge, not always a key)
+    const unsigned long long Km = fast_kth(src, sh, (unsigned)m.km, lo_ord, hi_ord);
+    // one pass over the top-k_sel: among the top-km, the smallest ord
+    // (s_(km-1)) and how many keys hold it (the ties the top-km keeps); below
+    // them, the largest ord (s_(km): the (km+1)-th key, a tie or not)
+    unsigned mn = 0xFFFFFFFFu, nmn = 0u, below = 0u;
+    for (int i = tid; i < src.n; i += kFT) {
+        const unsigned long long kk = src.key(i);
+        if (kk != 0ull && kk >= K) {
+            const unsigned o = key_ord(kk);
+            if (kk >= Km) {
+                nmn = o < mn ? 1u : (o == mn ? nmn + 1u : nmn);
+                mn = o < mn ? o : mn;
+            } else {
+                below = o > below ? o : below;
+            }
+        }
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+        const unsigned om = __shfl_xor_sync(0xFFFFFFFFu, mn, off);
+        const unsigned on = __shfl_xor_sync(0xFFFFFFFFu, nmn, off);
+        nmn = om < mn ? on : (om == mn ? nmn + on : nmn);
+        mn = om < mn ? om : mn;
+    }
+    below = __reduce_max_sync(0xFFFFFFFFu, below);
+    if (lane == 0) {
+        sh.hist[1][warp] = mn;
+        sh.hist[1][kFWarps + warp] = nmn;
+        sh.hist[1][2 * kFWarps + warp] = below;
+    }
+    __syncthreads();
+    if (tid == 0) {
+        unsigned v1 = 0xFFFFFFFFu, ties = 0u, v2 = 0u;
+#pragma unroll
+        for (int w = 0; w < kFWarps; ++w) {
+            const unsigned om = sh.hist[1][w], on = sh.hist[1][kFWarps + w], ob = sh.hist[1][2 * kFWarps + w];
+            ties = om < v1 ? on : (om == v1 ? ties + on : ties);
+            v1 = om < v1 ? om : v1;
+            v2 = ob > v2 ? ob : v2;
+        }
+        const float f0 = ord_score(hi_ord), f1 = ord_score(v1), f2 = ord_score(v2);
+        const float num = f1 - f2, den = f0 - f2;
+        *m.sigma = den > 0.0f ? num / den : 0.0f;
+        *m.vk = v1;
+        *m.need = (int)ties;
+    }
+}
+
+// Top-k of a candidate row (keys at or above `floor_ord`, positions <= bound),
+// and its cutoff margin when m.km > 0.
 __device__ void fast_cand_row(const unsigned long long *buf, int n, unsigned floor_ord, int bound, int k,
                               int *out_idx, float *out_score, FastShared &sh, unsigned long long *stage,
-                              int stage_cap, unsigned *bm, unsigned *wpre) {
+                              int stage_cap, unsigned *bm, const MarginOut &m) {
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const GCand g{buf, n, (unsigned long long)floor_ord << 32, 0xFFFFFFFFu - (unsigned)bound};
     if (tid == 0) {
@@ -865,7 +950,8 @@ __device__ void fast_cand_row(const unsigned long long *buf, int n, unsigned flo
     const int tail_words = used < stage_cap ? 2 * (stage_cap - used) : 0;
     if (ns <= k) {
         const SStage s{stage, ns};
-        nsel = fast_emit_bitmap(s, 1ull, bound, k, out_idx, out_score, sh, bm, tail, tail_words, wpre, true);
+        nsel = fast_emit_bitmap(s, 1ull, bound, k, out_idx, out_score, sh, bm, tail, tail_words, true);
+        if (m.km) fast_margin(s, 1ull, nsel, floor_ord, hi, m, sh);
     } else if (ns <= stage_cap) {
         const SStage s{stage, ns};
         // the first digit's histogram is in hist[0]: find its bin, then refine
@@ -899,7 +985,8 @@ __device__ void fast_cand_row(const unsigned long long *buf, int n, unsigned flo
             __syncthreads();
             K = fast_kth(s, sh, (unsigned)k, floor_ord, hi);
         }
-        nsel = fast_emit_bitmap(s, K, bound, k, out_idx, out_score, sh, bm, tail, tail_words, wpre, true);
+        nsel = fast_emit_bitmap(s, K, bound, k, out_idx, out_score, sh, bm, tail, tail_words, true);
+        if (m.km) fast_margin(s, K, nsel, floor_ord, hi, m, sh);
     } else {
         // more entries at or above the floor than the stage holds: the same
         // steps over the row in global memory (the whole stage is free)
@@ -907,7 +994,8 @@ __device__ void fast_cand_row(const unsigned long long *buf, int n, unsigned flo
         __syncthreads();
         const unsigned long long K = fast_kth(g, sh, (unsigned)k, floor_ord, hi);
         nsel = fast_emit_bitmap(g, K, bound, k, out_idx, out_score, sh, bm, reinterpret_cast<unsigned *>(stage),
-                                2 * stage_cap, wpre);
+                                2 * stage_cap);
+        if (m.km) fast_margin(g, K, nsel, floor_ord, hi, m, sh);
     }
     fast_pad(nsel, k, out_idx, out_score);
 }
@@ -916,7 +1004,7 @@ __device__ void fast_cand_row(const unsigned long long *buf, int n, unsigned flo
 // -1 = none), masked to positions <= bound.
 __device__ void fast_member_row(const float *sc, const int *pos, int n, int bound, int k, int *out_idx,
                                 float *out_score, FastShared &sh, unsigned long long *stage, int stage_cap,
-                                unsigned *bm, unsigned *wpre) {
+                                unsigned *bm) {
     const int tid = threadIdx.x, lane = tid & 31;
     const GScore g{sc, pos, n, bound};
     if (tid == 0) {
@@ -973,7 +1061,7 @@ __device__ void fast_member_row(const float *sc, const int *pos, int n, int boun
     } else {
         const unsigned long long K = nv <= (unsigned)k ? 1ull : fast_kth(g, sh, (unsigned)k, lo, hi);
         nsel = fast_emit_bitmap(g, K, bound, k, out_idx, out_score, sh, bm, reinterpret_cast<unsigned *>(stage),
-                                2 * stage_cap, wpre);
+                                2 * stage_cap);
     }
     fast_pad(nsel, k, out_idx, out_score);
 }
@@ -985,39 +1073,50 @@ __global__ void __launch_bounds__(kFT, 4) select_fast_kernel(SelectArgs a) {
     unsigned *bm = reinterpret_cast<unsigned *>(fast_smem);
     unsigned long long *stage = fast_smem + kChunkWords / 2;
     const int scap = a.stage_cap;
-    // per-word ranks of the bitmap walk, for the scores (when they are output)
-    unsigned *wpre = a.out_score ? reinterpret_cast<unsigned *>(stage + scap) : nullptr;
     int *oi = a.out_idx + (long long)row * a.k;
     float *os = a.out_score ? a.out_score + (long long)row * a.k : nullptr;
     // per-row scratch of prefill calls starts at the call's first scored row
     // (plan[6]); member scores at the first member of that row (plan[8])
     const long long p0 = a.kind == SEL_DEC_MEMBER ? 0 : a.plan[6];
-    auto cand = [&](long long r, int bound, int k) {
+    // the cutoff margin of dense rows (adaptive budget), per output row
+    const MarginOut mo = a.kind == SEL_DENSE_CAND && a.kmargin > 0
+                             ? MarginOut{a.kmargin, a.m_sigma + row, a.m_vk + row, a.m_need + row}
+                             : MarginOut{0, nullptr, nullptr, nullptr};
+    auto cand = [&](long long r, int bound, int k, const MarginOut &m) {
         const long long sr = r - p0;
         const unsigned n = a.cnt[sr];
         fast_cand_row(a.buf + sr * a.cap, (int)(n < a.cap ? n : a.cap), a.floor ? a.floor[sr] : 0u, bound, k, oi, os,
-                      sh, stage, scap, bm, os ? wpre : nullptr);
+                      sh, stage, scap, bm, m);
     };
+    const MarginOut none{0, nullptr, nullptr, nullptr};
     switch (a.kind) {
     case SEL_DENSE_CAND:
     case SEL_REUSE_CAND:
     case SEL_MEMBER_SCORES: {
-        if (!a.plan[0]) { fast_pad(0, a.k, oi, os); return; }
+        if (!a.plan[0]) {
+            fast_pad(0, a.k, oi, os);
+            if (mo.km && threadIdx.x == 0) {
+                *mo.sigma = __uint_as_float(0x7FC00000u);
+                *mo.vk = 0u;
+                *mo.need = 0;
+            }
+            return;
+        }
         if (row < a.plan[4] || row >= a.plan[5]) return;  // not an output row of this call
         const int b = find_seg(a.cu, a.S, row);
         const int t = row - a.cu[b];
         if (a.kind == SEL_DENSE_CAND) {
-            cand(row, t, a.k);
+            cand(row, t, a.k, mo);
         } else {
             const int n = a.cu[b + 1] - a.cu[b];
             const int p = a.plan[a.pl.rp() + b] + group_of(t, n, a.g, a.db);
             // Reuse, and members scored on their own (guardrail): the top-k of
             // the scored row's candidates inside the member's prefix
             if (a.kind == SEL_REUSE_CAND || t < dense_rows(n, a.g, a.db))
-                cand(p, t, a.k);
+                cand(p, t, a.k, none);
             else
                 fast_member_row(a.scores + ((long long)row - a.plan[8]) * a.ld, a.cand + (p - p0) * a.c, a.c, t,
-                                a.k, oi, os, sh, stage, scap, bm, os ? wpre : nullptr);
+                                a.k, oi, os, sh, stage, scap, bm);
         }
         return;
     }
@@ -1036,7 +1135,7 @@ __global__ void __launch_bounds__(kFT, 4) select_fast_kernel(SelectArgs a) {
             if (i < dense_rows(n, a.g, a.db)) return;
             oi = po;
             os = nullptr;
-            cand(row, row_bound(i, n, a.g, a.db), a.k);
+            cand(row, row_bound(i, n, a.g, a.db), a.k, none);
             return;
         }
         const int tl = row_bound(i, n, a.g);
@@ -1045,7 +1144,7 @@ __global__ void __launch_bounds__(kFT, 4) select_fast_kernel(SelectArgs a) {
         if (kr > 0) {
             oi = po;
             os = nullptr;
-            cand(row, key_bound(tl, kBlockShift), kr);
+            cand(row, key_bound(tl, kBlockShift), kr, none);
         }
         for (int r = (kr > 0 ? kr : 0) + (int)threadIdx.x; r < a.k; r += kFT) po[r] = -1;
         return;
@@ -1059,7 +1158,7 @@ __global__ void __launch_bounds__(kFT, 4) select_fast_kernel(SelectArgs a) {
             return;
         }
         fast_member_row(a.scores + (long long)row * a.ld, a.cand + (long long)b * a.c, a.c, kv - a.G + m, a.k, oi,
-                        os, sh, stage, scap, bm, os ? wpre : nullptr);
+                        os, sh, stage, scap, bm);
         return;
     }
     default:
@@ -1086,11 +1185,10 @@ cudaError_t launch_select_fast(const SelectArgs &a, cudaStream_t st) {
     if (member && a.c > room) room = a.c;
     if (room < kFastMinRoom) room = kFastMinRoom;
     room = (room + 255) / 256 * 256;
-    const size_t wpre_bytes = a.out_score ? (size_t)kChunkWords * 4 : 0;  // per-word ranks
-    const size_t limit = 232448 - sizeof(FastShared) - 1024 - (size_t)kChunkWords * 4 - wpre_bytes;
+    const size_t limit = 232448 - sizeof(FastShared) - 1024 - (size_t)kChunkWords * 4;
     if ((size_t)room * 8 > limit) room = (long long)(limit / 8) & ~1LL;
     b.stage_cap = (int)room;
-    const size_t smem = (size_t)kChunkWords * 4 + (size_t)room * 8 + wpre_bytes;
+    const size_t smem = (size_t)kChunkWords * 4 + (size_t)room * 8;
     cudaError_t e = cudaFuncSetAttribute(select_fast_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     TraceScope ts("select", st);
