@@ -139,22 +139,26 @@ AdaptiveWs adaptive_ws(int T, int H, int d, int topk, int rho, int S, idx_dtype 
 }
 
 struct DecodeWs {
-    size_t status, qbar, wbar, spill, cand, msc, ckeys, total;
+    size_t status, qbar, wbar, spill, cand, msc, ckeys, nlen, cblk, total;
 };
 
+// mode BLOCK: the decode block pre-filter (the proxy scans block means, then
+// the members re-score the chosen blocks' keys as in Refine)
 DecodeWs decode_ws(int B, int G, int n_max, int H, int d, int c, idx_mode mode, idx_dtype dt) {
     DecodeWs L{};
     Carve cv;
+    const bool blocks = mode == IDX_MODE_BLOCK, sets = mode == IDX_MODE_REFINE || blocks;
     const int rows = mode == IDX_MODE_DENSE ? B * G : B;
     L.status = cv.take(16);
     L.qbar = mode != IDX_MODE_DENSE ? cv.take((size_t)B * H * d * esize(dt)) : 0;
     L.wbar = mode != IDX_MODE_DENSE ? cv.take((size_t)B * H * 4) : 0;
-    L.spill = cv.take((size_t)rows * n_max * 4);
-    L.cand = mode == IDX_MODE_REFINE ? cv.take((size_t)B * c * 4) : 0;
-    L.msc = mode == IDX_MODE_REFINE ? cv.take((size_t)B * G * c * 4) : 0;
-    L.ckeys = (mode == IDX_MODE_REFINE && tc_gather_supported(H, d, (int)dt, G, c))
-                  ? cv.take((size_t)B * c_pad_of(c) * d * esize(dt))
-                  : 0;
+    L.spill = cv.take((size_t)rows * (blocks ? n_max >> kBlockShift : n_max) * 4);
+    L.cand = sets ? cv.take((size_t)B * c * 4) : 0;
+    L.msc = sets ? cv.take((size_t)B * G * c * 4) : 0;
+    L.ckeys = (sets && tc_gather_supported(H, d, (int)dt, G, c)) ? cv.take((size_t)B * c_pad_of(c) * d * esize(dt))
+                                                                 : 0;
+    L.nlen = blocks ? cv.take((size_t)B * 4) : 0;
+    L.cblk = blocks ? cv.take((size_t)B * (c >> kBlockShift) * 4) : 0;
     L.total = cv.off;
     return L;
 }
@@ -525,6 +529,7 @@ struct Decode {
     const int *bt = nullptr;  // paged cache: block table [B, max_pages], else NULL
     int page = 0, max_pages = 0;
     long long num_pages = 0;
+    const void *kbar = nullptr;  // block mode: block means [B, n_max / 64, d]
 
     unsigned *status() const { return reinterpret_cast<unsigned *>(ws + L.status); }
 
@@ -585,11 +590,29 @@ idx_status Decode::run(int *out_idx, float *out_score) const {
         return cuda_st(launch_select(sargs(SEL_DEC_DENSE, B * G, topk, out_idx, out_score, spill, n_max), st));
     }
     TRY_CUDA(launch_decode_proxy(q, w, B, G, H, d, (int)dt, ws + L.qbar, reinterpret_cast<float *>(ws + L.wbar), st));
-    TRY_CUDA(scan(dargs(true, spill)));
-    if (mode == IDX_MODE_REUSE)
-        return cuda_st(launch_select(sargs(SEL_DEC_REUSE, B * G, topk, out_idx, out_score, spill, n_max), st));
     int *cand = reinterpret_cast<int *>(ws + L.cand);
-    TRY_CUDA(launch_select(sargs(SEL_DEC_PROXY_TO_C, B, c, cand, nullptr, spill, n_max), st));
+    if (mode == IDX_MODE_BLOCK) {
+        // the proxy against the block means of the complete blocks, then the
+        // chosen blocks (and the partial block) become the candidate set
+        int *nlen = reinterpret_cast<int *>(ws + L.nlen);
+        int *cblk = reinterpret_cast<int *>(ws + L.cblk);
+        TRY_CUDA(launch_decode_block_len(kv, B, G, n_max, nlen, st));
+        DecodeArgs a = dargs(true, spill);
+        a.kc = kbar;
+        a.kv_len = nlen;
+        a.G = 1;
+        a.n_max = n_max >> kBlockShift;
+        TRY_CUDA(scan(a));
+        TRY_CUDA(launch_select(sargs(SEL_DEC_PROXY_TO_BLOCKS, B, c >> kBlockShift, cblk, nullptr, spill,
+                                     n_max >> kBlockShift),
+                               st));
+        TRY_CUDA(launch_decode_block_expand(kv, B, G, n_max, cblk, cand, c, st));
+    } else {
+        TRY_CUDA(scan(dargs(true, spill)));
+        if (mode == IDX_MODE_REUSE)
+            return cuda_st(launch_select(sargs(SEL_DEC_REUSE, B * G, topk, out_idx, out_score, spill, n_max), st));
+        TRY_CUDA(launch_select(sargs(SEL_DEC_PROXY_TO_C, B, c, cand, nullptr, spill, n_max), st));
+    }
     const GatherArgs ga = gargs();
     TRY_CUDA(tc_gather_supported(H, d, (int)dt, G, c) ? launch_gather_tc(ga, st)
                                                      : launch_gather_simt(ga, (int)dt, st));
@@ -645,6 +668,49 @@ idx_status idx_decode_paged_topk(const void *q, const void *kpool, const int *bl
     D.page = page;
     D.max_pages = max_pages;
     D.num_pages = num_pages;
+    return D.run(out_idx, out_score);
+}
+
+namespace {
+
+idx_status check_decode_block(int B, int G, int n_max, int H, int d, int topk, int c, idx_dtype dt) {
+    if (B < 1 || G < 1 || n_max < G || topk < 1 || !shape_ok(H, d, dt)) return IDX_ERR_INVALID;
+    if (n_max % kBlockN != 0 || c < topk || c < kBlockN || c % kBlockN != 0) return IDX_ERR_INVALID;
+    if (G > RB || n_max > kMaxLen || !path_ok(H, d, dt)) return IDX_ERR_UNSUPPORTED;
+    return IDX_OK;
+}
+
+}  // namespace
+
+size_t idx_decode_block_workspace_size(int B, int G, int n_max, int H, int d, int topk, int c, idx_dtype dtype) {
+    if (check_decode_block(B, G, n_max, H, d, topk, c, dtype) != IDX_OK) return 0;
+    return decode_ws(B, G, n_max, H, d, c, IDX_MODE_BLOCK, dtype).total;
+}
+
+idx_status idx_decode_block_means(const void *kcache, int B, int n_max, int d, idx_dtype dtype, int first_block,
+                                  void *kbar, idx_stream_t stream) {
+    if (!kcache || !kbar || B < 1 || n_max < kBlockN || n_max % kBlockN != 0 || first_block < 0 ||
+        !shape_ok(1, d, dtype))
+        return IDX_ERR_INVALID;
+    if (n_max > kMaxLen) return IDX_ERR_UNSUPPORTED;
+    TracePhase phase("decode_block");
+    return cuda_st(launch_decode_block_means(kcache, B, n_max, d, (int)dtype, first_block, kbar,
+                                             reinterpret_cast<cudaStream_t>(stream)));
+}
+
+idx_status idx_decode_block_topk(const void *q, const void *kcache, const void *kbar, const int *kv_len,
+                                 const float *w, int B, int G, int n_max, int H, int d, int topk, int c,
+                                 idx_dtype dtype, int *out_idx, float *out_score, void *ws, size_t ws_bytes,
+                                 idx_stream_t stream) {
+    if (!q || !kcache || !kbar || !kv_len || !w || !out_idx) return IDX_ERR_INVALID;
+    idx_status s = check_decode_block(B, G, n_max, H, d, topk, c, dtype);
+    if (s != IDX_OK) return s;
+    const size_t need = decode_ws(B, G, n_max, H, d, c, IDX_MODE_BLOCK, dtype).total;
+    if (!ws || (reinterpret_cast<uintptr_t>(ws) % kAlign) != 0 || ws_bytes < need) return IDX_ERR_WORKSPACE;
+    TracePhase phase("decode_block");
+    Decode D{q, kcache, kv_len, w, B, G, n_max, H, d, topk, c, IDX_MODE_BLOCK, dtype, static_cast<char *>(ws),
+             decode_ws(B, G, n_max, H, d, c, IDX_MODE_BLOCK, dtype), reinterpret_cast<cudaStream_t>(stream)};
+    D.kbar = kbar;
     return D.run(out_idx, out_score);
 }
 

@@ -141,8 +141,9 @@ enum SelKind {
     SEL_DEC_REUSE = 5,      // decode: proxy spill row b restricted to member m
     SEL_DEC_PROXY_TO_C = 6, // decode: candidate set of request b
     SEL_DEC_MEMBER = 7,     // decode: member scores over the candidate set
-    SEL_PROXY_TO_BLOCKS = 8 // block pre-filter: complete blocks of a proxy row (k = c / kBlockN, one
-                            // fewer when the row's prefix ends inside a block), block indices only
+    SEL_PROXY_TO_BLOCKS = 8, // block pre-filter: complete blocks of a proxy row (k = c / kBlockN, one
+                             // fewer when the row's prefix ends inside a block), block indices only
+    SEL_DEC_PROXY_TO_BLOCKS = 9 // decode block mode: the same over request b's block-score spill row
 };
 
 struct SelectArgs {
@@ -251,6 +252,13 @@ cudaError_t launch_block_expand(const int *cu, int S, int g, const int *plan, co
                                 const int *cblk, int *cand, int c, int R, cudaStream_t st);
 cudaError_t launch_decode_proxy(const void *q, const float *w, int B, int G, int H, int d, int dtype,
                                 void *qbar, float *wbar, cudaStream_t st);
+// decode block mode: block means of a cache [B, n_max, d] (blocks >= first_block),
+// the complete blocks per request, and candidate positions from the selected blocks
+cudaError_t launch_decode_block_means(const void *kc, int B, int n_max, int d, int dtype, int first_block,
+                                      void *kbar, cudaStream_t st);
+cudaError_t launch_decode_block_len(const int *kv_len, int B, int G, int n_max, int *nlen, cudaStream_t st);
+cudaError_t launch_decode_block_expand(const int *kv_len, int B, int G, int n_max, const int *cblk, int *cand,
+                                       int c, cudaStream_t st);
 size_t simt_smem_bytes(int H, int d, int dtype);
 bool tc_supported(int H, int d, int dtype);
 bool tc_decode_supported(int H, int d, int dtype, int rows_per_request);

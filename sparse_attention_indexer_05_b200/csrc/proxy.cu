@@ -148,6 +148,76 @@ __global__ void __launch_bounds__(kProxyThreads) block_mean_kernel(const T *k, c
     Vec<T>::store(kb + x * d + e, acc);
 }
 
+// Block means of a decode cache kc [B, n_max, d] (n_max a multiple of 64):
+// block j of request b (rows 64 j .. 64 j + 63) to row b * (n_max / 64) + j
+// of kbar, for blocks j >= first_block only (an update after appends), with
+// the same arithmetic as block_mean_kernel.  Rows past a request's kv_len
+// take part like any other: only the blocks below kv_len / 64 are ever read
+// by the decode block scan.  One thread per 8 dimensions of one block row.
+template <typename T>
+__global__ void __launch_bounds__(kProxyThreads) decode_block_mean_kernel(const T *kc, int B, int n_max, int d,
+                                                                          int first_block, T *kbar) {
+    const int per_row = d / 8;
+    const int nb = n_max >> kBlockShift, nu = nb - first_block;
+    const long long u = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    if (nu <= 0 || u >= (long long)B * nu * per_row) return;
+    const long long x = u / per_row;  // (request, block) pair
+    const int e = (int)(u - x * per_row) * 8;
+    const int b = (int)(x / nu), j = first_block + (int)(x - (long long)b * nu);
+    const T *src = kc + ((long long)b * n_max + (long long)j * kBlockN) * d + e;
+    float acc[8], v[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) acc[i] = 0.0f;
+    for (int r = 0; r < kBlockN; ++r) {
+        Vec<T>::load(src + (long long)r * d, v);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) acc[i] = __fadd_rn(acc[i], v[i]);
+    }
+#pragma unroll
+    for (int i = 0; i < 8; ++i) acc[i] = __fdiv_rn(acc[i], (float)kBlockN);
+    Vec<T>::store(kbar + ((long long)b * nb + j) * d + e, acc);
+}
+
+// Decode block mode: the complete blocks each request's proxy scans,
+// kv_len[b] / 64 (0 for a request whose kv_len is out of range; the block
+// select flags it).
+__global__ void decode_block_len_kernel(const int *kv_len, int B, int G, int n_max, int *nlen) {
+    const int b = blockIdx.x * blockDim.x + threadIdx.x;
+    if (b >= B) return;
+    const int kv = kv_len[b];
+    nlen[b] = (kv < G || kv > n_max) ? 0 : kv >> kBlockShift;
+}
+
+// Decode block mode: candidate set of request b from its selected blocks
+// cblk [B, c / 64] (ascending, -1 padded) and the partial block that holds
+// the last query (position kv_len[b] - 1), as block_expand_kernel does for
+// a prefill proxy.
+__global__ void __launch_bounds__(kProxyThreads) decode_block_expand_kernel(const int *kv_len, int G, int n_max,
+                                                                            const int *cblk, int *cand, int c) {
+    const int b = blockIdx.x;
+    const int kv = kv_len[b];
+    int *out = cand + (long long)b * c;
+    const int nb = c >> kBlockShift;
+    const bool ok = kv >= G && kv <= n_max;
+    const int tl = kv - 1;
+    const int part0 = (tl + 1) & ~(kBlockN - 1);
+    const bool partial = ok && part0 <= tl;
+    const int *sel = cblk + (long long)b * nb;
+    for (int j = threadIdx.x; j < c; j += blockDim.x) {
+        const int slot = j >> kBlockShift, r = j & (kBlockN - 1);
+        int v = -1;
+        if (ok) {
+            if (partial && slot == nb - 1) {
+                v = part0 + r <= tl ? part0 + r : -1;
+            } else {
+                const int blk = sel[slot];
+                v = blk >= 0 ? blk * kBlockN + r : -1;
+            }
+        }
+        out[j] = v;
+    }
+}
+
 // Candidate set of each proxy row in block mode: slot j of cblk [R, nb]
 // (a selected block, or -1) expands to the 64 positions of that block; the
 // partial block that holds the proxy's last member t_last fills the last
@@ -220,6 +290,34 @@ cudaError_t launch_proxy(const void *q, const float *w, const int *cu, int S, in
     else
         proxy_kernel<__nv_bfloat16><<<max_proxies, kProxyThreads, 0, st>>>(
             (const __nv_bfloat16 *)q, w, cu, S, H, d, g, db, plan, pl, (__nv_bfloat16 *)qbar, wbar);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_decode_block_means(const void *kc, int B, int n_max, int d, int dtype, int first_block,
+                                      void *kbar, cudaStream_t st) {
+    const int nu = (n_max >> kBlockShift) - first_block;
+    if (B <= 0 || nu <= 0) return cudaSuccess;
+    const long long units = (long long)B * nu * (d / 8);
+    const unsigned grid = (unsigned)((units + kProxyThreads - 1) / kProxyThreads);
+    TraceScope ts("block_means", st);
+    if (dtype == 1)
+        decode_block_mean_kernel<float><<<grid, kProxyThreads, 0, st>>>((const float *)kc, B, n_max, d, first_block,
+                                                                        (float *)kbar);
+    else
+        decode_block_mean_kernel<__nv_bfloat16><<<grid, kProxyThreads, 0, st>>>(
+            (const __nv_bfloat16 *)kc, B, n_max, d, first_block, (__nv_bfloat16 *)kbar);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_decode_block_len(const int *kv_len, int B, int G, int n_max, int *nlen, cudaStream_t st) {
+    decode_block_len_kernel<<<(B + 127) / 128, 128, 0, st>>>(kv_len, B, G, n_max, nlen);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_decode_block_expand(const int *kv_len, int B, int G, int n_max, const int *cblk, int *cand,
+                                       int c, cudaStream_t st) {
+    TraceScope ts("block_expand", st);
+    decode_block_expand_kernel<<<B, kProxyThreads, 0, st>>>(kv_len, G, n_max, cblk, cand, c);
     return cudaGetLastError();
 }
 

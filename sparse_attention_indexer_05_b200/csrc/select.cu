@@ -406,6 +406,27 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(SelectArgs a) {
         }
         return;
     }
+    case SEL_DEC_PROXY_TO_BLOCKS: {
+        // the proxy's top blocks among request b's complete blocks: k = c / 64
+        // slots, one of them kept for the partial block when kv_len[b] ends
+        // inside a block; the slots not taken are -1
+        const int b = row;
+        const int kv = a.kv_len[b];
+        if (kv < a.G || kv > a.n_max) {
+            if (threadIdx.x == 0) raise_status(a.status, ST_INVALID);
+            pad_all();
+            return;
+        }
+        const int nfull = kv >> kBlockShift;
+        const int want = a.k - ((kv & (kBlockN - 1)) != 0 ? 1 : 0);
+        const int take = want < nfull ? want : nfull;
+        if (take > 0) {
+            ScoreSrc src{a.scores + (long long)b * a.ld, nullptr, nfull, nfull - 1};
+            block_select(src, take, oi, nullptr, sh, stage, a.stage_cap, bm, gpre, wcap, a.status);
+        }
+        for (int r = (take > 0 ? take : 0) + threadIdx.x; r < a.k; r += blockDim.x) oi[r] = -1;
+        return;
+    }
     default:  // the other kinds run in select_fast_kernel
         return;
     }

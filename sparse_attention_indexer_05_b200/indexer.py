@@ -202,6 +202,40 @@ def decode_paged_topk(q, kpool, block_table, kv_len, w, topk: int, c: int = 0, m
     return (out_idx, out_score) if return_scores else out_idx
 
 
+def decode_block_means(kcache, kbar=None, first_block: int = 0, stream=None):
+    """Block means [B, n_max/64, d] of a decode cache kcache [B, n_max, d]
+    (n_max a multiple of 64); blocks >= first_block are (re)written."""
+    B, n_max, d = kcache.shape
+    if kbar is None:
+        kbar = torch.empty(B, n_max // 64, d, dtype=kcache.dtype, device=kcache.device)
+    N.check(N.lib().idx_decode_block_means(_dev(kcache, "kcache"), B, n_max, d, _dtype_code(kcache), first_block,
+                                           _dev(kbar, "kbar", kcache.dtype), _stream(stream)),
+            "idx_decode_block_means")
+    return kbar
+
+
+def decode_block_workspace_size(B, G, n_max, H, d, topk, c, dtype=torch.bfloat16) -> int:
+    dt = N.BF16 if dtype == torch.bfloat16 else N.F32
+    return int(N.lib().idx_decode_block_workspace_size(B, G, n_max, H, d, topk, c, dt))
+
+
+def decode_block_topk(q, kcache, kbar, kv_len, w, topk: int, c: int, out_idx=None, out_score=None, workspace=None,
+                      stream=None, return_scores=False):
+    """One decode step with the block pre-filter: q [B,G,H,d], kcache [B,n_max,d],
+    kbar [B,n_max/64,d] (decode_block_means), kv_len int32 [B], w [B,G,H]."""
+    B, G, H, d = q.shape
+    n_max = kcache.shape[1]
+    dt = _dtype_code(q)
+    ws = _ws(workspace, decode_block_workspace_size(B, G, n_max, H, d, topk, c, q.dtype), q.device)
+    out_idx, out_score = _outs((B, G), topk, q.device, out_idx, out_score, return_scores)
+    N.check(N.lib().idx_decode_block_topk(
+        _dev(q, "q"), _dev(kcache, "kcache", q.dtype), _dev(kbar, "kbar", q.dtype), _dev(kv_len, "kv_len", torch.int32),
+        _dev(w, "w", torch.float32), B, G, n_max, H, d, topk, c, dt, _dev(out_idx, "out_idx", torch.int32),
+        _dev(out_score, "out_score", torch.float32) if out_score is not None else None,
+        ws.data_ptr(), ws.numel(), _stream(stream)), "idx_decode_block_topk")
+    return (out_idx, out_score) if return_scores else out_idx
+
+
 def sparse_attn(q, kv, idx, cu_q, cu_kv, scale: float, out=None, lse=None, workspace=None, stream=None,
                 return_lse=False):
     """Token-sparse attention over the selected positions: q [R,H,576] bf16,

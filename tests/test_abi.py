@@ -26,7 +26,7 @@ def declared_functions():
 
 def test_exports_every_declared_symbol(lib):
     names = declared_functions()
-    assert len(names) == 25
+    assert len(names) == 28
     for n in names:
         assert hasattr(lib, n), n
         assert n in N.SIGNATURES, n
@@ -151,3 +151,39 @@ def test_sparse_attn_argument_checks(lib):
     assert call(H=256) == 2                        # more heads than the MMA's M
     assert call(ws_bytes=16) == 3                  # workspace too small
     assert call(ws=ctypes.c_void_p(264)) == 3      # misaligned workspace
+
+
+def test_decode_block_workspace_and_argument_checks(lib):
+    size = lib.idx_decode_block_workspace_size
+    ok = size(64, 2, 131072, 64, 128, 2048, 4096, 0)
+    assert ok > 0
+    # the block-score spill is a 64th of the token-score one
+    assert ok < lib.idx_decode_workspace_size(64, 2, 131072, 64, 128, 2048, 4096, 2, 0)
+    assert size(64, 2, 131072 - 1, 64, 128, 2048, 4096, 0) == 0    # n_max not a multiple of 64
+    assert size(64, 2, 131072, 64, 128, 2048, 4096 + 32, 0) == 0   # c not a multiple of 64
+    assert size(64, 2, 131072, 64, 128, 2048, 1024, 0) == 0        # c < topk
+    assert size(64, 9, 131072, 64, 128, 2048, 4096, 0) == 0        # G above one row block
+    fake = 256  # never dereferenced: the checks fail before any launch
+    f = lib.idx_decode_block_topk
+    args = [fake, fake, fake, fake, fake, 4, 2, 4096, 64, 128, 64, 128, 0, fake, None, fake, 1 << 40, None]
+    for i in (0, 1, 2, 3, 4, 13):  # q, kcache, kbar, kv_len, w, out_idx
+        a = list(args)
+        a[i] = None
+        assert f(*a) == 1, i
+    a = list(args)
+    a[11] = 96                      # c not a multiple of 64
+    assert f(*a) == 1
+    a = list(args)
+    a[7] = 4000                     # n_max not a multiple of 64
+    assert f(*a) == 1
+    a = list(args)
+    a[6] = 9                        # G > 8
+    assert f(*a) == 2
+    a = list(args)
+    a[16] = 16                      # workspace too small
+    assert f(*a) == 3
+    m = lib.idx_decode_block_means
+    assert m(None, 4, 4096, 128, 0, 0, fake, None) == 1
+    assert m(fake, 4, 4000, 128, 0, 0, fake, None) == 1   # n_max not a multiple of 64
+    assert m(fake, 4, 4096, 12, 0, 0, fake, None) == 1    # d % 8 != 0
+    assert m(fake, 4, 4096, 128, 0, -1, fake, None) == 1  # negative first block

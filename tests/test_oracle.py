@@ -522,13 +522,41 @@ def pin_gaussian_mean_score():
     assert abs(tot / pred - 1.0) < 0.05, tot / pred
 
 
+def pin_decode_block_full_budget_is_dense():
+    """Decode block mode whose budget covers every block of the cache (and the
+    partial one) gives every query its whole prefix as candidates: the dense
+    decode top-k; a budget of one block with kv_len inside a block gives the
+    partial block's positions up to each query."""
+    rng = np.random.default_rng(41)
+    B, G, H, d, n_max, bn = 4, 2, 4, 16, 256, 64
+    kc = _bf(rng.standard_normal((B, n_max, d)))
+    qd = _bf(rng.standard_normal((B, G, H, d)))
+    wd = rng.random((B, G, H)).astype(np.float32)
+    kv = np.array([256, 130, 64, 7], np.int32)
+    dense = O.decode_topk(qd, kc, wd, kv, 9, 0, O.DENSE)
+    blk = O.decode_topk(qd, kc, wd, kv, 9, n_max + bn, O.BLOCK, bn=bn)
+    assert np.array_equal(blk, dense)
+    kv1 = np.array([200, 130, 71, 7], np.int32)
+    one = O.decode_topk(qd, kc, wd, kv1, 9, bn, O.BLOCK, bn=bn)
+    for b in range(B):
+        part0 = (kv1[b] // bn) * bn
+        for m in range(G):
+            t = kv1[b] - G + m
+            want = list(range(part0, t + 1))[:9] if t >= part0 else []
+            got = [x for x in one[b, m].tolist() if x >= 0]
+            if t + 1 - part0 <= 9:
+                assert got == want, (b, m, got, want)
+            else:
+                assert len(got) == 9 and all(part0 <= x <= t for x in got)
+
+
 ALL_PINS = [pin_hand_scores, pin_hand_topk, pin_hand_guardrail, pin_guardrail_reductions, pin_hand_decode, pin_bruteforce_dense,
             pin_bruteforce_pivot, pin_exact_integer_inputs, pin_textbook_single_head,
             pin_pivot_special_cases, pin_invariants, pin_reuse_within_proxy_ranking,
             pin_proxy_exact_mean, pin_decode_matches_prefill, pin_gaussian_mean_score,
             pin_block_mean_exact, pin_block_reductions, pin_block_constant_keys_equal_refine,
             pin_block_partial_closed_form, pin_attn_single_entry, pin_attn_equal_logits_mean,
-            pin_attn_library_sdpa, pin_attn_large_logits]
+            pin_attn_library_sdpa, pin_attn_large_logits, pin_decode_block_full_budget_is_dense]
 
 
 @pytest.mark.parametrize("pin", ALL_PINS, ids=[p.__name__ for p in ALL_PINS])
