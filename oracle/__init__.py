@@ -21,7 +21,7 @@ import numpy as np
 from . import build as _build
 
 BF16, F32 = 0, 1
-DENSE, REUSE, REFINE, BLOCK = 0, 1, 2, 3
+DENSE, REUSE, REFINE, BLOCK, QUEST = 0, 1, 2, 3, 4
 
 _libs = {}
 _active = [None]
@@ -165,7 +165,8 @@ def dense_topk(q, k, w, cu_seqlens, topk: int, rows=None, threads=None) -> np.nd
 def pivot_topk(q, k, w, cu_seqlens, topk: int, g: int, c: int, mode: int, rows=None,
                threads=None, bn: int = 64, dense_below: int = 0) -> np.ndarray:
     """PIVOT Reuse (mode=REUSE), Refine (mode=REFINE) or Refine over block
-    pre-filter candidates (mode=BLOCK, block size bn) top-k of member rows.
+    pre-filter candidates (block size bn; blocks ranked by their mean key,
+    mode=BLOCK, or by the Quest min/max bound, mode=QUEST) top-k of member rows.
     Groups whose last member's prefix holds at most dense_below keys take the
     dense top-k (the guardrail; 0 = off)."""
     q = np.ascontiguousarray(q); k = np.ascontiguousarray(k); w = _c(w, np.float32)

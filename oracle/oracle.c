@@ -49,6 +49,17 @@
  *    counts tokens (c / bn blocks, one of them the partial block if there
  *    is one); the mean key is rounded like the proxy (fp32 sum in key order,
  *    IEEE division, bf16 round-to-nearest-even).
+ *  - Block pre-filter with the Quest bound (mode ORA_QUEST): the same
+ *    candidate generator, but a block is summarised by the per-dimension
+ *    minimum and maximum of its keys, and its score for a query is the
+ *    coordinate-wise upper bound of q . k over the block ("Uncertainty-gated
+ *    selection for block-sparse attention", Sec. 3.1, Eq. (2), after Quest):
+ *    sum over dimensions of max(q_d * kmax_d, q_d * kmin_d).  Reading: the
+ *    indexer scores each head's bound as it scores a dot product, so the
+ *    block score is sum_j w_j * max(0, bound_j); everything else (complete
+ *    blocks only, the partial block always a candidate, c / bn blocks) is
+ *    as in ORA_BLOCK.  The minimum and maximum of bf16 keys are bf16 keys:
+ *    no rounding step.
  *  - Token-sparse attention (ora_sparse_attn), the consumer of the selected
  *    sets: the PIVOT page's introduction says the selected set feeds sparse
  *    MLA attention.  The pages give no formula; the reading used here is
@@ -76,7 +87,7 @@
 #include <string.h>
 
 enum { ORA_BF16 = 0, ORA_F32 = 1 };
-enum { ORA_DENSE = 0, ORA_REUSE = 1, ORA_REFINE = 2, ORA_BLOCK = 3 };
+enum { ORA_DENSE = 0, ORA_REUSE = 1, ORA_REFINE = 2, ORA_BLOCK = 3, ORA_QUEST = 4 };
 
 /* ---------------------------------------------------------------- inputs */
 
@@ -221,6 +232,31 @@ static void block_mean(const void *k, int dtype, int d, long long r0, int bn, vo
 }
 
 /* Exported for tests of the block-mean step alone. */
+/* Quest block score of the proxy (qbar [H, d], wbar [H]) for key rows
+ * r0 .. r0+bn-1: per head the coordinate-wise upper bound of q . k over the
+ * block, sum_d max(q_d * kmax_d, q_d * kmin_d), then the indexer's weighted
+ * ReLU over the heads. */
+static double quest_score(const void *qbar, const float *wbar, const void *k, int dtype, int H, int d,
+                          long long r0, int bn) {
+    double total = 0.0;
+    for (int j = 0; j < H; ++j) {
+        double bound = 0.0;
+        for (int i = 0; i < d; ++i) {
+            double lo = load_elem(k, dtype, (size_t)r0 * d + i), hi = lo;
+            for (int r = 1; r < bn; ++r) {
+                double v = load_elem(k, dtype, (size_t)(r0 + r) * d + i);
+                if (v < lo) lo = v;
+                if (v > hi) hi = v;
+            }
+            double qd = load_elem(qbar, dtype, (size_t)j * d + i);
+            double a = qd * hi, b = qd * lo;
+            bound += a > b ? a : b;
+        }
+        if (bound > 0.0) total += (double)wbar[j] * bound;
+    }
+    return total;
+}
+
 int ora_block_mean(const void *k, int dtype, int d, long long r0, int bn, void *kbar) {
     if (!k || !kbar || bn <= 0 || d <= 0) return 1;
     block_mean(k, dtype, d, r0, bn, kbar);
@@ -240,7 +276,7 @@ int ora_group_proxy(const void *q, const float *w, int dtype, int H, int d, long
  *         are pos0 .. pos0+cnt-1 (request-local); the group's last member
  *         sits at t_last = pos0+cnt-1.
  *   keys: key rows key0 + s for s = 0 .. t_last.
- *   mode: ORA_REUSE, ORA_REFINE or ORA_BLOCK; c: candidate budget (Refine,
+ *   mode: ORA_REUSE, ORA_REFINE, ORA_BLOCK or ORA_QUEST; c: candidate budget (Refine,
  *         Block); bn: block size (Block).
  *   member: which member (0..cnt-1) to produce; out: k entries. */
 static int grouped_member_topk(const void *q, const void *k, const float *w, int dtype, int H, int d,
@@ -256,9 +292,10 @@ static int grouped_member_topk(const void *q, const void *k, const float *w, int
     group_proxy(q, w, dtype, H, d, m0, cnt, qbar, wbar);
     int t = pos0 + member;
     int rc = 0;
-    if (mode == ORA_BLOCK) {
+    if (mode == ORA_BLOCK || mode == ORA_QUEST) {
         /* complete blocks [j*bn, (j+1)*bn) inside the prefix, scored by the
-         * proxy against their mean keys; the partial block [part0, n) */
+         * proxy against their mean keys (ORA_BLOCK) or by the Quest bound
+         * (ORA_QUEST); the partial block [part0, n) */
         int nfull = n / bn;
         int part0 = nfull * bn;
         int want = c / bn - (part0 < n ? 1 : 0);
@@ -269,8 +306,12 @@ static int grouped_member_topk(const void *q, const void *k, const float *w, int
         cand_t *mc = (cand_t *)malloc(sizeof(cand_t) * (size_t)n);
         if (!kbar || !mc) { free(kbar); free(mc); rc = 2; goto done; }
         for (int j = 0; j < nfull; ++j) {
-            block_mean(k, dtype, d, key0 + (long long)j * bn, bn, kbar);
-            pc[j].score = index_score(qbar, 0, kbar, 0, wbar, H, d, dtype);
+            if (mode == ORA_QUEST) {
+                pc[j].score = quest_score(qbar, wbar, k, dtype, H, d, key0 + (long long)j * bn, bn);
+            } else {
+                block_mean(k, dtype, d, key0 + (long long)j * bn, bn, kbar);
+                pc[j].score = index_score(qbar, 0, kbar, 0, wbar, H, d, dtype);
+            }
             pc[j].pos = j;
         }
         qsort(pc, (size_t)nfull, sizeof(cand_t), by_score_desc_pos_asc);
@@ -477,9 +518,9 @@ int ora_dense_topk(const void *q, const void *k, const float *w, int dtype, cons
     return run_job(&J, nthreads);
 }
 
-/* PIVOT top-k (mode ORA_REUSE, ORA_REFINE or ORA_BLOCK) for the given
+/* PIVOT top-k (mode ORA_REUSE, ORA_REFINE, ORA_BLOCK or ORA_QUEST) for the given
  * global member rows; same layouts as ora_dense_topk; g >= 1; Refine and
- * Block need c >= topk; Block needs bn >= 1 (c / bn blocks).  Groups whose
+ * Block / Quest need c >= topk and bn >= 1 (c / bn blocks).  Groups whose
  * last member's prefix holds at most dense_below keys (0 = none) take the
  * dense top-k instead. */
 int ora_pivot_topk(const void *q, const void *k, const float *w, int dtype, const int *cu_seqlens,
@@ -488,9 +529,9 @@ int ora_pivot_topk(const void *q, const void *k, const float *w, int dtype, cons
     if (!q || !k || !w || !out || (nrows > 0 && !rows) || H <= 0 || d <= 0 || topk <= 0 || g <= 0 ||
         dense_below < 0)
         return 1;
-    if (mode != ORA_REUSE && mode != ORA_REFINE && mode != ORA_BLOCK) return 1;
-    if ((mode == ORA_REFINE || mode == ORA_BLOCK) && c < topk) return 1;
-    if (mode == ORA_BLOCK && bn < 1) return 1;
+    if (mode != ORA_REUSE && mode != ORA_REFINE && mode != ORA_BLOCK && mode != ORA_QUEST) return 1;
+    if ((mode == ORA_REFINE || mode == ORA_BLOCK || mode == ORA_QUEST) && c < topk) return 1;
+    if ((mode == ORA_BLOCK || mode == ORA_QUEST) && bn < 1) return 1;
     if (check_requests(cu_seqlens, num_seqs)) return 1;
     for (int i = 0; i < nrows; ++i)
         if (rows[i] < 0 || rows[i] >= cu_seqlens[num_seqs]) return 1;
@@ -507,17 +548,18 @@ int ora_pivot_topk(const void *q, const void *k, const float *w, int dtype, cons
  * q [B,G,H,d], kcache [B,n_max,d], w [B,G,H]; kv_len host [B] with
  * G <= kv_len[b] <= n_max; query m of request b sits at position
  * kv_len[b]-G+m and the cache already holds the keys of the group.
- * mode ORA_DENSE, ORA_REUSE, ORA_REFINE (c >= topk) or ORA_BLOCK (c >= topk,
- * bn >= 1); out [nreqs,G,topk]. */
+ * mode ORA_DENSE, ORA_REUSE, ORA_REFINE (c >= topk), ORA_BLOCK or ORA_QUEST
+ * (c >= topk, bn >= 1); out [nreqs,G,topk]. */
 int ora_decode_topk(const void *q, const void *kcache, const float *w, int dtype, const int *kv_len,
                     int B, int G, int n_max, int H, int d, int topk, int c, int mode, int bn,
                     const long long *reqs, int nreqs, int *out, int nthreads) {
     if (!q || !kcache || !w || !kv_len || !out || (nreqs > 0 && !reqs) || H <= 0 || d <= 0 ||
         topk <= 0 || G <= 0)
         return 1;
-    if (mode != ORA_DENSE && mode != ORA_REUSE && mode != ORA_REFINE && mode != ORA_BLOCK) return 1;
-    if ((mode == ORA_REFINE || mode == ORA_BLOCK) && c < topk) return 1;
-    if (mode == ORA_BLOCK && bn < 1) return 1;
+    if (mode != ORA_DENSE && mode != ORA_REUSE && mode != ORA_REFINE && mode != ORA_BLOCK && mode != ORA_QUEST)
+        return 1;
+    if ((mode == ORA_REFINE || mode == ORA_BLOCK || mode == ORA_QUEST) && c < topk) return 1;
+    if ((mode == ORA_BLOCK || mode == ORA_QUEST) && bn < 1) return 1;
     for (int i = 0; i < nreqs; ++i) {
         if (reqs[i] < 0 || reqs[i] >= B) return 1;
         int n = kv_len[reqs[i]];

@@ -550,13 +550,74 @@ def pin_decode_block_full_budget_is_dense():
                 assert len(got) == 9 and all(part0 <= x <= t for x in got)
 
 
+def pin_quest_hand_blocks():
+    """Quest bound, worked by hand (one head, w = 1, d = 1, blocks of 2, one
+    member at t = 4 that is its own proxy, c = 4 tokens = one complete block
+    plus the partial block {4}):
+      keys -10, 10, 3, 3, 1 and q = +1: block A = {-10, 10} has bound
+      max(1*10, 1*-10) = 10, block B = {3, 3} has 3: A is kept, candidates
+      {0, 1, 4} score 0, 10, 1, so the top-1 is position 1.  (The block
+      means rank B first, 3 > 0, giving position 2; so would a bound taken
+      from the minimum.)  With q = +2 and top-2: scores 0, 20, 2 -> {1, 4}.
+      keys -10, 10, -5, -5, 1 and q = -1: A's bound is max(-10, 10) = 10,
+      B's is max(5, 5) = 5: A is kept, candidates score 10, 0, 0, so the
+      top-1 is position 0.  (A bound from the maximum alone gives A -10 ->
+      0 and B 5, keeping B and giving position 2.)"""
+    w = np.ones((5, 1), np.float32)
+    cu = np.array([0, 5], np.int32)
+    k1 = _bf(np.array([[-10.0], [10.0], [3.0], [3.0], [1.0]], np.float32))
+    k2 = _bf(np.array([[-10.0], [10.0], [-5.0], [-5.0], [1.0]], np.float32))
+    for k, qv, topk, want in ((k1, 1.0, 1, [1]), (k1, 2.0, 2, [1, 4]), (k2, -1.0, 1, [0])):
+        q = _bf(np.full((5, 1, 1), qv, np.float32))
+        got = O.pivot_topk(q, k, w, cu, topk, 1, 4, O.QUEST, rows=np.array([4]), bn=2)
+        assert got[0].tolist() == want, (qv, got)
+    q = _bf(np.full((5, 1, 1), 1.0, np.float32))
+    assert O.pivot_topk(q, k1, w, cu, 1, 1, 4, O.BLOCK, rows=np.array([4]), bn=2)[0].tolist() == [2]
+
+
+def pin_quest_reductions():
+    """Quest: keys constant inside each block make the bound the exact dot
+    product, so Quest ranks blocks as the block means do; a budget covering
+    the prefix is dense; and decode Quest equals prefill Quest."""
+    rng = np.random.default_rng(43)
+    T, H, d, bn = 96, 3, 8, 4
+    base = rng.standard_normal((T // bn, d)).astype(np.float32)
+    k = _bf(np.repeat(base, bn, axis=0))
+    q = _bf(rng.standard_normal((T, H, d)))
+    w = rng.random((T, H)).astype(np.float32)
+    cu = np.array([0, 60, T], np.int32)
+    for g, c in ((4, 8), (3, 12)):
+        a = O.pivot_topk(q, k, w, cu, 5, g, c, O.QUEST, bn=bn)
+        b = O.pivot_topk(q, k, w, cu, 5, g, c, O.BLOCK, bn=bn)
+        assert np.array_equal(a, b), (g, c)
+    k2 = _bf(rng.standard_normal((T, d)))
+    a = O.pivot_topk(q, k2, w, cu, 5, 4, 128, O.QUEST, bn=bn)
+    assert np.array_equal(a, O.dense_topk(q, k2, w, cu, 5))
+    B, G, n_max = 2, 2, 40
+    kc = _bf(rng.standard_normal((B, n_max, d)))
+    qd = _bf(rng.standard_normal((B, G, H, d)))
+    wd = rng.random((B, G, H)).astype(np.float32)
+    kv = np.array([40, 22], np.int32)
+    got = O.decode_topk(qd, kc, wd, kv, 5, 8, O.QUEST, bn=4)
+    for b in range(B):
+        n = kv[b]
+        qq = np.zeros((n, H, d), np.uint16)
+        ww = np.zeros((n, H), np.float32)
+        qq[n - G:] = qd[b]
+        ww[n - G:] = wd[b]
+        want = O.pivot_topk(qq, kc[b, :n], ww, np.array([0, n], np.int32), 5, G, 8, O.QUEST,
+                            rows=np.arange(n - G, n), bn=4)
+        assert np.array_equal(got[b], want), b
+
+
 ALL_PINS = [pin_hand_scores, pin_hand_topk, pin_hand_guardrail, pin_guardrail_reductions, pin_hand_decode, pin_bruteforce_dense,
             pin_bruteforce_pivot, pin_exact_integer_inputs, pin_textbook_single_head,
             pin_pivot_special_cases, pin_invariants, pin_reuse_within_proxy_ranking,
             pin_proxy_exact_mean, pin_decode_matches_prefill, pin_gaussian_mean_score,
             pin_block_mean_exact, pin_block_reductions, pin_block_constant_keys_equal_refine,
             pin_block_partial_closed_form, pin_attn_single_entry, pin_attn_equal_logits_mean,
-            pin_attn_library_sdpa, pin_attn_large_logits, pin_decode_block_full_budget_is_dense]
+            pin_attn_library_sdpa, pin_attn_large_logits, pin_decode_block_full_budget_is_dense,
+            pin_quest_hand_blocks, pin_quest_reductions]
 
 
 @pytest.mark.parametrize("pin", ALL_PINS, ids=[p.__name__ for p in ALL_PINS])
@@ -601,6 +662,10 @@ MUTANTS = {
                               "if (J->dense_below > 0 && lo + 1 <= J->dense_below) {"),
     "guard_by_own_position": ("if (J->dense_below > 0 && hi <= J->dense_below) {",
                               "if (J->dense_below > 0 && t + 1 <= J->dense_below) {"),
+    "quest_bound_from_minimum": ("bound += a > b ? a : b;", "bound += a < b ? a : b;"),
+    "quest_bound_max_only": ("bound += a > b ? a : b;", "bound += a;"),
+    "quest_relu_dropped": ("if (bound > 0.0) total += (double)wbar[j] * bound;", "total += (double)wbar[j] * bound;"),
+    "quest_scored_by_mean": ("            if (mode == ORA_QUEST) {\n", "            if (0) {\n"),
 }
 
 
