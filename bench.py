@@ -875,33 +875,36 @@ def main():
             dec[mode] = {"ms_per_step": step_ms, "scan_kernel_ms": scan_ms,
                          "scan_GBps": gbs, "scan_frac_hbm": (gbs / hbm_peak) if gbs else None,
                          "kernels": {n: {"launches": c, "ms_per_step": t / args.steps} for n, (c, t) in trd.items()}}
-        # the block pre-filter: the proxy scans the cache's block means (kept by
-        # the caller beside the cache, so built once here, outside the timing),
+        # the block pre-filter: the proxy scans the cache's block summaries
+        # (kept by the caller beside the cache, so built once here, outside the
+        # timing: block means, or per-block key min/max for the Quest rule),
         # then the chosen blocks' keys are re-scored
-        kbar = idx.decode_block_means(dkc)
-        wsb = torch.empty(idx.decode_block_workspace_size(DEC_B, DEC_G, DEC_N, H, D, TOPK, C_REF), dtype=torch.uint8,
-                          device=dev)
-        for _ in range(args.warmup):
-            idx.decode_block_topk(dq_, dkc, kbar, dkv, dw_, TOPK, C_REF, out_idx=od, workspace=wsb)
-        torch.cuda.synchronize()
-        assert idx.device_status(wsb) == "IDX_OK"
-        lib.idx_trace_enable(1)
-        e0.record(stream)
-        for _ in range(args.steps):
-            idx.decode_block_topk(dq_, dkc, kbar, dkv, dw_, TOPK, C_REF, out_idx=od, workspace=wsb)
-        e1.record(stream)
-        torch.cuda.synchronize()
-        lib.idx_trace_enable(0)
-        _, trd = trace_report(lib)
-        step_ms = max_over_ranks(e0.elapsed_time(e1) / args.steps)
-        # bytes the step must read: the block means of every request and the
-        # c candidate keys of each (plus the queries)
-        kb_bytes = kbar.numel() * kbar.element_size()
-        cand_bytes = DEC_B * C_REF * D * dkc.element_size()
-        dec["block"] = {"ms_per_step": step_ms, "block_means_bytes": kb_bytes, "candidate_key_bytes": cand_bytes,
-                        "speedup_vs_dense": (dec["dense"]["ms_per_step"] / step_ms) if step_ms > 0 else None,
-                        "kernels": {n: {"launches": c, "ms_per_step": t / args.steps} for n, (c, t) in trd.items()}}
-        del kbar, wsb
+        for rule in ("mean", "quest"):
+            ksum = idx.decode_block_means(dkc) if rule == "mean" else idx.decode_block_minmax(dkc)
+            wsb = torch.empty(idx.decode_block_workspace_size(DEC_B, DEC_G, DEC_N, H, D, TOPK, C_REF, rule),
+                              dtype=torch.uint8, device=dev)
+            for _ in range(args.warmup):
+                idx.decode_block_topk(dq_, dkc, ksum, dkv, dw_, TOPK, C_REF, rule, out_idx=od, workspace=wsb)
+            torch.cuda.synchronize()
+            assert idx.device_status(wsb) == "IDX_OK"
+            lib.idx_trace_enable(1)
+            e0.record(stream)
+            for _ in range(args.steps):
+                idx.decode_block_topk(dq_, dkc, ksum, dkv, dw_, TOPK, C_REF, rule, out_idx=od, workspace=wsb)
+            e1.record(stream)
+            torch.cuda.synchronize()
+            lib.idx_trace_enable(0)
+            _, trd = trace_report(lib)
+            step_ms = max_over_ranks(e0.elapsed_time(e1) / args.steps)
+            # bytes the step must read: the block summaries of every request and
+            # the c candidate keys of each (plus the queries)
+            ks_bytes = ksum.numel() * ksum.element_size()
+            cand_bytes = DEC_B * C_REF * D * dkc.element_size()
+            dec["block_" + rule] = {
+                "ms_per_step": step_ms, "block_summary_bytes": ks_bytes, "candidate_key_bytes": cand_bytes,
+                "speedup_vs_dense": (dec["dense"]["ms_per_step"] / step_ms) if step_ms > 0 else None,
+                "kernels": {n: {"launches": c, "ms_per_step": t / args.steps} for n, (c, t) in trd.items()}}
+            del ksum, wsb
         dec["hbm_peak_GBps"] = hbm_peak
         del dpool, dbt, perm
 

@@ -249,27 +249,34 @@ idx_status idx_decode_paged_topk(const void *q, const void *kpool, const int *bl
 
 /* Decode with the block pre-filter as the candidate generator (page
  * "Uncertainty-gated selection for block-sparse attention", Sec. 3.1, step
- * 1: a block of 64 keys is summarised by its mean key; page "Not All Tokens
+ * 1: a block of 64 keys is summarised by its mean key, Eq. (1), or by its
+ * per-dimension key minimum and maximum, Eq. (2), after Quest; page "Not All Tokens
  * Deserve Equal Resolution", abstract: chunk summaries are scored first, the
  * tokens of the chosen chunks are then scored exactly).  The decode group of
  * request b (its G queries, PIVOT page, Method, decode paragraph) is one
- * group: its proxy (mean query, mean w) scores the mean keys of the
- * complete blocks below kv_len[b]; the c / 64 best blocks (one fewer when
+ * group: its proxy (mean query, mean w) scores the complete blocks below
+ * kv_len[b] -- rule 0: the indexer score of the proxy against the block's
+ * mean key; rule 1 (Quest): sum_h wbar_h * max(0, sum_i max(qbar_hi * kmax_i,
+ * qbar_hi * kmin_i)), the indexer's weighted ReLU of each head's upper
+ * bound of q . k over the block -- and the c / 64 best blocks (one fewer when
  * kv_len[b] ends inside a block, whose partial block is then always taken),
  * ties to the lower block, give the candidate positions; each query
  * re-scores the candidates inside its own prefix and keeps its top-k.  This
  * is the prefill block mode (idx_pivot_topk with IDX_MODE_BLOCK) applied to
  * the decode group.
  *
- * The block means are a cache the caller keeps beside the key cache, so a
- * decode step reads them (n / 64 rows per request) and the chosen blocks'
- * keys instead of the whole cache:
- *   kbar  [B, n_max / 64, d] dtype   row b * (n_max / 64) + j = the mean of
- *         rows 64 j .. 64 j + 63 of request b's cache: fp32 sum in row order,
- *         one IEEE fp32 division by 64, round-to-nearest-even to bf16 for
- *         bf16 keys (the same rule as the group proxy).  Rows of blocks at or
- *         past kv_len[b] / 64 are never read.
- * idx_decode_block_means writes it from the key cache. */
+ * The block summaries are a cache the caller keeps beside the key cache,
+ * so a decode step reads them (n / 64 rows per request) and the chosen
+ * blocks' keys instead of the whole cache:
+ *   rule 0: kbar [B, n_max / 64, d] dtype   row b * (n_max / 64) + j = the
+ *         mean of rows 64 j .. 64 j + 63 of request b's cache: fp32 sum in
+ *         row order, one IEEE fp32 division by 64, round-to-nearest-even to
+ *         bf16 for bf16 keys (the same rule as the group proxy);
+ *         idx_decode_block_means writes it;
+ *   rule 1: kminmax [B, n_max / 64, 2, d] dtype   for block j of request b,
+ *         the per-dimension minimum of its 64 rows, then their maximum;
+ *         idx_decode_block_minmax writes it.
+ * Blocks at or past kv_len[b] / 64 are never read. */
 
 /* kbar rows of the blocks j >= first_block (j < n_max / 64) of every request
  * from kcache [B, n_max, d]; first_block = 0 fills all of it, and after keys
@@ -279,19 +286,27 @@ idx_status idx_decode_paged_topk(const void *q, const void *kpool, const int *bl
 idx_status idx_decode_block_means(const void *kcache, int B, int n_max, int d, idx_dtype dtype,
                                   int first_block, void *kbar, idx_stream_t stream);
 
+/* The same for rule 1: kminmax rows of blocks j >= first_block (exact: every
+ * value is a key element). */
+idx_status idx_decode_block_minmax(const void *kcache, int B, int n_max, int d, idx_dtype dtype,
+                                   int first_block, void *kminmax, idx_stream_t stream);
+
 /* Workspace bytes for idx_decode_block_topk (0 for arguments it rejects). */
-size_t idx_decode_block_workspace_size(int B, int G, int n_max, int H, int d, int topk, int c,
+size_t idx_decode_block_workspace_size(int B, int G, int n_max, int H, int d, int topk, int c, int rule,
                                        idx_dtype dtype);
 
 /* One decode step with the block pre-filter.  q, kcache, kv_len, w, out_idx,
- * out_score and the status word as in idx_decode_topk; kbar as above.
+ * out_score and the status word as in idx_decode_topk; ksum = kbar (rule 0)
+ * or kminmax (rule 1) as above.
  *   c  candidate budget in tokens: a multiple of 64, >= 64 and >= topk
  *   n_max a multiple of 64
- * Argument errors return IDX_ERR_INVALID before any launch; G > 8, n_max >
- * 2^20 or a shape neither score path serves return IDX_ERR_UNSUPPORTED. */
-idx_status idx_decode_block_topk(const void *q, const void *kcache, const void *kbar, const int *kv_len,
-                                 const float *w, int B, int G, int n_max, int H, int d, int topk, int c,
-                                 idx_dtype dtype, int *out_idx, float *out_score, void *ws,
+ * Argument errors (a rule other than 0 or 1 included) return
+ * IDX_ERR_INVALID before any launch; G > 8, n_max > 2^20, a shape neither
+ * score path serves, or rule 1 with H * d * 8 bytes above the shared memory
+ * of one block return IDX_ERR_UNSUPPORTED. */
+idx_status idx_decode_block_topk(const void *q, const void *kcache, const void *ksum, int rule,
+                                 const int *kv_len, const float *w, int B, int G, int n_max, int H, int d,
+                                 int topk, int c, idx_dtype dtype, int *out_idx, float *out_score, void *ws,
                                  size_t ws_bytes, idx_stream_t stream);
 
 /* ----------------------------------------------- no-allocation variant */

@@ -47,9 +47,10 @@ SIGNATURES = {
     "idx_trace_enable": (_i, [_i]),
     "idx_debug_wait_probe": (_i, [_vp, ctypes.c_uint, _vp]),
     "idx_decode_block_means": (_i, [_vp, _i, _i, _i, _i, _i, _vp, _vp]),
-    "idx_decode_block_workspace_size": (_sz, [_i, _i, _i, _i, _i, _i, _i, _i]),
-    "idx_decode_block_topk": (_i, [_vp, _vp, _vp, _ip, _fp, _i, _i, _i, _i, _i, _i, _i, _i, _ip, _fp, _vp, _sz,
-                                   _vp]),
+    "idx_decode_block_minmax": (_i, [_vp, _i, _i, _i, _i, _i, _vp, _vp]),
+    "idx_decode_block_workspace_size": (_sz, [_i, _i, _i, _i, _i, _i, _i, _i, _i]),
+    "idx_decode_block_topk": (_i, [_vp, _vp, _vp, _i, _ip, _fp, _i, _i, _i, _i, _i, _i, _i, _i, _ip, _fp, _vp,
+                                   _sz, _vp]),
     "idx_decode_topk_noalloc": (_i, [_vp, _vp, _ip, _fp, _i, _i, _i, _i, _i, _i, _i, _ip, _fp, _vp]),
     "idx_decode_noalloc_status": (_i, [_vp]),
     "idx_trace_report": (_ll, [ctypes.c_char_p, _sz]),

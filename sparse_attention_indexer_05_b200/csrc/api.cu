@@ -529,7 +529,8 @@ struct Decode {
     const int *bt = nullptr;  // paged cache: block table [B, max_pages], else NULL
     int page = 0, max_pages = 0;
     long long num_pages = 0;
-    const void *kbar = nullptr;  // block mode: block means [B, n_max / 64, d]
+    const void *kbar = nullptr;  // block mode: block means [B, n_max / 64, d], or
+    int rule = 0;                // (rule 1, Quest) per-block key min and max [B, n_max / 64, 2, d]
 
     unsigned *status() const { return reinterpret_cast<unsigned *>(ws + L.status); }
 
@@ -597,12 +598,17 @@ idx_status Decode::run(int *out_idx, float *out_score) const {
         int *nlen = reinterpret_cast<int *>(ws + L.nlen);
         int *cblk = reinterpret_cast<int *>(ws + L.cblk);
         TRY_CUDA(launch_decode_block_len(kv, B, G, n_max, nlen, st));
-        DecodeArgs a = dargs(true, spill);
-        a.kc = kbar;
-        a.kv_len = nlen;
-        a.G = 1;
-        a.n_max = n_max >> kBlockShift;
-        TRY_CUDA(scan(a));
+        if (rule == 1) {
+            TRY_CUDA(launch_decode_quest_scan(ws + L.qbar, reinterpret_cast<const float *>(ws + L.wbar), kbar, nlen,
+                                              B, n_max >> kBlockShift, H, d, (int)dt, spill, st));
+        } else {
+            DecodeArgs a = dargs(true, spill);
+            a.kc = kbar;
+            a.kv_len = nlen;
+            a.G = 1;
+            a.n_max = n_max >> kBlockShift;
+            TRY_CUDA(scan(a));
+        }
         TRY_CUDA(launch_select(sargs(SEL_DEC_PROXY_TO_BLOCKS, B, c >> kBlockShift, cblk, nullptr, spill,
                                      n_max >> kBlockShift),
                                st));
@@ -673,17 +679,20 @@ idx_status idx_decode_paged_topk(const void *q, const void *kpool, const int *bl
 
 namespace {
 
-idx_status check_decode_block(int B, int G, int n_max, int H, int d, int topk, int c, idx_dtype dt) {
+idx_status check_decode_block(int B, int G, int n_max, int H, int d, int topk, int c, int rule, idx_dtype dt) {
     if (B < 1 || G < 1 || n_max < G || topk < 1 || !shape_ok(H, d, dt)) return IDX_ERR_INVALID;
-    if (n_max % kBlockN != 0 || c < topk || c < kBlockN || c % kBlockN != 0) return IDX_ERR_INVALID;
+    if (n_max % kBlockN != 0 || c < topk || c < kBlockN || c % kBlockN != 0 || (rule != 0 && rule != 1))
+        return IDX_ERR_INVALID;
     if (G > RB || n_max > kMaxLen || !path_ok(H, d, dt)) return IDX_ERR_UNSUPPORTED;
+    if (rule == 1 && quest_scan_smem(H, d) > kMaxSmem) return IDX_ERR_UNSUPPORTED;
     return IDX_OK;
 }
 
 }  // namespace
 
-size_t idx_decode_block_workspace_size(int B, int G, int n_max, int H, int d, int topk, int c, idx_dtype dtype) {
-    if (check_decode_block(B, G, n_max, H, d, topk, c, dtype) != IDX_OK) return 0;
+size_t idx_decode_block_workspace_size(int B, int G, int n_max, int H, int d, int topk, int c, int rule,
+                                       idx_dtype dtype) {
+    if (check_decode_block(B, G, n_max, H, d, topk, c, rule, dtype) != IDX_OK) return 0;
     return decode_ws(B, G, n_max, H, d, c, IDX_MODE_BLOCK, dtype).total;
 }
 
@@ -698,19 +707,31 @@ idx_status idx_decode_block_means(const void *kcache, int B, int n_max, int d, i
                                              reinterpret_cast<cudaStream_t>(stream)));
 }
 
-idx_status idx_decode_block_topk(const void *q, const void *kcache, const void *kbar, const int *kv_len,
+idx_status idx_decode_block_minmax(const void *kcache, int B, int n_max, int d, idx_dtype dtype, int first_block,
+                                   void *kminmax, idx_stream_t stream) {
+    if (!kcache || !kminmax || B < 1 || n_max < kBlockN || n_max % kBlockN != 0 || first_block < 0 ||
+        !shape_ok(1, d, dtype))
+        return IDX_ERR_INVALID;
+    if (n_max > kMaxLen) return IDX_ERR_UNSUPPORTED;
+    TracePhase phase("decode_quest");
+    return cuda_st(launch_decode_block_minmax(kcache, B, n_max, d, (int)dtype, first_block, kminmax,
+                                              reinterpret_cast<cudaStream_t>(stream)));
+}
+
+idx_status idx_decode_block_topk(const void *q, const void *kcache, const void *ksum, int rule, const int *kv_len,
                                  const float *w, int B, int G, int n_max, int H, int d, int topk, int c,
                                  idx_dtype dtype, int *out_idx, float *out_score, void *ws, size_t ws_bytes,
                                  idx_stream_t stream) {
-    if (!q || !kcache || !kbar || !kv_len || !w || !out_idx) return IDX_ERR_INVALID;
-    idx_status s = check_decode_block(B, G, n_max, H, d, topk, c, dtype);
+    if (!q || !kcache || !ksum || !kv_len || !w || !out_idx) return IDX_ERR_INVALID;
+    idx_status s = check_decode_block(B, G, n_max, H, d, topk, c, rule, dtype);
     if (s != IDX_OK) return s;
     const size_t need = decode_ws(B, G, n_max, H, d, c, IDX_MODE_BLOCK, dtype).total;
     if (!ws || (reinterpret_cast<uintptr_t>(ws) % kAlign) != 0 || ws_bytes < need) return IDX_ERR_WORKSPACE;
-    TracePhase phase("decode_block");
+    TracePhase phase(rule == 1 ? "decode_quest" : "decode_block");
     Decode D{q, kcache, kv_len, w, B, G, n_max, H, d, topk, c, IDX_MODE_BLOCK, dtype, static_cast<char *>(ws),
              decode_ws(B, G, n_max, H, d, c, IDX_MODE_BLOCK, dtype), reinterpret_cast<cudaStream_t>(stream)};
-    D.kbar = kbar;
+    D.kbar = ksum;
+    D.rule = rule;
     return D.run(out_idx, out_score);
 }
 

@@ -257,6 +257,13 @@ cudaError_t launch_decode_proxy(const void *q, const float *w, int B, int G, int
 cudaError_t launch_decode_block_means(const void *kc, int B, int n_max, int d, int dtype, int first_block,
                                       void *kbar, cudaStream_t st);
 cudaError_t launch_decode_block_len(const int *kv_len, int B, int G, int n_max, int *nlen, cudaStream_t st);
+// decode block mode with the Quest bound: per-block key minimum and maximum
+// [B, n_max / 64, 2, d], and the proxy's bound scores of the complete blocks
+cudaError_t launch_decode_block_minmax(const void *kc, int B, int n_max, int d, int dtype, int first_block,
+                                       void *kq, cudaStream_t st);
+size_t quest_scan_smem(int H, int d);
+cudaError_t launch_decode_quest_scan(const void *qbar, const float *wbar, const void *kq, const int *nlen, int B,
+                                     int nb, int H, int d, int dtype, float *spill, cudaStream_t st);
 cudaError_t launch_decode_block_expand(const int *kv_len, int B, int G, int n_max, const int *cblk, int *cand,
                                        int c, cudaStream_t st);
 size_t simt_smem_bytes(int H, int d, int dtype);

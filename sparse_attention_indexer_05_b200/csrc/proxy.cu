@@ -178,6 +178,130 @@ __global__ void __launch_bounds__(kProxyThreads) decode_block_mean_kernel(const 
     Vec<T>::store(kbar + ((long long)b * nb + j) * d + e, acc);
 }
 
+__device__ __forceinline__ float to_float(float x) { return x; }
+__device__ __forceinline__ float to_float(__nv_bfloat16 x) { return __bfloat162float(x); }
+
+// Block summaries for the Quest bound ("Uncertainty-gated selection for
+// block-sparse attention", Sec. 3.1, Eq. (2)): the per-dimension minimum and
+// maximum of the 64 keys of block j of request b, to rows 2 (b * nb + j) and
+// 2 (b * nb + j) + 1 of kq [B, nb, 2, d] (exact: they are keys), blocks j >=
+// first_block only.  One thread per 8 dimensions of one block.
+template <typename T>
+__global__ void __launch_bounds__(kProxyThreads) decode_block_minmax_kernel(const T *kc, int B, int n_max, int d,
+                                                                            int first_block, T *kq) {
+    const int per_row = d / 8;
+    const int nb = n_max >> kBlockShift, nu = nb - first_block;
+    const long long u = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    if (nu <= 0 || u >= (long long)B * nu * per_row) return;
+    const long long x = u / per_row;
+    const int e = (int)(u - x * per_row) * 8;
+    const int b = (int)(x / nu), j = first_block + (int)(x - (long long)b * nu);
+    const T *src = kc + ((long long)b * n_max + (long long)j * kBlockN) * d + e;
+    float lo[8], hi[8], v[8];
+    Vec<T>::load(src, lo);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) hi[i] = lo[i];
+    for (int r = 1; r < kBlockN; ++r) {
+        Vec<T>::load(src + (long long)r * d, v);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            lo[i] = fminf(lo[i], v[i]);
+            hi[i] = fmaxf(hi[i], v[i]);
+        }
+    }
+    T *dst = kq + ((long long)b * nb + j) * 2 * d + e;
+    Vec<T>::store(dst, lo);
+    Vec<T>::store(dst + d, hi);
+}
+
+// Decode block scores by the Quest bound: for the proxy of request b (qbar
+// [H, d], wbar [H]) and each complete block j < nlen[b],
+//     bound_h = sum_i max(q_hi * kmax_i, q_hi * kmin_i)   (i ascending, fp32)
+//     score   = sum_h wbar_h * max(bound_h, 0)           (h ascending)
+// to spill [b * nb + j].  max(q a, q b) with a >= b is q a for q >= 0 and q b
+// otherwise, so the bound is accumulated as two FMAs with q+ = max(q, 0) and
+// q- = min(q, 0) (the zero product adds nothing).  The proxy's q+ and q- sit
+// in shared memory as fp32 (H * d * 8 bytes) and are read as broadcasts;
+// each thread scores two blocks (kQuestPer), so every shared load feeds two
+// blocks' FMAs, with heads in chunks of 32 whose partial bounds stay in
+// registers.
+constexpr int kQuestThreads = 128;
+constexpr int kQuestPer = 2;
+
+template <typename T>
+__global__ void __launch_bounds__(kQuestThreads) decode_quest_scan_kernel(const T *qbar, const float *wbar,
+                                                                          const T *kq, const int *nlen, int nb,
+                                                                          int H, int d, float *spill) {
+    extern __shared__ __align__(16) float qs[];  // [H][d] q+, then [H][d] q-
+    const int b = blockIdx.y;
+    const int j0 = blockIdx.x * (kQuestThreads * kQuestPer) + threadIdx.x;  // blocks j0, j0 + kQuestThreads
+    const int nl = nlen[b];
+    if (blockIdx.x * (kQuestThreads * kQuestPer) >= nl) return;
+    const int HD = H * d;
+    for (int i = threadIdx.x; i < HD; i += blockDim.x) {
+        const float v = to_float(qbar[(long long)b * HD + i]);
+        qs[i] = v > 0.0f ? v : 0.0f;
+        qs[HD + i] = v < 0.0f ? v : 0.0f;
+    }
+    __syncthreads();
+    if (j0 >= nl) return;
+    const T *row[kQuestPer];  // kmin, then kmax; a block past nlen repeats the first (not stored)
+#pragma unroll
+    for (int u = 0; u < kQuestPer; ++u) {
+        const int j = j0 + u * kQuestThreads < nl ? j0 + u * kQuestThreads : j0;
+        row[u] = kq + ((long long)b * nb + j) * 2 * d;
+    }
+    float total[kQuestPer];
+#pragma unroll
+    for (int u = 0; u < kQuestPer; ++u) total[u] = 0.0f;
+    for (int h0 = 0; h0 < H; h0 += 32) {
+        float acc[kQuestPer][32];
+#pragma unroll
+        for (int u = 0; u < kQuestPer; ++u)
+#pragma unroll
+            for (int hh = 0; hh < 32; ++hh) acc[u][hh] = 0.0f;
+        for (int e = 0; e < d; e += 8) {
+            float lo[kQuestPer][8], hi[kQuestPer][8];
+#pragma unroll
+            for (int u = 0; u < kQuestPer; ++u) {
+                Vec<T>::load(row[u] + e, lo[u]);
+                Vec<T>::load(row[u] + d + e, hi[u]);
+            }
+#pragma unroll
+            for (int hh = 0; hh < 32; ++hh) {
+                if (h0 + hh < H) {
+                    const float4 *pp = reinterpret_cast<const float4 *>(qs + (h0 + hh) * d + e);
+                    const float4 *pn = reinterpret_cast<const float4 *>(qs + HD + (h0 + hh) * d + e);
+                    const float4 p0 = pp[0], p1 = pp[1], n0 = pn[0], n1 = pn[1];
+                    const float qp[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
+                    const float qn[8] = {n0.x, n0.y, n0.z, n0.w, n1.x, n1.y, n1.z, n1.w};
+#pragma unroll
+                    for (int u = 0; u < kQuestPer; ++u) {
+                        float a = acc[u][hh];
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) {
+                            a = fmaf(qp[i], hi[u][i], a);
+                            a = fmaf(qn[i], lo[u][i], a);
+                        }
+                        acc[u][hh] = a;
+                    }
+                }
+            }
+        }
+#pragma unroll
+        for (int hh = 0; hh < 32; ++hh) {
+            if (h0 + hh < H) {
+                const float wh = wbar[(long long)b * H + h0 + hh];
+#pragma unroll
+                for (int u = 0; u < kQuestPer; ++u) total[u] = fmaf(wh, fmaxf(acc[u][hh], 0.0f), total[u]);
+            }
+        }
+    }
+#pragma unroll
+    for (int u = 0; u < kQuestPer; ++u)
+        if (j0 + u * kQuestThreads < nl) spill[(long long)b * nb + j0 + u * kQuestThreads] = total[u];
+}
+
 // Decode block mode: the complete blocks each request's proxy scans,
 // kv_len[b] / 64 (0 for a request whose kv_len is out of range; the block
 // select flags it).
@@ -306,6 +430,44 @@ cudaError_t launch_decode_block_means(const void *kc, int B, int n_max, int d, i
     else
         decode_block_mean_kernel<__nv_bfloat16><<<grid, kProxyThreads, 0, st>>>(
             (const __nv_bfloat16 *)kc, B, n_max, d, first_block, (__nv_bfloat16 *)kbar);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_decode_block_minmax(const void *kc, int B, int n_max, int d, int dtype, int first_block,
+                                       void *kq, cudaStream_t st) {
+    const int nu = (n_max >> kBlockShift) - first_block;
+    if (B <= 0 || nu <= 0) return cudaSuccess;
+    const long long units = (long long)B * nu * (d / 8);
+    const unsigned grid = (unsigned)((units + kProxyThreads - 1) / kProxyThreads);
+    TraceScope ts("block_minmax", st);
+    if (dtype == 1)
+        decode_block_minmax_kernel<float><<<grid, kProxyThreads, 0, st>>>((const float *)kc, B, n_max, d,
+                                                                          first_block, (float *)kq);
+    else
+        decode_block_minmax_kernel<__nv_bfloat16><<<grid, kProxyThreads, 0, st>>>(
+            (const __nv_bfloat16 *)kc, B, n_max, d, first_block, (__nv_bfloat16 *)kq);
+    return cudaGetLastError();
+}
+
+size_t quest_scan_smem(int H, int d) { return (size_t)H * d * 8; }
+
+cudaError_t launch_decode_quest_scan(const void *qbar, const float *wbar, const void *kq, const int *nlen, int B,
+                                     int nb, int H, int d, int dtype, float *spill, cudaStream_t st) {
+    const size_t smem = quest_scan_smem(H, d);
+    cudaError_t e = dtype == 1 ? cudaFuncSetAttribute(decode_quest_scan_kernel<float>,
+                                                      cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)
+                               : cudaFuncSetAttribute(decode_quest_scan_kernel<__nv_bfloat16>,
+                                                      cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    const int per_cta = kQuestThreads * kQuestPer;
+    const dim3 grid((unsigned)((nb + per_cta - 1) / per_cta), (unsigned)B);
+    TraceScope ts("quest_scan", st);
+    if (dtype == 1)
+        decode_quest_scan_kernel<float><<<grid, kQuestThreads, smem, st>>>((const float *)qbar, wbar,
+                                                                           (const float *)kq, nlen, nb, H, d, spill);
+    else
+        decode_quest_scan_kernel<__nv_bfloat16><<<grid, kQuestThreads, smem, st>>>(
+            (const __nv_bfloat16 *)qbar, wbar, (const __nv_bfloat16 *)kq, nlen, nb, H, d, spill);
     return cudaGetLastError();
 }
 

@@ -214,23 +214,42 @@ def decode_block_means(kcache, kbar=None, first_block: int = 0, stream=None):
     return kbar
 
 
-def decode_block_workspace_size(B, G, n_max, H, d, topk, c, dtype=torch.bfloat16) -> int:
+def decode_block_minmax(kcache, kminmax=None, first_block: int = 0, stream=None):
+    """Per-block key minimum and maximum [B, n_max/64, 2, d] of a decode cache
+    kcache [B, n_max, d] (the Quest rule's block summaries); blocks >=
+    first_block are (re)written."""
+    B, n_max, d = kcache.shape
+    if kminmax is None:
+        kminmax = torch.empty(B, n_max // 64, 2, d, dtype=kcache.dtype, device=kcache.device)
+    N.check(N.lib().idx_decode_block_minmax(_dev(kcache, "kcache"), B, n_max, d, _dtype_code(kcache), first_block,
+                                            _dev(kminmax, "kminmax", kcache.dtype), _stream(stream)),
+            "idx_decode_block_minmax")
+    return kminmax
+
+
+_RULES = {"mean": 0, "quest": 1}
+
+
+def decode_block_workspace_size(B, G, n_max, H, d, topk, c, rule="mean", dtype=torch.bfloat16) -> int:
     dt = N.BF16 if dtype == torch.bfloat16 else N.F32
-    return int(N.lib().idx_decode_block_workspace_size(B, G, n_max, H, d, topk, c, dt))
+    return int(N.lib().idx_decode_block_workspace_size(B, G, n_max, H, d, topk, c, _RULES[rule], dt))
 
 
-def decode_block_topk(q, kcache, kbar, kv_len, w, topk: int, c: int, out_idx=None, out_score=None, workspace=None,
-                      stream=None, return_scores=False):
+def decode_block_topk(q, kcache, ksum, kv_len, w, topk: int, c: int, rule="mean", out_idx=None, out_score=None,
+                      workspace=None, stream=None, return_scores=False):
     """One decode step with the block pre-filter: q [B,G,H,d], kcache [B,n_max,d],
-    kbar [B,n_max/64,d] (decode_block_means), kv_len int32 [B], w [B,G,H]."""
+    kv_len int32 [B], w [B,G,H]; ksum = block means [B,n_max/64,d] for
+    rule="mean" (decode_block_means) or block min/max [B,n_max/64,2,d] for
+    rule="quest" (decode_block_minmax)."""
     B, G, H, d = q.shape
     n_max = kcache.shape[1]
     dt = _dtype_code(q)
-    ws = _ws(workspace, decode_block_workspace_size(B, G, n_max, H, d, topk, c, q.dtype), q.device)
+    ws = _ws(workspace, decode_block_workspace_size(B, G, n_max, H, d, topk, c, rule, q.dtype), q.device)
     out_idx, out_score = _outs((B, G), topk, q.device, out_idx, out_score, return_scores)
     N.check(N.lib().idx_decode_block_topk(
-        _dev(q, "q"), _dev(kcache, "kcache", q.dtype), _dev(kbar, "kbar", q.dtype), _dev(kv_len, "kv_len", torch.int32),
-        _dev(w, "w", torch.float32), B, G, n_max, H, d, topk, c, dt, _dev(out_idx, "out_idx", torch.int32),
+        _dev(q, "q"), _dev(kcache, "kcache", q.dtype), _dev(ksum, "ksum", q.dtype), _RULES[rule],
+        _dev(kv_len, "kv_len", torch.int32), _dev(w, "w", torch.float32), B, G, n_max, H, d, topk, c, dt,
+        _dev(out_idx, "out_idx", torch.int32),
         _dev(out_score, "out_score", torch.float32) if out_score is not None else None,
         ws.data_ptr(), ws.numel(), _stream(stream)), "idx_decode_block_topk")
     return (out_idx, out_score) if return_scores else out_idx

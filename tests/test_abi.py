@@ -26,7 +26,7 @@ def declared_functions():
 
 def test_exports_every_declared_symbol(lib):
     names = declared_functions()
-    assert len(names) == 28
+    assert len(names) == 29
     for n in names:
         assert hasattr(lib, n), n
         assert n in N.SIGNATURES, n
@@ -155,35 +155,34 @@ def test_sparse_attn_argument_checks(lib):
 
 def test_decode_block_workspace_and_argument_checks(lib):
     size = lib.idx_decode_block_workspace_size
-    ok = size(64, 2, 131072, 64, 128, 2048, 4096, 0)
-    assert ok > 0
-    # the block-score spill is a 64th of the token-score one
-    assert ok < lib.idx_decode_workspace_size(64, 2, 131072, 64, 128, 2048, 4096, 2, 0)
-    assert size(64, 2, 131072 - 1, 64, 128, 2048, 4096, 0) == 0    # n_max not a multiple of 64
-    assert size(64, 2, 131072, 64, 128, 2048, 4096 + 32, 0) == 0   # c not a multiple of 64
-    assert size(64, 2, 131072, 64, 128, 2048, 1024, 0) == 0        # c < topk
-    assert size(64, 9, 131072, 64, 128, 2048, 4096, 0) == 0        # G above one row block
+    for rule in (0, 1):
+        ok = size(64, 2, 131072, 64, 128, 2048, 4096, rule, 0)
+        assert ok > 0
+        # the block-score spill is a 64th of the token-score one
+        assert ok < lib.idx_decode_workspace_size(64, 2, 131072, 64, 128, 2048, 4096, 2, 0)
+        assert size(64, 2, 131072 - 1, 64, 128, 2048, 4096, rule, 0) == 0    # n_max not a multiple of 64
+        assert size(64, 2, 131072, 64, 128, 2048, 4096 + 32, rule, 0) == 0   # c not a multiple of 64
+        assert size(64, 2, 131072, 64, 128, 2048, 1024, rule, 0) == 0        # c < topk
+        assert size(64, 9, 131072, 64, 128, 2048, 4096, rule, 0) == 0        # G above one row block
+    assert size(64, 2, 131072, 64, 128, 2048, 4096, 2, 0) == 0               # no rule 2
+    assert size(64, 2, 131072, 256, 256, 2048, 4096, 1, 0) == 0              # Quest proxy above shared memory
     fake = 256  # never dereferenced: the checks fail before any launch
     f = lib.idx_decode_block_topk
-    args = [fake, fake, fake, fake, fake, 4, 2, 4096, 64, 128, 64, 128, 0, fake, None, fake, 1 << 40, None]
-    for i in (0, 1, 2, 3, 4, 13):  # q, kcache, kbar, kv_len, w, out_idx
+    args = [fake, fake, fake, 0, fake, fake, 4, 2, 4096, 64, 128, 64, 128, 0, fake, None, fake, 1 << 40, None]
+    for i in (0, 1, 2, 4, 5, 14):  # q, kcache, ksum, kv_len, w, out_idx
         a = list(args)
         a[i] = None
         assert f(*a) == 1, i
-    a = list(args)
-    a[11] = 96                      # c not a multiple of 64
-    assert f(*a) == 1
-    a = list(args)
-    a[7] = 4000                     # n_max not a multiple of 64
-    assert f(*a) == 1
-    a = list(args)
-    a[6] = 9                        # G > 8
-    assert f(*a) == 2
-    a = list(args)
-    a[16] = 16                      # workspace too small
-    assert f(*a) == 3
-    m = lib.idx_decode_block_means
-    assert m(None, 4, 4096, 128, 0, 0, fake, None) == 1
-    assert m(fake, 4, 4000, 128, 0, 0, fake, None) == 1   # n_max not a multiple of 64
-    assert m(fake, 4, 4096, 12, 0, 0, fake, None) == 1    # d % 8 != 0
-    assert m(fake, 4, 4096, 128, 0, -1, fake, None) == 1  # negative first block
+    for i, v, code in ((12, 96, 1),    # c not a multiple of 64
+                       (8, 4000, 1),   # n_max not a multiple of 64
+                       (3, 2, 1),      # no rule 2
+                       (7, 9, 2),      # G > 8
+                       (17, 16, 3)):   # workspace too small
+        a = list(args)
+        a[i] = v
+        assert f(*a) == code, (i, v)
+    for m in (lib.idx_decode_block_means, lib.idx_decode_block_minmax):
+        assert m(None, 4, 4096, 128, 0, 0, fake, None) == 1
+        assert m(fake, 4, 4000, 128, 0, 0, fake, None) == 1   # n_max not a multiple of 64
+        assert m(fake, 4, 4096, 12, 0, 0, fake, None) == 1    # d % 8 != 0
+        assert m(fake, 4, 4096, 128, 0, -1, fake, None) == 1  # negative first block

@@ -1,10 +1,13 @@
-"""GPU parity of decode with the block pre-filter (idx_decode_block_topk)
-and of the block means it reads (idx_decode_block_means), against the
-oracle's decode block mode (ora_decode_topk with ORA_BLOCK, block size 64).
+"""GPU parity of decode with the block pre-filter (idx_decode_block_topk,
+blocks ranked by their mean key or by the Quest bound) and of the block
+summaries it reads (idx_decode_block_means, idx_decode_block_minmax),
+against the oracle's decode block modes (ora_decode_topk with ORA_BLOCK or
+ORA_QUEST, block size 64).
 
   * block means: every row of kbar equals the oracle's mean of the same 64
     cache rows bit for bit (bf16 and fp32); an update from a first block on
-    equals the full computation and leaves the earlier rows untouched;
+    equals the full computation and leaves the earlier rows untouched; the
+    Quest summaries equal numpy's minimum and maximum of those rows;
   * the top-k: rows are well formed and hold as many positions as the
     oracle's (its candidate set has the same blocks and partial block), and
     index recall against the oracle is >= 0.999 on the tensor-core path
@@ -36,14 +39,17 @@ def idx():
     return m
 
 
-def _run(idx, D, topk, c):
+def _run(idx, D, topk, c, rule="mean"):
     q, kc, w, kv = to_dev(D.q), to_dev(D.kcache), to_dev(D.w), to_dev(D.kv_len)
-    kbar = idx.decode_block_means(kc)
+    ksum = idx.decode_block_means(kc) if rule == "mean" else idx.decode_block_minmax(kc)
     B, G, H, d = q.shape
-    ws = torch.empty(idx.decode_block_workspace_size(B, G, kc.shape[1], H, d, topk, c, q.dtype), dtype=torch.uint8,
-                     device="cuda")
-    out = idx.decode_block_topk(q, kc, kbar, kv, w, topk, c, workspace=ws)
-    return out.cpu().numpy(), idx.device_status(ws), kbar
+    ws = torch.empty(idx.decode_block_workspace_size(B, G, kc.shape[1], H, d, topk, c, rule, q.dtype),
+                     dtype=torch.uint8, device="cuda")
+    out = idx.decode_block_topk(q, kc, ksum, kv, w, topk, c, rule, workspace=ws)
+    return out.cpu().numpy(), idx.device_status(ws), ksum
+
+
+_MODE = {"mean": O.BLOCK, "quest": O.QUEST}
 
 
 def _check(got, want, kv, G, topk):
@@ -72,6 +78,14 @@ def test_block_means_bit_exact_and_update(idx, dtype):
             want = O.block_mean(kc_h[b], j * 64, 64)
             assert np.array_equal(got[b, j].view(np.uint32 if dtype == "f32" else np.uint16),
                                   want.view(np.uint32 if dtype == "f32" else np.uint16)), (b, j)
+    # the Quest summaries: per-dimension minimum, then maximum, of each block
+    kq = idx.decode_block_minmax(kc).cpu()
+    kq = kq.view(torch.int16).numpy().view(np.uint16) if dtype == "bf16" else kq.numpy()
+    vals_k = W.bf16_to_f32(kc_h) if dtype == "bf16" else kc_h
+    blocks = vals_k.reshape(B, n_max // 64, 64, d)
+    want_q = np.stack([blocks.min(axis=2), blocks.max(axis=2)], axis=2)
+    got_q = W.bf16_to_f32(kq) if dtype == "bf16" else kq
+    assert np.array_equal(got_q, want_q)
     # an update from block 7 on: rows 0..6 keep their (here: poisoned) values
     kbar2 = kbar.clone()
     kbar2[:, :7] = 0
@@ -81,32 +95,35 @@ def test_block_means_bit_exact_and_update(idx, dtype):
     assert (kbar2[:, :7] == 0).all()
 
 
-def test_decode_block_bf16_tensor_cores(idx):
+@pytest.mark.parametrize("rule", ["mean", "quest"])
+def test_decode_block_bf16_tensor_cores(idx, rule):
     topk, c, G = 64, 256, 2
     kv = [2560, 2000, 130, 64, 7, 63, 1025]
     D = W.decode(B=len(kv), n=2560, G=G, H=64, d=128, topk=topk, seed=11, kv_len=kv)
-    got, st, _ = _run(idx, D, topk, c)
+    got, st, _ = _run(idx, D, topk, c, rule)
     assert st == "IDX_OK"
-    want = O.decode_topk(D.q, D.kcache, D.w, D.kv_len, topk, c, O.BLOCK, bn=64)
+    want = O.decode_topk(D.q, D.kcache, D.w, D.kv_len, topk, c, _MODE[rule], bn=64)
     _check(got, want, D.kv_len, G, topk)
     assert recall(got, want) >= 0.999
 
 
-def test_decode_block_mtp_group_and_fp32(idx):
+@pytest.mark.parametrize("rule", ["mean", "quest"])
+def test_decode_block_mtp_group_and_fp32(idx, rule):
     # G = 4 MTP queries, fp32 (CUDA-core scan and re-score)
     topk, c, G = 16, 128, 4
     kv = [700, 4, 200, 129]
     D = W.decode(B=len(kv), n=704, G=G, H=4, d=64, topk=topk, seed=12, kv_len=kv)
     D.q = W.bf16_to_f32(D.q)
     D.kcache = W.bf16_to_f32(D.kcache)
-    got, st, _ = _run(idx, D, topk, c)
+    got, st, _ = _run(idx, D, topk, c, rule)
     assert st == "IDX_OK"
-    want = O.decode_topk(D.q, D.kcache, D.w, D.kv_len, topk, c, O.BLOCK, bn=64)
+    want = O.decode_topk(D.q, D.kcache, D.w, D.kv_len, topk, c, _MODE[rule], bn=64)
     _check(got, want, D.kv_len, G, topk)
     assert recall(got, want) >= 0.999
 
 
-def test_decode_block_exact_integer_inputs(idx):
+@pytest.mark.parametrize("rule", ["mean", "quest"])
+def test_decode_block_exact_integer_inputs(idx, rule):
     topk, c, G = 8, 128, 2
     B, n_max, H, d = 4, 512, 64, 128
     rng = np.random.default_rng(13)
@@ -114,20 +131,21 @@ def test_decode_block_exact_integer_inputs(idx):
     D.q = W.bf16_bits(rng.integers(-8, 9, size=D.q.shape).astype(np.float32))
     D.kcache = W.bf16_bits(rng.integers(-8, 9, size=D.kcache.shape).astype(np.float32))
     D.w = rng.choice(np.array([0.0, 0.25, 0.5, 1.0], np.float32), size=D.w.shape)
-    got, st, _ = _run(idx, D, topk, c)
+    got, st, _ = _run(idx, D, topk, c, rule)
     assert st == "IDX_OK"
-    want = O.decode_topk(D.q, D.kcache, D.w, D.kv_len, topk, c, O.BLOCK, bn=64)
+    want = O.decode_topk(D.q, D.kcache, D.w, D.kv_len, topk, c, _MODE[rule], bn=64)
     _check(got, want, D.kv_len, G, topk)
     assert recall(got, want) >= 0.99
 
 
-def test_decode_block_full_length(idx):
-    # the bench's request length, sampled requests checked against the oracle
+@pytest.mark.parametrize("rule", ["mean", "quest"])
+def test_decode_block_full_length(idx, rule):
+    # the bench's request length, requests of several lengths checked against the oracle
     topk, c, G = 2048, 4096, 2
     D = W.decode(B=4, n=131072, G=G, H=64, d=128, topk=topk, seed=14, kv_len=[131072, 100000, 65536, 4097])
-    got, st, _ = _run(idx, D, topk, c)
+    got, st, _ = _run(idx, D, topk, c, rule)
     assert st == "IDX_OK"
-    want = O.decode_topk(D.q, D.kcache, D.w, D.kv_len, topk, c, O.BLOCK, bn=64)
+    want = O.decode_topk(D.q, D.kcache, D.w, D.kv_len, topk, c, _MODE[rule], bn=64)
     _check(got, want, D.kv_len, G, topk)
     assert recall(got, want) >= 0.999
 
@@ -139,7 +157,7 @@ def test_decode_block_invalid_kv_len(idx):
     kv = torch.tensor([256, 1, 257], dtype=torch.int32, device="cuda")   # 1 < G, 257 > n_max
     kbar = idx.decode_block_means(kc)
     ws = torch.empty(idx.decode_block_workspace_size(3, G, 256, 64, 128, topk, c), dtype=torch.uint8, device="cuda")
-    out = idx.decode_block_topk(q, kc, kbar, kv, w, topk, c, workspace=ws).cpu().numpy()
+    out = idx.decode_block_topk(q, kc, kbar, kv, w, topk, c, "mean", workspace=ws).cpu().numpy()
     assert idx.device_status(ws) == "IDX_ERR_INVALID"
     assert (out[1] == -1).all() and (out[2] == -1).all()
     want = O.decode_topk(D.q, D.kcache, D.w, np.array([256, 256, 256], np.int32), topk, c, O.BLOCK, bn=64)
