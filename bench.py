@@ -734,7 +734,35 @@ def main():
         blk = {"workload": f"block_prefilter_refine_2x{L // 2}_g{G_REF}_c{C_REF}_bn64", "ms_per_step": bms,
                "queries_per_s": world * L / (bms / 1000.0), "overlap_with_refine_topk": ov,
                "kernels": {n: {"launches": c, "ms_per_step": t / args.steps} for n, (c, t) in trb.items()}}
-        del ws3, o3
+        del ws3
+        # the same with the blocks ranked by the Quest bound (CUDA-core block scan)
+        ws4 = torch.empty(idx.pivot_workspace_size(L, H, D, TOPK, 2, G_REF, C_REF, "quest"), dtype=torch.uint8,
+                          device=dev)
+
+        def qstep():
+            idx.pivot_topk(q, k, w, cu2, TOPK, G_REF, C_REF, "quest", out_idx=o3, workspace=ws4)
+
+        for _ in range(args.warmup):
+            qstep()
+        torch.cuda.synchronize()
+        assert idx.device_status(ws4) == "IDX_OK"
+        barrier()
+        lib.idx_trace_enable(1)
+        e0.record(stream)
+        for _ in range(args.steps):
+            qstep()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        lib.idx_trace_enable(0)
+        barrier()
+        qms = max_over_ranks(e0.elapsed_time(e1) / args.steps)
+        _, trq = trace_report(lib)
+        a, b_ = o2[srows].cpu().numpy(), o3[srows].cpu().numpy()
+        ovq = float(np.mean([len(set(x[x >= 0]) & set(y[y >= 0])) / max(1, (x >= 0).sum()) for x, y in zip(a, b_)]))
+        blk["quest"] = {"ms_per_step": qms, "queries_per_s": world * L / (qms / 1000.0),
+                        "overlap_with_refine_topk": ovq,
+                        "kernels": {n: {"launches": c, "ms_per_step": t / args.steps} for n, (c, t) in trq.items()}}
+        del ws4, o3
 
     # ------------------------------- token-sparse attention on the selections
     att = None

@@ -40,6 +40,16 @@
  *                      t_last.  Members then re-score C as in Refine.  No
  *                      key after t_last takes part.  c must be a multiple of
  *                      64 and >= topk.
+ *   - IDX_MODE_QUEST:  IDX_MODE_BLOCK with the blocks ranked by the Quest
+ *                      bound instead of the mean key (same page, Sec. 3.1,
+ *                      Eq. (2)): a block is summarised by the per-dimension
+ *                      minimum and maximum of its keys, and its proxy score
+ *                      is sum_h wbar_h * max(0, sum_i max(qbar_hi * kmax_i,
+ *                      qbar_hi * kmin_i)), the indexer's weighted ReLU of
+ *                      each head's upper bound of q . k over the block.
+ *                      Scored on CUDA cores in fp32; H * d * 8 bytes must fit
+ *                      in one block's shared memory (else
+ *                      IDX_ERR_UNSUPPORTED).
  *
  * Decode form (same page, Method, decode paragraph): the G queries of one
  * MTP step form one group; query m of request b sits at position
@@ -85,7 +95,13 @@ typedef enum {
 
 typedef enum { IDX_BF16 = 0, IDX_F32 = 1 } idx_dtype;
 
-typedef enum { IDX_MODE_DENSE = 0, IDX_MODE_REUSE = 1, IDX_MODE_REFINE = 2, IDX_MODE_BLOCK = 3 } idx_mode;
+typedef enum {
+    IDX_MODE_DENSE = 0,
+    IDX_MODE_REUSE = 1,
+    IDX_MODE_REFINE = 2,
+    IDX_MODE_BLOCK = 3,
+    IDX_MODE_QUEST = 4
+} idx_mode;
 
 /* ------------------------------------------------------------ prefill */
 
@@ -141,7 +157,7 @@ idx_status idx_adaptive_topk(const void *q, const void *k, const float *w, const
                              idx_dtype dtype, int *out_idx, float *out_score, float *out_sigma,
                              uint8_t *out_trigger, void *ws, size_t ws_bytes, idx_stream_t stream);
 
-/* Workspace bytes for idx_pivot_topk (mode REUSE, REFINE or BLOCK) with the
+/* Workspace bytes for idx_pivot_topk (mode REUSE, REFINE, BLOCK or QUEST) with the
  * same dense_below; 0 for arguments idx_pivot_topk would reject. */
 size_t idx_pivot_workspace_size(int T, int H, int d, int topk, int num_seqs, idx_dtype dtype, int g,
                                 int c, idx_mode mode, int dense_below);
@@ -149,9 +165,9 @@ size_t idx_pivot_workspace_size(int T, int H, int d, int topk, int num_seqs, idx
 /* PIVOT grouped indexer + top-k (Reuse, Refine or block pre-filter Refine)
  * over a packed batch.  Same tensors and layouts as idx_dense_topk, plus
  *   g     group size (>= 1); groups are request-local [m*g, min((m+1)*g, n))
- *   c     candidate budget in tokens for REFINE and BLOCK (c >= topk; BLOCK:
- *         a multiple of 64); ignored for REUSE
- *   mode  IDX_MODE_REUSE, IDX_MODE_REFINE or IDX_MODE_BLOCK
+ *   c     candidate budget in tokens for REFINE, BLOCK and QUEST (c >= topk;
+ *         BLOCK, QUEST: a multiple of 64); ignored for REUSE
+ *   mode  IDX_MODE_REUSE, IDX_MODE_REFINE, IDX_MODE_BLOCK or IDX_MODE_QUEST
  *   dense_below  the guardrail (PIVOT page, Results, indexer speed: PIVOT
  *         falls back to a dense scan for short groups, so that it is never
  *         slower than the dense indexer; the page gives no threshold).  A
@@ -160,8 +176,8 @@ size_t idx_pivot_workspace_size(int T, int H, int d, int topk, int num_seqs, idx
  *         dense top-k, exactly as idx_dense_topk would.  Those groups are
  *         the first min(n, floor(dense_below / g) * g) tokens of a request
  *         (all n when n <= dense_below); the other groups are unchanged.
- *         0 turns it off.  REUSE and REFINE only (BLOCK: IDX_ERR_UNSUPPORTED
- *         for dense_below > 0).  For REFINE a threshold of at most c changes
+ *         0 turns it off.  REUSE and REFINE only (BLOCK, QUEST:
+ *         IDX_ERR_UNSUPPORTED for dense_below > 0).  For REFINE a threshold of at most c changes
  *         no result: such a group's candidate set is its whole prefix.
  * IDX_ERR_INVALID for g < 1, dense_below < 0, an unknown mode or a c these
  * rules reject. */

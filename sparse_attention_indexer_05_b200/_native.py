@@ -10,7 +10,7 @@ LIB_PATH = os.path.join(HERE, "libidx.so")
 STATUS = {0: "IDX_OK", 1: "IDX_ERR_INVALID", 2: "IDX_ERR_UNSUPPORTED", 3: "IDX_ERR_WORKSPACE",
           4: "IDX_ERR_CUDA", 5: "IDX_ERR_TIMEOUT", 6: "IDX_ERR_OVERFLOW"}
 BF16, F32 = 0, 1
-MODE_DENSE, MODE_REUSE, MODE_REFINE, MODE_BLOCK = 0, 1, 2, 3
+MODE_DENSE, MODE_REUSE, MODE_REFINE, MODE_BLOCK, MODE_QUEST = 0, 1, 2, 3, 4
 
 # every entry point of include/idx.h: name -> (restype, argtypes)
 _vp, _fp, _ip = ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p

@@ -55,10 +55,13 @@ struct PrefillWs {
     long long Rb;         // scored rows of one call's output rows (per-row scratch)
     long long Mb;         // members of one call's groups (member scores)
     unsigned cap, ksel;
-    size_t status, plan, slot, qbar, wbar, cnt, floor, buf, cand, msc, ckeys, kblk, cblk, total;
+    size_t status, plan, slot, qbar, wbar, cnt, floor, buf, cand, msc, ckeys, kblk, cblk, qspill, total;
+    long long nbmax;      // Quest: blocks of the longest request (spill row stride)
 };
 
-bool refines(idx_mode m) { return m == IDX_MODE_REFINE || m == IDX_MODE_BLOCK; }
+// the block pre-filter, blocks ranked by their mean key or by the Quest bound
+bool blocky(idx_mode m) { return m == IDX_MODE_BLOCK || m == IDX_MODE_QUEST; }
+bool refines(idx_mode m) { return m == IDX_MODE_REFINE || blocky(m); }
 
 long long block_rows(int T) { return (T >> kBlockShift) > 0 ? (T >> kBlockShift) : 1; }
 
@@ -95,9 +98,10 @@ PrefillWs prefill_ws(int T, int H, int d, int topk, int S, idx_dtype dt, int g, 
     L.pl.maxtiles = (int)(nbound(T) / KT + 1);
     L.ksel = mode == IDX_MODE_REUSE    ? (unsigned)(topk + g - 1)
              : mode == IDX_MODE_REFINE ? (unsigned)c
-             : mode == IDX_MODE_BLOCK  ? (unsigned)(c >> kBlockShift)
+             : blocky(mode)            ? (unsigned)(c >> kBlockShift)
                                        : (unsigned)topk;
-    L.cap = mode == IDX_MODE_BLOCK ? cap_for(L.ksel, (nbound(T) >> kBlockShift) + 1) : cap_for(L.ksel, nbound(T));
+    L.cap = blocky(mode) ? cap_for(L.ksel, (nbound(T) >> kBlockShift) + 1) : cap_for(L.ksel, nbound(T));
+    L.nbmax = (nbound(T) >> kBlockShift) + 1;
     Carve cv;
     L.status = cv.take(16);
     L.plan = cv.take(L.pl.words() * 4);
@@ -112,8 +116,11 @@ PrefillWs prefill_ws(int T, int H, int d, int topk, int S, idx_dtype dt, int g, 
     L.ckeys = (refines(mode) && tc_gather_supported(H, d, (int)dt, g, c))
                   ? cv.take((size_t)L.Rb * c_pad_of(c) * d * esize(dt))
                   : 0;
-    L.kblk = mode == IDX_MODE_BLOCK ? cv.take((size_t)block_rows(T) * d * esize(dt)) : 0;
-    L.cblk = mode == IDX_MODE_BLOCK ? cv.take((size_t)L.Rb * (c >> kBlockShift) * 4) : 0;
+    // block means [T / 64, d], or the Quest rule's per-block min and max [T / 64, 2, d]
+    L.kblk = blocky(mode) ? cv.take((size_t)block_rows(T) * d * esize(dt) * (mode == IDX_MODE_QUEST ? 2 : 1)) : 0;
+    L.cblk = blocky(mode) ? cv.take((size_t)L.Rb * (c >> kBlockShift) * 4) : 0;
+    // Quest: the proxies' block scores, one row of nbmax per scored proxy
+    L.qspill = mode == IDX_MODE_QUEST ? cv.take((size_t)L.Rb * L.nbmax * 4) : 0;
     L.total = cv.off;
     return L;
 }
@@ -264,6 +271,8 @@ struct Prefill {
                              reinterpret_cast<float *>(ws + L.wbar), (int)L.R, st);
         if (e == cudaSuccess && mode == IDX_MODE_BLOCK)
             e = launch_block_means(k, cu, S, T, d, (int)dt, ws + L.kblk, st);
+        if (e == cudaSuccess && mode == IDX_MODE_QUEST)
+            e = launch_block_minmax(k, cu, S, T, d, (int)dt, ws + L.kblk, st);
         return e;
     }
 
@@ -431,10 +440,11 @@ size_t idx_pivot_workspace_size_rows(int T, int H, int d, int topk, int num_seqs
                                      idx_mode mode, int dense_below, int max_rows) {
     if (T < 1 || num_seqs < 1 || topk < 1 || g < 1 || dense_below < 0 || max_rows < 0 || !shape_ok(H, d, dtype))
         return 0;
-    if (mode != IDX_MODE_REUSE && mode != IDX_MODE_REFINE && mode != IDX_MODE_BLOCK) return 0;
+    if (mode != IDX_MODE_REUSE && mode != IDX_MODE_REFINE && !blocky(mode)) return 0;
     if (mode == IDX_MODE_REUSE) c = topk;
     if (refines(mode) && c < topk) return 0;
-    if (mode == IDX_MODE_BLOCK && (c < kBlockN || c % kBlockN != 0 || dense_below > 0)) return 0;
+    if (blocky(mode) && (c < kBlockN || c % kBlockN != 0 || dense_below > 0)) return 0;
+    if (mode == IDX_MODE_QUEST && quest_scan_smem(H, d) > kMaxSmem) return 0;
     return prefill_ws(T, H, d, topk, num_seqs, dtype, g, c, mode, dense_below, max_rows).total;
 }
 
@@ -447,12 +457,13 @@ idx_status idx_pivot_topk_rows(const void *q, const void *k, const float *w, con
                                int T, int H, int d, int topk, idx_dtype dtype, int g, int c, idx_mode mode,
                                int dense_below, int row_lo, int row_hi, int *out_idx, float *out_score, void *ws,
                                size_t ws_bytes, idx_stream_t stream) {
-    if (g < 1 || dense_below < 0 || (mode != IDX_MODE_REUSE && mode != IDX_MODE_REFINE && mode != IDX_MODE_BLOCK))
+    if (g < 1 || dense_below < 0 || (mode != IDX_MODE_REUSE && mode != IDX_MODE_REFINE && !blocky(mode)))
         return IDX_ERR_INVALID;
     if (row_lo < 0 || row_hi < row_lo || row_hi > T) return IDX_ERR_INVALID;
     if (refines(mode) && c < topk) return IDX_ERR_INVALID;
-    if (mode == IDX_MODE_BLOCK && (c < kBlockN || c % kBlockN != 0)) return IDX_ERR_INVALID;
-    if (mode == IDX_MODE_BLOCK && dense_below > 0) return IDX_ERR_UNSUPPORTED;
+    if (blocky(mode) && (c < kBlockN || c % kBlockN != 0)) return IDX_ERR_INVALID;
+    if (blocky(mode) && dense_below > 0) return IDX_ERR_UNSUPPORTED;
+    if (mode == IDX_MODE_QUEST && quest_scan_smem(H, d) > kMaxSmem) return IDX_ERR_UNSUPPORTED;
     // every request is at most T tokens long: with dense_below >= T every
     // group is short and the call is the dense call (the same rows, without
     // the grouped pipeline's extra work)
@@ -471,7 +482,10 @@ idx_status idx_pivot_topk_rows(const void *q, const void *k, const float *w, con
                                  need);
     if (s != IDX_OK) return s;
     if (row_lo == row_hi) return IDX_OK;
-    TracePhase phase(mode == IDX_MODE_REUSE ? "reuse" : mode == IDX_MODE_REFINE ? "refine" : "block");
+    TracePhase phase(mode == IDX_MODE_REUSE    ? "reuse"
+                     : mode == IDX_MODE_REFINE ? "refine"
+                     : mode == IDX_MODE_BLOCK  ? "block"
+                                               : "quest");
     Prefill P{q, k, w, cu_seqlens, num_seqs, T, H, d, topk, dtype, g, c, mode, static_cast<char *>(ws),
               prefill_ws(T, H, d, topk, num_seqs, dtype, g, c, mode, dense_below, m),
               reinterpret_cast<cudaStream_t>(stream)};
@@ -479,10 +493,28 @@ idx_status idx_pivot_topk_rows(const void *q, const void *k, const float *w, con
     P.row_lo = row_lo;
     P.row_hi = row_hi;
     TRY_CUDA(P.prepare());
+    int *cand = reinterpret_cast<int *>(P.ws + P.L.cand);
+    if (mode == IDX_MODE_QUEST) {
+        // the proxies' Quest bounds of their complete blocks, the top blocks
+        // of each, then the candidate positions as in the block-mean rule
+        float *qsp = reinterpret_cast<float *>(P.ws + P.L.qspill);
+        int *cblk = reinterpret_cast<int *>(P.ws + P.L.cblk);
+        TRY_CUDA(launch_prefill_quest_scan(P.ws + P.L.qbar, reinterpret_cast<const float *>(P.ws + P.L.wbar),
+                                           P.ws + P.L.kblk, cu_seqlens, num_seqs, g, P.plan(), P.L.pl, (int)P.L.R,
+                                           (int)P.L.nbmax, H, d, (int)dtype, qsp, P.L.nbmax, P.st));
+        SelectArgs sa = P.select_args(SEL_PROXY_SPILL_TO_BLOCKS, (int)P.L.R, c >> kBlockShift, cblk, nullptr);
+        sa.scores = qsp;
+        sa.ld = P.L.nbmax;
+        TRY_CUDA(launch_select(sa, P.st));
+        TRY_CUDA(launch_block_expand(cu_seqlens, num_seqs, g, P.plan(), P.L.pl, cblk, cand, c, (int)P.L.R, P.st));
+        const GatherArgs ga = P.gather_args();
+        TRY_CUDA(tc_gather_supported(H, d, (int)dtype, g, c) ? launch_gather_tc(ga, P.st)
+                                                           : launch_gather_simt(ga, (int)dtype, P.st));
+        return cuda_st(launch_select(P.select_args(SEL_MEMBER_SCORES, T, topk, out_idx, out_score), P.st));
+    }
     TRY_CUDA(P.score(P.score_args(true)));
     if (mode == IDX_MODE_REUSE)
         return cuda_st(launch_select(P.select_args(SEL_REUSE_CAND, T, topk, out_idx, out_score), P.st));
-    int *cand = reinterpret_cast<int *>(P.ws + P.L.cand);
     if (mode == IDX_MODE_BLOCK) {
         int *cblk = reinterpret_cast<int *>(P.ws + P.L.cblk);
         TRY_CUDA(launch_select(P.select_args(SEL_PROXY_TO_BLOCKS, (int)P.L.R, c >> kBlockShift, cblk, nullptr),

@@ -143,7 +143,9 @@ enum SelKind {
     SEL_DEC_MEMBER = 7,     // decode: member scores over the candidate set
     SEL_PROXY_TO_BLOCKS = 8, // block pre-filter: complete blocks of a proxy row (k = c / kBlockN, one
                              // fewer when the row's prefix ends inside a block), block indices only
-    SEL_DEC_PROXY_TO_BLOCKS = 9 // decode block mode: the same over request b's block-score spill row
+    SEL_DEC_PROXY_TO_BLOCKS = 9, // decode block mode: the same over request b's block-score spill row
+    SEL_PROXY_SPILL_TO_BLOCKS = 10 // prefill block mode, Quest rule: the same over a proxy's block-score
+                                   // spill row (scores, ld), into cand = the selected blocks [R, k]
 };
 
 struct SelectArgs {
@@ -262,6 +264,14 @@ cudaError_t launch_decode_block_len(const int *kv_len, int B, int G, int n_max, 
 cudaError_t launch_decode_block_minmax(const void *kc, int B, int n_max, int d, int dtype, int first_block,
                                        void *kq, cudaStream_t st);
 size_t quest_scan_smem(int H, int d);
+// prefill block mode with the Quest bound: per-block key min/max of every
+// request ([T / 64, 2, d], placed as the block means), and the proxy rows'
+// bound scores of their complete blocks into spill rows (stride ld)
+cudaError_t launch_block_minmax(const void *k, const int *cu, int S, int T, int d, int dtype, void *kq,
+                                cudaStream_t st);
+cudaError_t launch_prefill_quest_scan(const void *qbar, const float *wbar, const void *kq, const int *cu, int S,
+                                      int g, const int *plan, const PlanLayout &pl, int R, int nbmax, int H, int d,
+                                      int dtype, float *spill, long long ld, cudaStream_t st);
 cudaError_t launch_decode_quest_scan(const void *qbar, const float *wbar, const void *kq, const int *nlen, int B,
                                      int nb, int H, int d, int dtype, float *spill, cudaStream_t st);
 cudaError_t launch_decode_block_expand(const int *kv_len, int B, int G, int n_max, const int *cblk, int *cand,

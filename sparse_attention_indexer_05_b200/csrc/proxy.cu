@@ -214,42 +214,40 @@ __global__ void __launch_bounds__(kProxyThreads) decode_block_minmax_kernel(cons
     Vec<T>::store(dst + d, hi);
 }
 
-// Decode block scores by the Quest bound: for the proxy of request b (qbar
-// [H, d], wbar [H]) and each complete block j < nlen[b],
+// Block scores by the Quest bound ("Uncertainty-gated selection for
+// block-sparse attention", Sec. 3.1, Eq. (2)): for one proxy (qbar [H, d],
+// wbar [H]) and each complete block j < nl of its request,
 //     bound_h = sum_i max(q_hi * kmax_i, q_hi * kmin_i)   (i ascending, fp32)
 //     score   = sum_h wbar_h * max(bound_h, 0)           (h ascending)
-// to spill [b * nb + j].  max(q a, q b) with a >= b is q a for q >= 0 and q b
-// otherwise, so the bound is accumulated as two FMAs with q+ = max(q, 0) and
-// q- = min(q, 0) (the zero product adds nothing).  The proxy's q+ and q- sit
-// in shared memory as fp32 (H * d * 8 bytes) and are read as broadcasts;
-// each thread scores two blocks (kQuestPer), so every shared load feeds two
+// to out[j].  max(q a, q b) with a >= b is q a for q >= 0 and q b otherwise,
+// so the bound is accumulated as two FMAs with q+ = max(q, 0) and q- =
+// min(q, 0) (the zero product adds nothing).  The proxy's q+ and q- sit in
+// shared memory as fp32 (H * d * 8 bytes) and are read as broadcasts; each
+// thread scores two blocks (kQuestPer), so every shared load feeds two
 // blocks' FMAs, with heads in chunks of 32 whose partial bounds stay in
-// registers.
+// registers.  kq holds the request's blocks from block 0: [*, 2, d] (kmin,
+// kmax).
 constexpr int kQuestThreads = 128;
 constexpr int kQuestPer = 2;
 
 template <typename T>
-__global__ void __launch_bounds__(kQuestThreads) decode_quest_scan_kernel(const T *qbar, const float *wbar,
-                                                                          const T *kq, const int *nlen, int nb,
-                                                                          int H, int d, float *spill) {
-    extern __shared__ __align__(16) float qs[];  // [H][d] q+, then [H][d] q-
-    const int b = blockIdx.y;
-    const int j0 = blockIdx.x * (kQuestThreads * kQuestPer) + threadIdx.x;  // blocks j0, j0 + kQuestThreads
-    const int nl = nlen[b];
-    if (blockIdx.x * (kQuestThreads * kQuestPer) >= nl) return;
-    const int HD = H * d;
+__device__ void quest_load_proxy(const T *qbar, int HD, float *qs) {
     for (int i = threadIdx.x; i < HD; i += blockDim.x) {
-        const float v = to_float(qbar[(long long)b * HD + i]);
+        const float v = to_float(qbar[i]);
         qs[i] = v > 0.0f ? v : 0.0f;
         qs[HD + i] = v < 0.0f ? v : 0.0f;
     }
-    __syncthreads();
-    if (j0 >= nl) return;
-    const T *row[kQuestPer];  // kmin, then kmax; a block past nlen repeats the first (not stored)
+}
+
+template <typename T>
+__device__ void quest_block_scores(const float *qs, const float *wbar, const T *kq, int nl, int j0, int H, int d,
+                                   float *out) {
+    const int HD = H * d;
+    const T *row[kQuestPer];  // a block past nl repeats the first (not stored)
 #pragma unroll
     for (int u = 0; u < kQuestPer; ++u) {
         const int j = j0 + u * kQuestThreads < nl ? j0 + u * kQuestThreads : j0;
-        row[u] = kq + ((long long)b * nb + j) * 2 * d;
+        row[u] = kq + (long long)j * 2 * d;
     }
     float total[kQuestPer];
 #pragma unroll
@@ -291,7 +289,7 @@ __global__ void __launch_bounds__(kQuestThreads) decode_quest_scan_kernel(const 
 #pragma unroll
         for (int hh = 0; hh < 32; ++hh) {
             if (h0 + hh < H) {
-                const float wh = wbar[(long long)b * H + h0 + hh];
+                const float wh = wbar[h0 + hh];
 #pragma unroll
                 for (int u = 0; u < kQuestPer; ++u) total[u] = fmaf(wh, fmaxf(acc[u][hh], 0.0f), total[u]);
             }
@@ -299,7 +297,94 @@ __global__ void __launch_bounds__(kQuestThreads) decode_quest_scan_kernel(const 
     }
 #pragma unroll
     for (int u = 0; u < kQuestPer; ++u)
-        if (j0 + u * kQuestThreads < nl) spill[(long long)b * nb + j0 + u * kQuestThreads] = total[u];
+        if (j0 + u * kQuestThreads < nl) out[j0 + u * kQuestThreads] = total[u];
+}
+
+// Decode: the proxy of request b against its complete blocks j < nlen[b];
+// kq [B, nb, 2, d], scores to spill [b * nb + j].
+template <typename T>
+__global__ void __launch_bounds__(kQuestThreads, 3) decode_quest_scan_kernel(const T *qbar, const float *wbar,
+                                                                          const T *kq, const int *nlen, int nb,
+                                                                          int H, int d, float *spill) {
+    extern __shared__ __align__(16) float qs[];  // [H][d] q+, then [H][d] q-
+    const int b = blockIdx.y;
+    const int j0 = blockIdx.x * (kQuestThreads * kQuestPer) + threadIdx.x;
+    const int nl = nlen[b];
+    if (blockIdx.x * (kQuestThreads * kQuestPer) >= nl) return;
+    quest_load_proxy(qbar + (long long)b * H * d, H * d, qs);
+    __syncthreads();
+    if (j0 >= nl) return;
+    quest_block_scores(qs, wbar + (long long)b * H, kq + (long long)b * nb * 2 * d, nl, j0, H, d,
+                       spill + (long long)b * nb);
+}
+
+// Prefill block mode with the Quest bound: proxy row p (its request b, its
+// group's last member t_last) against the complete blocks j < (t_last + 1) /
+// 64 of its request; kq [T / 64, 2, d] with request b's blocks from row
+// cu[b] / 64; scores to spill [(p - plan[6]) * ld + j] (the call's scratch
+// rows, as the other per-row scratch).
+template <typename T>
+__global__ void __launch_bounds__(kQuestThreads, 3) prefill_quest_scan_kernel(const T *qbar, const float *wbar,
+                                                                           const T *kq, const int *cu, int S,
+                                                                           int g, const int *plan, PlanLayout pl,
+                                                                           int H, int d, float *spill, long long ld) {
+    extern __shared__ __align__(16) float qs[];
+    const int p = blockIdx.y;
+    if (!plan[0] || p >= plan[2] || !scored_in_range(plan, p)) return;
+    const int *rp = plan + pl.rp();
+    const int b = find_seg(rp, S, p);
+    const int i = p - rp[b];
+    const int n = cu[b + 1] - cu[b];
+    const int tl = row_bound(i, n, g);
+    const int nl = (tl + 1) >> kBlockShift;
+    const int j0 = blockIdx.x * (kQuestThreads * kQuestPer) + threadIdx.x;
+    if (blockIdx.x * (kQuestThreads * kQuestPer) >= nl) return;
+    quest_load_proxy(qbar + (long long)p * H * d, H * d, qs);
+    __syncthreads();
+    if (j0 >= nl) return;
+    quest_block_scores(qs, wbar + (long long)p * H, kq + (long long)(cu[b] >> kBlockShift) * 2 * d, nl, j0, H, d,
+                       spill + ((long long)p - plan[6]) * ld);
+}
+
+// Prefill block summaries for the Quest bound: the per-dimension minimum and
+// maximum of each complete block of each request, block i of request b to
+// rows 2 x and 2 x + 1 of kq, x = (cu[b] >> 6) + i (as block_mean_kernel
+// places its means); rows that belong to no complete block are zero.
+template <typename T>
+__global__ void __launch_bounds__(kProxyThreads) block_minmax_kernel(const T *k, const int *cu, int S, int T_,
+                                                                     int d, long long nrows, T *kq) {
+    const int per_row = d / 8;
+    const long long u = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    if (u >= nrows * per_row) return;
+    const long long x = u / per_row;
+    const int e = (int)(u - x * per_row) * 8;
+    int lo = 0, hi = S;
+    while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if ((long long)(cu[mid] >> kBlockShift) <= x) lo = mid; else hi = mid;
+    }
+    const long long i = x - (cu[lo] >> kBlockShift);
+    const bool ok = cu[lo] >= 0 && cu[lo] <= cu[lo + 1] && cu[lo + 1] <= T_;
+    const int nfull = ok ? (cu[lo + 1] - cu[lo]) >> kBlockShift : 0;
+    float mn[8], mx[8], v[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) mn[j] = mx[j] = 0.0f;
+    if (i < nfull) {
+        const T *src = k + ((long long)cu[lo] + i * kBlockN) * d + e;
+        Vec<T>::load(src, mn);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) mx[j] = mn[j];
+        for (int r = 1; r < kBlockN; ++r) {
+            Vec<T>::load(src + (long long)r * d, v);
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                mn[j] = fminf(mn[j], v[j]);
+                mx[j] = fmaxf(mx[j], v[j]);
+            }
+        }
+    }
+    Vec<T>::store(kq + x * 2 * d + e, mn);
+    Vec<T>::store(kq + x * 2 * d + d + e, mx);
 }
 
 // Decode block mode: the complete blocks each request's proxy scans,
@@ -468,6 +553,43 @@ cudaError_t launch_decode_quest_scan(const void *qbar, const float *wbar, const 
     else
         decode_quest_scan_kernel<__nv_bfloat16><<<grid, kQuestThreads, smem, st>>>(
             (const __nv_bfloat16 *)qbar, wbar, (const __nv_bfloat16 *)kq, nlen, nb, H, d, spill);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_block_minmax(const void *k, const int *cu, int S, int T, int d, int dtype, void *kq,
+                                cudaStream_t st) {
+    const long long nrows = (T >> kBlockShift) > 0 ? (T >> kBlockShift) : 1;
+    const long long units = nrows * (d / 8);
+    TraceScope ts("block_minmax", st);
+    const unsigned grid = (unsigned)((units + kProxyThreads - 1) / kProxyThreads);
+    if (dtype == 1)
+        block_minmax_kernel<float><<<grid, kProxyThreads, 0, st>>>((const float *)k, cu, S, T, d, nrows,
+                                                                   (float *)kq);
+    else
+        block_minmax_kernel<__nv_bfloat16><<<grid, kProxyThreads, 0, st>>>((const __nv_bfloat16 *)k, cu, S, T, d,
+                                                                           nrows, (__nv_bfloat16 *)kq);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_prefill_quest_scan(const void *qbar, const float *wbar, const void *kq, const int *cu, int S,
+                                      int g, const int *plan, const PlanLayout &pl, int R, int nbmax, int H, int d,
+                                      int dtype, float *spill, long long ld, cudaStream_t st) {
+    if (R <= 0 || nbmax <= 0) return cudaSuccess;
+    const size_t smem = quest_scan_smem(H, d);
+    cudaError_t e = dtype == 1 ? cudaFuncSetAttribute(prefill_quest_scan_kernel<float>,
+                                                      cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)
+                               : cudaFuncSetAttribute(prefill_quest_scan_kernel<__nv_bfloat16>,
+                                                      cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    const int per_cta = kQuestThreads * kQuestPer;
+    const dim3 grid((unsigned)((nbmax + per_cta - 1) / per_cta), (unsigned)R);
+    TraceScope ts("quest_scan", st);
+    if (dtype == 1)
+        prefill_quest_scan_kernel<float><<<grid, kQuestThreads, smem, st>>>(
+            (const float *)qbar, wbar, (const float *)kq, cu, S, g, plan, pl, H, d, spill, ld);
+    else
+        prefill_quest_scan_kernel<__nv_bfloat16><<<grid, kQuestThreads, smem, st>>>(
+            (const __nv_bfloat16 *)qbar, wbar, (const __nv_bfloat16 *)kq, cu, S, g, plan, pl, H, d, spill, ld);
     return cudaGetLastError();
 }
 

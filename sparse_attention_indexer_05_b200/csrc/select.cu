@@ -406,6 +406,30 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(SelectArgs a) {
         }
         return;
     }
+    case SEL_PROXY_SPILL_TO_BLOCKS: {
+        // prefill block mode (Quest rule): proxy row p's top blocks among the
+        // complete blocks of its prefix (t_last + 1) / 64, k = c / 64 slots,
+        // one of them kept for the partial block when the prefix ends inside
+        // a block; rows of the call's scratch from plan[6]
+        const int p = row;
+        if (!a.plan[0] || p >= a.plan[2] || !scored_in_range(a.plan, p)) return;
+        const long long sp = (long long)p - a.plan[6];
+        int *ob = a.out_idx + sp * a.k;
+        const int *rp = a.plan + a.pl.rp();
+        const int b = find_seg(rp, a.S, p);
+        const int i = p - rp[b];
+        const int n = a.cu[b + 1] - a.cu[b];
+        const int tl = row_bound(i, n, a.g);
+        const int nfull = (tl + 1) >> kBlockShift;
+        const int want = a.k - (((tl + 1) & (kBlockN - 1)) != 0 ? 1 : 0);
+        const int take = want < nfull ? want : nfull;
+        if (take > 0) {
+            ScoreSrc src{a.scores + sp * a.ld, nullptr, nfull, nfull - 1};
+            block_select(src, take, ob, nullptr, sh, stage, a.stage_cap, bm, gpre, wcap, a.status);
+        }
+        for (int r = (take > 0 ? take : 0) + threadIdx.x; r < a.k; r += blockDim.x) ob[r] = -1;
+        return;
+    }
     case SEL_DEC_PROXY_TO_BLOCKS: {
         // the proxy's top blocks among request b's complete blocks: k = c / 64
         // slots, one of them kept for the partial block when kv_len[b] ends

@@ -22,7 +22,8 @@ import torch
 
 from . import _native as N
 
-MODES = {"dense": N.MODE_DENSE, "reuse": N.MODE_REUSE, "refine": N.MODE_REFINE, "block": N.MODE_BLOCK}
+MODES = {"dense": N.MODE_DENSE, "reuse": N.MODE_REUSE, "refine": N.MODE_REFINE, "block": N.MODE_BLOCK,
+         "quest": N.MODE_QUEST}
 
 
 def _mode(m) -> int:

@@ -53,6 +53,12 @@ def test_workspace_sizes(lib):
     assert lib.idx_pivot_workspace_size(65536, 64, 128, 2048, 1, 0, 4, 4096, 2, 1 << 20) >= guard
     assert lib.idx_pivot_workspace_size(65536, 64, 128, 2048, 1, 0, 4, 4096, 2, -1) == 0  # negative threshold
     assert lib.idx_pivot_workspace_size(65536, 64, 128, 2048, 1, 0, 4, 4096, 3, 64) == 0  # block mode
+    # the Quest rule: block mode's rules, and the proxy's q+/q- in shared memory
+    assert lib.idx_pivot_workspace_size(65536, 64, 128, 2048, 1, 0, 16, 4096, 4, 0) > 0
+    assert lib.idx_pivot_workspace_size(65536, 64, 128, 2048, 1, 0, 16, 4096 + 32, 4, 0) == 0
+    assert lib.idx_pivot_workspace_size(65536, 64, 128, 2048, 1, 0, 16, 4096, 4, 64) == 0
+    assert lib.idx_pivot_workspace_size(65536, 256, 256, 2048, 1, 0, 16, 4096, 4, 0) == 0
+    assert lib.idx_pivot_workspace_size(65536, 64, 128, 2048, 1, 0, 16, 4096, 5, 0) == 0   # no mode 5
     # row-range calls: the per-row scratch covers the call's rows only
     full = lib.idx_dense_workspace_size(131072, 64, 128, 2048, 1, 0)
     assert lib.idx_dense_workspace_size_rows(131072, 64, 128, 2048, 1, 0, 0) == full
