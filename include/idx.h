@@ -49,7 +49,10 @@
  *                      each head's upper bound of q . k over the block.
  *                      Scored on CUDA cores in fp32; H * d * 8 bytes must fit
  *                      in one block's shared memory (else
- *                      IDX_ERR_UNSUPPORTED).
+ *                      IDX_ERR_UNSUPPORTED).  The workspace holds one fp32
+ *                      score per (scored proxy, block of the longest
+ *                      request): 4 * (T / g) * (T / 64) bytes for one
+ *                      request of T tokens, bounded by row-range calls.
  *
  * Decode form (same page, Method, decode paragraph): the G queries of one
  * MTP step form one group; query m of request b sits at position

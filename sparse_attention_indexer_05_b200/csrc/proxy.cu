@@ -307,10 +307,10 @@ __global__ void __launch_bounds__(kQuestThreads, 3) decode_quest_scan_kernel(con
                                                                           const T *kq, const int *nlen, int nb,
                                                                           int H, int d, float *spill) {
     extern __shared__ __align__(16) float qs[];  // [H][d] q+, then [H][d] q-
-    const int b = blockIdx.y;
-    const int j0 = blockIdx.x * (kQuestThreads * kQuestPer) + threadIdx.x;
+    const int b = blockIdx.x;  // request (grid x: no 65535 limit); block chunk on grid y
+    const int j0 = blockIdx.y * (kQuestThreads * kQuestPer) + threadIdx.x;
     const int nl = nlen[b];
-    if (blockIdx.x * (kQuestThreads * kQuestPer) >= nl) return;
+    if (blockIdx.y * (kQuestThreads * kQuestPer) >= nl) return;
     quest_load_proxy(qbar + (long long)b * H * d, H * d, qs);
     __syncthreads();
     if (j0 >= nl) return;
@@ -329,7 +329,7 @@ __global__ void __launch_bounds__(kQuestThreads, 3) prefill_quest_scan_kernel(co
                                                                            int g, const int *plan, PlanLayout pl,
                                                                            int H, int d, float *spill, long long ld) {
     extern __shared__ __align__(16) float qs[];
-    const int p = blockIdx.y;
+    const int p = blockIdx.x;  // proxy row (grid x: no 65535 limit); block chunk on grid y
     if (!plan[0] || p >= plan[2] || !scored_in_range(plan, p)) return;
     const int *rp = plan + pl.rp();
     const int b = find_seg(rp, S, p);
@@ -337,8 +337,8 @@ __global__ void __launch_bounds__(kQuestThreads, 3) prefill_quest_scan_kernel(co
     const int n = cu[b + 1] - cu[b];
     const int tl = row_bound(i, n, g);
     const int nl = (tl + 1) >> kBlockShift;
-    const int j0 = blockIdx.x * (kQuestThreads * kQuestPer) + threadIdx.x;
-    if (blockIdx.x * (kQuestThreads * kQuestPer) >= nl) return;
+    const int j0 = blockIdx.y * (kQuestThreads * kQuestPer) + threadIdx.x;
+    if (blockIdx.y * (kQuestThreads * kQuestPer) >= nl) return;
     quest_load_proxy(qbar + (long long)p * H * d, H * d, qs);
     __syncthreads();
     if (j0 >= nl) return;
@@ -545,7 +545,7 @@ cudaError_t launch_decode_quest_scan(const void *qbar, const float *wbar, const 
                                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     const int per_cta = kQuestThreads * kQuestPer;
-    const dim3 grid((unsigned)((nb + per_cta - 1) / per_cta), (unsigned)B);
+    const dim3 grid((unsigned)B, (unsigned)((nb + per_cta - 1) / per_cta));
     TraceScope ts("quest_scan", st);
     if (dtype == 1)
         decode_quest_scan_kernel<float><<<grid, kQuestThreads, smem, st>>>((const float *)qbar, wbar,
@@ -582,7 +582,7 @@ cudaError_t launch_prefill_quest_scan(const void *qbar, const float *wbar, const
                                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     const int per_cta = kQuestThreads * kQuestPer;
-    const dim3 grid((unsigned)((nbmax + per_cta - 1) / per_cta), (unsigned)R);
+    const dim3 grid((unsigned)R, (unsigned)((nbmax + per_cta - 1) / per_cta));
     TraceScope ts("quest_scan", st);
     if (dtype == 1)
         prefill_quest_scan_kernel<float><<<grid, kQuestThreads, smem, st>>>(
