@@ -933,6 +933,39 @@ def main():
                 "speedup_vs_dense": (dec["dense"]["ms_per_step"] / step_ms) if step_ms > 0 else None,
                 "kernels": {n: {"launches": c, "ms_per_step": t / args.steps} for n, (c, t) in trd.items()}}
             del ksum, wsb
+        # the same steps captured once in a CUDA graph and replayed (a serving
+        # loop's form: no per-launch host work between the kernels)
+        graph = {}
+        kbar_g = idx.decode_block_means(dkc)
+        wsb_g = torch.empty(idx.decode_block_workspace_size(DEC_B, DEC_G, DEC_N, H, D, TOPK, C_REF),
+                            dtype=torch.uint8, device=dev)
+        gsteps = {"dense": lambda: idx.decode_topk(dq_, dkc, dkv, dw_, TOPK, C_REF, "dense", out_idx=od,
+                                                   workspace=wsd),
+                  "refine": lambda: idx.decode_topk(dq_, dkc, dkv, dw_, TOPK, C_REF, "refine", out_idx=od,
+                                                    workspace=wsd),
+                  "block_mean": lambda: idx.decode_block_topk(dq_, dkc, kbar_g, dkv, dw_, TOPK, C_REF, "mean",
+                                                              out_idx=od, workspace=wsb_g)}
+        for name, fn in gsteps.items():
+            gs = torch.cuda.Stream(dev)
+            gs.wait_stream(torch.cuda.current_stream())
+            with torch.cuda.stream(gs):
+                fn()
+            torch.cuda.synchronize()
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=gs):
+                fn()
+            for _ in range(args.warmup):
+                g.replay()
+            torch.cuda.synchronize()
+            e0.record(stream)
+            for _ in range(args.steps):
+                g.replay()
+            e1.record(stream)
+            torch.cuda.synchronize()
+            graph[name] = max_over_ranks(e0.elapsed_time(e1) / args.steps)
+            del g
+        dec["graph_ms_per_step"] = graph
+        del kbar_g, wsb_g
         dec["hbm_peak_GBps"] = hbm_peak
         del dpool, dbt, perm
 
