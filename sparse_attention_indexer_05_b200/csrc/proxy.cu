@@ -223,12 +223,13 @@ __global__ void __launch_bounds__(kProxyThreads) decode_block_minmax_kernel(cons
 // so the bound is accumulated as two FMAs with q+ = max(q, 0) and q- =
 // min(q, 0) (the zero product adds nothing).  The proxy's q+ and q- sit in
 // shared memory as fp32 (H * d * 8 bytes) and are read as broadcasts; each
-// thread scores two blocks (kQuestPer), so every shared load feeds two
-// blocks' FMAs, with heads in chunks of 32 whose partial bounds stay in
-// registers.  kq holds the request's blocks from block 0: [*, 2, d] (kmin,
+// thread scores four blocks (kQuestPer), so every shared load feeds four
+// blocks' FMAs and four independent FMA chains run per head, with heads in
+// chunks of 16 whose partial bounds stay in registers.  kq holds the request's blocks from block 0: [*, 2, d] (kmin,
 // kmax).
 constexpr int kQuestThreads = 128;
-constexpr int kQuestPer = 2;
+constexpr int kQuestPer = 4;
+constexpr int kQuestHeads = 16;  // heads per register chunk
 
 template <typename T>
 __device__ void quest_load_proxy(const T *qbar, int HD, float *qs) {
@@ -252,12 +253,12 @@ __device__ void quest_block_scores(const float *qs, const float *wbar, const T *
     float total[kQuestPer];
 #pragma unroll
     for (int u = 0; u < kQuestPer; ++u) total[u] = 0.0f;
-    for (int h0 = 0; h0 < H; h0 += 32) {
-        float acc[kQuestPer][32];
+    for (int h0 = 0; h0 < H; h0 += kQuestHeads) {
+        float acc[kQuestPer][kQuestHeads];
 #pragma unroll
         for (int u = 0; u < kQuestPer; ++u)
 #pragma unroll
-            for (int hh = 0; hh < 32; ++hh) acc[u][hh] = 0.0f;
+            for (int hh = 0; hh < kQuestHeads; ++hh) acc[u][hh] = 0.0f;
         for (int e = 0; e < d; e += 8) {
             float lo[kQuestPer][8], hi[kQuestPer][8];
 #pragma unroll
@@ -266,7 +267,7 @@ __device__ void quest_block_scores(const float *qs, const float *wbar, const T *
                 Vec<T>::load(row[u] + d + e, hi[u]);
             }
 #pragma unroll
-            for (int hh = 0; hh < 32; ++hh) {
+            for (int hh = 0; hh < kQuestHeads; ++hh) {
                 if (h0 + hh < H) {
                     const float4 *pp = reinterpret_cast<const float4 *>(qs + (h0 + hh) * d + e);
                     const float4 *pn = reinterpret_cast<const float4 *>(qs + HD + (h0 + hh) * d + e);
@@ -287,7 +288,7 @@ __device__ void quest_block_scores(const float *qs, const float *wbar, const T *
             }
         }
 #pragma unroll
-        for (int hh = 0; hh < 32; ++hh) {
+        for (int hh = 0; hh < kQuestHeads; ++hh) {
             if (h0 + hh < H) {
                 const float wh = wbar[h0 + hh];
 #pragma unroll

@@ -90,3 +90,27 @@ def test_quest_row_ranges_stitch_and_guardrail_refused(idx):
                                 N.BF16, g, c, N.MODE_QUEST, 256, oi.data_ptr(), None, ws.data_ptr(), ws.numel(),
                                 torch.cuda.current_stream().cuda_stream)
     assert rc == 2, N.STATUS.get(rc, rc)
+
+
+def test_quest_full_size_packed_2x65536_g16(idx):
+    # the bench's block leg: 2 x 65536 tokens, g = 16, c = 4096, sampled rows
+    # (the first and last of each request, the group edges around them, and
+    # random rows) against the oracle, and every row well formed
+    topk, g, c = 2048, 16, 4096
+    P = W.cfg_long_packed(seed=0)
+    q, k, w, cu = to_dev(P.q), to_dev(P.k), to_dev(P.w), to_dev(P.cu_seqlens)
+    ws = torch.empty(idx.pivot_workspace_size(P.T, 64, 128, topk, 2, g, c, "quest"), dtype=torch.uint8,
+                     device="cuda")
+    got = idx.pivot_topk(q, k, w, cu, topk, g, c, "quest", workspace=ws).cpu().numpy()
+    assert idx.device_status(ws) == "IDX_OK"
+    rng = np.random.default_rng(54)
+    rows = np.unique(np.concatenate([[0, 15, 16, 4095, 4096, 65535, 65536, 65551, 131071],
+                                     rng.integers(0, P.T, 16)])).astype(np.int64)
+    want = O.pivot_topk(P.q, P.k, P.w, P.cu_seqlens, topk, g, c, O.QUEST, rows=rows, bn=64)
+    assert recall(got[rows], want) >= 0.999
+    for r, wr in zip(rows, want):
+        t = int(r - (65536 if r >= 65536 else 0))
+        row = got[r]
+        sel = row[row >= 0]
+        assert len(sel) == int((wr >= 0).sum()), r
+        assert (np.diff(sel) > 0).all() and (sel <= t).all(), r
