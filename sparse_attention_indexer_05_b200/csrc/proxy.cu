@@ -225,8 +225,8 @@ __global__ void __launch_bounds__(kProxyThreads) decode_block_minmax_kernel(cons
 // shared memory as fp32 (H * d * 8 bytes) and are read as broadcasts; each
 // thread scores four blocks (kQuestPer), so every shared load feeds four
 // blocks' FMAs and four independent FMA chains run per head, with heads in
-// chunks of 16 whose partial bounds stay in registers.  kq holds the request's blocks from block 0: [*, 2, d] (kmin,
-// kmax).
+// chunks of 16 whose partial bounds stay in registers.  kq holds the
+// request's blocks from block 0: [*, 2, d] (kmin, kmax).
 constexpr int kQuestThreads = 128;
 constexpr int kQuestPer = 4;
 constexpr int kQuestHeads = 16;  // heads per register chunk
