@@ -99,17 +99,33 @@ def proxy_pairs(n, g):
     return tot
 
 
-SCORE_SOURCES = ["score_tc.cu", "tc.cuh", "common.cuh", "internal.h", "plan.cuh"]
+SCORE_SOURCES = ["score_tc.cu", "tc.cuh", "common.cuh", "plan.cuh"]
+# the parts of internal.h the score kernel reads: its constants, the plan
+# layout and its argument struct (other declarations there do not change it)
+SCORE_DECLS = [r"constexpr int (RB|KT|kMaxLen|kBlockShift|kBlockN) = [^;]*;",
+               r"struct PlanLayout \{.*?\n\};", r"enum Sink \{[^}]*\};", r"struct ScoreArgs \{.*?\n\};"]
 
 
 def score_sources_sha():
     """sha256 over the sources of the dense score kernel (to tell whether a
-    recorded ncu traffic figure still describes the kernel that runs)."""
+    recorded ncu traffic figure still describes the kernel that runs): its
+    source files whole, and from internal.h the declarations it uses."""
     import hashlib
+    import re
+    csrc = os.path.join(ROOT, "sparse_attention_indexer_05_b200", "csrc")
     h = hashlib.sha256()
     for f in SCORE_SOURCES:
-        with open(os.path.join(ROOT, "sparse_attention_indexer_05_b200", "csrc", f), "rb") as fh:
+        with open(os.path.join(csrc, f), "rb") as fh:
             h.update(fh.read())
+    with open(os.path.join(csrc, "internal.h")) as fh:
+        text = fh.read()
+    for pat in SCORE_DECLS:
+        found = re.findall(pat, text, flags=re.S) if "struct" in pat or "enum" in pat else \
+            [m.group(0) for m in re.finditer(pat, text)]
+        if not found:
+            raise RuntimeError(f"declaration not found in internal.h: {pat}")
+        for m in found:
+            h.update((m if isinstance(m, str) else m[0]).encode())
     return h.hexdigest()
 
 
