@@ -323,14 +323,17 @@ __global__ void __launch_bounds__(kQuestThreads, 3) decode_quest_scan_kernel(con
 // group's last member t_last) against the complete blocks j < (t_last + 1) /
 // 64 of its request; kq [T / 64, 2, d] with request b's blocks from row
 // cu[b] / 64; scores to spill [(p - plan[6]) * ld + j] (the call's scratch
-// rows, as the other per-row scratch).
+// rows, as the other per-row scratch).  One CTA per proxy walks all of its
+// blocks, so the proxy is loaded into shared memory once.
 template <typename T>
 __global__ void __launch_bounds__(kQuestThreads, 3) prefill_quest_scan_kernel(const T *qbar, const float *wbar,
                                                                            const T *kq, const int *cu, int S,
                                                                            int g, const int *plan, PlanLayout pl,
                                                                            int H, int d, float *spill, long long ld) {
     extern __shared__ __align__(16) float qs[];
-    const int p = blockIdx.x;  // proxy row (grid x: no 65535 limit); block chunk on grid y
+    // proxy row, the last first (a request's later proxies have the longer
+    // prefixes, so the grid's tail holds the short ones)
+    const int p = (int)(gridDim.x - 1 - blockIdx.x);
     if (!plan[0] || p >= plan[2] || !scored_in_range(plan, p)) return;
     const int *rp = plan + pl.rp();
     const int b = find_seg(rp, S, p);
@@ -338,13 +341,15 @@ __global__ void __launch_bounds__(kQuestThreads, 3) prefill_quest_scan_kernel(co
     const int n = cu[b + 1] - cu[b];
     const int tl = row_bound(i, n, g);
     const int nl = (tl + 1) >> kBlockShift;
-    const int j0 = blockIdx.y * (kQuestThreads * kQuestPer) + threadIdx.x;
-    if (blockIdx.y * (kQuestThreads * kQuestPer) >= nl) return;
+    if (nl <= 0) return;
     quest_load_proxy(qbar + (long long)p * H * d, H * d, qs);
     __syncthreads();
-    if (j0 >= nl) return;
-    quest_block_scores(qs, wbar + (long long)p * H, kq + (long long)(cu[b] >> kBlockShift) * 2 * d, nl, j0, H, d,
-                       spill + ((long long)p - plan[6]) * ld);
+    const T *kb = kq + (long long)(cu[b] >> kBlockShift) * 2 * d;
+    float *out = spill + ((long long)p - plan[6]) * ld;
+    for (int base = 0; base < nl; base += kQuestThreads * kQuestPer) {
+        const int j0 = base + threadIdx.x;
+        if (j0 < nl) quest_block_scores(qs, wbar + (long long)p * H, kb, nl, j0, H, d, out);
+    }
 }
 
 // Prefill block summaries for the Quest bound: the per-dimension minimum and
@@ -582,8 +587,7 @@ cudaError_t launch_prefill_quest_scan(const void *qbar, const float *wbar, const
                                : cudaFuncSetAttribute(prefill_quest_scan_kernel<__nv_bfloat16>,
                                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    const int per_cta = kQuestThreads * kQuestPer;
-    const dim3 grid((unsigned)R, (unsigned)((nbmax + per_cta - 1) / per_cta));
+    const unsigned grid = (unsigned)R;
     TraceScope ts("quest_scan", st);
     if (dtype == 1)
         prefill_quest_scan_kernel<float><<<grid, kQuestThreads, smem, st>>>(
