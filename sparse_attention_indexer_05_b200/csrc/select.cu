@@ -929,6 +929,7 @@ __device__ void fast_cand_row(const unsigned long long *buf, int n, unsigned flo
         for (int j = tid; j < nclr; j += kFT) bm[j] = 0u;
     }
     unsigned mx = 0u;
+    const unsigned long long lo1 = g.lo > 1ull ? g.lo : 1ull;
     // 8 keys per thread and round, as four 16-byte loads (rows start 2 KB
     // aligned); the next round's loads are issued before this round's keys
     // are filtered, so their latency overlaps the work
@@ -955,11 +956,11 @@ __device__ void fast_cand_row(const unsigned long long *buf, int n, unsigned flo
         unsigned cnt = 0;
 #pragma unroll
         for (int u = 0; u < 8; ++u) {
-            const bool ok = kv[u] >= g.lo && (unsigned)kv[u] >= g.pmin && kv[u] != 0ull;
+            // lo1 >= 1 also drops the empty key 0; a dropped key becomes 0 (ord 0)
+            const bool ok = kv[u] >= lo1 && (unsigned)kv[u] >= g.pmin;
             if (!ok) kv[u] = 0ull;
             cnt += ok ? 1u : 0u;
-            const unsigned o = key_ord(kv[u]);
-            mx = ok && o > mx ? o : mx;
+            mx = max(mx, key_ord(kv[u]));
         }
         unsigned inc = cnt;
 #pragma unroll
