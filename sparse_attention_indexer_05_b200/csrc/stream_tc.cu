@@ -120,46 +120,41 @@ __device__ __forceinline__ Item item_info(const GatherArgs &g, const DecodeArgs 
     return it;
 }
 
-// sum_j w[j] * max(v[j], 0) over 32 heads; w 16-byte aligned, read as float4
-__device__ __forceinline__ float reduce32(const uint32_t (&v)[32], const float *w) {
-    const float4 *w4 = reinterpret_cast<const float4 *>(w);
-    float a[8];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) a[i] = 0.0f;
-#pragma unroll
-    for (int j4 = 0; j4 < 8; ++j4) {
-        const float4 wv = w4[j4];
-        a[(4 * j4 + 0) & 7] = fmaf(wv.x, fmaxf(__uint_as_float(v[4 * j4 + 0]), 0.0f), a[(4 * j4 + 0) & 7]);
-        a[(4 * j4 + 1) & 7] = fmaf(wv.y, fmaxf(__uint_as_float(v[4 * j4 + 1]), 0.0f), a[(4 * j4 + 1) & 7]);
-        a[(4 * j4 + 2) & 7] = fmaf(wv.z, fmaxf(__uint_as_float(v[4 * j4 + 2]), 0.0f), a[(4 * j4 + 2) & 7]);
-        a[(4 * j4 + 3) & 7] = fmaf(wv.w, fmaxf(__uint_as_float(v[4 * j4 + 3]), 0.0f), a[(4 * j4 + 3) & 7]);
-    }
-    return ((a[0] + a[1]) + (a[2] + a[3])) + ((a[4] + a[5]) + (a[6] + a[7]));
+// Packed (2 x fp32) fused multiply-add: acc.{x,y} = w.{x,y} * r.{x,y} + acc.{x,y},
+// each lane of the pair rounded separately (the sm_100 fma.rn.f32x2).
+__device__ __forceinline__ unsigned long long ffma2(unsigned long long acc, float w0, float w1, float r0, float r1) {
+    unsigned long long wp, rp;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(wp) : "f"(w0), "f"(w1));
+    asm("mov.b64 %0, {%1, %2};" : "=l"(rp) : "f"(r0), "f"(r1));
+    asm("fma.rn.f32x2 %0, %1, %2, %0;" : "+l"(acc) : "l"(wp), "l"(rp));
+    return acc;
 }
 
-// sum_j w[j] * max(v[j], 0) over 64 heads; w 16-byte aligned, read as float4
-__device__ __forceinline__ float reduce64(const uint32_t (&v0)[32], const uint32_t (&v1)[32], const float *w) {
-    const float4 *w4 = reinterpret_cast<const float4 *>(w);
-    float a[8];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) a[i] = 0.0f;
+// v + |v| = 2 max(v, 0), exactly for every finite v below FLT_MAX / 2; an
+// fp32 add on the FMA pipe instead of a max on the half-rate ALU pipe.
+__device__ __forceinline__ float twice_relu(uint32_t x) {
+    const float f = __uint_as_float(x);
+    return f + fabsf(f);
+}
+
+// sum_j w[j] * max(v[j], 0) over 32 heads, given w2 = w / 2 (read as float4,
+// 16-byte aligned): each term is w2[j] * (v[j] + |v[j]|), the same fp32
+// product.  8 independent partial sums kept as 4 packed pairs, so each two
+// heads cost two adds and one packed fma.
+__device__ __forceinline__ float reduce32(const uint32_t (&v)[32], const float *w2) {
+    const float4 *w4 = reinterpret_cast<const float4 *>(w2);
+    unsigned long long a[4] = {0ull, 0ull, 0ull, 0ull};
 #pragma unroll
     for (int j4 = 0; j4 < 8; ++j4) {
         const float4 wv = w4[j4];
-        a[(4 * j4 + 0) & 7] = fmaf(wv.x, fmaxf(__uint_as_float(v0[4 * j4 + 0]), 0.0f), a[(4 * j4 + 0) & 7]);
-        a[(4 * j4 + 1) & 7] = fmaf(wv.y, fmaxf(__uint_as_float(v0[4 * j4 + 1]), 0.0f), a[(4 * j4 + 1) & 7]);
-        a[(4 * j4 + 2) & 7] = fmaf(wv.z, fmaxf(__uint_as_float(v0[4 * j4 + 2]), 0.0f), a[(4 * j4 + 2) & 7]);
-        a[(4 * j4 + 3) & 7] = fmaf(wv.w, fmaxf(__uint_as_float(v0[4 * j4 + 3]), 0.0f), a[(4 * j4 + 3) & 7]);
+        a[(2 * j4) & 3] = ffma2(a[(2 * j4) & 3], wv.x, wv.y, twice_relu(v[4 * j4 + 0]), twice_relu(v[4 * j4 + 1]));
+        a[(2 * j4 + 1) & 3] =
+            ffma2(a[(2 * j4 + 1) & 3], wv.z, wv.w, twice_relu(v[4 * j4 + 2]), twice_relu(v[4 * j4 + 3]));
     }
+    float s[8];
 #pragma unroll
-    for (int j4 = 0; j4 < 8; ++j4) {
-        const float4 wv = w4[8 + j4];
-        a[(4 * j4 + 0) & 7] = fmaf(wv.x, fmaxf(__uint_as_float(v1[4 * j4 + 0]), 0.0f), a[(4 * j4 + 0) & 7]);
-        a[(4 * j4 + 1) & 7] = fmaf(wv.y, fmaxf(__uint_as_float(v1[4 * j4 + 1]), 0.0f), a[(4 * j4 + 1) & 7]);
-        a[(4 * j4 + 2) & 7] = fmaf(wv.z, fmaxf(__uint_as_float(v1[4 * j4 + 2]), 0.0f), a[(4 * j4 + 2) & 7]);
-        a[(4 * j4 + 3) & 7] = fmaf(wv.w, fmaxf(__uint_as_float(v1[4 * j4 + 3]), 0.0f), a[(4 * j4 + 3) & 7]);
-    }
-    return ((a[0] + a[1]) + (a[2] + a[3])) + ((a[4] + a[5]) + (a[6] + a[7]));
+    for (int i = 0; i < 4; ++i) asm("mov.b64 {%0, %1}, %2;" : "=f"(s[2 * i]), "=f"(s[2 * i + 1]) : "l"(a[i]));
+    return ((s[0] + s[1]) + (s[2] + s[3])) + ((s[4] + s[5]) + (s[6] + s[7]));
 }
 
 template <bool GATHER>
@@ -215,8 +210,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         const Item it = item_info<GATHER>(g, dd, item);
         if (!it.valid) continue;
         __syncthreads();
+        // the halved head weights (exact) of the item's rows, for reduce32
         for (int i = threadIdx.x; i < 4 * S_H; i += kThreads)
-            wsm[i] = (i / S_H) < it.m ? wsrc[it.qrow0 * S_H + i] : 0.0f;
+            wsm[i] = (i / S_H) < it.m ? 0.5f * wsrc[it.qrow0 * S_H + i] : 0.0f;
         __syncthreads();
         const uint32_t idesc = tc::idesc_bf16_f32(128, 64 * it.m);
 
