@@ -224,6 +224,10 @@ cudaError_t launch_decode_tc(const DecodeArgs &a, cudaStream_t st);
 cudaError_t launch_gather_simt(const GatherArgs &a, int dtype, cudaStream_t st);
 cudaError_t launch_gather_tc(const GatherArgs &a, cudaStream_t st);
 cudaError_t launch_select(const SelectArgs &a, cudaStream_t st);
+// dec_select.cu: the decode score rows (SEL_DEC_DENSE, _REUSE, _PROXY_TO_C),
+// one cluster of CTAs per row
+bool dec_select_kind(int kind);
+cudaError_t launch_dec_select(const SelectArgs &a, cudaStream_t st);
 cudaError_t launch_adaptive(const AdaptiveArgs &a, cudaStream_t st);
 cudaError_t launch_proxy(const void *q, const float *w, const int *cu, int S, int T, int H, int d,
                          int g, int db, int dtype, const int *plan, const PlanLayout &pl, void *qbar,

@@ -4,9 +4,11 @@
 // are ranked by key = (ord(score) << 32) | (0xFFFFFFFF - s), so the top-k is
 // "highest score first, ties to the lower position".
 //
-// Two kernels:
-//  - select_kernel: decode score rows (a full fp32 score row per query or
-//    proxy over its whole cache, up to 2^20 entries, few rows), below;
+// Two kernels here (the decode score rows, a full fp32 row per query or
+// proxy over its whole cache, take a cluster of CTAs per row: dec_select.cu):
+//  - select_kernel: the block-score rows of the block pre-filter (a proxy's
+//    scores over the complete blocks of its prefix, prefill Quest rule and
+//    decode), below;
 //  - select_fast_kernel: candidate buffers with a floor (dense, Reuse,
 //    proxy -> C, proxy -> blocks) and Refine member rows over a candidate
 //    set, further down.
@@ -380,32 +382,6 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(SelectArgs a) {
         }
     };
     switch (a.kind) {
-    case SEL_DEC_DENSE:
-    case SEL_DEC_REUSE:
-    case SEL_DEC_PROXY_TO_C: {
-        const bool per_member = a.kind != SEL_DEC_PROXY_TO_C;
-        const int b = per_member ? row / a.G : row;
-        const int m = per_member ? row % a.G : 0;
-        const int kv = a.kv_len[b];
-        if (kv < a.G || kv > a.n_max) {
-            if (threadIdx.x == 0) raise_status(a.status, ST_INVALID);
-            pad_all();
-            return;
-        }
-        if (a.kind == SEL_DEC_DENSE) {
-            const int bound = kv - a.G + m;
-            ScoreSrc src{a.scores + (long long)row * a.ld, nullptr, bound + 1, bound};
-            block_select(src, a.k, oi, os, sh, stage, a.stage_cap, bm, gpre, wcap, a.status);
-        } else if (a.kind == SEL_DEC_REUSE) {
-            const int bound = kv - a.G + m;
-            ScoreSrc src{a.scores + (long long)b * a.ld, nullptr, bound + 1, bound};
-            block_select(src, a.k, oi, os, sh, stage, a.stage_cap, bm, gpre, wcap, a.status);
-        } else {  // SEL_DEC_PROXY_TO_C
-            ScoreSrc src{a.scores + (long long)b * a.ld, nullptr, kv, kv - 1};
-            block_select(src, a.k, oi, nullptr, sh, stage, a.stage_cap, bm, gpre, wcap, a.status);
-        }
-        return;
-    }
     case SEL_PROXY_SPILL_TO_BLOCKS: {
         // prefill block mode (Quest rule): proxy row p's top blocks among the
         // complete blocks of its prefix (t_last + 1) / 64, k = c / 64 slots,
@@ -486,7 +462,8 @@ constexpr int kChunkWords = kChunkBits / 32;      // 4096 words = 16 KB
 struct __align__(16) FastShared {
     unsigned hist[2][256];
     unsigned wtot[kFWarps];
-    unsigned blkpre[kFT];  // emit: chunk-local rank of each lane block's first bit
+    unsigned blkpre[kFT];           // emit: chunk-local rank of each lane block's first bit
+    unsigned short blkmid[kFT];     // emit: rank of its ninth word's first bit within the block
     unsigned nstage;
     unsigned maxord;
     unsigned minord;
@@ -608,8 +585,10 @@ __device__ unsigned long long fast_kth(const Src &src, FastShared &sh, unsigned 
     return fast_kth_run(src, sh, need, prefix, mask, 64 - lead, 0);
 }
 
-// Keys staged in shared memory, read relative to a floor ord: key - floor << 32
-// (all staged keys have ord >= floor; the result is never 0).
+// Keys staged in shared memory, read relative to a base ord: key - base << 32.
+// A key whose ord is at or above the base gives a nonzero result; a key below
+// it (or an empty slot) wraps around to a value whose top bits are set, which
+// matches none of the prefixes the callers search.
 struct SStageOff {
     const unsigned long long *st;
     int n;
@@ -659,21 +638,34 @@ __device__ __forceinline__ int emit_word(int L, int per) {
 }
 
 // List the nonzero keys >= K of src in ascending position through a bitmap
-// (chunks of kChunkBits positions over 0..bound); returns how many.
+// (chunks of kChunkBits positions over 0..bound); returns how many.  Each
+// chunk: the selected keys set their bits; each lane block's count is ranked
+// by a warp scan and a block scan; then every selected key is placed at its
+// rank = its lane block's first rank + the bits before it in the block.  The
+// bits before it in its word come from one popcount, those of the block's
+// earlier words from a per-word table (8 bits a word: the rank of the word's
+// first bit within its run of 8 words; the second run's offset is kept per
+// block) in `buf` when it has room, else from popcounts of those words.  The
+// lists are built in `buf` after the table and copied out with coalesced
+// stores; without room they are written directly.
 template <class Src>
 __device__ int fast_emit_bitmap(const Src &src, unsigned long long K, int bound, int k, int *out_idx,
                                 float *out_score, FastShared &sh, unsigned *bm, unsigned *buf, int buf_words,
                                 bool bm_clear = false) {
-    const int tid = threadIdx.x;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    // the first chunk is the widest: its table size serves every chunk
+    const int tw0 = kFT * emit_per(bound / 32 + 1 < kChunkWords ? bound / 32 + 1 : kChunkWords);
+    const bool tab = buf_words >= tw0 / 4;
+    unsigned char *rk = reinterpret_cast<unsigned char *>(buf);
+    unsigned *lst = buf + (tab ? tw0 / 4 : 0);
+    const int lw = buf_words - (tab ? tw0 / 4 : 0);
+    const bool via_smem = lw >= (out_score ? 2 * k : k);
+    int *pi = via_smem ? reinterpret_cast<int *>(lst) : out_idx;
+    float *ps = via_smem ? reinterpret_cast<float *>(lst + k) : out_score;
     int base = 0;
-    // the list is built in shared memory (buf: free stage room) and copied
-    // out with coalesced stores; without room it is written directly
-    const bool via_smem = buf_words >= (out_score ? 2 * k : k);
-    int *pi = via_smem ? reinterpret_cast<int *>(buf) : out_idx;
-    float *ps = via_smem ? reinterpret_cast<float *>(buf + k) : out_score;
     for (int c0 = 0; c0 <= bound; c0 += kChunkBits) {
         const int nwords = (bound - c0) / 32 + 1 < kChunkWords ? (bound - c0) / 32 + 1 : kChunkWords;
-        const int per = emit_per(nwords);
+        const int per = emit_per(nwords), lg = 31 - __clz(per);
         if (!(bm_clear && c0 == 0)) {  // the caller may have cleared it for the first chunk
             for (int j = tid; j < kFT * per; j += kFT) bm[j] = 0u;
             __syncthreads();
@@ -687,11 +679,21 @@ __device__ int fast_emit_bitmap(const Src &src, unsigned long long K, int bound,
         }
         __syncthreads();
         // lane `lane` of warp `warp` owns logical words wb + lane * per .. + per - 1,
-        // stored at wb + 32 j + lane
-        const int lane = tid & 31, warp = tid >> 5;
+        // stored at wb + 32 j + lane; the table entry of a word sits at its
+        // storage index
         const int wb = warp * 32 * per;
-        unsigned cnt = 0;
-        for (int j = 0; j < per; ++j) cnt += __popc(bm[wb + 32 * j + lane]);
+        unsigned cnt = 0, run = 0;
+        for (int j = 0; j < per; ++j) {
+            const int w = wb + 32 * j + lane;
+            if (j == 8) {  // per <= kChunkWords / kFT = 16: at most two runs
+                sh.blkmid[tid] = (unsigned short)cnt;
+                run = 0;
+            }
+            if (tab) rk[w] = (unsigned char)run;  // at most 7 * 32 = 224
+            const unsigned c = __popc(bm[w]);
+            cnt += c;
+            run += c;
+        }
         unsigned inc = cnt;  // inclusive warp prefix of the lanes' counts
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
@@ -707,40 +709,31 @@ __device__ int fast_emit_bitmap(const Src &src, unsigned long long K, int bound,
             before += w < warp ? t : 0u;
             total += t;
         }
-        unsigned at = base + before + inc - cnt;
-        sh.blkpre[tid] = at - base;
-        const int pos0 = c0 + (wb + lane * per) * 32;  // first position of the lane's block
-        for (int j = 0; j < per; ++j) {
-            const int w = wb + 32 * j + lane;
-            unsigned x = bm[w];
-            while (x) {
-                const int bit = __ffs(x) - 1;
-                x &= x - 1u;
-                if (at < (unsigned)k) pi[at] = pos0 + 32 * j + bit;  // never past the row
-                ++at;
-            }
-        }
-        if (out_score) {
-            __syncthreads();  // every block's rank is recorded; the bitmap is intact
-            const int lg = 31 - __clz(per);
-            for (int i = tid; i < src.n; i += kFT) {
-                const unsigned long long kk = src.key(i);
-                if (kk != 0ull && kk >= K) {
-                    const int p = key_pos(kk) - c0;
-                    if (p >= 0 && p < kChunkBits) {
-                        // rank = the block's first rank + the bits before p in its block:
-                        // the block's earlier words sit 32, 64, .. words below
-                        const int L = p >> 5, w = emit_word(L, per);
-                        unsigned rk = sh.blkpre[L >> lg] + __popc(bm[w] & ((1u << (p & 31)) - 1u));
-                        for (int t = 1; t <= (L & (per - 1)); ++t) rk += __popc(bm[w - 32 * t]);
-                        if (base + (int)rk < k) ps[base + rk] = ord_score(key_ord(kk));
+        sh.blkpre[tid] = before + inc - cnt;  // chunk-local rank of the lane block's first bit
+        __syncthreads();
+        for (int i = tid; i < src.n; i += kFT) {
+            const unsigned long long kk = src.key(i);
+            if (kk != 0ull && kk >= K) {
+                const int p = key_pos(kk) - c0;
+                if (p >= 0 && p < kChunkBits) {
+                    const int L = p >> 5, w = emit_word(L, per), j = L & (per - 1);
+                    unsigned r = sh.blkpre[L >> lg] + __popc(bm[w] & ((1u << (p & 31)) - 1u));
+                    if (tab) {
+                        r += rk[w] + (j >= 8 ? sh.blkmid[L >> lg] : 0u);
+                    } else {  // the block's earlier words sit 32, 64, .. words below
+                        for (int t = 1; t <= j; ++t) r += __popc(bm[w - 32 * t]);
+                    }
+                    const int at = base + (int)r;
+                    if (at < k) {  // never past the row
+                        pi[at] = c0 + p;
+                        if (out_score) ps[at] = ord_score(key_ord(kk));
                     }
                 }
             }
         }
         base += (int)total;
         if (base > k) base = k;
-        __syncthreads();  // the bitmap is cleared again by the next chunk
+        __syncthreads();  // the bitmap and the table are rewritten by the next chunk
     }
     if (via_smem) {
         fast_copy_out(pi, out_idx, base);
@@ -907,33 +900,23 @@ __device__ void fast_margin(const Src &src, unsigned long long K, int nsel, unsi
     }
 }
 
-// Top-k of a candidate row (keys at or above `floor_ord`, positions <= bound),
-// and its cutoff margin when m.km > 0.
-__device__ void fast_cand_row(const unsigned long long *buf, int n, unsigned floor_ord, int bound, int k,
-                              int *out_idx, float *out_score, FastShared &sh, unsigned long long *stage,
-                              int stage_cap, unsigned *bm, const MarginOut &m) {
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const GCand g{buf, n, (unsigned long long)floor_ord << 32, 0xFFFFFFFFu - (unsigned)bound};
-    if (tid == 0) {
-        sh.nstage = 0u;
-        sh.maxord = 0u;
-    }
-    sh.hist[0][tid] = 0u;
-    sh.hist[1][tid] = 0u;
-    __syncthreads();
-    // the emit's bitmap (first chunk, the words the walk reads), cleared here
-    // (ordered before it by the barrier below)
-    {
-        const int nw = bound / 32 + 1 < kChunkWords ? bound / 32 + 1 : kChunkWords;
-        const int nclr = kFT * emit_per(nw);
-        for (int j = tid; j < nclr; j += kFT) bm[j] = 0u;
-    }
+// Staging pass of a candidate row: every key with ord >= max(floor_ord, 1)
+// (ord 0 is the empty key; no arithmetic result has it) goes to the stage,
+// and the first radix digit of each is counted in sh.hist[0].  kPos: the
+// buffer may hold positions past the bound (a Reuse member reading its
+// proxy's buffer), which are dropped too; without it every buffered position
+// is within the bound (the score pass appends only keys the row may see).
+// Returns this thread's largest staged ord (0: none).
+template <bool kPos>
+__device__ unsigned stage_cand(const GCand &g, unsigned floor_ord, FastShared &sh, unsigned long long *stage,
+                               int stage_cap) {
+    const int tid = threadIdx.x, lane = tid & 31, n = g.n;
+    const unsigned f1 = floor_ord > 0u ? floor_ord : 1u;
     unsigned mx = 0u;
-    const unsigned long long lo1 = g.lo > 1ull ? g.lo : 1ull;
     // 8 keys per thread and round, as four 16-byte loads (rows start 2 KB
     // aligned); the next round's loads are issued before this round's keys
     // are filtered, so their latency overlaps the work
-    const ulonglong2 *b2 = reinterpret_cast<const ulonglong2 *>(buf);
+    const ulonglong2 *b2 = reinterpret_cast<const ulonglong2 *>(g.buf);
     ulonglong2 nx[4];
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
@@ -953,15 +936,20 @@ __device__ void fast_cand_row(const unsigned long long *buf, int n, unsigned flo
             const int i = base + kFT * 8 + u * (kFT * 2) + tid * 2;
             if (i < n) nx[u] = b2[i >> 1];
         }
-        unsigned cnt = 0;
+        unsigned okm = 0u;
 #pragma unroll
         for (int u = 0; u < 8; ++u) {
-            // lo1 >= 1 also drops the empty key 0; a dropped key becomes 0 (ord 0)
-            const bool ok = kv[u] >= lo1 && (unsigned)kv[u] >= g.pmin;
-            if (!ok) kv[u] = 0ull;
-            cnt += ok ? 1u : 0u;
-            mx = max(mx, key_ord(kv[u]));
+            const unsigned o = key_ord(kv[u]);
+            bool ok = o >= f1;
+            if (kPos) {
+                ok = ok && (unsigned)kv[u] >= g.pmin;
+                mx = max(mx, ok ? o : 0u);
+            } else {
+                mx = max(mx, o);
+            }
+            okm |= ok ? 1u << u : 0u;
         }
+        const unsigned cnt = __popc(okm);
         unsigned inc = cnt;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
@@ -975,7 +963,7 @@ __device__ void fast_cand_row(const unsigned long long *buf, int n, unsigned flo
             b = __shfl_sync(0xFFFFFFFFu, b, 31) + inc - cnt;
 #pragma unroll
             for (int u = 0; u < 8; ++u) {
-                if (kv[u] != 0ull) {
+                if (okm & (1u << u)) {
                     if (b < (unsigned)stage_cap) stage[b] = kv[u];
                     ++b;
                     // the radix's first digit, counted here
@@ -984,6 +972,34 @@ __device__ void fast_cand_row(const unsigned long long *buf, int n, unsigned flo
             }
         }
     }
+    // without kPos the largest ord is staged exactly when it reaches f1
+    if (!kPos && mx < f1) mx = 0u;
+    return mx;
+}
+
+// Top-k of a candidate row (keys at or above `floor_ord`, positions <= bound),
+// and its cutoff margin when m.km > 0.
+__device__ void fast_cand_row(const unsigned long long *buf, int n, unsigned floor_ord, int bound, int k,
+                              int *out_idx, float *out_score, FastShared &sh, unsigned long long *stage,
+                              int stage_cap, unsigned *bm, const MarginOut &m, bool pos_check) {
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const GCand g{buf, n, (unsigned long long)floor_ord << 32, 0xFFFFFFFFu - (unsigned)bound};
+    if (tid == 0) {
+        sh.nstage = 0u;
+        sh.maxord = 0u;
+    }
+    sh.hist[0][tid] = 0u;
+    sh.hist[1][tid] = 0u;
+    __syncthreads();
+    // the emit's bitmap (first chunk, the words the walk reads), cleared here
+    // (ordered before it by the barrier below)
+    {
+        const int nw = bound / 32 + 1 < kChunkWords ? bound / 32 + 1 : kChunkWords;
+        const int nclr = kFT * emit_per(nw);
+        for (int j = tid; j < nclr; j += kFT) bm[j] = 0u;
+    }
+    unsigned mx = pos_check ? stage_cand<true>(g, floor_ord, sh, stage, stage_cap)
+                            : stage_cand<false>(g, floor_ord, sh, stage, stage_cap);
     mx = warp_max_u(mx);
     if (lane == 0 && mx) atomicMax(&sh.maxord, mx);
     __syncthreads();
@@ -1062,27 +1078,77 @@ __device__ void fast_member_row(const float *sc, const int *pos, int n, int boun
     __syncthreads();
     unsigned mx = 0u, mn = 0xFFFFFFFFu, cnt = 0;
     const bool staged = n <= stage_cap;
-    // 8 entries per thread and round, every load issued before any is used
-    for (int base = 0; base < n; base += kFT * 8) {
-        int pv[8];
-        float sv[8];
+    const bool vec = staged && pos != nullptr &&
+                     ((reinterpret_cast<uintptr_t>(sc) | reinterpret_cast<uintptr_t>(pos)) & 15u) == 0;
+    // 8 entries per thread and round, every load issued before any is used:
+    // with 16-byte aligned rows as two runs of 4 (16-byte loads and stores),
+    // else one entry at a time
+    if (vec) {
+        for (int base = 0; base < n; base += kFT * 8) {
+            float4 sv[2];
+            int4 pv[2];
 #pragma unroll
-        for (int u = 0; u < 8; ++u) {
-            const int i = base + u * kFT + tid;
-            pv[u] = i < n ? (pos ? pos[i] : i) : -1;
-            sv[u] = i < n ? sc[i] : 0.0f;
+            for (int u = 0; u < 2; ++u) {
+                const int i = base + (u * kFT + tid) * 4;
+                if (i + 3 < n) {
+                    sv[u] = *reinterpret_cast<const float4 *>(sc + i);
+                    pv[u] = *reinterpret_cast<const int4 *>(pos + i);
+                } else {
+                    sv[u] = make_float4(i < n ? sc[i] : 0.0f, i + 1 < n ? sc[i + 1] : 0.0f,
+                                        i + 2 < n ? sc[i + 2] : 0.0f, 0.0f);
+                    pv[u] = make_int4(i < n ? pos[i] : -1, i + 1 < n ? pos[i + 1] : -1, i + 2 < n ? pos[i + 2] : -1,
+                                      -1);
+                }
+            }
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+                const int i = base + (u * kFT + tid) * 4;
+                const float s4[4] = {sv[u].x, sv[u].y, sv[u].z, sv[u].w};
+                const int p4[4] = {pv[u].x, pv[u].y, pv[u].z, pv[u].w};
+                unsigned long long kk[4];
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    kk[j] = (p4[j] >= 0 && p4[j] <= bound) ? make_key(score_ord(s4[j]), p4[j]) : 0ull;
+                    if (kk[j] != 0ull) {
+                        const unsigned o = key_ord(kk[j]);
+                        mx = o > mx ? o : mx;
+                        mn = o < mn ? o : mn;
+                        ++cnt;
+                    }
+                }
+                if (i + 3 < n) {
+                    ulonglong2 *d2 = reinterpret_cast<ulonglong2 *>(stage + i);
+                    d2[0] = make_ulonglong2(kk[0], kk[1]);
+                    d2[1] = make_ulonglong2(kk[2], kk[3]);
+                } else {
+#pragma unroll
+                    for (int j = 0; j < 4; ++j)
+                        if (i + j < n) stage[i + j] = kk[j];
+                }
+            }
         }
+    } else {
+        for (int base = 0; base < n; base += kFT * 8) {
+            int pv[8];
+            float sv[8];
 #pragma unroll
-        for (int u = 0; u < 8; ++u) {
-            const int i = base + u * kFT + tid;
-            const unsigned long long kk =
-                (pv[u] >= 0 && pv[u] <= bound) ? make_key(score_ord(sv[u]), pv[u]) : 0ull;
-            if (staged && i < n) stage[i] = kk;
-            if (kk != 0ull) {
-                const unsigned o = key_ord(kk);
-                mx = o > mx ? o : mx;
-                mn = o < mn ? o : mn;
-                ++cnt;
+            for (int u = 0; u < 8; ++u) {
+                const int i = base + u * kFT + tid;
+                pv[u] = i < n ? (pos ? pos[i] : i) : -1;
+                sv[u] = i < n ? sc[i] : 0.0f;
+            }
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const int i = base + u * kFT + tid;
+                const unsigned long long kk =
+                    (pv[u] >= 0 && pv[u] <= bound) ? make_key(score_ord(sv[u]), pv[u]) : 0ull;
+                if (staged && i < n) stage[i] = kk;
+                if (kk != 0ull) {
+                    const unsigned o = key_ord(kk);
+                    mx = o > mx ? o : mx;
+                    mn = o < mn ? o : mn;
+                    ++cnt;
+                }
             }
         }
     }
@@ -1128,11 +1194,12 @@ __global__ void __launch_bounds__(kFT, 4) select_fast_kernel(SelectArgs a) {
     const MarginOut mo = a.kind == SEL_DENSE_CAND && a.kmargin > 0
                              ? MarginOut{a.kmargin, a.m_sigma + row, a.m_vk + row, a.m_need + row}
                              : MarginOut{0, nullptr, nullptr, nullptr};
-    auto cand = [&](long long r, int bound, int k, const MarginOut &m) {
+    // own: the buffer is the output row's own (scored with the same bound)
+    auto cand = [&](long long r, int bound, int k, const MarginOut &m, bool own) {
         const long long sr = r - p0;
         const unsigned n = a.cnt[sr];
         fast_cand_row(a.buf + sr * a.cap, (int)(n < a.cap ? n : a.cap), a.floor ? a.floor[sr] : 0u, bound, k, oi, os,
-                      sh, stage, scap, bm, m);
+                      sh, stage, scap, bm, m, !own);
     };
     const MarginOut none{0, nullptr, nullptr, nullptr};
     switch (a.kind) {
@@ -1152,14 +1219,14 @@ __global__ void __launch_bounds__(kFT, 4) select_fast_kernel(SelectArgs a) {
         const int b = find_seg(a.cu, a.S, row);
         const int t = row - a.cu[b];
         if (a.kind == SEL_DENSE_CAND) {
-            cand(row, t, a.k, mo);
+            cand(row, t, a.k, mo, true);
         } else {
             const int n = a.cu[b + 1] - a.cu[b];
             const int p = a.plan[a.pl.rp() + b] + group_of(t, n, a.g, a.db);
             // Reuse, and members scored on their own (guardrail): the top-k of
             // the scored row's candidates inside the member's prefix
             if (a.kind == SEL_REUSE_CAND || t < dense_rows(n, a.g, a.db))
-                cand(p, t, a.k, none);
+                cand(p, t, a.k, none, false);
             else
                 fast_member_row(a.scores + ((long long)row - a.plan[8]) * a.ld, a.cand + (p - p0) * a.c, a.c, t,
                                 a.k, oi, os, sh, stage, scap, bm);
@@ -1181,7 +1248,7 @@ __global__ void __launch_bounds__(kFT, 4) select_fast_kernel(SelectArgs a) {
             if (i < dense_rows(n, a.g, a.db)) return;
             oi = po;
             os = nullptr;
-            cand(row, row_bound(i, n, a.g, a.db), a.k, none);
+            cand(row, row_bound(i, n, a.g, a.db), a.k, none, true);
             return;
         }
         const int tl = row_bound(i, n, a.g);
@@ -1190,7 +1257,7 @@ __global__ void __launch_bounds__(kFT, 4) select_fast_kernel(SelectArgs a) {
         if (kr > 0) {
             oi = po;
             os = nullptr;
-            cand(row, key_bound(tl, kBlockShift), kr, none);
+            cand(row, key_bound(tl, kBlockShift), kr, none, false);
         }
         for (int r = (kr > 0 ? kr : 0) + (int)threadIdx.x; r < a.k; r += kFT) po[r] = -1;
         return;
@@ -1247,6 +1314,7 @@ cudaError_t launch_select_fast(const SelectArgs &a, cudaStream_t st) {
 cudaError_t launch_select(const SelectArgs &a, cudaStream_t st) {
     if (a.nrows <= 0) return cudaSuccess;
     if (fast_kind(a.kind)) return launch_select_fast(a, st);
+    if (dec_select_kind(a.kind)) return launch_dec_select(a, st);
     SelectArgs b = a;
     const size_t tail = ((size_t)a.bitmap_words * 2 + 32) * 4;  // bitmap + per-word prefix + warp totals
     const size_t limit = 232448 - sizeof(SelShared) - 1024;
