@@ -196,6 +196,30 @@ def test_decode_modes(idx):
                         assert np.array_equal(reselect(mm[keep], topk, Cv[keep]), got[b, m])
 
 
+def test_decode_exact_integer_inputs(idx):
+    """Integer q and cache in [-2, 2] (exact in bf16) and dyadic w: every decode
+    score is an exact fp32 integer, ties are frequent, and the selected indices
+    must equal the oracle's bit for bit.  n_max = 5000 and the ragged kv_len
+    leave segments of the decode select that end inside a 32-position run; the
+    tensor-core scan (H = 64, d = 128) and the CUDA-core scan (H = 4, d = 16)."""
+    for H, d in ((64, 128), (4, 16)):
+        B, G, n_max, topk, c = 3, 2, 5000, 512, 1024
+        rng = np.random.default_rng(11)
+        q = W.bf16_bits(rng.integers(-2, 3, size=(B, G, H, d)).astype(np.float32))
+        kc = W.bf16_bits(rng.integers(-2, 3, size=(B, n_max, d)).astype(np.float32))
+        w = rng.choice(np.array([0.0, 0.25, 0.5, 1.0], np.float32), size=(B, G, H)).astype(np.float32)
+        kv_len = np.array([5000, 4097, 1500], np.int32)
+        qd, kd, wd, kvd = to_dev(q), to_dev(kc), to_dev(w), to_dev(kv_len)
+        for mode, om in (("dense", O.DENSE), ("reuse", O.REUSE), ("refine", O.REFINE)):
+            ws = torch.empty(idx.decode_workspace_size(B, G, n_max, H, d, topk, c, mode, qd.dtype),
+                             dtype=torch.uint8, device="cuda")
+            out = idx.decode_topk(qd, kd, kvd, wd, topk, c, mode, workspace=ws)
+            assert idx.device_status(ws) == "IDX_OK"
+            got = out.cpu().numpy().reshape(B * G, topk)
+            want = O.decode_topk(q, kc, w, kv_len, topk, c, om).reshape(B * G, topk)
+            assert np.array_equal(got, want), (H, d, mode)
+
+
 def test_edges_short_prefixes_and_empty_request(idx):
     # topk larger than every prefix; an empty request in the middle; T = 1 case
     P = W.prefill([300, 0, 150], H=64, d=128, topk=512, rho=0.9, planted=0.0, seed=9)
