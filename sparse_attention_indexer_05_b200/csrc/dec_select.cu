@@ -272,9 +272,10 @@ __global__ void __cluster_dims__(kDC, 1, 1) __launch_bounds__(kDT, 2) dec_select
         }
         const unsigned long long base = (unsigned long long)LO << 32;
         const unsigned span = HI - LO;
-        // `shift` is the bit below the digits placed so far.  The first digit,
-        // bits [shift - 11, shift) of x, covers ord - LO exactly: it is
-        // (ord - LO) >> sh1, 32-bit arithmetic on the ord alone
+        // `shift` is the lowest bit of the current digit.  The first digit,
+        // bits [32 + sh1, 43 + sh1) of x, covers ord - LO exactly: it is
+        // (ord - LO) >> sh1, 32-bit arithmetic on the ord alone; each later
+        // round takes the next (up to) 11 bits below it
         const int sh1 = span >= (unsigned)kDBins ? 32 - kDBits - __clz(span) : 0;
         int shift = 32 + sh1;
         unsigned long long prefix = 0ull, mask = 0ull;

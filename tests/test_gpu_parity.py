@@ -196,6 +196,30 @@ def test_decode_modes(idx):
                         assert np.array_equal(reselect(mm[keep], topk, Cv[keep]), got[b, m])
 
 
+def test_decode_rows_longer_than_the_select_cache(idx):
+    """n_max = 140000: each of the 8 CTAs of a row's cluster holds 17504
+    positions, more than it keeps in shared memory, so the decode select reads
+    its segment from global memory on every pass.  Dense and Reuse indices
+    equal the oracle's rule re-applied to the GPU's own scores."""
+    topk, c, n_max = 2048, 4096, 140000
+    D = W.decode(B=2, n=n_max, G=2, H=64, d=128, topk=topk, c=c, seed=5, kv_len=[140000, 70001], n_max=n_max)
+    q, kc, w, kv = to_dev(D.q), to_dev(D.kcache), to_dev(D.w), to_dev(D.kv_len)
+    for mode in ("dense", "reuse"):
+        ws = torch.empty(max(idx.decode_workspace_size(2, 2, n_max, 64, 128, topk, c, m, q.dtype)
+                             for m in ("dense", mode)), dtype=torch.uint8, device="cuda")
+        got = idx.decode_topk(q, kc, kv, w, topk, c, mode, workspace=ws).cpu().numpy()
+        assert idx.device_status(ws) == "IDX_OK"
+        bounds = [int(n) - 2 + m for n in D.kv_len for m in range(2)]
+        check_rows_wellformed(got, bounds, topk)
+        stage = 0 if mode == "dense" else 1
+        sc = idx.debug_decode_scores(stage, q, kc, kv, w, topk, c, mode, workspace=ws).cpu().numpy()
+        for b in range(2):
+            for m in range(2):
+                t = int(D.kv_len[b]) - 2 + m
+                row = sc[b * 2 + m, :t + 1] if mode == "dense" else sc[b, :t + 1]
+                assert np.array_equal(reselect(row, topk), got[b, m]), (mode, b, m)
+
+
 def test_decode_exact_integer_inputs(idx):
     """Integer q and cache in [-2, 2] (exact in bf16) and dyadic w: every decode
     score is an exact fp32 integer, ties are frequent, and the selected indices
