@@ -14,9 +14,12 @@
 //      holds more than kList keys (after one round it holds a few dozen: the
 //      digits spread the row's range over 2048 bins);
 //   3. the CTAs copy the bin's keys from every segment into one short list and
-//      each finishes the radix on it (8-bit digits), all reaching the same K;
-//   4. each CTA counts its keys >= K; a prefix over the cluster's counts gives
-//      its offset, and it writes its selected positions in ascending order.
+//      each finishes the radix on it (8-bit digits), all reaching the same K.
+//      The pass that collects a segment's keys of the bin also counts, per
+//      warp, the keys above the bin; with the bin's keys >= K (from the list)
+//      that gives each warp's count of selected keys without another pass;
+//   4. a prefix over the cluster's counts gives each CTA its offset, and it
+//      writes its selected positions in ascending order.
 // Cluster barriers separate the steps.  Every decision between them comes
 // from values all CTAs of a cluster share (the row's bound and k, the summed
 // histogram), so all CTAs take the same barriers; the last barrier keeps each
@@ -249,6 +252,10 @@ __global__ void __cluster_dims__(kDC, 1, 1) __launch_bounds__(kDT, 2) dec_select
             }
         }
     }
+    // warp w's part of the segment in steps 3 and 4: [wj0, wj1)
+    const int wseg = ((len + kDWarps - 1) / kDWarps + 31) & ~31;
+    const int wj0 = warp * wseg, wj1 = wj0 + wseg < len ? wj0 + wseg : len;
+    bool counted = false;  // sh.wtot holds each warp's count of keys >= K
     unsigned long long K = 1ull;  // n <= k: every position
     if (r.n > r.k) {
         mn = __reduce_min_sync(0xFFFFFFFFu, mn);
@@ -319,17 +326,28 @@ __global__ void __cluster_dims__(kDC, 1, 1) __launch_bounds__(kDT, 2) dec_select
             one_round = false;
         }
         if (!done) {
-            // 3. the bin's keys from every segment, resolved in each CTA
+            // 3. the bin's keys from every segment, resolved in each CTA; the
+            // same pass counts each warp's keys above the bin, all selected
             if (tid == 0) sh.nlist = 0u;
             __syncthreads();
             const unsigned b1 = (unsigned)(prefix >> shift);  // the first digit, when it is the only one
-            for (int j0 = warp * 32; j0 < len; j0 += kDT) {
+            unsigned above_cnt = 0;
+            for (int j0 = wj0; j0 < wj1; j0 += 32) {
                 const int j = j0 + lane;
-                bool in = false;
-                if (j < len) {
+                bool in = false, up = false;
+                if (j < wj1) {
                     const unsigned o = ord_at(j);
-                    in = one_round ? ((o - LO) >> sh1) == b1 : ((make_key(o, s0 + j) - base) & mask) == prefix;
+                    if (one_round) {
+                        const unsigned d1 = (o - LO) >> sh1;
+                        in = d1 == b1;
+                        up = d1 > b1;
+                    } else {
+                        const unsigned long long xm = (make_key(o, s0 + j) - base) & mask;
+                        in = xm == prefix;
+                        up = xm > prefix;
+                    }
                 }
+                above_cnt += __popc(__ballot_sync(0xFFFFFFFFu, up));
                 const unsigned m = __ballot_sync(0xFFFFFFFFu, in);
                 if (m) {
                     unsigned at = 0;
@@ -364,27 +382,40 @@ __global__ void __cluster_dims__(kDC, 1, 1) __launch_bounds__(kDT, 2) dec_select
             }
             __syncthreads();
             prefix = local_kth(sh.merged, nm, base, prefix, mask, shift, need, sh);
+            // each warp's count: its keys above the bin, plus its keys of the
+            // bin (all in this CTA's list) that reach K
+            const unsigned long long Kb = prefix + base;
+            if (lane == 0) sh.wtot[warp] = above_cnt;
+            __syncthreads();
+            const int nown = (int)(sh.nlist < (unsigned)kList ? sh.nlist : (unsigned)kList);
+            for (int i = tid; i < nown; i += kDT) {
+                const unsigned long long kk = sh.list[i];
+                if (kk >= Kb) atomicAdd(&sh.wtot[(key_pos(kk) - s0) / wseg], 1u);
+            }
+            __syncthreads();
+            counted = true;
         }
         K = prefix + base;
     }
 
     // 4. this segment's selected keys, at the cluster offset, in ascending position
-    const int wseg = ((len + kDWarps - 1) / kDWarps + 31) & ~31;
-    const int j0 = warp * wseg, j1 = j0 + wseg < len ? j0 + wseg : len;
+    const int j0 = wj0, j1 = wj1;
     // key >= K  <=>  ord > Kord, or ord == Kord and position <= Kpos
     const unsigned Kord = (unsigned)(K >> 32), Kpos = 0xFFFFFFFFu - (unsigned)K;
     auto selected = [&](int j) {
         const unsigned o = ord_at(j);
         return o > Kord || (o == Kord && (unsigned)(s0 + j) <= Kpos);
     };
-    unsigned cnt = 0;
-    for (int j = j0; j < j1; j += 32) {
-        const int jj = j + lane;
-        const bool sel = jj < j1 && selected(jj);
-        cnt += __popc(__ballot_sync(0xFFFFFFFFu, sel));
+    if (!counted) {  // the bin closed at K, or every position is selected
+        unsigned cnt = 0;
+        for (int j = j0; j < j1; j += 32) {
+            const int jj = j + lane;
+            const bool sel = jj < j1 && selected(jj);
+            cnt += __popc(__ballot_sync(0xFFFFFFFFu, sel));
+        }
+        if (lane == 0) sh.wtot[warp] = cnt;
+        __syncthreads();
     }
-    if (lane == 0) sh.wtot[warp] = cnt;
-    __syncthreads();
     unsigned wbefore = 0, own = 0;
     for (int w = 0; w < kDWarps; ++w) {
         wbefore += w < warp ? sh.wtot[w] : 0u;
