@@ -180,6 +180,9 @@ struct SelectArgs {
     float *m_sigma;
     unsigned *m_vk;
     int *m_need;
+    // SEL_MEMBER_SCORES in select_fast_kernel: the member rows are selected by
+    // member_select_kernel; only the guardrail's own rows are left here
+    int skip_members;
 };
 
 // adaptive.cu: the adaptive budget from the cutoff margin over the rows of a
@@ -228,6 +231,10 @@ cudaError_t launch_select(const SelectArgs &a, cudaStream_t st);
 // one cluster of CTAs per row
 bool dec_select_kind(int kind);
 cudaError_t launch_dec_select(const SelectArgs &a, cudaStream_t st);
+// member_select.cu: Refine member rows (SEL_MEMBER_SCORES, SEL_DEC_MEMBER)
+// whose candidate lists fit in shared memory, one 128-thread CTA per row
+bool member_select_fits(const SelectArgs &a);
+cudaError_t launch_member_select(const SelectArgs &a, cudaStream_t st);
 cudaError_t launch_adaptive(const AdaptiveArgs &a, cudaStream_t st);
 cudaError_t launch_proxy(const void *q, const float *w, const int *cu, int S, int T, int H, int d,
                          int g, int db, int dtype, const int *plan, const PlanLayout &pl, void *qbar,

@@ -1227,7 +1227,7 @@ __global__ void __launch_bounds__(kFT, 4) select_fast_kernel(SelectArgs a) {
             // the scored row's candidates inside the member's prefix
             if (a.kind == SEL_REUSE_CAND || t < dense_rows(n, a.g, a.db))
                 cand(p, t, a.k, none, false);
-            else
+            else if (!a.skip_members)
                 fast_member_row(a.scores + ((long long)row - a.plan[8]) * a.ld, a.cand + (p - p0) * a.c, a.c, t,
                                 a.k, oi, os, sh, stage, scap, bm);
         }
@@ -1313,6 +1313,13 @@ cudaError_t launch_select_fast(const SelectArgs &a, cudaStream_t st) {
 
 cudaError_t launch_select(const SelectArgs &a, cudaStream_t st) {
     if (a.nrows <= 0) return cudaSuccess;
+    if (member_select_fits(a)) {
+        const cudaError_t e = launch_member_select(a, st);
+        if (e != cudaSuccess || a.kind != SEL_MEMBER_SCORES || a.db <= 0 || a.g <= 1) return e;
+        SelectArgs b = a;  // the guardrail's members scored on their own
+        b.skip_members = 1;
+        return launch_select_fast(b, st);
+    }
     if (fast_kind(a.kind)) return launch_select_fast(a, st);
     if (dec_select_kind(a.kind)) return launch_dec_select(a, st);
     SelectArgs b = a;
