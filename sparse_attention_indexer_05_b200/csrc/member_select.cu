@@ -2,7 +2,7 @@
 // over its group's candidate list (ascending positions, -1 = none), masked to
 // positions <= the member's own, prefill and decode alike.
 //
-// One CTA of 128 threads per row, up to eight CTAs an SM.  A row needs only
+// One CTA of 128 threads per row, up to ten CTAs an SM (48 registers).  A row needs only
 // the scores' ords: its candidates' positions ascend with their index, so
 // among equal scores the lower position is the lower index, and the top-k
 // by (score, then lower position) is
@@ -142,7 +142,7 @@ __device__ __forceinline__ unsigned member_ord(float s, int p, int bound, unsign
     return o;
 }
 
-__global__ void __launch_bounds__(kMT, 8) member_select_kernel(SelectArgs a) {
+__global__ void __launch_bounds__(kMT, 10) member_select_kernel(SelectArgs a) {
     extern __shared__ __align__(16) unsigned mem_ords[];
     __shared__ MemShared sh;
     const int row = blockIdx.x;
